@@ -1,0 +1,177 @@
+"""CPU oracle of the 1-bit Adam compressed-phase step -- TEST INFRASTRUCTURE.
+
+Thin numpy/ctypes wrapper around ``onebit_oracle.c`` (plain single-threaded C).
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package.  The product library
+(``bit_adam_error_b200``) never imports it and shares no code with it.
+
+Every function mirrors one step of the method as the pages state it; see the
+header of ``onebit_oracle.c`` for the passages followed and the readings taken
+where the pages are silent.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from typing import Optional, Tuple
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "onebit_oracle.c")
+_LIB = os.path.join(_HERE, "libonebit_oracle.so")
+
+F32, BF16 = 0, 1
+ADAM, LAMB = 0, 1
+STATUS_NONFINITE = 1
+
+CFLAGS = ["-O2", "-ffp-contract=off", "-fno-fast-math", "-fPIC", "-shared", "-std=c11"]
+
+
+def build(force: bool = False, src: str = _SRC, out: str = _LIB, defines=()) -> str:
+    """Compile the oracle with gcc (no FMA contraction).  Returns the .so path."""
+    if not force and os.path.exists(out) and os.path.getmtime(out) >= os.path.getmtime(src):
+        return out
+    cmd = ["gcc", *CFLAGS, *[f"-D{d}" for d in defines], "-o", out, src, "-lm"]
+    subprocess.run(cmd, check=True)
+    return out
+
+
+_P = ctypes.c_void_p
+_I32 = ctypes.c_int32
+_I64 = ctypes.c_int64
+_F = ctypes.c_float
+_U32 = ctypes.c_uint32
+
+_SIGS = {
+    "orc_words_total": (_I64, [_I32, _P]),
+    "orc_compress": (_U32, [_I32, _I64, _I32, _P, _P, _I32, _F, _P, _P, _P]),
+    "orc_server_reduce": (_U32, [_I32, _I64, _I32, _P, _P, _P, _P, _P, _P]),
+    "orc_adam_apply": (_U32, [_I64, _I32, _P, _P, _P, _F, _F, _F, _P, _P, _P]),
+    "orc_lamb_apply": (_U32, [_I64, _I32, _P, _P, _P, _F, _F, _F, _P, _P, _P, _P]),
+    "orc_warmup": (_U32, [_I32, _I64, _I32, _P, _P, _I32, _I32, _F, _F, _F, _F, _P, _P, _P]),
+    "orc_step": (_U32, [_I32, _I64, _I32, _P, _P, _I32, _I32, _F, _F, _F, _F,
+                        _P, _P, _P, _P, _P, _P, _P, _P, _P]),
+}
+
+
+class Oracle:
+    """ctypes handle on one build of the oracle library."""
+
+    def __init__(self, path: Optional[str] = None):
+        self.path = path or build()
+        self.lib = ctypes.CDLL(self.path)
+        for name, (res, args) in _SIGS.items():
+            fn = getattr(self.lib, name)
+            fn.restype = res
+            fn.argtypes = args
+
+    # -- helpers -----------------------------------------------------------------
+    @staticmethod
+    def _ptr(a: Optional[np.ndarray]):
+        if a is None:
+            return None
+        assert a.flags["C_CONTIGUOUS"], "oracle arrays must be contiguous"
+        return a.ctypes.data
+
+    @staticmethod
+    def _off(offsets) -> np.ndarray:
+        return np.ascontiguousarray(offsets, dtype=np.int64)
+
+    def words_total(self, offsets) -> int:
+        off = self._off(offsets)
+        return int(self.lib.orc_words_total(len(off) - 1, self._ptr(off)))
+
+    @staticmethod
+    def _dtype_of(grads: np.ndarray) -> int:
+        if grads.dtype == np.float32:
+            return F32
+        if grads.dtype == np.uint16:
+            return BF16
+        raise TypeError("grads must be float32 values or uint16 bfloat16 bit patterns")
+
+    # -- stages ------------------------------------------------------------------
+    def compress(self, offsets, grads: np.ndarray, err: np.ndarray, clip: float = 0.0
+                 ) -> Tuple[np.ndarray, np.ndarray, int]:
+        """Worker stage.  ``grads``/``err``: [W, n]; ``err`` updated in place.
+
+        Returns (bits_w [W, words], s_w [W, C], flags).
+        """
+        off = self._off(offsets)
+        W, n = grads.shape
+        C = len(off) - 1
+        words = self.words_total(off)
+        bits_w = np.zeros((W, words), np.uint32)
+        s_w = np.zeros((W, C), np.float32)
+        flags = self.lib.orc_compress(W, n, C, self._ptr(off), self._ptr(grads),
+                                      self._dtype_of(grads), float(clip), self._ptr(err),
+                                      self._ptr(bits_w), self._ptr(s_w))
+        return bits_w, s_w, int(flags)
+
+    def server_reduce(self, offsets, bits_w: np.ndarray, s_w: np.ndarray, srv_err: np.ndarray
+                      ) -> Tuple[np.ndarray, np.ndarray, int]:
+        """Server stage.  ``srv_err`` [n] updated in place.  Returns (bits_srv, s_srv, flags)."""
+        off = self._off(offsets)
+        W = bits_w.shape[0]
+        C = len(off) - 1
+        n = int(off[-1])
+        words = self.words_total(off)
+        bits_srv = np.zeros(words, np.uint32)
+        s_srv = np.zeros(C, np.float32)
+        flags = self.lib.orc_server_reduce(W, n, C, self._ptr(off), self._ptr(bits_w),
+                                           self._ptr(s_w), self._ptr(srv_err),
+                                           self._ptr(bits_srv), self._ptr(s_srv))
+        return bits_srv, s_srv, int(flags)
+
+    def adam_apply(self, offsets, bits_srv, s_srv, m, v, p, beta1, lr, eps) -> int:
+        off = self._off(offsets)
+        return int(self.lib.orc_adam_apply(int(off[-1]), len(off) - 1, self._ptr(off),
+                                           self._ptr(bits_srv), self._ptr(s_srv), beta1, lr,
+                                           eps, self._ptr(m), self._ptr(v), self._ptr(p)))
+
+    def lamb_apply(self, offsets, bits_srv, s_srv, m, v, p, beta1, lr, eps
+                   ) -> Tuple[np.ndarray, int]:
+        off = self._off(offsets)
+        r = np.zeros(len(off) - 1, np.float32)
+        flags = self.lib.orc_lamb_apply(int(off[-1]), len(off) - 1, self._ptr(off),
+                                        self._ptr(bits_srv), self._ptr(s_srv), beta1, lr, eps,
+                                        self._ptr(m), self._ptr(v), self._ptr(p), self._ptr(r))
+        return r, int(flags)
+
+    def warmup(self, offsets, grads, m, v, p, beta1, beta2, lr, eps, optimizer=ADAM) -> int:
+        off = self._off(offsets)
+        W, n = grads.shape
+        return int(self.lib.orc_warmup(W, n, len(off) - 1, self._ptr(off), self._ptr(grads),
+                                       self._dtype_of(grads), optimizer, beta1, beta2, lr, eps,
+                                       self._ptr(m), self._ptr(v), self._ptr(p)))
+
+    def step(self, offsets, grads, state: dict, beta1, lr, eps, clip=0.0, optimizer=ADAM) -> int:
+        """One compressed step.  ``state`` holds p, m, v, err, srv_err (updated in place)
+        and receives bits_w, s_w, bits_srv, s_srv."""
+        off = self._off(offsets)
+        W, n = grads.shape
+        C = len(off) - 1
+        words = self.words_total(off)
+        for key, shape, dt in (("bits_w", (W, words), np.uint32), ("s_w", (W, C), np.float32),
+                               ("bits_srv", (words,), np.uint32), ("s_srv", (C,), np.float32)):
+            if key not in state or state[key].shape != shape:
+                state[key] = np.zeros(shape, dt)
+        return int(self.lib.orc_step(
+            W, n, C, self._ptr(off), self._ptr(grads), self._dtype_of(grads), optimizer,
+            float(clip), beta1, lr, eps, self._ptr(state["p"]), self._ptr(state["m"]),
+            self._ptr(state["v"]), self._ptr(state["err"]), self._ptr(state["srv_err"]),
+            self._ptr(state["bits_w"]), self._ptr(state["s_w"]), self._ptr(state["bits_srv"]),
+            self._ptr(state["s_srv"])))
+
+
+_default: Optional[Oracle] = None
+
+
+def get() -> Oracle:
+    """The default (unmodified) oracle build."""
+    global _default
+    if _default is None:
+        _default = Oracle()
+    return _default

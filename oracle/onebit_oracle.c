@@ -1,0 +1,329 @@
+/*
+ * onebit_oracle.c -- TEST INFRASTRUCTURE, not the product.
+ *
+ * A plain, slow, single-threaded CPU statement of what the 1-bit Adam
+ * compressed-phase step computes.  It is the oracle the CUDA path is checked
+ * against.  Only tests/, __graft_entry__.smoke() and the CPU-baseline leg of
+ * bench.py may load it; the library under bit_adam_error_b200/ never does, and
+ * the two share no code, header, table or constant.
+ *
+ * Sources followed (page title, section):
+ *  - "DeepSpeed Communication Compression and Hiding", section "1-bit Adam:
+ *    预热、冻结方差、误差反馈 / 机制": the step structure -- warmup with full Adam
+ *    moments while step < freeze_step; afterwards compensated = local_grad +
+ *    error, one_bit_quantize -> (q, scale), compressed_allreduce, dequantize,
+ *    error = compensated - dequantized, m = beta1 m + (1 - beta1) g_hat with v
+ *    frozen, param -= lr m / (sqrt(v_frozen) + eps).
+ *  - same page, section "基线：Adam 为什么难压缩": the Adam moment equations.
+ *  - same page, section "1-bit LAMB": r_l = ||w_l|| / ||u_l||,
+ *    w_l <- w_l - eta r_l u_l, computed from the reconstructed global direction.
+ *  - the CANN 1-bit Adam article (intelliparadigm.com), section 3.2
+ *    "核心算法实现细节": clipping of extreme gradient
+ *    values before quantisation (threshold 5.0) and a NaN check after the
+ *    error update.
+ *  - where the pages name a step but give no formula, this oracle fixes it as:
+ *    scale s = ||c||_2 / sqrt(n) per chunk, sign(0) = +1, signs packed into
+ *    uint32 words, err = c - s * sign(c) per worker, and a server stage that
+ *    unpacks the W workers, averages their scaled signs and re-compresses the
+ *    average with its own server error buffer.
+ *
+ * Readings where the pages are silent (each listed in the design notes):
+ *  - bit = (c >= 0.0f): +0 and -0 give +1; NaN gives -1 and raises
+ *    ORC_STATUS_NONFINITE.
+ *  - element i of a chunk -> bit (i % 32) of word (i / 32) of that chunk;
+ *    every chunk starts on a fresh word; padding bits are 0.
+ *  - norms are accumulated in double, in ascending element order; the scale is
+ *    (float)(sqrt(S) / sqrt((double)n_k)); an empty chunk has scale 0.
+ *  - the server average is sum over w = 0..W-1 (ascending) of +-s_w in float,
+ *    then divided by (float)W.
+ *  - no bias correction; warmup averages the W gradients in float, ascending w.
+ *  - clip (when > 0) clamps the raw gradient before the error is added; a NaN
+ *    gradient passes through unchanged.
+ *  - LAMB: layer = chunk; u = m / (sqrtf(v) + eps); r = ||p|| / ||u|| with the
+ *    pre-update p, and r = 1 when either norm is 0; no weight decay.
+ *
+ * Parity pins: every function here is checked by tests/test_oracle_pins.py
+ * against hand-worked cases, closed forms, invariants and brute force.
+ *
+ * Build: gcc -O2 -ffp-contract=off -fPIC -shared (no FMA contraction, plain
+ * IEEE float/double).  All arrays are host memory, caller-owned.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define ORC_F32 0
+#define ORC_BF16 1
+#define ORC_ADAM 0
+#define ORC_LAMB 1
+#define ORC_STATUS_NONFINITE 1u
+
+/* ---- small helpers -------------------------------------------------------- */
+
+static int64_t words_of(int64_t n) { return (n + 31) / 32; }
+
+/* First word of every chunk: chunks start on a fresh word. */
+static void word_offsets(int32_t C, const int64_t* off, int64_t* wo) {
+  wo[0] = 0;
+  for (int32_t k = 0; k < C; ++k) wo[k + 1] = wo[k] + words_of(off[k + 1] - off[k]);
+}
+
+/* bf16 -> float is exact: the 16 bits are the top half of the float32. */
+static float grad_at(const void* grads, int32_t dtype, int64_t idx) {
+  if (dtype == ORC_BF16) {
+    uint32_t u = (uint32_t)((const uint16_t*)grads)[idx] << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return f;
+  }
+  return ((const float*)grads)[idx];
+}
+
+static float clip_grad(float g, float clip) {
+  if (!(clip > 0.0f)) return g;
+  if (g > clip) return clip;
+  if (g < -clip) return -clip;
+  return g; /* NaN falls through */
+}
+
+static int is_nonfinite(float x) { return !isfinite(x); }
+
+/* one_bit_quantize, scale part: s = ||c||_2 / sqrt(n). */
+static float quantize_scale(const float* c, int64_t n) {
+  if (n == 0) return 0.0f;
+  double S = 0.0;
+  for (int64_t i = 0; i < n; ++i) S += (double)c[i] * (double)c[i];
+  return (float)(sqrt(S) / sqrt((double)n));
+}
+
+/* one_bit_quantize, sign part: bit i = (c_i >= 0), LSB-first in uint32 words. */
+static void quantize_signs(const float* c, int64_t n, uint32_t* words) {
+  int64_t nw = words_of(n);
+  for (int64_t j = 0; j < nw; ++j) words[j] = 0u;
+  for (int64_t i = 0; i < n; ++i)
+    if (c[i] >= 0.0f) words[i / 32] |= 1u << (i % 32);
+}
+
+static int sign_bit(const uint32_t* words, int64_t i) {
+  return (int)((words[i / 32] >> (i % 32)) & 1u);
+}
+
+/* dequantize: +scale for a set bit, -scale otherwise. */
+static float dequantize(const uint32_t* words, float scale, int64_t i) {
+  return sign_bit(words, i) ? scale : -scale;
+}
+
+/* ---- exported --------------------------------------------------------------- */
+
+int64_t orc_words_total(int32_t C, const int64_t* off) {
+  int64_t t = 0;
+  for (int32_t k = 0; k < C; ++k) t += words_of(off[k + 1] - off[k]);
+  return t;
+}
+
+/*
+ * Worker stage, every worker w and chunk k:
+ *   compensated c = clip(g_w) + err_w
+ *   (q, s_wk)     = one_bit_quantize(c)
+ *   err_w         = c - dequantize(q, s_wk)
+ * grads: [W][n] (float32 or bf16 bits); err: [W][n] in/out;
+ * bits_w: [W][words_total] out; s_w: [W][C] out.  Returns status flags.
+ */
+uint32_t orc_compress(int32_t W, int64_t n, int32_t C, const int64_t* off,
+                      const void* grads, int32_t dtype, float clip, float* err,
+                      uint32_t* bits_w, float* s_w) {
+  uint32_t flags = 0;
+  int64_t* wo = (int64_t*)malloc(sizeof(int64_t) * (size_t)(C + 1));
+  word_offsets(C, off, wo);
+  int64_t words_total = wo[C];
+  for (int32_t k = 0; k < C; ++k) {
+    int64_t o = off[k], nk = off[k + 1] - off[k];
+    float* c = (float*)malloc(sizeof(float) * (size_t)(nk > 0 ? nk : 1));
+    for (int32_t w = 0; w < W; ++w) {
+      float* e = err + (int64_t)w * n + o;
+      uint32_t* q = bits_w + (int64_t)w * words_total + wo[k];
+      for (int64_t i = 0; i < nk; ++i) {
+        c[i] = clip_grad(grad_at(grads, dtype, (int64_t)w * n + o + i), clip) + e[i];
+        if (is_nonfinite(c[i])) flags |= ORC_STATUS_NONFINITE;
+      }
+      float s = quantize_scale(c, nk);
+      quantize_signs(c, nk, q);
+      s_w[(int64_t)w * C + k] = s;
+      for (int64_t i = 0; i < nk; ++i) e[i] = c[i] - dequantize(q, s, i);
+    }
+    free(c);
+  }
+  free(wo);
+  return flags;
+}
+
+/*
+ * Server stage (the compressed allreduce), every chunk k:
+ *   avg_i  = (sum_{w=0..W-1} dequantize(q_w, s_wk)_i) / W
+ *   c_srv  = avg + srv_err
+ *   (q', s_srv_k) = one_bit_quantize(c_srv)
+ *   srv_err = c_srv - dequantize(q', s_srv_k)
+ * bits_w: [W][words_total]; s_w: [W][C]; srv_err: [n] in/out;
+ * bits_srv: [words_total] out; s_srv: [C] out.  Returns status flags.
+ */
+uint32_t orc_server_reduce(int32_t W, int64_t n, int32_t C, const int64_t* off,
+                           const uint32_t* bits_w, const float* s_w,
+                           float* srv_err, uint32_t* bits_srv, float* s_srv) {
+  (void)n;
+  uint32_t flags = 0;
+  int64_t* wo = (int64_t*)malloc(sizeof(int64_t) * (size_t)(C + 1));
+  word_offsets(C, off, wo);
+  int64_t words_total = wo[C];
+  for (int32_t k = 0; k < C; ++k) {
+    int64_t o = off[k], nk = off[k + 1] - off[k];
+    float* c = (float*)malloc(sizeof(float) * (size_t)(nk > 0 ? nk : 1));
+    for (int64_t i = 0; i < nk; ++i) {
+      float acc = 0.0f;
+      for (int32_t w = 0; w < W; ++w)
+        acc += dequantize(bits_w + (int64_t)w * words_total + wo[k], s_w[(int64_t)w * C + k], i);
+      float avg = acc / (float)W;
+      c[i] = avg + srv_err[o + i];
+      if (is_nonfinite(c[i])) flags |= ORC_STATUS_NONFINITE;
+    }
+    float s = quantize_scale(c, nk);
+    uint32_t* q = bits_srv + wo[k];
+    quantize_signs(c, nk, q);
+    s_srv[k] = s;
+    for (int64_t i = 0; i < nk; ++i) srv_err[o + i] = c[i] - dequantize(q, s, i);
+    free(c);
+  }
+  free(wo);
+  return flags;
+}
+
+/*
+ * Compressed-phase Adam update with frozen v:
+ *   g_hat = dequantize(q', s_srv)
+ *   m = beta1 m + (1 - beta1) g_hat
+ *   p = p - lr m / (sqrtf(v) + eps)
+ */
+uint32_t orc_adam_apply(int64_t n, int32_t C, const int64_t* off,
+                        const uint32_t* bits_srv, const float* s_srv, float beta1,
+                        float lr, float eps, float* m, const float* v, float* p) {
+  (void)n;
+  uint32_t flags = 0;
+  int64_t* wo = (int64_t*)malloc(sizeof(int64_t) * (size_t)(C + 1));
+  word_offsets(C, off, wo);
+  const float one_minus_b1 = 1.0f - beta1;
+  for (int32_t k = 0; k < C; ++k) {
+    int64_t o = off[k], nk = off[k + 1] - off[k];
+    for (int64_t i = 0; i < nk; ++i) {
+      float g_hat = dequantize(bits_srv + wo[k], s_srv[k], i);
+      float mi = beta1 * m[o + i] + one_minus_b1 * g_hat;
+      m[o + i] = mi;
+      float pi = p[o + i] - lr * mi / (sqrtf(v[o + i]) + eps);
+      if (is_nonfinite(pi)) flags |= ORC_STATUS_NONFINITE;
+      p[o + i] = pi;
+    }
+  }
+  free(wo);
+  return flags;
+}
+
+/* Per-layer trust ratio r = ||p|| / ||u|| (pre-update p), 1 if either is 0. */
+static float trust_ratio(const float* p, const float* m, const float* v, float eps, int64_t nk) {
+  double P = 0.0, U = 0.0;
+  for (int64_t i = 0; i < nk; ++i) {
+    float u = m[i] / (sqrtf(v[i]) + eps);
+    P += (double)p[i] * (double)p[i];
+    U += (double)u * (double)u;
+  }
+  if (P > 0.0 && U > 0.0) return (float)(sqrt(P) / sqrt(U));
+  return 1.0f;
+}
+
+static uint32_t lamb_update_layer(float* p, const float* m, const float* v, float lr,
+                                  float eps, int64_t nk) {
+  uint32_t flags = 0;
+  float r = trust_ratio(p, m, v, eps, nk);
+  for (int64_t i = 0; i < nk; ++i) {
+    float u = m[i] / (sqrtf(v[i]) + eps);
+    float pi = p[i] - lr * r * u;
+    if (is_nonfinite(pi)) flags |= ORC_STATUS_NONFINITE;
+    p[i] = pi;
+  }
+  return flags;
+}
+
+/*
+ * Compressed-phase 1-bit LAMB update (layer = chunk), v frozen:
+ *   m = beta1 m + (1 - beta1) g_hat;  u = m / (sqrtf(v) + eps)
+ *   r_l = ||p_l|| / ||u_l||;          p -= lr r_l u
+ * r_out (may be NULL): [C] trust ratios used.
+ */
+uint32_t orc_lamb_apply(int64_t n, int32_t C, const int64_t* off,
+                        const uint32_t* bits_srv, const float* s_srv, float beta1,
+                        float lr, float eps, float* m, const float* v, float* p,
+                        float* r_out) {
+  (void)n;
+  uint32_t flags = 0;
+  int64_t* wo = (int64_t*)malloc(sizeof(int64_t) * (size_t)(C + 1));
+  word_offsets(C, off, wo);
+  const float one_minus_b1 = 1.0f - beta1;
+  for (int32_t k = 0; k < C; ++k) {
+    int64_t o = off[k], nk = off[k + 1] - off[k];
+    for (int64_t i = 0; i < nk; ++i) {
+      float g_hat = dequantize(bits_srv + wo[k], s_srv[k], i);
+      m[o + i] = beta1 * m[o + i] + one_minus_b1 * g_hat;
+    }
+    if (r_out) r_out[k] = trust_ratio(p + o, m + o, v + o, eps, nk);
+    flags |= lamb_update_layer(p + o, m + o, v + o, lr, eps, nk);
+  }
+  free(wo);
+  return flags;
+}
+
+/*
+ * Full-precision warmup step (step < freeze_step):
+ *   g = (sum_{w=0..W-1} g_w) / W
+ *   m = beta1 m + (1 - beta1) g;  v = beta2 v + (1 - beta2) g^2
+ *   Adam: p -= lr m / (sqrtf(v) + eps);  LAMB: trust-ratio update as above.
+ * Error buffers are not touched.
+ */
+uint32_t orc_warmup(int32_t W, int64_t n, int32_t C, const int64_t* off,
+                    const void* grads, int32_t dtype, int32_t optimizer, float beta1,
+                    float beta2, float lr, float eps, float* m, float* v, float* p) {
+  uint32_t flags = 0;
+  const float one_minus_b1 = 1.0f - beta1;
+  const float one_minus_b2 = 1.0f - beta2;
+  for (int64_t i = 0; i < n; ++i) {
+    float acc = 0.0f;
+    for (int32_t w = 0; w < W; ++w) acc += grad_at(grads, dtype, (int64_t)w * n + i);
+    float g = acc / (float)W;
+    if (is_nonfinite(g)) flags |= ORC_STATUS_NONFINITE;
+    m[i] = beta1 * m[i] + one_minus_b1 * g;
+    v[i] = beta2 * v[i] + one_minus_b2 * (g * g);
+    if (optimizer == ORC_ADAM) {
+      float pi = p[i] - lr * m[i] / (sqrtf(v[i]) + eps);
+      if (is_nonfinite(pi)) flags |= ORC_STATUS_NONFINITE;
+      p[i] = pi;
+    }
+  }
+  if (optimizer == ORC_LAMB)
+    for (int32_t k = 0; k < C; ++k) {
+      int64_t o = off[k], nk = off[k + 1] - off[k];
+      flags |= lamb_update_layer(p + o, m + o, v + o, lr, eps, nk);
+    }
+  return flags;
+}
+
+/* One whole compressed-phase step: worker stage, server stage, update. */
+uint32_t orc_step(int32_t W, int64_t n, int32_t C, const int64_t* off,
+                  const void* grads, int32_t dtype, int32_t optimizer, float clip,
+                  float beta1, float lr, float eps, float* p, float* m, const float* v,
+                  float* err, float* srv_err, uint32_t* bits_w, float* s_w,
+                  uint32_t* bits_srv, float* s_srv) {
+  uint32_t flags = orc_compress(W, n, C, off, grads, dtype, clip, err, bits_w, s_w);
+  flags |= orc_server_reduce(W, n, C, off, bits_w, s_w, srv_err, bits_srv, s_srv);
+  if (optimizer == ORC_LAMB)
+    flags |= orc_lamb_apply(n, C, off, bits_srv, s_srv, beta1, lr, eps, m, v, p, NULL);
+  else
+    flags |= orc_adam_apply(n, C, off, bits_srv, s_srv, beta1, lr, eps, m, v, p);
+  return flags;
+}

@@ -1,0 +1,462 @@
+"""Pins of the CPU oracle against things other than itself.
+
+Each ``pin_*`` function takes an ``oracle.Oracle`` and raises AssertionError
+when the oracle disagrees with a hand-worked case, a closed form, an
+invariant of the method, an exact (rational) brute-force computation, or an
+independent library routine (numpy's bit packing, norms, means).  They are
+run against the real oracle (tests/test_oracle_pins.py) and against oracle
+builds with planted mistakes, each of which must fail at least one pin
+(tests/test_oracle_mutants.py).
+
+Passages the checks rest on ('DeepSpeed Communication Compression and
+Hiding', section '1-bit Adam' 机制; same page '基线' for the Adam moments and
+'1-bit LAMB' for the trust ratio; the CANN article section 3.2 for clipping and
+the NaN check), with the scale s = ||c||_2/sqrt(n), sign(0) = +1, LSB-first
+uint32 packing, per-worker error c - s*sign(c), and the server stage that
+averages scaled signs and re-compresses with its own error buffer.
+"""
+
+from __future__ import annotations
+
+import json
+import math
+import os
+from fractions import Fraction
+
+import numpy as np
+
+from workloads import aux_bits, aux_normal, aux_uniform
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+SEED = 0x0B17
+B1, B2, LR, EPS = np.float32(0.9), np.float32(0.999), np.float32(1e-4), np.float32(1e-8)
+
+
+# -- independent helpers (numpy library routines, no oracle code) ---------------
+
+def offsets_of(sizes):
+    off = np.zeros(len(sizes) + 1, np.int64)
+    np.cumsum(np.asarray(sizes, np.int64), out=off[1:])
+    return off
+
+
+def word_base(sizes):
+    wb = [0]
+    for s in sizes:
+        wb.append(wb[-1] + (s + 31) // 32)
+    return wb
+
+
+def pack_ref(mask: np.ndarray) -> np.ndarray:
+    """Pack booleans LSB-first into uint32 words with numpy (independent packer)."""
+    nw = (len(mask) + 31) // 32
+    padded = np.zeros(nw * 32, np.uint8)
+    padded[: len(mask)] = mask
+    return np.packbits(padded, bitorder="little").view("<u4").astype(np.uint32)
+
+
+def unpack_ref(words: np.ndarray, nk: int) -> np.ndarray:
+    bits = np.unpackbits(np.ascontiguousarray(words, dtype="<u4").view(np.uint8), bitorder="little")
+    return bits[:nk].astype(bool)
+
+
+def ulp32(x) -> np.ndarray:
+    return np.spacing(np.abs(np.asarray(x, np.float32))).astype(np.float64)
+
+
+# -- hand-worked cases ----------------------------------------------------------
+
+def _case_c(case) -> np.ndarray:
+    if "c" in case:
+        return np.array([float(v) for v in case["c"]], np.float32)
+    name = case["name"]
+    if name.startswith("n33"):
+        return np.array([(-1) ** i * (i + 1) for i in range(33)], np.float32)
+    if name.startswith("n64"):
+        return np.array([i - 31.5 for i in range(64)], np.float32)
+    raise KeyError(name)
+
+
+def pin_hand_cases(o):
+    cases = json.load(open(os.path.join(GOLDEN, "pack_hand_cases.json")))["cases"]
+    for case in cases:
+        c = _case_c(case)
+        n = len(c)
+        g = c[None, :].copy()
+        err = np.zeros_like(g)
+        bits, s, flags = o.compress([0, n], g, err)
+        want_words = [int(w, 16) for w in case["words"]]
+        assert [int(x) for x in bits[0]] == want_words, (case["name"], [hex(x) for x in bits[0]])
+        assert sum(bin(int(x)).count("1") for x in bits[0]) == case["popcount"], case["name"]
+        assert flags == 0
+        s_exact = math.sqrt(float(Fraction(case["s_squared"])))
+        assert abs(float(s[0, 0]) - s_exact) <= ulp32(s_exact), (case["name"], s[0, 0], s_exact)
+        assert Fraction(case["sum_sq"]) == sum(Fraction(float(x)) ** 2 for x in c)
+        sign = np.where(unpack_ref(bits[0], n), 1.0, -1.0)
+        want_err = c.astype(np.float64) - float(s[0, 0]) * sign
+        assert np.all(np.abs(err[0] - want_err) <= 0.5 * ulp32(err[0])), case["name"]
+
+
+# -- worker stage invariants ----------------------------------------------------
+
+RAGGED = [33, 64, 1, 100, 0, 257, 31, 32]
+
+
+def _worker_inputs(W, sizes, key, gscale=1e-3, escale=1e-3):
+    n = int(sum(sizes))
+    g = aux_normal(SEED, (1, *key), W * n, gscale).reshape(W, n)
+    err = aux_normal(SEED, (2, *key), W * n, escale).reshape(W, n)
+    return g, err
+
+
+def pin_worker_invariants(o):
+    W, sizes = 3, RAGGED
+    off, wb = offsets_of(sizes), word_base(sizes)
+    g, err0 = _worker_inputs(W, sizes, (10,))
+    err = err0.copy()
+    bits, s, flags = o.compress(off, g, err)
+    assert flags == 0
+    assert bits.shape == (W, wb[-1]) and s.shape == (W, len(sizes))
+    c = g + err0  # float32 addition: the compensated gradient
+    for w in range(W):
+        for k, nk in enumerate(sizes):
+            lo, hi = off[k], off[k + 1]
+            q = bits[w, wb[k]: wb[k + 1]]
+            ck = c[w, lo:hi]
+            # packing: LSB-first, bit = (c >= 0), fresh word per chunk, zero padding
+            assert np.array_equal(q, pack_ref(ck >= 0)), (w, k)
+            assert sum(bin(int(x)).count("1") for x in q) == int(np.count_nonzero(ck >= 0))
+            if nk == 0:
+                assert s[w, k] == 0.0
+                continue
+            # scale: ||s * sign(c)||_2 = s sqrt(n) = ||c||_2
+            norm = np.linalg.norm(ck.astype(np.float64))
+            assert abs(float(s[w, k]) * math.sqrt(nk) - norm) <= 2e-7 * norm, (w, k)
+            # error: c = s*sign(c) + err, exact up to one rounding of err
+            sign = np.where(unpack_ref(q, nk), 1.0, -1.0)
+            exact = ck.astype(np.float64) - float(s[w, k]) * sign
+            assert np.all(np.abs(err[w, lo:hi] - exact) <= 0.5 * ulp32(err[w, lo:hi])), (w, k)
+
+
+def pin_chunk_independence(o):
+    """A multi-chunk call equals the chunks compressed one at a time."""
+    W, sizes = 2, RAGGED
+    off, wb = offsets_of(sizes), word_base(sizes)
+    g, err0 = _worker_inputs(W, sizes, (11,))
+    err = err0.copy()
+    bits, s, _ = o.compress(off, g, err)
+    for k, nk in enumerate(sizes):
+        lo, hi = off[k], off[k + 1]
+        ek = np.ascontiguousarray(err0[:, lo:hi])
+        bk, sk, _ = o.compress([0, nk], np.ascontiguousarray(g[:, lo:hi]), ek)
+        assert np.array_equal(bk, bits[:, wb[k]: wb[k + 1]]), k
+        assert np.array_equal(sk[:, 0], s[:, k]), k
+        assert np.array_equal(ek, err[:, lo:hi]), k
+
+
+def pin_clip(o):
+    g = np.array([[10.0, -10.0, 3.0, -7.0]], np.float32)
+    e = np.zeros_like(g)
+    _, s, _ = o.compress([0, 4], g, e, clip=5.0)
+    assert abs(float(s[0, 0]) - math.sqrt(21.0)) <= ulp32(math.sqrt(21.0))  # c = [5,-5,3,-5]
+    want = np.array([5 - math.sqrt(21), -5 + math.sqrt(21), 3 - math.sqrt(21), -5 + math.sqrt(21)])
+    assert np.all(np.abs(e[0] - want) <= ulp32(math.sqrt(21.0)) + ulp32(want))
+    e = np.zeros_like(g)
+    _, s, _ = o.compress([0, 4], g, e, clip=0.0)
+    assert abs(float(s[0, 0]) - math.sqrt(64.5)) <= ulp32(math.sqrt(64.5))  # no clip
+
+
+def pin_nonfinite(o):
+    g = np.array([[1.0, float("nan"), -2.0, 0.5]], np.float32)
+    e = np.zeros_like(g)
+    bits, s, flags = o.compress([0, 4], g, e)
+    assert flags & 1
+    assert int(bits[0, 0]) == 0b1001  # NaN quantises to -1 (bit 0)
+    g = np.array([[1.0, 2.0, -2.0, 0.5]], np.float32)
+    e = np.zeros_like(g)
+    _, _, flags = o.compress([0, 4], g, e)
+    assert flags == 0
+
+
+# bfloat16 bit patterns with their exact values, decoded by hand:
+# 0x3C23 = +2^(120-127) * (1 + 35/128);  0xBA83 = -2^(117-127) * (1 + 3/128)
+BF16_TABLE = [(0x3F80, 1.0), (0xBF80, -1.0), (0x4040, 3.0), (0x3F00, 0.5), (0xC0A0, -5.0),
+              (0x0000, 0.0), (0x8000, -0.0), (0x3C23, 0.00994873046875),
+              (0xBA83, -0.00099945068359375)]
+
+
+def pin_bf16(o):
+    bits16 = np.array([[b for b, _ in BF16_TABLE]], np.uint16)
+    vals = np.array([[v for _, v in BF16_TABLE]], np.float32)
+    n = bits16.shape[1]
+    e1, e2 = np.zeros((1, n), np.float32), np.zeros((1, n), np.float32)
+    b1, s1, _ = o.compress([0, n], bits16, e1)
+    b2, s2, _ = o.compress([0, n], vals, e2)
+    assert np.array_equal(b1, b2) and np.array_equal(s1, s2) and np.array_equal(e1, e2)
+
+
+def pin_empty_chunk(o):
+    sizes = [0, 8, 0]
+    g = np.array([[0.5, -1, 0, 2, -0.0, -3, 1, -2]], np.float32)
+    e = np.zeros_like(g)
+    bits, s, _ = o.compress(offsets_of(sizes), g, e)
+    assert bits.shape == (1, 1) and int(bits[0, 0]) == 0x5D
+    assert s[0, 0] == 0.0 and s[0, 2] == 0.0 and s[0, 1] > 0
+
+
+# -- server stage ----------------------------------------------------------------
+
+def pin_server_single_worker(o):
+    """W = 1 and a zero server error: the server re-quantisation is the identity."""
+    sizes = [40, 64, 1, 77]
+    off = offsets_of(sizes)
+    g, err = _worker_inputs(1, sizes, (20,))
+    bits_w, s_w, _ = o.compress(off, g, err)
+    srv_err = np.zeros(off[-1], np.float32)
+    bits_srv, s_srv, _ = o.server_reduce(off, bits_w, s_w, srv_err)
+    assert np.array_equal(bits_srv, bits_w[0])
+    assert np.array_equal(s_srv, s_w[0])
+    assert np.all(srv_err == 0.0)
+
+
+def pin_server_identical_workers(o):
+    sizes = [40, 64, 1, 77]
+    off = offsets_of(sizes)
+    for W in (2, 4):
+        g1, e1 = _worker_inputs(1, sizes, (21,))
+        g, err = np.repeat(g1, W, 0), np.repeat(e1, W, 0)
+        bits_w, s_w, _ = o.compress(off, g, err)
+        srv_err = np.zeros(off[-1], np.float32)
+        bits_srv, s_srv, _ = o.server_reduce(off, bits_w, s_w, srv_err)
+        assert np.array_equal(bits_srv, bits_w[0]) and np.array_equal(s_srv, s_w[0]), W
+        assert np.all(srv_err == 0.0), W
+
+
+def pin_server_opposite_workers(o):
+    """Two workers with opposite gradients: the scaled signs cancel exactly."""
+    sizes = [40, 64, 33]
+    off, wb = offsets_of(sizes), word_base(sizes)
+    g1, _ = _worker_inputs(1, sizes, (22,))
+    g = np.concatenate([g1, -g1])
+    err = np.zeros_like(g)
+    bits_w, s_w, _ = o.compress(off, g, err)
+    srv_err = np.zeros(off[-1], np.float32)
+    bits_srv, s_srv, _ = o.server_reduce(off, bits_w, s_w, srv_err)
+    assert np.all(s_srv == 0.0)
+    assert np.all(srv_err == 0.0)
+    for k, nk in enumerate(sizes):
+        assert np.array_equal(bits_srv[wb[k]: wb[k + 1]], pack_ref(np.ones(nk, bool)))
+
+
+def pin_server_bruteforce(o):
+    """Exact rational reconstruction of the server stage on tiny random inputs."""
+    sizes = [5, 32, 33, 64, 17]
+    off, wb = offsets_of(sizes), word_base(sizes)
+    n = int(off[-1])
+    for W in (1, 2, 3, 4):
+        bits_w = np.stack([aux_bits(SEED, (30, W, w), wb[-1]) for w in range(W)])
+        for w in range(W):  # padding bits must be zero on input as well
+            for k, nk in enumerate(sizes):
+                bits_w[w, wb[k]: wb[k + 1]] &= pack_ref(np.ones(nk, bool))
+        s_w = aux_uniform(SEED, (31, W), W * len(sizes), 0.1, 2.0).reshape(W, len(sizes))
+        srv0 = aux_normal(SEED, (32, W), n, 0.5)
+        srv_err = srv0.copy()
+        bits_srv, s_srv, _ = o.server_reduce(off, bits_w, s_w, srv_err)
+        for k, nk in enumerate(sizes):
+            lo = int(off[k])
+            exact = []
+            for i in range(nk):
+                acc = Fraction(0)
+                for w in range(W):
+                    bit = unpack_ref(bits_w[w, wb[k]: wb[k + 1]], nk)[i]
+                    acc += Fraction(float(s_w[w, k])) * (1 if bit else -1)
+                exact.append(acc / W + Fraction(float(srv0[lo + i])))
+            ex = np.array([float(x) for x in exact])
+            mag = np.max(np.abs(s_w[:, k])) + np.max(np.abs(srv0[lo: lo + nk]))
+            tol = (W + 3) * float(np.spacing(np.float32(mag)))
+            s_exact = math.sqrt(float(sum(x * x for x in exact)) / nk)
+            assert abs(float(s_srv[k]) - s_exact) <= 4 * tol, (W, k)
+            sgn = unpack_ref(bits_srv[wb[k]: wb[k + 1]], nk)
+            clear = np.abs(ex) > tol
+            assert np.array_equal(sgn[clear], ex[clear] >= 0), (W, k)
+            rec = srv_err[lo: lo + nk].astype(np.float64) + float(s_srv[k]) * np.where(sgn, 1.0, -1.0)
+            assert np.all(np.abs(rec - ex) <= 2 * tol), (W, k)
+            assert np.array_equal(bits_srv[wb[k]: wb[k + 1]], pack_ref(sgn))
+
+
+def pin_error_feedback_telescopes(o):
+    """Over T steps the transmitted directions add up to the gradients minus the
+    final residuals:  sum_t g_hat_t = mean_w(sum_t g_w,t - err_w,T) - srv_err_T."""
+    W, T, sizes = 3, 6, [50, 64, 33]
+    off, wb = offsets_of(sizes), word_base(sizes)
+    n = int(off[-1])
+    st = {"p": aux_normal(SEED, (40,), n, 0.02), "m": np.zeros(n, np.float32),
+          "v": aux_uniform(SEED, (41,), n, 1e-8, 1e-6),
+          "err": np.zeros((W, n), np.float32), "srv_err": np.zeros(n, np.float32)}
+    gsum = np.zeros((W, n))
+    ghat_sum = np.zeros(n)
+    for t in range(T):
+        g = aux_normal(SEED, (42, t), W * n, 1e-3).reshape(W, n)
+        gsum += g
+        o.step(off, g, st, B1, LR, EPS)
+        for k, nk in enumerate(sizes):
+            sg = np.where(unpack_ref(st["bits_srv"][wb[k]: wb[k + 1]], nk), 1.0, -1.0)
+            ghat_sum[off[k]: off[k + 1]] += float(st["s_srv"][k]) * sg
+    want = (gsum - st["err"]).mean(0) - st["srv_err"]
+    assert np.max(np.abs(ghat_sum - want)) <= 1e-8, np.max(np.abs(ghat_sum - want))
+
+
+# -- updates ---------------------------------------------------------------------
+
+def _fixed_direction(sizes, key):
+    wb = word_base(sizes)
+    bits = aux_bits(SEED, key, wb[-1])
+    for k, nk in enumerate(sizes):
+        bits[wb[k]: wb[k + 1]] &= pack_ref(np.ones(nk, bool))
+    return bits
+
+
+def _ghat(bits, s, sizes):
+    wb = word_base(sizes)
+    out = []
+    for k, nk in enumerate(sizes):
+        out.append(float(s[k]) * np.where(unpack_ref(bits[wb[k]: wb[k + 1]], nk), 1.0, -1.0))
+    return np.concatenate(out)
+
+
+def pin_adam_closed_form(o):
+    """Constant g_hat from m = 0: m_t = (1 - b1^t) g_hat and
+    p_t = p_0 - lr g_hat/(sqrt(v)+eps) * (t - b1 (1 - b1^t)/(1 - b1)); v untouched."""
+    sizes, T = [40, 24], 20
+    off = offsets_of(sizes)
+    n = int(off[-1])
+    bits = _fixed_direction(sizes, (50,))
+    s = np.array([0.3, 0.7], np.float32)
+    m = np.zeros(n, np.float32)
+    v = aux_uniform(SEED, (51,), n, 1e-4, 1e-2)
+    v0 = v.copy()
+    p0 = aux_normal(SEED, (52,), n, 0.02)
+    p = p0.copy()
+    for _ in range(T):
+        o.adam_apply(off, bits, s, m, v, p, B1, LR, EPS)
+    gh = _ghat(bits, s, sizes)
+    b1 = float(B1)
+    assert np.allclose(m, (1 - b1 ** T) * gh, rtol=2e-6, atol=0)
+    sum_m = T - b1 * (1 - b1 ** T) / (1 - b1)
+    want_p = p0 - float(LR) * gh * sum_m / (np.sqrt(v0.astype(np.float64)) + float(EPS))
+    assert np.max(np.abs(p - want_p)) <= 2e-7, np.max(np.abs(p - want_p))
+    assert np.array_equal(v, v0)
+
+
+def pin_lamb_proportional(o):
+    """With u proportional to p inside a layer the trust ratio cancels the scale:
+    p_new = (1 - lr) p; a zero layer takes r = 1."""
+    sizes = [48, 40, 16]
+    off, wb = offsets_of(sizes), word_base(sizes)
+    n = int(off[-1])
+    bits = _fixed_direction(sizes, (60,))
+    s = np.array([0.25, 0.5, 0.125], np.float32)
+    sgn = _ghat(bits, np.ones(3, np.float32), sizes)
+    a = np.repeat(np.array([0.05, 2.0, 0.0]), sizes)
+    p0 = (a * sgn).astype(np.float32)
+    p = p0.copy()
+    m = np.zeros(n, np.float32)
+    v = np.full(n, 0.04, np.float32)
+    r, _ = o.lamb_apply(off, bits, s, m, v, p, B1, LR, EPS)
+    lr = float(LR)
+    l0 = slice(0, sizes[0] + sizes[1])
+    assert np.allclose(p[l0], (1 - lr) * p0[l0].astype(np.float64), rtol=1e-6, atol=0)
+    beta = (1 - float(B1)) * s.astype(np.float64) / (math.sqrt(0.04) + float(EPS))
+    assert abs(float(r[0]) - 0.05 / beta[0]) <= 1e-6 * 0.05 / beta[0]
+    assert abs(float(r[1]) - 2.0 / beta[1]) <= 1e-6 * 2.0 / beta[1]
+    assert float(r[2]) == 1.0
+    u2 = (1 - float(B1)) * 0.125 * sgn[off[2]:] / (0.2 + float(EPS))
+    assert np.allclose(p[off[2]:], -lr * u2, rtol=1e-6, atol=0)
+
+
+def pin_lamb_step_norm(o):
+    """Every LAMB update moves a layer by exactly lr * ||p_l|| (r ||u|| = ||p||)."""
+    sizes = [64, 33, 100]
+    off = offsets_of(sizes)
+    n = int(off[-1])
+    bits = _fixed_direction(sizes, (61,))
+    s = np.array([1e-3, 2e-3, 5e-4], np.float32)
+    p0 = aux_normal(SEED, (62,), n, 0.02)
+    p = p0.copy()
+    m = aux_normal(SEED, (63,), n, 1e-3)
+    v = aux_uniform(SEED, (64,), n, 1e-8, 1e-6)
+    o.lamb_apply(off, bits, s, m, v, p, B1, LR, EPS)
+    for k in range(len(sizes)):
+        sl = slice(off[k], off[k + 1])
+        step = np.linalg.norm((p[sl] - p0[sl]).astype(np.float64))
+        want = float(LR) * np.linalg.norm(p0[sl].astype(np.float64))
+        assert abs(step - want) <= 1e-3 * want, (k, step, want)
+
+
+def pin_warmup_closed_form(o):
+    """From m = v = 0 with a constant gradient g (mean over workers):
+    m_t = (1 - b1^t) g, v_t = (1 - b2^t) g^2, and the first Adam move is
+    lr (1 - b1) g / (sqrt(1 - b2)|g| + eps)."""
+    W, sizes = 4, [60, 40]
+    off = offsets_of(sizes)
+    n = int(off[-1])
+    grads = aux_normal(SEED, (70,), W * n, 1e-3).reshape(W, n)
+    gbar = grads.astype(np.float64).mean(0)
+    m, v = np.zeros(n, np.float32), np.zeros(n, np.float32)
+    p0 = aux_normal(SEED, (71,), n, 0.02)
+    p = p0.copy()
+    o.warmup(off, grads, m, v, p, B1, B2, LR, EPS)
+    b1, b2, lr, eps = float(B1), float(B2), float(LR), float(EPS)
+    assert np.allclose(m, (1 - b1) * gbar, rtol=1e-5, atol=0)
+    assert np.allclose(v, (1 - b2) * gbar ** 2, rtol=1e-4, atol=0)
+    move = lr * (1 - b1) * gbar / (math.sqrt(1 - b2) * np.abs(gbar) + eps)
+    assert np.all(np.abs((p0.astype(np.float64) - p) - move) <= 2 * ulp32(p) + 1e-5 * np.abs(move))
+    o.warmup(off, grads, m, v, p, B1, B2, LR, EPS)
+    assert np.allclose(m, (1 - b1 ** 2) * gbar, rtol=1e-5, atol=0)
+    assert np.allclose(v, (1 - b2 ** 2) * gbar ** 2, rtol=1e-4, atol=0)
+
+
+def pin_warmup_lamb(o):
+    """Warmup with the LAMB update: each layer moves by lr ||p_l|| along -m."""
+    W, sizes = 2, [60, 40]
+    off = offsets_of(sizes)
+    n = int(off[-1])
+    grads = aux_normal(SEED, (72,), W * n, 1e-3).reshape(W, n)
+    m, v = np.zeros(n, np.float32), np.zeros(n, np.float32)
+    p0 = aux_normal(SEED, (73,), n, 0.02)
+    p = p0.copy()
+    o.warmup(off, grads, m, v, p, B1, B2, LR, EPS, optimizer=1)
+    for k in range(len(sizes)):
+        sl = slice(off[k], off[k + 1])
+        d = (p[sl] - p0[sl]).astype(np.float64)
+        want = float(LR) * np.linalg.norm(p0[sl].astype(np.float64))
+        assert abs(np.linalg.norm(d) - want) <= 1e-3 * want
+        assert np.all(np.sign(d) == -np.sign(m[sl]))
+
+
+def pin_step_composition(o):
+    """The whole-step entry equals its three stages called in order."""
+    W, sizes = 3, [50, 64, 33]
+    off = offsets_of(sizes)
+    n = int(off[-1])
+    g = aux_normal(SEED, (80,), W * n, 1e-3).reshape(W, n)
+    base = {"p": aux_normal(SEED, (81,), n, 0.02), "m": aux_normal(SEED, (82,), n, 1e-4),
+            "v": aux_uniform(SEED, (83,), n, 1e-8, 1e-6),
+            "err": aux_normal(SEED, (84,), W * n, 1e-4).reshape(W, n),
+            "srv_err": aux_normal(SEED, (85,), n, 1e-4)}
+    for opt in (0, 1):
+        a = {k: v.copy() for k, v in base.items()}
+        o.step(off, g, a, B1, LR, EPS, optimizer=opt)
+        b = {k: v.copy() for k, v in base.items()}
+        bw, sw, _ = o.compress(off, g, b["err"])
+        bs, ss, _ = o.server_reduce(off, bw, sw, b["srv_err"])
+        if opt == 0:
+            o.adam_apply(off, bs, ss, b["m"], b["v"], b["p"], B1, LR, EPS)
+        else:
+            o.lamb_apply(off, bs, ss, b["m"], b["v"], b["p"], B1, LR, EPS)
+        for key in ("p", "m", "err", "srv_err"):
+            assert np.array_equal(a[key], b[key]), (opt, key)
+        assert np.array_equal(a["bits_w"], bw) and np.array_equal(a["bits_srv"], bs)
+
+
+ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_") and callable(v)]

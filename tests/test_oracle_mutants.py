@@ -1,0 +1,69 @@
+"""Planted mistakes in the oracle must be caught by the pins.
+
+Each case copies onebit_oracle.c to a temporary directory, plants one
+plausible mistake (a dropped term, a wrong sign, a wrong index, an inverted
+ratio, ...), builds it with the same flags, and checks that at least one pin
+of tests/oracle_pins.py fails on it.  CPU only; nothing here touches the
+product library.
+"""
+
+import os
+
+import pytest
+
+import oracle
+from oracle_pins import ALL_PINS
+
+SRC = os.path.join(os.path.dirname(oracle.__file__), "onebit_oracle.c")
+
+MUTANTS = {
+    "error_sign": ("e[i] = c[i] - dequantize(q, s, i)", "e[i] = c[i] + dequantize(q, s, i)"),
+    "error_not_added": ("clip) + e[i];", "clip) + 0.0f;"),
+    "sign_of_zero": ("if (c[i] >= 0.0f) words", "if (c[i] > 0.0f) words"),
+    "bit_order": ("words[i / 32] |= 1u << (i % 32)", "words[i / 32] |= 1u << (31 - i % 32)"),
+    "scale_no_sqrt": ("return (float)(sqrt(S) / sqrt((double)n));", "return (float)(S / (double)n);"),
+    "scale_no_mean": ("return (float)(sqrt(S) / sqrt((double)n));", "return (float)sqrt(S);"),
+    "server_sum_not_mean": ("float avg = acc / (float)W;", "float avg = acc;"),
+    "server_error_dropped": ("c[i] = avg + srv_err[o + i];", "c[i] = avg;"),
+    "server_error_sign": ("srv_err[o + i] = c[i] - dequantize(q, s, i)",
+                          "srv_err[o + i] = dequantize(q, s, i) - c[i]"),
+    "server_first_worker_only": ("for (int32_t w = 0; w < W; ++w)\n        acc +=",
+                                 "for (int32_t w = 0; w < 1; ++w)\n        acc +="),
+    "momentum_coeff": ("float mi = beta1 * m[o + i] + one_minus_b1 * g_hat;",
+                       "float mi = one_minus_b1 * m[o + i] + beta1 * g_hat;"),
+    "param_sign": ("float pi = p[o + i] - lr * mi", "float pi = p[o + i] + lr * mi"),
+    "frozen_v_sqrt_dropped": ("lr * mi / (sqrtf(v[o + i]) + eps)", "lr * mi / (v[o + i] + eps)"),
+    "trust_ratio_inverted": ("return (float)(sqrt(P) / sqrt(U));", "return (float)(sqrt(U) / sqrt(P));"),
+    "lamb_ratio_dropped": ("float pi = p[i] - lr * r * u;", "float pi = p[i] - lr * u;"),
+    "warmup_v_not_squared": ("one_minus_b2 * (g * g)", "one_minus_b2 * g"),
+    "warmup_first_worker_only": ("for (int32_t w = 0; w < W; ++w) acc += grad_at",
+                                 "for (int32_t w = 0; w < 1; ++w) acc += grad_at"),
+    "clip_ignored": ("if (g > clip) return clip;", "if (g > clip) return g;"),
+    "bf16_shift": ("[idx] << 16;", "[idx] << 15;"),
+    "chunk_word_base": ("wo[k + 1] = wo[k] + words_of(off[k + 1] - off[k]);",
+                        "wo[k + 1] = wo[k] + (off[k + 1] - off[k]) / 32;"),
+    "nan_not_flagged": ("static int is_nonfinite(float x) { return !isfinite(x); }",
+                        "static int is_nonfinite(float x) { return isinf(x); }"),
+}
+
+
+@pytest.fixture(scope="module")
+def src_text():
+    return open(SRC).read()
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_mutant_is_caught(name, src_text, tmp_path):
+    old, new = MUTANTS[name]
+    assert src_text.count(old) == 1, f"mutation anchor for {name} not unique/present"
+    mutated = tmp_path / "onebit_oracle.c"
+    mutated.write_text(src_text.replace(old, new))
+    lib = oracle.build(force=True, src=str(mutated), out=str(tmp_path / f"lib_{name}.so"))
+    o = oracle.Oracle(lib)
+    caught = []
+    for pin in ALL_PINS:
+        try:
+            pin(o)
+        except (AssertionError, ValueError, FloatingPointError):
+            caught.append(pin.__name__)
+    assert caught, f"planted mistake {name!r} passed every pin"
