@@ -1,0 +1,433 @@
+#!/usr/bin/env python
+"""Benchmark of the 1-bit Adam compressed-phase step on B200.
+
+One step = one pass of the whole fused compressed step (worker stage with
+per-chunk scales, server stage, frozen-v Adam update) over one batch of
+synthetic gradients of the workload, through ``OneBitAdam.step`` ->
+``ob_step``.  Default workload: the flat 1.5e9-element GPT-2-XL-sized buffer
+(23 chunks of 2^26 elements, W = 1 worker, bf16 gradients, fp32 state).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints one JSON line (rank 0).  ``value`` is whole-job Gelem/s (elements of
+all replicas / max-over-ranks device time per step), measured with CUDA
+events with all inputs resident in HBM; ``e2e`` is the same metric through
+the public call with host (pinned) gradients, so the host-to-device copy of
+every step's gradients and a device-to-host read of its scales are inside
+the timed region.  ``roofline`` reports the dominant kernel's algorithmic
+bytes per launch over its CUDA-event time on its launch stream against the
+measured HBM copy bandwidth.  ``--impl reference`` times the CPU oracle (the
+plain C statement of the method) on a bounded sample of the same workload.
+
+Multi-GPU: every rank runs an independent replica of the workload (the
+virtual workers of one replica live in one GPU's memory); no collective is on
+the data path, so scaling is weak.
+"""
+
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+METRIC = "compressed-phase 1-bit Adam step: Gelem/s and HBM GB/s as % of B200 peak"
+UNIT = "Gelem/s"
+FALLBACK_HBM_GBS = 6650.0
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "ncu_traffic.txt")
+KERNEL_SOURCES = [os.path.join(ROOT, "bit_adam_error_b200", "csrc", f)
+                  for f in ("kernels.cuh", "onebit.cu")]
+
+
+def parse_args():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="gpt2xl-flat")
+    ap.add_argument("--grad-buffers", type=int, default=2,
+                    help="distinct gradient batches cycled through the timed steps")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    a = ap.parse_args()
+    if a.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if a.steps < 1:
+        ap.error("--steps must be >= 1")
+    return a
+
+
+# -- algorithmic traffic per element (three-pass schedule) ---------------------------
+
+def algo_bytes_per_elem(kind: str, wl) -> float:
+    """HBM bytes per element that kernel kind must move in the fused step."""
+    W, gb = wl.W, wl.grad_bytes
+    if kind == "k_worker_norm":          # read g, err for every worker
+        return (gb + 4) * W
+    if kind == "k_worker_pack":          # read g, err, write err, signs; read srv_err
+        return (gb + 8) * W + W / 8 + 4
+    if kind == "k_server_update":
+        if wl.optimizer == "lamb":       # signs, srv_err r/w, server signs, m r/w, v, p reads
+            return W / 8 + 8 + 1 / 8 + 16
+        return W / 8 + 8 + 1 / 8 + 20    # + m, v, p reads and m, p writes
+    if kind == "k_lamb_param":           # m, v, p reads, p write
+        return 16.0
+    return 0.0                           # finalisers: a few bytes per chunk
+
+
+def step_bytes_per_elem(wl) -> float:
+    kinds = ["k_worker_norm", "k_worker_pack", "k_server_update"]
+    if wl.optimizer == "lamb":
+        kinds.append("k_lamb_param")
+    return sum(algo_bytes_per_elem(k, wl) for k in kinds)
+
+
+def measured_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_sha() -> str:
+    h = hashlib.sha256()
+    for p in KERNEL_SOURCES:
+        with open(p, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch of `kernel` from the committed ncu summary, or None
+    when there is none for this kernel/workload or the kernel source changed."""
+    if not os.path.exists(TRAFFIC_FILE):
+        return None
+    sha = kernel_source_sha()
+    with open(TRAFFIC_FILE) as f:
+        for line in f:
+            parts = line.split()
+            if len(parts) < 3 or line.startswith("#"):
+                continue
+            kv = dict(p.split("=", 1) for p in parts[2:] if "=" in p)
+            if parts[0] == kernel and parts[1] == workload and kv.get("source_sha") == sha:
+                return float(kv["dram_bytes_per_launch"])
+    return None
+
+
+# -- clocks during the timed region ------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+    REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(prefix="clocks_", suffix=".csv")
+            self.fh = os.fdopen(fd, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "50", "-i", self.gpu_id], stdout=self.fh, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self, t0: float, t1: float):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "note": "nvidia-smi unavailable"}
+        time.sleep(0.1)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.fh.close()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                p = [x.strip() for x in line.split(",")]
+                if len(p) < 8:
+                    continue
+                try:
+                    ts = datetime.datetime.strptime(p[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                    rows.append((ts, float(p[1]), float(p[2]), float(p[3]) if p[3] not in ("[N/A]", "") else 0.0,
+                                 p[4:8]))
+                except ValueError:
+                    continue
+        os.unlink(self.path)
+        inside = [r for r in rows if t0 - 0.05 <= r[0] <= t1 + 0.05] or rows
+        if not inside:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "note": "no samples"}
+        reasons = sorted({name for r in inside for name, val in zip(self.REASONS, r[4])
+                          if val.lower() == "active"})
+        return {"sm_mhz": statistics.median(r[1] for r in inside),
+                "sm_max_mhz": max(r[2] for r in inside),
+                "reasons": reasons, "samples": len(inside),
+                "power_w_max": max(r[3] for r in inside)}
+
+
+# -- distributed plumbing ------------------------------------------------------------------
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def init_dist(world, local):
+    import torch
+    import torch.distributed as dist
+    if world > 1 and not dist.is_initialized():
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    return dist if world > 1 else None
+
+
+def barrier(dist):
+    if dist is not None:
+        dist.barrier()
+
+
+def max_over_ranks(dist, x: float, device) -> float:
+    if dist is None:
+        return x
+    import torch
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# -- CPU oracle timing ----------------------------------------------------------------------
+
+def oracle_rate(wl, chunks, max_elems=None, min_seconds=0.0, steps=1):
+    """Time the single-threaded oracle's compressed step on whole chunks (or on
+    the first max_elems elements of a chunk, taken as one chunk)."""
+    import oracle
+    import workloads as WL
+    o = oracle.get()
+    f = np.float32
+    elems = 0
+    secs = 0.0
+    per_step = []
+    used = []
+    for k in chunks:
+        nk = wl.sizes[k] if max_elems is None else min(max_elems, wl.sizes[k])
+        g = np.stack([WL.chunk_grads(wl, 0, w, k, 0, nk) for w in range(wl.W)])
+        p, v = WL.chunk_state(wl, k)
+        st = {"p": p[:nk].copy(), "m": np.zeros(nk, np.float32), "v": v[:nk].copy(),
+              "err": np.zeros((wl.W, nk), np.float32), "srv_err": np.zeros(nk, np.float32)}
+        for _ in range(steps):
+            t = time.perf_counter()
+            o.step([0, nk], g, st, f(wl.beta1), f(wl.lr), f(wl.eps), clip=wl.clip,
+                   optimizer=oracle.LAMB if wl.optimizer == "lamb" else oracle.ADAM)
+            dt = time.perf_counter() - t
+            per_step.append(dt)
+            secs += dt
+            elems += nk
+        used.append((k, nk))
+        if secs >= min_seconds:
+            break
+    return elems, secs, per_step, used
+
+
+def run_reference(args):
+    world, rank, local = dist_env()
+    if rank != 0:
+        return 0
+    import workloads as WL
+    wl = WL.get_workload(args.workload)
+    sample = 1 << 23
+    elems, secs, per_step, used = oracle_rate(wl, [0], max_elems=sample, steps=args.warmup + args.steps)
+    timed = per_step[args.warmup:]
+    ms = 1e3 * sum(timed) / len(timed)
+    value = used[0][1] / (ms / 1e3) / 1e9
+    sample_txt = (f"first {used[0][1]} elements of chunk 0 of {wl.name} taken as one chunk, "
+                  f"W={wl.W}, one compressed step per bench step, single thread")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": workload_config(wl, args.gpus),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
+                             "sample": sample_txt},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def workload_config(wl, n_gpus):
+    return {"workload": f"{wl.name}: {wl.description}", "n": wl.n, "chunks": wl.C, "W": wl.W,
+            "grad_dtype": wl.grad_dtype, "state_dtype": "f32", "optimizer": wl.optimizer,
+            "global_batch": wl.W * n_gpus, "parallelism": f"{n_gpus} replica(s) x {wl.W} virtual workers",
+            "l2": f"inputs larger than L2: {step_bytes_per_elem(wl) * wl.n / 1e9:.1f} GB of traffic per step"}
+
+
+# -- our arm -------------------------------------------------------------------------------
+
+def run_ours(args):
+    import torch
+    world, rank, local = dist_env()
+    if world != args.gpus:
+        print(f"warning: --gpus {args.gpus} but WORLD_SIZE={world}", file=sys.stderr)
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    dist = init_dist(world, local)
+
+    import workloads as WL
+    from bit_adam_error_b200 import OneBitAdam, _lib as L
+
+    wl = WL.get_workload(args.workload)
+    n, W = wl.n, wl.W
+    gdt = torch.bfloat16 if wl.grad_dtype == "bf16" else torch.float32
+
+    # State: seeded p, v on the host, uploaded once.
+    p_h = np.empty(n, np.float32)
+    v_h = np.empty(n, np.float32)
+    WL.fill_state(wl.with_(freeze_step=0), p_h, v_h)
+    opt = OneBitAdam(wl.offsets, W, grad_dtype=wl.grad_dtype, optimizer=wl.optimizer, clip=wl.clip,
+                     freeze_step=0, lr=wl.lr, beta1=wl.beta1, beta2=wl.beta2, eps=wl.eps,
+                     device=device, p=torch.from_numpy(p_h).to(device), v=torch.from_numpy(v_h).to(device))
+    del p_h, v_h
+
+    # Gradient batches: generated into pinned host buffers (kept for e2e), copied to HBM.
+    nbuf = max(1, args.grad_buffers)
+    host_g, dev_g = [], []
+    for b in range(nbuf):
+        h = torch.empty((W, n), dtype=gdt, pin_memory=True)
+        arr = h.view(torch.int16).numpy().view(np.uint16) if wl.grad_dtype == "bf16" else h.numpy()
+        WL.fill_grads(wl, b + 1000 * rank, arr)
+        host_g.append(h)
+        dev_g.append(h.to(device))
+    stream = torch.cuda.current_stream(device)
+
+    for i in range(args.warmup):
+        opt.step(dev_g[i % nbuf])
+    torch.cuda.synchronize()
+
+    # -- timed region: inputs resident in HBM ------------------------------------
+    per_step_launches = 5 if wl.optimizer == "adam" else 7
+    L.ob_profile_start(opt.ctx, args.steps * per_step_launches)
+    launches0 = L.ob_launch_count(opt.ctx)
+    sampler = ClockSampler(gpu_id(device))
+    sampler.start()
+    time.sleep(0.3)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(dist)
+    torch.cuda.synchronize()
+    w0 = time.time()
+    e0.record(stream)
+    for i in range(args.steps):
+        opt.step(dev_g[i % nbuf])
+    e1.record(stream)
+    torch.cuda.synchronize()
+    w1 = time.time()
+    barrier(dist)
+    clocks = sampler.stop(w0, w1)
+    launches = L.ob_launch_count(opt.ctx) - launches0
+    prof = L.ob_profile_stop(opt.ctx)
+    ms = e0.elapsed_time(e1) / args.steps
+    ms_max = max_over_ranks(dist, ms, device)
+    status = opt.status()
+
+    # Dominant kernel roofline (this rank's CUDA events on the launch stream).
+    peak, peak_src = measured_peak()
+    dom = max(prof, key=lambda k: prof[k][0])
+    dom_ms = prof[dom][0] / prof[dom][1]
+    dom_bytes = algo_bytes_per_elem(dom, wl) * n
+    achieved = dom_bytes / (dom_ms / 1e3) / 1e9
+    traffic = ncu_traffic(dom, wl.name)
+    total_ms = sum(v[0] for v in prof.values())
+    roofline = {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": peak,
+                "peak_source": f"{peak_src} (copy bandwidth)", "unit": "GB/s",
+                "frac": achieved / peak, "traffic": traffic,
+                "algorithmic_bytes_per_launch": dom_bytes, "launch_ms": dom_ms,
+                "share_of_kernel_time": prof[dom][0] / total_ms}
+    kernels = {k: {"ms_per_launch": v[0] / v[1], "launches": v[1], "share": v[0] / total_ms,
+                   "algorithmic_GBps": (algo_bytes_per_elem(k, wl) * n / (v[0] / v[1] / 1e3) / 1e9)
+                   if algo_bytes_per_elem(k, wl) else None}
+               for k, v in prof.items()}
+    step_gbs = step_bytes_per_elem(wl) * n / (ms_max / 1e3) / 1e9
+
+    # -- end to end: host gradients through the public call ---------------------------
+    e2e = None
+    if not args.no_e2e:
+        s_host = torch.empty(wl.C, dtype=torch.float32, pin_memory=True)
+        for i in range(2):
+            opt.step(host_g[i % nbuf])
+        torch.cuda.synchronize()
+        barrier(dist)
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for i in range(args.steps):
+            opt.step(host_g[i % nbuf])
+            s_host.copy_(opt.s_srv, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier(dist)
+        ms_e2e = max_over_ranks(dist, e0.elapsed_time(e1) / args.steps, device)
+        e2e = {"value": world * n / (ms_e2e / 1e3) / 1e9, "unit": UNIT, "ms_per_step": ms_e2e,
+               "h2d_bytes_per_step": W * n * wl.grad_bytes, "d2h_bytes_per_step": 4 * wl.C}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        elems, secs, _, used = oracle_rate(wl, list(range(wl.C)), min_seconds=10.0)
+        cpu = {"value": elems / secs / 1e9, "unit": UNIT, "cores": 1, "kind": "oracle",
+               "sample": f"{len(used)} whole chunk(s) {[k for k, _ in used]} of {wl.name} "
+                         f"({elems} elements), one compressed step each, single thread, "
+                         f"{secs:.1f} s"}
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": world * n / (ms_max / 1e3) / 1e9, "unit": UNIT,
+                "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+                "data": "synthetic (seeded Philox streams; shapes and distributions of the workload)",
+                "config": workload_config(wl, world),
+                "hbm": {"step_achieved_GBps": step_gbs, "step_frac": step_gbs / peak,
+                        "algorithmic_bytes_per_elem": step_bytes_per_elem(wl), "peak": peak,
+                        "peak_source": peak_src},
+                "roofline": roofline, "kernels": kernels, "cpu_baseline": cpu, "e2e": e2e,
+                "gpu_launches": launches, "status_flags": status, "clocks": clocks}
+        print(json.dumps(line), flush=True)
+    opt.close()
+    if dist is not None:
+        dist.destroy_process_group()
+    return 0
+
+
+def gpu_id(device) -> str:
+    import torch
+    try:
+        return "GPU-" + str(torch.cuda.get_device_properties(device).uuid)
+    except Exception:
+        return str(device.index)
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

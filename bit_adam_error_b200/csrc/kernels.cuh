@@ -1,0 +1,719 @@
+// kernels.cuh -- sm_100a streaming kernels of the 1-bit Adam compressed-phase step.
+//
+// Method ("DeepSpeed Communication Compression and Hiding", section "1-bit Adam",
+// 机制; "1-bit LAMB" for the trust ratio; CANN 1-bit Adam article section 3.2 for
+// the clip and the NaN check):
+//   worker w, chunk k:  c = clip(g_w) + err_w,  s_wk = ||c||_2 / sqrt(n_k),
+//                       bit = (c >= 0),  err_w = c - s_wk * sign
+//   server:             c_srv = (sum_w s_wk sign_w) / W + srv_err,
+//                       s_srv = ||c_srv|| / sqrt(n_k),  srv_err = c_srv - s_srv sign'
+//   update:             g_hat = s_srv sign';  m = b1 m + (1-b1) g_hat;
+//                       p -= lr m / (sqrt(v) + eps)     (v frozen)
+//
+// Everything here is HBM streaming: no contraction, so no tensor cores.  The
+// step is three element passes because two per-chunk norms gate the writes:
+//   pass 1  k_worker_norm      reads g, err               -> per-tile sum c^2
+//   pass 2  k_worker_pack      reads g, err, srv_err      -> err, bits_w, per-tile sum c_srv^2
+//   pass 3  k_server_update    reads bits_w, srv_err, m, v, p -> bits_srv, srv_err, m, p
+// with a tiny deterministic finalize (per-chunk fp64 sum of the tile partials,
+// fixed order) between passes.
+//
+// Work unit: a warp tile of kTile = 512 consecutive elements of ONE chunk (a
+// chunk is cut into ceil(n_k / 512) tiles; tiles never straddle chunks).  Warps
+// stride over tiles (persistent grid), so chunks of any size mix freely and the
+// per-tile partial norm lands at a fixed index: sums are reproducible run to run.
+//
+// Vector path (chunk start and length multiples of 8 elements, and the worker
+// row stride a multiple of 8): lane L of a 256-element group holds elements
+// 8L..8L+7 (two 16-byte fp32 loads, or one 16-byte bf16 load), so its 8 sign bits
+// form byte (L % 4) of word (L / 4) of the group; two xor-shuffles assemble the
+// eight 32-bit words, LSB-first.  Any other chunk takes the scalar path: lane L
+// holds element 32j + L and one ballot is one word.
+//
+// Floating point: fp32 arithmetic in the order written, built with -fmad=false,
+// IEEE division and square root, so every per-element value is the one the
+// plain C statement of the method gives for the same scales.  Norms are summed
+// in double with an explicit fma (c*c is exact in double, so fma(c, c, acc)
+// equals acc + c*c rounded once).
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace ob {
+
+constexpr int kWarp = 32;
+constexpr int kVec = 8;                          // elements per lane per group
+constexpr int kGroupElems = kWarp * kVec;        // 256 elements = 8 words
+constexpr int kGroups = 2;                       // groups per warp tile
+constexpr int kTile = kGroupElems * kGroups;     // 512 elements per warp tile
+constexpr int kTileWords = kTile / 32;
+constexpr int kBlock = 256;                      // threads per CTA (8 warps)
+constexpr int kWarpsPerBlock = kBlock / kWarp;
+constexpr int kFinalizeThreads = 256;
+constexpr unsigned kFull = 0xffffffffu;
+constexpr uint32_t kStatusNonfinite = 1u;
+
+// Chunk tables in device memory (owned by the ctx scratch).
+struct Layout {
+  const int64_t* off;   // [C+1] first element of every chunk
+  const int64_t* wo;    // [C+1] first word of every chunk within a packed row
+  const int64_t* tp;    // [C+1] first warp tile of every chunk
+  const uint8_t* vec;   // [C]   1: 8-wide vector path, 0: scalar path
+  int64_t n;            // elements per row
+  int64_t T;            // warp tiles per row
+  int64_t words;        // packed words per row
+  int32_t C;
+};
+
+struct Hyper {
+  float lr, b1, omb1, b2, omb2, eps, clip;   // omb = 1 - b, computed in float on the host
+};
+
+struct Tile {
+  int k;
+  int64_t ck0;   // element index of the chunk start
+  int64_t nk;    // chunk length
+  int64_t rel;   // chunk-relative index of the tile's first element
+  int64_t w0;    // word index of the chunk's first word
+  bool vec;
+};
+
+// Largest k with tp[k] <= t (tp non-decreasing, tp[C] = T > t): the chunk that
+// owns tile t; empty chunks are skipped automatically.
+__device__ __forceinline__ int find_chunk(const Layout& L, int64_t t, int hint) {
+  if (L.tp[hint] <= t && t < L.tp[hint + 1]) return hint;
+  int lo = 0, hi = L.C;
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (L.tp[mid] <= t) lo = mid; else hi = mid;
+  }
+  return lo;
+}
+
+__device__ __forceinline__ Tile tile_at(const Layout& L, int64_t t, int& hint) {
+  const int k = find_chunk(L, t, hint);
+  hint = k;
+  Tile r;
+  r.k = k;
+  r.ck0 = L.off[k];
+  r.nk = L.off[k + 1] - r.ck0;
+  r.rel = (t - L.tp[k]) * kTile;
+  r.w0 = L.wo[k];
+  r.vec = L.vec[k] != 0;
+  return r;
+}
+
+// ---- element access ------------------------------------------------------------
+
+__device__ __forceinline__ void ld8_ro(const float* p, float (&x)[8]) {
+  const float4 a = __ldg(reinterpret_cast<const float4*>(p));
+  const float4 b = __ldg(reinterpret_cast<const float4*>(p) + 1);
+  x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
+  x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+}
+
+// bf16 -> fp32 is exact: the 16 bits are the top half of the float.
+__device__ __forceinline__ void ld8_ro(const uint16_t* p, float (&x)[8]) {
+  const uint4 u = __ldg(reinterpret_cast<const uint4*>(p));
+  x[0] = __uint_as_float(u.x << 16); x[1] = __uint_as_float(u.x & 0xffff0000u);
+  x[2] = __uint_as_float(u.y << 16); x[3] = __uint_as_float(u.y & 0xffff0000u);
+  x[4] = __uint_as_float(u.z << 16); x[5] = __uint_as_float(u.z & 0xffff0000u);
+  x[6] = __uint_as_float(u.w << 16); x[7] = __uint_as_float(u.w & 0xffff0000u);
+}
+
+// Read-write buffers: plain (coherent) loads.
+__device__ __forceinline__ void ld8(const float* p, float (&x)[8]) {
+  const float4 a = reinterpret_cast<const float4*>(p)[0];
+  const float4 b = reinterpret_cast<const float4*>(p)[1];
+  x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
+  x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+}
+
+__device__ __forceinline__ void st8(float* p, const float (&x)[8]) {
+  reinterpret_cast<float4*>(p)[0] = make_float4(x[0], x[1], x[2], x[3]);
+  reinterpret_cast<float4*>(p)[1] = make_float4(x[4], x[5], x[6], x[7]);
+}
+
+__device__ __forceinline__ float ld1_ro(const float* p) { return __ldg(p); }
+__device__ __forceinline__ float ld1_ro(const uint16_t* p) {
+  return __uint_as_float(static_cast<uint32_t>(__ldg(p)) << 16);
+}
+
+__device__ __forceinline__ void zero8(float (&x)[8]) {
+#pragma unroll
+  for (int j = 0; j < 8; ++j) x[j] = 0.0f;
+}
+
+// ---- method pieces -------------------------------------------------------------
+
+// Clamp the raw gradient to [-clip, clip] when clip > 0; NaN passes through.
+__device__ __forceinline__ float clip_grad(float g, float clip) {
+  if (!(clip > 0.0f)) return g;
+  if (g > clip) return clip;
+  if (g < -clip) return -clip;
+  return g;
+}
+
+__device__ __forceinline__ float signed_scale(bool bit, float s) { return bit ? s : -s; }
+
+// Lanes 4q..4q+3 each hold one byte of word q (LSB-first); returns the whole
+// word in every lane of the quad (lane 4q writes it).
+__device__ __forceinline__ uint32_t quad_word(uint32_t byte, int lane) {
+  uint32_t v = byte << (8 * (lane & 3));
+  v |= __shfl_xor_sync(kFull, v, 1);
+  v |= __shfl_xor_sync(kFull, v, 2);
+  return v;
+}
+
+__device__ __forceinline__ uint32_t lane_byte(uint32_t word, int lane) {
+  return (word >> (8 * (lane & 3))) & 0xffu;
+}
+
+__device__ __forceinline__ double warp_sum(double x) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(kFull, x, o);
+  return x;
+}
+
+__device__ __forceinline__ void flag_nonfinite(bool bad, uint32_t* status) {
+  if (__any_sync(kFull, bad) && (threadIdx.x & 31) == 0) atomicOr(status, kStatusNonfinite);
+}
+
+__device__ __forceinline__ int64_t warp_id() {
+  return (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+}
+__device__ __forceinline__ int64_t warp_count() {
+  return (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+}
+
+// ---- pass 1: per-tile sum of c^2 for every worker ----------------------------------
+// part[w * T + t] = sum over tile t of (clip(g_w) + err_w)^2.
+template <typename GT>
+__global__ void __launch_bounds__(kBlock)
+k_worker_norm(Layout L, int W, const GT* __restrict__ grads, const float* __restrict__ err,
+              float clip, double* __restrict__ part, uint32_t* __restrict__ status) {
+  const int lane = threadIdx.x & 31;
+  const int64_t items = static_cast<int64_t>(W) * L.T;
+  int hint = 0;
+  for (int64_t it = warp_id(); it < items; it += warp_count()) {
+    const int w = static_cast<int>(it / L.T);
+    const int64_t t = it - static_cast<int64_t>(w) * L.T;
+    const Tile tl = tile_at(L, t, hint);
+    const GT* g = grads + static_cast<int64_t>(w) * L.n + tl.ck0;
+    const float* e = err + static_cast<int64_t>(w) * L.n + tl.ck0;
+    double acc = 0.0;
+    bool bad = false;
+    if (tl.vec) {
+      float gv[kGroups][8], ev[kGroups][8];
+#pragma unroll
+      for (int q = 0; q < kGroups; ++q) {
+        const int64_t i0 = tl.rel + q * kGroupElems + lane * kVec;
+        if (i0 < tl.nk) { ld8_ro(g + i0, gv[q]); ld8_ro(e + i0, ev[q]); }
+        else { zero8(gv[q]); zero8(ev[q]); }
+      }
+#pragma unroll
+      for (int q = 0; q < kGroups; ++q)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const float c = clip_grad(gv[q][j], clip) + ev[q][j];
+          acc = fma(static_cast<double>(c), static_cast<double>(c), acc);
+          bad |= !isfinite(c);
+        }
+    } else {
+      for (int j = 0; j < kTileWords; ++j) {
+        const int64_t i = tl.rel + j * 32 + lane;
+        if (i < tl.nk) {
+          const float c = clip_grad(ld1_ro(g + i), clip) + __ldg(e + i);
+          acc = fma(static_cast<double>(c), static_cast<double>(c), acc);
+          bad |= !isfinite(c);
+        }
+      }
+    }
+    acc = warp_sum(acc);
+    if (lane == 0) part[it] = acc;
+    flag_nonfinite(bad, status);
+  }
+}
+
+// ---- finalize: per-chunk scale from tile partials ----------------------------------
+// out[r * C + k] = sqrt(sum_t part[r * T + t]) / sqrt(n_k), t over chunk k's tiles,
+// summed in a fixed order; 0 for an empty chunk.  grid = (C, R).
+__device__ __forceinline__ double block_sum_fixed(double x, double* sm) {
+  const int tid = threadIdx.x;
+  sm[tid] = x;
+  __syncthreads();
+#pragma unroll
+  for (int s = kFinalizeThreads / 2; s > 0; s >>= 1) {
+    if (tid < s) sm[tid] += sm[tid + s];
+    __syncthreads();
+  }
+  const double r = sm[0];
+  __syncthreads();
+  return r;
+}
+
+__global__ void __launch_bounds__(kFinalizeThreads)
+k_finalize_scale(Layout L, const double* __restrict__ part, float* __restrict__ out) {
+  __shared__ double sm[kFinalizeThreads];
+  const int k = blockIdx.x, r = blockIdx.y;
+  const double* pr = part + static_cast<int64_t>(r) * L.T;
+  double acc = 0.0;
+  for (int64_t t = L.tp[k] + threadIdx.x; t < L.tp[k + 1]; t += kFinalizeThreads) acc += pr[t];
+  const double S = block_sum_fixed(acc, sm);
+  if (threadIdx.x == 0) {
+    const int64_t nk = L.off[k + 1] - L.off[k];
+    out[static_cast<int64_t>(r) * L.C + k] =
+        nk > 0 ? __double2float_rn(__ddiv_rn(__dsqrt_rn(S), __dsqrt_rn(static_cast<double>(nk))))
+               : 0.0f;
+  }
+}
+
+// LAMB trust ratio per layer (chunk): r = sqrt(P) / sqrt(U), 1 if either is 0.  grid = C.
+__global__ void __launch_bounds__(kFinalizeThreads)
+k_finalize_ratio(Layout L, const double* __restrict__ partP, const double* __restrict__ partU,
+                 float* __restrict__ ratio) {
+  __shared__ double sm[kFinalizeThreads];
+  const int k = blockIdx.x;
+  double a = 0.0, b = 0.0;
+  for (int64_t t = L.tp[k] + threadIdx.x; t < L.tp[k + 1]; t += kFinalizeThreads) {
+    a += partP[t];
+    b += partU[t];
+  }
+  const double P = block_sum_fixed(a, sm);
+  const double U = block_sum_fixed(b, sm);
+  if (threadIdx.x == 0)
+    ratio[k] = (P > 0.0 && U > 0.0) ? __double2float_rn(__ddiv_rn(__dsqrt_rn(P), __dsqrt_rn(U)))
+                                    : 1.0f;
+}
+
+// ---- pass 2: worker pack (+ server accumulation) -------------------------------------
+// For every worker: c = clip(g) + err, bit = (c >= 0), err = c - s_w sign, bits_w.
+// SERVER: also c_srv = (sum_w s_w sign_w) / W + srv_err and part_srv[t] = sum c_srv^2.
+template <typename GT, bool SERVER>
+__global__ void __launch_bounds__(kBlock)
+k_worker_pack(Layout L, int W, const GT* __restrict__ grads, float* __restrict__ err,
+              const float* __restrict__ s_w, uint32_t* __restrict__ bits_w,
+              const float* __restrict__ srv_err, double* __restrict__ part_srv, float clip,
+              uint32_t* __restrict__ status) {
+  const int lane = threadIdx.x & 31;
+  const float Wf = static_cast<float>(W);
+  int hint = 0;
+  for (int64_t t = warp_id(); t < L.T; t += warp_count()) {
+    const Tile tl = tile_at(L, t, hint);
+    double tsum = 0.0;
+    bool bad = false;
+    if (tl.vec) {
+      float acc[kGroups][8], sv[kGroups][8];
+      bool in[kGroups];
+#pragma unroll
+      for (int q = 0; q < kGroups; ++q) {
+        const int64_t i0 = tl.rel + q * kGroupElems + lane * kVec;
+        in[q] = i0 < tl.nk;
+        zero8(acc[q]);
+        if (SERVER) {
+          if (in[q]) ld8_ro(srv_err + tl.ck0 + i0, sv[q]); else zero8(sv[q]);
+        }
+      }
+      for (int w = 0; w < W; ++w) {
+        const GT* g = grads + static_cast<int64_t>(w) * L.n + tl.ck0;
+        float* e = err + static_cast<int64_t>(w) * L.n + tl.ck0;
+        const float s = __ldg(s_w + static_cast<int64_t>(w) * L.C + tl.k);
+        float gv[kGroups][8], ev[kGroups][8];
+#pragma unroll
+        for (int q = 0; q < kGroups; ++q) {
+          const int64_t i0 = tl.rel + q * kGroupElems + lane * kVec;
+          if (in[q]) { ld8_ro(g + i0, gv[q]); ld8(e + i0, ev[q]); }
+          else { zero8(gv[q]); zero8(ev[q]); }
+        }
+#pragma unroll
+        for (int q = 0; q < kGroups; ++q) {
+          const int64_t i0 = tl.rel + q * kGroupElems + lane * kVec;
+          uint32_t byte = 0;
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const float c = clip_grad(gv[q][j], clip) + ev[q][j];
+            const bool b = c >= 0.0f;
+            const float d = signed_scale(b, s);
+            byte |= static_cast<uint32_t>(b) << j;
+            ev[q][j] = c - d;
+            acc[q][j] = acc[q][j] + d;
+            bad |= in[q] && !isfinite(c);
+          }
+          if (!in[q]) byte = 0;
+          else st8(e + i0, ev[q]);
+          const uint32_t word = quad_word(byte, lane);
+          const int64_t wrel = (tl.rel + q * kGroupElems) / 32 + (lane >> 2);
+          if ((lane & 3) == 0 && wrel * 32 < tl.nk)
+            bits_w[static_cast<int64_t>(w) * L.words + tl.w0 + wrel] = word;
+        }
+      }
+      if (SERVER) {
+#pragma unroll
+        for (int q = 0; q < kGroups; ++q)
+          if (in[q]) {
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              const float cs = __fdiv_rn(acc[q][j], Wf) + sv[q][j];
+              tsum = fma(static_cast<double>(cs), static_cast<double>(cs), tsum);
+              bad |= !isfinite(cs);
+            }
+          }
+      }
+    } else {
+      for (int j = 0; j < kTileWords; ++j) {
+        const int64_t i = tl.rel + j * 32 + lane;
+        const bool inb = i < tl.nk;
+        float acc = 0.0f;
+        for (int w = 0; w < W; ++w) {
+          const float s = __ldg(s_w + static_cast<int64_t>(w) * L.C + tl.k);
+          float* e = err + static_cast<int64_t>(w) * L.n + tl.ck0;
+          bool b = false;
+          if (inb) {
+            const float c = clip_grad(ld1_ro(grads + static_cast<int64_t>(w) * L.n + tl.ck0 + i), clip) + e[i];
+            b = c >= 0.0f;
+            const float d = signed_scale(b, s);
+            e[i] = c - d;
+            acc = acc + d;
+            bad |= !isfinite(c);
+          }
+          const uint32_t word = __ballot_sync(kFull, b);
+          if (lane == 0 && (tl.rel + j * 32) < tl.nk)
+            bits_w[static_cast<int64_t>(w) * L.words + tl.w0 + tl.rel / 32 + j] = word;
+        }
+        if (SERVER && inb) {
+          const float cs = __fdiv_rn(acc, Wf) + __ldg(srv_err + tl.ck0 + i);
+          tsum = fma(static_cast<double>(cs), static_cast<double>(cs), tsum);
+          bad |= !isfinite(cs);
+        }
+      }
+    }
+    if (SERVER) {
+      tsum = warp_sum(tsum);
+      if (lane == 0) part_srv[t] = tsum;
+    }
+    flag_nonfinite(bad, status);
+  }
+}
+
+// ---- server average recomputed from the packed worker signs ---------------------------
+// acc[j] = sum_w s_w[w][k] * sign_w(element), in ascending w (the same float
+// additions pass 2 made), for the 8 elements of this lane in group (rel0).
+__device__ __forceinline__ void server_sum8(const Layout& L, int W, const uint32_t* __restrict__ bits_w,
+                                            const float* __restrict__ s_w, const Tile& tl,
+                                            int64_t wrel, bool word_in, int lane, float (&acc)[8]) {
+  zero8(acc);
+  for (int w = 0; w < W; ++w) {
+    const float s = __ldg(s_w + static_cast<int64_t>(w) * L.C + tl.k);
+    const uint32_t word =
+        word_in ? __ldg(bits_w + static_cast<int64_t>(w) * L.words + tl.w0 + wrel) : 0u;
+    const uint32_t byte = lane_byte(word, lane);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc[j] = acc[j] + signed_scale((byte >> j) & 1u, s);
+  }
+}
+
+// Server norm only (stage-wise call): part_srv[t] = sum over the tile of c_srv^2.
+__global__ void __launch_bounds__(kBlock)
+k_server_norm(Layout L, int W, const uint32_t* __restrict__ bits_w, const float* __restrict__ s_w,
+              const float* __restrict__ srv_err, double* __restrict__ part_srv,
+              uint32_t* __restrict__ status) {
+  const int lane = threadIdx.x & 31;
+  const float Wf = static_cast<float>(W);
+  int hint = 0;
+  for (int64_t t = warp_id(); t < L.T; t += warp_count()) {
+    const Tile tl = tile_at(L, t, hint);
+    double tsum = 0.0;
+    bool bad = false;
+    if (tl.vec) {
+#pragma unroll
+      for (int q = 0; q < kGroups; ++q) {
+        const int64_t i0 = tl.rel + q * kGroupElems + lane * kVec;
+        const int64_t wrel = (tl.rel + q * kGroupElems) / 32 + (lane >> 2);
+        float acc[8];
+        server_sum8(L, W, bits_w, s_w, tl, wrel, wrel * 32 < tl.nk, lane, acc);
+        if (i0 < tl.nk) {
+          float sv[8];
+          ld8_ro(srv_err + tl.ck0 + i0, sv);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const float cs = __fdiv_rn(acc[j], Wf) + sv[j];
+            tsum = fma(static_cast<double>(cs), static_cast<double>(cs), tsum);
+            bad |= !isfinite(cs);
+          }
+        }
+      }
+    } else {
+      for (int j = 0; j < kTileWords; ++j) {
+        const int64_t i = tl.rel + j * 32 + lane;
+        if (i < tl.nk) {
+          float acc = 0.0f;
+          for (int w = 0; w < W; ++w) {
+            const float s = __ldg(s_w + static_cast<int64_t>(w) * L.C + tl.k);
+            const uint32_t word = __ldg(bits_w + static_cast<int64_t>(w) * L.words + tl.w0 + tl.rel / 32 + j);
+            acc = acc + signed_scale((word >> lane) & 1u, s);
+          }
+          const float cs = __fdiv_rn(acc, Wf) + __ldg(srv_err + tl.ck0 + i);
+          tsum = fma(static_cast<double>(cs), static_cast<double>(cs), tsum);
+          bad |= !isfinite(cs);
+        }
+      }
+    }
+    tsum = warp_sum(tsum);
+    if (lane == 0) part_srv[t] = tsum;
+    flag_nonfinite(bad, status);
+  }
+}
+
+// ---- pass 3: server pack + update ------------------------------------------------------
+enum class Upd : int {
+  kNone = 0,   // server pack + server error only (stage-wise call)
+  kAdam = 1,   // + m and p (frozen-v Adam)
+  kLambM = 2,  // + m, and per-tile sums of p^2 and u^2 for the LAMB trust ratio
+};
+
+// Per element: the update given g_hat = d.
+template <Upd U>
+__device__ __forceinline__ void update_elem(float d, float& m, float v, float& p, const Hyper& h,
+                                            double& P, double& Usum, bool& bad) {
+  if (U == Upd::kAdam) {
+    m = h.b1 * m + h.omb1 * d;
+    p = p - __fdiv_rn(h.lr * m, __fsqrt_rn(v) + h.eps);
+    bad |= !isfinite(p);
+  } else if (U == Upd::kLambM) {
+    m = h.b1 * m + h.omb1 * d;
+    const float u = __fdiv_rn(m, __fsqrt_rn(v) + h.eps);
+    P = fma(static_cast<double>(p), static_cast<double>(p), P);
+    Usum = fma(static_cast<double>(u), static_cast<double>(u), Usum);
+  }
+}
+
+// FROM_WORKERS: c_srv from bits_w/s_w/srv_err, quantised with s_srv, bits_srv and
+// srv_err written (the compressed allreduce's second half).  Otherwise g_hat is
+// read back from bits_srv/s_srv (the update-only stage call).
+template <Upd U, bool FROM_WORKERS>
+__global__ void __launch_bounds__(kBlock)
+k_server_update(Layout L, int W, const uint32_t* __restrict__ bits_w, const float* __restrict__ s_w,
+                const float* __restrict__ s_srv, float* __restrict__ srv_err,
+                uint32_t* __restrict__ bits_srv, float* __restrict__ m, const float* __restrict__ v,
+                float* __restrict__ p, Hyper h, double* __restrict__ partP,
+                double* __restrict__ partU, uint32_t* __restrict__ status) {
+  const int lane = threadIdx.x & 31;
+  const float Wf = static_cast<float>(W);
+  int hint = 0;
+  for (int64_t t = warp_id(); t < L.T; t += warp_count()) {
+    const Tile tl = tile_at(L, t, hint);
+    const float s2 = __ldg(s_srv + tl.k);
+    double Psum = 0.0, Usum = 0.0;
+    bool bad = false;
+    if (tl.vec) {
+#pragma unroll
+      for (int q = 0; q < kGroups; ++q) {
+        const int64_t i0 = tl.rel + q * kGroupElems + lane * kVec;
+        const int64_t wrel = (tl.rel + q * kGroupElems) / 32 + (lane >> 2);
+        const bool word_in = wrel * 32 < tl.nk;
+        const bool in = i0 < tl.nk;
+        const int64_t gi = tl.ck0 + i0;
+        float sv[8], mv[8], vv[8], pv[8];
+        if (in) {
+          if (FROM_WORKERS) ld8(srv_err + gi, sv);
+          if (U != Upd::kNone) { ld8(m + gi, mv); ld8_ro(v + gi, vv); ld8(p + gi, pv); }
+        }
+        uint32_t byte = 0;
+        if (FROM_WORKERS) {
+          float acc[8];
+          server_sum8(L, W, bits_w, s_w, tl, wrel, word_in, lane, acc);
+          if (in) {
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              const float cs = __fdiv_rn(acc[j], Wf) + sv[j];
+              const bool b = cs >= 0.0f;
+              const float d = signed_scale(b, s2);
+              byte |= static_cast<uint32_t>(b) << j;
+              sv[j] = cs - d;
+              bad |= !isfinite(cs);
+              update_elem<U>(d, mv[j], vv[j], pv[j], h, Psum, Usum, bad);
+            }
+            st8(srv_err + gi, sv);
+          }
+          const uint32_t word = quad_word(byte, lane);
+          if ((lane & 3) == 0 && word_in) bits_srv[tl.w0 + wrel] = word;
+        } else {
+          const uint32_t word = word_in ? __ldg(bits_srv + tl.w0 + wrel) : 0u;
+          byte = lane_byte(word, lane);
+          if (in) {
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+              update_elem<U>(signed_scale((byte >> j) & 1u, s2), mv[j], vv[j], pv[j], h, Psum, Usum, bad);
+          }
+        }
+        if (in && U != Upd::kNone) {
+          st8(m + gi, mv);
+          if (U == Upd::kAdam) st8(p + gi, pv);
+        }
+      }
+    } else {
+      for (int j = 0; j < kTileWords; ++j) {
+        const int64_t i = tl.rel + j * 32 + lane;
+        const bool inb = i < tl.nk;
+        const int64_t gi = tl.ck0 + i;
+        const int64_t wi = tl.w0 + tl.rel / 32 + j;
+        bool b = false;
+        float d = 0.0f;
+        if (FROM_WORKERS) {
+          if (inb) {
+            float acc = 0.0f;
+            for (int w = 0; w < W; ++w) {
+              const float s = __ldg(s_w + static_cast<int64_t>(w) * L.C + tl.k);
+              const uint32_t word = __ldg(bits_w + static_cast<int64_t>(w) * L.words + wi);
+              acc = acc + signed_scale((word >> lane) & 1u, s);
+            }
+            const float cs = __fdiv_rn(acc, Wf) + srv_err[gi];
+            b = cs >= 0.0f;
+            d = signed_scale(b, s2);
+            srv_err[gi] = cs - d;
+            bad |= !isfinite(cs);
+          }
+          const uint32_t word = __ballot_sync(kFull, b);
+          if (lane == 0 && (tl.rel + j * 32) < tl.nk) bits_srv[wi] = word;
+        } else if (inb) {
+          d = signed_scale((__ldg(bits_srv + wi) >> lane) & 1u, s2);
+        }
+        if (inb && U != Upd::kNone) {
+          float mv = m[gi], pv = p[gi];
+          update_elem<U>(d, mv, __ldg(v + gi), pv, h, Psum, Usum, bad);
+          m[gi] = mv;
+          if (U == Upd::kAdam) p[gi] = pv;
+        }
+      }
+    }
+    if (U == Upd::kLambM) {
+      Psum = warp_sum(Psum);
+      Usum = warp_sum(Usum);
+      if (lane == 0) { partP[t] = Psum; partU[t] = Usum; }
+    }
+    flag_nonfinite(bad, status);
+  }
+}
+
+// ---- LAMB parameter step: p -= lr * r_k * m / (sqrt(v) + eps) ---------------------------
+__global__ void __launch_bounds__(kBlock)
+k_lamb_param(Layout L, const float* __restrict__ m, const float* __restrict__ v,
+             float* __restrict__ p, const float* __restrict__ ratio, Hyper h,
+             uint32_t* __restrict__ status) {
+  const int lane = threadIdx.x & 31;
+  int hint = 0;
+  for (int64_t t = warp_id(); t < L.T; t += warp_count()) {
+    const Tile tl = tile_at(L, t, hint);
+    const float lr_r = h.lr * __ldg(ratio + tl.k);
+    bool bad = false;
+    if (tl.vec) {
+#pragma unroll
+      for (int q = 0; q < kGroups; ++q) {
+        const int64_t i0 = tl.rel + q * kGroupElems + lane * kVec;
+        if (i0 < tl.nk) {
+          const int64_t gi = tl.ck0 + i0;
+          float mv[8], vv[8], pv[8];
+          ld8_ro(m + gi, mv); ld8_ro(v + gi, vv); ld8(p + gi, pv);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const float u = __fdiv_rn(mv[j], __fsqrt_rn(vv[j]) + h.eps);
+            pv[j] = pv[j] - lr_r * u;
+            bad |= !isfinite(pv[j]);
+          }
+          st8(p + gi, pv);
+        }
+      }
+    } else {
+      for (int j = 0; j < kTileWords; ++j) {
+        const int64_t i = tl.rel + j * 32 + lane;
+        if (i < tl.nk) {
+          const int64_t gi = tl.ck0 + i;
+          const float u = __fdiv_rn(__ldg(m + gi), __fsqrt_rn(__ldg(v + gi)) + h.eps);
+          const float pn = p[gi] - lr_r * u;
+          bad |= !isfinite(pn);
+          p[gi] = pn;
+        }
+      }
+    }
+    flag_nonfinite(bad, status);
+  }
+}
+
+// ---- full-precision warmup -------------------------------------------------------------
+// g = (sum_w g_w) / W; m = b1 m + (1-b1) g; v = b2 v + (1-b2) g^2;
+// Adam: p -= lr m / (sqrt(v) + eps).  LAMB: per-tile sums of p^2 and u^2 instead
+// (the parameter step follows in k_lamb_param).
+template <typename GT, bool LAMB>
+__global__ void __launch_bounds__(kBlock)
+k_warmup(Layout L, int W, const GT* __restrict__ grads, float* __restrict__ m,
+         float* __restrict__ v, float* __restrict__ p, Hyper h, double* __restrict__ partP,
+         double* __restrict__ partU, uint32_t* __restrict__ status) {
+  const int lane = threadIdx.x & 31;
+  const float Wf = static_cast<float>(W);
+  int hint = 0;
+  for (int64_t t = warp_id(); t < L.T; t += warp_count()) {
+    const Tile tl = tile_at(L, t, hint);
+    double Psum = 0.0, Usum = 0.0;
+    bool bad = false;
+    auto elem = [&](float gsum, float& mm, float& vv, float& pp) {
+      const float g = __fdiv_rn(gsum, Wf);
+      bad |= !isfinite(g);
+      mm = h.b1 * mm + h.omb1 * g;
+      vv = h.b2 * vv + h.omb2 * (g * g);
+      if (LAMB) {
+        const float u = __fdiv_rn(mm, __fsqrt_rn(vv) + h.eps);
+        Psum = fma(static_cast<double>(pp), static_cast<double>(pp), Psum);
+        Usum = fma(static_cast<double>(u), static_cast<double>(u), Usum);
+      } else {
+        pp = pp - __fdiv_rn(h.lr * mm, __fsqrt_rn(vv) + h.eps);
+        bad |= !isfinite(pp);
+      }
+    };
+    if (tl.vec) {
+#pragma unroll
+      for (int q = 0; q < kGroups; ++q) {
+        const int64_t i0 = tl.rel + q * kGroupElems + lane * kVec;
+        if (i0 < tl.nk) {
+          const int64_t gi = tl.ck0 + i0;
+          float acc[8], mv[8], vv[8], pv[8];
+          zero8(acc);
+          ld8(m + gi, mv); ld8(v + gi, vv); ld8(p + gi, pv);
+          for (int w = 0; w < W; ++w) {
+            float gv[8];
+            ld8_ro(grads + static_cast<int64_t>(w) * L.n + gi, gv);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) acc[j] = acc[j] + gv[j];
+          }
+#pragma unroll
+          for (int j = 0; j < 8; ++j) elem(acc[j], mv[j], vv[j], pv[j]);
+          st8(m + gi, mv);
+          st8(v + gi, vv);
+          if (!LAMB) st8(p + gi, pv);
+        }
+      }
+    } else {
+      for (int j = 0; j < kTileWords; ++j) {
+        const int64_t i = tl.rel + j * 32 + lane;
+        if (i < tl.nk) {
+          const int64_t gi = tl.ck0 + i;
+          float acc = 0.0f;
+          for (int w = 0; w < W; ++w) acc = acc + ld1_ro(grads + static_cast<int64_t>(w) * L.n + gi);
+          float mm = m[gi], vv = v[gi], pp = p[gi];
+          elem(acc, mm, vv, pp);
+          m[gi] = mm;
+          v[gi] = vv;
+          if (!LAMB) p[gi] = pp;
+        }
+      }
+    }
+    if (LAMB) {
+      Psum = warp_sum(Psum);
+      Usum = warp_sum(Usum);
+      if (lane == 0) { partP[t] = Psum; partU[t] = Usum; }
+    }
+    flag_nonfinite(bad, status);
+  }
+}
+
+}  // namespace ob

@@ -1,0 +1,589 @@
+// onebit.cu -- host side of the C ABI declared in include/onebit.h.
+//
+// Validates arguments, owns the per-ctx scratch (chunk tables, per-tile partial
+// norms, LAMB ratios, status word) and enqueues the kernels of kernels.cuh on the
+// caller's stream.  No call allocates or synchronises after ob_create, except
+// ob_get_status (one 4-byte read-back).
+#include <algorithm>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <new>
+#include <vector>
+
+#include <cuda_runtime.h>
+
+#include "onebit.h"
+#include "kernels.cuh"
+
+namespace {
+
+thread_local char g_last_error[512] = "";
+
+ob_err fail(ob_err code, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  std::vsnprintf(g_last_error, sizeof g_last_error, fmt, ap);
+  va_end(ap);
+  return code;
+}
+
+ob_err cuda_fail(cudaError_t e, const char* what) {
+  return fail(OB_ECUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int64_t words_of(int64_t n) { return (n + 31) / 32; }
+
+// Checks everything about a config that needs no device.
+ob_err check_config(const ob_config* c) {
+  if (!c) return fail(OB_EINVAL, "config is NULL");
+  if (c->n < 0) return fail(OB_EINVAL, "n = %lld < 0", (long long)c->n);
+  if (c->num_chunks < 1) return fail(OB_EINVAL, "num_chunks = %d < 1", c->num_chunks);
+  if (!c->chunk_offsets) return fail(OB_EINVAL, "chunk_offsets is NULL");
+  if (c->chunk_offsets[0] != 0) return fail(OB_EINVAL, "chunk_offsets[0] must be 0");
+  for (int32_t k = 0; k < c->num_chunks; ++k)
+    if (c->chunk_offsets[k + 1] < c->chunk_offsets[k])
+      return fail(OB_EINVAL, "chunk_offsets decrease at chunk %d", k);
+  if (c->chunk_offsets[c->num_chunks] != c->n)
+    return fail(OB_EINVAL, "chunk_offsets[C] = %lld != n = %lld",
+                (long long)c->chunk_offsets[c->num_chunks], (long long)c->n);
+  if (c->W < 1 || c->W > 1024) return fail(OB_EINVAL, "W = %d outside [1, 1024]", c->W);
+  if (c->grad_dtype != OB_F32 && c->grad_dtype != OB_BF16)
+    return fail(OB_EINVAL, "grad_dtype = %d is neither OB_F32 nor OB_BF16", c->grad_dtype);
+  if (c->optimizer != OB_ADAM && c->optimizer != OB_LAMB)
+    return fail(OB_EINVAL, "optimizer = %d is neither OB_ADAM nor OB_LAMB", c->optimizer);
+  const float hp[] = {c->lr, c->beta1, c->beta2, c->eps, c->clip};
+  for (float x : hp)
+    if (!std::isfinite(x)) return fail(OB_EINVAL, "hyper-parameters must be finite");
+  if (c->freeze_step < 0) return fail(OB_EINVAL, "freeze_step = %d < 0", c->freeze_step);
+  // Element and word indices of [W][n] rows must fit in int64 comfortably.
+  if (c->n > (int64_t(1) << 50) / c->W) return fail(OB_EINVAL, "W * n too large");
+  return OB_OK;
+}
+
+// A device buffer argument: NULL only when it holds no element; 16-byte
+// aligned; device (or managed) memory of the current device.
+ob_err check_dev(const void* p, int64_t count, const char* name, int device) {
+  if (count == 0) return OB_OK;
+  if (!p) return fail(OB_EINVAL, "%s is NULL", name);
+  if (!aligned16(p)) return fail(OB_EINVAL, "%s is not 16-byte aligned", name);
+  cudaPointerAttributes a;
+  cudaError_t e = cudaPointerGetAttributes(&a, p);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return cuda_fail(e, name);
+  }
+  if (a.type != cudaMemoryTypeDevice && a.type != cudaMemoryTypeManaged)
+    return fail(OB_EINVAL, "%s is not device memory", name);
+  if (a.type == cudaMemoryTypeDevice && a.device != device)
+    return fail(OB_EINVAL, "%s lives on device %d, ctx on device %d", name, a.device, device);
+  return OB_OK;
+}
+
+}  // namespace
+
+struct ob_ctx {
+  ob_config cfg;
+  std::vector<int64_t> off;       // host copy of the chunk offsets
+  int64_t words = 0, T = 0;
+  int device = 0, num_sms = 0;
+  int64_t step = 0;
+  float *p, *m, *v, *err, *srv_err, *s_w, *s_srv;
+  uint32_t *bits_w, *bits_srv;
+  // scratch (one cudaMalloc)
+  void* scratch = nullptr;
+  ob::Layout L{};
+  double *part_w = nullptr, *part_srv = nullptr, *partP = nullptr, *partU = nullptr;
+  float* ratio = nullptr;
+  uint32_t* status = nullptr;
+  ob::Hyper h{};
+  const void* grads_checked = nullptr;   // last grads pointer that passed check_dev
+  std::vector<std::pair<const void*, int>> occ;  // kernel -> resident CTAs per SM
+  // profiling: event pairs around launches
+  int64_t launches = 0;
+  bool prof_on = false;
+  int32_t prof_cap = 0, prof_used = 0;
+  std::vector<cudaEvent_t> prof_ev;
+  std::vector<int32_t> prof_kind;
+};
+
+namespace {
+
+// Persistent grid: enough CTAs to cover `warps` warp-items, at most one full
+// wave of resident CTAs (num_sms x occupancy).
+template <typename K>
+int grid_for(ob_ctx* c, K kernel, int64_t warps) {
+  const void* key = reinterpret_cast<const void*>(kernel);
+  int per_sm = 0;
+  for (auto& kv : c->occ)
+    if (kv.first == key) per_sm = kv.second;
+  if (per_sm == 0) {
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, ob::kBlock, 0) != cudaSuccess ||
+        per_sm < 1) {
+      cudaGetLastError();
+      per_sm = 1;
+    }
+    c->occ.emplace_back(key, per_sm);
+  }
+  const int64_t need = (warps + ob::kWarpsPerBlock - 1) / ob::kWarpsPerBlock;
+  return static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(need, int64_t(c->num_sms) * per_sm)));
+}
+
+// Run fn with the ctx's device current; restore the caller's device after.
+struct DeviceGuard {
+  int prev = -1;
+  bool ok = true;
+  explicit DeviceGuard(int dev) {
+    if (cudaGetDevice(&prev) != cudaSuccess) { ok = false; return; }
+    if (prev != dev && cudaSetDevice(dev) != cudaSuccess) ok = false;
+  }
+  ~DeviceGuard() {
+    int cur = -1;
+    if (prev >= 0 && cudaGetDevice(&cur) == cudaSuccess && cur != prev) cudaSetDevice(prev);
+  }
+};
+
+// Enqueue one kernel launch (fn), with an event pair around it while profiling.
+template <typename Fn>
+void launch(ob_ctx* c, int kind, cudaStream_t st, Fn&& fn) {
+  const bool rec = c->prof_on && c->prof_used < c->prof_cap;
+  if (rec) cudaEventRecord(c->prof_ev[2 * c->prof_used], st);
+  fn();
+  if (rec) {
+    cudaEventRecord(c->prof_ev[2 * c->prof_used + 1], st);
+    c->prof_kind[c->prof_used++] = kind;
+  }
+  ++c->launches;
+}
+
+ob_err check_launch(const char* what) {
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, what);
+  return OB_OK;
+}
+
+ob_err check_grads(ob_ctx* c, const void* grads) {
+  if (grads == c->grads_checked && grads) return OB_OK;
+  const int64_t count = int64_t(c->cfg.W) * c->cfg.n;
+  ob_err r = check_dev(grads, count, "grads", c->device);
+  if (r == OB_OK) c->grads_checked = grads;
+  return r;
+}
+
+// ---- enqueue helpers (no validation) ----------------------------------------------
+
+void enqueue_finalize_scale(ob_ctx* c, const double* part, float* out, int rows, cudaStream_t st) {
+  launch(c, OB_K_FINALIZE_SCALE, st, [&] {
+    ob::k_finalize_scale<<<dim3(c->cfg.num_chunks, rows), ob::kFinalizeThreads, 0, st>>>(c->L, part, out);
+  });
+}
+
+template <typename GT>
+void enqueue_worker(ob_ctx* c, const GT* grads, bool with_server, cudaStream_t st) {
+  const int W = c->cfg.W;
+  if (c->T > 0) {
+    auto k1 = ob::k_worker_norm<GT>;
+    const int g1 = grid_for(c, k1, W * c->T);
+    launch(c, OB_K_WORKER_NORM, st, [&] {
+      k1<<<g1, ob::kBlock, 0, st>>>(c->L, W, grads, c->err, c->h.clip, c->part_w, c->status);
+    });
+  }
+  enqueue_finalize_scale(c, c->part_w, c->s_w, W, st);
+  if (c->T > 0) {
+    auto k2 = with_server ? ob::k_worker_pack<GT, true> : ob::k_worker_pack<GT, false>;
+    const int g2 = grid_for(c, k2, c->T);
+    launch(c, OB_K_WORKER_PACK, st, [&] {
+      k2<<<g2, ob::kBlock, 0, st>>>(c->L, W, grads, c->err, c->s_w, c->bits_w, c->srv_err,
+                                    c->part_srv, c->h.clip, c->status);
+    });
+  }
+  if (with_server) enqueue_finalize_scale(c, c->part_srv, c->s_srv, 1, st);
+}
+
+template <ob::Upd U, bool FROM_WORKERS>
+void enqueue_server_update(ob_ctx* c, cudaStream_t st) {
+  if (c->T == 0) return;
+  auto k3 = ob::k_server_update<U, FROM_WORKERS>;
+  const int g3 = grid_for(c, k3, c->T);
+  launch(c, OB_K_SERVER_UPDATE, st, [&] {
+    k3<<<g3, ob::kBlock, 0, st>>>(c->L, c->cfg.W, c->bits_w, c->s_w, c->s_srv, c->srv_err,
+                                  c->bits_srv, c->m, c->v, c->p, c->h, c->partP, c->partU,
+                                  c->status);
+  });
+}
+
+void enqueue_lamb_param(ob_ctx* c, cudaStream_t st) {
+  launch(c, OB_K_FINALIZE_RATIO, st, [&] {
+    ob::k_finalize_ratio<<<c->cfg.num_chunks, ob::kFinalizeThreads, 0, st>>>(c->L, c->partP, c->partU, c->ratio);
+  });
+  if (c->T == 0) return;
+  auto k = ob::k_lamb_param;
+  const int g = grid_for(c, k, c->T);
+  launch(c, OB_K_LAMB_PARAM, st, [&] {
+    k<<<g, ob::kBlock, 0, st>>>(c->L, c->m, c->v, c->p, c->ratio, c->h, c->status);
+  });
+}
+
+// Update from the packed worker signs (fused) or from bits_srv (stage call).
+void enqueue_update(ob_ctx* c, bool from_workers, cudaStream_t st) {
+  const bool lamb = c->cfg.optimizer == OB_LAMB;
+  if (from_workers) {
+    if (lamb) enqueue_server_update<ob::Upd::kLambM, true>(c, st);
+    else enqueue_server_update<ob::Upd::kAdam, true>(c, st);
+  } else {
+    if (lamb) enqueue_server_update<ob::Upd::kLambM, false>(c, st);
+    else enqueue_server_update<ob::Upd::kAdam, false>(c, st);
+  }
+  if (lamb) enqueue_lamb_param(c, st);
+}
+
+template <typename GT>
+void enqueue_warmup(ob_ctx* c, const GT* grads, cudaStream_t st) {
+  const bool lamb = c->cfg.optimizer == OB_LAMB;
+  if (c->T > 0) {
+    auto k = lamb ? ob::k_warmup<GT, true> : ob::k_warmup<GT, false>;
+    const int g = grid_for(c, k, c->T);
+    launch(c, OB_K_WARMUP, st, [&] {
+      k<<<g, ob::kBlock, 0, st>>>(c->L, c->cfg.W, grads, c->m, c->v, c->p, c->h, c->partP,
+                                  c->partU, c->status);
+    });
+  }
+  if (lamb) enqueue_lamb_param(c, st);
+}
+
+void enqueue_server_stage(ob_ctx* c, cudaStream_t st) {
+  if (c->T > 0) {
+    auto k = ob::k_server_norm;
+    const int g = grid_for(c, k, c->T);
+    launch(c, OB_K_SERVER_NORM, st, [&] {
+      k<<<g, ob::kBlock, 0, st>>>(c->L, c->cfg.W, c->bits_w, c->s_w, c->srv_err, c->part_srv,
+                                  c->status);
+    });
+  }
+  enqueue_finalize_scale(c, c->part_srv, c->s_srv, 1, st);
+  enqueue_server_update<ob::Upd::kNone, true>(c, st);
+}
+
+ob_err fused_step(ob_ctx* c, const void* grads, cudaStream_t st) {
+  if (c->cfg.grad_dtype == OB_BF16)
+    enqueue_worker<uint16_t>(c, static_cast<const uint16_t*>(grads), true, st);
+  else
+    enqueue_worker<float>(c, static_cast<const float*>(grads), true, st);
+  enqueue_update(c, true, st);
+  ob_err r = check_launch("ob_step");
+  if (r == OB_OK) ++c->step;
+  return r;
+}
+
+ob_err check_ctx(const ob_ctx* c) {
+  if (!c) return fail(OB_EINVAL, "ctx is NULL");
+  return OB_OK;
+}
+
+ob_err require_compressed(const ob_ctx* c, const char* call) {
+  if (c->step < c->cfg.freeze_step)
+    return fail(OB_EPHASE, "%s: step %lld is in the warmup phase (freeze_step = %d)", call,
+                (long long)c->step, c->cfg.freeze_step);
+  return OB_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+ob_err ob_layout(const ob_config* cfg, int64_t* words_total) {
+  ob_err r = check_config(cfg);
+  if (r != OB_OK) return r;
+  if (!words_total) return fail(OB_EINVAL, "words_total is NULL");
+  int64_t t = 0;
+  for (int32_t k = 0; k < cfg->num_chunks; ++k)
+    t += words_of(cfg->chunk_offsets[k + 1] - cfg->chunk_offsets[k]);
+  *words_total = t;
+  return OB_OK;
+}
+
+ob_err ob_create(const ob_config* cfg, float* p, float* m, float* v, float* err, float* srv_err,
+                 uint32_t* bits_w, float* s_w, uint32_t* bits_srv, float* s_srv, ob_ctx** out) {
+  if (!out) return fail(OB_EINVAL, "out is NULL");
+  *out = nullptr;
+  int64_t words = 0;
+  ob_err r = ob_layout(cfg, &words);
+  if (r != OB_OK) return r;
+  const int64_t n = cfg->n, W = cfg->W, C = cfg->num_chunks;
+
+  int device = 0;
+  cudaError_t e = cudaGetDevice(&device);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  struct { const void* p; int64_t count; const char* name; } bufs[] = {
+      {p, n, "p"}, {m, n, "m"}, {v, n, "v"}, {err, W * n, "err"}, {srv_err, n, "srv_err"},
+      {bits_w, W * words, "bits_w"}, {s_w, W * C, "s_w"}, {bits_srv, words, "bits_srv"},
+      {s_srv, C, "s_srv"}};
+  for (auto& b : bufs)
+    if ((r = check_dev(b.p, b.count, b.name, device)) != OB_OK) return r;
+
+  ob_ctx* c = new (std::nothrow) ob_ctx();
+  if (!c) return fail(OB_ENOMEM, "ctx allocation failed");
+  c->cfg = *cfg;
+  c->off.assign(cfg->chunk_offsets, cfg->chunk_offsets + C + 1);
+  c->cfg.chunk_offsets = c->off.data();
+  c->device = device;
+  c->words = words;
+  c->p = p; c->m = m; c->v = v; c->err = err; c->srv_err = srv_err;
+  c->bits_w = bits_w; c->s_w = s_w; c->bits_srv = bits_srv; c->s_srv = s_srv;
+  c->h.lr = cfg->lr;
+  c->h.b1 = cfg->beta1;
+  c->h.omb1 = 1.0f - cfg->beta1;
+  c->h.b2 = cfg->beta2;
+  c->h.omb2 = 1.0f - cfg->beta2;
+  c->h.eps = cfg->eps;
+  c->h.clip = cfg->clip;
+  if ((e = cudaDeviceGetAttribute(&c->num_sms, cudaDevAttrMultiProcessorCount, device)) != cudaSuccess) {
+    delete c;
+    return cuda_fail(e, "cudaDeviceGetAttribute");
+  }
+
+  // Chunk tables.
+  std::vector<int64_t> wo(C + 1), tp(C + 1);
+  std::vector<uint8_t> vec(C);
+  wo[0] = tp[0] = 0;
+  for (int64_t k = 0; k < C; ++k) {
+    const int64_t o = c->off[k], nk = c->off[k + 1] - o;
+    wo[k + 1] = wo[k] + words_of(nk);
+    tp[k + 1] = tp[k] + (nk + ob::kTile - 1) / ob::kTile;
+    // 8-wide path: chunk start and length multiples of 8, and every worker row
+    // starts on a multiple of 8 elements (16 bytes of bf16, 32 bytes of fp32).
+    vec[k] = (o % 8 == 0) && (nk % 8 == 0) && (W == 1 || n % 8 == 0);
+  }
+  c->T = tp[C];
+
+  // Scratch layout: tables, then partials, every piece 256-byte aligned.
+  auto up256 = [](size_t x) { return (x + 255) & ~size_t(255); };
+  const size_t sz_tab = up256(sizeof(int64_t) * (C + 1));
+  const size_t sz_vec = up256(size_t(C));
+  const size_t sz_pw = up256(sizeof(double) * size_t(W) * size_t(c->T));
+  const size_t sz_pt = up256(sizeof(double) * size_t(c->T));
+  const size_t sz_ratio = up256(sizeof(float) * size_t(C));
+  const size_t total = 3 * sz_tab + sz_vec + sz_pw + 3 * sz_pt + sz_ratio + 256;
+  if ((e = cudaMalloc(&c->scratch, total)) != cudaSuccess) {
+    cudaGetLastError();
+    delete c;
+    return fail(OB_ENOMEM, "cudaMalloc of %zu scratch bytes failed: %s", total, cudaGetErrorString(e));
+  }
+  char* base = static_cast<char*>(c->scratch);
+  int64_t* d_off = reinterpret_cast<int64_t*>(base); base += sz_tab;
+  int64_t* d_wo = reinterpret_cast<int64_t*>(base); base += sz_tab;
+  int64_t* d_tp = reinterpret_cast<int64_t*>(base); base += sz_tab;
+  uint8_t* d_vec = reinterpret_cast<uint8_t*>(base); base += sz_vec;
+  c->part_w = reinterpret_cast<double*>(base); base += sz_pw;
+  c->part_srv = reinterpret_cast<double*>(base); base += sz_pt;
+  c->partP = reinterpret_cast<double*>(base); base += sz_pt;
+  c->partU = reinterpret_cast<double*>(base); base += sz_pt;
+  c->ratio = reinterpret_cast<float*>(base); base += sz_ratio;
+  c->status = reinterpret_cast<uint32_t*>(base);
+
+  const struct { void* dst; const void* src; size_t bytes; } copies[] = {
+      {d_off, c->off.data(), sizeof(int64_t) * (C + 1)},
+      {d_wo, wo.data(), sizeof(int64_t) * (C + 1)},
+      {d_tp, tp.data(), sizeof(int64_t) * (C + 1)},
+      {d_vec, vec.data(), size_t(C)}};
+  for (auto& cp : copies)
+    if ((e = cudaMemcpy(cp.dst, cp.src, cp.bytes, cudaMemcpyHostToDevice)) != cudaSuccess) {
+      cudaFree(c->scratch);
+      delete c;
+      return cuda_fail(e, "cudaMemcpy of chunk tables");
+    }
+  if ((e = cudaMemset(c->status, 0, sizeof(uint32_t))) != cudaSuccess ||
+      (e = cudaDeviceSynchronize()) != cudaSuccess) {
+    cudaFree(c->scratch);
+    delete c;
+    return cuda_fail(e, "scratch initialisation");
+  }
+  c->L.off = d_off;
+  c->L.wo = d_wo;
+  c->L.tp = d_tp;
+  c->L.vec = d_vec;
+  c->L.n = n;
+  c->L.T = c->T;
+  c->L.words = words;
+  c->L.C = static_cast<int32_t>(C);
+  *out = c;
+  return OB_OK;
+}
+
+ob_err ob_warmup_step(ob_ctx* c, const void* grads, void* stream) {
+  ob_err r = check_ctx(c);
+  if (r != OB_OK) return r;
+  if (c->step >= c->cfg.freeze_step)
+    return fail(OB_EPHASE, "ob_warmup_step: step %lld >= freeze_step %d", (long long)c->step,
+                c->cfg.freeze_step);
+  DeviceGuard dg(c->device);
+  if (!dg.ok) return fail(OB_ECUDA, "cannot select device %d", c->device);
+  if ((r = check_grads(c, grads)) != OB_OK) return r;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (c->cfg.grad_dtype == OB_BF16) enqueue_warmup<uint16_t>(c, static_cast<const uint16_t*>(grads), st);
+  else enqueue_warmup<float>(c, static_cast<const float*>(grads), st);
+  if ((r = check_launch("ob_warmup_step")) != OB_OK) return r;
+  ++c->step;
+  return OB_OK;
+}
+
+ob_err ob_compress(ob_ctx* c, const void* grads, void* stream) {
+  ob_err r = check_ctx(c);
+  if (r != OB_OK) return r;
+  if ((r = require_compressed(c, "ob_compress")) != OB_OK) return r;
+  DeviceGuard dg(c->device);
+  if (!dg.ok) return fail(OB_ECUDA, "cannot select device %d", c->device);
+  if ((r = check_grads(c, grads)) != OB_OK) return r;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (c->cfg.grad_dtype == OB_BF16) enqueue_worker<uint16_t>(c, static_cast<const uint16_t*>(grads), false, st);
+  else enqueue_worker<float>(c, static_cast<const float*>(grads), false, st);
+  return check_launch("ob_compress");
+}
+
+ob_err ob_server_reduce(ob_ctx* c, void* stream) {
+  ob_err r = check_ctx(c);
+  if (r != OB_OK) return r;
+  if ((r = require_compressed(c, "ob_server_reduce")) != OB_OK) return r;
+  DeviceGuard dg(c->device);
+  if (!dg.ok) return fail(OB_ECUDA, "cannot select device %d", c->device);
+  enqueue_server_stage(c, static_cast<cudaStream_t>(stream));
+  return check_launch("ob_server_reduce");
+}
+
+ob_err ob_step(ob_ctx* c, const void* grads, void* stream) {
+  ob_err r = check_ctx(c);
+  if (r != OB_OK) return r;
+  if ((r = require_compressed(c, "ob_step")) != OB_OK) return r;
+  DeviceGuard dg(c->device);
+  if (!dg.ok) return fail(OB_ECUDA, "cannot select device %d", c->device);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (grads) {
+    if ((r = check_grads(c, grads)) != OB_OK) return r;
+    return fused_step(c, grads, st);
+  }
+  enqueue_update(c, false, st);
+  if ((r = check_launch("ob_step")) != OB_OK) return r;
+  ++c->step;
+  return OB_OK;
+}
+
+ob_err ob_step_host(ob_ctx* c, const void* host_grads, void* dev_staging, void* stream) {
+  ob_err r = check_ctx(c);
+  if (r != OB_OK) return r;
+  if ((r = require_compressed(c, "ob_step_host")) != OB_OK) return r;
+  const int64_t count = int64_t(c->cfg.W) * c->cfg.n;
+  if (count > 0 && !host_grads) return fail(OB_EINVAL, "host_grads is NULL");
+  DeviceGuard dg(c->device);
+  if (!dg.ok) return fail(OB_ECUDA, "cannot select device %d", c->device);
+  if ((r = check_grads(c, dev_staging)) != OB_OK) return r;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t bytes = size_t(count) * (c->cfg.grad_dtype == OB_BF16 ? 2 : 4);
+  if (bytes > 0) {
+    cudaError_t e = cudaMemcpyAsync(dev_staging, host_grads, bytes, cudaMemcpyHostToDevice, st);
+    if (e != cudaSuccess) return cuda_fail(e, "ob_step_host: host-to-device copy");
+  }
+  return fused_step(c, dev_staging, st);
+}
+
+ob_err ob_destroy(ob_ctx* c) {
+  if (!c) return OB_OK;
+  ob_err r = OB_OK;
+  for (auto& ev : c->prof_ev) cudaEventDestroy(ev);
+  if (c->scratch) {
+    DeviceGuard dg(c->device);
+    cudaError_t e = cudaFree(c->scratch);
+    if (e != cudaSuccess) r = cuda_fail(e, "cudaFree");
+  }
+  delete c;
+  return r;
+}
+
+ob_err ob_get_status(ob_ctx* c, uint32_t* flags, int32_t clear, void* stream) {
+  ob_err r = check_ctx(c);
+  if (r != OB_OK) return r;
+  if (!flags) return fail(OB_EINVAL, "flags is NULL");
+  DeviceGuard dg(c->device);
+  if (!dg.ok) return fail(OB_ECUDA, "cannot select device %d", c->device);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint32_t h = 0;
+  cudaError_t e = cudaMemcpyAsync(&h, c->status, sizeof h, cudaMemcpyDeviceToHost, st);
+  if (e == cudaSuccess && clear) e = cudaMemsetAsync(c->status, 0, sizeof(uint32_t), st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return cuda_fail(e, "ob_get_status");
+  *flags = h;
+  return OB_OK;
+}
+
+int64_t ob_get_step(const ob_ctx* c) { return c ? c->step : -1; }
+
+ob_err ob_set_step(ob_ctx* c, int64_t step) {
+  ob_err r = check_ctx(c);
+  if (r != OB_OK) return r;
+  if (step < 0) return fail(OB_EINVAL, "step = %lld < 0", (long long)step);
+  c->step = step;
+  return OB_OK;
+}
+
+ob_err ob_profile_start(ob_ctx* c, int32_t capacity) {
+  ob_err r = check_ctx(c);
+  if (r != OB_OK) return r;
+  if (capacity < 1 || capacity > (1 << 20)) return fail(OB_EINVAL, "capacity = %d outside [1, 2^20]", capacity);
+  if (c->prof_on) return fail(OB_EINVAL, "profiling already started");
+  DeviceGuard dg(c->device);
+  if (!dg.ok) return fail(OB_ECUDA, "cannot select device %d", c->device);
+  c->prof_ev.assign(2 * size_t(capacity), nullptr);
+  for (auto& ev : c->prof_ev) {
+    cudaError_t e = cudaEventCreate(&ev);
+    if (e != cudaSuccess) {
+      for (auto& x : c->prof_ev) if (x) cudaEventDestroy(x);
+      c->prof_ev.clear();
+      return cuda_fail(e, "cudaEventCreate");
+    }
+  }
+  c->prof_kind.assign(size_t(capacity), 0);
+  c->prof_cap = capacity;
+  c->prof_used = 0;
+  c->prof_on = true;
+  return OB_OK;
+}
+
+ob_err ob_profile_stop(ob_ctx* c, double* ms, int64_t* launches) {
+  ob_err r = check_ctx(c);
+  if (r != OB_OK) return r;
+  if (!ms || !launches) return fail(OB_EINVAL, "ms / launches is NULL");
+  if (!c->prof_on) return fail(OB_EINVAL, "profiling not started");
+  DeviceGuard dg(c->device);
+  for (int k = 0; k < OB_K_KINDS; ++k) { ms[k] = 0.0; launches[k] = 0; }
+  cudaError_t first = cudaSuccess;
+  for (int32_t i = 0; i < c->prof_used; ++i) {
+    float t = 0.0f;
+    cudaError_t e = cudaEventSynchronize(c->prof_ev[2 * i + 1]);
+    if (e == cudaSuccess) e = cudaEventElapsedTime(&t, c->prof_ev[2 * i], c->prof_ev[2 * i + 1]);
+    if (e != cudaSuccess) { if (first == cudaSuccess) first = e; continue; }
+    ms[c->prof_kind[i]] += t;
+    launches[c->prof_kind[i]] += 1;
+  }
+  for (auto& ev : c->prof_ev) cudaEventDestroy(ev);
+  c->prof_ev.clear();
+  c->prof_kind.clear();
+  c->prof_on = false;
+  c->prof_cap = c->prof_used = 0;
+  if (first != cudaSuccess) return cuda_fail(first, "ob_profile_stop");
+  return OB_OK;
+}
+
+const char* ob_kernel_name(int32_t kind) {
+  static const char* names[OB_K_KINDS] = {
+      "k_worker_norm", "k_finalize_scale", "k_worker_pack", "k_server_norm",
+      "k_server_update", "k_lamb_param", "k_warmup", "k_finalize_ratio"};
+  return (kind >= 0 && kind < OB_K_KINDS) ? names[kind] : "";
+}
+
+int64_t ob_launch_count(const ob_ctx* c) { return c ? c->launches : -1; }
+
+const char* ob_last_error(void) { return g_last_error; }
+
+}  // extern "C"

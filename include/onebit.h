@@ -1,0 +1,183 @@
+/*
+ * onebit.h -- C ABI of the B200 (sm_100a) 1-bit Adam compressed-phase library.
+ *
+ * The calls follow the step as stated in "DeepSpeed Communication Compression
+ * and Hiding", section "1-bit Adam: 预热、冻结方差、误差反馈" (机制):
+ *
+ *     if step < freeze_step:  g = allreduce(local_grad); m, v = adam_moments(g, m, v)
+ *     else:                   compensated = local_grad + error
+ *                             q, scale    = one_bit_quantize(compensated)
+ *                             q_global    = compressed_allreduce(q, scale)
+ *                             g_hat       = dequantize(q_global)
+ *                             error       = compensated - g_hat
+ *                             m           = beta1 m + (1 - beta1) g_hat   (v frozen)
+ *     param -= lr m / (sqrt(v_frozen) + eps)
+ *
+ * with W data-parallel workers held in one GPU's memory.  Where the page gives
+ * no formula the library fixes it as follows:
+ *   - the gradient is cut into chunks (one per parameter tensor or per flat
+ *     slice); each chunk has its own scale s = ||c||_2 / sqrt(n_k);
+ *   - sign(c) is the bit (c >= 0.0f): +0 and -0 send +1, NaN sends -1;
+ *   - element i of chunk k -> bit (i % 32) of word (i / 32) of that chunk's
+ *     words; every chunk starts on a fresh uint32 word; padding bits are 0;
+ *   - the worker error is local, err_w = c - s_wk * sign(c);
+ *   - the compressed allreduce unpacks the W workers, averages the scaled signs
+ *     (sum over w = 0..W-1 in float, then / W), adds a server error buffer,
+ *     re-quantises that sum with its own per-chunk scale, and keeps
+ *     srv_err = c_srv - s_srv * sign(c_srv); g_hat = s_srv * sign(c_srv);
+ *   - norms are accumulated in double and rounded once to float;
+ *   - no bias correction; the warmup averages the W gradients in float.
+ * The 1-bit LAMB variant ("DeepSpeed Communication Compression and Hiding",
+ * section "1-bit LAMB") replaces the last line by u = m / (sqrt(v) + eps),
+ * r_l = ||p_l|| / ||u_l|| per layer (layer = chunk, pre-update p, r = 1 if
+ * either norm is 0), p -= lr r_l u.  Clipping before quantisation (CANN 1-bit
+ * Adam article, section 3.2) clamps the raw gradient to [-clip, clip].
+ *
+ * Conventions for every call:
+ *   - Device buffers are caller-owned and must stay valid for the ctx's life.
+ *     The ctx stores their pointers and owns only its own scratch (per-tile
+ *     partial norms, chunk tables, status word), allocated in ob_create.
+ *   - Every device pointer must be 16-byte aligned; otherwise OB_EINVAL.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *     Calls only enqueue work on it and return; none synchronises except
+ *     ob_get_status and ob_create.
+ *   - Calls return ob_err and never abort or trap.  On failure
+ *     ob_last_error() returns a message (thread-local, valid until the next
+ *     call on the same thread).
+ *   - Calls on one ctx must be ordered (same stream, or synchronised); two
+ *     ctxs may share no state buffer.
+ *   - The step counter advances in ob_warmup_step, ob_step and ob_step_host,
+ *     never in the stage calls.
+ */
+#ifndef ONEBIT_H_
+#define ONEBIT_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct ob_ctx ob_ctx; /* opaque */
+
+typedef enum {
+  OB_OK = 0,
+  OB_EINVAL = -1, /* bad argument: null/misaligned pointer, bad size or layout */
+  OB_ECUDA = -2,  /* a CUDA runtime call or kernel launch failed */
+  OB_EPHASE = -3, /* call not allowed in the current phase (warmup vs compressed) */
+  OB_ENOMEM = -4  /* scratch allocation failed */
+} ob_err;
+
+enum { OB_F32 = 0, OB_BF16 = 1 };  /* gradient element type */
+enum { OB_ADAM = 0, OB_LAMB = 1 }; /* update rule after the compressed allreduce */
+
+#define OB_STATUS_NONFINITE 1u /* a compensated value, server value or parameter was NaN/Inf */
+
+typedef struct {
+  int64_t n;                    /* total elements (parameters); >= 0 */
+  int32_t num_chunks;           /* C >= 1 */
+  const int64_t* chunk_offsets; /* HOST array of C+1 entries: [0] = 0, non-decreasing, [C] = n;
+                                   copied in ob_create.  Empty chunks are allowed (scale 0). */
+  int32_t W;                    /* virtual workers, 1 <= W <= 1024 */
+  int32_t grad_dtype;           /* OB_F32 or OB_BF16 */
+  int32_t optimizer;            /* OB_ADAM or OB_LAMB (LAMB layers = chunks) */
+  float lr, beta1, beta2, eps;
+  float clip;                   /* <= 0: off; else clamp the raw gradient to [-clip, clip] */
+  int32_t freeze_step;          /* steps 0..freeze_step-1 are full-precision warmup */
+} ob_config;
+
+/* Number of uint32 words one packed sign row holds: sum_k ceil(n_k / 32).
+ * Host-only; validates the config.  words_total must be non-NULL. */
+ob_err ob_layout(const ob_config* cfg, int64_t* words_total);
+
+/* Create a ctx over caller-owned DEVICE buffers (float32 unless stated):
+ *   p, m, v, srv_err: [n];  err: [W][n] (worker-major);
+ *   bits_w: uint32 [W][words_total];  s_w: [W][C];
+ *   bits_srv: uint32 [words_total];  s_srv: [C].
+ * Does not initialise them (the caller sets p, m, v; err and srv_err start at 0).
+ * Allocates the ctx scratch with cudaMalloc on the current device and
+ * synchronises once.  *out receives the ctx (NULL on failure). */
+ob_err ob_create(const ob_config* cfg, float* p, float* m, float* v, float* err,
+                 float* srv_err, uint32_t* bits_w, float* s_w, uint32_t* bits_srv,
+                 float* s_srv, ob_ctx** out);
+
+/* One full-precision warmup step (step < freeze_step, else OB_EPHASE):
+ *   g = (sum_w g_w) / W;  m = b1 m + (1-b1) g;  v = b2 v + (1-b2) g^2;
+ *   Adam: p -= lr m / (sqrt(v) + eps);  LAMB: per-layer trust-ratio update.
+ * grads: DEVICE [W][n] of grad_dtype.  Error buffers are not touched. */
+ob_err ob_warmup_step(ob_ctx* ctx, const void* grads, void* stream);
+
+/* Worker stage only (compressed phase): for every worker and chunk,
+ * c = clip(g_w) + err_w, s_w = ||c|| / sqrt(n_k), bits_w = sign(c),
+ * err_w = c - s_w sign(c).  grads: DEVICE [W][n].  Step counter unchanged. */
+ob_err ob_compress(ob_ctx* ctx, const void* grads, void* stream);
+
+/* Server stage only (the compressed allreduce) from bits_w / s_w:
+ * c_srv = mean_w(s_w sign_w) + srv_err, s_srv = ||c_srv|| / sqrt(n_k),
+ * bits_srv = sign(c_srv), srv_err = c_srv - s_srv sign(c_srv). */
+ob_err ob_server_reduce(ob_ctx* ctx, void* stream);
+
+/* grads != NULL: the whole fused compressed step (worker stage, server stage,
+ * update) on DEVICE grads [W][n].  grads == NULL: the update alone from
+ * bits_srv / s_srv (g_hat = s_srv sign), after ob_compress + ob_server_reduce.
+ * Advances the step counter.  OB_EPHASE while step < freeze_step. */
+ob_err ob_step(ob_ctx* ctx, const void* grads, void* stream);
+
+/* Same as ob_step(ctx, grads, ...) with the gradients in HOST memory:
+ * enqueues one host-to-device copy of [W][n] grad_dtype elements from
+ * host_grads into dev_staging (a caller-owned DEVICE buffer of that size,
+ * 16-byte aligned), then the fused step.  host_grads should be page-locked
+ * for the copy to be asynchronous.  Advances the step counter. */
+ob_err ob_step_host(ob_ctx* ctx, const void* host_grads, void* dev_staging, void* stream);
+
+/* Destroy a ctx and free its scratch (not the caller's buffers).  NULL is OK. */
+ob_err ob_destroy(ob_ctx* ctx);
+
+/* Copy the status flags (OB_STATUS_*) accumulated since the last clear into
+ * *flags (HOST); synchronises `stream`.  If clear != 0 the flags are reset. */
+ob_err ob_get_status(ob_ctx* ctx, uint32_t* flags, int32_t clear, void* stream);
+
+/* Step counter (number of completed warmup + compressed steps) for
+ * checkpoint/resume.  ob_get_step returns -1 for a NULL ctx. */
+int64_t ob_get_step(const ob_ctx* ctx);
+ob_err ob_set_step(ob_ctx* ctx, int64_t step);
+
+/* ---- profiling (not part of the method) ----------------------------------
+ * Kernel kinds the library launches, for per-kernel timing: */
+enum {
+  OB_K_WORKER_NORM = 0,    /* pass 1: per-tile sums of c^2, every worker */
+  OB_K_FINALIZE_SCALE = 1, /* per-chunk scale from tile partials */
+  OB_K_WORKER_PACK = 2,    /* pass 2: signs, worker error (+ server sums when fused) */
+  OB_K_SERVER_NORM = 3,    /* server sums alone (stage call) */
+  OB_K_SERVER_UPDATE = 4,  /* pass 3: server signs + error, and/or the update */
+  OB_K_LAMB_PARAM = 5,     /* LAMB parameter step */
+  OB_K_WARMUP = 6,         /* full-precision warmup step */
+  OB_K_FINALIZE_RATIO = 7, /* LAMB trust ratio per layer */
+  OB_K_KINDS = 8
+};
+
+/* Start recording a CUDA event pair around each of the next `capacity`
+ * kernel launches of this ctx, on the stream each is launched on.  Creates
+ * 2*capacity events (a set-up call: do it outside any timed region).
+ * capacity must be in [1, 1<<20]. */
+ob_err ob_profile_start(ob_ctx* ctx, int32_t capacity);
+
+/* Stop recording, wait for the recorded events, and write per kind the total
+ * elapsed milliseconds ms[OB_K_KINDS] and the number of timed launches
+ * launches[OB_K_KINDS] (both HOST arrays).  Destroys the events. */
+ob_err ob_profile_stop(ob_ctx* ctx, double* ms, int64_t* launches);
+
+/* Name of a kernel kind ("" if out of range). */
+const char* ob_kernel_name(int32_t kind);
+
+/* Kernel launches this ctx has enqueued since ob_create (-1 for NULL). */
+int64_t ob_launch_count(const ob_ctx* ctx);
+
+/* Message of the last failed call on this thread ("" if none). */
+const char* ob_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ONEBIT_H_ */

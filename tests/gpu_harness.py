@@ -1,0 +1,156 @@
+"""Shared helpers of the GPU parity tests: run the CUDA path (through the C ABI,
+via the OneBitAdam binding) and the CPU oracle on the same seeded inputs, and
+compare them.
+
+Comparison bar (per step, identical input state):
+  * packed sign words: bit-exact;
+  * scales: relative error <= 1e-5;
+  * state tensors X (err, srv_err, m, v, p), per row and per chunk:
+      max_i |X_gpu - X_ref| <= 1e-5 * max(|X_ref,i|, RMS_chunk(X_ref)).
+"""
+
+from __future__ import annotations
+
+from typing import Dict, Optional, Sequence
+
+import numpy as np
+import torch
+
+import oracle
+import workloads as WL
+from bit_adam_error_b200 import OneBitAdam
+
+RTOL = 1e-5
+HP = dict(lr=1e-4, beta1=0.9, beta2=0.999, eps=1e-8)
+F = {k: np.float32(v) for k, v in HP.items()}
+
+
+def dev():
+    return torch.device("cuda", 0)
+
+
+def to_dev(a: np.ndarray) -> torch.Tensor:
+    if a.dtype == np.uint16:
+        return torch.from_numpy(a.view(np.int16).copy()).to(dev()).view(torch.bfloat16)
+    if a.dtype == np.uint32:
+        return torch.from_numpy(a.view(np.int32).copy()).to(dev())
+    return torch.from_numpy(np.ascontiguousarray(a)).to(dev())
+
+
+def np_of(t: torch.Tensor) -> np.ndarray:
+    a = t.detach().cpu().contiguous().numpy()
+    return a.view(np.uint32) if a.dtype == np.int32 else a
+
+
+def assert_bits(name, got: np.ndarray, ref: np.ndarray):
+    got, ref = np.asarray(got, np.uint32), np.asarray(ref, np.uint32)
+    assert got.shape == ref.shape, (name, got.shape, ref.shape)
+    bad = np.nonzero(got != ref)
+    assert bad[0].size == 0, f"{name}: {bad[0].size} words differ, first at {tuple(b[0] for b in bad)}"
+
+
+def assert_scales(name, got, ref, rtol=RTOL):
+    got, ref = np.asarray(got, np.float64), np.asarray(ref, np.float64)
+    same_nan = np.isnan(got) & np.isnan(ref)
+    with np.errstate(invalid="ignore"):
+        ok = same_nan | (got == ref) | (np.abs(got - ref) <= rtol * np.abs(ref))
+    assert ok.all(), f"{name}: max rel err {np.nanmax(np.abs(got - ref) / np.maximum(np.abs(ref), 1e-300))}"
+
+
+def assert_state(name, got, ref, offsets, rtol=RTOL):
+    got = np.atleast_2d(np.asarray(got, np.float64))
+    ref = np.atleast_2d(np.asarray(ref, np.float64))
+    assert got.shape == ref.shape, (name, got.shape, ref.shape)
+    for r in range(ref.shape[0]):
+        for k in range(len(offsets) - 1):
+            lo, hi = int(offsets[k]), int(offsets[k + 1])
+            if hi == lo:
+                continue
+            g, x = got[r, lo:hi], ref[r, lo:hi]
+            fin = np.isfinite(x)
+            assert np.array_equal(np.isnan(g), np.isnan(x)), f"{name}[{r}] chunk {k}: NaN pattern"
+            inf = np.isinf(x)
+            assert np.array_equal(g[inf], x[inf]), f"{name}[{r}] chunk {k}: infinities differ"
+            if not fin.any():
+                continue
+            rms = np.sqrt(np.mean(x[fin] ** 2))
+            bound = rtol * np.maximum(np.abs(x[fin]), rms)
+            err = np.abs(g[fin] - x[fin])
+            assert (err <= bound).all(), (
+                f"{name}[{r}] chunk {k}: max |diff| {err.max():.3e} vs bound {bound[np.argmax(err - bound)]:.3e}")
+
+
+class Pair:
+    """A GPU optimizer and the oracle state it is compared with."""
+
+    def __init__(self, offsets: Sequence[int], W: int, *, grad_dtype="f32", optimizer="adam",
+                 clip=0.0, freeze_step=0, p0: Optional[np.ndarray] = None,
+                 v0: Optional[np.ndarray] = None, m0: Optional[np.ndarray] = None,
+                 err0: Optional[np.ndarray] = None, srv0: Optional[np.ndarray] = None):
+        self.off = np.asarray(offsets, np.int64)
+        self.n = int(self.off[-1])
+        self.W = W
+        self.clip = clip
+        self.optimizer = optimizer
+        self.orc = oracle.get()
+        n = self.n
+        p0 = np.zeros(n, np.float32) if p0 is None else p0
+        v0 = np.zeros(n, np.float32) if v0 is None else v0
+        m0 = np.zeros(n, np.float32) if m0 is None else m0
+        err0 = np.zeros((W, n), np.float32) if err0 is None else err0
+        srv0 = np.zeros(n, np.float32) if srv0 is None else srv0
+        self.gpu = OneBitAdam(self.off, W, grad_dtype=grad_dtype, optimizer=optimizer, clip=clip,
+                              freeze_step=freeze_step, device=dev(), p=to_dev(p0),
+                              m=to_dev(m0), v=to_dev(v0), **HP)
+        if err0.any():
+            self.gpu.err.copy_(to_dev(err0))
+        if srv0.any():
+            self.gpu.srv_err.copy_(to_dev(srv0))
+        self.ref: Dict[str, np.ndarray] = {"p": p0.copy(), "m": m0.copy(), "v": v0.copy(),
+                                           "err": err0.copy(), "srv_err": srv0.copy()}
+        self.ref_flags = 0
+
+    @property
+    def opt_code(self):
+        return oracle.LAMB if self.optimizer == "lamb" else oracle.ADAM
+
+    def step(self, g: np.ndarray, warm: bool) -> None:
+        self.gpu.step(to_dev(g))
+        r = self.ref
+        if warm:
+            self.ref_flags |= self.orc.warmup(self.off, g, r["m"], r["v"], r["p"], F["beta1"],
+                                              F["beta2"], F["lr"], F["eps"], optimizer=self.opt_code)
+        else:
+            self.ref_flags |= self.orc.step(self.off, g, r, F["beta1"], F["lr"], F["eps"],
+                                            clip=self.clip, optimizer=self.opt_code)
+
+    def compare(self, what=("p", "m", "v", "err", "srv_err"), bits=True, tag=""):
+        torch.cuda.synchronize()
+        for k in what:
+            got = np_of(getattr(self.gpu, k))
+            assert_state(f"{tag}{k}", got, self.ref[k].reshape(got.shape), self.off)
+        if bits and "bits_w" in self.ref:
+            assert_bits(f"{tag}bits_w", np_of(self.gpu.bits_w), self.ref["bits_w"])
+            assert_bits(f"{tag}bits_srv", np_of(self.gpu.bits_srv), self.ref["bits_srv"])
+            assert_scales(f"{tag}s_w", np_of(self.gpu.s_w), self.ref["s_w"])
+            assert_scales(f"{tag}s_srv", np_of(self.gpu.s_srv), self.ref["s_srv"])
+
+    def exact(self) -> bool:
+        """True when every state tensor equals the oracle's bit for bit."""
+        torch.cuda.synchronize()
+        return all(np.array_equal(np_of(getattr(self.gpu, k)).reshape(-1), self.ref[k].reshape(-1))
+                   for k in ("p", "m", "v", "err", "srv_err"))
+
+
+def grads_for(wl: WL.Workload, step: int) -> np.ndarray:
+    dt = np.uint16 if wl.grad_dtype == "bf16" else np.float32
+    g = np.zeros((wl.W, wl.n), dt)
+    WL.fill_grads(wl, step, g)
+    return g
+
+
+def state_for(wl: WL.Workload):
+    p = np.zeros(wl.n, np.float32)
+    v = np.zeros(wl.n, np.float32)
+    WL.fill_state(wl, p, v)
+    return p, v

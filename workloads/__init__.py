@@ -11,6 +11,7 @@ from .gen import (  # noqa: F401
     chunk_grads,
     chunk_state,
     fill_grads,
+    fill_grads_row,
     fill_state,
     f32_to_bf16_bits,
     bf16_bits_to_f32,

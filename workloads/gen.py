@@ -119,22 +119,32 @@ def _threads() -> int:
     return max(1, min(32, os.cpu_count() or 1))
 
 
-def fill_grads(wl: Workload, step: int, out: np.ndarray, workers=None) -> None:
-    """Fill ``out`` (shape [W, n]; float32 or uint16) with the step's gradients."""
-    workers = range(wl.W) if workers is None else workers
+def fill_grads(wl: Workload, step: int, out: np.ndarray, workers=None, rows=None) -> None:
+    """Fill ``out`` (shape [W, n]; float32 or uint16) with the step's gradients.
+
+    ``workers`` selects which workers to generate; ``rows`` (same length) the
+    rows of ``out`` they go to (default: row = worker).
+    """
+    workers = list(range(wl.W)) if workers is None else list(workers)
+    rows = workers if rows is None else list(rows)
     off = wl.offsets
-    jobs = [(w, k, b, lo, hi) for w in workers for k in range(wl.C)
+    jobs = [(w, r, k, b, lo, hi) for w, r in zip(workers, rows) for k in range(wl.C)
             for b, lo, hi in _blocks(wl.sizes[k])]
 
     def run(job):
-        w, k, b, lo, hi = job
+        w, r, k, b, lo, hi = job
         g = _grad_block(wl, step, w, k, b, hi - lo)
         if wl.grad_dtype == "bf16":
             g = f32_to_bf16_bits(g)
-        out[w, off[k] + lo: off[k] + hi] = g
+        out[r, off[k] + lo: off[k] + hi] = g
 
     with ThreadPoolExecutor(_threads()) as ex:
         list(ex.map(run, jobs))
+
+
+def fill_grads_row(wl: Workload, step: int, worker: int, out: np.ndarray) -> None:
+    """Fill the flat row ``out`` (length n) with one worker's gradients at ``step``."""
+    fill_grads(wl, step, out.reshape(1, -1), workers=[worker], rows=[0])
 
 
 def fill_state(wl: Workload, p_out: np.ndarray, v_out: Optional[np.ndarray]) -> None:
