@@ -45,6 +45,7 @@ import numpy as np  # noqa: E402
 METRIC = "compressed-phase 1-bit Adam step: Gelem/s and HBM GB/s as % of B200 peak"
 UNIT = "Gelem/s"
 FALLBACK_HBM_GBS = 6650.0
+E2E_MAX_HOST_BYTES = 16e9        # pinned host gradients per step the e2e leg may hold
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "ncu_traffic.txt")
 KERNEL_SOURCES = [os.path.join(ROOT, "bit_adam_error_b200", "csrc", f)
                   for f in ("kernels.cuh", "onebit.cu")]
@@ -57,6 +58,8 @@ def parse_args():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="gpt2xl-flat")
+    ap.add_argument("--chunks", type=int, default=0,
+                    help="use only the first K chunks of the workload (a smaller case, e.g. for ncu)")
     ap.add_argument("--grad-buffers", type=int, default=2,
                     help="distinct gradient batches cycled through the timed steps")
     ap.add_argument("--no-e2e", action="store_true")
@@ -255,8 +258,7 @@ def run_reference(args):
     world, rank, local = dist_env()
     if rank != 0:
         return 0
-    import workloads as WL
-    wl = WL.get_workload(args.workload)
+    wl = select_workload(args)
     sample = 1 << 23
     elems, secs, per_step, used = oracle_rate(wl, [0], max_elems=sample, steps=args.warmup + args.steps)
     timed = per_step[args.warmup:]
@@ -273,6 +275,16 @@ def run_reference(args):
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
+
+
+def select_workload(args):
+    import workloads as WL
+    wl = WL.get_workload(args.workload)
+    if args.chunks:
+        k = min(args.chunks, wl.C)
+        wl = wl.with_(sizes=wl.sizes[:k], name=f"{wl.name}-first{k}",
+                      description=f"first {k} chunk(s) of {wl.name} ({wl.description})")
+    return wl
 
 
 def workload_config(wl, n_gpus):
@@ -296,28 +308,31 @@ def run_ours(args):
     import workloads as WL
     from bit_adam_error_b200 import OneBitAdam, _lib as L
 
-    wl = WL.get_workload(args.workload)
+    wl = select_workload(args)
     n, W = wl.n, wl.W
     gdt = torch.bfloat16 if wl.grad_dtype == "bf16" else torch.float32
 
-    # State: seeded p, v on the host, uploaded once.
-    p_h = np.empty(n, np.float32)
-    v_h = np.empty(n, np.float32)
-    WL.fill_state(wl.with_(freeze_step=0), p_h, v_h)
+    # State: seeded p, v generated a chunk group at a time and uploaded once.
     opt = OneBitAdam(wl.offsets, W, grad_dtype=wl.grad_dtype, optimizer=wl.optimizer, clip=wl.clip,
                      freeze_step=0, lr=wl.lr, beta1=wl.beta1, beta2=wl.beta2, eps=wl.eps,
-                     device=device, p=torch.from_numpy(p_h).to(device), v=torch.from_numpy(v_h).to(device))
+                     device=device)
+    swl = wl.with_(freeze_step=0)
+    for k0, k1 in WL.chunk_groups(wl):
+        lo, hi = int(wl.offsets[k0]), int(wl.offsets[k1])
+        p_h = np.empty(hi - lo, np.float32)
+        v_h = np.empty(hi - lo, np.float32)
+        WL.fill_state(swl, p_h, v_h, chunks=(k0, k1))
+        opt.p[lo:hi].copy_(torch.from_numpy(p_h))
+        opt.v[lo:hi].copy_(torch.from_numpy(v_h))
     del p_h, v_h
 
-    # Gradient batches: generated into pinned host buffers (kept for e2e), copied to HBM.
+    # Gradient batches in HBM (distinct seeded steps), generated a chunk group at a time.
     nbuf = max(1, args.grad_buffers)
-    host_g, dev_g = [], []
+    dev_g = []
     for b in range(nbuf):
-        h = torch.empty((W, n), dtype=gdt, pin_memory=True)
-        arr = h.view(torch.int16).numpy().view(np.uint16) if wl.grad_dtype == "bf16" else h.numpy()
-        WL.fill_grads(wl, b + 1000 * rank, arr)
-        host_g.append(h)
-        dev_g.append(h.to(device))
+        G = torch.empty((W, n), dtype=gdt, device=device)
+        fill_device_grads(wl, b + 1000 * rank, G)
+        dev_g.append(G)
     stream = torch.cuda.current_stream(device)
 
     for i in range(args.warmup):
@@ -370,23 +385,36 @@ def run_ours(args):
 
     # -- end to end: host gradients through the public call ---------------------------
     e2e = None
-    if not args.no_e2e:
+    host_bytes = W * n * wl.grad_bytes
+    if not args.no_e2e and host_bytes > E2E_MAX_HOST_BYTES:
+        e2e = {"value": None, "unit": UNIT, "note": f"skipped: {host_bytes / 1e9:.1f} GB of pinned host "
+               f"gradients per step exceeds the {E2E_MAX_HOST_BYTES / 1e9:.0f} GB cap"}
+    elif not args.no_e2e:
+        # Pinned host copies of the gradient batches, filled from the same seeded streams.
+        host_g = []
+        for b in range(min(nbuf, 2)):
+            h = torch.empty((W, n), dtype=gdt, pin_memory=True)
+            arr = h.view(torch.int16).numpy().view(np.uint16) if wl.grad_dtype == "bf16" else h.numpy()
+            WL.fill_grads(wl, b + 1000 * rank, arr)
+            host_g.append(h)
+        nh = len(host_g)
         s_host = torch.empty(wl.C, dtype=torch.float32, pin_memory=True)
         for i in range(2):
-            opt.step(host_g[i % nbuf])
+            opt.step(host_g[i % nh])
         torch.cuda.synchronize()
         barrier(dist)
         torch.cuda.synchronize()
         e0.record(stream)
         for i in range(args.steps):
-            opt.step(host_g[i % nbuf])
+            opt.step(host_g[i % nh])
             s_host.copy_(opt.s_srv, non_blocking=True)
         e1.record(stream)
         torch.cuda.synchronize()
         barrier(dist)
         ms_e2e = max_over_ranks(dist, e0.elapsed_time(e1) / args.steps, device)
         e2e = {"value": world * n / (ms_e2e / 1e3) / 1e9, "unit": UNIT, "ms_per_step": ms_e2e,
-               "h2d_bytes_per_step": W * n * wl.grad_bytes, "d2h_bytes_per_step": 4 * wl.C}
+               "h2d_bytes_per_step": host_bytes, "d2h_bytes_per_step": 4 * wl.C}
+        del host_g
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -412,6 +440,21 @@ def run_ours(args):
     if dist is not None:
         dist.destroy_process_group()
     return 0
+
+
+def fill_device_grads(wl, step, G) -> None:
+    """Seeded gradients of one step into the device tensor G [W, n], a worker row
+    and a chunk group at a time."""
+    import torch
+    import workloads as WL
+    bf = wl.grad_dtype == "bf16"
+    for w in range(wl.W):
+        for k0, k1 in WL.chunk_groups(wl):
+            lo, hi = int(wl.offsets[k0]), int(wl.offsets[k1])
+            row = np.empty(hi - lo, np.uint16 if bf else np.float32)
+            WL.fill_grads_row(wl, step, w, row, chunks=(k0, k1))
+            src = torch.from_numpy(row.view(np.int16)).view(torch.bfloat16) if bf else torch.from_numpy(row)
+            G[w, lo:hi].copy_(src)
 
 
 def gpu_id(device) -> str:

@@ -154,3 +154,28 @@ def state_for(wl: WL.Workload):
     v = np.zeros(wl.n, np.float32)
     WL.fill_state(wl, p, v)
     return p, v
+
+
+def upload_state(wl: WL.Workload, p_dev: torch.Tensor, v_dev: torch.Tensor) -> None:
+    """Seeded initial p, v of the workload into device tensors, a chunk group at a
+    time (bounded host memory)."""
+    for k0, k1 in WL.chunk_groups(wl):
+        lo, hi = int(wl.offsets[k0]), int(wl.offsets[k1])
+        p = np.empty(hi - lo, np.float32)
+        v = np.empty(hi - lo, np.float32)
+        WL.fill_state(wl, p, v, chunks=(k0, k1))
+        p_dev[lo:hi].copy_(torch.from_numpy(p))
+        v_dev[lo:hi].copy_(torch.from_numpy(v))
+
+
+def upload_grads(wl: WL.Workload, step: int, G: torch.Tensor) -> None:
+    """The step's gradients into the device tensor G [W, n], a worker row and a
+    chunk group at a time."""
+    bf = wl.grad_dtype == "bf16"
+    for w in range(wl.W):
+        for k0, k1 in WL.chunk_groups(wl):
+            lo, hi = int(wl.offsets[k0]), int(wl.offsets[k1])
+            row = np.empty(hi - lo, np.uint16 if bf else np.float32)
+            WL.fill_grads_row(wl, step, w, row, chunks=(k0, k1))
+            src = torch.from_numpy(row.view(np.int16)).view(torch.bfloat16) if bf else torch.from_numpy(row)
+            G[w, lo:hi].copy_(src)

@@ -16,20 +16,10 @@ import torch
 import oracle
 import workloads as WL
 from bit_adam_error_b200 import OneBitAdam
-from gpu_harness import F, HP, assert_bits, assert_scales, assert_state, dev, np_of
+from gpu_harness import (F, HP, assert_bits, assert_scales, assert_state, dev, np_of,
+                         upload_grads, upload_state)
 
 pytestmark = [pytest.mark.gpu, pytest.mark.slow]
-
-
-def fill_device_grads(wl, step, G):
-    """Generate the step's gradients row by row into the device tensor G [W, n]."""
-    dt = np.uint16 if wl.grad_dtype == "bf16" else np.float32
-    row = np.zeros(wl.n, dt)
-    for w in range(wl.W):
-        WL.fill_grads_row(wl, step, w, row)
-        src = torch.from_numpy(row.view(np.int16)).view(torch.bfloat16) if dt == np.uint16 \
-            else torch.from_numpy(row)
-        G[w].copy_(src)
 
 
 def sampled_chunks(wl):
@@ -42,17 +32,13 @@ def test_full_size_sampled_chunks(name):
     wl = WL.get_workload(name)
     steps = wl.freeze_step + 1
     torch.cuda.empty_cache()
-    p = np.zeros(wl.n, np.float32)
-    v = np.zeros(wl.n, np.float32)
-    WL.fill_state(wl, p, v)
     opt = OneBitAdam(wl.offsets, wl.W, grad_dtype=wl.grad_dtype, optimizer=wl.optimizer,
-                     clip=wl.clip, freeze_step=wl.freeze_step, device=dev(),
-                     p=torch.from_numpy(p).to(dev()), v=torch.from_numpy(v).to(dev()), **HP)
-    del p, v
+                     clip=wl.clip, freeze_step=wl.freeze_step, device=dev(), **HP)
+    upload_state(wl, opt.p, opt.v)
     gdt = torch.bfloat16 if wl.grad_dtype == "bf16" else torch.float32
     G = torch.empty((wl.W, wl.n), dtype=gdt, device=dev())
     for t in range(steps):
-        fill_device_grads(wl, t, G)
+        upload_grads(wl, t, G)
         opt.step(G)
     torch.cuda.synchronize()
     assert opt.status() == 0

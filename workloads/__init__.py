@@ -10,6 +10,7 @@ from .configs import WORKLOADS, Workload, get_workload  # noqa: F401
 from .gen import (  # noqa: F401
     chunk_grads,
     chunk_state,
+    chunk_groups,
     fill_grads,
     fill_grads_row,
     fill_state,

@@ -119,16 +119,32 @@ def _threads() -> int:
     return max(1, min(32, os.cpu_count() or 1))
 
 
-def fill_grads(wl: Workload, step: int, out: np.ndarray, workers=None, rows=None) -> None:
+def chunk_groups(wl: Workload, max_elems: int = 1 << 28):
+    """Consecutive chunk ranges [k0, k1) holding at most max_elems elements each
+    (a single larger chunk forms a group of its own)."""
+    k0, tot = 0, 0
+    for k, s in enumerate(wl.sizes):
+        if k > k0 and tot + s > max_elems:
+            yield k0, k
+            k0, tot = k, 0
+        tot += s
+    if k0 < wl.C:
+        yield k0, wl.C
+
+
+def fill_grads(wl: Workload, step: int, out: np.ndarray, workers=None, rows=None,
+               chunks=None) -> None:
     """Fill ``out`` (shape [W, n]; float32 or uint16) with the step's gradients.
 
     ``workers`` selects which workers to generate; ``rows`` (same length) the
-    rows of ``out`` they go to (default: row = worker).
+    rows of ``out`` they go to (default: row = worker).  ``chunks = (k0, k1)``
+    restricts it to those chunks; ``out`` then holds only their elements.
     """
     workers = list(range(wl.W)) if workers is None else list(workers)
     rows = workers if rows is None else list(rows)
-    off = wl.offsets
-    jobs = [(w, r, k, b, lo, hi) for w, r in zip(workers, rows) for k in range(wl.C)
+    k0, k1 = (0, wl.C) if chunks is None else chunks
+    off = wl.offsets - wl.offsets[k0]
+    jobs = [(w, r, k, b, lo, hi) for w, r in zip(workers, rows) for k in range(k0, k1)
             for b, lo, hi in _blocks(wl.sizes[k])]
 
     def run(job):
@@ -142,15 +158,18 @@ def fill_grads(wl: Workload, step: int, out: np.ndarray, workers=None, rows=None
         list(ex.map(run, jobs))
 
 
-def fill_grads_row(wl: Workload, step: int, worker: int, out: np.ndarray) -> None:
-    """Fill the flat row ``out`` (length n) with one worker's gradients at ``step``."""
-    fill_grads(wl, step, out.reshape(1, -1), workers=[worker], rows=[0])
+def fill_grads_row(wl: Workload, step: int, worker: int, out: np.ndarray, chunks=None) -> None:
+    """Fill the flat row ``out`` with one worker's gradients at ``step`` (all
+    chunks, or chunks = (k0, k1) only)."""
+    fill_grads(wl, step, out.reshape(1, -1), workers=[worker], rows=[0], chunks=chunks)
 
 
-def fill_state(wl: Workload, p_out: np.ndarray, v_out: Optional[np.ndarray]) -> None:
-    """Fill flat ``p_out`` / ``v_out`` (float32, length n) with the initial state."""
-    off = wl.offsets
-    jobs = [(k, b, lo, hi) for k in range(wl.C) for b, lo, hi in _blocks(wl.sizes[k])]
+def fill_state(wl: Workload, p_out: np.ndarray, v_out: Optional[np.ndarray], chunks=None) -> None:
+    """Fill flat ``p_out`` / ``v_out`` (float32) with the initial state of all
+    chunks (length n) or of chunks = (k0, k1) only."""
+    k0, k1 = (0, wl.C) if chunks is None else chunks
+    off = wl.offsets - wl.offsets[k0]
+    jobs = [(k, b, lo, hi) for k in range(k0, k1) for b, lo, hi in _blocks(wl.sizes[k])]
 
     def run(job):
         k, b, lo, hi = job
