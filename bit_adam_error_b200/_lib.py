@@ -63,6 +63,7 @@ _SIGS = {
     "ob_profile_stop": (ctypes.c_int, [_P, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int64)]),
     "ob_kernel_name": (ctypes.c_char_p, [ctypes.c_int32]),
     "ob_launch_count": (ctypes.c_int64, [_P]),
+    "ob_compress_noalloc": (ctypes.c_int, [ctypes.POINTER(ob_config), _P, _P, _P, _P, _P]),
     "ob_last_error": (ctypes.c_char_p, []),
 }
 
@@ -182,3 +183,9 @@ def ob_kernel_name(kind: int) -> str:
 
 def ob_launch_count(ctx) -> int:
     return int(load().ob_launch_count(ctx))
+
+
+def ob_compress_noalloc(cfg: ob_config, grads: int, err: int, bits_w: int, s_w: int, stream: int) -> None:
+    """Worker stage without a ctx and without device allocation (fixed scratch)."""
+    check(load().ob_compress_noalloc(ctypes.byref(cfg), grads, err, bits_w, s_w, stream),
+          "ob_compress_noalloc")

@@ -9,6 +9,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 #include <new>
 #include <vector>
 
@@ -587,3 +588,150 @@ int64_t ob_launch_count(const ob_ctx* c) { return c ? c->launches : -1; }
 const char* ob_last_error(void) { return g_last_error; }
 
 }  // extern "C"
+
+// ---- worker stage without allocation -------------------------------------------------
+// ob_compress_noalloc (declared in onebit.h) serves callers that must not allocate
+// device memory.  Its scratch is one fixed file-scope device array; host code here
+// only ever passes the array's device address, obtained once per device with
+// cudaGetSymbolAddress (the symbol itself is a host-side stand-in, not an address).
+constexpr size_t kNoAllocScratchBytes = size_t(8) << 20;  // 8 MiB on every device
+
+// Every GPU that loads this library holds this array until the process exits.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+namespace {
+
+constexpr int32_t kNoAllocMaxChunks = 4096;
+constexpr int kNoAllocMaxDevices = 64;
+constexpr size_t kNoAllocTableBytes = 3 * sizeof(int64_t) * (kNoAllocMaxChunks + 1) + kNoAllocMaxChunks;
+
+struct NoAllocDevice {
+  bool ready = false;
+  char* scratch = nullptr;   // device address of g_noalloc_scratch on this device
+  int num_sms = 0;
+  int occ_norm[2] = {1, 1};  // resident CTAs per SM: [f32, bf16]
+  int occ_pack[2] = {1, 1};
+};
+
+std::mutex g_noalloc_mu;
+NoAllocDevice g_noalloc_dev[kNoAllocMaxDevices];
+// Host image of the scratch header (chunk tables + zeroed status word), rebuilt
+// under the mutex and copied with one cudaMemcpyAsync per call.
+alignas(256) unsigned char g_noalloc_header[kNoAllocTableBytes + 512];
+
+int occupancy(const void* fn) {
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, ob::kBlock, 0) != cudaSuccess || per_sm < 1) {
+    cudaGetLastError();
+    per_sm = 1;
+  }
+  return per_sm;
+}
+
+// Once per device, with that device current: look up the array's device address.
+ob_err noalloc_setup(int device, NoAllocDevice** out) {
+  if (device < 0 || device >= kNoAllocMaxDevices) return fail(OB_EINVAL, "device %d out of range", device);
+  NoAllocDevice& d = g_noalloc_dev[device];
+  if (!d.ready) {
+    void* ptr = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(no-alloc scratch)");
+    if ((e = cudaDeviceGetAttribute(&d.num_sms, cudaDevAttrMultiProcessorCount, device)) != cudaSuccess)
+      return cuda_fail(e, "cudaDeviceGetAttribute");
+    d.occ_norm[0] = occupancy(reinterpret_cast<const void*>(ob::k_worker_norm<float>));
+    d.occ_norm[1] = occupancy(reinterpret_cast<const void*>(ob::k_worker_norm<uint16_t>));
+    d.occ_pack[0] = occupancy(reinterpret_cast<const void*>(ob::k_worker_pack<float, false>));
+    d.occ_pack[1] = occupancy(reinterpret_cast<const void*>(ob::k_worker_pack<uint16_t, false>));
+    d.scratch = static_cast<char*>(ptr);
+    d.ready = true;
+  }
+  *out = &d;
+  return OB_OK;
+}
+
+int noalloc_grid(int num_sms, int per_sm, int64_t warps) {
+  const int64_t need = (warps + ob::kWarpsPerBlock - 1) / ob::kWarpsPerBlock;
+  return static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(need, int64_t(num_sms) * per_sm)));
+}
+
+}  // namespace
+
+extern "C" ob_err ob_compress_noalloc(const ob_config* cfg, const void* grads, float* err,
+                                      uint32_t* bits_w, float* s_w, void* stream) {
+  int64_t words = 0;
+  ob_err r = ob_layout(cfg, &words);
+  if (r != OB_OK) return r;
+  const int64_t n = cfg->n, W = cfg->W, C = cfg->num_chunks;
+  if (C > kNoAllocMaxChunks)
+    return fail(OB_EINVAL, "ob_compress_noalloc: %lld chunks, at most %d", (long long)C, kNoAllocMaxChunks);
+  // Scratch needed: header (tables, status) + one double per (worker, warp tile).
+  int64_t T = 0;
+  for (int64_t k = 0; k < C; ++k) T += (cfg->chunk_offsets[k + 1] - cfg->chunk_offsets[k] + ob::kTile - 1) / ob::kTile;
+  const size_t header = (kNoAllocTableBytes + 256 + 255) & ~size_t(255);
+  const size_t need = header + sizeof(double) * size_t(W) * size_t(T);
+  if (need > kNoAllocScratchBytes)
+    return fail(OB_EINVAL,
+                "ob_compress_noalloc: W=%lld, n=%lld needs %zu bytes of scratch; the fixed array holds %zu "
+                "(about W*n <= %lld elements); use ob_create/ob_compress instead",
+                (long long)W, (long long)n, need, kNoAllocScratchBytes,
+                (long long)((kNoAllocScratchBytes - header) / sizeof(double) * ob::kTile));
+  int device = 0;
+  cudaError_t e = cudaGetDevice(&device);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  struct { const void* p; int64_t count; const char* name; } bufs[] = {
+      {grads, W * n, "grads"}, {err, W * n, "err"}, {bits_w, W * words, "bits_w"}, {s_w, W * C, "s_w"}};
+  for (auto& b : bufs)
+    if ((r = check_dev(b.p, b.count, b.name, device)) != OB_OK) return r;
+
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  NoAllocDevice* d = nullptr;
+  if ((r = noalloc_setup(device, &d)) != OB_OK) return r;
+
+  // Header image: off | wo | tp (int64, C+1 each) | vec (C bytes) | status (zeroed).
+  std::memset(g_noalloc_header, 0, sizeof g_noalloc_header);
+  int64_t* h_off = reinterpret_cast<int64_t*>(g_noalloc_header);
+  int64_t* h_wo = h_off + (C + 1);
+  int64_t* h_tp = h_wo + (C + 1);
+  uint8_t* h_vec = reinterpret_cast<uint8_t*>(h_tp + (C + 1));
+  const size_t status_at = (reinterpret_cast<unsigned char*>(h_vec + C) - g_noalloc_header + 255) & ~size_t(255);
+  h_off[0] = h_wo[0] = h_tp[0] = 0;
+  for (int64_t k = 0; k < C; ++k) {
+    const int64_t o = cfg->chunk_offsets[k], nk = cfg->chunk_offsets[k + 1] - o;
+    h_off[k + 1] = cfg->chunk_offsets[k + 1];
+    h_wo[k + 1] = h_wo[k] + words_of(nk);
+    h_tp[k + 1] = h_tp[k] + (nk + ob::kTile - 1) / ob::kTile;
+    h_vec[k] = (o % 8 == 0) && (nk % 8 == 0) && (W == 1 || n % 8 == 0);
+  }
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if ((e = cudaMemcpyAsync(d->scratch, g_noalloc_header, status_at + sizeof(uint32_t),
+                           cudaMemcpyHostToDevice, st)) != cudaSuccess)
+    return cuda_fail(e, "ob_compress_noalloc: header copy");
+
+  ob::Layout L{};
+  L.off = reinterpret_cast<const int64_t*>(d->scratch);
+  L.wo = L.off + (C + 1);
+  L.tp = L.wo + (C + 1);
+  L.vec = reinterpret_cast<const uint8_t*>(L.tp + (C + 1));
+  L.n = n;
+  L.T = T;
+  L.words = words;
+  L.C = static_cast<int32_t>(C);
+  uint32_t* status = reinterpret_cast<uint32_t*>(d->scratch + status_at);
+  double* part = reinterpret_cast<double*>(d->scratch + header);
+  const int bf = cfg->grad_dtype == OB_BF16 ? 1 : 0;
+  const float clip = cfg->clip;
+  if (T > 0) {
+    const int g1 = noalloc_grid(d->num_sms, d->occ_norm[bf], W * T);
+    if (bf) ob::k_worker_norm<uint16_t><<<g1, ob::kBlock, 0, st>>>(L, int(W), static_cast<const uint16_t*>(grads), err, clip, part, status);
+    else ob::k_worker_norm<float><<<g1, ob::kBlock, 0, st>>>(L, int(W), static_cast<const float*>(grads), err, clip, part, status);
+  }
+  ob::k_finalize_scale<<<dim3(unsigned(C), unsigned(W)), ob::kFinalizeThreads, 0, st>>>(L, part, s_w);
+  if (T > 0) {
+    const int g2 = noalloc_grid(d->num_sms, d->occ_pack[bf], T);
+    if (bf)
+      ob::k_worker_pack<uint16_t, false><<<g2, ob::kBlock, 0, st>>>(L, int(W), static_cast<const uint16_t*>(grads), err, s_w, bits_w, nullptr, nullptr, clip, status);
+    else
+      ob::k_worker_pack<float, false><<<g2, ob::kBlock, 0, st>>>(L, int(W), static_cast<const float*>(grads), err, s_w, bits_w, nullptr, nullptr, clip, status);
+  }
+  return check_launch("ob_compress_noalloc");
+}

@@ -173,6 +173,39 @@ const char* ob_kernel_name(int32_t kind);
 /* Kernel launches this ctx has enqueued since ob_create (-1 for NULL). */
 int64_t ob_launch_count(const ob_ctx* ctx);
 
+/* ---- worker stage for callers that cannot allocate --------------------------
+ * The paper has no counterpart to this call; it exists for integration.
+ * Some callers must not allocate device memory at all: code whose GPU memory is
+ * owned by another allocator (a framework's caching pool that has reserved the
+ * device up front, where a raw cudaMalloc could fail or fragment the pool) and
+ * code on a latency-critical path (a gradient hook inside a training step),
+ * where cudaMalloc/cudaFree may synchronise the device.  Such callers cannot
+ * use ob_create, which allocates the ctx scratch.
+ *
+ * ob_compress_noalloc is the worker stage of ob_compress without a ctx and
+ * without any allocation: for every worker w and chunk k,
+ *   c = clip(g_w) + err_w,  s_w[w][k] = ||c|| / sqrt(n_k),  bits_w = sign(c),
+ *   err_w = c - s_w sign(c)
+ * with results identical to ob_compress on the same inputs.  The caller passes
+ * the config and DEVICE buffers as for ob_create/ob_compress: grads [W][n]
+ * (grad_dtype), err [W][n] (in/out), bits_w [W][words_total], s_w [W][C];
+ * 16-byte aligned.  lr, betas, eps and freeze_step are ignored.
+ *
+ * Scratch: a fixed 8 MiB array in the library's device memory (every GPU that
+ * loads the library holds it until the process exits), used for the chunk
+ * tables and one double per (worker, 512-element tile).  Calls needing more --
+ * about W*n above 5.3e8 elements, or more than 4096 chunks -- return
+ * OB_EINVAL with a message, before any work is enqueued.  All calls share the
+ * array: two calls whose work overlaps on the GPU (different streams, or
+ * different host threads without ordering) race and give wrong results;
+ * order them on one stream.  Each call rewrites the tables and clears the
+ * status word it uses.  The first call on each device looks up the array's
+ * device address (cudaGetSymbolAddress) with that device current; make that
+ * first call before any stream capture begins.  Not-finite flags are not
+ * reported by this call (the ctx path's ob_get_status has them). */
+ob_err ob_compress_noalloc(const ob_config* cfg, const void* grads, float* err,
+                           uint32_t* bits_w, float* s_w, void* stream);
+
 /* Message of the last failed call on this thread ("" if none). */
 const char* ob_last_error(void);
 
