@@ -51,6 +51,8 @@ constexpr int kTileWords = kTile / 32;
 constexpr int kBlock = 256;                      // threads per CTA (8 warps)
 constexpr int kWarpsPerBlock = kBlock / kWarp;
 constexpr int kFinalizeThreads = 256;
+constexpr bool kWide = false;                    // 256-bit (v8.f32) global accesses for fp32 arrays
+constexpr int kPackGroupsInFlight = kGroups;     // pass 2: groups whose loads are issued together
 constexpr unsigned kFull = 0xffffffffu;
 constexpr uint32_t kStatusNonfinite = 1u;
 
@@ -58,10 +60,12 @@ constexpr uint32_t kStatusNonfinite = 1u;
 struct Layout {
   const int64_t* off;   // [C+1] first element of every chunk
   const int64_t* wo;    // [C+1] first word of every chunk within a packed row
-  const int64_t* tp;    // [C+1] first warp tile of every chunk
+  const int64_t* tp;    // [C+1] first warp tile (kTile elements) of every chunk
+  const int64_t* tpb;   // [C+1] first block tile (kBT elements, pipelined passes) of every chunk
   const uint8_t* vec;   // [C]   1: 8-wide vector path, 0: scalar path
   int64_t n;            // elements per row
   int64_t T;            // warp tiles per row
+  int64_t Tb;           // block tiles per row
   int64_t words;        // packed words per row
   int32_t C;
 };
@@ -107,10 +111,16 @@ __device__ __forceinline__ Tile tile_at(const Layout& L, int64_t t, int& hint) {
 // ---- element access ------------------------------------------------------------
 
 __device__ __forceinline__ void ld8_ro(const float* p, float (&x)[8]) {
-  const float4 a = __ldg(reinterpret_cast<const float4*>(p));
-  const float4 b = __ldg(reinterpret_cast<const float4*>(p) + 1);
-  x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
-  x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+  if constexpr (kWide) {
+    asm("ld.global.nc.L1::no_allocate.v8.f32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+        : "=f"(x[0]), "=f"(x[1]), "=f"(x[2]), "=f"(x[3]), "=f"(x[4]), "=f"(x[5]), "=f"(x[6]), "=f"(x[7])
+        : "l"(p));
+  } else {
+    const float4 a = __ldg(reinterpret_cast<const float4*>(p));
+    const float4 b = __ldg(reinterpret_cast<const float4*>(p) + 1);
+    x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
+    x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+  }
 }
 
 // bf16 -> fp32 is exact: the 16 bits are the top half of the float.
@@ -122,17 +132,30 @@ __device__ __forceinline__ void ld8_ro(const uint16_t* p, float (&x)[8]) {
   x[6] = __uint_as_float(u.w << 16); x[7] = __uint_as_float(u.w & 0xffff0000u);
 }
 
-// Read-write buffers: plain (coherent) loads.
+// Read-write buffers: plain (coherent) loads; each element is read once, then
+// written once by the same thread, so no load is ever moved past its store.
 __device__ __forceinline__ void ld8(const float* p, float (&x)[8]) {
-  const float4 a = reinterpret_cast<const float4*>(p)[0];
-  const float4 b = reinterpret_cast<const float4*>(p)[1];
-  x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
-  x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+  if constexpr (kWide) {
+    asm("ld.global.L1::no_allocate.v8.f32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+        : "=f"(x[0]), "=f"(x[1]), "=f"(x[2]), "=f"(x[3]), "=f"(x[4]), "=f"(x[5]), "=f"(x[6]), "=f"(x[7])
+        : "l"(p));
+  } else {
+    const float4 a = reinterpret_cast<const float4*>(p)[0];
+    const float4 b = reinterpret_cast<const float4*>(p)[1];
+    x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
+    x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+  }
 }
 
 __device__ __forceinline__ void st8(float* p, const float (&x)[8]) {
-  reinterpret_cast<float4*>(p)[0] = make_float4(x[0], x[1], x[2], x[3]);
-  reinterpret_cast<float4*>(p)[1] = make_float4(x[4], x[5], x[6], x[7]);
+  if constexpr (kWide) {
+    asm volatile("st.global.v8.f32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(p), "f"(x[0]), "f"(x[1]),
+                 "f"(x[2]), "f"(x[3]), "f"(x[4]), "f"(x[5]), "f"(x[6]), "f"(x[7])
+                 : "memory");
+  } else {
+    reinterpret_cast<float4*>(p)[0] = make_float4(x[0], x[1], x[2], x[3]);
+    reinterpret_cast<float4*>(p)[1] = make_float4(x[4], x[5], x[6], x[7]);
+  }
 }
 
 __device__ __forceinline__ float ld1_ro(const float* p) { return __ldg(p); }
@@ -237,8 +260,10 @@ k_worker_norm(Layout L, int W, const GT* __restrict__ grads, const float* __rest
 }
 
 // ---- finalize: per-chunk scale from tile partials ----------------------------------
-// out[r * C + k] = sqrt(sum_t part[r * T + t]) / sqrt(n_k), t over chunk k's tiles,
-// summed in a fixed order; 0 for an empty chunk.  grid = (C, R).
+// Partial slots of chunk k are [tpx[k] * mult, tpx[k+1] * mult) of each row (tpx =
+// warp-tile prefix with mult 1, or block-tile prefix with one slot per consumer
+// warp).  out[r * C + k] = sqrt(sum of the slots, fixed order) / sqrt(n_k); 0 for
+// an empty chunk.  grid = (C, R).
 __device__ __forceinline__ double block_sum_fixed(double x, double* sm) {
   const int tid = threadIdx.x;
   sm[tid] = x;
@@ -254,12 +279,13 @@ __device__ __forceinline__ double block_sum_fixed(double x, double* sm) {
 }
 
 __global__ void __launch_bounds__(kFinalizeThreads)
-k_finalize_scale(Layout L, const double* __restrict__ part, float* __restrict__ out) {
+k_finalize_scale(Layout L, const double* __restrict__ part, const int64_t* __restrict__ tpx,
+                 int mult, int64_t row_stride, float* __restrict__ out) {
   __shared__ double sm[kFinalizeThreads];
   const int k = blockIdx.x, r = blockIdx.y;
-  const double* pr = part + static_cast<int64_t>(r) * L.T;
+  const double* pr = part + static_cast<int64_t>(r) * row_stride;
   double acc = 0.0;
-  for (int64_t t = L.tp[k] + threadIdx.x; t < L.tp[k + 1]; t += kFinalizeThreads) acc += pr[t];
+  for (int64_t t = tpx[k] * mult + threadIdx.x; t < tpx[k + 1] * mult; t += kFinalizeThreads) acc += pr[t];
   const double S = block_sum_fixed(acc, sm);
   if (threadIdx.x == 0) {
     const int64_t nk = L.off[k + 1] - L.off[k];
@@ -272,11 +298,11 @@ k_finalize_scale(Layout L, const double* __restrict__ part, float* __restrict__ 
 // LAMB trust ratio per layer (chunk): r = sqrt(P) / sqrt(U), 1 if either is 0.  grid = C.
 __global__ void __launch_bounds__(kFinalizeThreads)
 k_finalize_ratio(Layout L, const double* __restrict__ partP, const double* __restrict__ partU,
-                 float* __restrict__ ratio) {
+                 const int64_t* __restrict__ tpx, int mult, float* __restrict__ ratio) {
   __shared__ double sm[kFinalizeThreads];
   const int k = blockIdx.x;
   double a = 0.0, b = 0.0;
-  for (int64_t t = L.tp[k] + threadIdx.x; t < L.tp[k + 1]; t += kFinalizeThreads) {
+  for (int64_t t = tpx[k] * mult + threadIdx.x; t < tpx[k + 1] * mult; t += kFinalizeThreads) {
     a += partP[t];
     b += partU[t];
   }
@@ -304,61 +330,65 @@ k_worker_pack(Layout L, int W, const GT* __restrict__ grads, float* __restrict__
     double tsum = 0.0;
     bool bad = false;
     if (tl.vec) {
-      float acc[kGroups][8], sv[kGroups][8];
-      bool in[kGroups];
+      constexpr int GP = kPackGroupsInFlight;
+#pragma unroll 1
+      for (int q0 = 0; q0 < kGroups; q0 += GP) {
+        float acc[GP][8], sv[GP][8];
+        bool in[GP];
 #pragma unroll
-      for (int q = 0; q < kGroups; ++q) {
-        const int64_t i0 = tl.rel + q * kGroupElems + lane * kVec;
-        in[q] = i0 < tl.nk;
-        zero8(acc[q]);
-        if (SERVER) {
-          if (in[q]) ld8_ro(srv_err + tl.ck0 + i0, sv[q]); else zero8(sv[q]);
-        }
-      }
-      for (int w = 0; w < W; ++w) {
-        const GT* g = grads + static_cast<int64_t>(w) * L.n + tl.ck0;
-        float* e = err + static_cast<int64_t>(w) * L.n + tl.ck0;
-        const float s = __ldg(s_w + static_cast<int64_t>(w) * L.C + tl.k);
-        float gv[kGroups][8], ev[kGroups][8];
-#pragma unroll
-        for (int q = 0; q < kGroups; ++q) {
-          const int64_t i0 = tl.rel + q * kGroupElems + lane * kVec;
-          if (in[q]) { ld8_ro(g + i0, gv[q]); ld8(e + i0, ev[q]); }
-          else { zero8(gv[q]); zero8(ev[q]); }
-        }
-#pragma unroll
-        for (int q = 0; q < kGroups; ++q) {
-          const int64_t i0 = tl.rel + q * kGroupElems + lane * kVec;
-          uint32_t byte = 0;
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const float c = clip_grad(gv[q][j], clip) + ev[q][j];
-            const bool b = c >= 0.0f;
-            const float d = signed_scale(b, s);
-            byte |= static_cast<uint32_t>(b) << j;
-            ev[q][j] = c - d;
-            acc[q][j] = acc[q][j] + d;
-            bad |= in[q] && !isfinite(c);
+        for (int u = 0; u < GP; ++u) {
+          const int64_t i0 = tl.rel + (q0 + u) * kGroupElems + lane * kVec;
+          in[u] = i0 < tl.nk;
+          zero8(acc[u]);
+          if (SERVER) {
+            if (in[u]) ld8_ro(srv_err + tl.ck0 + i0, sv[u]); else zero8(sv[u]);
           }
-          if (!in[q]) byte = 0;
-          else st8(e + i0, ev[q]);
-          const uint32_t word = quad_word(byte, lane);
-          const int64_t wrel = (tl.rel + q * kGroupElems) / 32 + (lane >> 2);
-          if ((lane & 3) == 0 && wrel * 32 < tl.nk)
-            bits_w[static_cast<int64_t>(w) * L.words + tl.w0 + wrel] = word;
         }
-      }
-      if (SERVER) {
+        for (int w = 0; w < W; ++w) {
+          const GT* g = grads + static_cast<int64_t>(w) * L.n + tl.ck0;
+          float* e = err + static_cast<int64_t>(w) * L.n + tl.ck0;
+          const float s = __ldg(s_w + static_cast<int64_t>(w) * L.C + tl.k);
+          float gv[GP][8], ev[GP][8];
 #pragma unroll
-        for (int q = 0; q < kGroups; ++q)
-          if (in[q]) {
+          for (int u = 0; u < GP; ++u) {
+            const int64_t i0 = tl.rel + (q0 + u) * kGroupElems + lane * kVec;
+            if (in[u]) { ld8_ro(g + i0, gv[u]); ld8(e + i0, ev[u]); }
+            else { zero8(gv[u]); zero8(ev[u]); }
+          }
+#pragma unroll
+          for (int u = 0; u < GP; ++u) {
+            const int64_t i0 = tl.rel + (q0 + u) * kGroupElems + lane * kVec;
+            uint32_t byte = 0;
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
-              const float cs = __fdiv_rn(acc[q][j], Wf) + sv[q][j];
-              tsum = fma(static_cast<double>(cs), static_cast<double>(cs), tsum);
-              bad |= !isfinite(cs);
+              const float c = clip_grad(gv[u][j], clip) + ev[u][j];
+              const bool b = c >= 0.0f;
+              const float d = signed_scale(b, s);
+              byte |= static_cast<uint32_t>(b) << j;
+              ev[u][j] = c - d;
+              acc[u][j] = acc[u][j] + d;
+              bad |= in[u] && !isfinite(c);
             }
+            if (!in[u]) byte = 0;
+            else st8(e + i0, ev[u]);
+            const uint32_t word = quad_word(byte, lane);
+            const int64_t wrel = (tl.rel + (q0 + u) * kGroupElems) / 32 + (lane >> 2);
+            if ((lane & 3) == 0 && wrel * 32 < tl.nk)
+              bits_w[static_cast<int64_t>(w) * L.words + tl.w0 + wrel] = word;
           }
+        }
+        if (SERVER) {
+#pragma unroll
+          for (int u = 0; u < GP; ++u)
+            if (in[u]) {
+#pragma unroll
+              for (int j = 0; j < 8; ++j) {
+                const float cs = __fdiv_rn(acc[u][j], Wf) + sv[u][j];
+                tsum = fma(static_cast<double>(cs), static_cast<double>(cs), tsum);
+                bad |= !isfinite(cs);
+              }
+            }
+        }
       }
     } else {
       for (int j = 0; j < kTileWords; ++j) {

@@ -72,6 +72,7 @@ enum { OB_F32 = 0, OB_BF16 = 1 };  /* gradient element type */
 enum { OB_ADAM = 0, OB_LAMB = 1 }; /* update rule after the compressed allreduce */
 
 #define OB_STATUS_NONFINITE 1u /* a compensated value, server value or parameter was NaN/Inf */
+#define OB_STATUS_TIMEOUT 2u   /* a kernel gave up a bounded wait on its copy pipeline (results invalid) */
 
 typedef struct {
   int64_t n;                    /* total elements (parameters); >= 0 */
@@ -153,7 +154,9 @@ enum {
   OB_K_LAMB_PARAM = 5,     /* LAMB parameter step */
   OB_K_WARMUP = 6,         /* full-precision warmup step */
   OB_K_FINALIZE_RATIO = 7, /* LAMB trust ratio per layer */
-  OB_K_KINDS = 8
+  OB_K_WORKER_PACK_PIPE = 8,   /* pass 2 of the fused step, bulk-copy pipelined */
+  OB_K_SERVER_UPDATE_PIPE = 9, /* pass 3 of the fused step, bulk-copy pipelined */
+  OB_K_KINDS = 10
 };
 
 /* Start recording a CUDA event pair around each of the next `capacity`

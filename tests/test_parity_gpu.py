@@ -130,6 +130,7 @@ def run_chain(wl, steps, compare_every=True, **pair_kw):
         pr.step(grads_for(wl, t), warm=t < wl.freeze_step)
         if compare_every or t == steps - 1:
             pr.compare(tag=f"step {t} ", bits=t >= wl.freeze_step)
+    assert pr.gpu.status() == 0      # no non-finite value, no pipeline timeout
     return pr
 
 
@@ -154,6 +155,20 @@ def test_warmup_then_compressed(opt):
     sizes = WL.configs.bert_tensor_sizes(64, 2, 256, 1000)
     wl = small(sizes, 8, optimizer=opt, grad_dist="normal_layer", freeze_step=3)
     run_chain(wl, 6)
+
+
+@pytest.mark.parametrize("W,gdt,opt", [(1, "bf16", "adam"), (3, "f32", "adam"), (2, "f32", "lamb")])
+def test_fused_steps_many_tiles_per_cta(W, gdt, opt):
+    # ~12M elements: every CTA of the pipelined passes cycles its stage ring many
+    # times (block tiles of 2048 elements, one CTA per SM); chunks of uneven size.
+    wl = small([1 << 23, 3 * (1 << 20) + 2048 * 7 + 8, 40, 2048 * 300 - 8 * 3], W, grad_dtype=gdt,
+               optimizer=opt)
+    run_chain(wl, 3)
+
+
+def test_fused_steps_many_workers_fallback():
+    # W = 1024: the pass-3 stage would not fit shared memory; the warp-tile kernel runs.
+    run_chain(small([2048, 1000, 24], 1024), 2)
 
 
 def test_hundred_chained_steps_parameter_norm():
