@@ -48,7 +48,7 @@ FALLBACK_HBM_GBS = 6650.0
 E2E_MAX_HOST_BYTES = 16e9        # pinned host gradients per step the e2e leg may hold
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "ncu_traffic.txt")
 KERNEL_SOURCES = [os.path.join(ROOT, "bit_adam_error_b200", "csrc", f)
-                  for f in ("kernels.cuh", "pipeline.cuh", "onebit.cu")]
+                  for f in ("kernels.cuh", "onebit.cu")]
 
 
 def parse_args():
@@ -79,9 +79,9 @@ def algo_bytes_per_elem(kind: str, wl) -> float:
     W, gb = wl.W, wl.grad_bytes
     if kind == "k_worker_norm":          # read g, err for every worker
         return (gb + 4) * W
-    if kind in ("k_worker_pack", "k_pack_server_pipe"):  # read g, err, write err, signs; read srv_err
+    if kind == "k_worker_pack":          # read g, err, write err, signs; read srv_err
         return (gb + 8) * W + W / 8 + 4
-    if kind in ("k_server_update", "k_server_update_pipe"):
+    if kind == "k_server_update":
         if wl.optimizer == "lamb":       # signs, srv_err r/w, server signs, m r/w, v, p reads
             return W / 8 + 8 + 1 / 8 + 16
         return W / 8 + 8 + 1 / 8 + 20    # + m, v, p reads and m, p writes

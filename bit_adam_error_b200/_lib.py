@@ -17,7 +17,6 @@ OB_OK, OB_EINVAL, OB_ECUDA, OB_EPHASE, OB_ENOMEM = 0, -1, -2, -3, -4
 OB_F32, OB_BF16 = 0, 1
 OB_ADAM, OB_LAMB = 0, 1
 OB_STATUS_NONFINITE = 1
-OB_STATUS_TIMEOUT = 2
 
 ERR_NAMES = {OB_OK: "OB_OK", OB_EINVAL: "OB_EINVAL", OB_ECUDA: "OB_ECUDA",
              OB_EPHASE: "OB_EPHASE", OB_ENOMEM: "OB_ENOMEM"}
@@ -68,7 +67,7 @@ _SIGS = {
     "ob_last_error": (ctypes.c_char_p, []),
 }
 
-OB_K_KINDS = 10
+OB_K_KINDS = 8
 
 _lib = None
 

@@ -25,7 +25,7 @@
 //
 // Vector path (chunk start and length multiples of 8 elements, and the worker
 // row stride a multiple of 8): lane L of a 256-element group holds elements
-// 8L..8L+7 (two 16-byte fp32 loads, or one 16-byte bf16 load), so its 8 sign bits
+// 8L..8L+7 (one 32-byte v8.f32 access, or one 16-byte load of 8 bf16), so its 8 sign bits
 // form byte (L % 4) of word (L / 4) of the group; two xor-shuffles assemble the
 // eight 32-bit words, LSB-first.  Any other chunk takes the scalar path: lane L
 // holds element 32j + L and one ballot is one word.
@@ -51,8 +51,8 @@ constexpr int kTileWords = kTile / 32;
 constexpr int kBlock = 256;                      // threads per CTA (8 warps)
 constexpr int kWarpsPerBlock = kBlock / kWarp;
 constexpr int kFinalizeThreads = 256;
-constexpr bool kWide = false;                    // 256-bit (v8.f32) global accesses for fp32 arrays
-constexpr int kPackGroupsInFlight = kGroups;     // pass 2: groups whose loads are issued together
+constexpr bool kWide = true;                     // 256-bit (v8.f32) global accesses for fp32 arrays
+constexpr int kUpdateMinBlocks = 2;              // pass 3: resident CTAs per SM asked of ptxas
 constexpr unsigned kFull = 0xffffffffu;
 constexpr uint32_t kStatusNonfinite = 1u;
 
@@ -61,11 +61,9 @@ struct Layout {
   const int64_t* off;   // [C+1] first element of every chunk
   const int64_t* wo;    // [C+1] first word of every chunk within a packed row
   const int64_t* tp;    // [C+1] first warp tile (kTile elements) of every chunk
-  const int64_t* tpb;   // [C+1] first block tile (kBT elements, pipelined passes) of every chunk
   const uint8_t* vec;   // [C]   1: 8-wide vector path, 0: scalar path
   int64_t n;            // elements per row
   int64_t T;            // warp tiles per row
-  int64_t Tb;           // block tiles per row
   int64_t words;        // packed words per row
   int32_t C;
 };
@@ -180,6 +178,35 @@ __device__ __forceinline__ float clip_grad(float g, float clip) {
 
 __device__ __forceinline__ float signed_scale(bool bit, float s) { return bit ? s : -s; }
 
+// The mean of W scaled signs, acc / W: IEEE division, or the product with 1/W when
+// W is a power of two -- x / 2^k and x * 2^-k round the same exact value, so the
+// result is identical and the division's instruction sequence is saved.
+// POW2 is a template parameter of the kernels (chosen on the host from W), so the
+// choice is never a branch inside an element loop.
+template <bool POW2>
+struct Mean {
+  float Wf, invW;
+  __device__ __forceinline__ float operator()(float acc) const {
+    if constexpr (POW2) return acc * invW;
+    else return __fdiv_rn(acc, Wf);
+  }
+};
+
+template <bool POW2>
+__device__ __forceinline__ Mean<POW2> make_mean(int W) {
+  Mean<POW2> m;
+  m.Wf = static_cast<float>(W);
+  m.invW = __fdiv_rn(1.0f, m.Wf);
+  return m;
+}
+
+// A sum of squares of finite floats cannot overflow a double, so a non-finite
+// tile sum means a non-finite value in the tile: one check per tile replaces a
+// check per element.
+__device__ __forceinline__ void flag_tile_sum(double sum, uint32_t* status) {
+  if (!isfinite(sum)) atomicOr(status, kStatusNonfinite);
+}
+
 // Lanes 4q..4q+3 each hold one byte of word q (LSB-first); returns the whole
 // word in every lane of the quad (lane 4q writes it).
 __device__ __forceinline__ uint32_t quad_word(uint32_t byte, int lane) {
@@ -211,8 +238,9 @@ __device__ __forceinline__ int64_t warp_count() {
 }
 
 // ---- pass 1: per-tile sum of c^2 for every worker ----------------------------------
-// part[w * T + t] = sum over tile t of (clip(g_w) + err_w)^2.
-template <typename GT>
+// part[w * T + t] = sum over tile t of (clip(g_w) + err_w)^2; a non-finite sum
+// (some c is NaN/Inf) raises the status flag.
+template <typename GT, bool CLIP>
 __global__ void __launch_bounds__(kBlock)
 k_worker_norm(Layout L, int W, const GT* __restrict__ grads, const float* __restrict__ err,
               float clip, double* __restrict__ part, uint32_t* __restrict__ status) {
@@ -226,7 +254,6 @@ k_worker_norm(Layout L, int W, const GT* __restrict__ grads, const float* __rest
     const GT* g = grads + static_cast<int64_t>(w) * L.n + tl.ck0;
     const float* e = err + static_cast<int64_t>(w) * L.n + tl.ck0;
     double acc = 0.0;
-    bool bad = false;
     if (tl.vec) {
       float gv[kGroups][8], ev[kGroups][8];
 #pragma unroll
@@ -239,23 +266,23 @@ k_worker_norm(Layout L, int W, const GT* __restrict__ grads, const float* __rest
       for (int q = 0; q < kGroups; ++q)
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
-          const float c = clip_grad(gv[q][j], clip) + ev[q][j];
+          const float c = (CLIP ? clip_grad(gv[q][j], clip) : gv[q][j]) + ev[q][j];
           acc = fma(static_cast<double>(c), static_cast<double>(c), acc);
-          bad |= !isfinite(c);
         }
     } else {
       for (int j = 0; j < kTileWords; ++j) {
         const int64_t i = tl.rel + j * 32 + lane;
         if (i < tl.nk) {
-          const float c = clip_grad(ld1_ro(g + i), clip) + __ldg(e + i);
+          const float c = (CLIP ? clip_grad(ld1_ro(g + i), clip) : ld1_ro(g + i)) + __ldg(e + i);
           acc = fma(static_cast<double>(c), static_cast<double>(c), acc);
-          bad |= !isfinite(c);
         }
       }
     }
     acc = warp_sum(acc);
-    if (lane == 0) part[it] = acc;
-    flag_nonfinite(bad, status);
+    if (lane == 0) {
+      part[it] = acc;
+      flag_tile_sum(acc, status);
+    }
   }
 }
 
@@ -316,21 +343,23 @@ k_finalize_ratio(Layout L, const double* __restrict__ partP, const double* __res
 // ---- pass 2: worker pack (+ server accumulation) -------------------------------------
 // For every worker: c = clip(g) + err, bit = (c >= 0), err = c - s_w sign, bits_w.
 // SERVER: also c_srv = (sum_w s_w sign_w) / W + srv_err and part_srv[t] = sum c_srv^2.
-template <typename GT, bool SERVER>
-__global__ void __launch_bounds__(kBlock)
+// Non-finite c were flagged by pass 1 (same values); non-finite c_srv by the tile sum.
+// GP = groups of one tile whose loads are issued together: 1 keeps the kernel
+// under 80 registers (3 CTAs per SM), best when W is small and a tile carries few
+// bytes per instruction; 2 keeps more bytes in flight per warp, best for large W.
+template <typename GT, bool SERVER, bool CLIP, bool POW2, int GP>
+__global__ void __launch_bounds__(kBlock, GP == 1 ? 3 : 2)
 k_worker_pack(Layout L, int W, const GT* __restrict__ grads, float* __restrict__ err,
               const float* __restrict__ s_w, uint32_t* __restrict__ bits_w,
               const float* __restrict__ srv_err, double* __restrict__ part_srv, float clip,
               uint32_t* __restrict__ status) {
   const int lane = threadIdx.x & 31;
-  const float Wf = static_cast<float>(W);
+  const auto mean = make_mean<POW2>(W);
   int hint = 0;
   for (int64_t t = warp_id(); t < L.T; t += warp_count()) {
     const Tile tl = tile_at(L, t, hint);
     double tsum = 0.0;
-    bool bad = false;
     if (tl.vec) {
-      constexpr int GP = kPackGroupsInFlight;
 #pragma unroll 1
       for (int q0 = 0; q0 < kGroups; q0 += GP) {
         float acc[GP][8], sv[GP][8];
@@ -361,13 +390,12 @@ k_worker_pack(Layout L, int W, const GT* __restrict__ grads, float* __restrict__
             uint32_t byte = 0;
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
-              const float c = clip_grad(gv[u][j], clip) + ev[u][j];
+              const float c = (CLIP ? clip_grad(gv[u][j], clip) : gv[u][j]) + ev[u][j];
               const bool b = c >= 0.0f;
               const float d = signed_scale(b, s);
               byte |= static_cast<uint32_t>(b) << j;
               ev[u][j] = c - d;
               acc[u][j] = acc[u][j] + d;
-              bad |= in[u] && !isfinite(c);
             }
             if (!in[u]) byte = 0;
             else st8(e + i0, ev[u]);
@@ -383,9 +411,8 @@ k_worker_pack(Layout L, int W, const GT* __restrict__ grads, float* __restrict__
             if (in[u]) {
 #pragma unroll
               for (int j = 0; j < 8; ++j) {
-                const float cs = __fdiv_rn(acc[u][j], Wf) + sv[u][j];
+                const float cs = mean(acc[u][j]) + sv[u][j];
                 tsum = fma(static_cast<double>(cs), static_cast<double>(cs), tsum);
-                bad |= !isfinite(cs);
               }
             }
         }
@@ -400,29 +427,30 @@ k_worker_pack(Layout L, int W, const GT* __restrict__ grads, float* __restrict__
           float* e = err + static_cast<int64_t>(w) * L.n + tl.ck0;
           bool b = false;
           if (inb) {
-            const float c = clip_grad(ld1_ro(grads + static_cast<int64_t>(w) * L.n + tl.ck0 + i), clip) + e[i];
+            const float g = ld1_ro(grads + static_cast<int64_t>(w) * L.n + tl.ck0 + i);
+            const float c = (CLIP ? clip_grad(g, clip) : g) + e[i];
             b = c >= 0.0f;
             const float d = signed_scale(b, s);
             e[i] = c - d;
             acc = acc + d;
-            bad |= !isfinite(c);
           }
           const uint32_t word = __ballot_sync(kFull, b);
           if (lane == 0 && (tl.rel + j * 32) < tl.nk)
             bits_w[static_cast<int64_t>(w) * L.words + tl.w0 + tl.rel / 32 + j] = word;
         }
         if (SERVER && inb) {
-          const float cs = __fdiv_rn(acc, Wf) + __ldg(srv_err + tl.ck0 + i);
+          const float cs = mean(acc) + __ldg(srv_err + tl.ck0 + i);
           tsum = fma(static_cast<double>(cs), static_cast<double>(cs), tsum);
-          bad |= !isfinite(cs);
         }
       }
     }
     if (SERVER) {
       tsum = warp_sum(tsum);
-      if (lane == 0) part_srv[t] = tsum;
+      if (lane == 0) {
+        part_srv[t] = tsum;
+        flag_tile_sum(tsum, status);
+      }
     }
-    flag_nonfinite(bad, status);
   }
 }
 
@@ -444,17 +472,17 @@ __device__ __forceinline__ void server_sum8(const Layout& L, int W, const uint32
 }
 
 // Server norm only (stage-wise call): part_srv[t] = sum over the tile of c_srv^2.
+template <bool POW2>
 __global__ void __launch_bounds__(kBlock)
 k_server_norm(Layout L, int W, const uint32_t* __restrict__ bits_w, const float* __restrict__ s_w,
               const float* __restrict__ srv_err, double* __restrict__ part_srv,
               uint32_t* __restrict__ status) {
   const int lane = threadIdx.x & 31;
-  const float Wf = static_cast<float>(W);
+  const auto mean = make_mean<POW2>(W);
   int hint = 0;
   for (int64_t t = warp_id(); t < L.T; t += warp_count()) {
     const Tile tl = tile_at(L, t, hint);
     double tsum = 0.0;
-    bool bad = false;
     if (tl.vec) {
 #pragma unroll
       for (int q = 0; q < kGroups; ++q) {
@@ -467,9 +495,8 @@ k_server_norm(Layout L, int W, const uint32_t* __restrict__ bits_w, const float*
           ld8_ro(srv_err + tl.ck0 + i0, sv);
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
-            const float cs = __fdiv_rn(acc[j], Wf) + sv[j];
+            const float cs = mean(acc[j]) + sv[j];
             tsum = fma(static_cast<double>(cs), static_cast<double>(cs), tsum);
-            bad |= !isfinite(cs);
           }
         }
       }
@@ -483,15 +510,16 @@ k_server_norm(Layout L, int W, const uint32_t* __restrict__ bits_w, const float*
             const uint32_t word = __ldg(bits_w + static_cast<int64_t>(w) * L.words + tl.w0 + tl.rel / 32 + j);
             acc = acc + signed_scale((word >> lane) & 1u, s);
           }
-          const float cs = __fdiv_rn(acc, Wf) + __ldg(srv_err + tl.ck0 + i);
+          const float cs = mean(acc) + __ldg(srv_err + tl.ck0 + i);
           tsum = fma(static_cast<double>(cs), static_cast<double>(cs), tsum);
-          bad |= !isfinite(cs);
         }
       }
     }
     tsum = warp_sum(tsum);
-    if (lane == 0) part_srv[t] = tsum;
-    flag_nonfinite(bad, status);
+    if (lane == 0) {
+      part_srv[t] = tsum;
+      flag_tile_sum(tsum, status);
+    }
   }
 }
 
@@ -521,15 +549,15 @@ __device__ __forceinline__ void update_elem(float d, float& m, float v, float& p
 // FROM_WORKERS: c_srv from bits_w/s_w/srv_err, quantised with s_srv, bits_srv and
 // srv_err written (the compressed allreduce's second half).  Otherwise g_hat is
 // read back from bits_srv/s_srv (the update-only stage call).
-template <Upd U, bool FROM_WORKERS>
-__global__ void __launch_bounds__(kBlock)
+template <Upd U, bool FROM_WORKERS, bool POW2>
+__global__ void __launch_bounds__(kBlock, kUpdateMinBlocks)
 k_server_update(Layout L, int W, const uint32_t* __restrict__ bits_w, const float* __restrict__ s_w,
                 const float* __restrict__ s_srv, float* __restrict__ srv_err,
                 uint32_t* __restrict__ bits_srv, float* __restrict__ m, const float* __restrict__ v,
                 float* __restrict__ p, Hyper h, double* __restrict__ partP,
                 double* __restrict__ partU, uint32_t* __restrict__ status) {
   const int lane = threadIdx.x & 31;
-  const float Wf = static_cast<float>(W);
+  const auto mean = make_mean<POW2>(W);
   int hint = 0;
   for (int64_t t = warp_id(); t < L.T; t += warp_count()) {
     const Tile tl = tile_at(L, t, hint);
@@ -556,12 +584,11 @@ k_server_update(Layout L, int W, const uint32_t* __restrict__ bits_w, const floa
           if (in) {
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
-              const float cs = __fdiv_rn(acc[j], Wf) + sv[j];
+              const float cs = mean(acc[j]) + sv[j];
               const bool b = cs >= 0.0f;
               const float d = signed_scale(b, s2);
               byte |= static_cast<uint32_t>(b) << j;
               sv[j] = cs - d;
-              bad |= !isfinite(cs);
               update_elem<U>(d, mv[j], vv[j], pv[j], h, Psum, Usum, bad);
             }
             st8(srv_err + gi, sv);
@@ -598,11 +625,10 @@ k_server_update(Layout L, int W, const uint32_t* __restrict__ bits_w, const floa
               const uint32_t word = __ldg(bits_w + static_cast<int64_t>(w) * L.words + wi);
               acc = acc + signed_scale((word >> lane) & 1u, s);
             }
-            const float cs = __fdiv_rn(acc, Wf) + srv_err[gi];
+            const float cs = mean(acc) + srv_err[gi];
             b = cs >= 0.0f;
             d = signed_scale(b, s2);
             srv_err[gi] = cs - d;
-            bad |= !isfinite(cs);
           }
           const uint32_t word = __ballot_sync(kFull, b);
           if (lane == 0 && (tl.rel + j * 32) < tl.nk) bits_srv[wi] = word;
@@ -674,20 +700,20 @@ k_lamb_param(Layout L, const float* __restrict__ m, const float* __restrict__ v,
 // g = (sum_w g_w) / W; m = b1 m + (1-b1) g; v = b2 v + (1-b2) g^2;
 // Adam: p -= lr m / (sqrt(v) + eps).  LAMB: per-tile sums of p^2 and u^2 instead
 // (the parameter step follows in k_lamb_param).
-template <typename GT, bool LAMB>
+template <typename GT, bool LAMB, bool POW2>
 __global__ void __launch_bounds__(kBlock)
 k_warmup(Layout L, int W, const GT* __restrict__ grads, float* __restrict__ m,
          float* __restrict__ v, float* __restrict__ p, Hyper h, double* __restrict__ partP,
          double* __restrict__ partU, uint32_t* __restrict__ status) {
   const int lane = threadIdx.x & 31;
-  const float Wf = static_cast<float>(W);
+  const auto mean = make_mean<POW2>(W);
   int hint = 0;
   for (int64_t t = warp_id(); t < L.T; t += warp_count()) {
     const Tile tl = tile_at(L, t, hint);
     double Psum = 0.0, Usum = 0.0;
     bool bad = false;
     auto elem = [&](float gsum, float& mm, float& vv, float& pp) {
-      const float g = __fdiv_rn(gsum, Wf);
+      const float g = mean(gsum);
       bad |= !isfinite(g);
       mm = h.b1 * mm + h.omb1 * g;
       vv = h.b2 * vv + h.omb2 * (g * g);

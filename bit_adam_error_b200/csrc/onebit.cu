@@ -17,16 +17,10 @@
 
 #include "onebit.h"
 #include "kernels.cuh"
-#include "pipeline.cuh"
 
 namespace {
 
 thread_local char g_last_error[512] = "";
-
-// Shared memory the pipelined passes 2 and 3 may use per SM (split over
-// kPipeCtasPerSm CTAs); 0 keeps that pass on its warp-tile kernel.
-constexpr size_t kPipe2SmemBudget = 0;
-constexpr size_t kPipe3SmemBudget = 0;
 
 ob_err fail(ob_err code, const char* fmt, ...) {
   va_list ap;
@@ -40,7 +34,8 @@ ob_err cuda_fail(cudaError_t e, const char* what) {
   return fail(OB_ECUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
 }
 
-bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+// 32 bytes: the kernels move 8 fp32 elements per lane in one 256-bit access.
+bool aligned32(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 31u) == 0; }
 
 int64_t words_of(int64_t n) { return (n + 31) / 32; }
 
@@ -71,12 +66,12 @@ ob_err check_config(const ob_config* c) {
   return OB_OK;
 }
 
-// A device buffer argument: NULL only when it holds no element; 16-byte
+// A device buffer argument: NULL only when it holds no element; 32-byte
 // aligned; device (or managed) memory of the current device.
 ob_err check_dev(const void* p, int64_t count, const char* name, int device) {
   if (count == 0) return OB_OK;
   if (!p) return fail(OB_EINVAL, "%s is NULL", name);
-  if (!aligned16(p)) return fail(OB_EINVAL, "%s is not 16-byte aligned", name);
+  if (!aligned32(p)) return fail(OB_EINVAL, "%s is not 32-byte aligned", name);
   cudaPointerAttributes a;
   cudaError_t e = cudaPointerGetAttributes(&a, p);
   if (e != cudaSuccess) {
@@ -104,9 +99,6 @@ struct ob_ctx {
   void* scratch = nullptr;
   ob::Layout L{};
   double *part_w = nullptr, *part_srv = nullptr, *partP = nullptr, *partU = nullptr;
-  int64_t Tb = 0;                 // block tiles (pipelined passes)
-  int pipe_s2 = 0, pipe_s3 = 0;   // ring stages of the pipelined passes (0: warp-tile kernels)
-  size_t pipe_b2 = 0, pipe_b3 = 0;  // dynamic shared memory of one launch
   float* ratio = nullptr;
   uint32_t* status = nullptr;
   ob::Hyper h{};
@@ -194,32 +186,30 @@ void enqueue_finalize_scale(ob_ctx* c, const double* part, float* out, int rows,
   });
 }
 
-template <typename GT>
-void enqueue_worker(ob_ctx* c, const GT* grads, bool with_server, cudaStream_t st) {
+// W a power of two: the server mean is an exact multiply (see ob::Mean).
+bool pow2_workers(const ob_ctx* c) { return (c->cfg.W & (c->cfg.W - 1)) == 0; }
+
+// Pass 2 issues one group of a tile at a time (3 CTAs per SM) up to this many
+// workers, two groups at a time (2 CTAs per SM) above it -- measured on B200:
+// W = 1 bf16 3.19 vs 3.47 ms per 1.5e9 elements, W = 16 fp32 10.30 vs 10.05 ms.
+constexpr int kPackOneGroupMaxW = 2;
+
+template <typename GT, bool CLIP, bool POW2>
+void enqueue_worker_t(ob_ctx* c, const GT* grads, bool with_server, cudaStream_t st) {
   const int W = c->cfg.W;
   if (c->T > 0) {
-    auto k1 = ob::k_worker_norm<GT>;
+    auto k1 = ob::k_worker_norm<GT, CLIP>;
     const int g1 = grid_for(c, k1, W * c->T);
     launch(c, OB_K_WORKER_NORM, st, [&] {
       k1<<<g1, ob::kBlock, 0, st>>>(c->L, W, grads, c->err, c->h.clip, c->part_w, c->status);
     });
   }
   enqueue_finalize_scale(c, c->part_w, c->s_w, W, c->L.tp, 1, c->T, st);
-  if (with_server && c->pipe_s2 > 0) {
-    // Pipelined pass 2: bulk-copy ring, server sums in one slot per (block tile, consumer warp).
-    if (c->Tb > 0) {
-      const int g2 = static_cast<int>(std::min<int64_t>(int64_t(c->num_sms) * ob::kPipeCtasPerSm, c->Tb));
-      launch(c, OB_K_WORKER_PACK_PIPE, st, [&] {
-        ob::k_pack_server_pipe<GT><<<g2, ob::kPipeThreads, c->pipe_b2, st>>>(
-            c->L, W, grads, c->err, c->s_w, c->bits_w, c->srv_err, c->part_srv, c->h.clip,
-            c->pipe_s2, c->status);
-      });
-    }
-    enqueue_finalize_scale(c, c->part_srv, c->s_srv, 1, c->L.tpb, ob::kConsumers, 0, st);
-    return;
-  }
   if (c->T > 0) {
-    auto k2 = with_server ? ob::k_worker_pack<GT, true> : ob::k_worker_pack<GT, false>;
+    // The stage call (no server part) never uses the mean: one instantiation each.
+    const bool one = W <= kPackOneGroupMaxW;
+    auto k2 = with_server ? (one ? ob::k_worker_pack<GT, true, CLIP, POW2, 1> : ob::k_worker_pack<GT, true, CLIP, POW2, 2>)
+                          : (one ? ob::k_worker_pack<GT, false, CLIP, false, 1> : ob::k_worker_pack<GT, false, CLIP, false, 2>);
     const int g2 = grid_for(c, k2, c->T);
     launch(c, OB_K_WORKER_PACK, st, [&] {
       k2<<<g2, ob::kBlock, 0, st>>>(c->L, W, grads, c->err, c->s_w, c->bits_w, c->srv_err,
@@ -229,10 +219,20 @@ void enqueue_worker(ob_ctx* c, const GT* grads, bool with_server, cudaStream_t s
   if (with_server) enqueue_finalize_scale(c, c->part_srv, c->s_srv, 1, c->L.tp, 1, 0, st);
 }
 
+template <typename GT>
+void enqueue_worker(ob_ctx* c, const GT* grads, bool with_server, cudaStream_t st) {
+  const bool clip = c->h.clip > 0.0f, p2 = pow2_workers(c);
+  if (clip && p2) enqueue_worker_t<GT, true, true>(c, grads, with_server, st);
+  else if (clip) enqueue_worker_t<GT, true, false>(c, grads, with_server, st);
+  else if (p2) enqueue_worker_t<GT, false, true>(c, grads, with_server, st);
+  else enqueue_worker_t<GT, false, false>(c, grads, with_server, st);
+}
+
 template <ob::Upd U, bool FROM_WORKERS>
 void enqueue_server_update(ob_ctx* c, cudaStream_t st) {
   if (c->T == 0) return;
-  auto k3 = ob::k_server_update<U, FROM_WORKERS>;
+  auto k3 = pow2_workers(c) ? ob::k_server_update<U, FROM_WORKERS, true>
+                            : ob::k_server_update<U, FROM_WORKERS, false>;
   const int g3 = grid_for(c, k3, c->T);
   launch(c, OB_K_SERVER_UPDATE, st, [&] {
     k3<<<g3, ob::kBlock, 0, st>>>(c->L, c->cfg.W, c->bits_w, c->s_w, c->s_srv, c->srv_err,
@@ -241,11 +241,11 @@ void enqueue_server_update(ob_ctx* c, cudaStream_t st) {
   });
 }
 
-// LAMB: trust ratio per layer from partial slots [tpx[k]*mult, tpx[k+1]*mult), then p.
-void enqueue_lamb_param(ob_ctx* c, const int64_t* tpx, int mult, cudaStream_t st) {
+// LAMB: trust ratio per layer from the tile partials, then the parameter step.
+void enqueue_lamb_param(ob_ctx* c, cudaStream_t st) {
   launch(c, OB_K_FINALIZE_RATIO, st, [&] {
     ob::k_finalize_ratio<<<c->cfg.num_chunks, ob::kFinalizeThreads, 0, st>>>(c->L, c->partP, c->partU,
-                                                                             tpx, mult, c->ratio);
+                                                                             c->L.tp, 1, c->ratio);
   });
   if (c->T == 0) return;
   auto k = ob::k_lamb_param;
@@ -255,29 +255,9 @@ void enqueue_lamb_param(ob_ctx* c, const int64_t* tpx, int mult, cudaStream_t st
   });
 }
 
-template <ob::Upd U>
-void enqueue_server_update_pipe(ob_ctx* c, cudaStream_t st) {
-  if (c->Tb == 0) return;
-  const int g3 = static_cast<int>(std::min<int64_t>(int64_t(c->num_sms) * ob::kPipeCtasPerSm, c->Tb));
-  launch(c, OB_K_SERVER_UPDATE_PIPE, st, [&] {
-    ob::k_server_update_pipe<U><<<g3, ob::kPipeThreads, c->pipe_b3, st>>>(
-        c->L, c->cfg.W, c->bits_w, c->s_w, c->s_srv, c->srv_err, c->bits_srv, c->m, c->v, c->p,
-        c->h, c->partP, c->partU, c->pipe_s3, c->status);
-  });
-}
-
 // Update from the packed worker signs (fused) or from bits_srv (stage call).
 void enqueue_update(ob_ctx* c, bool from_workers, cudaStream_t st) {
   const bool lamb = c->cfg.optimizer == OB_LAMB;
-  if (from_workers && c->pipe_s3 > 0) {
-    if (lamb) {
-      enqueue_server_update_pipe<ob::Upd::kLambM>(c, st);
-      enqueue_lamb_param(c, c->L.tpb, ob::kConsumers, st);
-    } else {
-      enqueue_server_update_pipe<ob::Upd::kAdam>(c, st);
-    }
-    return;
-  }
   if (from_workers) {
     if (lamb) enqueue_server_update<ob::Upd::kLambM, true>(c, st);
     else enqueue_server_update<ob::Upd::kAdam, true>(c, st);
@@ -285,26 +265,27 @@ void enqueue_update(ob_ctx* c, bool from_workers, cudaStream_t st) {
     if (lamb) enqueue_server_update<ob::Upd::kLambM, false>(c, st);
     else enqueue_server_update<ob::Upd::kAdam, false>(c, st);
   }
-  if (lamb) enqueue_lamb_param(c, c->L.tp, 1, st);
+  if (lamb) enqueue_lamb_param(c, st);
 }
 
 template <typename GT>
 void enqueue_warmup(ob_ctx* c, const GT* grads, cudaStream_t st) {
-  const bool lamb = c->cfg.optimizer == OB_LAMB;
+  const bool lamb = c->cfg.optimizer == OB_LAMB, p2 = pow2_workers(c);
   if (c->T > 0) {
-    auto k = lamb ? ob::k_warmup<GT, true> : ob::k_warmup<GT, false>;
+    auto k = lamb ? (p2 ? ob::k_warmup<GT, true, true> : ob::k_warmup<GT, true, false>)
+                  : (p2 ? ob::k_warmup<GT, false, true> : ob::k_warmup<GT, false, false>);
     const int g = grid_for(c, k, c->T);
     launch(c, OB_K_WARMUP, st, [&] {
       k<<<g, ob::kBlock, 0, st>>>(c->L, c->cfg.W, grads, c->m, c->v, c->p, c->h, c->partP,
                                   c->partU, c->status);
     });
   }
-  if (lamb) enqueue_lamb_param(c, c->L.tp, 1, st);
+  if (lamb) enqueue_lamb_param(c, st);
 }
 
 void enqueue_server_stage(ob_ctx* c, cudaStream_t st) {
   if (c->T > 0) {
-    auto k = ob::k_server_norm;
+    auto k = pow2_workers(c) ? ob::k_server_norm<true> : ob::k_server_norm<false>;
     const int g = grid_for(c, k, c->T);
     launch(c, OB_K_SERVER_NORM, st, [&] {
       k<<<g, ob::kBlock, 0, st>>>(c->L, c->cfg.W, c->bits_w, c->s_w, c->srv_err, c->part_srv,
@@ -394,62 +375,27 @@ ob_err ob_create(const ob_config* cfg, float* p, float* m, float* v, float* err,
   }
 
   // Chunk tables.
-  std::vector<int64_t> wo(C + 1), tp(C + 1), tpb(C + 1);
+  std::vector<int64_t> wo(C + 1), tp(C + 1);
   std::vector<uint8_t> vec(C);
-  wo[0] = tp[0] = tpb[0] = 0;
+  wo[0] = tp[0] = 0;
   for (int64_t k = 0; k < C; ++k) {
     const int64_t o = c->off[k], nk = c->off[k + 1] - o;
     wo[k + 1] = wo[k] + words_of(nk);
     tp[k + 1] = tp[k] + (nk + ob::kTile - 1) / ob::kTile;
-    tpb[k + 1] = tpb[k] + (nk + ob::kBT - 1) / ob::kBT;
     // 8-wide path: chunk start and length multiples of 8, and every worker row
     // starts on a multiple of 8 elements (16 bytes of bf16, 32 bytes of fp32).
     vec[k] = (o % 8 == 0) && (nk % 8 == 0) && (W == 1 || n % 8 == 0);
   }
   c->T = tp[C];
-  c->Tb = tpb[C];
-
-  // Pipelined passes: ring stages that fit the shared-memory budget of one CTA
-  // per SM; fewer than 2 stages -> the warp-tile kernels.
-  {
-    int optin = 0;
-    cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, device);
-    const size_t cap = size_t(optin) > 4096 ? size_t(optin) - 4096 : 0;
-    const size_t budget2 = std::min(cap, kPipe2SmemBudget) / ob::kPipeCtasPerSm;
-    const size_t budget3 = std::min(cap, kPipe3SmemBudget) / ob::kPipeCtasPerSm;
-    const size_t budget = std::max(budget2, budget3);
-    const size_t st2 = size_t(ob::kBT) * ((cfg->grad_dtype == OB_BF16 ? 2 : 4) + 8);
-    const size_t st3 = size_t(ob::kBT) * 16 + size_t(W) * ob::kBTWords * 4;
-    const int s2 = static_cast<int>(std::min<size_t>(16, budget2 / st2));
-    const int s3 = static_cast<int>(std::min<size_t>(16, budget3 / st3));
-    bool ok = true;
-    if (s2 >= 2) {
-      c->pipe_s2 = s2;
-      c->pipe_b2 = size_t(s2) * st2;
-      ok &= cudaFuncSetAttribute(ob::k_pack_server_pipe<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(budget)) == cudaSuccess;
-      ok &= cudaFuncSetAttribute(ob::k_pack_server_pipe<uint16_t>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(budget)) == cudaSuccess;
-    }
-    if (s3 >= 2) {
-      c->pipe_s3 = s3;
-      c->pipe_b3 = size_t(s3) * st3;
-      ok &= cudaFuncSetAttribute(ob::k_server_update_pipe<ob::Upd::kAdam>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(budget)) == cudaSuccess;
-      ok &= cudaFuncSetAttribute(ob::k_server_update_pipe<ob::Upd::kLambM>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(budget)) == cudaSuccess;
-    }
-    if (!ok) {  // keep the warp-tile kernels
-      cudaGetLastError();
-      c->pipe_s2 = c->pipe_s3 = 0;
-    }
-  }
 
   // Scratch layout: tables, then partials, every piece 256-byte aligned.
   auto up256 = [](size_t x) { return (x + 255) & ~size_t(255); };
   const size_t sz_tab = up256(sizeof(int64_t) * (C + 1));
   const size_t sz_vec = up256(size_t(C));
   const size_t sz_pw = up256(sizeof(double) * size_t(W) * size_t(c->T));
-  const size_t slots = std::max<size_t>(size_t(c->T), size_t(c->Tb) * ob::kConsumers);
-  const size_t sz_pt = up256(sizeof(double) * slots);
+  const size_t sz_pt = up256(sizeof(double) * size_t(c->T));
   const size_t sz_ratio = up256(sizeof(float) * size_t(C));
-  const size_t total = 4 * sz_tab + sz_vec + sz_pw + 3 * sz_pt + sz_ratio + 256;
+  const size_t total = 3 * sz_tab + sz_vec + sz_pw + 3 * sz_pt + sz_ratio + 256;
   if ((e = cudaMalloc(&c->scratch, total)) != cudaSuccess) {
     cudaGetLastError();
     delete c;
@@ -459,7 +405,6 @@ ob_err ob_create(const ob_config* cfg, float* p, float* m, float* v, float* err,
   int64_t* d_off = reinterpret_cast<int64_t*>(base); base += sz_tab;
   int64_t* d_wo = reinterpret_cast<int64_t*>(base); base += sz_tab;
   int64_t* d_tp = reinterpret_cast<int64_t*>(base); base += sz_tab;
-  int64_t* d_tpb = reinterpret_cast<int64_t*>(base); base += sz_tab;
   uint8_t* d_vec = reinterpret_cast<uint8_t*>(base); base += sz_vec;
   c->part_w = reinterpret_cast<double*>(base); base += sz_pw;
   c->part_srv = reinterpret_cast<double*>(base); base += sz_pt;
@@ -472,7 +417,6 @@ ob_err ob_create(const ob_config* cfg, float* p, float* m, float* v, float* err,
       {d_off, c->off.data(), sizeof(int64_t) * (C + 1)},
       {d_wo, wo.data(), sizeof(int64_t) * (C + 1)},
       {d_tp, tp.data(), sizeof(int64_t) * (C + 1)},
-      {d_tpb, tpb.data(), sizeof(int64_t) * (C + 1)},
       {d_vec, vec.data(), size_t(C)}};
   for (auto& cp : copies)
     if ((e = cudaMemcpy(cp.dst, cp.src, cp.bytes, cudaMemcpyHostToDevice)) != cudaSuccess) {
@@ -489,11 +433,9 @@ ob_err ob_create(const ob_config* cfg, float* p, float* m, float* v, float* err,
   c->L.off = d_off;
   c->L.wo = d_wo;
   c->L.tp = d_tp;
-  c->L.tpb = d_tpb;
   c->L.vec = d_vec;
   c->L.n = n;
   c->L.T = c->T;
-  c->L.Tb = c->Tb;
   c->L.words = words;
   c->L.C = static_cast<int32_t>(C);
   *out = c;
@@ -665,8 +607,7 @@ ob_err ob_profile_stop(ob_ctx* c, double* ms, int64_t* launches) {
 const char* ob_kernel_name(int32_t kind) {
   static const char* names[OB_K_KINDS] = {
       "k_worker_norm", "k_finalize_scale", "k_worker_pack", "k_server_norm",
-      "k_server_update", "k_lamb_param", "k_warmup", "k_finalize_ratio",
-      "k_pack_server_pipe", "k_server_update_pipe"};
+      "k_server_update", "k_lamb_param", "k_warmup", "k_finalize_ratio"};
   return (kind >= 0 && kind < OB_K_KINDS) ? names[kind] : "";
 }
 
@@ -725,10 +666,10 @@ ob_err noalloc_setup(int device, NoAllocDevice** out) {
     if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(no-alloc scratch)");
     if ((e = cudaDeviceGetAttribute(&d.num_sms, cudaDevAttrMultiProcessorCount, device)) != cudaSuccess)
       return cuda_fail(e, "cudaDeviceGetAttribute");
-    d.occ_norm[0] = occupancy(reinterpret_cast<const void*>(ob::k_worker_norm<float>));
-    d.occ_norm[1] = occupancy(reinterpret_cast<const void*>(ob::k_worker_norm<uint16_t>));
-    d.occ_pack[0] = occupancy(reinterpret_cast<const void*>(ob::k_worker_pack<float, false>));
-    d.occ_pack[1] = occupancy(reinterpret_cast<const void*>(ob::k_worker_pack<uint16_t, false>));
+    d.occ_norm[0] = occupancy(reinterpret_cast<const void*>(ob::k_worker_norm<float, true>));
+    d.occ_norm[1] = occupancy(reinterpret_cast<const void*>(ob::k_worker_norm<uint16_t, true>));
+    d.occ_pack[0] = occupancy(reinterpret_cast<const void*>(ob::k_worker_pack<float, false, true, false, 2>));
+    d.occ_pack[1] = occupancy(reinterpret_cast<const void*>(ob::k_worker_pack<uint16_t, false, true, false, 2>));
     d.scratch = static_cast<char*>(ptr);
     d.ready = true;
   }
@@ -807,18 +748,25 @@ extern "C" ob_err ob_compress_noalloc(const ob_config* cfg, const void* grads, f
   double* part = reinterpret_cast<double*>(d->scratch + header);
   const int bf = cfg->grad_dtype == OB_BF16 ? 1 : 0;
   const float clip = cfg->clip;
+  const bool cl = clip > 0.0f;
   if (T > 0) {
     const int g1 = noalloc_grid(d->num_sms, d->occ_norm[bf], W * T);
-    if (bf) ob::k_worker_norm<uint16_t><<<g1, ob::kBlock, 0, st>>>(L, int(W), static_cast<const uint16_t*>(grads), err, clip, part, status);
-    else ob::k_worker_norm<float><<<g1, ob::kBlock, 0, st>>>(L, int(W), static_cast<const float*>(grads), err, clip, part, status);
+    const uint16_t* gh = static_cast<const uint16_t*>(grads);
+    const float* gf = static_cast<const float*>(grads);
+    if (bf && cl) ob::k_worker_norm<uint16_t, true><<<g1, ob::kBlock, 0, st>>>(L, int(W), gh, err, clip, part, status);
+    else if (bf) ob::k_worker_norm<uint16_t, false><<<g1, ob::kBlock, 0, st>>>(L, int(W), gh, err, clip, part, status);
+    else if (cl) ob::k_worker_norm<float, true><<<g1, ob::kBlock, 0, st>>>(L, int(W), gf, err, clip, part, status);
+    else ob::k_worker_norm<float, false><<<g1, ob::kBlock, 0, st>>>(L, int(W), gf, err, clip, part, status);
   }
   ob::k_finalize_scale<<<dim3(unsigned(C), unsigned(W)), ob::kFinalizeThreads, 0, st>>>(L, part, L.tp, 1, T, s_w);
   if (T > 0) {
     const int g2 = noalloc_grid(d->num_sms, d->occ_pack[bf], T);
-    if (bf)
-      ob::k_worker_pack<uint16_t, false><<<g2, ob::kBlock, 0, st>>>(L, int(W), static_cast<const uint16_t*>(grads), err, s_w, bits_w, nullptr, nullptr, clip, status);
-    else
-      ob::k_worker_pack<float, false><<<g2, ob::kBlock, 0, st>>>(L, int(W), static_cast<const float*>(grads), err, s_w, bits_w, nullptr, nullptr, clip, status);
+    const uint16_t* gh = static_cast<const uint16_t*>(grads);
+    const float* gf = static_cast<const float*>(grads);
+    if (bf && cl) ob::k_worker_pack<uint16_t, false, true, false, 2><<<g2, ob::kBlock, 0, st>>>(L, int(W), gh, err, s_w, bits_w, nullptr, nullptr, clip, status);
+    else if (bf) ob::k_worker_pack<uint16_t, false, false, false, 2><<<g2, ob::kBlock, 0, st>>>(L, int(W), gh, err, s_w, bits_w, nullptr, nullptr, clip, status);
+    else if (cl) ob::k_worker_pack<float, false, true, false, 2><<<g2, ob::kBlock, 0, st>>>(L, int(W), gf, err, s_w, bits_w, nullptr, nullptr, clip, status);
+    else ob::k_worker_pack<float, false, false, false, 2><<<g2, ob::kBlock, 0, st>>>(L, int(W), gf, err, s_w, bits_w, nullptr, nullptr, clip, status);
   }
   return check_launch("ob_compress_noalloc");
 }

@@ -1,18 +1,14 @@
 /*
  * onebit.h -- C ABI of the B200 (sm_100a) 1-bit Adam compressed-phase library.
  *
- * The calls follow the step as stated in "DeepSpeed Communication Compression
- * and Hiding", section "1-bit Adam: 预热、冻结方差、误差反馈" (机制):
- *
- *     if step < freeze_step:  g = allreduce(local_grad); m, v = adam_moments(g, m, v)
- *     else:                   compensated = local_grad + error
- *                             q, scale    = one_bit_quantize(compensated)
- *                             q_global    = compressed_allreduce(q, scale)
- *                             g_hat       = dequantize(q_global)
- *                             error       = compensated - g_hat
- *                             m           = beta1 m + (1 - beta1) g_hat   (v frozen)
- *     param -= lr m / (sqrt(v_frozen) + eps)
- *
+ * The calls follow the step described in "DeepSpeed Communication Compression
+ * and Hiding", section "1-bit Adam: 预热、冻结方差、误差反馈" (机制).  Before freeze_step
+ * the averaged gradient drives ordinary Adam moments (m and v).  From then on
+ * each worker adds its error buffer to its gradient, sends the sum as one sign
+ * bit per element plus a scale, the workers' messages are combined by a
+ * compressed allreduce and expanded back into a direction g_hat, the error
+ * buffer keeps what quantisation dropped, m follows g_hat while v stays
+ * frozen, and the parameters move by lr * m / (sqrt(v) + eps) --
  * with W data-parallel workers held in one GPU's memory.  Where the page gives
  * no formula the library fixes it as follows:
  *   - the gradient is cut into chunks (one per parameter tensor or per flat
@@ -37,7 +33,8 @@
  *   - Device buffers are caller-owned and must stay valid for the ctx's life.
  *     The ctx stores their pointers and owns only its own scratch (per-tile
  *     partial norms, chunk tables, status word), allocated in ob_create.
- *   - Every device pointer must be 16-byte aligned; otherwise OB_EINVAL.
+ *   - Every device pointer must be 32-byte aligned (cudaMalloc and the PyTorch
+ *     caching allocator give 256 or more); otherwise OB_EINVAL.
  *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
  *     Calls only enqueue work on it and return; none synchronises except
  *     ob_get_status and ob_create.
@@ -72,7 +69,6 @@ enum { OB_F32 = 0, OB_BF16 = 1 };  /* gradient element type */
 enum { OB_ADAM = 0, OB_LAMB = 1 }; /* update rule after the compressed allreduce */
 
 #define OB_STATUS_NONFINITE 1u /* a compensated value, server value or parameter was NaN/Inf */
-#define OB_STATUS_TIMEOUT 2u   /* a kernel gave up a bounded wait on its copy pipeline (results invalid) */
 
 typedef struct {
   int64_t n;                    /* total elements (parameters); >= 0 */
@@ -127,7 +123,7 @@ ob_err ob_step(ob_ctx* ctx, const void* grads, void* stream);
 /* Same as ob_step(ctx, grads, ...) with the gradients in HOST memory:
  * enqueues one host-to-device copy of [W][n] grad_dtype elements from
  * host_grads into dev_staging (a caller-owned DEVICE buffer of that size,
- * 16-byte aligned), then the fused step.  host_grads should be page-locked
+ * 32-byte aligned), then the fused step.  host_grads should be page-locked
  * for the copy to be asynchronous.  Advances the step counter. */
 ob_err ob_step_host(ob_ctx* ctx, const void* host_grads, void* dev_staging, void* stream);
 
@@ -154,9 +150,7 @@ enum {
   OB_K_LAMB_PARAM = 5,     /* LAMB parameter step */
   OB_K_WARMUP = 6,         /* full-precision warmup step */
   OB_K_FINALIZE_RATIO = 7, /* LAMB trust ratio per layer */
-  OB_K_WORKER_PACK_PIPE = 8,   /* pass 2 of the fused step, bulk-copy pipelined */
-  OB_K_SERVER_UPDATE_PIPE = 9, /* pass 3 of the fused step, bulk-copy pipelined */
-  OB_K_KINDS = 10
+  OB_K_KINDS = 8
 };
 
 /* Start recording a CUDA event pair around each of the next `capacity`
@@ -192,7 +186,7 @@ int64_t ob_launch_count(const ob_ctx* ctx);
  * with results identical to ob_compress on the same inputs.  The caller passes
  * the config and DEVICE buffers as for ob_create/ob_compress: grads [W][n]
  * (grad_dtype), err [W][n] (in/out), bits_w [W][words_total], s_w [W][C];
- * 16-byte aligned.  lr, betas, eps and freeze_step are ignored.
+ * 32-byte aligned.  lr, betas, eps and freeze_step are ignored.
  *
  * Scratch: a fixed 8 MiB array in the library's device memory (every GPU that
  * loads the library holds it until the process exits), used for the chunk

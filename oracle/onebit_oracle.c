@@ -9,11 +9,12 @@
  *
  * Sources followed (page title, section):
  *  - "DeepSpeed Communication Compression and Hiding", section "1-bit Adam:
- *    预热、冻结方差、误差反馈 / 机制": the step structure -- warmup with full Adam
- *    moments while step < freeze_step; afterwards compensated = local_grad +
- *    error, one_bit_quantize -> (q, scale), compressed_allreduce, dequantize,
- *    error = compensated - dequantized, m = beta1 m + (1 - beta1) g_hat with v
- *    frozen, param -= lr m / (sqrt(v_frozen) + eps).
+ *    预热、冻结方差、误差反馈 / 机制": the structure of the step -- full Adam moments
+ *    on the averaged gradient during warmup (step < freeze_step); afterwards each
+ *    worker's gradient plus its error buffer is reduced to signs and a scale,
+ *    the workers' messages are combined by a compressed allreduce and expanded
+ *    into the direction g_hat, the error buffer keeps what quantisation lost,
+ *    m follows g_hat with v frozen, and p moves by lr m / (sqrt(v) + eps).
  *  - same page, section "基线：Adam 为什么难压缩": the Adam moment equations.
  *  - same page, section "1-bit LAMB": r_l = ||w_l|| / ||u_l||,
  *    w_l <- w_l - eta r_l u_l, computed from the reconstructed global direction.
