@@ -312,6 +312,33 @@ ob_err check_ctx(const ob_ctx* c) {
   return OB_OK;
 }
 
+// The buffers each call touches; a ctx may be created without the others
+// (e.g. a server-only ctx on the rank that owns some chunks).
+enum Need : unsigned {
+  kNeedUpdate = 1u,  // p, m, v, bits_srv, s_srv
+  kNeedWarm = 2u,    // p, m, v
+  kNeedWorker = 4u,  // err, bits_w, s_w
+  kNeedServer = 8u,  // srv_err, bits_w, s_w, bits_srv, s_srv
+};
+
+ob_err require_buffers(const ob_ctx* c, unsigned need, const char* call) {
+  const int64_t n = c->cfg.n, W = c->cfg.W, C = c->cfg.num_chunks;
+  const struct { unsigned mask; const void* p; int64_t count; const char* name; } list[] = {
+      {kNeedUpdate | kNeedWarm, c->p, n, "p"},
+      {kNeedUpdate | kNeedWarm, c->m, n, "m"},
+      {kNeedUpdate | kNeedWarm, c->v, n, "v"},
+      {kNeedWorker, c->err, W * n, "err"},
+      {kNeedServer, c->srv_err, n, "srv_err"},
+      {kNeedWorker | kNeedServer, c->bits_w, W * c->words, "bits_w"},
+      {kNeedWorker | kNeedServer, c->s_w, W * C, "s_w"},
+      {kNeedUpdate | kNeedServer, c->bits_srv, c->words, "bits_srv"},
+      {kNeedUpdate | kNeedServer, c->s_srv, C, "s_srv"}};
+  for (const auto& b : list)
+    if ((b.mask & need) && b.count > 0 && !b.p)
+      return fail(OB_EINVAL, "%s: the ctx was created without %s", call, b.name);
+  return OB_OK;
+}
+
 ob_err require_compressed(const ob_ctx* c, const char* call) {
   if (c->step < c->cfg.freeze_step)
     return fail(OB_EPHASE, "%s: step %lld is in the warmup phase (freeze_step = %d)", call,
@@ -350,8 +377,8 @@ ob_err ob_create(const ob_config* cfg, float* p, float* m, float* v, float* err,
       {p, n, "p"}, {m, n, "m"}, {v, n, "v"}, {err, W * n, "err"}, {srv_err, n, "srv_err"},
       {bits_w, W * words, "bits_w"}, {s_w, W * C, "s_w"}, {bits_srv, words, "bits_srv"},
       {s_srv, C, "s_srv"}};
-  for (auto& b : bufs)
-    if ((r = check_dev(b.p, b.count, b.name, device)) != OB_OK) return r;
+  for (auto& b : bufs)  // NULL: the ctx is created without that buffer (see require_buffers)
+    if (b.p && (r = check_dev(b.p, b.count, b.name, device)) != OB_OK) return r;
 
   ob_ctx* c = new (std::nothrow) ob_ctx();
   if (!c) return fail(OB_ENOMEM, "ctx allocation failed");
@@ -448,6 +475,7 @@ ob_err ob_warmup_step(ob_ctx* c, const void* grads, void* stream) {
   if (c->step >= c->cfg.freeze_step)
     return fail(OB_EPHASE, "ob_warmup_step: step %lld >= freeze_step %d", (long long)c->step,
                 c->cfg.freeze_step);
+  if ((r = require_buffers(c, kNeedWarm, "ob_warmup_step")) != OB_OK) return r;
   DeviceGuard dg(c->device);
   if (!dg.ok) return fail(OB_ECUDA, "cannot select device %d", c->device);
   if ((r = check_grads(c, grads)) != OB_OK) return r;
@@ -463,6 +491,7 @@ ob_err ob_compress(ob_ctx* c, const void* grads, void* stream) {
   ob_err r = check_ctx(c);
   if (r != OB_OK) return r;
   if ((r = require_compressed(c, "ob_compress")) != OB_OK) return r;
+  if ((r = require_buffers(c, kNeedWorker, "ob_compress")) != OB_OK) return r;
   DeviceGuard dg(c->device);
   if (!dg.ok) return fail(OB_ECUDA, "cannot select device %d", c->device);
   if ((r = check_grads(c, grads)) != OB_OK) return r;
@@ -476,6 +505,7 @@ ob_err ob_server_reduce(ob_ctx* c, void* stream) {
   ob_err r = check_ctx(c);
   if (r != OB_OK) return r;
   if ((r = require_compressed(c, "ob_server_reduce")) != OB_OK) return r;
+  if ((r = require_buffers(c, kNeedServer, "ob_server_reduce")) != OB_OK) return r;
   DeviceGuard dg(c->device);
   if (!dg.ok) return fail(OB_ECUDA, "cannot select device %d", c->device);
   enqueue_server_stage(c, static_cast<cudaStream_t>(stream));
@@ -486,6 +516,8 @@ ob_err ob_step(ob_ctx* c, const void* grads, void* stream) {
   ob_err r = check_ctx(c);
   if (r != OB_OK) return r;
   if ((r = require_compressed(c, "ob_step")) != OB_OK) return r;
+  if ((r = require_buffers(c, grads ? (kNeedWorker | kNeedServer | kNeedUpdate) : kNeedUpdate, "ob_step")) != OB_OK)
+    return r;
   DeviceGuard dg(c->device);
   if (!dg.ok) return fail(OB_ECUDA, "cannot select device %d", c->device);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -503,6 +535,7 @@ ob_err ob_step_host(ob_ctx* c, const void* host_grads, void* dev_staging, void* 
   ob_err r = check_ctx(c);
   if (r != OB_OK) return r;
   if ((r = require_compressed(c, "ob_step_host")) != OB_OK) return r;
+  if ((r = require_buffers(c, kNeedWorker | kNeedServer | kNeedUpdate, "ob_step_host")) != OB_OK) return r;
   const int64_t count = int64_t(c->cfg.W) * c->cfg.n;
   if (count > 0 && !host_grads) return fail(OB_EINVAL, "host_grads is NULL");
   DeviceGuard dg(c->device);

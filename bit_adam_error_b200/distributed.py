@@ -1,0 +1,305 @@
+"""1-bit Adam across real GPUs: worker w = rank w, one process per GPU.
+
+The single-GPU library keeps W virtual workers in one GPU's memory.  Here the
+W workers are the ranks of a torch.distributed group and the compressed
+allreduce ("DeepSpeed Communication Compression and Hiding", section "1-bit
+Adam", 机制) becomes two exchanges of packed words:
+
+  1. every rank runs the worker stage on its own gradient (one worker):
+     signs + per-chunk scales + its worker error;
+  2. exchange 1: the words and scales of chunk k go to the rank that owns k;
+  3. every owner runs the server stage over the W workers of its chunks
+     (server error kept only by the owner);
+  4. exchange 2: the owners' server words and scales go to every rank;
+  5. every rank applies the update to its replica of p, m (v frozen).
+
+Chunks are owned whole (greedy balance by size), so each chunk's server scale
+and every float operation are the ones the single-GPU path (and the oracle)
+computes with W workers: the result is the same, bit for bit.  The flat
+buffer groups chunks by owner, so each exchange moves one contiguous slice
+per peer: about n/32 words plus C scales in each direction per step, 1/32 of an
+fp32 allreduce.  Warmup steps all-gather the full-precision gradients and run
+the W-worker warmup kernel, which sums them in rank order like the oracle.
+
+The arithmetic runs in the CUDA library (``CudaStages``); this module only
+plans the layout and moves packed words between ranks (NCCL on GPUs; gloo
+stages CUDA tensors through host memory).  The stage backend is an object with
+a fixed interface, so the exchange logic can also be exercised on CPU ranks.
+"""
+
+from __future__ import annotations
+
+from dataclasses import dataclass
+from typing import List, Optional, Sequence, Tuple
+
+import numpy as np
+import torch
+import torch.distributed as dist
+
+
+# ---- layout ------------------------------------------------------------------------
+
+@dataclass(frozen=True)
+class DPLayout:
+    """Chunk ownership and the owner-grouped flat layout.
+
+    ``sizes`` are the chunks in the caller's order; ``order`` lists them in
+    layout order (grouped by owner rank, ascending chunk index inside a group).
+    Offsets and word offsets are in layout order.
+    """
+
+    sizes: Tuple[int, ...]
+    world: int
+    owner: Tuple[int, ...]           # owner rank of each chunk (caller's order)
+    order: Tuple[int, ...]           # caller's chunk index at each layout position
+    offsets: np.ndarray              # [C+1] element offsets, layout order
+    words: np.ndarray                # [C+1] packed-word offsets, layout order
+    kbounds: Tuple[int, ...]         # [world+1] layout positions: rank r owns [kbounds[r], kbounds[r+1])
+
+    @property
+    def n(self) -> int:
+        return int(self.offsets[-1])
+
+    @property
+    def C(self) -> int:
+        return len(self.sizes)
+
+    def kslice(self, r: int) -> slice:
+        return slice(self.kbounds[r], self.kbounds[r + 1])
+
+    def eslice(self, r: int) -> slice:
+        return slice(int(self.offsets[self.kbounds[r]]), int(self.offsets[self.kbounds[r + 1]]))
+
+    def wslice(self, r: int) -> slice:
+        return slice(int(self.words[self.kbounds[r]]), int(self.words[self.kbounds[r + 1]]))
+
+    def to_layout(self, per_chunk: Sequence[np.ndarray]) -> np.ndarray:
+        """Concatenate per-chunk arrays (caller's order) in layout order."""
+        return np.concatenate([per_chunk[k] for k in self.order]) if self.C else np.zeros(0)
+
+    def chunk_position(self, k: int) -> int:
+        return self.order.index(k)
+
+
+def plan(sizes: Sequence[int], world: int) -> DPLayout:
+    """Assign chunks to ranks (largest first to the least-loaded rank, ties to the
+    lower rank) and lay the buffer out grouped by owner."""
+    sizes = tuple(int(s) for s in sizes)
+    if world < 1:
+        raise ValueError("world must be >= 1")
+    load = [0] * world
+    owner = [0] * len(sizes)
+    for k in sorted(range(len(sizes)), key=lambda k: (-sizes[k], k)):
+        r = min(range(world), key=lambda r: (load[r], r))
+        owner[k] = r
+        load[r] += sizes[k]
+    order = tuple(sorted(range(len(sizes)), key=lambda k: (owner[k], k)))
+    lay_sizes = [sizes[k] for k in order]
+    offsets = np.zeros(len(sizes) + 1, np.int64)
+    np.cumsum(np.asarray(lay_sizes, np.int64), out=offsets[1:])
+    words = np.zeros(len(sizes) + 1, np.int64)
+    np.cumsum(np.asarray([(s + 31) // 32 for s in lay_sizes], np.int64), out=words[1:])
+    kb = [0] * (world + 1)
+    for r in range(world):
+        kb[r + 1] = kb[r] + sum(1 for k in order if owner[k] == r)
+    return DPLayout(sizes, world, tuple(owner), order, offsets, words, tuple(kb))
+
+
+# ---- CUDA stage backend ------------------------------------------------------------------
+
+class CudaStages:
+    """Per-rank state and the C-ABI ctxs that compute on it.
+
+    local  (W = 1): p, m, v, this rank's err, its words/scales, the full server
+                    words/scales (filled by exchange 2) -> worker stage, update.
+    server (W = world, owned chunks only): srv_err, the W workers' words/scales
+                    of the owned chunks (filled by exchange 1) -> server stage.
+    warm   (W = world, shares p, m, v): the full-precision warmup step.
+    Phases are the driver's: every ctx is created with freeze_step 0 (local,
+    server) or never leaving warmup (warm).
+    """
+
+    def __init__(self, layout: DPLayout, rank: int, *, grad_dtype: str = "f32",
+                 optimizer: str = "adam", lr: float = 1e-4, beta1: float = 0.9,
+                 beta2: float = 0.999, eps: float = 1e-8, clip: float = 0.0,
+                 warmup: bool = True, device=None):
+        from . import _lib as L
+        self.L = L
+        self.device = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
+        self.layout, self.rank = layout, rank
+        W, n, C = layout.world, layout.n, layout.C
+        gd = L.OB_BF16 if grad_dtype == "bf16" else L.OB_F32
+        opt = L.OB_LAMB if optimizer == "lamb" else L.OB_ADAM
+        hp = dict(lr=lr, beta1=beta1, beta2=beta2, eps=eps, clip=clip)
+        dev, f32, i32 = self.device, torch.float32, torch.int32
+        words = int(layout.words[-1])
+        z = lambda shape, dt=f32: torch.zeros(shape, dtype=dt, device=dev)  # noqa: E731
+        self.p, self.m, self.v = z(n), z(n), z(n)
+        self.err = z((1, n))
+        self.bits_w, self.s_w = z((1, words), i32), z((1, C))
+        self.bits_srv, self.s_srv = z(words, i32), z(C)
+        ptr = lambda t: 0 if t is None or t.numel() == 0 else int(t.data_ptr())  # noqa: E731
+        self._keep = []
+
+        def cfg(offsets, workers, freeze):
+            c, arr = L.make_config(int(offsets[-1]), offsets, workers, gd, opt, freeze_step=freeze, **hp)
+            self._keep.append(arr)
+            return c
+
+        with torch.cuda.device(dev):
+            self.local = L.ob_create(cfg(layout.offsets, 1, 0), ptr(self.p), ptr(self.m), ptr(self.v),
+                                     ptr(self.err), 0, ptr(self.bits_w), ptr(self.s_w),
+                                     ptr(self.bits_srv), ptr(self.s_srv))
+            ks = layout.kslice(rank)
+            off_own = layout.offsets[ks.start: ks.stop + 1] - layout.offsets[ks.start]
+            self.n_own, self.C_own = int(off_own[-1]), ks.stop - ks.start
+            w_own = layout.wslice(rank).stop - layout.wslice(rank).start
+            self.srv_err = z(self.n_own)
+            self.bits_w_srv, self.s_w_srv = z((W, w_own), i32), z((W, self.C_own))
+            self.bits_srv_own, self.s_srv_own = z(w_own, i32), z(self.C_own)
+            self.server = 0
+            if self.C_own > 0:
+                self.server = L.ob_create(cfg(off_own, W, 0), 0, 0, 0, 0, ptr(self.srv_err),
+                                          ptr(self.bits_w_srv), ptr(self.s_w_srv),
+                                          ptr(self.bits_srv_own), ptr(self.s_srv_own))
+            self.warm = 0
+            if warmup:
+                self.warm = L.ob_create(cfg(layout.offsets, W, 1 << 30), ptr(self.p), ptr(self.m),
+                                        ptr(self.v), 0, 0, 0, 0, 0, 0)
+
+    def _stream(self) -> int:
+        return int(torch.cuda.current_stream(self.device).cuda_stream)
+
+    def warmup(self, gathered: torch.Tensor) -> None:
+        self.L.ob_warmup_step(self.warm, int(gathered.data_ptr()), self._stream())
+
+    def compress(self, grad: torch.Tensor) -> None:
+        self.L.ob_compress(self.local, int(grad.data_ptr()), self._stream())
+
+    def server_reduce(self) -> None:
+        if self.server:
+            self.L.ob_server_reduce(self.server, self._stream())
+
+    def apply(self) -> None:
+        self.L.ob_step(self.local, None, self._stream())
+
+    def status(self) -> int:
+        st = self._stream()
+        f = self.L.ob_get_status(self.local, False, st)
+        if self.server:
+            f |= self.L.ob_get_status(self.server, False, st)
+        if self.warm:
+            f |= self.L.ob_get_status(self.warm, False, st)
+        return f
+
+    def close(self) -> None:
+        for name in ("local", "server", "warm"):
+            h = getattr(self, name, 0)
+            if h:
+                self.L.ob_destroy(h)
+                setattr(self, name, 0)
+
+
+# ---- the data-parallel optimizer -------------------------------------------------------
+
+class DistributedOneBitAdam:
+    """One rank of data-parallel 1-bit Adam (worker w = rank w).
+
+    ``step(grad)`` takes this rank's gradient as a flat tensor in layout order
+    (``layout.to_layout`` / ``layout.eslice``) and runs a warmup step while
+    ``step_count < freeze_step``, the compressed step afterwards.
+    """
+
+    def __init__(self, layout: DPLayout, stages, *, freeze_step: int = 0, group=None):
+        self.layout, self.stages = layout, stages
+        self.group = group
+        self.rank = dist.get_rank(group)
+        self.world = dist.get_world_size(group)
+        if self.world != layout.world:
+            raise ValueError(f"layout planned for {layout.world} ranks, group has {self.world}")
+        self.freeze_step = int(freeze_step)
+        self.step_count = 0
+        self._stage_on_host = dist.get_backend(group) == "gloo"
+
+    # -- point-to-point with optional host staging (gloo has no CUDA transport) --
+    def _p2p(self, sends: List[Tuple[torch.Tensor, int]], recvs: List[Tuple[torch.Tensor, int]]) -> None:
+        host = self._stage_on_host
+        ops, copy_back = [], []
+        for t, peer in sends:
+            if t.numel():
+                src = t.detach().to("cpu") if host and t.is_cuda else t.contiguous()
+                ops.append(dist.P2POp(dist.isend, src, peer, self.group))
+        for t, peer in recvs:
+            if t.numel():
+                dst = torch.empty(t.shape, dtype=t.dtype) if host and t.is_cuda else t
+                ops.append(dist.P2POp(dist.irecv, dst, peer, self.group))
+                if dst is not t:
+                    copy_back.append((t, dst))
+        if ops:
+            for req in dist.batch_isend_irecv(ops):
+                req.wait()
+        for t, dst in copy_back:
+            t.copy_(dst)
+
+    def _to_owners(self) -> None:
+        """Exchange 1: this rank's words/scales of owner o's chunks -> rank o."""
+        L, s, r = self.layout, self.stages, self.rank
+        sends, recvs = [], []
+        for o in range(self.world):
+            wsl, ksl = L.wslice(o), L.kslice(o)
+            if o == r:
+                s.bits_w_srv[r].copy_(s.bits_w[0, wsl])
+                s.s_w_srv[r].copy_(s.s_w[0, ksl])
+            else:
+                sends += [(s.bits_w[0, wsl], o), (s.s_w[0, ksl], o)]
+                recvs += [(s.bits_w_srv[o], o), (s.s_w_srv[o], o)]
+        self._p2p(sends, recvs)
+
+    def _from_owners(self) -> None:
+        """Exchange 2: owner o's server words/scales -> every rank."""
+        L, s, r = self.layout, self.stages, self.rank
+        sends, recvs = [], []
+        for o in range(self.world):
+            wsl, ksl = L.wslice(o), L.kslice(o)
+            if o == r:
+                s.bits_srv[wsl].copy_(s.bits_srv_own)
+                s.s_srv[ksl].copy_(s.s_srv_own)
+            else:
+                sends += [(s.bits_srv_own, o), (s.s_srv_own, o)]
+                recvs += [(s.bits_srv[wsl], o), (s.s_srv[ksl], o)]
+        self._p2p(sends, recvs)
+
+    def _gather_grads(self, grad: torch.Tensor) -> torch.Tensor:
+        """All ranks' full-precision gradients, rank-major [world, n] (warmup)."""
+        if self._stage_on_host and grad.is_cuda:
+            parts = [torch.empty(grad.shape, dtype=grad.dtype) for _ in range(self.world)]
+            dist.all_gather(parts, grad.to("cpu"), group=self.group)
+            return torch.stack(parts).to(grad.device)
+        parts = [torch.empty_like(grad) for _ in range(self.world)]
+        dist.all_gather(parts, grad, group=self.group)
+        return torch.stack(parts)
+
+    @property
+    def in_warmup(self) -> bool:
+        return self.step_count < self.freeze_step
+
+    def step(self, grad: torch.Tensor) -> None:
+        if grad.numel() != self.layout.n:
+            raise ValueError(f"gradient must hold {self.layout.n} elements (layout order)")
+        if self.in_warmup:
+            self.stages.warmup(self._gather_grads(grad.reshape(-1)))
+        else:
+            self.stages.compress(grad)
+            self._to_owners()
+            self.stages.server_reduce()
+            self._from_owners()
+            self.stages.apply()
+        self.step_count += 1
+
+    def status(self) -> int:
+        """Status flags OR-ed over all ranks."""
+        f = torch.tensor([self.stages.status()], dtype=torch.int64)
+        if not self._stage_on_host and torch.cuda.is_available():
+            f = f.to(self.stages.device)
+        dist.all_reduce(f, op=dist.ReduceOp.MAX, group=self.group)  # one flag bit in use
+        return int(f.item())

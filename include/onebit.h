@@ -41,8 +41,8 @@
  *   - Calls return ob_err and never abort or trap.  On failure
  *     ob_last_error() returns a message (thread-local, valid until the next
  *     call on the same thread).
- *   - Calls on one ctx must be ordered (same stream, or synchronised); two
- *     ctxs may share no state buffer.
+ *   - Calls on one ctx must be ordered (same stream, or synchronised); ctxs
+ *     that share a state buffer must order their calls the same way.
  *   - The step counter advances in ob_warmup_step, ob_step and ob_step_host,
  *     never in the stage calls.
  */
@@ -92,6 +92,13 @@ ob_err ob_layout(const ob_config* cfg, int64_t* words_total);
  *   bits_w: uint32 [W][words_total];  s_w: [W][C];
  *   bits_srv: uint32 [words_total];  s_srv: [C].
  * Does not initialise them (the caller sets p, m, v; err and srv_err start at 0).
+ * A buffer may be NULL when the ctx never makes a call that touches it; calls
+ * return OB_EINVAL when one of theirs is missing:
+ *   ob_warmup_step: p, m, v          ob_compress: err, bits_w, s_w
+ *   ob_server_reduce: srv_err, bits_w, s_w, bits_srv, s_srv
+ *   ob_step(NULL): p, m, v, bits_srv, s_srv    ob_step(grads), ob_step_host: all
+ * (e.g. a rank that owns some chunks in a multi-GPU step keeps a server-only
+ * ctx).  Several ctxs may share a buffer if their calls are ordered.
  * Allocates the ctx scratch with cudaMalloc on the current device and
  * synchronises once.  *out receives the ctx (NULL on failure). */
 ob_err ob_create(const ob_config* cfg, float* p, float* m, float* v, float* err,

@@ -1,0 +1,248 @@
+"""Multi-rank harness for the data-parallel driver (bit_adam_error_b200.distributed).
+
+``OracleStages`` is a CPU stage backend with the interface of ``CudaStages``,
+computing with the oracle, so the driver's ownership plan and both exchanges
+run under gloo on CPU ranks; ``run_ranks`` spawns the ranks and collects each
+rank's final state; ``reference`` runs the same workload as one W-worker
+oracle problem in the caller's chunk order.  Test infrastructure only.
+"""
+
+from __future__ import annotations
+
+import datetime
+import os
+import socket
+import traceback
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+HP = dict(lr=1e-4, beta1=0.9, beta2=0.999, eps=1e-8)
+
+
+class OracleStages:
+    def __init__(self, layout, rank, optimizer="adam", clip=0.0):
+        import oracle
+        self.o = oracle.get()
+        self.layout, self.rank = layout, rank
+        self.opt = oracle.LAMB if optimizer == "lamb" else oracle.ADAM
+        self.clip = clip
+        self.device = torch.device("cpu")
+        W, n, C = layout.world, layout.n, layout.C
+        words = int(layout.words[-1])
+        f32, i32 = torch.float32, torch.int32
+        self.p, self.m, self.v = torch.zeros(n), torch.zeros(n), torch.zeros(n)
+        self.err = torch.zeros((1, n))
+        self.bits_w, self.s_w = torch.zeros((1, words), dtype=i32), torch.zeros((1, C))
+        self.bits_srv, self.s_srv = torch.zeros(words, dtype=i32), torch.zeros(C)
+        ks, wsl = layout.kslice(rank), layout.wslice(rank)
+        self.off_own = layout.offsets[ks.start: ks.stop + 1] - layout.offsets[ks.start]
+        self.srv_err = torch.zeros(int(self.off_own[-1]))
+        self.bits_w_srv = torch.zeros((W, wsl.stop - wsl.start), dtype=i32)
+        self.s_w_srv = torch.zeros((W, ks.stop - ks.start), dtype=f32)
+        self.bits_srv_own = torch.zeros(wsl.stop - wsl.start, dtype=i32)
+        self.s_srv_own = torch.zeros(ks.stop - ks.start, dtype=f32)
+        self.flags = 0
+
+    @staticmethod
+    def _u32(t):
+        return t.numpy().view(np.uint32)
+
+    def warmup(self, gathered):
+        f = {k: np.float32(v) for k, v in HP.items()}
+        self.flags |= self.o.warmup(self.layout.offsets, np.ascontiguousarray(gathered.numpy()),
+                                    self.m.numpy(), self.v.numpy(), self.p.numpy(), f["beta1"],
+                                    f["beta2"], f["lr"], f["eps"], optimizer=self.opt)
+
+    def compress(self, grad):
+        if grad.dtype == torch.bfloat16:
+            g = np.ascontiguousarray(grad.view(torch.int16).numpy().view(np.uint16).reshape(1, -1))
+        else:
+            g = np.ascontiguousarray(grad.numpy().reshape(1, -1))
+        bits, s, fl = self.o.compress(self.layout.offsets, g, self.err.numpy(), clip=self.clip)
+        self._u32(self.bits_w)[:] = bits
+        self.s_w.numpy()[:] = s
+        self.flags |= fl
+
+    def server_reduce(self):
+        if self.s_w_srv.shape[1] == 0:
+            return
+        bits, s, fl = self.o.server_reduce(self.off_own, np.ascontiguousarray(self._u32(self.bits_w_srv)),
+                                           np.ascontiguousarray(self.s_w_srv.numpy()), self.srv_err.numpy())
+        self._u32(self.bits_srv_own)[:] = bits
+        self.s_srv_own.numpy()[:] = s
+        self.flags |= fl
+
+    def apply(self):
+        f = {k: np.float32(v) for k, v in HP.items()}
+        args = (self.layout.offsets, self._u32(self.bits_srv), self.s_srv.numpy(), self.m.numpy(),
+                self.v.numpy(), self.p.numpy(), f["beta1"], f["lr"], f["eps"])
+        if self.opt:
+            self.flags |= self.o.lamb_apply(*args)[1]
+        else:
+            self.flags |= self.o.adam_apply(*args)
+
+    def status(self):
+        return self.flags
+
+
+def free_port() -> int:
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def workload(sizes, world, **kw):
+    import workloads as WL
+    return WL.get_workload("tiny").with_(sizes=tuple(sizes), W=world, **kw)
+
+
+def rank_inputs(wl, layout, rank, step):
+    """This rank's gradient at `step` in layout order (worker = rank)."""
+    import workloads as WL
+    return layout.to_layout([WL.chunk_grads(wl, step, rank, k) for k in range(wl.C)])
+
+
+def initial_state(wl, layout):
+    import workloads as WL
+    ps, vs = zip(*[WL.chunk_state(wl, k) for k in range(wl.C)])
+    return layout.to_layout(ps).astype(np.float32), layout.to_layout(vs).astype(np.float32)
+
+
+def _rank_main(rank, world, port, sizes, wl_kw, steps, backend, device, q):
+    try:
+        import sys
+        sys.path.insert(0, ROOT)
+        sys.path.insert(0, os.path.join(ROOT, "tests"))
+        import torch.distributed as dist
+        from bit_adam_error_b200.distributed import DistributedOneBitAdam, plan
+        os.environ["MASTER_ADDR"] = "127.0.0.1"
+        os.environ["MASTER_PORT"] = str(port)
+        if device != "cpu":
+            torch.cuda.set_device(torch.device(device))
+        dist.init_process_group(backend, rank=rank, world_size=world,
+                                timeout=datetime.timedelta(seconds=120))
+        wl = workload(sizes, world, **wl_kw)
+        layout = plan(sizes, world)
+        if device == "cpu":
+            stages = OracleStages(layout, rank, optimizer=wl.optimizer, clip=wl.clip)
+        else:
+            from bit_adam_error_b200.distributed import CudaStages
+            stages = CudaStages(layout, rank, grad_dtype=wl.grad_dtype, optimizer=wl.optimizer,
+                                clip=wl.clip, warmup=wl.freeze_step > 0, device=device, **HP)
+        p0, v0 = initial_state(wl, layout)
+        stages.p.copy_(torch.from_numpy(p0))
+        stages.v.copy_(torch.from_numpy(v0))
+        drv = DistributedOneBitAdam(layout, stages, freeze_step=wl.freeze_step)
+        for t in range(steps):
+            g = rank_inputs(wl, layout, rank, t)
+            gt = torch.from_numpy(g.view(np.int16)).view(torch.bfloat16) if g.dtype == np.uint16 \
+                else torch.from_numpy(g)
+            drv.step(gt.to(stages.device))
+        flags = drv.status()
+        if device != "cpu":
+            torch.cuda.synchronize()
+
+        def host(t):
+            a = t.detach().cpu().numpy()
+            return a.view(np.uint32) if a.dtype == np.int32 else a.copy()
+
+        out = {k: host(getattr(stages, k)) for k in ("p", "m", "v", "err", "srv_err", "bits_srv", "s_srv")}
+        out["flags"] = flags
+        if hasattr(stages, "close"):
+            stages.close()
+        dist.destroy_process_group()
+        q.put((rank, out))
+    except Exception:
+        q.put((rank, {"error": traceback.format_exc()}))
+
+
+def run_ranks(sizes, world, wl_kw, steps, backend="gloo", device="cpu", timeout=600):
+    """Spawn `world` ranks; returns the list of per-rank final states."""
+    import multiprocessing as mp
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = free_port()
+    procs = [ctx.Process(target=_rank_main, args=(r, world, port, sizes, wl_kw, steps, backend, device, q))
+             for r in range(world)]
+    for pr in procs:
+        pr.start()
+    results = {}
+    try:
+        for _ in range(world):
+            r, out = q.get(timeout=timeout)
+            results[r] = out
+    finally:
+        for pr in procs:
+            pr.join(timeout=30)
+            if pr.is_alive():
+                pr.kill()
+    for r, out in results.items():
+        assert "error" not in out, f"rank {r} failed:\n{out['error']}"
+    return [results[r] for r in range(world)]
+
+
+def reference(sizes, world, wl_kw, steps):
+    """The same workload as one W-worker oracle problem (caller's chunk order)."""
+    import oracle
+    import workloads as WL
+    wl = workload(sizes, world, **wl_kw)
+    o = oracle.get()
+    n = wl.n
+    p = np.zeros(n, np.float32)
+    v = np.zeros(n, np.float32)
+    WL.fill_state(wl, p, v)
+    st = {"p": p, "m": np.zeros(n, np.float32), "v": v, "err": np.zeros((world, n), np.float32),
+          "srv_err": np.zeros(n, np.float32)}
+    f = {k: np.float32(x) for k, x in HP.items()}
+    opt = oracle.LAMB if wl.optimizer == "lamb" else oracle.ADAM
+    for t in range(steps):
+        dt = np.uint16 if wl.grad_dtype == "bf16" else np.float32
+        g = np.zeros((world, n), dt)
+        WL.fill_grads(wl, t, g)
+        if t < wl.freeze_step:
+            o.warmup(wl.offsets, g, st["m"], st["v"], st["p"], f["beta1"], f["beta2"], f["lr"], f["eps"],
+                     optimizer=opt)
+        else:
+            o.step(wl.offsets, g, st, f["beta1"], f["lr"], f["eps"], clip=wl.clip, optimizer=opt)
+    return wl, st
+
+
+def compare(layout, wl, ref, outs, exact=True):
+    """Every rank's state against the W-worker oracle, mapped to layout order:
+    bit for bit (exact) or to the parity bar of the GPU tests."""
+    off = wl.offsets
+
+    def lay(a):  # caller-order flat array -> layout order
+        return layout.to_layout([a[..., off[k]:off[k + 1]] for k in range(wl.C)]) if a.ndim == 1 else \
+            np.stack([lay(r) for r in a])
+
+    wb = np.zeros(wl.C + 1, np.int64)
+    np.cumsum([(s + 31) // 32 for s in wl.sizes], out=wb[1:])
+    bits_ref = layout.to_layout([ref["bits_srv"][wb[k]:wb[k + 1]] for k in range(wl.C)]).astype(np.uint32)
+    s_ref = np.array([ref["s_srv"][k] for k in layout.order], np.float32)
+    srv_ref = lay(ref["srv_err"])
+    if exact:
+        same = lambda name, got, want: np.testing.assert_array_equal(got, want, err_msg=name)  # noqa: E731
+        scales = same
+    else:
+        from gpu_harness import assert_scales, assert_state
+        same = lambda name, got, want: assert_state(name, got, want, layout.offsets)  # noqa: E731
+        scales = assert_scales
+    for r, out in enumerate(outs):
+        for key in ("p", "m", "v"):
+            same(f"rank {r} {key}", out[key], lay(ref[key]))
+        same(f"rank {r} err", out["err"][0], lay(ref["err"][r]))
+        if "bits_w" in ref:
+            assert np.array_equal(out["bits_srv"], bits_ref), (r, "bits_srv")
+            scales(f"rank {r} s_srv", out["s_srv"], s_ref)
+            es = layout.eslice(r)
+            own_off = layout.offsets[layout.kslice(r).start: layout.kslice(r).stop + 1] - es.start
+            got, want = out["srv_err"], srv_ref[es]
+            if exact:
+                np.testing.assert_array_equal(got, want, err_msg=f"rank {r} srv_err")
+            else:
+                from gpu_harness import assert_state
+                assert_state(f"rank {r} srv_err", got, want, own_off)

@@ -1,0 +1,43 @@
+"""Data-parallel driver on CPU ranks (gloo, world size 2 and 3).
+
+The ranks exchange packed words with the driver's real exchange code; the
+per-rank arithmetic is the oracle (OracleStages).  Every rank's final state
+must equal the single-process W-worker oracle, bit for bit: chunk ownership
+and the two exchanges must not change a single operation.
+"""
+
+import numpy as np
+import pytest
+
+from bit_adam_error_b200.distributed import plan
+from dist_harness import compare, reference, run_ranks
+
+SIZES = [40, 1000, 64, 33, 2048, 7, 512, 96, 0, 300]
+
+
+def test_plan_balances_and_groups_by_owner():
+    lay = plan(SIZES, 3)
+    loads = [sum(SIZES[k] for k in range(len(SIZES)) if lay.owner[k] == r) for r in range(3)]
+    assert max(loads) - min(loads) <= max(SIZES)
+    assert [lay.owner[k] for k in lay.order] == sorted(lay.owner)
+    assert lay.offsets[-1] == sum(SIZES)
+    for r in range(3):
+        ks = lay.kslice(r)
+        assert all(lay.owner[lay.order[i]] == r for i in range(ks.start, ks.stop))
+    one = plan(SIZES, 1)
+    assert one.order == tuple(range(len(SIZES)))
+    many = plan([10, 20], 4)            # more ranks than chunks: some own nothing
+    assert sum(many.kslice(r).stop - many.kslice(r).start for r in range(4)) == 2
+
+
+@pytest.mark.parametrize("world,wl_kw,steps", [
+    (2, dict(), 4),
+    (3, dict(freeze_step=2), 4),
+    (2, dict(optimizer="lamb", freeze_step=1), 3),
+    (3, dict(grad_dtype="bf16", clip=5.0, grad_dist="student_t_zeros", zero_frac=0.05), 3),
+])
+def test_ranks_match_single_process_oracle(world, wl_kw, steps):
+    outs = run_ranks(SIZES, world, wl_kw, steps)
+    wl, ref = reference(SIZES, world, wl_kw, steps)
+    compare(plan(SIZES, world), wl, ref, outs)
+    assert all(o["flags"] == 0 for o in outs)
