@@ -62,6 +62,12 @@ def parse_args():
                     help="use only the first K chunks of the workload (a smaller case, e.g. for ncu)")
     ap.add_argument("--grad-buffers", type=int, default=2,
                     help="distinct gradient batches cycled through the timed steps")
+    ap.add_argument("--phase", choices=["compressed", "refresh"], default="compressed",
+                    help="time the compressed step (default) or the full-precision variance-refresh "
+                         "step of 0/1 Adam")
+    ap.add_argument("--dp", action="store_true",
+                    help="time the real data-parallel path (worker w = rank w, NCCL exchanges) "
+                         "instead of per-GPU replicas of the single-GPU step")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     a = ap.parse_args()
@@ -87,10 +93,14 @@ def algo_bytes_per_elem(kind: str, wl) -> float:
         return W / 8 + 8 + 1 / 8 + 20    # + m, v, p reads and m, p writes
     if kind == "k_lamb_param":           # m, v, p reads, p write
         return 16.0
+    if kind == "k_warmup":               # g (xW), m, v, p reads; m, v (+ p for Adam) writes
+        return gb * W + (20 if wl.optimizer == "lamb" else 24)
     return 0.0                           # finalisers: a few bytes per chunk
 
 
-def step_bytes_per_elem(wl) -> float:
+def step_bytes_per_elem(wl, phase: str = "compressed") -> float:
+    if phase == "refresh":
+        return algo_bytes_per_elem("k_warmup", wl) + (16.0 if wl.optimizer == "lamb" else 0.0)
     kinds = ["k_worker_norm", "k_worker_pack", "k_server_update"]
     if wl.optimizer == "lamb":
         kinds.append("k_lamb_param")
@@ -223,9 +233,10 @@ def max_over_ranks(dist, x: float, device) -> float:
 
 # -- CPU oracle timing ----------------------------------------------------------------------
 
-def oracle_rate(wl, chunks, max_elems=None, min_seconds=0.0, steps=1):
-    """Time the single-threaded oracle's compressed step on whole chunks (or on
-    the first max_elems elements of a chunk, taken as one chunk)."""
+def oracle_rate(wl, chunks, max_elems=None, min_seconds=0.0, steps=1, phase="compressed"):
+    """Time the single-threaded oracle's compressed step (or full-precision
+    refresh step) on whole chunks (or on the first max_elems elements of a
+    chunk, taken as one chunk)."""
     import oracle
     import workloads as WL
     o = oracle.get()
@@ -240,10 +251,14 @@ def oracle_rate(wl, chunks, max_elems=None, min_seconds=0.0, steps=1):
         p, v = WL.chunk_state(wl, k)
         st = {"p": p[:nk].copy(), "m": np.zeros(nk, np.float32), "v": v[:nk].copy(),
               "err": np.zeros((wl.W, nk), np.float32), "srv_err": np.zeros(nk, np.float32)}
+        opt = oracle.LAMB if wl.optimizer == "lamb" else oracle.ADAM
         for _ in range(steps):
             t = time.perf_counter()
-            o.step([0, nk], g, st, f(wl.beta1), f(wl.lr), f(wl.eps), clip=wl.clip,
-                   optimizer=oracle.LAMB if wl.optimizer == "lamb" else oracle.ADAM)
+            if phase == "refresh":
+                o.warmup([0, nk], g, st["m"], st["v"], st["p"], f(wl.beta1), f(wl.beta2), f(wl.lr),
+                         f(wl.eps), optimizer=opt)
+            else:
+                o.step([0, nk], g, st, f(wl.beta1), f(wl.lr), f(wl.eps), clip=wl.clip, optimizer=opt)
             dt = time.perf_counter() - t
             per_step.append(dt)
             secs += dt
@@ -335,12 +350,13 @@ def run_ours(args):
         dev_g.append(G)
     stream = torch.cuda.current_stream(device)
 
+    step_fn = opt.refresh_step if args.phase == "refresh" else opt.step
     for i in range(args.warmup):
-        opt.step(dev_g[i % nbuf])
+        step_fn(dev_g[i % nbuf])
     torch.cuda.synchronize()
 
     # -- timed region: inputs resident in HBM ------------------------------------
-    per_step_launches = 5 if wl.optimizer == "adam" else 7
+    per_step_launches = 8
     L.ob_profile_start(opt.ctx, args.steps * per_step_launches)
     launches0 = L.ob_launch_count(opt.ctx)
     sampler = ClockSampler(gpu_id(device))
@@ -352,7 +368,7 @@ def run_ours(args):
     w0 = time.time()
     e0.record(stream)
     for i in range(args.steps):
-        opt.step(dev_g[i % nbuf])
+        step_fn(dev_g[i % nbuf])
     e1.record(stream)
     torch.cuda.synchronize()
     w1 = time.time()
@@ -381,12 +397,14 @@ def run_ours(args):
                    "algorithmic_GBps": (algo_bytes_per_elem(k, wl) * n / (v[0] / v[1] / 1e3) / 1e9)
                    if algo_bytes_per_elem(k, wl) else None}
                for k, v in prof.items()}
-    step_gbs = step_bytes_per_elem(wl) * n / (ms_max / 1e3) / 1e9
+    step_gbs = step_bytes_per_elem(wl, args.phase) * n / (ms_max / 1e3) / 1e9
 
     # -- end to end: host gradients through the public call ---------------------------
     e2e = None
     host_bytes = W * n * wl.grad_bytes
-    if not args.no_e2e and host_bytes > E2E_MAX_HOST_BYTES:
+    if not args.no_e2e and args.phase != "compressed":
+        e2e = {"value": None, "unit": UNIT, "note": "host gradients are taken by the compressed step only"}
+    elif not args.no_e2e and host_bytes > E2E_MAX_HOST_BYTES:
         e2e = {"value": None, "unit": UNIT, "note": f"skipped: {host_bytes / 1e9:.1f} GB of pinned host "
                f"gradients per step exceeds the {E2E_MAX_HOST_BYTES / 1e9:.0f} GB cap"}
     elif not args.no_e2e:
@@ -418,10 +436,10 @@ def run_ours(args):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        elems, secs, _, used = oracle_rate(wl, list(range(wl.C)), min_seconds=10.0)
+        elems, secs, _, used = oracle_rate(wl, list(range(wl.C)), min_seconds=10.0, phase=args.phase)
         cpu = {"value": elems / secs / 1e9, "unit": UNIT, "cores": 1, "kind": "oracle",
                "sample": f"{len(used)} whole chunk(s) {[k for k, _ in used]} of {wl.name} "
-                         f"({elems} elements), one compressed step each, single thread, "
+                         f"({elems} elements), one {args.phase} step each, single thread, "
                          f"{secs:.1f} s"}
 
     if rank == 0:
@@ -430,8 +448,9 @@ def run_ours(args):
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
                 "data": "synthetic (seeded Philox streams; shapes and distributions of the workload)",
                 "config": workload_config(wl, world),
+                "phase": args.phase,
                 "hbm": {"step_achieved_GBps": step_gbs, "step_frac": step_gbs / peak,
-                        "algorithmic_bytes_per_elem": step_bytes_per_elem(wl), "peak": peak,
+                        "algorithmic_bytes_per_elem": step_bytes_per_elem(wl, args.phase), "peak": peak,
                         "peak_source": peak_src},
                 "roofline": roofline, "kernels": kernels, "cpu_baseline": cpu, "e2e": e2e,
                 "gpu_launches": launches, "status_flags": status, "clocks": clocks}
@@ -457,6 +476,75 @@ def fill_device_grads(wl, step, G) -> None:
             G[w, lo:hi].copy_(src)
 
 
+def run_dp(args):
+    """Data-parallel 1-bit Adam over the ranks: each rank is one worker (W = N),
+    compresses its own gradient, serves the chunks it owns and applies the update."""
+    import torch
+    world, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    import torch.distributed as tdist
+    if not tdist.is_initialized():
+        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+        os.environ.setdefault("MASTER_PORT", "29517")
+        os.environ.setdefault("RANK", str(rank))
+        os.environ.setdefault("WORLD_SIZE", str(world))
+        tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=device)
+    import workloads as WL
+    from bit_adam_error_b200.distributed import CudaStages, DistributedOneBitAdam, plan
+    wl = select_workload(args).with_(W=world, freeze_step=0)
+    layout = plan(wl.sizes, world)
+    stages = CudaStages(layout, rank, grad_dtype=wl.grad_dtype, optimizer=wl.optimizer, clip=wl.clip,
+                        lr=wl.lr, beta1=wl.beta1, beta2=wl.beta2, eps=wl.eps, warmup=False, device=device)
+    bf = wl.grad_dtype == "bf16"
+    gdt = torch.bfloat16 if bf else torch.float32
+    nbuf = max(1, args.grad_buffers)
+    G = [torch.empty(layout.n, dtype=gdt, device=device) for _ in range(nbuf)]
+    for pos, k in enumerate(layout.order):            # layout order: chunks grouped by owner
+        lo, hi = int(layout.offsets[pos]), int(layout.offsets[pos + 1])
+        p_h = np.empty(hi - lo, np.float32)
+        v_h = np.empty(hi - lo, np.float32)
+        WL.fill_state(wl, p_h, v_h, chunks=(k, k + 1))
+        stages.p[lo:hi].copy_(torch.from_numpy(p_h))
+        stages.v[lo:hi].copy_(torch.from_numpy(v_h))
+        for b in range(nbuf):
+            row = np.empty(hi - lo, np.uint16 if bf else np.float32)
+            WL.fill_grads_row(wl, b, rank, row, chunks=(k, k + 1))
+            src = torch.from_numpy(row.view(np.int16)).view(torch.bfloat16) if bf else torch.from_numpy(row)
+            G[b][lo:hi].copy_(src)
+    drv = DistributedOneBitAdam(layout, stages, freeze_step=0)
+    stream = torch.cuda.current_stream(device)
+    for i in range(args.warmup):
+        drv.step(G[i % nbuf])
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(tdist)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for i in range(args.steps):
+        drv.step(G[i % nbuf])
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier(tdist)
+    ms = max_over_ranks(tdist, e0.elapsed_time(e1) / args.steps, device)
+    flags = drv.status()
+    if rank == 0:
+        own = [layout.eslice(r).stop - layout.eslice(r).start for r in range(world)]
+        line = {"metric": METRIC, "value": world * layout.n / (ms / 1e3) / 1e9, "unit": UNIT,
+                "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+                "data": "synthetic (seeded Philox streams; shapes and distributions of the workload)",
+                "config": dict(workload_config(wl, world), parallelism=f"dp{world}: worker w = rank w, "
+                               f"chunk-owner server stage, NCCL point-to-point exchanges",
+                               owned_elements=own),
+                "exchange_bytes_per_step_per_rank": 2 * 4 * (int(layout.words[-1]) + layout.C),
+                "status_flags": flags, "e2e": None}
+        print(json.dumps(line), flush=True)
+    stages.close()
+    tdist.destroy_process_group()
+    return 0
+
+
 def gpu_id(device) -> str:
     import torch
     try:
@@ -469,6 +557,8 @@ def main():
     args = parse_args()
     if args.impl == "reference":
         return run_reference(args)
+    if args.dp:
+        return run_dp(args)
     return run_ours(args)
 
 

@@ -51,6 +51,7 @@ _SIGS = {
     "ob_create": (ctypes.c_int, [ctypes.POINTER(ob_config), _P, _P, _P, _P, _P, _P, _P, _P, _P,
                                  ctypes.POINTER(_P)]),
     "ob_warmup_step": (ctypes.c_int, [_P, _P, _P]),
+    "ob_refresh_step": (ctypes.c_int, [_P, _P, _P]),
     "ob_compress": (ctypes.c_int, [_P, _P, _P]),
     "ob_server_reduce": (ctypes.c_int, [_P, _P]),
     "ob_step": (ctypes.c_int, [_P, _P, _P]),
@@ -129,6 +130,10 @@ def ob_create(cfg: ob_config, p, m, v, err, srv_err, bits_w, s_w, bits_srv, s_sr
 
 def ob_warmup_step(ctx: int, grads: int, stream: int) -> None:
     check(load().ob_warmup_step(ctx, grads, stream), "ob_warmup_step")
+
+
+def ob_refresh_step(ctx: int, grads: int, stream: int) -> None:
+    check(load().ob_refresh_step(ctx, grads, stream), "ob_refresh_step")
 
 
 def ob_compress(ctx: int, grads: int, stream: int) -> None:

@@ -104,6 +104,13 @@ struct ob_ctx {
   ob::Hyper h{};
   const void* grads_checked = nullptr;   // last grads pointer that passed check_dev
   std::vector<std::pair<const void*, int>> occ;  // kernel -> resident CTAs per SM
+  // ob_step_host: internal copy stream, "copied" event, and per staging buffer
+  // an event recorded after the last kernels that read it.
+  cudaStream_t copy_stream = nullptr;
+  cudaEvent_t copied = nullptr;
+  struct Staging { const void* ptr = nullptr; cudaEvent_t free_ev = nullptr; bool used = false; };
+  Staging staging[4];
+  int staging_next = 0;
   // profiling: event pairs around launches
   int64_t launches = 0;
   bool prof_on = false;
@@ -469,22 +476,38 @@ ob_err ob_create(const ob_config* cfg, float* p, float* m, float* v, float* err,
   return OB_OK;
 }
 
-ob_err ob_warmup_step(ob_ctx* c, const void* grads, void* stream) {
-  ob_err r = check_ctx(c);
+namespace {
+
+// Full-precision step (warmup, or a 0/1 Adam variance refresh): no phase check.
+ob_err full_precision_step(ob_ctx* c, const void* grads, void* stream, const char* call) {
+  ob_err r = require_buffers(c, kNeedWarm, call);
   if (r != OB_OK) return r;
-  if (c->step >= c->cfg.freeze_step)
-    return fail(OB_EPHASE, "ob_warmup_step: step %lld >= freeze_step %d", (long long)c->step,
-                c->cfg.freeze_step);
-  if ((r = require_buffers(c, kNeedWarm, "ob_warmup_step")) != OB_OK) return r;
   DeviceGuard dg(c->device);
   if (!dg.ok) return fail(OB_ECUDA, "cannot select device %d", c->device);
   if ((r = check_grads(c, grads)) != OB_OK) return r;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (c->cfg.grad_dtype == OB_BF16) enqueue_warmup<uint16_t>(c, static_cast<const uint16_t*>(grads), st);
   else enqueue_warmup<float>(c, static_cast<const float*>(grads), st);
-  if ((r = check_launch("ob_warmup_step")) != OB_OK) return r;
+  if ((r = check_launch(call)) != OB_OK) return r;
   ++c->step;
   return OB_OK;
+}
+
+}  // namespace
+
+ob_err ob_warmup_step(ob_ctx* c, const void* grads, void* stream) {
+  ob_err r = check_ctx(c);
+  if (r != OB_OK) return r;
+  if (c->step >= c->cfg.freeze_step)
+    return fail(OB_EPHASE, "ob_warmup_step: step %lld >= freeze_step %d", (long long)c->step,
+                c->cfg.freeze_step);
+  return full_precision_step(c, grads, stream, "ob_warmup_step");
+}
+
+ob_err ob_refresh_step(ob_ctx* c, const void* grads, void* stream) {
+  ob_err r = check_ctx(c);
+  if (r != OB_OK) return r;
+  return full_precision_step(c, grads, stream, "ob_refresh_step");
 }
 
 ob_err ob_compress(ob_ctx* c, const void* grads, void* stream) {
@@ -531,6 +554,27 @@ ob_err ob_step(ob_ctx* c, const void* grads, void* stream) {
   return OB_OK;
 }
 
+namespace {
+
+// The staging slot of `ptr`, created (with its event) on first use; with more
+// than 4 distinct buffers the oldest slot is recycled after its event completes.
+ob_err staging_slot(ob_ctx* c, const void* ptr, ob_ctx::Staging** out) {
+  for (auto& s : c->staging)
+    if (s.ptr == ptr && s.free_ev) { *out = &s; return OB_OK; }
+  ob_ctx::Staging& s = c->staging[c->staging_next];
+  c->staging_next = (c->staging_next + 1) % 4;
+  cudaError_t e = cudaSuccess;
+  if (s.free_ev && s.used) e = cudaEventSynchronize(s.free_ev);
+  if (e == cudaSuccess && !s.free_ev) e = cudaEventCreateWithFlags(&s.free_ev, cudaEventDisableTiming);
+  if (e != cudaSuccess) return cuda_fail(e, "ob_step_host: staging event");
+  s.ptr = ptr;
+  s.used = false;
+  *out = &s;
+  return OB_OK;
+}
+
+}  // namespace
+
 ob_err ob_step_host(ob_ctx* c, const void* host_grads, void* dev_staging, void* stream) {
   ob_err r = check_ctx(c);
   if (r != OB_OK) return r;
@@ -543,17 +587,41 @@ ob_err ob_step_host(ob_ctx* c, const void* host_grads, void* dev_staging, void* 
   if ((r = check_grads(c, dev_staging)) != OB_OK) return r;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const size_t bytes = size_t(count) * (c->cfg.grad_dtype == OB_BF16 ? 2 : 4);
+  ob_ctx::Staging* slot = nullptr;
   if (bytes > 0) {
-    cudaError_t e = cudaMemcpyAsync(dev_staging, host_grads, bytes, cudaMemcpyHostToDevice, st);
+    cudaError_t e = cudaSuccess;
+    if (!c->copy_stream) e = cudaStreamCreateWithFlags(&c->copy_stream, cudaStreamNonBlocking);
+    if (e == cudaSuccess && !c->copied) e = cudaEventCreateWithFlags(&c->copied, cudaEventDisableTiming);
+    if (e != cudaSuccess) return cuda_fail(e, "ob_step_host: copy stream");
+    if ((r = staging_slot(c, dev_staging, &slot)) != OB_OK) return r;
+    // The upload waits only for the kernels that last read this staging buffer,
+    // so it overlaps the compute of the step before when buffers alternate.
+    if (slot->used) e = cudaStreamWaitEvent(c->copy_stream, slot->free_ev, 0);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(dev_staging, host_grads, bytes, cudaMemcpyHostToDevice, c->copy_stream);
+    if (e == cudaSuccess) e = cudaEventRecord(c->copied, c->copy_stream);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(st, c->copied, 0);
     if (e != cudaSuccess) return cuda_fail(e, "ob_step_host: host-to-device copy");
   }
-  return fused_step(c, dev_staging, st);
+  if ((r = fused_step(c, dev_staging, st)) != OB_OK) return r;
+  if (slot) {
+    cudaError_t e = cudaEventRecord(slot->free_ev, st);
+    if (e != cudaSuccess) return cuda_fail(e, "ob_step_host: staging event");
+    slot->used = true;
+  }
+  return OB_OK;
 }
 
 ob_err ob_destroy(ob_ctx* c) {
   if (!c) return OB_OK;
   ob_err r = OB_OK;
   for (auto& ev : c->prof_ev) cudaEventDestroy(ev);
+  if (c->copy_stream) {
+    cudaStreamSynchronize(c->copy_stream);
+    cudaStreamDestroy(c->copy_stream);
+  }
+  if (c->copied) cudaEventDestroy(c->copied);
+  for (auto& s : c->staging)
+    if (s.free_ev) cudaEventDestroy(s.free_ev);
   if (c->scratch) {
     DeviceGuard dg(c->device);
     cudaError_t e = cudaFree(c->scratch);

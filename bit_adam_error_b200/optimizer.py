@@ -72,7 +72,8 @@ class OneBitAdam:
             self.ctx = L.ob_create(self.cfg, _ptr(self.p), _ptr(self.m), _ptr(self.v),
                                    _ptr(self.err), _ptr(self.srv_err), _ptr(self.bits_w),
                                    _ptr(self.s_w), _ptr(self.bits_srv), _ptr(self.s_srv))
-        self._staging: Optional[torch.Tensor] = None
+        self._staging: list = []       # two device buffers for host gradients, used alternately
+        self._staging_turn = 0
 
     # -- plumbing -----------------------------------------------------------------
     def _stream(self) -> int:
@@ -104,17 +105,23 @@ class OneBitAdam:
 
         Device gradients run the warmup or the fused compressed step in place;
         CPU gradients (pinned for an asynchronous copy) go through
-        ``ob_step_host`` with a device staging buffer (compressed phase only).
+        ``ob_step_host`` with two device staging buffers used alternately, so
+        the upload of a step's gradients overlaps the previous step's compute
+        (compressed phase only; keep the host tensor unchanged until the
+        current stream has passed the step).
         """
         if grads.device.type == "cpu":
             if self.in_warmup:
                 raise L.OneBitError(L.OB_EPHASE, "step", "host gradients are taken in the compressed phase only")
-            if self._staging is None:
-                self._staging = torch.empty((self.W, self.n), dtype=self.grad_torch_dtype, device=self.device)
             if grads.dtype != self.grad_torch_dtype or not grads.is_contiguous() \
                     or grads.numel() != self.W * self.n:
                 raise ValueError("host grads must be contiguous, of the configured dtype and size")
-            L.ob_step_host(self.ctx, _ptr(grads), _ptr(self._staging), self._stream())
+            if not self._staging:
+                self._staging = [torch.empty((self.W, self.n), dtype=self.grad_torch_dtype, device=self.device)
+                                 for _ in range(2)]
+            staging = self._staging[self._staging_turn]
+            self._staging_turn ^= 1
+            L.ob_step_host(self.ctx, _ptr(grads), _ptr(staging), self._stream())
             return
         g = self._grads_ptr(grads)
         if self.in_warmup:
@@ -124,6 +131,11 @@ class OneBitAdam:
 
     def warmup_step(self, grads: torch.Tensor) -> None:
         L.ob_warmup_step(self.ctx, self._grads_ptr(grads), self._stream())
+
+    def refresh_step(self, grads: torch.Tensor) -> None:
+        """0/1 Adam variance refresh: a full-precision step (m and v) in any phase;
+        error buffers untouched.  Which steps refresh is the caller's schedule."""
+        L.ob_refresh_step(self.ctx, self._grads_ptr(grads), self._stream())
 
     def compress(self, grads: torch.Tensor) -> None:
         """Worker stage: err, bits_w, s_w."""

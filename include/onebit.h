@@ -111,6 +111,15 @@ ob_err ob_create(const ob_config* cfg, float* p, float* m, float* v, float* err,
  * grads: DEVICE [W][n] of grad_dtype.  Error buffers are not touched. */
 ob_err ob_warmup_step(ob_ctx* ctx, const void* grads, void* stream);
 
+/* Variance refresh of 0/1 Adam ("DeepSpeed Communication Compression and
+ * Hiding", section "0/1 Adam"): the same full-precision step as
+ * ob_warmup_step -- Adam (or LAMB) moments m AND v from the averaged gradient,
+ * then the parameter update -- allowed in any phase, so the frozen variance is
+ * refreshed between compressed steps.  Error buffers are not touched.  The
+ * pages give no refresh schedule; the caller chooses the steps.  Advances the
+ * step counter. */
+ob_err ob_refresh_step(ob_ctx* ctx, const void* grads, void* stream);
+
 /* Worker stage only (compressed phase): for every worker and chunk,
  * c = clip(g_w) + err_w, s_w = ||c|| / sqrt(n_k), bits_w = sign(c),
  * err_w = c - s_w sign(c).  grads: DEVICE [W][n].  Step counter unchanged. */
@@ -128,10 +137,15 @@ ob_err ob_server_reduce(ob_ctx* ctx, void* stream);
 ob_err ob_step(ob_ctx* ctx, const void* grads, void* stream);
 
 /* Same as ob_step(ctx, grads, ...) with the gradients in HOST memory:
- * enqueues one host-to-device copy of [W][n] grad_dtype elements from
- * host_grads into dev_staging (a caller-owned DEVICE buffer of that size,
- * 32-byte aligned), then the fused step.  host_grads should be page-locked
- * for the copy to be asynchronous.  Advances the step counter. */
+ * copies [W][n] grad_dtype elements from host_grads into dev_staging (a
+ * caller-owned DEVICE buffer of that size, 32-byte aligned), then runs the
+ * fused step on `stream`.  The copy runs on an internal copy stream (created on
+ * the first call, with a few events) and waits only for the kernels that last
+ * read the same dev_staging buffer; `stream` waits for the copy.  Passing two
+ * staging buffers alternately therefore overlaps the upload of one step's
+ * gradients with the previous step's compute.  host_grads should be page-
+ * locked, and must stay unchanged until `stream` has passed this step.
+ * Advances the step counter. */
 ob_err ob_step_host(ob_ctx* ctx, const void* host_grads, void* dev_staging, void* stream);
 
 /* Destroy a ctx and free its scratch (not the caller's buffers).  NULL is OK. */

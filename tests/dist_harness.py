@@ -111,7 +111,7 @@ def initial_state(wl, layout):
     return layout.to_layout(ps).astype(np.float32), layout.to_layout(vs).astype(np.float32)
 
 
-def _rank_main(rank, world, port, sizes, wl_kw, steps, backend, device, q):
+def _rank_main(rank, world, port, sizes, wl_kw, steps, backend, device, q, die=None, timeout_s=120):
     try:
         import sys
         sys.path.insert(0, ROOT)
@@ -123,7 +123,7 @@ def _rank_main(rank, world, port, sizes, wl_kw, steps, backend, device, q):
         if device != "cpu":
             torch.cuda.set_device(torch.device(device))
         dist.init_process_group(backend, rank=rank, world_size=world,
-                                timeout=datetime.timedelta(seconds=120))
+                                timeout=datetime.timedelta(seconds=timeout_s))
         wl = workload(sizes, world, **wl_kw)
         layout = plan(sizes, world)
         if device == "cpu":
@@ -137,6 +137,8 @@ def _rank_main(rank, world, port, sizes, wl_kw, steps, backend, device, q):
         stages.v.copy_(torch.from_numpy(v0))
         drv = DistributedOneBitAdam(layout, stages, freeze_step=wl.freeze_step)
         for t in range(steps):
+            if die is not None and die == (rank, t):
+                os._exit(17)             # an injected rank failure between steps
             g = rank_inputs(wl, layout, rank, t)
             gt = torch.from_numpy(g.view(np.int16)).view(torch.bfloat16) if g.dtype == np.uint16 \
                 else torch.from_numpy(g)
@@ -246,3 +248,27 @@ def compare(layout, wl, ref, outs, exact=True):
             else:
                 from gpu_harness import assert_state
                 assert_state(f"rank {r} srv_err", got, want, own_off)
+
+
+def run_with_dead_rank(sizes, world, wl_kw, steps, die, timeout_s=15):
+    """Spawn the ranks with rank die[0] exiting before its step die[1]; returns
+    ({rank: result or error}, {rank: exit code})."""
+    import multiprocessing as mp
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = free_port()
+    procs = [ctx.Process(target=_rank_main, args=(r, world, port, sizes, wl_kw, steps, "gloo", "cpu", q,
+                                                  die, timeout_s)) for r in range(world)]
+    for pr in procs:
+        pr.start()
+    results = {}
+    try:
+        for _ in range(world - 1):
+            r, out = q.get(timeout=timeout_s * 6)
+            results[r] = out
+    finally:
+        for pr in procs:
+            pr.join(timeout=30)
+            if pr.is_alive():
+                pr.kill()
+    return results, {r: pr.exitcode for r, pr in enumerate(procs)}

@@ -6,11 +6,13 @@ must equal the single-process W-worker oracle, bit for bit: chunk ownership
 and the two exchanges must not change a single operation.
 """
 
+import time
+
 import numpy as np
 import pytest
 
 from bit_adam_error_b200.distributed import plan
-from dist_harness import compare, reference, run_ranks
+from dist_harness import compare, reference, run_ranks, run_with_dead_rank
 
 SIZES = [40, 1000, 64, 33, 2048, 7, 512, 96, 0, 300]
 
@@ -41,3 +43,13 @@ def test_ranks_match_single_process_oracle(world, wl_kw, steps):
     wl, ref = reference(SIZES, world, wl_kw, steps)
     compare(plan(SIZES, world), wl, ref, outs)
     assert all(o["flags"] == 0 for o in outs)
+
+
+def test_a_dead_rank_ends_the_others_step_with_an_error():
+    """Failure detection on the host: rank 1 exits between steps; rank 0's next
+    exchange must fail (peer gone or process-group timeout), not hang."""
+    t0 = time.monotonic()
+    results, codes = run_with_dead_rank(SIZES, 2, dict(), steps=3, die=(1, 1), timeout_s=10)
+    assert codes[1] == 17
+    assert "error" in results[0], "the surviving rank finished instead of reporting the lost peer"
+    assert time.monotonic() - t0 < 120

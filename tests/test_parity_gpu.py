@@ -309,3 +309,72 @@ def test_host_buffer_entry_point_matches_device_path():
     for k in ("p", "m", "err", "srv_err", "bits_srv"):
         assert np.array_equal(np_of(getattr(a, k)), np_of(getattr(b, k))), k
     assert b.step_count == 3
+
+
+def test_host_entry_overlapped_steps_match_device_path():
+    """Back-to-back host-gradient steps (no synchronisation between them): the
+    upload of step t+1 overlaps step t's compute through the internal copy
+    stream and the alternating staging buffers; results equal the device path."""
+    wl = small([1 << 20, 4096, 40], 2)
+    p, v = state_for(wl)
+    a = OneBitAdam(wl.offsets, 2, device=dev(), p=to_dev(p), v=to_dev(v), **HP)
+    b = OneBitAdam(wl.offsets, 2, device=dev(), p=to_dev(p), v=to_dev(v), **HP)
+    hosts = [torch.from_numpy(grads_for(wl, t)).pin_memory() for t in range(4)]
+    for t in range(4):
+        a.step(hosts[t].to(dev()))
+    for t in range(4):
+        b.step(hosts[t])                 # no synchronisation in between
+    torch.cuda.synchronize()
+    for k in ("p", "m", "err", "srv_err", "bits_srv", "s_srv"):
+        assert np.array_equal(np_of(getattr(a, k)), np_of(getattr(b, k))), k
+    assert b.step_count == 4
+
+
+def test_step_replays_from_a_cuda_graph():
+    """The fused step's launches capture into a CUDA graph; replaying it equals
+    eager execution bit for bit (small workloads are launch-bound)."""
+    wl = WL.get_workload("tiny")
+    p, v = state_for(wl)
+    eager = OneBitAdam(wl.offsets, wl.W, device=dev(), p=to_dev(p), v=to_dev(v), **HP)
+    graphed = OneBitAdam(wl.offsets, wl.W, device=dev(), p=to_dev(p), v=to_dev(v), **HP)
+    G = torch.empty((wl.W, wl.n), dtype=torch.float32, device=dev())
+    s = torch.cuda.Stream(device=dev())
+    s.wait_stream(torch.cuda.current_stream())
+    graph = torch.cuda.CUDAGraph()
+    G.copy_(to_dev(grads_for(wl, 0)))
+    with torch.cuda.stream(s):
+        graphed.step(G)                   # first call outside capture (occupancy queries)
+    torch.cuda.current_stream().wait_stream(s)
+    with torch.cuda.graph(graph, stream=s):
+        graphed.step(G)
+    graphed.set_step(1)                   # the capture call counted a step without running it
+    eager.step(to_dev(grads_for(wl, 0)))
+    for t in range(1, 4):
+        gt = to_dev(grads_for(wl, t))
+        eager.step(gt)
+        G.copy_(gt)
+        graph.replay()
+    torch.cuda.synchronize()
+    for k in ("p", "m", "err", "srv_err", "bits_srv", "s_srv"):
+        assert np.array_equal(np_of(getattr(eager, k)), np_of(getattr(graphed, k))), k
+
+
+@pytest.mark.parametrize("opt", ["adam", "lamb"])
+def test_zero_one_adam_variance_refresh(opt):
+    """0/1 Adam: full-precision refresh steps (m and v) interleaved with
+    compressed steps; error buffers carry through the refreshes untouched."""
+    wl = small(ALIGNED, 3, optimizer=opt)
+    p, v = state_for(wl)
+    pr = Pair(wl.offsets, 3, optimizer=opt, p0=p, v0=v)
+    o = oracle.get()
+    for t, refresh in enumerate([False, False, True, False, True, True, False]):
+        g = grads_for(wl, t)
+        if refresh:
+            pr.gpu.refresh_step(to_dev(g))
+            r = pr.ref
+            o.warmup(wl.offsets, g, r["m"], r["v"], r["p"], F["beta1"], F["beta2"], F["lr"], F["eps"],
+                     optimizer=pr.opt_code)
+        else:
+            pr.step(g, warm=False)
+        pr.compare(tag=f"step {t} ", bits=not refresh)
+    assert pr.gpu.step_count == 7 and pr.gpu.status() == 0
