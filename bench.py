@@ -399,6 +399,18 @@ def run_ours(args):
                for k, v in prof.items()}
     step_gbs = step_bytes_per_elem(wl, args.phase) * n / (ms_max / 1e3) / 1e9
 
+    # -- error-buffer monitoring (one call, timed alone) -----------------------------
+    monitor = None
+    if args.phase == "compressed":
+        e0.record(stream)
+        opt.error_norms()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        mon_ms = e0.elapsed_time(e1)
+        mon_bytes = 4 * n * (W + 1)
+        monitor = {"ms": mon_ms, "GBps": mon_bytes / (mon_ms / 1e3) / 1e9,
+                   "frac": mon_bytes / (mon_ms / 1e3) / 1e9 / peak, "bytes": mon_bytes}
+
     # -- end to end: host gradients through the public call ---------------------------
     e2e = None
     host_bytes = W * n * wl.grad_bytes
@@ -452,7 +464,8 @@ def run_ours(args):
                 "hbm": {"step_achieved_GBps": step_gbs, "step_frac": step_gbs / peak,
                         "algorithmic_bytes_per_elem": step_bytes_per_elem(wl, args.phase), "peak": peak,
                         "peak_source": peak_src},
-                "roofline": roofline, "kernels": kernels, "cpu_baseline": cpu, "e2e": e2e,
+                "roofline": roofline, "kernels": kernels, "error_norms_call": monitor,
+                "cpu_baseline": cpu, "e2e": e2e,
                 "gpu_launches": launches, "status_flags": status, "clocks": clocks}
         print(json.dumps(line), flush=True)
     opt.close()

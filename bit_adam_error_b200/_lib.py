@@ -65,6 +65,7 @@ _SIGS = {
     "ob_kernel_name": (ctypes.c_char_p, [ctypes.c_int32]),
     "ob_launch_count": (ctypes.c_int64, [_P]),
     "ob_compress_noalloc": (ctypes.c_int, [ctypes.POINTER(ob_config), _P, _P, _P, _P, _P]),
+    "ob_error_norms": (ctypes.c_int, [_P, _P, _P, _P]),
     "ob_last_error": (ctypes.c_char_p, []),
 }
 
@@ -168,6 +169,10 @@ def ob_get_step(ctx) -> int:
 
 def ob_set_step(ctx: int, step: int) -> None:
     check(load().ob_set_step(ctx, step), "ob_set_step")
+
+
+def ob_error_norms(ctx: int, worker_norms: int, server_norms: int, stream: int) -> None:
+    check(load().ob_error_norms(ctx, worker_norms, server_norms, stream), "ob_error_norms")
 
 
 def ob_profile_start(ctx: int, capacity: int) -> None:

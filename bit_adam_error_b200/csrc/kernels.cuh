@@ -305,6 +305,7 @@ __device__ __forceinline__ double block_sum_fixed(double x, double* sm) {
   return r;
 }
 
+template <bool RMS>
 __global__ void __launch_bounds__(kFinalizeThreads)
 k_finalize_scale(Layout L, const double* __restrict__ part, const int64_t* __restrict__ tpx,
                  int mult, int64_t row_stride, float* __restrict__ out) {
@@ -316,9 +317,10 @@ k_finalize_scale(Layout L, const double* __restrict__ part, const int64_t* __res
   const double S = block_sum_fixed(acc, sm);
   if (threadIdx.x == 0) {
     const int64_t nk = L.off[k + 1] - L.off[k];
-    out[static_cast<int64_t>(r) * L.C + k] =
-        nk > 0 ? __double2float_rn(__ddiv_rn(__dsqrt_rn(S), __dsqrt_rn(static_cast<double>(nk))))
-               : 0.0f;
+    float o = 0.0f;
+    if (!RMS) o = __double2float_rn(__dsqrt_rn(S));   // plain L2 norm (monitoring)
+    else if (nk > 0) o = __double2float_rn(__ddiv_rn(__dsqrt_rn(S), __dsqrt_rn(static_cast<double>(nk))));
+    out[static_cast<int64_t>(r) * L.C + k] = o;
   }
 }
 
@@ -649,6 +651,43 @@ k_server_update(Layout L, int W, const uint32_t* __restrict__ bits_w, const floa
       if (lane == 0) { partP[t] = Psum; partU[t] = Usum; }
     }
     flag_nonfinite(bad, status);
+  }
+}
+
+// ---- monitoring: per-tile sums of squares of R fp32 rows [R][n] --------------------------
+__global__ void __launch_bounds__(kBlock)
+k_rows_sumsq(Layout L, int R, const float* __restrict__ x, double* __restrict__ part) {
+  const int lane = threadIdx.x & 31;
+  const int64_t items = static_cast<int64_t>(R) * L.T;
+  int hint = 0;
+  for (int64_t it = warp_id(); it < items; it += warp_count()) {
+    const int r = static_cast<int>(it / L.T);
+    const int64_t t = it - static_cast<int64_t>(r) * L.T;
+    const Tile tl = tile_at(L, t, hint);
+    const float* row = x + static_cast<int64_t>(r) * L.n + tl.ck0;
+    double acc = 0.0;
+    if (tl.vec) {
+#pragma unroll
+      for (int q = 0; q < kGroups; ++q) {
+        const int64_t i0 = tl.rel + q * kGroupElems + lane * kVec;
+        if (i0 < tl.nk) {
+          float v[8];
+          ld8_ro(row + i0, v);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) acc = fma(static_cast<double>(v[j]), static_cast<double>(v[j]), acc);
+        }
+      }
+    } else {
+      for (int j = 0; j < kTileWords; ++j) {
+        const int64_t i = tl.rel + j * 32 + lane;
+        if (i < tl.nk) {
+          const float v = __ldg(row + i);
+          acc = fma(static_cast<double>(v), static_cast<double>(v), acc);
+        }
+      }
+    }
+    acc = warp_sum(acc);
+    if (lane == 0) part[it] = acc;
   }
 }
 

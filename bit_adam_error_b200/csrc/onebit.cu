@@ -188,7 +188,7 @@ ob_err check_grads(ob_ctx* c, const void* grads) {
 void enqueue_finalize_scale(ob_ctx* c, const double* part, float* out, int rows,
                             const int64_t* tpx, int mult, int64_t row_stride, cudaStream_t st) {
   launch(c, OB_K_FINALIZE_SCALE, st, [&] {
-    ob::k_finalize_scale<<<dim3(c->cfg.num_chunks, rows), ob::kFinalizeThreads, 0, st>>>(
+    ob::k_finalize_scale<true><<<dim3(c->cfg.num_chunks, rows), ob::kFinalizeThreads, 0, st>>>(
         c->L, part, tpx, mult, row_stride, out);
   });
 }
@@ -657,6 +657,35 @@ ob_err ob_set_step(ob_ctx* c, int64_t step) {
   return OB_OK;
 }
 
+ob_err ob_error_norms(ob_ctx* c, float* worker_norms, float* server_norms, void* stream) {
+  ob_err r = check_ctx(c);
+  if (r != OB_OK) return r;
+  const int64_t W = c->cfg.W, C = c->cfg.num_chunks;
+  if (!worker_norms && !server_norms) return fail(OB_EINVAL, "ob_error_norms: no output");
+  if (worker_norms && !c->err && c->cfg.n > 0) return fail(OB_EINVAL, "ob_error_norms: the ctx has no err");
+  if (server_norms && !c->srv_err && c->cfg.n > 0) return fail(OB_EINVAL, "ob_error_norms: the ctx has no srv_err");
+  DeviceGuard dg(c->device);
+  if (!dg.ok) return fail(OB_ECUDA, "cannot select device %d", c->device);
+  if (worker_norms && (r = check_dev(worker_norms, W * C, "worker_norms", c->device)) != OB_OK) return r;
+  if (server_norms && (r = check_dev(server_norms, C, "server_norms", c->device)) != OB_OK) return r;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // Reuses the partial-sum scratch of the step: call it between steps on the same stream.
+  auto norms = [&](const float* x, int rows, double* part, float* out) {
+    if (c->T > 0) {
+      auto k = ob::k_rows_sumsq;
+      const int g = grid_for(c, k, rows * c->T);
+      launch(c, OB_K_WORKER_NORM, st, [&] { k<<<g, ob::kBlock, 0, st>>>(c->L, rows, x, part); });
+    }
+    launch(c, OB_K_FINALIZE_SCALE, st, [&] {
+      ob::k_finalize_scale<false><<<dim3(unsigned(C), unsigned(rows)), ob::kFinalizeThreads, 0, st>>>(
+          c->L, part, c->L.tp, 1, c->T, out);
+    });
+  };
+  if (worker_norms) norms(c->err, int(W), c->part_w, worker_norms);
+  if (server_norms) norms(c->srv_err, 1, c->part_srv, server_norms);
+  return check_launch("ob_error_norms");
+}
+
 ob_err ob_profile_start(ob_ctx* c, int32_t capacity) {
   ob_err r = check_ctx(c);
   if (r != OB_OK) return r;
@@ -859,7 +888,7 @@ extern "C" ob_err ob_compress_noalloc(const ob_config* cfg, const void* grads, f
     else if (cl) ob::k_worker_norm<float, true><<<g1, ob::kBlock, 0, st>>>(L, int(W), gf, err, clip, part, status);
     else ob::k_worker_norm<float, false><<<g1, ob::kBlock, 0, st>>>(L, int(W), gf, err, clip, part, status);
   }
-  ob::k_finalize_scale<<<dim3(unsigned(C), unsigned(W)), ob::kFinalizeThreads, 0, st>>>(L, part, L.tp, 1, T, s_w);
+  ob::k_finalize_scale<true><<<dim3(unsigned(C), unsigned(W)), ob::kFinalizeThreads, 0, st>>>(L, part, L.tp, 1, T, s_w);
   if (T > 0) {
     const int g2 = noalloc_grid(d->num_sms, d->occ_pack[bf], T);
     const uint16_t* gh = static_cast<const uint16_t*>(grads);

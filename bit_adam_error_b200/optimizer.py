@@ -149,6 +149,15 @@ class OneBitAdam:
         """Update from bits_srv / s_srv (after compress + server_reduce)."""
         L.ob_step(self.ctx, None, self._stream())
 
+    def error_norms(self):
+        """(worker norms [W, C], server norms [C]) of the error buffers, per chunk,
+        as device tensors (monitoring; the CANN article's error-norm check)."""
+        wn = torch.empty((self.W, self.C), dtype=torch.float32, device=self.device)
+        sn = torch.empty(self.C, dtype=torch.float32, device=self.device)
+        L.ob_error_norms(self.ctx, _ptr(wn) if wn.numel() else 0, _ptr(sn) if sn.numel() else 0,
+                         self._stream())
+        return wn, sn
+
     def status(self, clear: bool = False) -> int:
         return L.ob_get_status(self.ctx, clear, self._stream())
 

@@ -160,6 +160,15 @@ ob_err ob_get_status(ob_ctx* ctx, uint32_t* flags, int32_t clear, void* stream);
 int64_t ob_get_step(const ob_ctx* ctx);
 ob_err ob_set_step(ob_ctx* ctx, int64_t step);
 
+/* Error-feedback monitoring (CANN 1-bit Adam article, sections 6.2 and 8:
+ * watch the L2 norm of the error buffers; a norm that collapses towards 0
+ * signals vanishing updates): writes ||err_w restricted to chunk k||_2 to
+ * worker_norms[w * C + k] and ||srv_err on chunk k||_2 to server_norms[k]
+ * (DEVICE float arrays; either may be NULL).  Norms are summed in double in a
+ * fixed order.  Uses the ctx scratch, so it must be ordered with the ctx's
+ * steps (same stream); it does not change any state. */
+ob_err ob_error_norms(ob_ctx* ctx, float* worker_norms, float* server_norms, void* stream);
+
 /* ---- profiling (not part of the method) ----------------------------------
  * Kernel kinds the library launches, for per-kernel timing: */
 enum {

@@ -378,3 +378,21 @@ def test_zero_one_adam_variance_refresh(opt):
             pr.step(g, warm=False)
         pr.compare(tag=f"step {t} ", bits=not refresh)
     assert pr.gpu.step_count == 7 and pr.gpu.status() == 0
+
+
+@pytest.mark.parametrize("layout", sorted(LAYOUTS))
+def test_error_norms_monitoring(layout):
+    """Per-chunk L2 norms of the worker and server error buffers after a few
+    steps equal numpy's norms of the oracle's buffers (same state)."""
+    wl = small(LAYOUTS[layout], 3)
+    pr = run_chain(wl, 3, compare_every=False)
+    wn, sn = pr.gpu.error_norms()
+    torch.cuda.synchronize()
+    off = wl.offsets
+    want_w = np.array([[np.linalg.norm(pr.ref["err"][w, off[k]:off[k + 1]].astype(np.float64))
+                        for k in range(wl.C)] for w in range(3)])
+    want_s = np.array([np.linalg.norm(pr.ref["srv_err"][off[k]:off[k + 1]].astype(np.float64))
+                       for k in range(wl.C)])
+    assert_scales("worker error norms", np_of(wn), want_w)
+    assert_scales("server error norms", np_of(sn), want_s)
+    assert np.all(np_of(wn)[:, np.diff(off) == 0] == 0)
