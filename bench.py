@@ -65,6 +65,8 @@ def parse_args():
     ap.add_argument("--phase", choices=["compressed", "refresh"], default="compressed",
                     help="time the compressed step (default) or the full-precision variance-refresh "
                          "step of 0/1 Adam")
+    ap.add_argument("--err-dtype", choices=["f32", "bf16"], default=None,
+                    help="storage of the error buffers (default: the workload's, f32)")
     ap.add_argument("--dp", action="store_true",
                     help="time the real data-parallel path (worker w = rank w, NCCL exchanges) "
                          "instead of per-GPU replicas of the single-GPU step")
@@ -81,16 +83,17 @@ def parse_args():
 # -- algorithmic traffic per element (three-pass schedule) ---------------------------
 
 def algo_bytes_per_elem(kind: str, wl) -> float:
-    """HBM bytes per element that kernel kind must move in the fused step."""
-    W, gb = wl.W, wl.grad_bytes
+    """HBM bytes per element that kernel kind must move in the fused step
+    (gb = gradient bytes, eb = error-buffer bytes: 4, or 2 when stored as bf16)."""
+    W, gb, eb = wl.W, wl.grad_bytes, wl.err_bytes
     if kind == "k_worker_norm":          # read g, err for every worker
-        return (gb + 4) * W
+        return (gb + eb) * W
     if kind == "k_worker_pack":          # read g, err, write err, signs; read srv_err
-        return (gb + 8) * W + W / 8 + 4
+        return (gb + 2 * eb) * W + W / 8 + eb
     if kind == "k_server_update":
         if wl.optimizer == "lamb":       # signs, srv_err r/w, server signs, m r/w, v, p reads
-            return W / 8 + 8 + 1 / 8 + 16
-        return W / 8 + 8 + 1 / 8 + 20    # + m, v, p reads and m, p writes
+            return W / 8 + 2 * eb + 1 / 8 + 16
+        return W / 8 + 2 * eb + 1 / 8 + 20  # + m, v, p reads and m, p writes
     if kind == "k_lamb_param":           # m, v, p reads, p write
         return 16.0
     if kind == "k_warmup":               # g (xW), m, v, p reads; m, v (+ p for Adam) writes
@@ -249,8 +252,9 @@ def oracle_rate(wl, chunks, max_elems=None, min_seconds=0.0, steps=1, phase="com
         nk = wl.sizes[k] if max_elems is None else min(max_elems, wl.sizes[k])
         g = np.stack([WL.chunk_grads(wl, 0, w, k, 0, nk) for w in range(wl.W)])
         p, v = WL.chunk_state(wl, k)
+        edt = np.uint16 if wl.err_dtype == "bf16" else np.float32
         st = {"p": p[:nk].copy(), "m": np.zeros(nk, np.float32), "v": v[:nk].copy(),
-              "err": np.zeros((wl.W, nk), np.float32), "srv_err": np.zeros(nk, np.float32)}
+              "err": np.zeros((wl.W, nk), edt), "srv_err": np.zeros(nk, edt)}
         opt = oracle.LAMB if wl.optimizer == "lamb" else oracle.ADAM
         for _ in range(steps):
             t = time.perf_counter()
@@ -295,6 +299,8 @@ def run_reference(args):
 def select_workload(args):
     import workloads as WL
     wl = WL.get_workload(args.workload)
+    if getattr(args, "err_dtype", None):
+        wl = wl.with_(err_dtype=args.err_dtype)
     if args.chunks:
         k = min(args.chunks, wl.C)
         wl = wl.with_(sizes=wl.sizes[:k], name=f"{wl.name}-first{k}",
@@ -304,7 +310,8 @@ def select_workload(args):
 
 def workload_config(wl, n_gpus):
     return {"workload": f"{wl.name}: {wl.description}", "n": wl.n, "chunks": wl.C, "W": wl.W,
-            "grad_dtype": wl.grad_dtype, "state_dtype": "f32", "optimizer": wl.optimizer,
+            "grad_dtype": wl.grad_dtype, "state_dtype": "f32", "err_dtype": wl.err_dtype,
+            "optimizer": wl.optimizer,
             "global_batch": wl.W * n_gpus, "parallelism": f"{n_gpus} replica(s) x {wl.W} virtual workers",
             "l2": f"inputs larger than L2: {step_bytes_per_elem(wl) * wl.n / 1e9:.1f} GB of traffic per step"}
 
@@ -330,7 +337,7 @@ def run_ours(args):
     # State: seeded p, v generated a chunk group at a time and uploaded once.
     opt = OneBitAdam(wl.offsets, W, grad_dtype=wl.grad_dtype, optimizer=wl.optimizer, clip=wl.clip,
                      freeze_step=0, lr=wl.lr, beta1=wl.beta1, beta2=wl.beta2, eps=wl.eps,
-                     device=device)
+                     err_dtype=wl.err_dtype, device=device)
     swl = wl.with_(freeze_step=0)
     for k0, k1 in WL.chunk_groups(wl):
         lo, hi = int(wl.offsets[k0]), int(wl.offsets[k1])
@@ -407,7 +414,7 @@ def run_ours(args):
         e1.record(stream)
         torch.cuda.synchronize()
         mon_ms = e0.elapsed_time(e1)
-        mon_bytes = 4 * n * (W + 1)
+        mon_bytes = wl.err_bytes * n * (W + 1)
         monitor = {"ms": mon_ms, "GBps": mon_bytes / (mon_ms / 1e3) / 1e9,
                    "frac": mon_bytes / (mon_ms / 1e3) / 1e9 / peak, "bytes": mon_bytes}
 

@@ -36,6 +36,7 @@ class ob_config(ctypes.Structure):
         ("eps", ctypes.c_float),
         ("clip", ctypes.c_float),
         ("freeze_step", ctypes.c_int32),
+        ("err_dtype", ctypes.c_int32),
     ]
 
 
@@ -106,11 +107,12 @@ def check(code: int, call: str) -> None:
 
 
 def make_config(n, offsets, W, grad_dtype=OB_F32, optimizer=OB_ADAM, lr=1e-4, beta1=0.9,
-                beta2=0.999, eps=1e-8, clip=0.0, freeze_step=0):
+                beta2=0.999, eps=1e-8, clip=0.0, freeze_step=0, err_dtype=OB_F32):
     """Build an ob_config; returns (config, offsets_array) -- keep both alive."""
     arr = (ctypes.c_int64 * len(offsets))(*[int(x) for x in offsets])
     cfg = ob_config(int(n), len(offsets) - 1, arr, int(W), int(grad_dtype), int(optimizer),
-                    float(lr), float(beta1), float(beta2), float(eps), float(clip), int(freeze_step))
+                    float(lr), float(beta1), float(beta2), float(eps), float(clip), int(freeze_step),
+                    int(err_dtype))
     return cfg, arr
 
 

@@ -166,6 +166,45 @@ __device__ __forceinline__ void zero8(float (&x)[8]) {
   for (int j = 0; j < 8; ++j) x[j] = 0.0f;
 }
 
+// Error buffers: float32, or bfloat16 (uint16 patterns, rounded to nearest even on
+// store, widened exactly on load).  Arithmetic is float32 either way.
+__device__ __forceinline__ uint16_t bf16_rne(float x) {
+  const uint32_t u = __float_as_uint(x);
+  if ((u & 0x7fffffffu) > 0x7f800000u) return static_cast<uint16_t>((u >> 16) | 0x0040u);  // quiet NaN
+  return static_cast<uint16_t>((u + 0x7fffu + ((u >> 16) & 1u)) >> 16);
+}
+
+__device__ __forceinline__ void ld8(const uint16_t* p, float (&x)[8]) {
+  const uint4 u = *reinterpret_cast<const uint4*>(p);
+  x[0] = __uint_as_float(u.x << 16); x[1] = __uint_as_float(u.x & 0xffff0000u);
+  x[2] = __uint_as_float(u.y << 16); x[3] = __uint_as_float(u.y & 0xffff0000u);
+  x[4] = __uint_as_float(u.z << 16); x[5] = __uint_as_float(u.z & 0xffff0000u);
+  x[6] = __uint_as_float(u.w << 16); x[7] = __uint_as_float(u.w & 0xffff0000u);
+}
+
+// Two floats -> two bfloat16 (round to nearest even) packed low|high, in one
+// conversion instruction; equal to bf16_rne for every non-NaN input (a NaN
+// stays a NaN, possibly with another payload).
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+__device__ __forceinline__ void st8(uint16_t* p, const float (&x)[8]) {
+  uint4 u;
+  u.x = pack_bf16x2(x[0], x[1]);
+  u.y = pack_bf16x2(x[2], x[3]);
+  u.z = pack_bf16x2(x[4], x[5]);
+  u.w = pack_bf16x2(x[6], x[7]);
+  *reinterpret_cast<uint4*>(p) = u;
+}
+
+__device__ __forceinline__ float ld1(const float* p) { return *p; }
+__device__ __forceinline__ float ld1(const uint16_t* p) { return __uint_as_float(static_cast<uint32_t>(*p) << 16); }
+__device__ __forceinline__ void st1(float* p, float x) { *p = x; }
+__device__ __forceinline__ void st1(uint16_t* p, float x) { *p = bf16_rne(x); }
+
 // ---- method pieces -------------------------------------------------------------
 
 // Clamp the raw gradient to [-clip, clip] when clip > 0; NaN passes through.
@@ -240,9 +279,9 @@ __device__ __forceinline__ int64_t warp_count() {
 // ---- pass 1: per-tile sum of c^2 for every worker ----------------------------------
 // part[w * T + t] = sum over tile t of (clip(g_w) + err_w)^2; a non-finite sum
 // (some c is NaN/Inf) raises the status flag.
-template <typename GT, bool CLIP>
+template <typename GT, typename ET, bool CLIP>
 __global__ void __launch_bounds__(kBlock)
-k_worker_norm(Layout L, int W, const GT* __restrict__ grads, const float* __restrict__ err,
+k_worker_norm(Layout L, int W, const GT* __restrict__ grads, const ET* __restrict__ err,
               float clip, double* __restrict__ part, uint32_t* __restrict__ status) {
   const int lane = threadIdx.x & 31;
   const int64_t items = static_cast<int64_t>(W) * L.T;
@@ -252,7 +291,7 @@ k_worker_norm(Layout L, int W, const GT* __restrict__ grads, const float* __rest
     const int64_t t = it - static_cast<int64_t>(w) * L.T;
     const Tile tl = tile_at(L, t, hint);
     const GT* g = grads + static_cast<int64_t>(w) * L.n + tl.ck0;
-    const float* e = err + static_cast<int64_t>(w) * L.n + tl.ck0;
+    const ET* e = err + static_cast<int64_t>(w) * L.n + tl.ck0;
     double acc = 0.0;
     if (tl.vec) {
       float gv[kGroups][8], ev[kGroups][8];
@@ -273,7 +312,7 @@ k_worker_norm(Layout L, int W, const GT* __restrict__ grads, const float* __rest
       for (int j = 0; j < kTileWords; ++j) {
         const int64_t i = tl.rel + j * 32 + lane;
         if (i < tl.nk) {
-          const float c = (CLIP ? clip_grad(ld1_ro(g + i), clip) : ld1_ro(g + i)) + __ldg(e + i);
+          const float c = (CLIP ? clip_grad(ld1_ro(g + i), clip) : ld1_ro(g + i)) + ld1_ro(e + i);
           acc = fma(static_cast<double>(c), static_cast<double>(c), acc);
         }
       }
@@ -349,11 +388,11 @@ k_finalize_ratio(Layout L, const double* __restrict__ partP, const double* __res
 // GP = groups of one tile whose loads are issued together: 1 keeps the kernel
 // under 80 registers (3 CTAs per SM), best when W is small and a tile carries few
 // bytes per instruction; 2 keeps more bytes in flight per warp, best for large W.
-template <typename GT, bool SERVER, bool CLIP, bool POW2, int GP>
+template <typename GT, typename ET, bool SERVER, bool CLIP, bool POW2, int GP>
 __global__ void __launch_bounds__(kBlock, GP == 1 ? 3 : 2)
-k_worker_pack(Layout L, int W, const GT* __restrict__ grads, float* __restrict__ err,
+k_worker_pack(Layout L, int W, const GT* __restrict__ grads, ET* __restrict__ err,
               const float* __restrict__ s_w, uint32_t* __restrict__ bits_w,
-              const float* __restrict__ srv_err, double* __restrict__ part_srv, float clip,
+              const ET* __restrict__ srv_err, double* __restrict__ part_srv, float clip,
               uint32_t* __restrict__ status) {
   const int lane = threadIdx.x & 31;
   const auto mean = make_mean<POW2>(W);
@@ -377,7 +416,7 @@ k_worker_pack(Layout L, int W, const GT* __restrict__ grads, float* __restrict__
         }
         for (int w = 0; w < W; ++w) {
           const GT* g = grads + static_cast<int64_t>(w) * L.n + tl.ck0;
-          float* e = err + static_cast<int64_t>(w) * L.n + tl.ck0;
+          ET* e = err + static_cast<int64_t>(w) * L.n + tl.ck0;
           const float s = __ldg(s_w + static_cast<int64_t>(w) * L.C + tl.k);
           float gv[GP][8], ev[GP][8];
 #pragma unroll
@@ -426,14 +465,14 @@ k_worker_pack(Layout L, int W, const GT* __restrict__ grads, float* __restrict__
         float acc = 0.0f;
         for (int w = 0; w < W; ++w) {
           const float s = __ldg(s_w + static_cast<int64_t>(w) * L.C + tl.k);
-          float* e = err + static_cast<int64_t>(w) * L.n + tl.ck0;
+          ET* e = err + static_cast<int64_t>(w) * L.n + tl.ck0;
           bool b = false;
           if (inb) {
             const float g = ld1_ro(grads + static_cast<int64_t>(w) * L.n + tl.ck0 + i);
-            const float c = (CLIP ? clip_grad(g, clip) : g) + e[i];
+            const float c = (CLIP ? clip_grad(g, clip) : g) + ld1(e + i);
             b = c >= 0.0f;
             const float d = signed_scale(b, s);
-            e[i] = c - d;
+            st1(e + i, c - d);
             acc = acc + d;
           }
           const uint32_t word = __ballot_sync(kFull, b);
@@ -441,7 +480,7 @@ k_worker_pack(Layout L, int W, const GT* __restrict__ grads, float* __restrict__
             bits_w[static_cast<int64_t>(w) * L.words + tl.w0 + tl.rel / 32 + j] = word;
         }
         if (SERVER && inb) {
-          const float cs = mean(acc) + __ldg(srv_err + tl.ck0 + i);
+          const float cs = mean(acc) + ld1_ro(srv_err + tl.ck0 + i);
           tsum = fma(static_cast<double>(cs), static_cast<double>(cs), tsum);
         }
       }
@@ -474,10 +513,10 @@ __device__ __forceinline__ void server_sum8(const Layout& L, int W, const uint32
 }
 
 // Server norm only (stage-wise call): part_srv[t] = sum over the tile of c_srv^2.
-template <bool POW2>
+template <typename ET, bool POW2>
 __global__ void __launch_bounds__(kBlock)
 k_server_norm(Layout L, int W, const uint32_t* __restrict__ bits_w, const float* __restrict__ s_w,
-              const float* __restrict__ srv_err, double* __restrict__ part_srv,
+              const ET* __restrict__ srv_err, double* __restrict__ part_srv,
               uint32_t* __restrict__ status) {
   const int lane = threadIdx.x & 31;
   const auto mean = make_mean<POW2>(W);
@@ -512,7 +551,7 @@ k_server_norm(Layout L, int W, const uint32_t* __restrict__ bits_w, const float*
             const uint32_t word = __ldg(bits_w + static_cast<int64_t>(w) * L.words + tl.w0 + tl.rel / 32 + j);
             acc = acc + signed_scale((word >> lane) & 1u, s);
           }
-          const float cs = mean(acc) + __ldg(srv_err + tl.ck0 + i);
+          const float cs = mean(acc) + ld1_ro(srv_err + tl.ck0 + i);
           tsum = fma(static_cast<double>(cs), static_cast<double>(cs), tsum);
         }
       }
@@ -551,10 +590,10 @@ __device__ __forceinline__ void update_elem(float d, float& m, float v, float& p
 // FROM_WORKERS: c_srv from bits_w/s_w/srv_err, quantised with s_srv, bits_srv and
 // srv_err written (the compressed allreduce's second half).  Otherwise g_hat is
 // read back from bits_srv/s_srv (the update-only stage call).
-template <Upd U, bool FROM_WORKERS, bool POW2>
+template <Upd U, bool FROM_WORKERS, bool POW2, typename ET>
 __global__ void __launch_bounds__(kBlock, kUpdateMinBlocks)
 k_server_update(Layout L, int W, const uint32_t* __restrict__ bits_w, const float* __restrict__ s_w,
-                const float* __restrict__ s_srv, float* __restrict__ srv_err,
+                const float* __restrict__ s_srv, ET* __restrict__ srv_err,
                 uint32_t* __restrict__ bits_srv, float* __restrict__ m, const float* __restrict__ v,
                 float* __restrict__ p, Hyper h, double* __restrict__ partP,
                 double* __restrict__ partU, uint32_t* __restrict__ status) {
@@ -627,10 +666,10 @@ k_server_update(Layout L, int W, const uint32_t* __restrict__ bits_w, const floa
               const uint32_t word = __ldg(bits_w + static_cast<int64_t>(w) * L.words + wi);
               acc = acc + signed_scale((word >> lane) & 1u, s);
             }
-            const float cs = mean(acc) + srv_err[gi];
+            const float cs = mean(acc) + ld1(srv_err + gi);
             b = cs >= 0.0f;
             d = signed_scale(b, s2);
-            srv_err[gi] = cs - d;
+            st1(srv_err + gi, cs - d);
           }
           const uint32_t word = __ballot_sync(kFull, b);
           if (lane == 0 && (tl.rel + j * 32) < tl.nk) bits_srv[wi] = word;
@@ -655,8 +694,9 @@ k_server_update(Layout L, int W, const uint32_t* __restrict__ bits_w, const floa
 }
 
 // ---- monitoring: per-tile sums of squares of R fp32 rows [R][n] --------------------------
+template <typename ET>
 __global__ void __launch_bounds__(kBlock)
-k_rows_sumsq(Layout L, int R, const float* __restrict__ x, double* __restrict__ part) {
+k_rows_sumsq(Layout L, int R, const ET* __restrict__ x, double* __restrict__ part) {
   const int lane = threadIdx.x & 31;
   const int64_t items = static_cast<int64_t>(R) * L.T;
   int hint = 0;
@@ -664,7 +704,7 @@ k_rows_sumsq(Layout L, int R, const float* __restrict__ x, double* __restrict__ 
     const int r = static_cast<int>(it / L.T);
     const int64_t t = it - static_cast<int64_t>(r) * L.T;
     const Tile tl = tile_at(L, t, hint);
-    const float* row = x + static_cast<int64_t>(r) * L.n + tl.ck0;
+    const ET* row = x + static_cast<int64_t>(r) * L.n + tl.ck0;
     double acc = 0.0;
     if (tl.vec) {
 #pragma unroll
@@ -681,7 +721,7 @@ k_rows_sumsq(Layout L, int R, const float* __restrict__ x, double* __restrict__ 
       for (int j = 0; j < kTileWords; ++j) {
         const int64_t i = tl.rel + j * 32 + lane;
         if (i < tl.nk) {
-          const float v = __ldg(row + i);
+          const float v = ld1_ro(row + i);
           acc = fma(static_cast<double>(v), static_cast<double>(v), acc);
         }
       }

@@ -61,6 +61,8 @@ ob_err check_config(const ob_config* c) {
   for (float x : hp)
     if (!std::isfinite(x)) return fail(OB_EINVAL, "hyper-parameters must be finite");
   if (c->freeze_step < 0) return fail(OB_EINVAL, "freeze_step = %d < 0", c->freeze_step);
+  if (c->err_dtype != OB_F32 && c->err_dtype != OB_BF16)
+    return fail(OB_EINVAL, "err_dtype = %d is neither OB_F32 nor OB_BF16", c->err_dtype);
   // Element and word indices of [W][n] rows must fit in int64 comfortably.
   if (c->n > (int64_t(1) << 50) / c->W) return fail(OB_EINVAL, "W * n too large");
   return OB_OK;
@@ -93,7 +95,8 @@ struct ob_ctx {
   int64_t words = 0, T = 0;
   int device = 0, num_sms = 0;
   int64_t step = 0;
-  float *p, *m, *v, *err, *srv_err, *s_w, *s_srv;
+  float *p, *m, *v, *s_w, *s_srv;
+  void *err, *srv_err;              // float32 or bfloat16 (cfg.err_dtype)
   uint32_t *bits_w, *bits_srv;
   // scratch (one cudaMalloc)
   void* scratch = nullptr;
@@ -201,51 +204,67 @@ bool pow2_workers(const ob_ctx* c) { return (c->cfg.W & (c->cfg.W - 1)) == 0; }
 // W = 1 bf16 3.19 vs 3.47 ms per 1.5e9 elements, W = 16 fp32 10.30 vs 10.05 ms.
 constexpr int kPackOneGroupMaxW = 2;
 
-template <typename GT, bool CLIP, bool POW2>
+template <typename GT, typename ET, bool CLIP, bool POW2>
 void enqueue_worker_t(ob_ctx* c, const GT* grads, bool with_server, cudaStream_t st) {
   const int W = c->cfg.W;
+  ET* err = static_cast<ET*>(c->err);
+  const ET* srv_err = static_cast<const ET*>(c->srv_err);
   if (c->T > 0) {
-    auto k1 = ob::k_worker_norm<GT, CLIP>;
+    auto k1 = ob::k_worker_norm<GT, ET, CLIP>;
     const int g1 = grid_for(c, k1, W * c->T);
     launch(c, OB_K_WORKER_NORM, st, [&] {
-      k1<<<g1, ob::kBlock, 0, st>>>(c->L, W, grads, c->err, c->h.clip, c->part_w, c->status);
+      k1<<<g1, ob::kBlock, 0, st>>>(c->L, W, grads, err, c->h.clip, c->part_w, c->status);
     });
   }
   enqueue_finalize_scale(c, c->part_w, c->s_w, W, c->L.tp, 1, c->T, st);
   if (c->T > 0) {
     // The stage call (no server part) never uses the mean: one instantiation each.
     const bool one = W <= kPackOneGroupMaxW;
-    auto k2 = with_server ? (one ? ob::k_worker_pack<GT, true, CLIP, POW2, 1> : ob::k_worker_pack<GT, true, CLIP, POW2, 2>)
-                          : (one ? ob::k_worker_pack<GT, false, CLIP, false, 1> : ob::k_worker_pack<GT, false, CLIP, false, 2>);
+    auto k2 = with_server ? (one ? ob::k_worker_pack<GT, ET, true, CLIP, POW2, 1> : ob::k_worker_pack<GT, ET, true, CLIP, POW2, 2>)
+                          : (one ? ob::k_worker_pack<GT, ET, false, CLIP, false, 1> : ob::k_worker_pack<GT, ET, false, CLIP, false, 2>);
     const int g2 = grid_for(c, k2, c->T);
     launch(c, OB_K_WORKER_PACK, st, [&] {
-      k2<<<g2, ob::kBlock, 0, st>>>(c->L, W, grads, c->err, c->s_w, c->bits_w, c->srv_err,
+      k2<<<g2, ob::kBlock, 0, st>>>(c->L, W, grads, err, c->s_w, c->bits_w, srv_err,
                                     c->part_srv, c->h.clip, c->status);
     });
   }
   if (with_server) enqueue_finalize_scale(c, c->part_srv, c->s_srv, 1, c->L.tp, 1, 0, st);
 }
 
+template <typename GT, typename ET>
+void enqueue_worker_e(ob_ctx* c, const GT* grads, bool with_server, cudaStream_t st) {
+  const bool clip = c->h.clip > 0.0f, p2 = pow2_workers(c);
+  if (clip && p2) enqueue_worker_t<GT, ET, true, true>(c, grads, with_server, st);
+  else if (clip) enqueue_worker_t<GT, ET, true, false>(c, grads, with_server, st);
+  else if (p2) enqueue_worker_t<GT, ET, false, true>(c, grads, with_server, st);
+  else enqueue_worker_t<GT, ET, false, false>(c, grads, with_server, st);
+}
+
 template <typename GT>
 void enqueue_worker(ob_ctx* c, const GT* grads, bool with_server, cudaStream_t st) {
-  const bool clip = c->h.clip > 0.0f, p2 = pow2_workers(c);
-  if (clip && p2) enqueue_worker_t<GT, true, true>(c, grads, with_server, st);
-  else if (clip) enqueue_worker_t<GT, true, false>(c, grads, with_server, st);
-  else if (p2) enqueue_worker_t<GT, false, true>(c, grads, with_server, st);
-  else enqueue_worker_t<GT, false, false>(c, grads, with_server, st);
+  if (c->cfg.err_dtype == OB_BF16) enqueue_worker_e<GT, uint16_t>(c, grads, with_server, st);
+  else enqueue_worker_e<GT, float>(c, grads, with_server, st);
+}
+
+template <ob::Upd U, bool FROM_WORKERS, typename ET>
+void enqueue_server_update_e(ob_ctx* c, cudaStream_t st) {
+  auto k3 = pow2_workers(c) ? ob::k_server_update<U, FROM_WORKERS, true, ET>
+                            : ob::k_server_update<U, FROM_WORKERS, false, ET>;
+  const int g3 = grid_for(c, k3, c->T);
+  ET* srv_err = static_cast<ET*>(c->srv_err);
+  launch(c, OB_K_SERVER_UPDATE, st, [&] {
+    k3<<<g3, ob::kBlock, 0, st>>>(c->L, c->cfg.W, c->bits_w, c->s_w, c->s_srv, srv_err,
+                                  c->bits_srv, c->m, c->v, c->p, c->h, c->partP, c->partU,
+                                  c->status);
+  });
 }
 
 template <ob::Upd U, bool FROM_WORKERS>
 void enqueue_server_update(ob_ctx* c, cudaStream_t st) {
   if (c->T == 0) return;
-  auto k3 = pow2_workers(c) ? ob::k_server_update<U, FROM_WORKERS, true>
-                            : ob::k_server_update<U, FROM_WORKERS, false>;
-  const int g3 = grid_for(c, k3, c->T);
-  launch(c, OB_K_SERVER_UPDATE, st, [&] {
-    k3<<<g3, ob::kBlock, 0, st>>>(c->L, c->cfg.W, c->bits_w, c->s_w, c->s_srv, c->srv_err,
-                                  c->bits_srv, c->m, c->v, c->p, c->h, c->partP, c->partU,
-                                  c->status);
-  });
+  // The update-only call never reads the server error: one instantiation.
+  if (FROM_WORKERS && c->cfg.err_dtype == OB_BF16) enqueue_server_update_e<U, FROM_WORKERS, uint16_t>(c, st);
+  else enqueue_server_update_e<U, FROM_WORKERS, float>(c, st);
 }
 
 // LAMB: trust ratio per layer from the tile partials, then the parameter step.
@@ -290,14 +309,20 @@ void enqueue_warmup(ob_ctx* c, const GT* grads, cudaStream_t st) {
   if (lamb) enqueue_lamb_param(c, st);
 }
 
+template <typename ET>
+void enqueue_server_norm(ob_ctx* c, cudaStream_t st) {
+  auto k = pow2_workers(c) ? ob::k_server_norm<ET, true> : ob::k_server_norm<ET, false>;
+  const int g = grid_for(c, k, c->T);
+  const ET* srv_err = static_cast<const ET*>(c->srv_err);
+  launch(c, OB_K_SERVER_NORM, st, [&] {
+    k<<<g, ob::kBlock, 0, st>>>(c->L, c->cfg.W, c->bits_w, c->s_w, srv_err, c->part_srv, c->status);
+  });
+}
+
 void enqueue_server_stage(ob_ctx* c, cudaStream_t st) {
   if (c->T > 0) {
-    auto k = pow2_workers(c) ? ob::k_server_norm<true> : ob::k_server_norm<false>;
-    const int g = grid_for(c, k, c->T);
-    launch(c, OB_K_SERVER_NORM, st, [&] {
-      k<<<g, ob::kBlock, 0, st>>>(c->L, c->cfg.W, c->bits_w, c->s_w, c->srv_err, c->part_srv,
-                                  c->status);
-    });
+    if (c->cfg.err_dtype == OB_BF16) enqueue_server_norm<uint16_t>(c, st);
+    else enqueue_server_norm<float>(c, st);
   }
   enqueue_finalize_scale(c, c->part_srv, c->s_srv, 1, c->L.tp, 1, 0, st);
   enqueue_server_update<ob::Upd::kNone, true>(c, st);
@@ -368,7 +393,7 @@ ob_err ob_layout(const ob_config* cfg, int64_t* words_total) {
   return OB_OK;
 }
 
-ob_err ob_create(const ob_config* cfg, float* p, float* m, float* v, float* err, float* srv_err,
+ob_err ob_create(const ob_config* cfg, float* p, float* m, float* v, void* err, void* srv_err,
                  uint32_t* bits_w, float* s_w, uint32_t* bits_srv, float* s_srv, ob_ctx** out) {
   if (!out) return fail(OB_EINVAL, "out is NULL");
   *out = nullptr;
@@ -670,11 +695,21 @@ ob_err ob_error_norms(ob_ctx* c, float* worker_norms, float* server_norms, void*
   if (server_norms && (r = check_dev(server_norms, C, "server_norms", c->device)) != OB_OK) return r;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   // Reuses the partial-sum scratch of the step: call it between steps on the same stream.
-  auto norms = [&](const float* x, int rows, double* part, float* out) {
+  auto norms = [&](const void* x, int rows, double* part, float* out) {
     if (c->T > 0) {
-      auto k = ob::k_rows_sumsq;
-      const int g = grid_for(c, k, rows * c->T);
-      launch(c, OB_K_WORKER_NORM, st, [&] { k<<<g, ob::kBlock, 0, st>>>(c->L, rows, x, part); });
+      if (c->cfg.err_dtype == OB_BF16) {
+        auto k = ob::k_rows_sumsq<uint16_t>;
+        const int g = grid_for(c, k, rows * c->T);
+        launch(c, OB_K_WORKER_NORM, st, [&] {
+          k<<<g, ob::kBlock, 0, st>>>(c->L, rows, static_cast<const uint16_t*>(x), part);
+        });
+      } else {
+        auto k = ob::k_rows_sumsq<float>;
+        const int g = grid_for(c, k, rows * c->T);
+        launch(c, OB_K_WORKER_NORM, st, [&] {
+          k<<<g, ob::kBlock, 0, st>>>(c->L, rows, static_cast<const float*>(x), part);
+        });
+      }
     }
     launch(c, OB_K_FINALIZE_SCALE, st, [&] {
       ob::k_finalize_scale<false><<<dim3(unsigned(C), unsigned(rows)), ob::kFinalizeThreads, 0, st>>>(
@@ -796,10 +831,10 @@ ob_err noalloc_setup(int device, NoAllocDevice** out) {
     if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(no-alloc scratch)");
     if ((e = cudaDeviceGetAttribute(&d.num_sms, cudaDevAttrMultiProcessorCount, device)) != cudaSuccess)
       return cuda_fail(e, "cudaDeviceGetAttribute");
-    d.occ_norm[0] = occupancy(reinterpret_cast<const void*>(ob::k_worker_norm<float, true>));
-    d.occ_norm[1] = occupancy(reinterpret_cast<const void*>(ob::k_worker_norm<uint16_t, true>));
-    d.occ_pack[0] = occupancy(reinterpret_cast<const void*>(ob::k_worker_pack<float, false, true, false, 2>));
-    d.occ_pack[1] = occupancy(reinterpret_cast<const void*>(ob::k_worker_pack<uint16_t, false, true, false, 2>));
+    d.occ_norm[0] = occupancy(reinterpret_cast<const void*>(ob::k_worker_norm<float, float, true>));
+    d.occ_norm[1] = occupancy(reinterpret_cast<const void*>(ob::k_worker_norm<uint16_t, float, true>));
+    d.occ_pack[0] = occupancy(reinterpret_cast<const void*>(ob::k_worker_pack<float, float, false, true, false, 2>));
+    d.occ_pack[1] = occupancy(reinterpret_cast<const void*>(ob::k_worker_pack<uint16_t, float, false, true, false, 2>));
     d.scratch = static_cast<char*>(ptr);
     d.ready = true;
   }
@@ -820,6 +855,8 @@ extern "C" ob_err ob_compress_noalloc(const ob_config* cfg, const void* grads, f
   ob_err r = ob_layout(cfg, &words);
   if (r != OB_OK) return r;
   const int64_t n = cfg->n, W = cfg->W, C = cfg->num_chunks;
+  if (cfg->err_dtype != OB_F32)
+    return fail(OB_EINVAL, "ob_compress_noalloc: float32 error buffers only");
   if (C > kNoAllocMaxChunks)
     return fail(OB_EINVAL, "ob_compress_noalloc: %lld chunks, at most %d", (long long)C, kNoAllocMaxChunks);
   // Scratch needed: header (tables, status) + one double per (worker, warp tile).
@@ -883,20 +920,20 @@ extern "C" ob_err ob_compress_noalloc(const ob_config* cfg, const void* grads, f
     const int g1 = noalloc_grid(d->num_sms, d->occ_norm[bf], W * T);
     const uint16_t* gh = static_cast<const uint16_t*>(grads);
     const float* gf = static_cast<const float*>(grads);
-    if (bf && cl) ob::k_worker_norm<uint16_t, true><<<g1, ob::kBlock, 0, st>>>(L, int(W), gh, err, clip, part, status);
-    else if (bf) ob::k_worker_norm<uint16_t, false><<<g1, ob::kBlock, 0, st>>>(L, int(W), gh, err, clip, part, status);
-    else if (cl) ob::k_worker_norm<float, true><<<g1, ob::kBlock, 0, st>>>(L, int(W), gf, err, clip, part, status);
-    else ob::k_worker_norm<float, false><<<g1, ob::kBlock, 0, st>>>(L, int(W), gf, err, clip, part, status);
+    if (bf && cl) ob::k_worker_norm<uint16_t, float, true><<<g1, ob::kBlock, 0, st>>>(L, int(W), gh, err, clip, part, status);
+    else if (bf) ob::k_worker_norm<uint16_t, float, false><<<g1, ob::kBlock, 0, st>>>(L, int(W), gh, err, clip, part, status);
+    else if (cl) ob::k_worker_norm<float, float, true><<<g1, ob::kBlock, 0, st>>>(L, int(W), gf, err, clip, part, status);
+    else ob::k_worker_norm<float, float, false><<<g1, ob::kBlock, 0, st>>>(L, int(W), gf, err, clip, part, status);
   }
   ob::k_finalize_scale<true><<<dim3(unsigned(C), unsigned(W)), ob::kFinalizeThreads, 0, st>>>(L, part, L.tp, 1, T, s_w);
   if (T > 0) {
     const int g2 = noalloc_grid(d->num_sms, d->occ_pack[bf], T);
     const uint16_t* gh = static_cast<const uint16_t*>(grads);
     const float* gf = static_cast<const float*>(grads);
-    if (bf && cl) ob::k_worker_pack<uint16_t, false, true, false, 2><<<g2, ob::kBlock, 0, st>>>(L, int(W), gh, err, s_w, bits_w, nullptr, nullptr, clip, status);
-    else if (bf) ob::k_worker_pack<uint16_t, false, false, false, 2><<<g2, ob::kBlock, 0, st>>>(L, int(W), gh, err, s_w, bits_w, nullptr, nullptr, clip, status);
-    else if (cl) ob::k_worker_pack<float, false, true, false, 2><<<g2, ob::kBlock, 0, st>>>(L, int(W), gf, err, s_w, bits_w, nullptr, nullptr, clip, status);
-    else ob::k_worker_pack<float, false, false, false, 2><<<g2, ob::kBlock, 0, st>>>(L, int(W), gf, err, s_w, bits_w, nullptr, nullptr, clip, status);
+    if (bf && cl) ob::k_worker_pack<uint16_t, float, false, true, false, 2><<<g2, ob::kBlock, 0, st>>>(L, int(W), gh, err, s_w, bits_w, nullptr, nullptr, clip, status);
+    else if (bf) ob::k_worker_pack<uint16_t, float, false, false, false, 2><<<g2, ob::kBlock, 0, st>>>(L, int(W), gh, err, s_w, bits_w, nullptr, nullptr, clip, status);
+    else if (cl) ob::k_worker_pack<float, float, false, true, false, 2><<<g2, ob::kBlock, 0, st>>>(L, int(W), gf, err, s_w, bits_w, nullptr, nullptr, clip, status);
+    else ob::k_worker_pack<float, float, false, false, false, 2><<<g2, ob::kBlock, 0, st>>>(L, int(W), gf, err, s_w, bits_w, nullptr, nullptr, clip, status);
   }
   return check_launch("ob_compress_noalloc");
 }

@@ -4,8 +4,9 @@ PyTorch supplies device memory and the current CUDA stream; every step of the
 method runs in ``libonebit.so``.  The optimizer keeps the whole state resident
 in HBM as flat buffers:
 
-  p, m, v, srv_err : float32 [n]
-  err              : float32 [W, n]       (one error buffer per virtual worker)
+  p, m, v          : float32 [n]
+  err              : [W, n]  (one error buffer per virtual worker; float32 or bfloat16)
+  srv_err          : [n]     (server error buffer; same type as err)
   bits_w           : uint32  [W, words]   (packed worker signs; stored as int32)
   s_w              : float32 [W, C]
   bits_srv         : uint32  [words]
@@ -36,7 +37,7 @@ class OneBitAdam:
     def __init__(self, offsets: Sequence[int], W: int, *, grad_dtype: str = "f32",
                  optimizer: str = "adam", lr: float = 1e-4, beta1: float = 0.9,
                  beta2: float = 0.999, eps: float = 1e-8, clip: float = 0.0,
-                 freeze_step: int = 0, device=None,
+                 freeze_step: int = 0, err_dtype: str = "f32", device=None,
                  p: Optional[torch.Tensor] = None, m: Optional[torch.Tensor] = None,
                  v: Optional[torch.Tensor] = None):
         self.device = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
@@ -47,9 +48,11 @@ class OneBitAdam:
         self.grad_dtype = {"f32": L.OB_F32, "bf16": L.OB_BF16}[grad_dtype]
         self.grad_torch_dtype = torch.float32 if self.grad_dtype == L.OB_F32 else torch.bfloat16
         self.optimizer = {"adam": L.OB_ADAM, "lamb": L.OB_LAMB}[optimizer]
+        self.err_dtype = {"f32": L.OB_F32, "bf16": L.OB_BF16}[err_dtype]
+        edt = torch.float32 if self.err_dtype == L.OB_F32 else torch.bfloat16
         self.cfg, self._off_keep = L.make_config(self.n, self.offsets, self.W, self.grad_dtype,
                                                  self.optimizer, lr, beta1, beta2, eps, clip,
-                                                 freeze_step)
+                                                 freeze_step, self.err_dtype)
         self.words = L.ob_layout(self.cfg)
         dev, f32 = self.device, torch.float32
 
@@ -62,8 +65,8 @@ class OneBitAdam:
         self.p = state(p, (self.n,))
         self.m = state(m, (self.n,))
         self.v = state(v, (self.n,))
-        self.err = torch.zeros((self.W, self.n), dtype=f32, device=dev)
-        self.srv_err = torch.zeros(self.n, dtype=f32, device=dev)
+        self.err = torch.zeros((self.W, self.n), dtype=edt, device=dev)
+        self.srv_err = torch.zeros(self.n, dtype=edt, device=dev)
         self.bits_w = torch.zeros((self.W, self.words), dtype=torch.int32, device=dev)
         self.s_w = torch.zeros((self.W, self.C), dtype=f32, device=dev)
         self.bits_srv = torch.zeros(self.words, dtype=torch.int32, device=dev)

@@ -81,6 +81,9 @@ typedef struct {
   float lr, beta1, beta2, eps;
   float clip;                   /* <= 0: off; else clamp the raw gradient to [-clip, clip] */
   int32_t freeze_step;          /* steps 0..freeze_step-1 are full-precision warmup */
+  int32_t err_dtype;            /* OB_F32, or OB_BF16: err and srv_err stored as bfloat16
+                                   (rounded to nearest even; arithmetic stays float32) --
+                                   half the error-buffer bytes, different rounding */
 } ob_config;
 
 /* Number of uint32 words one packed sign row holds: sum_k ceil(n_k / 32).
@@ -88,7 +91,7 @@ typedef struct {
 ob_err ob_layout(const ob_config* cfg, int64_t* words_total);
 
 /* Create a ctx over caller-owned DEVICE buffers (float32 unless stated):
- *   p, m, v, srv_err: [n];  err: [W][n] (worker-major);
+ *   p, m, v: [n];  err: [W][n] (worker-major), srv_err: [n], both of err_dtype;
  *   bits_w: uint32 [W][words_total];  s_w: [W][C];
  *   bits_srv: uint32 [words_total];  s_srv: [C].
  * Does not initialise them (the caller sets p, m, v; err and srv_err start at 0).
@@ -101,8 +104,8 @@ ob_err ob_layout(const ob_config* cfg, int64_t* words_total);
  * ctx).  Several ctxs may share a buffer if their calls are ordered.
  * Allocates the ctx scratch with cudaMalloc on the current device and
  * synchronises once.  *out receives the ctx (NULL on failure). */
-ob_err ob_create(const ob_config* cfg, float* p, float* m, float* v, float* err,
-                 float* srv_err, uint32_t* bits_w, float* s_w, uint32_t* bits_srv,
+ob_err ob_create(const ob_config* cfg, float* p, float* m, float* v, void* err,
+                 void* srv_err, uint32_t* bits_w, float* s_w, uint32_t* bits_srv,
                  float* s_srv, ob_ctx** out);
 
 /* One full-precision warmup step (step < freeze_step, else OB_EPHASE):
@@ -215,8 +218,9 @@ int64_t ob_launch_count(const ob_ctx* ctx);
  *   err_w = c - s_w sign(c)
  * with results identical to ob_compress on the same inputs.  The caller passes
  * the config and DEVICE buffers as for ob_create/ob_compress: grads [W][n]
- * (grad_dtype), err [W][n] (in/out), bits_w [W][words_total], s_w [W][C];
- * 32-byte aligned.  lr, betas, eps and freeze_step are ignored.
+ * (grad_dtype), err [W][n] (float32, in/out; err_dtype must be OB_F32),
+ * bits_w [W][words_total], s_w [W][C]; 32-byte aligned.  lr, betas, eps and
+ * freeze_step are ignored.
  *
  * Scratch: a fixed 8 MiB array in the library's device memory (every GPU that
  * loads the library holds it until the process exits), used for the chunk

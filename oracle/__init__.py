@@ -47,13 +47,13 @@ _U32 = ctypes.c_uint32
 
 _SIGS = {
     "orc_words_total": (_I64, [_I32, _P]),
-    "orc_compress": (_U32, [_I32, _I64, _I32, _P, _P, _I32, _F, _P, _P, _P]),
-    "orc_server_reduce": (_U32, [_I32, _I64, _I32, _P, _P, _P, _P, _P, _P]),
+    "orc_compress": (_U32, [_I32, _I64, _I32, _P, _P, _I32, _F, _P, _I32, _P, _P]),
+    "orc_server_reduce": (_U32, [_I32, _I64, _I32, _P, _P, _P, _P, _I32, _P, _P]),
     "orc_adam_apply": (_U32, [_I64, _I32, _P, _P, _P, _F, _F, _F, _P, _P, _P]),
     "orc_lamb_apply": (_U32, [_I64, _I32, _P, _P, _P, _F, _F, _F, _P, _P, _P, _P]),
     "orc_warmup": (_U32, [_I32, _I64, _I32, _P, _P, _I32, _I32, _F, _F, _F, _F, _P, _P, _P]),
     "orc_step": (_U32, [_I32, _I64, _I32, _P, _P, _I32, _I32, _F, _F, _F, _F,
-                        _P, _P, _P, _P, _P, _P, _P, _P, _P]),
+                        _P, _P, _P, _P, _P, _I32, _P, _P, _P, _P]),
 }
 
 
@@ -85,6 +85,14 @@ class Oracle:
         return int(self.lib.orc_words_total(len(off) - 1, self._ptr(off)))
 
     @staticmethod
+    def _err_dtype(err: np.ndarray) -> int:
+        if err.dtype == np.float32:
+            return F32
+        if err.dtype == np.uint16:
+            return BF16
+        raise TypeError("error buffers must be float32 or uint16 bfloat16 bit patterns")
+
+    @staticmethod
     def _dtype_of(grads: np.ndarray) -> int:
         if grads.dtype == np.float32:
             return F32
@@ -107,7 +115,7 @@ class Oracle:
         s_w = np.zeros((W, C), np.float32)
         flags = self.lib.orc_compress(W, n, C, self._ptr(off), self._ptr(grads),
                                       self._dtype_of(grads), float(clip), self._ptr(err),
-                                      self._ptr(bits_w), self._ptr(s_w))
+                                      self._err_dtype(err), self._ptr(bits_w), self._ptr(s_w))
         return bits_w, s_w, int(flags)
 
     def server_reduce(self, offsets, bits_w: np.ndarray, s_w: np.ndarray, srv_err: np.ndarray
@@ -122,7 +130,8 @@ class Oracle:
         s_srv = np.zeros(C, np.float32)
         flags = self.lib.orc_server_reduce(W, n, C, self._ptr(off), self._ptr(bits_w),
                                            self._ptr(s_w), self._ptr(srv_err),
-                                           self._ptr(bits_srv), self._ptr(s_srv))
+                                           self._err_dtype(srv_err), self._ptr(bits_srv),
+                                           self._ptr(s_srv))
         return bits_srv, s_srv, int(flags)
 
     def adam_apply(self, offsets, bits_srv, s_srv, m, v, p, beta1, lr, eps) -> int:
@@ -148,8 +157,9 @@ class Oracle:
                                        self._ptr(m), self._ptr(v), self._ptr(p)))
 
     def step(self, offsets, grads, state: dict, beta1, lr, eps, clip=0.0, optimizer=ADAM) -> int:
-        """One compressed step.  ``state`` holds p, m, v, err, srv_err (updated in place)
-        and receives bits_w, s_w, bits_srv, s_srv."""
+        """One compressed step.  ``state`` holds p, m, v, err, srv_err (updated in place;
+        err and srv_err float32, or both uint16 bfloat16 patterns) and receives
+        bits_w, s_w, bits_srv, s_srv."""
         off = self._off(offsets)
         W, n = grads.shape
         C = len(off) - 1
@@ -162,6 +172,7 @@ class Oracle:
             W, n, C, self._ptr(off), self._ptr(grads), self._dtype_of(grads), optimizer,
             float(clip), beta1, lr, eps, self._ptr(state["p"]), self._ptr(state["m"]),
             self._ptr(state["v"]), self._ptr(state["err"]), self._ptr(state["srv_err"]),
+            self._err_dtype(state["err"]),
             self._ptr(state["bits_w"]), self._ptr(state["s_w"]), self._ptr(state["bits_srv"]),
             self._ptr(state["s_srv"])))
 

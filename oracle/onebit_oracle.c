@@ -42,6 +42,9 @@
  *    gradient passes through unchanged.
  *  - LAMB: layer = chunk; u = m / (sqrtf(v) + eps); r = ||p|| / ||u|| with the
  *    pre-update p, and r = 1 when either norm is 0; no weight decay.
+ *  - error buffers may be stored in bfloat16 (half the bytes; the gradient-
+ *    compression survey page suggests half-precision error storage): each
+ *    stored error is the float32 result rounded to nearest-even bfloat16.
  *
  * Parity pins: every function here is checked by tests/test_oracle_pins.py
  * against hand-worked cases, closed forms, invariants and brute force.
@@ -79,6 +82,27 @@ static float grad_at(const void* grads, int32_t dtype, int64_t idx) {
     return f;
   }
   return ((const float*)grads)[idx];
+}
+
+/* Error buffers are stored as float32, or as bfloat16 (the top 16 bits of the
+ * float32, rounded to nearest with ties to even; NaN stays NaN) and widened
+ * exactly on load; all arithmetic stays float32. */
+static uint16_t to_bf16_rne(float x) {
+  uint32_t u;
+  memcpy(&u, &x, sizeof u);
+  if ((u & 0x7fffffffu) > 0x7f800000u) return (uint16_t)((u >> 16) | 0x0040u); /* quiet NaN */
+  uint32_t lsb = (u >> 16) & 1u;
+  return (uint16_t)((u + 0x7fffu + lsb) >> 16);
+}
+
+static float err_get(const void* e, int32_t dtype, int64_t i) {
+  if (dtype == ORC_BF16) return grad_at(e, ORC_BF16, i);
+  return ((const float*)e)[i];
+}
+
+static void err_set(void* e, int32_t dtype, int64_t i, float x) {
+  if (dtype == ORC_BF16) ((uint16_t*)e)[i] = to_bf16_rne(x);
+  else ((float*)e)[i] = x;
 }
 
 static float clip_grad(float g, float clip) {
@@ -132,8 +156,8 @@ int64_t orc_words_total(int32_t C, const int64_t* off) {
  * bits_w: [W][words_total] out; s_w: [W][C] out.  Returns status flags.
  */
 uint32_t orc_compress(int32_t W, int64_t n, int32_t C, const int64_t* off,
-                      const void* grads, int32_t dtype, float clip, float* err,
-                      uint32_t* bits_w, float* s_w) {
+                      const void* grads, int32_t dtype, float clip, void* err,
+                      int32_t err_dtype, uint32_t* bits_w, float* s_w) {
   uint32_t flags = 0;
   int64_t* wo = (int64_t*)malloc(sizeof(int64_t) * (size_t)(C + 1));
   word_offsets(C, off, wo);
@@ -142,16 +166,16 @@ uint32_t orc_compress(int32_t W, int64_t n, int32_t C, const int64_t* off,
     int64_t o = off[k], nk = off[k + 1] - off[k];
     float* c = (float*)malloc(sizeof(float) * (size_t)(nk > 0 ? nk : 1));
     for (int32_t w = 0; w < W; ++w) {
-      float* e = err + (int64_t)w * n + o;
+      const int64_t e0 = (int64_t)w * n + o;
       uint32_t* q = bits_w + (int64_t)w * words_total + wo[k];
       for (int64_t i = 0; i < nk; ++i) {
-        c[i] = clip_grad(grad_at(grads, dtype, (int64_t)w * n + o + i), clip) + e[i];
+        c[i] = clip_grad(grad_at(grads, dtype, e0 + i), clip) + err_get(err, err_dtype, e0 + i);
         if (is_nonfinite(c[i])) flags |= ORC_STATUS_NONFINITE;
       }
       float s = quantize_scale(c, nk);
       quantize_signs(c, nk, q);
       s_w[(int64_t)w * C + k] = s;
-      for (int64_t i = 0; i < nk; ++i) e[i] = c[i] - dequantize(q, s, i);
+      for (int64_t i = 0; i < nk; ++i) err_set(err, err_dtype, e0 + i, c[i] - dequantize(q, s, i));
     }
     free(c);
   }
@@ -169,8 +193,8 @@ uint32_t orc_compress(int32_t W, int64_t n, int32_t C, const int64_t* off,
  * bits_srv: [words_total] out; s_srv: [C] out.  Returns status flags.
  */
 uint32_t orc_server_reduce(int32_t W, int64_t n, int32_t C, const int64_t* off,
-                           const uint32_t* bits_w, const float* s_w,
-                           float* srv_err, uint32_t* bits_srv, float* s_srv) {
+                           const uint32_t* bits_w, const float* s_w, void* srv_err,
+                           int32_t err_dtype, uint32_t* bits_srv, float* s_srv) {
   (void)n;
   uint32_t flags = 0;
   int64_t* wo = (int64_t*)malloc(sizeof(int64_t) * (size_t)(C + 1));
@@ -184,14 +208,14 @@ uint32_t orc_server_reduce(int32_t W, int64_t n, int32_t C, const int64_t* off,
       for (int32_t w = 0; w < W; ++w)
         acc += dequantize(bits_w + (int64_t)w * words_total + wo[k], s_w[(int64_t)w * C + k], i);
       float avg = acc / (float)W;
-      c[i] = avg + srv_err[o + i];
+      c[i] = avg + err_get(srv_err, err_dtype, o + i);
       if (is_nonfinite(c[i])) flags |= ORC_STATUS_NONFINITE;
     }
     float s = quantize_scale(c, nk);
     uint32_t* q = bits_srv + wo[k];
     quantize_signs(c, nk, q);
     s_srv[k] = s;
-    for (int64_t i = 0; i < nk; ++i) srv_err[o + i] = c[i] - dequantize(q, s, i);
+    for (int64_t i = 0; i < nk; ++i) err_set(srv_err, err_dtype, o + i, c[i] - dequantize(q, s, i));
     free(c);
   }
   free(wo);
@@ -318,10 +342,10 @@ uint32_t orc_warmup(int32_t W, int64_t n, int32_t C, const int64_t* off,
 uint32_t orc_step(int32_t W, int64_t n, int32_t C, const int64_t* off,
                   const void* grads, int32_t dtype, int32_t optimizer, float clip,
                   float beta1, float lr, float eps, float* p, float* m, const float* v,
-                  float* err, float* srv_err, uint32_t* bits_w, float* s_w,
+                  void* err, void* srv_err, int32_t err_dtype, uint32_t* bits_w, float* s_w,
                   uint32_t* bits_srv, float* s_srv) {
-  uint32_t flags = orc_compress(W, n, C, off, grads, dtype, clip, err, bits_w, s_w);
-  flags |= orc_server_reduce(W, n, C, off, bits_w, s_w, srv_err, bits_srv, s_srv);
+  uint32_t flags = orc_compress(W, n, C, off, grads, dtype, clip, err, err_dtype, bits_w, s_w);
+  flags |= orc_server_reduce(W, n, C, off, bits_w, s_w, srv_err, err_dtype, bits_srv, s_srv);
   if (optimizer == ORC_LAMB)
     flags |= orc_lamb_apply(n, C, off, bits_srv, s_srv, beta1, lr, eps, m, v, p, NULL);
   else

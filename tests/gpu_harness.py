@@ -38,8 +38,19 @@ def to_dev(a: np.ndarray) -> torch.Tensor:
 
 
 def np_of(t: torch.Tensor) -> np.ndarray:
-    a = t.detach().cpu().contiguous().numpy()
+    """Host copy; int32 words as uint32, bfloat16 as uint16 bit patterns."""
+    t = t.detach().cpu().contiguous()
+    if t.dtype == torch.bfloat16:
+        return t.view(torch.int16).numpy().view(np.uint16)
+    a = t.numpy()
     return a.view(np.uint32) if a.dtype == np.int32 else a
+
+
+def as_f32(a: np.ndarray) -> np.ndarray:
+    """bfloat16 patterns widened to float32 (other arrays unchanged)."""
+    if a.dtype == np.uint16:
+        return (a.astype(np.uint32) << np.uint32(16)).view(np.float32)
+    return a
 
 
 def assert_bits(name, got: np.ndarray, ref: np.ndarray):
@@ -84,7 +95,7 @@ class Pair:
     """A GPU optimizer and the oracle state it is compared with."""
 
     def __init__(self, offsets: Sequence[int], W: int, *, grad_dtype="f32", optimizer="adam",
-                 clip=0.0, freeze_step=0, p0: Optional[np.ndarray] = None,
+                 clip=0.0, freeze_step=0, err_dtype="f32", p0: Optional[np.ndarray] = None,
                  v0: Optional[np.ndarray] = None, m0: Optional[np.ndarray] = None,
                  err0: Optional[np.ndarray] = None, srv0: Optional[np.ndarray] = None):
         self.off = np.asarray(offsets, np.int64)
@@ -97,11 +108,12 @@ class Pair:
         p0 = np.zeros(n, np.float32) if p0 is None else p0
         v0 = np.zeros(n, np.float32) if v0 is None else v0
         m0 = np.zeros(n, np.float32) if m0 is None else m0
-        err0 = np.zeros((W, n), np.float32) if err0 is None else err0
-        srv0 = np.zeros(n, np.float32) if srv0 is None else srv0
+        edt = np.uint16 if err_dtype == "bf16" else np.float32
+        err0 = np.zeros((W, n), edt) if err0 is None else err0
+        srv0 = np.zeros(n, edt) if srv0 is None else srv0
         self.gpu = OneBitAdam(self.off, W, grad_dtype=grad_dtype, optimizer=optimizer, clip=clip,
-                              freeze_step=freeze_step, device=dev(), p=to_dev(p0),
-                              m=to_dev(m0), v=to_dev(v0), **HP)
+                              freeze_step=freeze_step, err_dtype=err_dtype, device=dev(),
+                              p=to_dev(p0), m=to_dev(m0), v=to_dev(v0), **HP)
         if err0.any():
             self.gpu.err.copy_(to_dev(err0))
         if srv0.any():
@@ -128,7 +140,8 @@ class Pair:
         torch.cuda.synchronize()
         for k in what:
             got = np_of(getattr(self.gpu, k))
-            assert_state(f"{tag}{k}", got, self.ref[k].reshape(got.shape), self.off)
+            want = self.ref[k].reshape(got.shape)       # bfloat16 buffers compare widened
+            assert_state(f"{tag}{k}", as_f32(got), as_f32(want), self.off)
         if bits and "bits_w" in self.ref:
             assert_bits(f"{tag}bits_w", np_of(self.gpu.bits_w), self.ref["bits_w"])
             assert_bits(f"{tag}bits_srv", np_of(self.gpu.bits_srv), self.ref["bits_srv"])

@@ -204,6 +204,48 @@ def pin_empty_chunk(o):
     assert s[0, 0] == 0.0 and s[0, 2] == 0.0 and s[0, 1] > 0
 
 
+def _bf16_of(a: np.ndarray) -> np.ndarray:
+    """float32 -> bfloat16 patterns with torch's conversion (round to nearest even)."""
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(a, np.float32)).to(torch.bfloat16) \
+        .view(torch.int16).numpy().view(np.uint16)
+
+
+def _widen(b: np.ndarray) -> np.ndarray:
+    return (b.astype(np.uint32) << np.uint32(16)).view(np.float32)
+
+
+def pin_bf16_error_storage(o):
+    """Error buffers stored as bfloat16 hold the float32 results rounded to
+    nearest-even (checked against torch's conversion, on data with exact ties),
+    and the next step reads them back widened exactly."""
+    W, sizes = 2, [1 << 18, 1000, 33]
+    off = offsets_of(sizes)
+    n = int(off[-1])
+    g = aux_normal(SEED, (90,), W * n, 1e-3).reshape(W, n)
+    e32 = np.zeros((W, n), np.float32)
+    e16 = np.zeros((W, n), np.uint16)
+    b32, s32, _ = o.compress(off, g, e32)
+    b16, s16, _ = o.compress(off, g, e16)
+    assert np.array_equal(b32, b16) and np.array_equal(s32, s16)
+    ties = (e32.view(np.uint32) & np.uint32(0xFFFF)) == np.uint32(0x8000)
+    assert ties.sum() >= 1, "no exact bfloat16 ties in the data"
+    assert np.array_equal(e16, _bf16_of(e32))
+    # step 2 from the stored bfloat16 errors == float32 mode fed their widened values
+    g2 = aux_normal(SEED, (91,), W * n, 1e-3).reshape(W, n)
+    e32b = _widen(e16)
+    o.compress(off, g2, e32b)
+    o.compress(off, g2, e16)
+    assert np.array_equal(e16, _bf16_of(e32b))
+    # server error buffer, from a state both modes can hold
+    srv16 = _bf16_of(aux_normal(SEED, (92,), n, 1e-3))
+    srv32 = _widen(srv16)
+    bs32, ss32, _ = o.server_reduce(off, b32, s32, srv32)
+    bs16, ss16, _ = o.server_reduce(off, b32, s32, srv16)
+    assert np.array_equal(bs32, bs16) and np.array_equal(ss32, ss16)
+    assert np.array_equal(srv16, _bf16_of(srv32))
+
+
 # -- server stage ----------------------------------------------------------------
 
 def pin_server_single_worker(o):

@@ -17,16 +17,20 @@ from oracle_pins import ALL_PINS
 SRC = os.path.join(os.path.dirname(oracle.__file__), "onebit_oracle.c")
 
 MUTANTS = {
-    "error_sign": ("e[i] = c[i] - dequantize(q, s, i)", "e[i] = c[i] + dequantize(q, s, i)"),
-    "error_not_added": ("clip) + e[i];", "clip) + 0.0f;"),
+    "error_sign": ("err_set(err, err_dtype, e0 + i, c[i] - dequantize(q, s, i))",
+                   "err_set(err, err_dtype, e0 + i, c[i] + dequantize(q, s, i))"),
+    "error_not_added": ("clip) + err_get(err, err_dtype, e0 + i);", "clip) + 0.0f;"),
     "sign_of_zero": ("if (c[i] >= 0.0f) words", "if (c[i] > 0.0f) words"),
     "bit_order": ("words[i / 32] |= 1u << (i % 32)", "words[i / 32] |= 1u << (31 - i % 32)"),
     "scale_no_sqrt": ("return (float)(sqrt(S) / sqrt((double)n));", "return (float)(S / (double)n);"),
     "scale_no_mean": ("return (float)(sqrt(S) / sqrt((double)n));", "return (float)sqrt(S);"),
     "server_sum_not_mean": ("float avg = acc / (float)W;", "float avg = acc;"),
-    "server_error_dropped": ("c[i] = avg + srv_err[o + i];", "c[i] = avg;"),
-    "server_error_sign": ("srv_err[o + i] = c[i] - dequantize(q, s, i)",
-                          "srv_err[o + i] = dequantize(q, s, i) - c[i]"),
+    "server_error_dropped": ("c[i] = avg + err_get(srv_err, err_dtype, o + i);", "c[i] = avg;"),
+    "server_error_sign": ("err_set(srv_err, err_dtype, o + i, c[i] - dequantize(q, s, i))",
+                          "err_set(srv_err, err_dtype, o + i, dequantize(q, s, i) - c[i])"),
+    "bf16_store_truncates": ("return (uint16_t)((u + 0x7fffu + lsb) >> 16);", "return (uint16_t)(u >> 16);"),
+    "bf16_store_ties_up": ("return (uint16_t)((u + 0x7fffu + lsb) >> 16);",
+                           "return (uint16_t)((u + 0x8000u) >> 16);"),
     "server_first_worker_only": ("for (int32_t w = 0; w < W; ++w)\n        acc +=",
                                  "for (int32_t w = 0; w < 1; ++w)\n        acc +="),
     "momentum_coeff": ("float mi = beta1 * m[o + i] + one_minus_b1 * g_hat;",

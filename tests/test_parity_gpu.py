@@ -122,8 +122,9 @@ def test_update_stage(layout, opt):
 
 # -- whole steps -------------------------------------------------------------------------
 
-def run_chain(wl, steps, compare_every=True, **pair_kw):
+def run_chain(wl, steps, compare_every=True, err_dtype="f32", **pair_kw):
     p, v = state_for(wl)
+    pair_kw["err_dtype"] = err_dtype
     pr = Pair(wl.offsets, wl.W, grad_dtype=wl.grad_dtype, optimizer=wl.optimizer, clip=wl.clip,
               freeze_step=wl.freeze_step, p0=p, v0=v, **pair_kw)
     for t in range(steps):
@@ -148,6 +149,44 @@ def test_fused_steps_ragged(layout, W, gdt, opt, clip):
     wl = small(LAYOUTS[layout], W, grad_dtype=gdt, optimizer=opt, clip=clip,
                grad_dist="student_t_zeros" if clip else "normal", zero_frac=0.05 if clip else 0.0)
     run_chain(wl, 4)
+
+
+@pytest.mark.parametrize("layout", sorted(LAYOUTS))
+@pytest.mark.parametrize("W,gdt,opt,clip", [(1, "bf16", "adam", 0.0), (4, "f32", "lamb", 0.0),
+                                            (16, "f32", "adam", 5.0), (3, "f32", "adam", 0.0)])
+def test_fused_steps_bf16_error_buffers(layout, W, gdt, opt, clip):
+    """Error buffers stored as bfloat16 (rounded to nearest even): every step
+    equals the oracle run with the same storage."""
+    wl = small(LAYOUTS[layout], W, grad_dtype=gdt, optimizer=opt, clip=clip,
+               grad_dist="student_t_zeros" if clip else "normal", zero_frac=0.05 if clip else 0.0)
+    pr = run_chain(wl, 4, err_dtype="bf16")
+    assert pr.gpu.err.dtype == torch.bfloat16
+
+
+def test_stages_bf16_error_buffers():
+    """Worker and server stages alone with bfloat16 error buffers."""
+    wl = small(RAGGED, 3)
+    p, v, m, err0, srv = aux_state(wl.n, 41, 3)
+    from oracle_pins import _bf16_of
+    err0, srv = _bf16_of(err0).reshape(3, -1), _bf16_of(srv)
+    pr = Pair(wl.offsets, 3, err_dtype="bf16", p0=p, v0=v, m0=m, err0=err0, srv0=srv)
+    g = grads_for(wl, 0)
+    pr.gpu.compress(to_dev(g))
+    pr.gpu.server_reduce()
+    e, sv = err0.copy(), srv.copy()
+    o = oracle.get()
+    bits_w, s_w, _ = o.compress(wl.offsets, g, e)
+    bits_srv, s_srv, _ = o.server_reduce(wl.offsets, bits_w, s_w, sv)
+    torch.cuda.synchronize()
+    assert_bits("bits_w", np_of(pr.gpu.bits_w), bits_w)
+    assert_bits("bits_srv", np_of(pr.gpu.bits_srv), bits_srv)
+    assert np.array_equal(np_of(pr.gpu.err), e) and np.array_equal(np_of(pr.gpu.srv_err), sv)
+    wn, sn = pr.gpu.error_norms()
+    torch.cuda.synchronize()
+    widen = lambda a: (a.astype(np.uint32) << np.uint32(16)).view(np.float32).astype(np.float64)  # noqa: E731
+    off = wl.offsets
+    want = np.array([np.linalg.norm(widen(sv[off[k]:off[k + 1]])) for k in range(wl.C)])
+    assert_scales("server error norms", np_of(sn), want)
 
 
 @pytest.mark.parametrize("opt", ["adam", "lamb"])

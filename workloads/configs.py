@@ -86,6 +86,7 @@ class Workload:
     sizes: Tuple[int, ...]
     W: int
     grad_dtype: str = "f32"          # "f32" | "bf16"
+    err_dtype: str = "f32"           # storage of the error buffers: "f32" | "bf16"
     optimizer: str = "adam"          # "adam" | "lamb"
     grad_dist: str = "normal"
     grad_scale: float = 1e-3
@@ -121,6 +122,10 @@ class Workload:
     @property
     def grad_bytes(self) -> int:
         return 2 if self.grad_dtype == "bf16" else 4
+
+    @property
+    def err_bytes(self) -> int:
+        return 2 if self.err_dtype == "bf16" else 4
 
     def with_(self, **kw) -> "Workload":
         d = {k: getattr(self, k) for k in self.__dataclass_fields__ if k != "_cache"}
