@@ -50,7 +50,7 @@ constexpr int kTile = kGroupElems * kGroups;     // 512 elements per warp tile
 constexpr int kTileWords = kTile / 32;
 constexpr int kBlock = 256;                      // threads per CTA (8 warps)
 constexpr int kWarpsPerBlock = kBlock / kWarp;
-constexpr int kFinalizeThreads = 256;
+constexpr int kFinalizeThreads = 1024;
 constexpr bool kWide = true;                     // 256-bit (v8.f32) global accesses for fp32 arrays
 constexpr int kUpdateMinBlocks = 2;              // pass 3: resident CTAs per SM asked of ptxas
 constexpr unsigned kFull = 0xffffffffu;
