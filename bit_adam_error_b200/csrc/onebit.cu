@@ -2,8 +2,12 @@
 //
 // Validates arguments, owns the per-ctx scratch (chunk tables, per-tile partial
 // norms, LAMB ratios, status word) and enqueues the kernels of kernels.cuh on the
-// caller's stream.  No call allocates or synchronises after ob_create, except
-// ob_get_status (one 4-byte read-back).
+// caller's stream.  After ob_create no call allocates device memory; the step
+// calls only enqueue work.  ob_get_status synchronises the stream (one 4-byte
+// read-back); ob_step_host creates its copy stream and events on first use;
+// ob_profile_start/stop create, wait for and destroy CUDA events; ob_destroy
+// waits for the copy stream.  ob_compress_noalloc (end of file) uses a fixed
+// static scratch array instead of a ctx.
 #include <algorithm>
 #include <cmath>
 #include <cstdarg>

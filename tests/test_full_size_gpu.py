@@ -71,3 +71,39 @@ def test_full_size_sampled_chunks(name):
         assert_scales(tag + "s_w", np_of(opt.s_w[:, k]), ref["s_w"][:, 0])
         assert_scales(tag + "s_srv", np_of(opt.s_srv[k:k + 1]), ref["s_srv"])
     opt.close()
+
+
+def test_row_longer_than_two_to_the_31():
+    """Maximum-size indexing: one worker row of 2^31 + 2^20 elements (bf16
+    gradients; about 48 GB resident), so element, word and tile indices pass
+    2^31.  The first chunk and the chunks past 2^31 are compared with the oracle."""
+    n = (1 << 31) + (1 << 20)
+    wl = WL.get_workload("gpt2xl-flat").with_(name="row-2^31", sizes=tuple(WL.configs.flat_slices(n, 1 << 26)))
+    torch.cuda.empty_cache()
+    opt = OneBitAdam(wl.offsets, 1, grad_dtype="bf16", device=dev(), **HP)
+    upload_state(wl, opt.p, opt.v)
+    G = torch.empty((1, n), dtype=torch.bfloat16, device=dev())
+    upload_grads(wl, 0, G)
+    opt.step(G)
+    torch.cuda.synchronize()
+    assert opt.status() == 0
+    del G
+    o = oracle.get()
+    wb = np.zeros(wl.C + 1, np.int64)
+    np.cumsum([(s + 31) // 32 for s in wl.sizes], out=wb[1:])
+    for k in (0, wl.C - 2, wl.C - 1):
+        nk = wl.sizes[k]
+        lo, hi = int(wl.offsets[k]), int(wl.offsets[k + 1])
+        off = np.array([0, nk], np.int64)
+        pk, vk = WL.chunk_state(wl, k)
+        ref = {"p": pk, "m": np.zeros(nk, np.float32), "v": vk, "err": np.zeros((1, nk), np.float32),
+               "srv_err": np.zeros(nk, np.float32)}
+        o.step(off, WL.chunk_grads(wl, 0, 0, k)[None, :], ref, F["beta1"], F["lr"], F["eps"])
+        tag = f"chunk {k} [{lo}, {hi}): "
+        for key in ("p", "m", "srv_err"):
+            assert_state(tag + key, np_of(getattr(opt, key)[lo:hi]), ref[key], off)
+        assert_state(tag + "err", np_of(opt.err[:, lo:hi]), ref["err"], off)
+        assert_bits(tag + "bits_srv", np_of(opt.bits_srv[wb[k]:wb[k + 1]]), ref["bits_srv"])
+        assert_scales(tag + "s_srv", np_of(opt.s_srv[k:k + 1]), ref["s_srv"])
+    assert wl.offsets[wl.C - 1] > (1 << 31)
+    opt.close()
