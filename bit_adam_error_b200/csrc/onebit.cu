@@ -38,8 +38,10 @@ ob_err cuda_fail(cudaError_t e, const char* what) {
   return fail(OB_ECUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
 }
 
-// 32 bytes: the kernels move 8 fp32 elements per lane in one 256-bit access.
-bool aligned32(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 31u) == 0; }
+// Element arrays need 32 bytes: the kernels move 8 fp32 elements per lane in one
+// 256-bit access.  Packed words and scales are read and written one 4-byte word
+// at a time, so 4 bytes suffice (slices of them can start on any word).
+constexpr uintptr_t kAlignElems = 32, kAlignWords = 4;
 
 int64_t words_of(int64_t n) { return (n + 31) / 32; }
 
@@ -72,12 +74,14 @@ ob_err check_config(const ob_config* c) {
   return OB_OK;
 }
 
-// A device buffer argument: NULL only when it holds no element; 32-byte
-// aligned; device (or managed) memory of the current device.
-ob_err check_dev(const void* p, int64_t count, const char* name, int device) {
+// A device buffer argument: NULL only when it holds no element; aligned to
+// `align` bytes; device (or managed) memory of the current device.
+ob_err check_dev(const void* p, int64_t count, const char* name, int device,
+                 uintptr_t align = kAlignElems) {
   if (count == 0) return OB_OK;
   if (!p) return fail(OB_EINVAL, "%s is NULL", name);
-  if (!aligned32(p)) return fail(OB_EINVAL, "%s is not 32-byte aligned", name);
+  if (reinterpret_cast<uintptr_t>(p) % align != 0)
+    return fail(OB_EINVAL, "%s is not %d-byte aligned", name, int(align));
   cudaPointerAttributes a;
   cudaError_t e = cudaPointerGetAttributes(&a, p);
   if (e != cudaSuccess) {
@@ -409,12 +413,13 @@ ob_err ob_create(const ob_config* cfg, float* p, float* m, float* v, void* err, 
   int device = 0;
   cudaError_t e = cudaGetDevice(&device);
   if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
-  struct { const void* p; int64_t count; const char* name; } bufs[] = {
-      {p, n, "p"}, {m, n, "m"}, {v, n, "v"}, {err, W * n, "err"}, {srv_err, n, "srv_err"},
-      {bits_w, W * words, "bits_w"}, {s_w, W * C, "s_w"}, {bits_srv, words, "bits_srv"},
-      {s_srv, C, "s_srv"}};
+  struct { const void* p; int64_t count; const char* name; uintptr_t align; } bufs[] = {
+      {p, n, "p", kAlignElems}, {m, n, "m", kAlignElems}, {v, n, "v", kAlignElems},
+      {err, W * n, "err", kAlignElems}, {srv_err, n, "srv_err", kAlignElems},
+      {bits_w, W * words, "bits_w", kAlignWords}, {s_w, W * C, "s_w", kAlignWords},
+      {bits_srv, words, "bits_srv", kAlignWords}, {s_srv, C, "s_srv", kAlignWords}};
   for (auto& b : bufs)  // NULL: the ctx is created without that buffer (see require_buffers)
-    if (b.p && (r = check_dev(b.p, b.count, b.name, device)) != OB_OK) return r;
+    if (b.p && (r = check_dev(b.p, b.count, b.name, device, b.align)) != OB_OK) return r;
 
   ob_ctx* c = new (std::nothrow) ob_ctx();
   if (!c) return fail(OB_ENOMEM, "ctx allocation failed");
@@ -695,8 +700,10 @@ ob_err ob_error_norms(ob_ctx* c, float* worker_norms, float* server_norms, void*
   if (server_norms && !c->srv_err && c->cfg.n > 0) return fail(OB_EINVAL, "ob_error_norms: the ctx has no srv_err");
   DeviceGuard dg(c->device);
   if (!dg.ok) return fail(OB_ECUDA, "cannot select device %d", c->device);
-  if (worker_norms && (r = check_dev(worker_norms, W * C, "worker_norms", c->device)) != OB_OK) return r;
-  if (server_norms && (r = check_dev(server_norms, C, "server_norms", c->device)) != OB_OK) return r;
+  if (worker_norms && (r = check_dev(worker_norms, W * C, "worker_norms", c->device, kAlignWords)) != OB_OK)
+    return r;
+  if (server_norms && (r = check_dev(server_norms, C, "server_norms", c->device, kAlignWords)) != OB_OK)
+    return r;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   // Reuses the partial-sum scratch of the step: call it between steps on the same stream.
   auto norms = [&](const void* x, int rows, double* part, float* out) {
@@ -877,10 +884,11 @@ extern "C" ob_err ob_compress_noalloc(const ob_config* cfg, const void* grads, f
   int device = 0;
   cudaError_t e = cudaGetDevice(&device);
   if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
-  struct { const void* p; int64_t count; const char* name; } bufs[] = {
-      {grads, W * n, "grads"}, {err, W * n, "err"}, {bits_w, W * words, "bits_w"}, {s_w, W * C, "s_w"}};
+  struct { const void* p; int64_t count; const char* name; uintptr_t align; } bufs[] = {
+      {grads, W * n, "grads", kAlignElems}, {err, W * n, "err", kAlignElems},
+      {bits_w, W * words, "bits_w", kAlignWords}, {s_w, W * C, "s_w", kAlignWords}};
   for (auto& b : bufs)
-    if ((r = check_dev(b.p, b.count, b.name, device)) != OB_OK) return r;
+    if ((r = check_dev(b.p, b.count, b.name, device, b.align)) != OB_OK) return r;
 
   std::lock_guard<std::mutex> lock(g_noalloc_mu);
   NoAllocDevice* d = nullptr;

@@ -33,8 +33,10 @@
  *   - Device buffers are caller-owned and must stay valid for the ctx's life.
  *     The ctx stores their pointers and owns only its own scratch (per-tile
  *     partial norms, chunk tables, status word), allocated in ob_create.
- *   - Every device pointer must be 32-byte aligned (cudaMalloc and the PyTorch
- *     caching allocator give 256 or more); otherwise OB_EINVAL.
+ *   - Element arrays (gradients, p, m, v, err, srv_err, staging) must be 32-byte
+ *     aligned (cudaMalloc and the PyTorch caching allocator give 256 or more);
+ *     packed words and scales (bits_w, bits_srv, s_w, s_srv, norm outputs) 4-byte
+ *     aligned; otherwise OB_EINVAL.
  *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
  *     Calls only enqueue work on it and return; none synchronises except
  *     ob_get_status and ob_create.
