@@ -25,6 +25,12 @@ The arithmetic runs in the CUDA library (``CudaStages``); this module only
 plans the layout and moves packed words between ranks (NCCL on GPUs; gloo
 stages CUDA tensors through host memory).  The stage backend is an object with
 a fixed interface, so the exchange logic can also be exercised on CPU ranks.
+
+Compression overlapped with transfer (the CANN 1-bit Adam article, section
+4.2): with one worker ctx per owner slice, each slice is compressed just
+before its exchange round is posted, and updated as soon as its owner's server
+words arrive.  On NCCL the transfers run on the communicator's own stream, so
+they overlap the kernels of the next slice.
 """
 
 from __future__ import annotations
@@ -122,7 +128,7 @@ class CudaStages:
     def __init__(self, layout: DPLayout, rank: int, *, grad_dtype: str = "f32",
                  optimizer: str = "adam", lr: float = 1e-4, beta1: float = 0.9,
                  beta2: float = 0.999, eps: float = 1e-8, clip: float = 0.0,
-                 warmup: bool = True, device=None):
+                 warmup: bool = True, pipelined: bool = True, device=None):
         from . import _lib as L
         self.L = L
         self.device = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
@@ -166,6 +172,23 @@ class CudaStages:
             if warmup:
                 self.warm = L.ob_create(cfg(layout.offsets, W, 1 << 30), ptr(self.p), ptr(self.m),
                                         ptr(self.v), 0, 0, 0, 0, 0, 0)
+            # One worker+update ctx per owner slice (views into the same buffers), so a
+            # slice can be compressed and sent while the next one is compressed.  Element
+            # arrays of a slice must start 32-byte aligned (16 bf16 elements).
+            self.slice_ctx: Optional[List[int]] = None
+            if pipelined and W > 1 and all(layout.eslice(o).start % 16 == 0 for o in range(W)):
+                self.slice_ctx = []
+                for o in range(W):
+                    ks, es, ws = layout.kslice(o), layout.eslice(o), layout.wslice(o)
+                    if ks.stop == ks.start:
+                        self.slice_ctx.append(0)
+                        continue
+                    so = layout.offsets[ks.start: ks.stop + 1] - es.start
+                    e4, w4, k4 = 4 * es.start, 4 * ws.start, 4 * ks.start
+                    self.slice_ctx.append(L.ob_create(
+                        cfg(so, 1, 0), ptr(self.p) + e4, ptr(self.m) + e4, ptr(self.v) + e4,
+                        ptr(self.err) + e4, 0, ptr(self.bits_w) + w4, ptr(self.s_w) + k4,
+                        ptr(self.bits_srv) + w4, ptr(self.s_srv) + k4))
 
     def _stream(self) -> int:
         return int(torch.cuda.current_stream(self.device).cuda_stream)
@@ -175,6 +198,18 @@ class CudaStages:
 
     def compress(self, grad: torch.Tensor) -> None:
         self.L.ob_compress(self.local, int(grad.data_ptr()), self._stream())
+
+    @property
+    def pipelined(self) -> bool:
+        return self.slice_ctx is not None
+
+    def compress_slice(self, o: int, grad_slice: torch.Tensor) -> None:
+        if self.slice_ctx[o]:
+            self.L.ob_compress(self.slice_ctx[o], int(grad_slice.data_ptr()), self._stream())
+
+    def apply_slice(self, o: int) -> None:
+        if self.slice_ctx[o]:
+            self.L.ob_step(self.slice_ctx[o], None, self._stream())
 
     def server_reduce(self) -> None:
         if self.server:
@@ -190,6 +225,9 @@ class CudaStages:
             f |= self.L.ob_get_status(self.server, False, st)
         if self.warm:
             f |= self.L.ob_get_status(self.warm, False, st)
+        for h in self.slice_ctx or []:
+            if h:
+                f |= self.L.ob_get_status(h, False, st)
         return f
 
     def close(self) -> None:
@@ -198,9 +236,27 @@ class CudaStages:
             if h:
                 self.L.ob_destroy(h)
                 setattr(self, name, 0)
+        for h in self.slice_ctx or []:
+            if h:
+                self.L.ob_destroy(h)
+        self.slice_ctx = None
 
 
 # ---- the data-parallel optimizer -------------------------------------------------------
+
+class _Pending:
+    """Posted point-to-point works plus the host-staged receives to copy back."""
+
+    def __init__(self, works, copy_back):
+        self.works, self.copy_back = works, copy_back
+
+    def wait(self) -> None:
+        for w in self.works:
+            w.wait()
+        for t, dst in self.copy_back:
+            t.copy_(dst)
+        self.works, self.copy_back = [], []
+
 
 class DistributedOneBitAdam:
     """One rank of data-parallel 1-bit Adam (worker w = rank w).
@@ -222,7 +278,11 @@ class DistributedOneBitAdam:
         self._stage_on_host = dist.get_backend(group) == "gloo"
 
     # -- point-to-point with optional host staging (gloo has no CUDA transport) --
-    def _p2p(self, sends: List[Tuple[torch.Tensor, int]], recvs: List[Tuple[torch.Tensor, int]]) -> None:
+    def _p2p(self, sends: List[Tuple[torch.Tensor, int]], recvs: List[Tuple[torch.Tensor, int]],
+             wait: bool = True) -> "_Pending":
+        """Post one grouped batch of sends and receives.  With ``wait=False`` the
+        caller waits on the returned handle later (on NCCL that makes the current
+        stream wait for the transfer, so kernels enqueued meanwhile overlap it)."""
         host = self._stage_on_host
         ops, copy_back = [], []
         for t, peer in sends:
@@ -235,11 +295,10 @@ class DistributedOneBitAdam:
                 ops.append(dist.P2POp(dist.irecv, dst, peer, self.group))
                 if dst is not t:
                     copy_back.append((t, dst))
-        if ops:
-            for req in dist.batch_isend_irecv(ops):
-                req.wait()
-        for t, dst in copy_back:
-            t.copy_(dst)
+        pending = _Pending(dist.batch_isend_irecv(ops) if ops else [], copy_back)
+        if wait:
+            pending.wait()
+        return pending
 
     def _to_owners(self) -> None:
         """Exchange 1: this rank's words/scales of owner o's chunks -> rank o."""
@@ -269,6 +328,41 @@ class DistributedOneBitAdam:
                 recvs += [(s.bits_srv[wsl], o), (s.s_srv[ksl], o)]
         self._p2p(sends, recvs)
 
+    def _compressed_step_pipelined(self, grad: torch.Tensor) -> None:
+        """Exchange 1 and 2 as W-1 shifted rounds.  In round i this rank sends to
+        rank r+i and receives from rank r-i, so every round pairs the ranks
+        consistently whatever their number.  Exchange 1: slice r+i is compressed
+        just before its round is posted, so its transfer overlaps the
+        compression of the next slice; the server stage waits for all rounds.
+        Exchange 2: all rounds are posted at once, then slice r-i is updated as
+        soon as round i has arrived."""
+        L, s, r, W = self.layout, self.stages, self.rank, self.world
+        pending = []
+        for i in range(1, W):
+            to, frm = (r + i) % W, (r - i) % W
+            s.compress_slice(to, grad[L.eslice(to)])
+            pending.append(self._p2p(
+                [(s.bits_w[0, L.wslice(to)], to), (s.s_w[0, L.kslice(to)], to)],
+                [(s.bits_w_srv[frm], frm), (s.s_w_srv[frm], frm)], wait=False))
+        s.compress_slice(r, grad[L.eslice(r)])
+        s.bits_w_srv[r].copy_(s.bits_w[0, L.wslice(r)])
+        s.s_w_srv[r].copy_(s.s_w[0, L.kslice(r)])
+        for pend in pending:
+            pend.wait()
+        s.server_reduce()
+        pending = []
+        for i in range(1, W):
+            to, frm = (r + i) % W, (r - i) % W
+            pending.append(self._p2p(
+                [(s.bits_srv_own, to), (s.s_srv_own, to)],
+                [(s.bits_srv[L.wslice(frm)], frm), (s.s_srv[L.kslice(frm)], frm)], wait=False))
+        s.bits_srv[L.wslice(r)].copy_(s.bits_srv_own)
+        s.s_srv[L.kslice(r)].copy_(s.s_srv_own)
+        s.apply_slice(r)
+        for i, pend in enumerate(pending, 1):
+            pend.wait()
+            s.apply_slice((r - i) % W)
+
     def _gather_grads(self, grad: torch.Tensor) -> torch.Tensor:
         """All ranks' full-precision gradients, rank-major [world, n] (warmup)."""
         if self._stage_on_host and grad.is_cuda:
@@ -288,6 +382,8 @@ class DistributedOneBitAdam:
             raise ValueError(f"gradient must hold {self.layout.n} elements (layout order)")
         if self.in_warmup:
             self.stages.warmup(self._gather_grads(grad.reshape(-1)))
+        elif getattr(self.stages, "pipelined", False):
+            self._compressed_step_pipelined(grad.reshape(-1))
         else:
             self.stages.compress(grad)
             self._to_owners()

@@ -23,7 +23,10 @@ HP = dict(lr=1e-4, beta1=0.9, beta2=0.999, eps=1e-8)
 
 
 class OracleStages:
-    def __init__(self, layout, rank, optimizer="adam", clip=0.0):
+    """``pipelined``: also offer the per-owner-slice stages (compress_slice,
+    apply_slice), so the driver takes its overlapped schedule."""
+
+    def __init__(self, layout, rank, optimizer="adam", clip=0.0, pipelined=False):
         import oracle
         self.o = oracle.get()
         self.layout, self.rank = layout, rank
@@ -45,6 +48,7 @@ class OracleStages:
         self.bits_srv_own = torch.zeros(wsl.stop - wsl.start, dtype=i32)
         self.s_srv_own = torch.zeros(ks.stop - ks.start, dtype=f32)
         self.flags = 0
+        self.pipelined = bool(pipelined) and layout.world > 1
 
     @staticmethod
     def _u32(t):
@@ -56,14 +60,33 @@ class OracleStages:
                                     self.m.numpy(), self.v.numpy(), self.p.numpy(), f["beta1"],
                                     f["beta2"], f["lr"], f["eps"], optimizer=self.opt)
 
-    def compress(self, grad):
+    @staticmethod
+    def _grad_rows(grad):
         if grad.dtype == torch.bfloat16:
-            g = np.ascontiguousarray(grad.view(torch.int16).numpy().view(np.uint16).reshape(1, -1))
-        else:
-            g = np.ascontiguousarray(grad.numpy().reshape(1, -1))
-        bits, s, fl = self.o.compress(self.layout.offsets, g, self.err.numpy(), clip=self.clip)
+            return np.ascontiguousarray(grad.view(torch.int16).numpy().view(np.uint16).reshape(1, -1))
+        return np.ascontiguousarray(grad.numpy().reshape(1, -1))
+
+    def compress(self, grad):
+        bits, s, fl = self.o.compress(self.layout.offsets, self._grad_rows(grad), self.err.numpy(),
+                                      clip=self.clip)
         self._u32(self.bits_w)[:] = bits
         self.s_w.numpy()[:] = s
+        self.flags |= fl
+
+    def _slice_offsets(self, o):
+        ks, es = self.layout.kslice(o), self.layout.eslice(o)
+        return self.layout.offsets[ks.start: ks.stop + 1] - es.start
+
+    def compress_slice(self, o, grad_slice):
+        L = self.layout
+        ks, es, wsl = L.kslice(o), L.eslice(o), L.wslice(o)
+        if ks.stop == ks.start:
+            return
+        err = self.err.numpy()[0, es].reshape(1, -1)
+        bits, s, fl = self.o.compress(self._slice_offsets(o), self._grad_rows(grad_slice), err,
+                                      clip=self.clip)
+        self._u32(self.bits_w)[0, wsl] = bits[0]
+        self.s_w.numpy()[0, ks] = s[0]
         self.flags |= fl
 
     def server_reduce(self):
@@ -79,6 +102,19 @@ class OracleStages:
         f = {k: np.float32(v) for k, v in HP.items()}
         args = (self.layout.offsets, self._u32(self.bits_srv), self.s_srv.numpy(), self.m.numpy(),
                 self.v.numpy(), self.p.numpy(), f["beta1"], f["lr"], f["eps"])
+        if self.opt:
+            self.flags |= self.o.lamb_apply(*args)[1]
+        else:
+            self.flags |= self.o.adam_apply(*args)
+
+    def apply_slice(self, o):
+        L = self.layout
+        ks, es, wsl = L.kslice(o), L.eslice(o), L.wslice(o)
+        if ks.stop == ks.start:
+            return
+        f = {k: np.float32(v) for k, v in HP.items()}
+        args = (self._slice_offsets(o), self._u32(self.bits_srv)[wsl], self.s_srv.numpy()[ks],
+                self.m.numpy()[es], self.v.numpy()[es], self.p.numpy()[es], f["beta1"], f["lr"], f["eps"])
         if self.opt:
             self.flags |= self.o.lamb_apply(*args)[1]
         else:
@@ -111,7 +147,8 @@ def initial_state(wl, layout):
     return layout.to_layout(ps).astype(np.float32), layout.to_layout(vs).astype(np.float32)
 
 
-def _rank_main(rank, world, port, sizes, wl_kw, steps, backend, device, q, die=None, timeout_s=120):
+def _rank_main(rank, world, port, sizes, wl_kw, steps, backend, device, q, die=None, timeout_s=120,
+               pipelined=False):
     try:
         import sys
         sys.path.insert(0, ROOT)
@@ -127,11 +164,12 @@ def _rank_main(rank, world, port, sizes, wl_kw, steps, backend, device, q, die=N
         wl = workload(sizes, world, **wl_kw)
         layout = plan(sizes, world)
         if device == "cpu":
-            stages = OracleStages(layout, rank, optimizer=wl.optimizer, clip=wl.clip)
+            stages = OracleStages(layout, rank, optimizer=wl.optimizer, clip=wl.clip, pipelined=pipelined)
         else:
             from bit_adam_error_b200.distributed import CudaStages
             stages = CudaStages(layout, rank, grad_dtype=wl.grad_dtype, optimizer=wl.optimizer,
-                                clip=wl.clip, warmup=wl.freeze_step > 0, device=device, **HP)
+                                clip=wl.clip, warmup=wl.freeze_step > 0, pipelined=pipelined,
+                                device=device, **HP)
         p0, v0 = initial_state(wl, layout)
         stages.p.copy_(torch.from_numpy(p0))
         stages.v.copy_(torch.from_numpy(v0))
@@ -144,6 +182,7 @@ def _rank_main(rank, world, port, sizes, wl_kw, steps, backend, device, q, die=N
                 else torch.from_numpy(g)
             drv.step(gt.to(stages.device))
         flags = drv.status()
+        schedule = "pipelined" if getattr(stages, "pipelined", False) else "grouped"
         if device != "cpu":
             torch.cuda.synchronize()
 
@@ -153,6 +192,7 @@ def _rank_main(rank, world, port, sizes, wl_kw, steps, backend, device, q, die=N
 
         out = {k: host(getattr(stages, k)) for k in ("p", "m", "v", "err", "srv_err", "bits_srv", "s_srv")}
         out["flags"] = flags
+        out["schedule"] = schedule
         if hasattr(stages, "close"):
             stages.close()
         dist.destroy_process_group()
@@ -161,14 +201,14 @@ def _rank_main(rank, world, port, sizes, wl_kw, steps, backend, device, q, die=N
         q.put((rank, {"error": traceback.format_exc()}))
 
 
-def run_ranks(sizes, world, wl_kw, steps, backend="gloo", device="cpu", timeout=600):
+def run_ranks(sizes, world, wl_kw, steps, backend="gloo", device="cpu", timeout=600, pipelined=False):
     """Spawn `world` ranks; returns the list of per-rank final states."""
     import multiprocessing as mp
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = free_port()
-    procs = [ctx.Process(target=_rank_main, args=(r, world, port, sizes, wl_kw, steps, backend, device, q))
-             for r in range(world)]
+    procs = [ctx.Process(target=_rank_main, args=(r, world, port, sizes, wl_kw, steps, backend, device, q),
+                         kwargs=dict(pipelined=pipelined)) for r in range(world)]
     for pr in procs:
         pr.start()
     results = {}

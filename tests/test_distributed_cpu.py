@@ -32,17 +32,29 @@ def test_plan_balances_and_groups_by_owner():
     assert sum(many.kslice(r).stop - many.kslice(r).start for r in range(4)) == 2
 
 
+@pytest.mark.parametrize("pipelined", [False, True], ids=["grouped", "pipelined"])
 @pytest.mark.parametrize("world,wl_kw,steps", [
     (2, dict(), 4),
     (3, dict(freeze_step=2), 4),
     (2, dict(optimizer="lamb", freeze_step=1), 3),
     (3, dict(grad_dtype="bf16", clip=5.0, grad_dist="student_t_zeros", zero_frac=0.05), 3),
 ])
-def test_ranks_match_single_process_oracle(world, wl_kw, steps):
-    outs = run_ranks(SIZES, world, wl_kw, steps)
+def test_ranks_match_single_process_oracle(world, wl_kw, steps, pipelined):
+    outs = run_ranks(SIZES, world, wl_kw, steps, pipelined=pipelined)
     wl, ref = reference(SIZES, world, wl_kw, steps)
     compare(plan(SIZES, world), wl, ref, outs)
     assert all(o["flags"] == 0 for o in outs)
+    assert all(o["schedule"] == ("pipelined" if pipelined else "grouped") for o in outs)
+
+
+@pytest.mark.parametrize("world", [4, 5])
+def test_pipelined_rounds_pair_every_rank(world):
+    """Shifted rounds with 4 and 5 ranks (the pairing differs from world 2/3;
+    with 5 ranks over 10 chunks some ranks own one chunk, one owns the empty one)."""
+    outs = run_ranks(SIZES, world, dict(freeze_step=1), 3, pipelined=True)
+    wl, ref = reference(SIZES, world, dict(freeze_step=1), 3)
+    compare(plan(SIZES, world), wl, ref, outs)
+    assert all(o["schedule"] == "pipelined" for o in outs)
 
 
 def test_a_dead_rank_ends_the_others_step_with_an_error():

@@ -17,14 +17,20 @@ pytestmark = pytest.mark.gpu
 SIZES = [4096, 1000, 640, 33, 20480, 7, 512, 96, 0, 3000]
 
 
-@pytest.mark.parametrize("world,backend,wl_kw,steps", [
-    (1, "nccl", dict(freeze_step=1), 3),
-    (2, "gloo", dict(), 4),
-    (2, "gloo", dict(freeze_step=2, optimizer="lamb"), 4),
-    (2, "gloo", dict(grad_dtype="bf16", clip=5.0, grad_dist="student_t_zeros", zero_frac=0.05), 3),
+@pytest.mark.parametrize("world,backend,wl_kw,steps,pipelined", [
+    (1, "nccl", dict(freeze_step=1), 3, True),
+    (2, "gloo", dict(), 4, False),
+    (2, "gloo", dict(), 4, True),
+    (2, "gloo", dict(freeze_step=2, optimizer="lamb"), 4, True),
+    (2, "gloo", dict(grad_dtype="bf16", clip=5.0, grad_dist="student_t_zeros", zero_frac=0.05), 3, False),
+    (3, "gloo", dict(grad_dtype="bf16", clip=5.0, grad_dist="student_t_zeros", zero_frac=0.05), 3, True),
 ])
-def test_gpu_ranks_match_oracle(world, backend, wl_kw, steps):
-    outs = run_ranks(SIZES, world, wl_kw, steps, backend=backend, device="cuda:0")
+def test_gpu_ranks_match_oracle(world, backend, wl_kw, steps, pipelined):
+    """Owner slices of SIZES start on 16-element boundaries for 2 and 3 ranks, so
+    the per-slice ctxs (pipelined schedule) are taken there."""
+    outs = run_ranks(SIZES, world, wl_kw, steps, backend=backend, device="cuda:0", pipelined=pipelined)
     wl, ref = reference(SIZES, world, wl_kw, steps)
     compare(plan(SIZES, world), wl, ref, outs, exact=False)
     assert all(o["flags"] == 0 for o in outs)
+    want = "pipelined" if pipelined and world > 1 else "grouped"
+    assert all(o["schedule"] == want for o in outs)
