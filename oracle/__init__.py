@@ -54,7 +54,15 @@ _SIGS = {
     "orc_warmup": (_U32, [_I32, _I64, _I32, _P, _P, _I32, _I32, _F, _F, _F, _F, _P, _P, _P]),
     "orc_step": (_U32, [_I32, _I64, _I32, _P, _P, _I32, _I32, _F, _F, _F, _F,
                         _P, _P, _P, _P, _P, _I32, _P, _P, _P, _P]),
+    "orc_code_words_total": (_I64, [_I32, _P]),
+    "orc_ternary_compress": (_U32, [_I32, _I64, _I32, _P, _P, _I32, _F, _F, _P, _I32, _P]),
+    "orc_ternary_server": (_U32, [_I32, _I32, _P, _P, _P]),
+    "orc_ternary_apply": (_U32, [_I64, _I32, _P, _I32, _P, _I32, _F, _F, _F, _P, _P, _P, _P]),
+    "orc_ternary_step": (_U32, [_I32, _I64, _I32, _P, _P, _I32, _I32, _F, _F, _F, _F,
+                                _P, _P, _P, _P, _I32, _P, _P]),
 }
+
+MAX_TERNARY_WORKERS = 127   # the int8 sum of W codes in {-1, 0, 1} is exact up to here
 
 
 class Oracle:
@@ -175,6 +183,63 @@ class Oracle:
             self._err_dtype(state["err"]),
             self._ptr(state["bits_w"]), self._ptr(state["s_w"]), self._ptr(state["bits_srv"]),
             self._ptr(state["s_srv"])))
+
+    # -- the momentum-error rule (int8 ternary codes) --------------------------------
+    def code_words_total(self, offsets) -> int:
+        off = self._off(offsets)
+        return int(self.lib.orc_code_words_total(len(off) - 1, self._ptr(off)))
+
+    def ternary_compress(self, offsets, grads: np.ndarray, err: np.ndarray, beta1, clip: float = 0.0
+                         ) -> Tuple[np.ndarray, int]:
+        """Worker stage.  ``grads``/``err``: [W, n]; ``err`` updated in place.
+
+        Returns (codes_w int8 [W, 4 * code_words], flags).
+        """
+        off = self._off(offsets)
+        W, n = grads.shape
+        codes = np.zeros((W, 4 * self.code_words_total(off)), np.int8)
+        flags = self.lib.orc_ternary_compress(W, n, len(off) - 1, self._ptr(off), self._ptr(grads),
+                                              self._dtype_of(grads), float(clip), beta1,
+                                              self._ptr(err), self._err_dtype(err), self._ptr(codes))
+        return codes, int(flags)
+
+    def ternary_server(self, offsets, codes_w: np.ndarray) -> np.ndarray:
+        """Per-element sum of the W workers' codes (int8, W <= 127)."""
+        off = self._off(offsets)
+        W = codes_w.shape[0]
+        if W > MAX_TERNARY_WORKERS:
+            raise ValueError(f"W = {W} > {MAX_TERNARY_WORKERS}: the int8 code sum could overflow")
+        out = np.zeros(4 * self.code_words_total(off), np.int8)
+        self.lib.orc_ternary_server(W, len(off) - 1, self._ptr(off),
+                                    self._ptr(np.ascontiguousarray(codes_w, np.int8)), self._ptr(out))
+        return out
+
+    def ternary_apply(self, offsets, W, codes_srv, m, v, p, beta1, lr, eps, optimizer=ADAM
+                      ) -> Tuple[np.ndarray, int]:
+        off = self._off(offsets)
+        r = np.zeros(len(off) - 1, np.float32)
+        flags = self.lib.orc_ternary_apply(int(off[-1]), len(off) - 1, self._ptr(off), int(W),
+                                           self._ptr(np.ascontiguousarray(codes_srv, np.int8)),
+                                           optimizer, beta1, lr, eps, self._ptr(m), self._ptr(v),
+                                           self._ptr(p), self._ptr(r))
+        return r, int(flags)
+
+    def ternary_step(self, offsets, grads, state: dict, beta1, lr, eps, clip=0.0, optimizer=ADAM) -> int:
+        """One compressed step of the momentum-error rule.  ``state`` holds p, m, v,
+        err (updated in place) and receives codes_w and codes_srv."""
+        off = self._off(offsets)
+        W, n = grads.shape
+        if W > MAX_TERNARY_WORKERS:
+            raise ValueError(f"W = {W} > {MAX_TERNARY_WORKERS}: the int8 code sum could overflow")
+        nb = 4 * self.code_words_total(off)
+        for key, shape in (("codes_w", (W, nb)), ("codes_srv", (nb,))):
+            if key not in state or state[key].shape != shape:
+                state[key] = np.zeros(shape, np.int8)
+        return int(self.lib.orc_ternary_step(
+            W, n, len(off) - 1, self._ptr(off), self._ptr(grads), self._dtype_of(grads), optimizer,
+            float(clip), beta1, lr, eps, self._ptr(state["p"]), self._ptr(state["m"]),
+            self._ptr(state["v"]), self._ptr(state["err"]), self._err_dtype(state["err"]),
+            self._ptr(state["codes_w"]), self._ptr(state["codes_srv"])))
 
 
 _default: Optional[Oracle] = None

@@ -352,3 +352,153 @@ uint32_t orc_step(int32_t W, int64_t n, int32_t C, const int64_t* off,
     flags |= orc_adam_apply(n, C, off, bits_srv, s_srv, beta1, lr, eps, m, v, p);
   return flags;
 }
+
+/* ---- the momentum-error rule ------------------------------------------------------
+ *
+ * The CANN 1-bit Adam article, section 2.1 "量化与误差补偿机制" (sign quantisation,
+ * error, momentum-form error compensation), section 2.2 "动量修正策略" (m follows
+ * the compressed gradient) and section 3.2 (clip before quantisation, NaN check
+ * after the error update, int8 storage of the compressed gradient).  Per worker
+ * w and element, with eps_w the worker's error buffer:
+ *   c      = clip(g_w) + eps_w
+ *   q      = sign(c)                        in {-1, 0, +1}, no scale
+ *   Delta  = c - q
+ *   eps_w  = beta1 eps_w + (1 - beta1) Delta
+ * The article's snippet is one worker.  Readings for W workers and the rest:
+ *  - q travels as an int8 code; the W codes of an element are combined by
+ *    their sum (exact in int8 for W <= 127), and the direction is their mean
+ *    g_hat = (float)sum / (float)W (the compressed allreduce of the DeepSpeed
+ *    page, section "机制", averaging the workers' messages);
+ *  - m = beta1 m + (1 - beta1) g_hat and the parameter step are the ones of
+ *    orc_adam_apply / orc_lamb_apply, v frozen;
+ *  - sign(+0) = sign(-0) = 0, and a NaN c gives code 0 (its error is NaN);
+ *  - the check after the error update flags any non-finite error (NaN or
+ *    +-inf), and a non-finite parameter as elsewhere;
+ *  - codes of chunk k occupy bytes [4 cw_k, 4 cw_k + n_k) of a row, where
+ *    every chunk starts on a fresh 32-bit word and takes ceil(n_k / 4) words;
+ *    padding bytes are 0.
+ */
+
+static int64_t code_words_of(int64_t n) { return (n + 3) / 4; }
+
+static void code_word_offsets(int32_t C, const int64_t* off, int64_t* cw) {
+  cw[0] = 0;
+  for (int32_t k = 0; k < C; ++k) cw[k + 1] = cw[k] + code_words_of(off[k + 1] - off[k]);
+}
+
+int64_t orc_code_words_total(int32_t C, const int64_t* off) {
+  int64_t t = 0;
+  for (int32_t k = 0; k < C; ++k) t += code_words_of(off[k + 1] - off[k]);
+  return t;
+}
+
+/* sign() with sign(0) = 0; NaN compares false both ways and gives 0. */
+static int8_t ternary_sign(float c) {
+  if (c > 0.0f) return 1;
+  if (c < 0.0f) return -1;
+  return 0;
+}
+
+/*
+ * Worker stage of the momentum-error rule.  grads: [W][n]; err: [W][n] in/out;
+ * codes_w: [W][4 * code_words_total] int8 out.  Returns status flags.
+ */
+uint32_t orc_ternary_compress(int32_t W, int64_t n, int32_t C, const int64_t* off,
+                              const void* grads, int32_t dtype, float clip, float beta1,
+                              void* err, int32_t err_dtype, int8_t* codes_w) {
+  uint32_t flags = 0;
+  const float one_minus_b1 = 1.0f - beta1;
+  int64_t* cw = (int64_t*)malloc(sizeof(int64_t) * (size_t)(C + 1));
+  code_word_offsets(C, off, cw);
+  const int64_t row_bytes = 4 * cw[C];
+  for (int32_t w = 0; w < W; ++w) {
+    int8_t* row = codes_w + (int64_t)w * row_bytes;
+    memset(row, 0, (size_t)row_bytes);
+    for (int32_t k = 0; k < C; ++k) {
+      int64_t o = off[k], nk = off[k + 1] - off[k];
+      for (int64_t i = 0; i < nk; ++i) {
+        const int64_t e = (int64_t)w * n + o + i;
+        float eps_old = err_get(err, err_dtype, e);
+        float c = clip_grad(grad_at(grads, dtype, e), clip) + eps_old;
+        int8_t q = ternary_sign(c);
+        float delta = c - (float)q;
+        float eps_new = beta1 * eps_old + one_minus_b1 * delta;
+        if (is_nonfinite(eps_new)) flags |= ORC_STATUS_NONFINITE;
+        err_set(err, err_dtype, e, eps_new);
+        row[4 * cw[k] + i] = q;
+      }
+    }
+  }
+  free(cw);
+  return flags;
+}
+
+/*
+ * Server stage of the momentum-error rule: codes_srv = sum over w = 0..W-1 of
+ * codes_w, per element (the caller keeps W <= 127).  codes_w: [W][row bytes];
+ * codes_srv: [row bytes] out, padding bytes 0.
+ */
+uint32_t orc_ternary_server(int32_t W, int32_t C, const int64_t* off, const int8_t* codes_w,
+                            int8_t* codes_srv) {
+  int64_t* cw = (int64_t*)malloc(sizeof(int64_t) * (size_t)(C + 1));
+  code_word_offsets(C, off, cw);
+  const int64_t row_bytes = 4 * cw[C];
+  memset(codes_srv, 0, (size_t)row_bytes);
+  for (int32_t k = 0; k < C; ++k) {
+    int64_t nk = off[k + 1] - off[k];
+    for (int64_t i = 0; i < nk; ++i) {
+      const int64_t b = 4 * cw[k] + i;
+      int sum = 0;
+      for (int32_t w = 0; w < W; ++w) sum += codes_w[(int64_t)w * row_bytes + b];
+      codes_srv[b] = (int8_t)sum;
+    }
+  }
+  free(cw);
+  return 0u;
+}
+
+/*
+ * Update of the momentum-error rule: g_hat = (float)codes_srv / (float)W, then
+ * m and p as orc_adam_apply (optimizer ORC_ADAM) or orc_lamb_apply (ORC_LAMB;
+ * r_out, may be NULL, receives the [C] trust ratios).
+ */
+uint32_t orc_ternary_apply(int64_t n, int32_t C, const int64_t* off, int32_t W,
+                           const int8_t* codes_srv, int32_t optimizer, float beta1, float lr,
+                           float eps, float* m, const float* v, float* p, float* r_out) {
+  (void)n;
+  uint32_t flags = 0;
+  int64_t* cw = (int64_t*)malloc(sizeof(int64_t) * (size_t)(C + 1));
+  code_word_offsets(C, off, cw);
+  const float one_minus_b1 = 1.0f - beta1;
+  for (int32_t k = 0; k < C; ++k) {
+    int64_t o = off[k], nk = off[k + 1] - off[k];
+    for (int64_t i = 0; i < nk; ++i) {
+      float g_hat = (float)codes_srv[4 * cw[k] + i] / (float)W;
+      float mi = beta1 * m[o + i] + one_minus_b1 * g_hat;
+      m[o + i] = mi;
+      if (optimizer == ORC_ADAM) {
+        float pi = p[o + i] - lr * mi / (sqrtf(v[o + i]) + eps);
+        if (is_nonfinite(pi)) flags |= ORC_STATUS_NONFINITE;
+        p[o + i] = pi;
+      }
+    }
+    if (optimizer == ORC_LAMB) {
+      if (r_out) r_out[k] = trust_ratio(p + o, m + o, v + o, eps, nk);
+      flags |= lamb_update_layer(p + o, m + o, v + o, lr, eps, nk);
+    }
+  }
+  free(cw);
+  return flags;
+}
+
+/* One whole compressed-phase step of the momentum-error rule. */
+uint32_t orc_ternary_step(int32_t W, int64_t n, int32_t C, const int64_t* off,
+                          const void* grads, int32_t dtype, int32_t optimizer, float clip,
+                          float beta1, float lr, float eps, float* p, float* m, const float* v,
+                          void* err, int32_t err_dtype, int8_t* codes_w, int8_t* codes_srv) {
+  uint32_t flags = orc_ternary_compress(W, n, C, off, grads, dtype, clip, beta1, err, err_dtype,
+                                        codes_w);
+  flags |= orc_ternary_server(W, C, off, codes_w, codes_srv);
+  flags |= orc_ternary_apply(n, C, off, W, codes_srv, optimizer, beta1, lr, eps, m, v, p, NULL);
+  return flags;
+}

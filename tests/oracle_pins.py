@@ -501,4 +501,257 @@ def pin_step_composition(o):
         assert np.array_equal(a["bits_w"], bw) and np.array_equal(a["bits_srv"], bs)
 
 
+
+
+# -- the momentum-error rule (int8 ternary codes) ---------------------------------------
+
+def _f32(x) -> np.float32:
+    return np.float32(float(x))
+
+
+def code_base(sizes):
+    """First 4-byte word of every chunk's codes (ceil(n_k / 4) words per chunk)."""
+    cb = [0]
+    for s in sizes:
+        cb.append(cb[-1] + (s + 3) // 4)
+    return cb
+
+
+def pin_ternary_hand_cases(o):
+    doc = json.load(open(os.path.join(GOLDEN, "ternary_hand_cases.json")))
+    for case in doc["cases"]:
+        sizes = case["sizes"]
+        g = np.array([[_f32(x) for x in case["g"]]], np.float32)
+        err = np.array([[_f32(x) for x in case["err0"]]], np.float32)
+        codes, flags = o.ternary_compress(offsets_of(sizes), g, err, _f32(case["beta1"]))
+        want = np.array([int(b, 16) for b in case["codes_bytes"]], np.uint8).view(np.int8)
+        assert np.array_equal(codes[0], want), (case["name"], codes[0])
+        want_err = [float(Fraction(str(x))) for x in case["err1"]]
+        assert [float(x) for x in err[0]] == want_err, (case["name"], err[0])
+        assert flags == 0
+    srv = doc["server"]
+    cw = np.array(srv["codes"], np.int8)
+    out = o.ternary_server([0, cw.shape[1]], cw)
+    assert [int(x) for x in out] == srv["sum"], out
+
+
+def _ternary_inputs(W, sizes, key, gscale=0.3, escale=0.1):
+    n = int(sum(sizes))
+    g = aux_normal(SEED, (70, *key), W * n, gscale).reshape(W, n)
+    err = aux_normal(SEED, (71, *key), W * n, escale).reshape(W, n)
+    return g, err
+
+
+def _codes_of(codes_row, sizes):
+    """Unpack one row of chunk-laid codes to one value per element."""
+    cb = code_base(sizes)
+    return np.concatenate([codes_row[4 * cb[k]: 4 * cb[k] + nk] for k, nk in enumerate(sizes)]) \
+        if sizes else np.zeros(0, np.int8)
+
+
+def pin_ternary_codes_are_signs(o):
+    """Every code is numpy's sign of the compensated value g + eps (float32 sum),
+    and every padding byte is 0."""
+    sizes = RAGGED
+    off, cb = offsets_of(sizes), code_base(sizes)
+    for W in (1, 3):
+        g, err = _ternary_inputs(W, sizes, (W,))
+        c = g + err
+        codes, flags = o.ternary_compress(off, g, err, B1)
+        assert flags == 0
+        for w in range(W):
+            assert np.array_equal(_codes_of(codes[w], sizes), np.sign(c[w]).astype(np.int8)), W
+            pad = np.ones(codes.shape[1], bool)
+            for k, nk in enumerate(sizes):
+                pad[4 * cb[k]: 4 * cb[k] + nk] = False
+            assert not codes[w][pad].any()
+
+
+def pin_ternary_error_telescopes(o):
+    """eps <- beta1 eps + (1 - beta1)(c - q) with c = g + eps is
+    eps <- eps + (1 - beta1)(g - q), since beta1 + (1 - beta1) = 1 exactly for the
+    float32 constants; so over T steps eps_T - eps_0 = (1 - beta1) sum_t (g_t - q_t),
+    up to the roundings of each step."""
+    sizes, T, W = [40, 33, 64], 40, 2
+    off = offsets_of(sizes)
+    n = int(off[-1])
+    omb1 = float(np.float32(1) - B1)
+    _, err = _ternary_inputs(W, sizes, (80,))
+    err0 = err.astype(np.float64)
+    acc = np.zeros((W, n))
+    tol = np.zeros((W, n))
+    for t in range(T):
+        g = aux_normal(SEED, (81, t), W * n, 0.3).reshape(W, n)
+        before = err.astype(np.float64)
+        codes, _ = o.ternary_compress(off, g, err, B1)
+        q = np.stack([_codes_of(codes[w], sizes) for w in range(W)]).astype(np.float64)
+        acc += g.astype(np.float64) - q
+        mag = np.abs(g) + np.abs(before) + np.abs(q) + np.abs(err)
+        tol += 4 * ulp32(mag)
+    diff = np.abs((err.astype(np.float64) - err0) - omb1 * acc)
+    assert np.all(diff <= tol), float(np.max(diff - tol))
+
+
+def pin_ternary_beta1_limits(o):
+    """beta1 = 1 keeps the error buffer bit for bit; beta1 = 0 leaves the plain
+    quantisation residual c - q."""
+    sizes = [40, 33]
+    off = offsets_of(sizes)
+    g, err = _ternary_inputs(2, sizes, (90,))
+    keep = err.copy()
+    o.ternary_compress(off, g, err, np.float32(1.0))
+    assert np.array_equal(err.view(np.uint32), keep.view(np.uint32))
+    c = g + keep
+    o.ternary_compress(off, g, err, np.float32(0.0))
+    assert np.array_equal(err, c - np.sign(c))
+
+
+def pin_ternary_server_bruteforce(o):
+    """The server sum equals an integer brute-force sum of the unpacked codes, for
+    W up to 127 (all +1 and all -1 reach the int8 limits); padding stays 0."""
+    sizes = RAGGED
+    off, cb = offsets_of(sizes), code_base(sizes)
+    nb = 4 * cb[-1]
+    for W in (1, 2, 5, 127):
+        u = aux_uniform(SEED, (100, W), W * int(off[-1]), 0.0, 3.0).reshape(W, -1)
+        vals = np.floor(u).astype(np.int64) - 1
+        vals = np.clip(vals, -1, 1)
+        if W == 127:
+            vals[:, :5] = 1
+            vals[:, 5:10] = -1
+        codes = np.zeros((W, nb), np.int8)
+        for w in range(W):
+            for k, nk in enumerate(sizes):
+                codes[w, 4 * cb[k]: 4 * cb[k] + nk] = vals[w, off[k]: off[k + 1]]
+        out = o.ternary_server(off, codes)
+        want = [sum(int(vals[w, i]) for w in range(W)) for i in range(int(off[-1]))]
+        assert [int(x) for x in _codes_of(out, sizes)] == want, W
+        pad = np.ones(nb, bool)
+        for k, nk in enumerate(sizes):
+            pad[4 * cb[k]: 4 * cb[k] + nk] = False
+        assert not out[pad].any()
+    try:
+        o.ternary_server(off, np.zeros((128, nb), np.int8))
+    except ValueError:
+        pass
+    else:
+        raise AssertionError("W = 128 accepted: the int8 code sum could overflow")
+
+
+def pin_ternary_adam_closed_form(o):
+    """Constant code sums per chunk with W = 4 give g_hat in {1, -1/2, 0, 3/4}
+    exactly; then m_t = (1 - b1^t) g_hat and p follows the closed form of
+    pin_adam_closed_form; v untouched."""
+    sizes, T, W = [8, 12, 5, 9], 20, 4
+    off, cb = offsets_of(sizes), code_base(sizes)
+    n = int(off[-1])
+    sums = [4, -2, 0, 3]
+    codes = np.zeros(4 * cb[-1], np.int8)
+    gh = np.zeros(n)
+    for k, nk in enumerate(sizes):
+        codes[4 * cb[k]: 4 * cb[k] + nk] = sums[k]
+        gh[off[k]: off[k + 1]] = sums[k] / W
+    m = np.zeros(n, np.float32)
+    v = aux_uniform(SEED, (110,), n, 1e-4, 1e-2)
+    v0 = v.copy()
+    p0 = aux_normal(SEED, (111,), n, 0.02)
+    p = p0.copy()
+    for _ in range(T):
+        _, flags = o.ternary_apply(off, W, codes, m, v, p, B1, LR, EPS)
+        assert flags == 0
+    b1 = float(B1)
+    assert np.allclose(m, (1 - b1 ** T) * gh, rtol=2e-6, atol=0)
+    sum_m = T - b1 * (1 - b1 ** T) / (1 - b1)
+    want_p = p0 - float(LR) * gh * sum_m / (np.sqrt(v0.astype(np.float64)) + float(EPS))
+    assert np.max(np.abs(p - want_p)) <= 2e-7, np.max(np.abs(p - want_p))
+    assert np.array_equal(v, v0)
+
+
+def pin_ternary_lamb_proportional(o):
+    """LAMB with the momentum-error rule: a layer whose u = m/(sqrt v + eps) is
+    proportional to p (constant g_hat, v and p of one sign) moves to (1 - lr) p;
+    a layer with all codes 0 has u = 0, r = 1 and keeps p."""
+    sizes, W = [16, 12], 2
+    off, cb = offsets_of(sizes), code_base(sizes)
+    n = int(off[-1])
+    codes = np.zeros(4 * cb[-1], np.int8)
+    codes[: sizes[0]] = 2                   # g_hat = 1 on layer 0, 0 on layer 1
+    m = np.zeros(n, np.float32)
+    v = np.full(n, 0.25, np.float32)
+    p = np.concatenate([np.full(sizes[0], 0.3), aux_normal(SEED, (120,), sizes[1], 0.02)]).astype(np.float32)
+    p0 = p.copy()
+    lr = np.float32(0.01)
+    r, flags = o.ternary_apply(off, W, codes, m, v, p, B1, lr, EPS, optimizer=1)
+    assert flags == 0
+    assert np.allclose(p[: sizes[0]], (1 - float(lr)) * 0.3, rtol=1e-6)
+    assert np.array_equal(p[sizes[0]:], p0[sizes[0]:]) and float(r[1]) == 1.0
+    u0 = float(np.float32(1) - B1) / (0.5 + float(EPS))
+    assert abs(float(r[0]) - 0.3 / u0) <= 1e-6 * 0.3 / u0
+
+
+def pin_ternary_step_composition(o):
+    """The whole step equals worker stage -> server sum -> update, Adam and LAMB."""
+    sizes, W = [40, 33, 64, 0, 7], 3
+    off = offsets_of(sizes)
+    n = int(off[-1])
+    for opt in (0, 1):
+        g, err = _ternary_inputs(W, sizes, (130, opt))
+        st = {"p": aux_normal(SEED, (131,), n, 0.02), "m": aux_normal(SEED, (132,), n, 1e-3),
+              "v": aux_uniform(SEED, (133,), n, 1e-8, 1e-6), "err": err.copy()}
+        ref = {k: v.copy() for k, v in st.items()}
+        flags = o.ternary_step(off, g, st, B1, LR, EPS, optimizer=opt)
+        codes, f1 = o.ternary_compress(off, g, ref["err"], B1)
+        srv = o.ternary_server(off, codes)
+        _, f2 = o.ternary_apply(off, W, srv, ref["m"], ref["v"], ref["p"], B1, LR, EPS, optimizer=opt)
+        assert flags == f1 | f2
+        for k in ("p", "m", "v", "err"):
+            assert np.array_equal(st[k], ref[k]), (opt, k)
+        assert np.array_equal(st["codes_w"], codes) and np.array_equal(st["codes_srv"], srv)
+
+
+def pin_ternary_nonfinite(o):
+    """A NaN gradient gives code 0 and a NaN error; +inf gives code +1 and an
+    infinite error; both raise the flag (the check after the error update).
+    Large finite values do not."""
+    off = [0, 4]
+    g = np.array([[np.nan, np.inf, -3e38, 1.0]], np.float32)
+    err = np.zeros_like(g)
+    codes, flags = o.ternary_compress(off, g, err, B1)
+    assert flags == 1
+    assert [int(x) for x in codes[0][:4]] == [0, 1, -1, 1]
+    assert np.isnan(err[0, 0]) and np.isposinf(err[0, 1]) and np.isfinite(err[0, 2:]).all()
+    g2 = np.array([[-3e38, 3e38, 0.0, 1.0]], np.float32)
+    _, flags = o.ternary_compress(off, g2, np.zeros_like(g2), B1)
+    assert flags == 0
+
+
+def pin_ternary_clip(o):
+    """clip > 0 clamps the raw gradient before eps is added: a clipped run equals
+    the run on numpy's clamped gradient, bit for bit; NaN passes through."""
+    sizes = [40, 33]
+    off = offsets_of(sizes)
+    g, err = _ternary_inputs(2, sizes, (140,), gscale=8.0)
+    e1, e2 = err.copy(), err.copy()
+    c1, _ = o.ternary_compress(off, g, e1, B1, clip=5.0)
+    c2, _ = o.ternary_compress(off, np.clip(g, -5, 5).astype(np.float32), e2, B1)
+    assert np.array_equal(c1, c2) and np.array_equal(e1, e2)
+    assert np.abs(g).max() > 5
+
+
+def pin_ternary_bf16(o):
+    """bf16 gradients widen exactly (same result as their float32 values); bf16
+    error storage keeps torch's round-to-nearest-even bfloat16 of the float32
+    result."""
+    sizes = RAGGED
+    off = offsets_of(sizes)
+    g, err = _ternary_inputs(2, sizes, (150,))
+    gb = _bf16_of(g)
+    eb = _bf16_of(err)
+    e32 = _widen(eb)
+    c_b, _ = o.ternary_compress(off, gb, eb, B1)
+    c_f, _ = o.ternary_compress(off, _widen(gb), e32, B1)
+    assert np.array_equal(c_b, c_f)
+    assert np.array_equal(eb, _bf16_of(e32))
+
+
 ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_") and callable(v)]

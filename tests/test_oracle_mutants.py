@@ -48,6 +48,24 @@ MUTANTS = {
                         "wo[k + 1] = wo[k] + (off[k + 1] - off[k]) / 32;"),
     "nan_not_flagged": ("static int is_nonfinite(float x) { return !isfinite(x); }",
                         "static int is_nonfinite(float x) { return isinf(x); }"),
+    # the momentum-error rule
+    "ternary_zero_is_positive": ("if (c > 0.0f) return 1;", "if (c >= 0.0f) return 1;"),
+    "ternary_error_coeffs_swapped": ("float eps_new = beta1 * eps_old + one_minus_b1 * delta;",
+                                     "float eps_new = one_minus_b1 * eps_old + beta1 * delta;"),
+    "ternary_error_not_compensated": ("clip_grad(grad_at(grads, dtype, e), clip) + eps_old;",
+                                      "clip_grad(grad_at(grads, dtype, e), clip) + 0.0f;"),
+    "ternary_delta_sign": ("float delta = c - (float)q;", "float delta = (float)q - c;"),
+    "ternary_error_is_delta": ("float eps_new = beta1 * eps_old + one_minus_b1 * delta;",
+                               "float eps_new = delta;"),
+    "ternary_server_first_worker_only": ("for (int32_t w = 0; w < W; ++w) sum += codes_w",
+                                         "for (int32_t w = 0; w < 1; ++w) sum += codes_w"),
+    "ternary_mean_not_divided": ("float g_hat = (float)codes_srv[4 * cw[k] + i] / (float)W;",
+                                 "float g_hat = (float)codes_srv[4 * cw[k] + i];"),
+    "ternary_code_word_base": ("cw[k + 1] = cw[k] + code_words_of(off[k + 1] - off[k]);",
+                               "cw[k + 1] = cw[k] + (off[k + 1] - off[k]) / 4;"),
+    "ternary_nan_check_dropped": ("if (is_nonfinite(eps_new)) flags |= ORC_STATUS_NONFINITE;", ""),
+    "ternary_clip_after_error": ("float c = clip_grad(grad_at(grads, dtype, e), clip) + eps_old;",
+                                 "float c = clip_grad(grad_at(grads, dtype, e) + eps_old, clip);"),
 }
 
 
