@@ -48,7 +48,7 @@ FALLBACK_HBM_GBS = 6650.0
 E2E_MAX_HOST_BYTES = 16e9        # pinned host gradients per step the e2e leg may hold
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "ncu_traffic.txt")
 KERNEL_SOURCES = [os.path.join(ROOT, "bit_adam_error_b200", "csrc", f)
-                  for f in ("kernels.cuh", "onebit.cu")]
+                  for f in ("kernels.cuh", "ternary.cuh", "onebit.cu")]
 
 
 def parse_args():
@@ -65,6 +65,9 @@ def parse_args():
     ap.add_argument("--phase", choices=["compressed", "refresh"], default="compressed",
                     help="time the compressed step (default) or the full-precision variance-refresh "
                          "step of 0/1 Adam")
+    ap.add_argument("--rule", choices=["scaled", "momentum"], default="scaled",
+                    help="compression rule: scaled sign bits with worker and server error "
+                         "(default), or the momentum-error rule with int8 ternary codes")
     ap.add_argument("--err-dtype", choices=["f32", "bf16"], default=None,
                     help="storage of the error buffers (default: the workload's, f32)")
     ap.add_argument("--dp", action="store_true",
@@ -98,12 +101,23 @@ def algo_bytes_per_elem(kind: str, wl) -> float:
         return 16.0
     if kind == "k_warmup":               # g (xW), m, v, p reads; m, v (+ p for Adam) writes
         return gb * W + (20 if wl.optimizer == "lamb" else 24)
+    # the momentum-error rule
+    if kind == "k_ternary_step":         # g, err r/w per worker; m r/w, v, p r (+ p w for Adam)
+        return (gb + 2 * eb) * W + (16 if wl.optimizer == "lamb" else 20)
+    if kind == "k_ternary_compress":     # g, err r/w, one code byte per worker
+        return (gb + 2 * eb + 1) * W
+    if kind == "k_ternary_server":       # W code bytes in, one sum byte out
+        return W + 1.0
+    if kind == "k_ternary_update":       # one sum byte, m r/w, v, p r (+ p w for Adam)
+        return 1 + (16 if wl.optimizer == "lamb" else 20)
     return 0.0                           # finalisers: a few bytes per chunk
 
 
-def step_bytes_per_elem(wl, phase: str = "compressed") -> float:
+def step_bytes_per_elem(wl, phase: str = "compressed", rule: str = "scaled") -> float:
     if phase == "refresh":
         return algo_bytes_per_elem("k_warmup", wl) + (16.0 if wl.optimizer == "lamb" else 0.0)
+    if rule == "momentum":
+        return algo_bytes_per_elem("k_ternary_step", wl) + (16.0 if wl.optimizer == "lamb" else 0.0)
     kinds = ["k_worker_norm", "k_worker_pack", "k_server_update"]
     if wl.optimizer == "lamb":
         kinds.append("k_lamb_param")
@@ -236,7 +250,7 @@ def max_over_ranks(dist, x: float, device) -> float:
 
 # -- CPU oracle timing ----------------------------------------------------------------------
 
-def oracle_rate(wl, chunks, max_elems=None, min_seconds=0.0, steps=1, phase="compressed"):
+def oracle_rate(wl, chunks, max_elems=None, min_seconds=0.0, steps=1, phase="compressed", rule="scaled"):
     """Time the single-threaded oracle's compressed step (or full-precision
     refresh step) on whole chunks (or on the first max_elems elements of a
     chunk, taken as one chunk)."""
@@ -261,6 +275,9 @@ def oracle_rate(wl, chunks, max_elems=None, min_seconds=0.0, steps=1, phase="com
             if phase == "refresh":
                 o.warmup([0, nk], g, st["m"], st["v"], st["p"], f(wl.beta1), f(wl.beta2), f(wl.lr),
                          f(wl.eps), optimizer=opt)
+            elif rule == "momentum":
+                o.ternary_step([0, nk], g, st, f(wl.beta1), f(wl.lr), f(wl.eps), clip=wl.clip,
+                               optimizer=opt)
             else:
                 o.step([0, nk], g, st, f(wl.beta1), f(wl.lr), f(wl.eps), clip=wl.clip, optimizer=opt)
             dt = time.perf_counter() - t
@@ -279,16 +296,17 @@ def run_reference(args):
         return 0
     wl = select_workload(args)
     sample = 1 << 23
-    elems, secs, per_step, used = oracle_rate(wl, [0], max_elems=sample, steps=args.warmup + args.steps)
+    elems, secs, per_step, used = oracle_rate(wl, [0], max_elems=sample, steps=args.warmup + args.steps,
+                                              rule=args.rule)
     timed = per_step[args.warmup:]
     ms = 1e3 * sum(timed) / len(timed)
     value = used[0][1] / (ms / 1e3) / 1e9
     sample_txt = (f"first {used[0][1]} elements of chunk 0 of {wl.name} taken as one chunk, "
-                  f"W={wl.W}, one compressed step per bench step, single thread")
+                  f"W={wl.W}, one compressed step per bench step ({args.rule} rule), single thread")
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-            "config": workload_config(wl, args.gpus),
+            "config": workload_config(wl, args.gpus, args.rule),
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
                              "sample": sample_txt},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -308,12 +326,13 @@ def select_workload(args):
     return wl
 
 
-def workload_config(wl, n_gpus):
+def workload_config(wl, n_gpus, rule="scaled"):
     return {"workload": f"{wl.name}: {wl.description}", "n": wl.n, "chunks": wl.C, "W": wl.W,
             "grad_dtype": wl.grad_dtype, "state_dtype": "f32", "err_dtype": wl.err_dtype,
-            "optimizer": wl.optimizer,
+            "optimizer": wl.optimizer, "rule": rule,
             "global_batch": wl.W * n_gpus, "parallelism": f"{n_gpus} replica(s) x {wl.W} virtual workers",
-            "l2": f"inputs larger than L2: {step_bytes_per_elem(wl) * wl.n / 1e9:.1f} GB of traffic per step"}
+            "l2": f"inputs larger than L2: {step_bytes_per_elem(wl, 'compressed', rule) * wl.n / 1e9:.1f} "
+                  "GB of traffic per step"}
 
 
 # -- our arm -------------------------------------------------------------------------------
@@ -337,7 +356,7 @@ def run_ours(args):
     # State: seeded p, v generated a chunk group at a time and uploaded once.
     opt = OneBitAdam(wl.offsets, W, grad_dtype=wl.grad_dtype, optimizer=wl.optimizer, clip=wl.clip,
                      freeze_step=0, lr=wl.lr, beta1=wl.beta1, beta2=wl.beta2, eps=wl.eps,
-                     err_dtype=wl.err_dtype, device=device)
+                     err_dtype=wl.err_dtype, rule=args.rule, device=device)
     swl = wl.with_(freeze_step=0)
     for k0, k1 in WL.chunk_groups(wl):
         lo, hi = int(wl.offsets[k0]), int(wl.offsets[k1])
@@ -404,7 +423,7 @@ def run_ours(args):
                    "algorithmic_GBps": (algo_bytes_per_elem(k, wl) * n / (v[0] / v[1] / 1e3) / 1e9)
                    if algo_bytes_per_elem(k, wl) else None}
                for k, v in prof.items()}
-    step_gbs = step_bytes_per_elem(wl, args.phase) * n / (ms_max / 1e3) / 1e9
+    step_gbs = step_bytes_per_elem(wl, args.phase, args.rule) * n / (ms_max / 1e3) / 1e9
 
     # -- error-buffer monitoring (one call, timed alone) -----------------------------
     monitor = None
@@ -414,7 +433,7 @@ def run_ours(args):
         e1.record(stream)
         torch.cuda.synchronize()
         mon_ms = e0.elapsed_time(e1)
-        mon_bytes = wl.err_bytes * n * (W + 1)
+        mon_bytes = wl.err_bytes * n * (W + (1 if opt.srv_err is not None else 0))
         monitor = {"ms": mon_ms, "GBps": mon_bytes / (mon_ms / 1e3) / 1e9,
                    "frac": mon_bytes / (mon_ms / 1e3) / 1e9 / peak, "bytes": mon_bytes}
 
@@ -435,6 +454,9 @@ def run_ours(args):
             WL.fill_grads(wl, b + 1000 * rank, arr)
             host_g.append(h)
         nh = len(host_g)
+        # The step's result read back each step: the server scales, or (the
+        # momentum-error rule has none) the first C parameters.
+        result = opt.s_srv if opt.s_srv is not None else opt.p[: wl.C]
         s_host = torch.empty(wl.C, dtype=torch.float32, pin_memory=True)
         for i in range(2):
             opt.step(host_g[i % nh])
@@ -444,7 +466,7 @@ def run_ours(args):
         e0.record(stream)
         for i in range(args.steps):
             opt.step(host_g[i % nh])
-            s_host.copy_(opt.s_srv, non_blocking=True)
+            s_host.copy_(result, non_blocking=True)
         e1.record(stream)
         torch.cuda.synchronize()
         barrier(dist)
@@ -455,10 +477,11 @@ def run_ours(args):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        elems, secs, _, used = oracle_rate(wl, list(range(wl.C)), min_seconds=10.0, phase=args.phase)
+        elems, secs, _, used = oracle_rate(wl, list(range(wl.C)), min_seconds=10.0, phase=args.phase,
+                                           rule=args.rule)
         cpu = {"value": elems / secs / 1e9, "unit": UNIT, "cores": 1, "kind": "oracle",
                "sample": f"{len(used)} whole chunk(s) {[k for k, _ in used]} of {wl.name} "
-                         f"({elems} elements), one {args.phase} step each, single thread, "
+                         f"({elems} elements), one {args.phase} step each ({args.rule} rule), single thread, "
                          f"{secs:.1f} s"}
 
     if rank == 0:
@@ -466,10 +489,11 @@ def run_ours(args):
                 "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max,
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
                 "data": "synthetic (seeded Philox streams; shapes and distributions of the workload)",
-                "config": workload_config(wl, world),
+                "config": workload_config(wl, world, args.rule),
                 "phase": args.phase,
                 "hbm": {"step_achieved_GBps": step_gbs, "step_frac": step_gbs / peak,
-                        "algorithmic_bytes_per_elem": step_bytes_per_elem(wl, args.phase), "peak": peak,
+                        "algorithmic_bytes_per_elem": step_bytes_per_elem(wl, args.phase, args.rule),
+                        "peak": peak,
                         "peak_source": peak_src},
                 "roofline": roofline, "kernels": kernels, "error_norms_call": monitor,
                 "cpu_baseline": cpu, "e2e": e2e,

@@ -16,6 +16,7 @@ LIB_PATH = os.path.join(_PKG, "libonebit.so")
 OB_OK, OB_EINVAL, OB_ECUDA, OB_EPHASE, OB_ENOMEM = 0, -1, -2, -3, -4
 OB_F32, OB_BF16 = 0, 1
 OB_ADAM, OB_LAMB = 0, 1
+OB_RULE_SCALED_SIGN, OB_RULE_MOMENTUM_ERROR = 0, 1
 OB_STATUS_NONFINITE = 1
 
 ERR_NAMES = {OB_OK: "OB_OK", OB_EINVAL: "OB_EINVAL", OB_ECUDA: "OB_ECUDA",
@@ -37,6 +38,7 @@ class ob_config(ctypes.Structure):
         ("clip", ctypes.c_float),
         ("freeze_step", ctypes.c_int32),
         ("err_dtype", ctypes.c_int32),
+        ("rule", ctypes.c_int32),
     ]
 
 
@@ -70,7 +72,7 @@ _SIGS = {
     "ob_last_error": (ctypes.c_char_p, []),
 }
 
-OB_K_KINDS = 8
+OB_K_KINDS = 12
 
 _lib = None
 
@@ -107,12 +109,13 @@ def check(code: int, call: str) -> None:
 
 
 def make_config(n, offsets, W, grad_dtype=OB_F32, optimizer=OB_ADAM, lr=1e-4, beta1=0.9,
-                beta2=0.999, eps=1e-8, clip=0.0, freeze_step=0, err_dtype=OB_F32):
+                beta2=0.999, eps=1e-8, clip=0.0, freeze_step=0, err_dtype=OB_F32,
+                rule=OB_RULE_SCALED_SIGN):
     """Build an ob_config; returns (config, offsets_array) -- keep both alive."""
     arr = (ctypes.c_int64 * len(offsets))(*[int(x) for x in offsets])
     cfg = ob_config(int(n), len(offsets) - 1, arr, int(W), int(grad_dtype), int(optimizer),
                     float(lr), float(beta1), float(beta2), float(eps), float(clip), int(freeze_step),
-                    int(err_dtype))
+                    int(err_dtype), int(rule))
     return cfg, arr
 
 

@@ -21,6 +21,7 @@
 
 #include "onebit.h"
 #include "kernels.cuh"
+#include "ternary.cuh"
 
 namespace {
 
@@ -44,6 +45,16 @@ ob_err cuda_fail(cudaError_t e, const char* what) {
 constexpr uintptr_t kAlignElems = 32, kAlignWords = 4;
 
 int64_t words_of(int64_t n) { return (n + 31) / 32; }
+
+bool momentum_rule(const ob_config* c) { return c->rule == OB_RULE_MOMENTUM_ERROR; }
+
+// Words of one chunk in a packed row: sign bits, or int8 codes four to a word.
+int64_t row_words_of(const ob_config* c, int64_t nk) {
+  return momentum_rule(c) ? (nk + 3) / 4 : words_of(nk);
+}
+
+// The int8 sum of W codes in {-1, 0, 1} is exact up to this many workers.
+constexpr int32_t kMaxMomentumWorkers = 127;
 
 // Checks everything about a config that needs no device.
 ob_err check_config(const ob_config* c) {
@@ -69,6 +80,10 @@ ob_err check_config(const ob_config* c) {
   if (c->freeze_step < 0) return fail(OB_EINVAL, "freeze_step = %d < 0", c->freeze_step);
   if (c->err_dtype != OB_F32 && c->err_dtype != OB_BF16)
     return fail(OB_EINVAL, "err_dtype = %d is neither OB_F32 nor OB_BF16", c->err_dtype);
+  if (c->rule != OB_RULE_SCALED_SIGN && c->rule != OB_RULE_MOMENTUM_ERROR)
+    return fail(OB_EINVAL, "rule = %d is neither OB_RULE_SCALED_SIGN nor OB_RULE_MOMENTUM_ERROR", c->rule);
+  if (momentum_rule(c) && c->W > kMaxMomentumWorkers)
+    return fail(OB_EINVAL, "W = %d > %d: the int8 sum of the codes could overflow", c->W, kMaxMomentumWorkers);
   // Element and word indices of [W][n] rows must fit in int64 comfortably.
   if (c->n > (int64_t(1) << 50) / c->W) return fail(OB_EINVAL, "W * n too large");
   return OB_OK;
@@ -336,7 +351,90 @@ void enqueue_server_stage(ob_ctx* c, cudaStream_t st) {
   enqueue_server_update<ob::Upd::kNone, true>(c, st);
 }
 
+// ---- the momentum-error rule ---------------------------------------------------------
+
+template <typename GT, typename ET, bool CLIP, bool POW2>
+void enqueue_ternary_step_t(ob_ctx* c, const GT* grads, cudaStream_t st) {
+  if (c->T == 0) return;
+  auto k = c->cfg.optimizer == OB_LAMB ? ob::k_ternary_step<GT, ET, CLIP, POW2, ob::Upd::kLambM>
+                                       : ob::k_ternary_step<GT, ET, CLIP, POW2, ob::Upd::kAdam>;
+  const int g = grid_for(c, k, c->T);
+  launch(c, OB_K_TERNARY_STEP, st, [&] {
+    k<<<g, ob::kBlock, 0, st>>>(c->L, c->cfg.W, grads, static_cast<ET*>(c->err), c->m, c->v, c->p,
+                                c->h, c->partP, c->partU, c->status);
+  });
+}
+
+template <typename GT, typename ET, bool CLIP>
+void enqueue_ternary_compress_t(ob_ctx* c, const GT* grads, cudaStream_t st) {
+  if (c->T == 0) return;
+  auto k = ob::k_ternary_compress<GT, ET, CLIP>;
+  const int g = grid_for(c, k, c->cfg.W * c->T);
+  launch(c, OB_K_TERNARY_COMPRESS, st, [&] {
+    k<<<g, ob::kBlock, 0, st>>>(c->L, c->cfg.W, grads, static_cast<ET*>(c->err), c->bits_w, c->h,
+                                c->status);
+  });
+}
+
+// Worker stage (fused = false) or the whole one-pass step (fused = true).
+template <typename GT, typename ET>
+void enqueue_ternary_e(ob_ctx* c, const GT* grads, bool fused, cudaStream_t st) {
+  const bool clip = c->h.clip > 0.0f, p2 = pow2_workers(c);
+  if (!fused) {
+    if (clip) enqueue_ternary_compress_t<GT, ET, true>(c, grads, st);
+    else enqueue_ternary_compress_t<GT, ET, false>(c, grads, st);
+    return;
+  }
+  if (clip && p2) enqueue_ternary_step_t<GT, ET, true, true>(c, grads, st);
+  else if (clip) enqueue_ternary_step_t<GT, ET, true, false>(c, grads, st);
+  else if (p2) enqueue_ternary_step_t<GT, ET, false, true>(c, grads, st);
+  else enqueue_ternary_step_t<GT, ET, false, false>(c, grads, st);
+  if (c->cfg.optimizer == OB_LAMB) enqueue_lamb_param(c, st);
+}
+
+void enqueue_ternary(ob_ctx* c, const void* grads, bool fused, cudaStream_t st) {
+  const bool bf16_err = c->cfg.err_dtype == OB_BF16;
+  if (c->cfg.grad_dtype == OB_BF16) {
+    const uint16_t* g = static_cast<const uint16_t*>(grads);
+    if (bf16_err) enqueue_ternary_e<uint16_t, uint16_t>(c, g, fused, st);
+    else enqueue_ternary_e<uint16_t, float>(c, g, fused, st);
+  } else {
+    const float* g = static_cast<const float*>(grads);
+    if (bf16_err) enqueue_ternary_e<float, uint16_t>(c, g, fused, st);
+    else enqueue_ternary_e<float, float>(c, g, fused, st);
+  }
+}
+
+void enqueue_ternary_server(ob_ctx* c, cudaStream_t st) {
+  if (c->words == 0) return;
+  auto k = ob::k_ternary_server;
+  const int g = grid_for(c, k, (c->words + 31) / 32);
+  launch(c, OB_K_TERNARY_SERVER, st, [&] {
+    k<<<g, ob::kBlock, 0, st>>>(c->cfg.W, c->words, c->bits_w, c->bits_srv);
+  });
+}
+
+void enqueue_ternary_update(ob_ctx* c, cudaStream_t st) {
+  const bool lamb = c->cfg.optimizer == OB_LAMB, p2 = pow2_workers(c);
+  if (c->T > 0) {
+    auto k = lamb ? (p2 ? ob::k_ternary_update<ob::Upd::kLambM, true> : ob::k_ternary_update<ob::Upd::kLambM, false>)
+                  : (p2 ? ob::k_ternary_update<ob::Upd::kAdam, true> : ob::k_ternary_update<ob::Upd::kAdam, false>);
+    const int g = grid_for(c, k, c->T);
+    launch(c, OB_K_TERNARY_UPDATE, st, [&] {
+      k<<<g, ob::kBlock, 0, st>>>(c->L, c->cfg.W, c->bits_srv, c->m, c->v, c->p, c->h, c->partP,
+                                  c->partU, c->status);
+    });
+  }
+  if (lamb) enqueue_lamb_param(c, st);
+}
+
 ob_err fused_step(ob_ctx* c, const void* grads, cudaStream_t st) {
+  if (momentum_rule(&c->cfg)) {
+    enqueue_ternary(c, grads, true, st);
+    ob_err r = check_launch("ob_step");
+    if (r == OB_OK) ++c->step;
+    return r;
+  }
   if (c->cfg.grad_dtype == OB_BF16)
     enqueue_worker<uint16_t>(c, static_cast<const uint16_t*>(grads), true, st);
   else
@@ -359,20 +457,23 @@ enum Need : unsigned {
   kNeedWarm = 2u,    // p, m, v
   kNeedWorker = 4u,  // err, bits_w, s_w
   kNeedServer = 8u,  // srv_err, bits_w, s_w, bits_srv, s_srv
+  kNeedErr = 16u,    // err alone (the one-pass step of the momentum-error rule)
 };
 
 ob_err require_buffers(const ob_ctx* c, unsigned need, const char* call) {
   const int64_t n = c->cfg.n, W = c->cfg.W, C = c->cfg.num_chunks;
+  // The momentum-error rule has no scales and no server error.
+  const unsigned scaled = momentum_rule(&c->cfg) ? 0u : ~0u;
   const struct { unsigned mask; const void* p; int64_t count; const char* name; } list[] = {
       {kNeedUpdate | kNeedWarm, c->p, n, "p"},
       {kNeedUpdate | kNeedWarm, c->m, n, "m"},
       {kNeedUpdate | kNeedWarm, c->v, n, "v"},
-      {kNeedWorker, c->err, W * n, "err"},
-      {kNeedServer, c->srv_err, n, "srv_err"},
+      {kNeedWorker | kNeedErr, c->err, W * n, "err"},
+      {kNeedServer & scaled, c->srv_err, n, "srv_err"},
       {kNeedWorker | kNeedServer, c->bits_w, W * c->words, "bits_w"},
-      {kNeedWorker | kNeedServer, c->s_w, W * C, "s_w"},
+      {(kNeedWorker | kNeedServer) & scaled, c->s_w, W * C, "s_w"},
       {kNeedUpdate | kNeedServer, c->bits_srv, c->words, "bits_srv"},
-      {kNeedUpdate | kNeedServer, c->s_srv, C, "s_srv"}};
+      {(kNeedUpdate | kNeedServer) & scaled, c->s_srv, C, "s_srv"}};
   for (const auto& b : list)
     if ((b.mask & need) && b.count > 0 && !b.p)
       return fail(OB_EINVAL, "%s: the ctx was created without %s", call, b.name);
@@ -396,7 +497,7 @@ ob_err ob_layout(const ob_config* cfg, int64_t* words_total) {
   if (!words_total) return fail(OB_EINVAL, "words_total is NULL");
   int64_t t = 0;
   for (int32_t k = 0; k < cfg->num_chunks; ++k)
-    t += words_of(cfg->chunk_offsets[k + 1] - cfg->chunk_offsets[k]);
+    t += row_words_of(cfg, cfg->chunk_offsets[k + 1] - cfg->chunk_offsets[k]);
   *words_total = t;
   return OB_OK;
 }
@@ -448,7 +549,7 @@ ob_err ob_create(const ob_config* cfg, float* p, float* m, float* v, void* err, 
   wo[0] = tp[0] = 0;
   for (int64_t k = 0; k < C; ++k) {
     const int64_t o = c->off[k], nk = c->off[k + 1] - o;
-    wo[k + 1] = wo[k] + words_of(nk);
+    wo[k + 1] = wo[k] + row_words_of(cfg, nk);
     tp[k + 1] = tp[k] + (nk + ob::kTile - 1) / ob::kTile;
     // 8-wide path: chunk start and length multiples of 8, and every worker row
     // starts on a multiple of 8 elements (16 bytes of bf16, 32 bytes of fp32).
@@ -553,7 +654,8 @@ ob_err ob_compress(ob_ctx* c, const void* grads, void* stream) {
   if (!dg.ok) return fail(OB_ECUDA, "cannot select device %d", c->device);
   if ((r = check_grads(c, grads)) != OB_OK) return r;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (c->cfg.grad_dtype == OB_BF16) enqueue_worker<uint16_t>(c, static_cast<const uint16_t*>(grads), false, st);
+  if (momentum_rule(&c->cfg)) enqueue_ternary(c, grads, false, st);
+  else if (c->cfg.grad_dtype == OB_BF16) enqueue_worker<uint16_t>(c, static_cast<const uint16_t*>(grads), false, st);
   else enqueue_worker<float>(c, static_cast<const float*>(grads), false, st);
   return check_launch("ob_compress");
 }
@@ -565,7 +667,8 @@ ob_err ob_server_reduce(ob_ctx* c, void* stream) {
   if ((r = require_buffers(c, kNeedServer, "ob_server_reduce")) != OB_OK) return r;
   DeviceGuard dg(c->device);
   if (!dg.ok) return fail(OB_ECUDA, "cannot select device %d", c->device);
-  enqueue_server_stage(c, static_cast<cudaStream_t>(stream));
+  if (momentum_rule(&c->cfg)) enqueue_ternary_server(c, static_cast<cudaStream_t>(stream));
+  else enqueue_server_stage(c, static_cast<cudaStream_t>(stream));
   return check_launch("ob_server_reduce");
 }
 
@@ -573,8 +676,11 @@ ob_err ob_step(ob_ctx* c, const void* grads, void* stream) {
   ob_err r = check_ctx(c);
   if (r != OB_OK) return r;
   if ((r = require_compressed(c, "ob_step")) != OB_OK) return r;
-  if ((r = require_buffers(c, grads ? (kNeedWorker | kNeedServer | kNeedUpdate) : kNeedUpdate, "ob_step")) != OB_OK)
-    return r;
+  // The fused step of the momentum-error rule touches p, m, v and err only.
+  const unsigned need = !grads ? kNeedUpdate
+                        : momentum_rule(&c->cfg) ? (kNeedWarm | kNeedErr)
+                                                 : (kNeedWorker | kNeedServer | kNeedUpdate);
+  if ((r = require_buffers(c, need, "ob_step")) != OB_OK) return r;
   DeviceGuard dg(c->device);
   if (!dg.ok) return fail(OB_ECUDA, "cannot select device %d", c->device);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -582,7 +688,8 @@ ob_err ob_step(ob_ctx* c, const void* grads, void* stream) {
     if ((r = check_grads(c, grads)) != OB_OK) return r;
     return fused_step(c, grads, st);
   }
-  enqueue_update(c, false, st);
+  if (momentum_rule(&c->cfg)) enqueue_ternary_update(c, st);
+  else enqueue_update(c, false, st);
   if ((r = check_launch("ob_step")) != OB_OK) return r;
   ++c->step;
   return OB_OK;
@@ -613,7 +720,8 @@ ob_err ob_step_host(ob_ctx* c, const void* host_grads, void* dev_staging, void* 
   ob_err r = check_ctx(c);
   if (r != OB_OK) return r;
   if ((r = require_compressed(c, "ob_step_host")) != OB_OK) return r;
-  if ((r = require_buffers(c, kNeedWorker | kNeedServer | kNeedUpdate, "ob_step_host")) != OB_OK) return r;
+  const unsigned need = momentum_rule(&c->cfg) ? (kNeedWarm | kNeedErr) : (kNeedWorker | kNeedServer | kNeedUpdate);
+  if ((r = require_buffers(c, need, "ob_step_host")) != OB_OK) return r;
   const int64_t count = int64_t(c->cfg.W) * c->cfg.n;
   if (count > 0 && !host_grads) return fail(OB_EINVAL, "host_grads is NULL");
   DeviceGuard dg(c->device);
@@ -697,6 +805,8 @@ ob_err ob_error_norms(ob_ctx* c, float* worker_norms, float* server_norms, void*
   const int64_t W = c->cfg.W, C = c->cfg.num_chunks;
   if (!worker_norms && !server_norms) return fail(OB_EINVAL, "ob_error_norms: no output");
   if (worker_norms && !c->err && c->cfg.n > 0) return fail(OB_EINVAL, "ob_error_norms: the ctx has no err");
+  if (server_norms && momentum_rule(&c->cfg))
+    return fail(OB_EINVAL, "ob_error_norms: the momentum-error rule has no server error");
   if (server_norms && !c->srv_err && c->cfg.n > 0) return fail(OB_EINVAL, "ob_error_norms: the ctx has no srv_err");
   DeviceGuard dg(c->device);
   if (!dg.ok) return fail(OB_ECUDA, "cannot select device %d", c->device);
@@ -783,7 +893,8 @@ ob_err ob_profile_stop(ob_ctx* c, double* ms, int64_t* launches) {
 const char* ob_kernel_name(int32_t kind) {
   static const char* names[OB_K_KINDS] = {
       "k_worker_norm", "k_finalize_scale", "k_worker_pack", "k_server_norm",
-      "k_server_update", "k_lamb_param", "k_warmup", "k_finalize_ratio"};
+      "k_server_update", "k_lamb_param", "k_warmup", "k_finalize_ratio",
+      "k_ternary_step", "k_ternary_compress", "k_ternary_server", "k_ternary_update"};
   return (kind >= 0 && kind < OB_K_KINDS) ? names[kind] : "";
 }
 
@@ -868,6 +979,8 @@ extern "C" ob_err ob_compress_noalloc(const ob_config* cfg, const void* grads, f
   const int64_t n = cfg->n, W = cfg->W, C = cfg->num_chunks;
   if (cfg->err_dtype != OB_F32)
     return fail(OB_EINVAL, "ob_compress_noalloc: float32 error buffers only");
+  if (cfg->rule != OB_RULE_SCALED_SIGN)
+    return fail(OB_EINVAL, "ob_compress_noalloc: the scaled-sign rule only");
   if (C > kNoAllocMaxChunks)
     return fail(OB_EINVAL, "ob_compress_noalloc: %lld chunks, at most %d", (long long)C, kNoAllocMaxChunks);
   // Scratch needed: header (tables, status) + one double per (worker, warp tile).

@@ -12,6 +12,11 @@ in HBM as flat buffers:
   bits_srv         : uint32  [words]
   s_srv            : float32 [C]
 
+With ``rule="momentum"`` (the momentum-error rule of the CANN 1-bit Adam
+article, sections 2.1-3.2) bits_w / bits_srv hold int8 codes and their sums
+(``codes_w`` / ``codes_srv`` give int8 views), and srv_err, s_w, s_srv are
+absent (None): that rule has no scale and no server error.
+
 Phases follow "DeepSpeed Communication Compression and Hiding" (section
 "1-bit Adam", 机制): ``step()`` runs the full-precision warmup while
 ``step_count < freeze_step`` and the fused compressed step afterwards (the
@@ -37,7 +42,7 @@ class OneBitAdam:
     def __init__(self, offsets: Sequence[int], W: int, *, grad_dtype: str = "f32",
                  optimizer: str = "adam", lr: float = 1e-4, beta1: float = 0.9,
                  beta2: float = 0.999, eps: float = 1e-8, clip: float = 0.0,
-                 freeze_step: int = 0, err_dtype: str = "f32", device=None,
+                 freeze_step: int = 0, err_dtype: str = "f32", rule: str = "scaled", device=None,
                  p: Optional[torch.Tensor] = None, m: Optional[torch.Tensor] = None,
                  v: Optional[torch.Tensor] = None):
         self.device = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
@@ -50,9 +55,11 @@ class OneBitAdam:
         self.optimizer = {"adam": L.OB_ADAM, "lamb": L.OB_LAMB}[optimizer]
         self.err_dtype = {"f32": L.OB_F32, "bf16": L.OB_BF16}[err_dtype]
         edt = torch.float32 if self.err_dtype == L.OB_F32 else torch.bfloat16
+        self.rule = {"scaled": L.OB_RULE_SCALED_SIGN, "momentum": L.OB_RULE_MOMENTUM_ERROR}[rule]
+        scaled = self.rule == L.OB_RULE_SCALED_SIGN
         self.cfg, self._off_keep = L.make_config(self.n, self.offsets, self.W, self.grad_dtype,
                                                  self.optimizer, lr, beta1, beta2, eps, clip,
-                                                 freeze_step, self.err_dtype)
+                                                 freeze_step, self.err_dtype, self.rule)
         self.words = L.ob_layout(self.cfg)
         dev, f32 = self.device, torch.float32
 
@@ -66,17 +73,27 @@ class OneBitAdam:
         self.m = state(m, (self.n,))
         self.v = state(v, (self.n,))
         self.err = torch.zeros((self.W, self.n), dtype=edt, device=dev)
-        self.srv_err = torch.zeros(self.n, dtype=edt, device=dev)
+        self.srv_err = torch.zeros(self.n, dtype=edt, device=dev) if scaled else None
         self.bits_w = torch.zeros((self.W, self.words), dtype=torch.int32, device=dev)
-        self.s_w = torch.zeros((self.W, self.C), dtype=f32, device=dev)
+        self.s_w = torch.zeros((self.W, self.C), dtype=f32, device=dev) if scaled else None
         self.bits_srv = torch.zeros(self.words, dtype=torch.int32, device=dev)
-        self.s_srv = torch.zeros(self.C, dtype=f32, device=dev)
+        self.s_srv = torch.zeros(self.C, dtype=f32, device=dev) if scaled else None
         with torch.cuda.device(dev):
             self.ctx = L.ob_create(self.cfg, _ptr(self.p), _ptr(self.m), _ptr(self.v),
                                    _ptr(self.err), _ptr(self.srv_err), _ptr(self.bits_w),
                                    _ptr(self.s_w), _ptr(self.bits_srv), _ptr(self.s_srv))
         self._staging: list = []       # two device buffers for host gradients, used alternately
         self._staging_turn = 0
+
+    @property
+    def codes_w(self) -> torch.Tensor:
+        """Momentum-error rule: the workers' int8 codes [W, 4 * words] (a view)."""
+        return self.bits_w.view(torch.int8)
+
+    @property
+    def codes_srv(self) -> torch.Tensor:
+        """Momentum-error rule: the per-element code sums, int8 [4 * words] (a view)."""
+        return self.bits_srv.view(torch.int8)
 
     # -- plumbing -----------------------------------------------------------------
     def _stream(self) -> int:
@@ -156,9 +173,10 @@ class OneBitAdam:
         """(worker norms [W, C], server norms [C]) of the error buffers, per chunk,
         as device tensors (monitoring; the CANN article's error-norm check)."""
         wn = torch.empty((self.W, self.C), dtype=torch.float32, device=self.device)
-        sn = torch.empty(self.C, dtype=torch.float32, device=self.device)
-        L.ob_error_norms(self.ctx, _ptr(wn) if wn.numel() else 0, _ptr(sn) if sn.numel() else 0,
-                         self._stream())
+        sn = torch.empty(self.C, dtype=torch.float32, device=self.device) \
+            if self.srv_err is not None else None
+        L.ob_error_norms(self.ctx, _ptr(wn) if wn.numel() else 0,
+                         _ptr(sn) if sn is not None and sn.numel() else 0, self._stream())
         return wn, sn
 
     def status(self, clear: bool = False) -> int:
@@ -166,14 +184,15 @@ class OneBitAdam:
 
     # -- checkpoint ----------------------------------------------------------------
     def state_dict(self) -> Dict[str, object]:
-        keys = ("p", "m", "v", "err", "srv_err")
+        keys = [k for k in ("p", "m", "v", "err", "srv_err") if getattr(self, k) is not None]
         sd: Dict[str, object] = {k: getattr(self, k).detach().cpu().clone() for k in keys}
         sd["step"] = self.step_count
         return sd
 
     def load_state_dict(self, sd: Dict[str, object]) -> None:
         for k in ("p", "m", "v", "err", "srv_err"):
-            getattr(self, k).copy_(sd[k])  # type: ignore[arg-type]
+            if getattr(self, k) is not None:
+                getattr(self, k).copy_(sd[k])  # type: ignore[arg-type]
         self.set_step(int(sd["step"]))  # type: ignore[arg-type]
 
     def close(self) -> None:

@@ -29,6 +29,15 @@
  * either norm is 0), p -= lr r_l u.  Clipping before quantisation (CANN 1-bit
  * Adam article, section 3.2) clamps the raw gradient to [-clip, clip].
  *
+ * A second compression rule, the momentum-error rule of the CANN 1-bit Adam
+ * article (sections 2.1, 2.2 and 3.2), is selected by ob_config.rule =
+ * OB_RULE_MOMENTUM_ERROR.  Per worker and element:
+ *   c = clip(g_w) + err_w;  q = sign(c) in {-1, 0, +1} (sign(+-0) = 0, no scale);
+ *   err_w = beta1 err_w + (1 - beta1) (c - q)
+ * q travels as an int8 code; the W codes of an element are summed (exact in
+ * int8, so W <= 127), g_hat = sum / W, and m, p move as above (v frozen).
+ * There is no server error and no scale under this rule.
+ *
  * Conventions for every call:
  *   - Device buffers are caller-owned and must stay valid for the ctx's life.
  *     The ctx stores their pointers and owns only its own scratch (per-tile
@@ -69,6 +78,10 @@ typedef enum {
 
 enum { OB_F32 = 0, OB_BF16 = 1 };  /* gradient element type */
 enum { OB_ADAM = 0, OB_LAMB = 1 }; /* update rule after the compressed allreduce */
+enum {                             /* compression rule (ob_config.rule) */
+  OB_RULE_SCALED_SIGN = 0,         /* sign bits + per-chunk scale, worker and server error */
+  OB_RULE_MOMENTUM_ERROR = 1       /* int8 ternary codes, momentum-form worker error */
+};
 
 #define OB_STATUS_NONFINITE 1u /* a compensated value, server value or parameter was NaN/Inf */
 
@@ -86,9 +99,14 @@ typedef struct {
   int32_t err_dtype;            /* OB_F32, or OB_BF16: err and srv_err stored as bfloat16
                                    (rounded to nearest even; arithmetic stays float32) --
                                    half the error-buffer bytes, different rounding */
+  int32_t rule;                 /* OB_RULE_SCALED_SIGN (default 0) or OB_RULE_MOMENTUM_ERROR
+                                   (then W <= 127) */
 } ob_config;
 
-/* Number of uint32 words one packed sign row holds: sum_k ceil(n_k / 32).
+/* Number of uint32 words one packed row holds.  OB_RULE_SCALED_SIGN: sign bits,
+ * sum_k ceil(n_k / 32).  OB_RULE_MOMENTUM_ERROR: int8 codes, sum_k ceil(n_k / 4);
+ * element i of chunk k is byte i of the chunk's words (byte b of a word is bits
+ * 8b..8b+7), every chunk starts on a fresh word, padding bytes are 0.
  * Host-only; validates the config.  words_total must be non-NULL. */
 ob_err ob_layout(const ob_config* cfg, int64_t* words_total);
 
@@ -104,6 +122,11 @@ ob_err ob_layout(const ob_config* cfg, int64_t* words_total);
  *   ob_step(NULL): p, m, v, bits_srv, s_srv    ob_step(grads), ob_step_host: all
  * (e.g. a rank that owns some chunks in a multi-GPU step keeps a server-only
  * ctx).  Several ctxs may share a buffer if their calls are ordered.
+ * Under OB_RULE_MOMENTUM_ERROR: bits_w holds the workers' int8 codes and
+ * bits_srv their per-element sums (int8), both in the ob_layout words; srv_err,
+ * s_w and s_srv are never used (pass NULL); ob_compress needs err and bits_w,
+ * ob_server_reduce bits_w and bits_srv, ob_step(NULL) p, m, v and bits_srv, and
+ * ob_step(grads) p, m, v and err only.
  * Allocates the ctx scratch with cudaMalloc on the current device and
  * synchronises once.  *out receives the ctx (NULL on failure). */
 ob_err ob_create(const ob_config* cfg, float* p, float* m, float* v, void* err,
@@ -127,18 +150,24 @@ ob_err ob_refresh_step(ob_ctx* ctx, const void* grads, void* stream);
 
 /* Worker stage only (compressed phase): for every worker and chunk,
  * c = clip(g_w) + err_w, s_w = ||c|| / sqrt(n_k), bits_w = sign(c),
- * err_w = c - s_w sign(c).  grads: DEVICE [W][n].  Step counter unchanged. */
+ * err_w = c - s_w sign(c).  grads: DEVICE [W][n].  Step counter unchanged.
+ * OB_RULE_MOMENTUM_ERROR: bits_w = int8 codes sign(c), err_w = beta1 err_w +
+ * (1 - beta1)(c - sign(c)). */
 ob_err ob_compress(ob_ctx* ctx, const void* grads, void* stream);
 
 /* Server stage only (the compressed allreduce) from bits_w / s_w:
  * c_srv = mean_w(s_w sign_w) + srv_err, s_srv = ||c_srv|| / sqrt(n_k),
- * bits_srv = sign(c_srv), srv_err = c_srv - s_srv sign(c_srv). */
+ * bits_srv = sign(c_srv), srv_err = c_srv - s_srv sign(c_srv).
+ * OB_RULE_MOMENTUM_ERROR: bits_srv = per-element sum of the W int8 codes. */
 ob_err ob_server_reduce(ob_ctx* ctx, void* stream);
 
 /* grads != NULL: the whole fused compressed step (worker stage, server stage,
  * update) on DEVICE grads [W][n].  grads == NULL: the update alone from
  * bits_srv / s_srv (g_hat = s_srv sign), after ob_compress + ob_server_reduce.
- * Advances the step counter.  OB_EPHASE while step < freeze_step. */
+ * Advances the step counter.  OB_EPHASE while step < freeze_step.
+ * OB_RULE_MOMENTUM_ERROR: g_hat = (int8 sum in bits_srv) / W; the fused step is
+ * one pass over the elements that keeps the codes in registers, so it writes
+ * neither bits_w nor bits_srv. */
 ob_err ob_step(ob_ctx* ctx, const void* grads, void* stream);
 
 /* Same as ob_step(ctx, grads, ...) with the gradients in HOST memory:
@@ -169,8 +198,8 @@ ob_err ob_set_step(ob_ctx* ctx, int64_t step);
  * watch the L2 norm of the error buffers; a norm that collapses towards 0
  * signals vanishing updates): writes ||err_w restricted to chunk k||_2 to
  * worker_norms[w * C + k] and ||srv_err on chunk k||_2 to server_norms[k]
- * (DEVICE float arrays; either may be NULL).  Norms are summed in double in a
- * fixed order.  Uses the ctx scratch, so it must be ordered with the ctx's
+ * (DEVICE float arrays; either may be NULL; server_norms must be NULL under
+ * OB_RULE_MOMENTUM_ERROR).  Norms are summed in double in a fixed order.  Uses the ctx scratch, so it must be ordered with the ctx's
  * steps (same stream); it does not change any state. */
 ob_err ob_error_norms(ob_ctx* ctx, float* worker_norms, float* server_norms, void* stream);
 
@@ -185,7 +214,11 @@ enum {
   OB_K_LAMB_PARAM = 5,     /* LAMB parameter step */
   OB_K_WARMUP = 6,         /* full-precision warmup step */
   OB_K_FINALIZE_RATIO = 7, /* LAMB trust ratio per layer */
-  OB_K_KINDS = 8
+  OB_K_TERNARY_STEP = 8,     /* momentum-error rule: the fused one-pass step */
+  OB_K_TERNARY_COMPRESS = 9, /* momentum-error rule: codes + worker error (stage call) */
+  OB_K_TERNARY_SERVER = 10,  /* momentum-error rule: sum of the workers' codes */
+  OB_K_TERNARY_UPDATE = 11,  /* momentum-error rule: update from the code sums */
+  OB_K_KINDS = 12
 };
 
 /* Start recording a CUDA event pair around each of the next `capacity`
@@ -220,7 +253,8 @@ int64_t ob_launch_count(const ob_ctx* ctx);
  *   err_w = c - s_w sign(c)
  * with results identical to ob_compress on the same inputs.  The caller passes
  * the config and DEVICE buffers as for ob_create/ob_compress: grads [W][n]
- * (grad_dtype), err [W][n] (float32, in/out; err_dtype must be OB_F32),
+ * (grad_dtype), err [W][n] (float32, in/out; err_dtype must be OB_F32 and
+ * rule OB_RULE_SCALED_SIGN),
  * bits_w [W][words_total], s_w [W][C]; 32-byte aligned.  lr, betas, eps and
  * freeze_step are ignored.
  *

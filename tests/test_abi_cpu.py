@@ -38,6 +38,14 @@ def test_layout_counts_words_per_chunk():
     assert L.ob_layout(cfg) == 0
 
 
+def test_layout_counts_code_words_under_the_momentum_rule():
+    """int8 codes, four to a word, every chunk on a fresh word."""
+    cfg, _k = L.make_config(100, [0, 33, 33, 97, 100], 3, rule=L.OB_RULE_MOMENTUM_ERROR)
+    assert L.ob_layout(cfg) == 9 + 0 + 16 + 1
+    cfg, _k = L.make_config(8, [0, 8], 127, rule=L.OB_RULE_MOMENTUM_ERROR)
+    assert L.ob_layout(cfg) == 2
+
+
 @pytest.mark.parametrize("kw,frag", [
     (dict(n=10, offsets=[0, 5, 9], W=1), "!= n"),
     (dict(n=10, offsets=[1, 10], W=1), "[0] must be 0"),
@@ -49,6 +57,8 @@ def test_layout_counts_words_per_chunk():
     (dict(n=10, offsets=[0, 10], W=1, lr=float("nan")), "finite"),
     (dict(n=10, offsets=[0, 10], W=1, freeze_step=-1), "freeze_step"),
     (dict(n=-1, offsets=[0, -1], W=1), "n = -1"),
+    (dict(n=10, offsets=[0, 10], W=1, rule=2), "rule = 2"),
+    (dict(n=10, offsets=[0, 10], W=128, rule=1), "W = 128 > 127"),
 ])
 def test_layout_rejects_bad_configs(kw, frag):
     n, off, W = kw.pop("n"), kw.pop("offsets"), kw.pop("W")

@@ -34,3 +34,23 @@ def test_warmup_below_three_is_rejected():
     r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
                         "--warmup", "2"], cwd=ROOT, capture_output=True, text=True, timeout=120)
     assert r.returncode != 0 and "warmup" in r.stderr
+
+
+def test_reference_arm_momentum_rule():
+    d = run_bench("--impl", "reference", "--workload", "tiny", "--rule", "momentum", "--steps", "2",
+                  "--warmup", "3")
+    assert d["config"]["rule"] == "momentum" and d["value"] > 0
+    assert "momentum rule" in d["cpu_baseline"]["sample"]
+
+
+def test_byte_model_of_the_one_pass_step():
+    """The one-pass step moves g and err (read and write) per worker, plus m, v, p."""
+    sys.path.insert(0, ROOT)
+    import bench
+    import workloads as WL
+    wl = WL.get_workload("gpt2xl-flat")
+    assert bench.step_bytes_per_elem(wl, "compressed", "momentum") == 2 + 8 + 20
+    bl = WL.get_workload("bert-large")
+    assert bench.step_bytes_per_elem(bl, "compressed", "momentum") == 16 * 12 + 20
+    lamb = WL.get_workload("lamb-1.3b")
+    assert bench.step_bytes_per_elem(lamb, "compressed", "momentum") == 4 * 12 + 16 + 16

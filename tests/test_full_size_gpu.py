@@ -107,3 +107,39 @@ def test_row_longer_than_two_to_the_31():
         assert_scales(tag + "s_srv", np_of(opt.s_srv[k:k + 1]), ref["s_srv"])
     assert wl.offsets[wl.C - 1] >= (1 << 31)
     opt.close()
+
+
+@pytest.mark.parametrize("name", ["gpt2xl-flat", "bert-large", "lamb-1.3b"])
+def test_full_size_momentum_rule(name):
+    """The momentum-error rule's one-pass step at full size (two compressed
+    steps from the seeded state), compared with the oracle on sampled chunks."""
+    wl = WL.get_workload(name)
+    steps = 2
+    torch.cuda.empty_cache()
+    opt = OneBitAdam(wl.offsets, wl.W, grad_dtype=wl.grad_dtype, optimizer=wl.optimizer,
+                     clip=wl.clip, rule="momentum", device=dev(), **HP)
+    upload_state(wl, opt.p, opt.v)
+    gdt = torch.bfloat16 if wl.grad_dtype == "bf16" else torch.float32
+    G = torch.empty((wl.W, wl.n), dtype=gdt, device=dev())
+    for t in range(steps):
+        upload_grads(wl, t, G)
+        opt.step(G)
+    torch.cuda.synchronize()
+    assert opt.status() == 0
+    del G
+    o = oracle.get()
+    opt_code = oracle.LAMB if wl.optimizer == "lamb" else oracle.ADAM
+    for k in sampled_chunks(wl):
+        nk = wl.sizes[k]
+        lo, hi = int(wl.offsets[k]), int(wl.offsets[k + 1])
+        off = np.array([0, nk], np.int64)
+        pk, vk = WL.chunk_state(wl, k)
+        ref = {"p": pk, "m": np.zeros(nk, np.float32), "v": vk, "err": np.zeros((wl.W, nk), np.float32)}
+        for t in range(steps):
+            g = np.stack([WL.chunk_grads(wl, t, w, k) for w in range(wl.W)])
+            o.ternary_step(off, g, ref, F["beta1"], F["lr"], F["eps"], clip=wl.clip, optimizer=opt_code)
+        tag = f"{name} chunk {k}: "
+        for key in ("p", "m", "v"):
+            assert_state(tag + key, np_of(getattr(opt, key)[lo:hi]), ref[key], off)
+        assert_state(tag + "err", np_of(opt.err[:, lo:hi]), ref["err"], off)
+    opt.close()

@@ -33,10 +33,12 @@ MUTANTS = {
                            "return (uint16_t)((u + 0x8000u) >> 16);"),
     "server_first_worker_only": ("for (int32_t w = 0; w < W; ++w)\n        acc +=",
                                  "for (int32_t w = 0; w < 1; ++w)\n        acc +="),
-    "momentum_coeff": ("float mi = beta1 * m[o + i] + one_minus_b1 * g_hat;",
-                       "float mi = one_minus_b1 * m[o + i] + beta1 * g_hat;"),
-    "param_sign": ("float pi = p[o + i] - lr * mi", "float pi = p[o + i] + lr * mi"),
-    "frozen_v_sqrt_dropped": ("lr * mi / (sqrtf(v[o + i]) + eps)", "lr * mi / (v[o + i] + eps)"),
+    # (anchors of the scaled-sign update: the s_srv line above, 6-space indentation)
+    "momentum_coeff": ("s_srv[k], i);\n      float mi = beta1 * m[o + i] + one_minus_b1 * g_hat;",
+                       "s_srv[k], i);\n      float mi = one_minus_b1 * m[o + i] + beta1 * g_hat;"),
+    "param_sign": ("\n      float pi = p[o + i] - lr * mi", "\n      float pi = p[o + i] + lr * mi"),
+    "frozen_v_sqrt_dropped": ("\n      float pi = p[o + i] - lr * mi / (sqrtf(v[o + i]) + eps);",
+                              "\n      float pi = p[o + i] - lr * mi / (v[o + i] + eps);"),
     "trust_ratio_inverted": ("return (float)(sqrt(P) / sqrt(U));", "return (float)(sqrt(U) / sqrt(P));"),
     "lamb_ratio_dropped": ("float pi = p[i] - lr * r * u;", "float pi = p[i] - lr * u;"),
     "warmup_v_not_squared": ("one_minus_b2 * (g * g)", "one_minus_b2 * g"),
@@ -64,6 +66,9 @@ MUTANTS = {
     "ternary_code_word_base": ("cw[k + 1] = cw[k] + code_words_of(off[k + 1] - off[k]);",
                                "cw[k + 1] = cw[k] + (off[k + 1] - off[k]) / 4;"),
     "ternary_nan_check_dropped": ("if (is_nonfinite(eps_new)) flags |= ORC_STATUS_NONFINITE;", ""),
+    "ternary_momentum_coeff": ("(float)W;\n      float mi = beta1 * m[o + i] + one_minus_b1 * g_hat;",
+                               "(float)W;\n      float mi = one_minus_b1 * m[o + i] + beta1 * g_hat;"),
+    "ternary_param_sign": ("\n        float pi = p[o + i] - lr * mi", "\n        float pi = p[o + i] + lr * mi"),
     "ternary_clip_after_error": ("float c = clip_grad(grad_at(grads, dtype, e), clip) + eps_old;",
                                  "float c = clip_grad(grad_at(grads, dtype, e) + eps_old, clip);"),
 }
