@@ -61,6 +61,7 @@ class DPLayout:
     offsets: np.ndarray              # [C+1] element offsets, layout order
     words: np.ndarray                # [C+1] packed-word offsets, layout order
     kbounds: Tuple[int, ...]         # [world+1] layout positions: rank r owns [kbounds[r], kbounds[r+1])
+    codes_per_word: int = 32         # 32 sign bits, or 4 int8 codes (momentum-error rule)
 
     @property
     def n(self) -> int:
@@ -87,9 +88,13 @@ class DPLayout:
         return self.order.index(k)
 
 
-def plan(sizes: Sequence[int], world: int) -> DPLayout:
+def plan(sizes: Sequence[int], world: int, codes_per_word: int = 32) -> DPLayout:
     """Assign chunks to ranks (largest first to the least-loaded rank, ties to the
-    lower rank) and lay the buffer out grouped by owner."""
+    lower rank) and lay the buffer out grouped by owner.  ``codes_per_word``: 32
+    for the sign bits of the scaled-sign rule, 4 for the int8 codes of the
+    momentum-error rule (every chunk starts on a fresh word either way)."""
+    if codes_per_word not in (4, 32):
+        raise ValueError("codes_per_word must be 32 (sign bits) or 4 (int8 codes)")
     sizes = tuple(int(s) for s in sizes)
     if world < 1:
         raise ValueError("world must be >= 1")
@@ -104,11 +109,12 @@ def plan(sizes: Sequence[int], world: int) -> DPLayout:
     offsets = np.zeros(len(sizes) + 1, np.int64)
     np.cumsum(np.asarray(lay_sizes, np.int64), out=offsets[1:])
     words = np.zeros(len(sizes) + 1, np.int64)
-    np.cumsum(np.asarray([(s + 31) // 32 for s in lay_sizes], np.int64), out=words[1:])
+    cpw = codes_per_word
+    np.cumsum(np.asarray([(s + cpw - 1) // cpw for s in lay_sizes], np.int64), out=words[1:])
     kb = [0] * (world + 1)
     for r in range(world):
         kb[r + 1] = kb[r] + sum(1 for k in order if owner[k] == r)
-    return DPLayout(sizes, world, tuple(owner), order, offsets, words, tuple(kb))
+    return DPLayout(sizes, world, tuple(owner), order, offsets, words, tuple(kb), cpw)
 
 
 # ---- CUDA stage backend ------------------------------------------------------------------
@@ -128,12 +134,18 @@ class CudaStages:
     def __init__(self, layout: DPLayout, rank: int, *, grad_dtype: str = "f32",
                  optimizer: str = "adam", lr: float = 1e-4, beta1: float = 0.9,
                  beta2: float = 0.999, eps: float = 1e-8, clip: float = 0.0,
-                 warmup: bool = True, pipelined: bool = True, device=None):
+                 warmup: bool = True, pipelined: bool = True, rule: str = "scaled", device=None):
         from . import _lib as L
         self.L = L
         self.device = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
         self.layout, self.rank = layout, rank
-        W, n, C = layout.world, layout.n, layout.C
+        W, n = layout.world, layout.n
+        momentum = rule == "momentum"
+        if layout.codes_per_word != (4 if momentum else 32):
+            raise ValueError(f"layout planned with {layout.codes_per_word} codes per word for rule {rule!r}")
+        # The momentum-error rule has no scales and no server error: those are empty.
+        C = 0 if momentum else layout.C
+        code_rule = L.OB_RULE_MOMENTUM_ERROR if momentum else L.OB_RULE_SCALED_SIGN
         gd = L.OB_BF16 if grad_dtype == "bf16" else L.OB_F32
         opt = L.OB_LAMB if optimizer == "lamb" else L.OB_ADAM
         hp = dict(lr=lr, beta1=beta1, beta2=beta2, eps=eps, clip=clip)
@@ -148,7 +160,8 @@ class CudaStages:
         self._keep = []
 
         def cfg(offsets, workers, freeze):
-            c, arr = L.make_config(int(offsets[-1]), offsets, workers, gd, opt, freeze_step=freeze, **hp)
+            c, arr = L.make_config(int(offsets[-1]), offsets, workers, gd, opt, freeze_step=freeze,
+                                   rule=code_rule, **hp)
             self._keep.append(arr)
             return c
 
@@ -160,9 +173,10 @@ class CudaStages:
             off_own = layout.offsets[ks.start: ks.stop + 1] - layout.offsets[ks.start]
             self.n_own, self.C_own = int(off_own[-1]), ks.stop - ks.start
             w_own = layout.wslice(rank).stop - layout.wslice(rank).start
-            self.srv_err = z(self.n_own)
-            self.bits_w_srv, self.s_w_srv = z((W, w_own), i32), z((W, self.C_own))
-            self.bits_srv_own, self.s_srv_own = z(w_own, i32), z(self.C_own)
+            self.srv_err = z(0 if momentum else self.n_own)
+            C_own_scales = 0 if momentum else self.C_own
+            self.bits_w_srv, self.s_w_srv = z((W, w_own), i32), z((W, C_own_scales))
+            self.bits_srv_own, self.s_srv_own = z(w_own, i32), z(C_own_scales)
             self.server = 0
             if self.C_own > 0:
                 self.server = L.ob_create(cfg(off_own, W, 0), 0, 0, 0, 0, ptr(self.srv_err),
@@ -185,10 +199,11 @@ class CudaStages:
                         continue
                     so = layout.offsets[ks.start: ks.stop + 1] - es.start
                     e4, w4, k4 = 4 * es.start, 4 * ws.start, 4 * ks.start
+                    at = lambda t, b: ptr(t) + b if t.numel() else 0  # noqa: E731
                     self.slice_ctx.append(L.ob_create(
-                        cfg(so, 1, 0), ptr(self.p) + e4, ptr(self.m) + e4, ptr(self.v) + e4,
-                        ptr(self.err) + e4, 0, ptr(self.bits_w) + w4, ptr(self.s_w) + k4,
-                        ptr(self.bits_srv) + w4, ptr(self.s_srv) + k4))
+                        cfg(so, 1, 0), at(self.p, e4), at(self.m, e4), at(self.v, e4),
+                        at(self.err, e4), 0, at(self.bits_w, w4), at(self.s_w, k4),
+                        at(self.bits_srv, w4), at(self.s_srv, k4)))
 
     def _stream(self) -> int:
         return int(torch.cuda.current_stream(self.device).cuda_stream)

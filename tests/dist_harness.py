@@ -26,14 +26,16 @@ class OracleStages:
     """``pipelined``: also offer the per-owner-slice stages (compress_slice,
     apply_slice), so the driver takes its overlapped schedule."""
 
-    def __init__(self, layout, rank, optimizer="adam", clip=0.0, pipelined=False):
+    def __init__(self, layout, rank, optimizer="adam", clip=0.0, pipelined=False, rule="scaled"):
         import oracle
         self.o = oracle.get()
         self.layout, self.rank = layout, rank
         self.opt = oracle.LAMB if optimizer == "lamb" else oracle.ADAM
         self.clip = clip
         self.device = torch.device("cpu")
-        W, n, C = layout.world, layout.n, layout.C
+        self.momentum = rule == "momentum"
+        W, n = layout.world, layout.n
+        C = 0 if self.momentum else layout.C
         words = int(layout.words[-1])
         f32, i32 = torch.float32, torch.int32
         self.p, self.m, self.v = torch.zeros(n), torch.zeros(n), torch.zeros(n)
@@ -42,11 +44,12 @@ class OracleStages:
         self.bits_srv, self.s_srv = torch.zeros(words, dtype=i32), torch.zeros(C)
         ks, wsl = layout.kslice(rank), layout.wslice(rank)
         self.off_own = layout.offsets[ks.start: ks.stop + 1] - layout.offsets[ks.start]
-        self.srv_err = torch.zeros(int(self.off_own[-1]))
+        c_own = 0 if self.momentum else ks.stop - ks.start
+        self.srv_err = torch.zeros(0 if self.momentum else int(self.off_own[-1]))
         self.bits_w_srv = torch.zeros((W, wsl.stop - wsl.start), dtype=i32)
-        self.s_w_srv = torch.zeros((W, ks.stop - ks.start), dtype=f32)
+        self.s_w_srv = torch.zeros((W, c_own), dtype=f32)
         self.bits_srv_own = torch.zeros(wsl.stop - wsl.start, dtype=i32)
-        self.s_srv_own = torch.zeros(ks.stop - ks.start, dtype=f32)
+        self.s_srv_own = torch.zeros(c_own, dtype=f32)
         self.flags = 0
         self.pipelined = bool(pipelined) and layout.world > 1
 
@@ -67,6 +70,12 @@ class OracleStages:
         return np.ascontiguousarray(grad.numpy().reshape(1, -1))
 
     def compress(self, grad):
+        if self.momentum:
+            codes, fl = self.o.ternary_compress(self.layout.offsets, self._grad_rows(grad), self.err.numpy(),
+                                                np.float32(HP["beta1"]), clip=self.clip)
+            self.bits_w.numpy().view(np.int8)[:] = codes
+            self.flags |= fl
+            return
         bits, s, fl = self.o.compress(self.layout.offsets, self._grad_rows(grad), self.err.numpy(),
                                       clip=self.clip)
         self._u32(self.bits_w)[:] = bits
@@ -83,6 +92,12 @@ class OracleStages:
         if ks.stop == ks.start:
             return
         err = self.err.numpy()[0, es].reshape(1, -1)
+        if self.momentum:
+            codes, fl = self.o.ternary_compress(self._slice_offsets(o), self._grad_rows(grad_slice), err,
+                                                np.float32(HP["beta1"]), clip=self.clip)
+            self.bits_w.numpy().view(np.int8)[0, 4 * wsl.start: 4 * wsl.stop] = codes[0]
+            self.flags |= fl
+            return
         bits, s, fl = self.o.compress(self._slice_offsets(o), self._grad_rows(grad_slice), err,
                                       clip=self.clip)
         self._u32(self.bits_w)[0, wsl] = bits[0]
@@ -90,6 +105,11 @@ class OracleStages:
         self.flags |= fl
 
     def server_reduce(self):
+        if self.momentum:
+            if self.bits_w_srv.shape[1]:
+                sums = self.o.ternary_server(self.off_own, np.ascontiguousarray(self.bits_w_srv.numpy().view(np.int8)))
+                self.bits_srv_own.numpy().view(np.int8)[:] = sums
+            return
         if self.s_w_srv.shape[1] == 0:
             return
         bits, s, fl = self.o.server_reduce(self.off_own, np.ascontiguousarray(self._u32(self.bits_w_srv)),
@@ -100,6 +120,12 @@ class OracleStages:
 
     def apply(self):
         f = {k: np.float32(v) for k, v in HP.items()}
+        if self.momentum:
+            self.flags |= self.o.ternary_apply(self.layout.offsets, self.layout.world,
+                                               self.bits_srv.numpy().view(np.int8), self.m.numpy(),
+                                               self.v.numpy(), self.p.numpy(), f["beta1"], f["lr"], f["eps"],
+                                               optimizer=self.opt)[1]
+            return
         args = (self.layout.offsets, self._u32(self.bits_srv), self.s_srv.numpy(), self.m.numpy(),
                 self.v.numpy(), self.p.numpy(), f["beta1"], f["lr"], f["eps"])
         if self.opt:
@@ -113,6 +139,12 @@ class OracleStages:
         if ks.stop == ks.start:
             return
         f = {k: np.float32(v) for k, v in HP.items()}
+        if self.momentum:
+            sums = np.ascontiguousarray(self.bits_srv.numpy().view(np.int8)[4 * wsl.start: 4 * wsl.stop])
+            self.flags |= self.o.ternary_apply(self._slice_offsets(o), L.world, sums, self.m.numpy()[es],
+                                               self.v.numpy()[es], self.p.numpy()[es], f["beta1"], f["lr"],
+                                               f["eps"], optimizer=self.opt)[1]
+            return
         args = (self._slice_offsets(o), self._u32(self.bits_srv)[wsl], self.s_srv.numpy()[ks],
                 self.m.numpy()[es], self.v.numpy()[es], self.p.numpy()[es], f["beta1"], f["lr"], f["eps"])
         if self.opt:
@@ -148,7 +180,7 @@ def initial_state(wl, layout):
 
 
 def _rank_main(rank, world, port, sizes, wl_kw, steps, backend, device, q, die=None, timeout_s=120,
-               pipelined=False):
+               pipelined=False, rule="scaled"):
     try:
         import sys
         sys.path.insert(0, ROOT)
@@ -162,14 +194,15 @@ def _rank_main(rank, world, port, sizes, wl_kw, steps, backend, device, q, die=N
         dist.init_process_group(backend, rank=rank, world_size=world,
                                 timeout=datetime.timedelta(seconds=timeout_s))
         wl = workload(sizes, world, **wl_kw)
-        layout = plan(sizes, world)
+        layout = plan(sizes, world, 4 if rule == "momentum" else 32)
         if device == "cpu":
-            stages = OracleStages(layout, rank, optimizer=wl.optimizer, clip=wl.clip, pipelined=pipelined)
+            stages = OracleStages(layout, rank, optimizer=wl.optimizer, clip=wl.clip, pipelined=pipelined,
+                                  rule=rule)
         else:
             from bit_adam_error_b200.distributed import CudaStages
             stages = CudaStages(layout, rank, grad_dtype=wl.grad_dtype, optimizer=wl.optimizer,
                                 clip=wl.clip, warmup=wl.freeze_step > 0, pipelined=pipelined,
-                                device=device, **HP)
+                                rule=rule, device=device, **HP)
         p0, v0 = initial_state(wl, layout)
         stages.p.copy_(torch.from_numpy(p0))
         stages.v.copy_(torch.from_numpy(v0))
@@ -201,14 +234,15 @@ def _rank_main(rank, world, port, sizes, wl_kw, steps, backend, device, q, die=N
         q.put((rank, {"error": traceback.format_exc()}))
 
 
-def run_ranks(sizes, world, wl_kw, steps, backend="gloo", device="cpu", timeout=600, pipelined=False):
+def run_ranks(sizes, world, wl_kw, steps, backend="gloo", device="cpu", timeout=600, pipelined=False,
+              rule="scaled"):
     """Spawn `world` ranks; returns the list of per-rank final states."""
     import multiprocessing as mp
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = free_port()
     procs = [ctx.Process(target=_rank_main, args=(r, world, port, sizes, wl_kw, steps, backend, device, q),
-                         kwargs=dict(pipelined=pipelined)) for r in range(world)]
+                         kwargs=dict(pipelined=pipelined, rule=rule)) for r in range(world)]
     for pr in procs:
         pr.start()
     results = {}
@@ -226,7 +260,7 @@ def run_ranks(sizes, world, wl_kw, steps, backend="gloo", device="cpu", timeout=
     return [results[r] for r in range(world)]
 
 
-def reference(sizes, world, wl_kw, steps):
+def reference(sizes, world, wl_kw, steps, rule="scaled"):
     """The same workload as one W-worker oracle problem (caller's chunk order)."""
     import oracle
     import workloads as WL
@@ -247,6 +281,8 @@ def reference(sizes, world, wl_kw, steps):
         if t < wl.freeze_step:
             o.warmup(wl.offsets, g, st["m"], st["v"], st["p"], f["beta1"], f["beta2"], f["lr"], f["eps"],
                      optimizer=opt)
+        elif rule == "momentum":
+            o.ternary_step(wl.offsets, g, st, f["beta1"], f["lr"], f["eps"], clip=wl.clip, optimizer=opt)
         else:
             o.step(wl.offsets, g, st, f["beta1"], f["lr"], f["eps"], clip=wl.clip, optimizer=opt)
     return wl, st
@@ -261,11 +297,12 @@ def compare(layout, wl, ref, outs, exact=True):
         return layout.to_layout([a[..., off[k]:off[k + 1]] for k in range(wl.C)]) if a.ndim == 1 else \
             np.stack([lay(r) for r in a])
 
-    wb = np.zeros(wl.C + 1, np.int64)
-    np.cumsum([(s + 31) // 32 for s in wl.sizes], out=wb[1:])
-    bits_ref = layout.to_layout([ref["bits_srv"][wb[k]:wb[k + 1]] for k in range(wl.C)]).astype(np.uint32)
-    s_ref = np.array([ref["s_srv"][k] for k in layout.order], np.float32)
-    srv_ref = lay(ref["srv_err"])
+    if "bits_srv" in ref:          # the scaled-sign rule: server words, scales, server error
+        wb = np.zeros(wl.C + 1, np.int64)
+        np.cumsum([(s + 31) // 32 for s in wl.sizes], out=wb[1:])
+        bits_ref = layout.to_layout([ref["bits_srv"][wb[k]:wb[k + 1]] for k in range(wl.C)]).astype(np.uint32)
+        s_ref = np.array([ref["s_srv"][k] for k in layout.order], np.float32)
+        srv_ref = lay(ref["srv_err"])
     if exact:
         same = lambda name, got, want: np.testing.assert_array_equal(got, want, err_msg=name)  # noqa: E731
         scales = same
@@ -277,6 +314,11 @@ def compare(layout, wl, ref, outs, exact=True):
         for key in ("p", "m", "v"):
             same(f"rank {r} {key}", out[key], lay(ref[key]))
         same(f"rank {r} err", out["err"][0], lay(ref["err"][r]))
+        if "codes_srv" in ref:        # momentum-error rule: the code sums, byte for byte
+            cb = np.zeros(wl.C + 1, np.int64)
+            np.cumsum([(s + 3) // 4 for s in wl.sizes], out=cb[1:])
+            want = layout.to_layout([ref["codes_srv"][4 * cb[k]: 4 * cb[k + 1]] for k in range(wl.C)])
+            assert np.array_equal(out["bits_srv"].view(np.int8), want.astype(np.int8)), (r, "code sums")
         if "bits_w" in ref:
             assert np.array_equal(out["bits_srv"], bits_ref), (r, "bits_srv")
             scales(f"rank {r} s_srv", out["s_srv"], s_ref)

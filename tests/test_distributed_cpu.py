@@ -65,3 +65,25 @@ def test_a_dead_rank_ends_the_others_step_with_an_error():
     assert codes[1] == 17
     assert "error" in results[0], "the surviving rank finished instead of reporting the lost peer"
     assert time.monotonic() - t0 < 120
+
+
+@pytest.mark.parametrize("pipelined", [False, True], ids=["grouped", "pipelined"])
+@pytest.mark.parametrize("world,wl_kw,steps", [
+    (2, dict(freeze_step=1), 3),
+    (3, dict(grad_dtype="bf16", clip=5.0, grad_dist="student_t_zeros", zero_frac=0.05), 3),
+    (3, dict(optimizer="lamb"), 2),
+])
+def test_momentum_rule_ranks_match_single_process_oracle(world, wl_kw, steps, pipelined):
+    """The momentum-error rule across ranks: int8 codes to the owners, code sums
+    back; every rank equals the W-worker oracle bit for bit."""
+    outs = run_ranks(SIZES, world, wl_kw, steps, pipelined=pipelined, rule="momentum")
+    wl, ref = reference(SIZES, world, wl_kw, steps, rule="momentum")
+    compare(plan(SIZES, world, 4), wl, ref, outs)
+    assert all(o["flags"] == 0 for o in outs)
+
+
+def test_plan_code_words():
+    lay = plan(SIZES, 3, 4)
+    assert int(lay.words[-1]) == sum((s + 3) // 4 for s in SIZES)
+    with pytest.raises(ValueError):
+        plan(SIZES, 2, 8)
