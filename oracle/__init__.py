@@ -60,6 +60,12 @@ _SIGS = {
     "orc_ternary_apply": (_U32, [_I64, _I32, _P, _I32, _P, _I32, _F, _F, _F, _P, _P, _P, _P]),
     "orc_ternary_step": (_U32, [_I32, _I64, _I32, _P, _P, _I32, _I32, _F, _F, _F, _F,
                                 _P, _P, _P, _P, _I32, _P, _P]),
+    "orc_words2_total": (_I64, [_I32, _P]),
+    "orc_twobit_compress": (_U32, [_I32, _I64, _I32, _P, _P, _I32, _F, _P, _I32, _P, _P]),
+    "orc_twobit_server": (_U32, [_I32, _I64, _I32, _P, _P, _P, _P, _I32, _P, _P]),
+    "orc_twobit_apply": (_U32, [_I64, _I32, _P, _P, _P, _I32, _F, _F, _F, _P, _P, _P, _P]),
+    "orc_twobit_step": (_U32, [_I32, _I64, _I32, _P, _P, _I32, _I32, _F, _F, _F, _F,
+                               _P, _P, _P, _P, _P, _I32, _P, _P, _P, _P]),
 }
 
 MAX_TERNARY_WORKERS = 127   # the int8 sum of W codes in {-1, 0, 1} is exact up to here
@@ -240,6 +246,69 @@ class Oracle:
             float(clip), beta1, lr, eps, self._ptr(state["p"]), self._ptr(state["m"]),
             self._ptr(state["v"]), self._ptr(state["err"]), self._err_dtype(state["err"]),
             self._ptr(state["codes_w"]), self._ptr(state["codes_srv"])))
+
+    # -- 2-bit Adam (two residual sign planes) ---------------------------------------
+    def words2_total(self, offsets) -> int:
+        off = self._off(offsets)
+        return int(self.lib.orc_words2_total(len(off) - 1, self._ptr(off)))
+
+    def twobit_compress(self, offsets, grads: np.ndarray, err: np.ndarray, clip: float = 0.0
+                        ) -> Tuple[np.ndarray, np.ndarray, int]:
+        """Worker stage.  Returns (bits_w [W, words2], s_w [W, C, 2], flags); err in place."""
+        off = self._off(offsets)
+        W, n = grads.shape
+        C = len(off) - 1
+        bits_w = np.zeros((W, self.words2_total(off)), np.uint32)
+        s_w = np.zeros((W, C, 2), np.float32)
+        flags = self.lib.orc_twobit_compress(W, n, C, self._ptr(off), self._ptr(grads),
+                                             self._dtype_of(grads), float(clip), self._ptr(err),
+                                             self._err_dtype(err), self._ptr(bits_w), self._ptr(s_w))
+        return bits_w, s_w, int(flags)
+
+    def twobit_server(self, offsets, bits_w: np.ndarray, s_w: np.ndarray, srv_err: np.ndarray
+                      ) -> Tuple[np.ndarray, np.ndarray, int]:
+        """Server stage.  Returns (bits_srv [words2], s_srv [C, 2], flags); srv_err in place."""
+        off = self._off(offsets)
+        W = bits_w.shape[0]
+        C = len(off) - 1
+        bits_srv = np.zeros(self.words2_total(off), np.uint32)
+        s_srv = np.zeros((C, 2), np.float32)
+        flags = self.lib.orc_twobit_server(W, int(off[-1]), C, self._ptr(off),
+                                           self._ptr(np.ascontiguousarray(bits_w, np.uint32)),
+                                           self._ptr(np.ascontiguousarray(s_w, np.float32)),
+                                           self._ptr(srv_err), self._err_dtype(srv_err),
+                                           self._ptr(bits_srv), self._ptr(s_srv))
+        return bits_srv, s_srv, int(flags)
+
+    def twobit_apply(self, offsets, bits_srv, s_srv, m, v, p, beta1, lr, eps, optimizer=ADAM
+                     ) -> Tuple[np.ndarray, int]:
+        off = self._off(offsets)
+        r = np.zeros(len(off) - 1, np.float32)
+        flags = self.lib.orc_twobit_apply(int(off[-1]), len(off) - 1, self._ptr(off),
+                                          self._ptr(np.ascontiguousarray(bits_srv, np.uint32)),
+                                          self._ptr(np.ascontiguousarray(s_srv, np.float32)), optimizer,
+                                          beta1, lr, eps, self._ptr(m), self._ptr(v), self._ptr(p),
+                                          self._ptr(r))
+        return r, int(flags)
+
+    def twobit_step(self, offsets, grads, state: dict, beta1, lr, eps, clip=0.0, optimizer=ADAM) -> int:
+        """One compressed step of 2-bit Adam; ``state`` as for ``step`` (bits_w,
+        s_w [W, C, 2], bits_srv, s_srv [C, 2] are (re)allocated when missing)."""
+        off = self._off(offsets)
+        W, n = grads.shape
+        C = len(off) - 1
+        words = self.words2_total(off)
+        for key, shape, dt in (("bits_w", (W, words), np.uint32), ("s_w", (W, C, 2), np.float32),
+                               ("bits_srv", (words,), np.uint32), ("s_srv", (C, 2), np.float32)):
+            if key not in state or state[key].shape != shape:
+                state[key] = np.zeros(shape, dt)
+        return int(self.lib.orc_twobit_step(
+            W, n, C, self._ptr(off), self._ptr(grads), self._dtype_of(grads), optimizer,
+            float(clip), beta1, lr, eps, self._ptr(state["p"]), self._ptr(state["m"]),
+            self._ptr(state["v"]), self._ptr(state["err"]), self._ptr(state["srv_err"]),
+            self._err_dtype(state["err"]),
+            self._ptr(state["bits_w"]), self._ptr(state["s_w"]), self._ptr(state["bits_srv"]),
+            self._ptr(state["s_srv"])))
 
 
 _default: Optional[Oracle] = None

@@ -46,6 +46,10 @@
  *    compression survey page suggests half-precision error storage): each
  *    stored error is the float32 result rounded to nearest-even bfloat16.
  *
+ * Two more compression rules follow the main one, each under its own heading
+ * with its passages and readings: the CANN article's momentum-error rule
+ * (int8 ternary codes) and 2-bit Adam (two residual sign planes).
+ *
  * Parity pins: every function here is checked by tests/test_oracle_pins.py
  * against hand-worked cases, closed forms, invariants and brute force.
  *
@@ -500,5 +504,145 @@ uint32_t orc_ternary_step(int32_t W, int64_t n, int32_t C, const int64_t* off,
                                         codes_w);
   flags |= orc_ternary_server(W, C, off, codes_w, codes_srv);
   flags |= orc_ternary_apply(n, C, off, W, codes_srv, optimizer, beta1, lr, eps, m, v, p, NULL);
+  return flags;
+}
+
+/* ---- 2-bit Adam ----------------------------------------------------------------------
+ *
+ * The CANN 1-bit Adam article names 2-bit Adam (section 5.1, table: 6.25% of the
+ * traffic; section 8: weaker compression for embedding layers) but gives no
+ * quantiser.  Reading: the 1-bit quantiser of this file applied twice, the
+ * second time to what the first left over -- two sign planes with one scale
+ * each, 2 bits per element plus 2 scales per chunk:
+ *   (q1, s1) = one_bit_quantize(c),        r   = c - dequantize(q1, s1)
+ *   (q2, s2) = one_bit_quantize(r),        err = r - dequantize(q2, s2)
+ *   dequantized value = dequantize(q1, s1) + dequantize(q2, s2)   (float add)
+ * Workers and server use it in place of one_bit_quantize; everything else
+ * (error feedback, server average and error, update) is unchanged.
+ * Layout: chunk k owns 2 ceil(n_k / 32) words of a row -- plane 1, then plane
+ * 2 -- starting on a fresh word; scales are [..][C][2] (plane 1, plane 2).
+ */
+
+static int64_t words2_of(int64_t n) { return 2 * words_of(n); }
+
+int64_t orc_words2_total(int32_t C, const int64_t* off) {
+  int64_t t = 0;
+  for (int32_t k = 0; k < C; ++k) t += words2_of(off[k + 1] - off[k]);
+  return t;
+}
+
+/* Two planes of c: words[0 .. 2 nw), s[0..1]; resid (may alias nothing) gets
+ * the final residual r - dequantize(q2, s2). */
+static void two_bit_quantize(const float* c, int64_t nk, uint32_t* words, float* s, float* r,
+                             float* resid) {
+  const int64_t nw = words_of(nk);
+  s[0] = quantize_scale(c, nk);
+  quantize_signs(c, nk, words);
+  for (int64_t i = 0; i < nk; ++i) r[i] = c[i] - dequantize(words, s[0], i);
+  s[1] = quantize_scale(r, nk);
+  quantize_signs(r, nk, words + nw);
+  for (int64_t i = 0; i < nk; ++i) resid[i] = r[i] - dequantize(words + nw, s[1], i);
+}
+
+static float dequantize2(const uint32_t* words, int64_t nw, const float* s, int64_t i) {
+  return dequantize(words, s[0], i) + dequantize(words + nw, s[1], i);
+}
+
+/* Worker stage of 2-bit Adam.  bits_w: [W][words2_total]; s_w: [W][C][2]. */
+uint32_t orc_twobit_compress(int32_t W, int64_t n, int32_t C, const int64_t* off,
+                             const void* grads, int32_t dtype, float clip, void* err,
+                             int32_t err_dtype, uint32_t* bits_w, float* s_w) {
+  uint32_t flags = 0;
+  int64_t* wo = (int64_t*)malloc(sizeof(int64_t) * (size_t)(C + 1));
+  wo[0] = 0;
+  for (int32_t k = 0; k < C; ++k) wo[k + 1] = wo[k] + words2_of(off[k + 1] - off[k]);
+  for (int32_t k = 0; k < C; ++k) {
+    int64_t o = off[k], nk = off[k + 1] - off[k];
+    size_t bytes = sizeof(float) * (size_t)(nk > 0 ? nk : 1);
+    float *c = (float*)malloc(bytes), *r = (float*)malloc(bytes), *e = (float*)malloc(bytes);
+    for (int32_t w = 0; w < W; ++w) {
+      const int64_t e0 = (int64_t)w * n + o;
+      for (int64_t i = 0; i < nk; ++i) {
+        c[i] = clip_grad(grad_at(grads, dtype, e0 + i), clip) + err_get(err, err_dtype, e0 + i);
+        if (is_nonfinite(c[i])) flags |= ORC_STATUS_NONFINITE;
+      }
+      two_bit_quantize(c, nk, bits_w + (int64_t)w * wo[C] + wo[k], s_w + ((int64_t)w * C + k) * 2, r, e);
+      for (int64_t i = 0; i < nk; ++i) err_set(err, err_dtype, e0 + i, e[i]);
+    }
+    free(c); free(r); free(e);
+  }
+  free(wo);
+  return flags;
+}
+
+/* Server stage of 2-bit Adam: c_srv = mean_w(dequantized worker w) + srv_err,
+ * quantised to two planes; srv_err keeps the residual. */
+uint32_t orc_twobit_server(int32_t W, int64_t n, int32_t C, const int64_t* off,
+                           const uint32_t* bits_w, const float* s_w, void* srv_err,
+                           int32_t err_dtype, uint32_t* bits_srv, float* s_srv) {
+  (void)n;
+  uint32_t flags = 0;
+  int64_t* wo = (int64_t*)malloc(sizeof(int64_t) * (size_t)(C + 1));
+  wo[0] = 0;
+  for (int32_t k = 0; k < C; ++k) wo[k + 1] = wo[k] + words2_of(off[k + 1] - off[k]);
+  for (int32_t k = 0; k < C; ++k) {
+    int64_t o = off[k], nk = off[k + 1] - off[k], nw = words_of(nk);
+    size_t bytes = sizeof(float) * (size_t)(nk > 0 ? nk : 1);
+    float *c = (float*)malloc(bytes), *r = (float*)malloc(bytes), *e = (float*)malloc(bytes);
+    for (int64_t i = 0; i < nk; ++i) {
+      float acc = 0.0f;
+      for (int32_t w = 0; w < W; ++w)
+        acc += dequantize2(bits_w + (int64_t)w * wo[C] + wo[k], nw, s_w + ((int64_t)w * C + k) * 2, i);
+      float avg = acc / (float)W;
+      c[i] = avg + err_get(srv_err, err_dtype, o + i);
+      if (is_nonfinite(c[i])) flags |= ORC_STATUS_NONFINITE;
+    }
+    two_bit_quantize(c, nk, bits_srv + wo[k], s_srv + 2 * k, r, e);
+    for (int64_t i = 0; i < nk; ++i) err_set(srv_err, err_dtype, o + i, e[i]);
+    free(c); free(r); free(e);
+  }
+  free(wo);
+  return flags;
+}
+
+/* Update of 2-bit Adam: g_hat = dequantized server planes; m and p as
+ * orc_adam_apply (ORC_ADAM) or orc_lamb_apply (ORC_LAMB; r_out may be NULL). */
+uint32_t orc_twobit_apply(int64_t n, int32_t C, const int64_t* off, const uint32_t* bits_srv,
+                          const float* s_srv, int32_t optimizer, float beta1, float lr, float eps,
+                          float* m, const float* v, float* p, float* r_out) {
+  (void)n;
+  uint32_t flags = 0;
+  const float one_minus_b1 = 1.0f - beta1;
+  int64_t wo = 0;
+  for (int32_t k = 0; k < C; ++k) {
+    int64_t o = off[k], nk = off[k + 1] - off[k], nw = words_of(nk);
+    for (int64_t i = 0; i < nk; ++i) {
+      float g_hat = dequantize2(bits_srv + wo, nw, s_srv + 2 * k, i);
+      float mi = beta1 * m[o + i] + one_minus_b1 * g_hat;
+      m[o + i] = mi;
+      if (optimizer == ORC_ADAM) {
+        float pi = p[o + i] - lr * mi / (sqrtf(v[o + i]) + eps);
+        if (is_nonfinite(pi)) flags |= ORC_STATUS_NONFINITE;
+        p[o + i] = pi;
+      }
+    }
+    if (optimizer == ORC_LAMB) {
+      if (r_out) r_out[k] = trust_ratio(p + o, m + o, v + o, eps, nk);
+      flags |= lamb_update_layer(p + o, m + o, v + o, lr, eps, nk);
+    }
+    wo += 2 * nw;
+  }
+  return flags;
+}
+
+/* One whole compressed-phase step of 2-bit Adam. */
+uint32_t orc_twobit_step(int32_t W, int64_t n, int32_t C, const int64_t* off,
+                         const void* grads, int32_t dtype, int32_t optimizer, float clip,
+                         float beta1, float lr, float eps, float* p, float* m, const float* v,
+                         void* err, void* srv_err, int32_t err_dtype, uint32_t* bits_w, float* s_w,
+                         uint32_t* bits_srv, float* s_srv) {
+  uint32_t flags = orc_twobit_compress(W, n, C, off, grads, dtype, clip, err, err_dtype, bits_w, s_w);
+  flags |= orc_twobit_server(W, n, C, off, bits_w, s_w, srv_err, err_dtype, bits_srv, s_srv);
+  flags |= orc_twobit_apply(n, C, off, bits_srv, s_srv, optimizer, beta1, lr, eps, m, v, p, NULL);
   return flags;
 }

@@ -754,4 +754,185 @@ def pin_ternary_bf16(o):
     assert np.array_equal(eb, _bf16_of(e32))
 
 
+
+
+# -- 2-bit Adam (two residual sign planes) ----------------------------------------------
+
+def _twobit_case_c(case):
+    if "c" in case:
+        return np.array(case["c"], np.float32)
+    return np.array([(-1) ** i * 3.0 for i in range(33)] + [2, -2, 2, -2], np.float32)
+
+
+def pin_twobit_hand_cases(o):
+    doc = json.load(open(os.path.join(GOLDEN, "twobit_hand_cases.json")))
+    for case in doc["cases"]:
+        c = _twobit_case_c(case)
+        sizes = case["sizes"]
+        g = c[None, :].copy()
+        err = np.zeros_like(g)
+        bits, s, flags = o.twobit_compress(offsets_of(sizes), g, err)
+        assert [int(x) for x in bits[0]] == [int(w, 16) for w in case["words"]], (case["name"], bits)
+        s1sq = case["s1_squared"] if isinstance(case["s1_squared"], list) else [case["s1_squared"]]
+        s2sq = case["s2_squared"] if isinstance(case["s2_squared"], list) else [case["s2_squared"]]
+        for k in range(len(sizes)):
+            for plane, sq in ((0, s1sq[k]), (1, s2sq[k])):
+                want = math.sqrt(float(Fraction(sq)))
+                assert abs(float(s[0, k, plane]) - want) <= ulp32(want), (case["name"], k, plane)
+        if "r" in case:
+            r = np.array(case["r"], np.float64)
+            sign2 = np.where(r >= 0, 1.0, -1.0)
+            want_err = r - float(s[0, 0, 1]) * sign2
+            assert np.all(np.abs(err[0] - want_err) <= 0.5 * ulp32(err[0])), case["name"]
+        assert flags == 0
+
+
+def pin_twobit_is_one_bit_twice(o):
+    """Plane 1 and s1 are the 1-bit stage of c; plane 2, s2 and the error are the
+    1-bit stage of the 1-bit residual (with a zero error buffer) -- bit for bit."""
+    sizes = RAGGED
+    off, wb = offsets_of(sizes), word_base(sizes)
+    for W, clip in ((1, 0.0), (3, 0.0), (2, 2e-3)):
+        g, err = _worker_inputs(W, sizes, (160, W))
+        e2 = err.copy()
+        bits2, s2, f2 = o.twobit_compress(off, g, e2, clip=clip)
+        e1 = err.copy()
+        b1, s1, _ = o.compress(off, g, e1, clip=clip)
+        zero = np.zeros_like(e1)
+        b1b, s1b, _ = o.compress(off, e1.copy(), zero)
+        for w in range(W):
+            for k, nk in enumerate(sizes):
+                nw = wb[k + 1] - wb[k]
+                base = 2 * wb[k]
+                assert np.array_equal(bits2[w, base: base + nw], b1[w, wb[k]: wb[k + 1]]), (W, k, 1)
+                assert np.array_equal(bits2[w, base + nw: base + 2 * nw], b1b[w, wb[k]: wb[k + 1]]), (W, k, 2)
+        assert np.array_equal(s2[:, :, 0], s1) and np.array_equal(s2[:, :, 1], s1b)
+        assert np.array_equal(e2, zero), W
+        assert f2 == 0
+
+
+def pin_twobit_residual_norm_identity(o):
+    """sum r^2 = sum c^2 - 2 s1 sum |c| + n s1^2 for r = c - s1 sign(c): the second
+    scale agrees with the closed form of the first plane's residual norm."""
+    sizes = [40, 64, 257, 1000]
+    off = offsets_of(sizes)
+    g, err = _worker_inputs(2, sizes, (170,))
+    c = (g + err).astype(np.float64)
+    _, s, _ = o.twobit_compress(off, g, err.copy())
+    for w in range(2):
+        for k, nk in enumerate(sizes):
+            ck = c[w, off[k]: off[k + 1]]
+            s1 = float(s[w, k, 0])
+            r2 = (ck ** 2).sum() - 2 * s1 * np.abs(ck).sum() + nk * s1 * s1
+            assert abs(float(s[w, k, 1]) - math.sqrt(r2 / nk)) <= 1e-5 * math.sqrt(r2 / nk), (w, k)
+
+
+def _ghat2(bits, s, sizes):
+    wb = word_base(sizes)
+    out = []
+    for k, nk in enumerate(sizes):
+        nw = wb[k + 1] - wb[k]
+        base = 2 * wb[k]
+        p1 = np.where(unpack_ref(bits[base: base + nw], nk), 1.0, -1.0)
+        p2 = np.where(unpack_ref(bits[base + nw: base + 2 * nw], nk), 1.0, -1.0)
+        out.append(float(s[k, 0]) * p1 + float(s[k, 1]) * p2)
+    return np.concatenate(out)
+
+
+def pin_twobit_error_feedback_telescopes(o):
+    """With two planes the two-level error feedback still telescopes:
+    sum_t g_hat_t = mean_w(sum_t g_w,t - err_w,T) - srv_err_T."""
+    W, T, sizes = 3, 6, [50, 64, 33]
+    off = offsets_of(sizes)
+    n = int(off[-1])
+    st = {"p": aux_normal(SEED, (180,), n, 0.02), "m": np.zeros(n, np.float32),
+          "v": aux_uniform(SEED, (181,), n, 1e-8, 1e-6),
+          "err": np.zeros((W, n), np.float32), "srv_err": np.zeros(n, np.float32)}
+    gsum = np.zeros((W, n))
+    ghat_sum = np.zeros(n)
+    for t in range(T):
+        g = aux_normal(SEED, (182, t), W * n, 1e-3).reshape(W, n)
+        gsum += g
+        o.twobit_step(off, g, st, B1, LR, EPS)
+        ghat_sum += _ghat2(st["bits_srv"], st["s_srv"], sizes)
+    want = (gsum - st["err"]).mean(0) - st["srv_err"]
+    assert np.max(np.abs(ghat_sum - want)) <= 1e-8, np.max(np.abs(ghat_sum - want))
+
+
+def pin_twobit_server_special_cases(o):
+    """Opposite workers cancel exactly, so the server quantises its own error
+    (= the worker stage applied to srv_err); two identical workers equal one."""
+    sizes = [40, 33, 64]
+    off = offsets_of(sizes)
+    n = int(off[-1])
+    g, err = _worker_inputs(1, sizes, (190,))
+    bits, s, _ = o.twobit_compress(off, g, err)
+    bits_neg = ~bits
+    srv0 = aux_normal(SEED, (191,), n, 1e-3)
+    wb = word_base(sizes)
+    for k, nk in enumerate(sizes):            # padding bits stay 0 in the negated message
+        for base in (2 * wb[k], 2 * wb[k] + (wb[k + 1] - wb[k])):
+            nw = wb[k + 1] - wb[k]
+            bits_neg[0, base: base + nw] &= pack_ref(np.ones(nk, bool))
+    srv = srv0.copy()
+    b_s, s_s, _ = o.twobit_server(off, np.concatenate([bits, bits_neg]), np.concatenate([s, s]), srv)
+    e = np.zeros((1, n), np.float32)
+    b_ref, s_ref, _ = o.twobit_compress(off, srv0[None, :].copy(), e)
+    assert np.array_equal(b_s, b_ref[0]) and np.array_equal(s_s, s_ref[0]) and np.array_equal(srv, e[0])
+    one = srv0.copy()
+    two = srv0.copy()
+    b1, s1, _ = o.twobit_server(off, bits, s, one)
+    b2, s2, _ = o.twobit_server(off, np.concatenate([bits, bits]), np.concatenate([s, s]), two)
+    assert np.array_equal(b1, b2) and np.array_equal(s1, s2) and np.array_equal(one, two)
+
+
+def pin_twobit_adam_closed_form(o):
+    """Constant server planes: m_t = (1 - b1^t) g_hat with g_hat = +-s1 +-s2 per
+    element, and p follows the closed form of pin_adam_closed_form."""
+    sizes, T = [40, 24], 20
+    off, wb = offsets_of(sizes), word_base(sizes)
+    n = int(off[-1])
+    bits = np.zeros(2 * wb[-1], np.uint32)
+    for k, nk in enumerate(sizes):
+        nw = wb[k + 1] - wb[k]
+        bits[2 * wb[k]: 2 * wb[k] + nw] = _fixed_direction([nk], (200, k, 1))
+        bits[2 * wb[k] + nw: 2 * wb[k + 1]] = _fixed_direction([nk], (200, k, 2))
+    s = np.array([[0.3, 0.125], [0.7, 0.25]], np.float32)
+    m = np.zeros(n, np.float32)
+    v = aux_uniform(SEED, (201,), n, 1e-4, 1e-2)
+    v0 = v.copy()
+    p0 = aux_normal(SEED, (202,), n, 0.02)
+    p = p0.copy()
+    for _ in range(T):
+        _, flags = o.twobit_apply(off, bits, s, m, v, p, B1, LR, EPS)
+        assert flags == 0
+    gh = _ghat2(bits, s, sizes)
+    b1 = float(B1)
+    assert np.allclose(m, (1 - b1 ** T) * gh, rtol=2e-6, atol=0)
+    sum_m = T - b1 * (1 - b1 ** T) / (1 - b1)
+    want_p = p0 - float(LR) * gh * sum_m / (np.sqrt(v0.astype(np.float64)) + float(EPS))
+    assert np.max(np.abs(p - want_p)) <= 2e-7, np.max(np.abs(p - want_p))
+    assert np.array_equal(v, v0)
+
+
+def pin_twobit_step_composition(o):
+    sizes, W = [40, 33, 64, 0, 7], 3
+    off = offsets_of(sizes)
+    n = int(off[-1])
+    for opt in (0, 1):
+        g, err = _worker_inputs(W, sizes, (210, opt))
+        st = {"p": aux_normal(SEED, (211,), n, 0.02), "m": aux_normal(SEED, (212,), n, 1e-3),
+              "v": aux_uniform(SEED, (213,), n, 1e-8, 1e-6), "err": err.copy(),
+              "srv_err": aux_normal(SEED, (214,), n, 1e-4)}
+        ref = {k: v.copy() for k, v in st.items()}
+        flags = o.twobit_step(off, g, st, B1, LR, EPS, optimizer=opt)
+        b, s, f1 = o.twobit_compress(off, g, ref["err"])
+        bs, ss, f2 = o.twobit_server(off, b, s, ref["srv_err"])
+        _, f3 = o.twobit_apply(off, bs, ss, ref["m"], ref["v"], ref["p"], B1, LR, EPS, optimizer=opt)
+        assert flags == f1 | f2 | f3
+        for k in ("p", "m", "v", "err", "srv_err"):
+            assert np.array_equal(st[k], ref[k]), (opt, k)
+        assert np.array_equal(st["bits_srv"], bs) and np.array_equal(st["s_srv"], ss)
+
+
 ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_") and callable(v)]

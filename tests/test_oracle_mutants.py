@@ -3,7 +3,10 @@
 Each case copies onebit_oracle.c to a temporary directory, plants one
 plausible mistake (a dropped term, a wrong sign, a wrong index, an inverted
 ratio, ...), builds it with the same flags, and checks that at least one pin
-of tests/oracle_pins.py fails on it.  CPU only; nothing here touches the
+of tests/oracle_pins.py fails on it.  Where the oracle repeats a statement
+(the same server average in the 1-bit and 2-bit stages, say), the mutant names
+the occurrence it plants.  Every planted mistake keeps memory accesses in
+bounds, so a mutant can only compute wrong values, never crash the run.  CPU only; nothing here touches the
 product library.
 """
 
@@ -19,20 +22,20 @@ SRC = os.path.join(os.path.dirname(oracle.__file__), "onebit_oracle.c")
 MUTANTS = {
     "error_sign": ("err_set(err, err_dtype, e0 + i, c[i] - dequantize(q, s, i))",
                    "err_set(err, err_dtype, e0 + i, c[i] + dequantize(q, s, i))"),
-    "error_not_added": ("clip) + err_get(err, err_dtype, e0 + i);", "clip) + 0.0f;"),
+    "error_not_added": ("clip) + err_get(err, err_dtype, e0 + i);", "clip) + 0.0f;", 0),
     "sign_of_zero": ("if (c[i] >= 0.0f) words", "if (c[i] > 0.0f) words"),
     "bit_order": ("words[i / 32] |= 1u << (i % 32)", "words[i / 32] |= 1u << (31 - i % 32)"),
     "scale_no_sqrt": ("return (float)(sqrt(S) / sqrt((double)n));", "return (float)(S / (double)n);"),
     "scale_no_mean": ("return (float)(sqrt(S) / sqrt((double)n));", "return (float)sqrt(S);"),
-    "server_sum_not_mean": ("float avg = acc / (float)W;", "float avg = acc;"),
-    "server_error_dropped": ("c[i] = avg + err_get(srv_err, err_dtype, o + i);", "c[i] = avg;"),
+    "server_sum_not_mean": ("float avg = acc / (float)W;", "float avg = acc;", 0),
+    "server_error_dropped": ("c[i] = avg + err_get(srv_err, err_dtype, o + i);", "c[i] = avg;", 0),
     "server_error_sign": ("err_set(srv_err, err_dtype, o + i, c[i] - dequantize(q, s, i))",
                           "err_set(srv_err, err_dtype, o + i, dequantize(q, s, i) - c[i])"),
     "bf16_store_truncates": ("return (uint16_t)((u + 0x7fffu + lsb) >> 16);", "return (uint16_t)(u >> 16);"),
     "bf16_store_ties_up": ("return (uint16_t)((u + 0x7fffu + lsb) >> 16);",
                            "return (uint16_t)((u + 0x8000u) >> 16);"),
     "server_first_worker_only": ("for (int32_t w = 0; w < W; ++w)\n        acc +=",
-                                 "for (int32_t w = 0; w < 1; ++w)\n        acc +="),
+                                 "for (int32_t w = 0; w < 1; ++w)\n        acc +=", 0),
     # (anchors of the scaled-sign update: the s_srv line above, 6-space indentation)
     "momentum_coeff": ("s_srv[k], i);\n      float mi = beta1 * m[o + i] + one_minus_b1 * g_hat;",
                        "s_srv[k], i);\n      float mi = one_minus_b1 * m[o + i] + beta1 * g_hat;"),
@@ -68,7 +71,22 @@ MUTANTS = {
     "ternary_nan_check_dropped": ("if (is_nonfinite(eps_new)) flags |= ORC_STATUS_NONFINITE;", ""),
     "ternary_momentum_coeff": ("(float)W;\n      float mi = beta1 * m[o + i] + one_minus_b1 * g_hat;",
                                "(float)W;\n      float mi = one_minus_b1 * m[o + i] + beta1 * g_hat;"),
-    "ternary_param_sign": ("\n        float pi = p[o + i] - lr * mi", "\n        float pi = p[o + i] + lr * mi"),
+    "ternary_param_sign": ("\n        float pi = p[o + i] - lr * mi", "\n        float pi = p[o + i] + lr * mi", 0),
+    # 2-bit Adam (a third entry: which occurrence of a shared statement is planted)
+    "twobit_error_not_added": ("clip) + err_get(err, err_dtype, e0 + i);", "clip) + 0.0f;", 1),
+    "twobit_server_sum_not_mean": ("float avg = acc / (float)W;", "float avg = acc;", 1),
+    "twobit_server_error_dropped": ("c[i] = avg + err_get(srv_err, err_dtype, o + i);", "c[i] = avg;", 1),
+    "twobit_server_first_worker_only": ("for (int32_t w = 0; w < W; ++w)\n        acc +=",
+                                        "for (int32_t w = 0; w < 1; ++w)\n        acc +=", 1),
+    "twobit_param_sign": ("\n        float pi = p[o + i] - lr * mi", "\n        float pi = p[o + i] + lr * mi", 1),
+    "twobit_second_plane_of_c": ("  quantize_signs(r, nk, words + nw);", "  quantize_signs(c, nk, words + nw);"),
+    "twobit_second_scale_of_c": ("  s[1] = quantize_scale(r, nk);", "  s[1] = quantize_scale(c, nk);"),
+    "twobit_error_drops_first_plane": ("resid[i] = r[i] - dequantize(words + nw, s[1], i);",
+                                       "resid[i] = c[i] - dequantize(words + nw, s[1], i);"),
+    "twobit_dequantize_first_plane_only": ("return dequantize(words, s[0], i) + dequantize(words + nw, s[1], i);",
+                                           "return dequantize(words, s[0], i);"),
+    "twobit_second_plane_shifted": ("  quantize_signs(r, nk, words + nw);", "  quantize_signs(r, nk, words + nw - 1);"),
+    "twobit_apply_word_step": ("    wo += 2 * nw;", "    wo += nw;"),
     "ternary_clip_after_error": ("float c = clip_grad(grad_at(grads, dtype, e), clip) + eps_old;",
                                  "float c = clip_grad(grad_at(grads, dtype, e) + eps_old, clip);"),
 }
@@ -81,10 +99,16 @@ def src_text():
 
 @pytest.mark.parametrize("name", sorted(MUTANTS))
 def test_mutant_is_caught(name, src_text, tmp_path):
-    old, new = MUTANTS[name]
-    assert src_text.count(old) == 1, f"mutation anchor for {name} not unique/present"
+    old, new, *nth = MUTANTS[name]
+    if nth:       # a statement the oracle repeats: plant only its nth occurrence
+        parts = src_text.split(old)
+        assert len(parts) > nth[0] + 1, f"mutation anchor for {name} has no occurrence {nth[0]}"
+        text = old.join(parts[: nth[0] + 1]) + new + old.join(parts[nth[0] + 1:])
+    else:
+        assert src_text.count(old) == 1, f"mutation anchor for {name} not unique/present"
+        text = src_text.replace(old, new)
     mutated = tmp_path / "onebit_oracle.c"
-    mutated.write_text(src_text.replace(old, new))
+    mutated.write_text(text)
     lib = oracle.build(force=True, src=str(mutated), out=str(tmp_path / f"lib_{name}.so"))
     o = oracle.Oracle(lib)
     caught = []
