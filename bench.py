@@ -48,7 +48,7 @@ FALLBACK_HBM_GBS = 6650.0
 E2E_MAX_HOST_BYTES = 16e9        # pinned host gradients per step the e2e leg may hold
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "ncu_traffic.txt")
 KERNEL_SOURCES = [os.path.join(ROOT, "bit_adam_error_b200", "csrc", f)
-                  for f in ("kernels.cuh", "ternary.cuh", "onebit.cu")]
+                  for f in ("kernels.cuh", "ternary.cuh", "twobit.cuh", "onebit.cu")]
 
 
 def parse_args():
@@ -65,9 +65,10 @@ def parse_args():
     ap.add_argument("--phase", choices=["compressed", "refresh"], default="compressed",
                     help="time the compressed step (default) or the full-precision variance-refresh "
                          "step of 0/1 Adam")
-    ap.add_argument("--rule", choices=["scaled", "momentum"], default="scaled",
+    ap.add_argument("--rule", choices=["scaled", "momentum", "twobit"], default="scaled",
                     help="compression rule: scaled sign bits with worker and server error "
-                         "(default), or the momentum-error rule with int8 ternary codes")
+                         "(default), the momentum-error rule with int8 ternary codes, or "
+                         "2-bit Adam (two residual sign planes)")
     ap.add_argument("--err-dtype", choices=["f32", "bf16"], default=None,
                     help="storage of the error buffers (default: the workload's, f32)")
     ap.add_argument("--dp", action="store_true",
@@ -110,6 +111,15 @@ def algo_bytes_per_elem(kind: str, wl) -> float:
         return W + 1.0
     if kind == "k_ternary_update":       # one sum byte, m r/w, v, p r (+ p w for Adam)
         return 1 + (16 if wl.optimizer == "lamb" else 20)
+    # 2-bit Adam: two sign planes per message
+    if kind == "k_tb_resid_norm":        # g, err again for the first plane's residual
+        return (gb + eb) * W
+    if kind == "k_tb_pack":              # g, err r/w, both planes; srv_err read
+        return (gb + 2 * eb) * W + W / 4 + eb
+    if kind == "k_tb_server_norm":       # both planes of every worker, srv_err
+        return W / 4 + eb
+    if kind == "k_tb_server_update":     # planes, srv_err r/w, server planes (+ m, v, p as Adam/LAMB)
+        return W / 4 + 2 * eb + 1 / 4 + (16 if wl.optimizer == "lamb" else 20)
     return 0.0                           # finalisers: a few bytes per chunk
 
 
@@ -118,6 +128,9 @@ def step_bytes_per_elem(wl, phase: str = "compressed", rule: str = "scaled") -> 
         return algo_bytes_per_elem("k_warmup", wl) + (16.0 if wl.optimizer == "lamb" else 0.0)
     if rule == "momentum":
         return algo_bytes_per_elem("k_ternary_step", wl) + (16.0 if wl.optimizer == "lamb" else 0.0)
+    if rule == "twobit":
+        kinds = ["k_worker_norm", "k_tb_resid_norm", "k_tb_pack", "k_tb_server_norm", "k_tb_server_update"]
+        return sum(algo_bytes_per_elem(k, wl) for k in kinds) + (16.0 if wl.optimizer == "lamb" else 0.0)
     kinds = ["k_worker_norm", "k_worker_pack", "k_server_update"]
     if wl.optimizer == "lamb":
         kinds.append("k_lamb_param")
@@ -278,6 +291,9 @@ def oracle_rate(wl, chunks, max_elems=None, min_seconds=0.0, steps=1, phase="com
             elif rule == "momentum":
                 o.ternary_step([0, nk], g, st, f(wl.beta1), f(wl.lr), f(wl.eps), clip=wl.clip,
                                optimizer=opt)
+            elif rule == "twobit":
+                o.twobit_step([0, nk], g, st, f(wl.beta1), f(wl.lr), f(wl.eps), clip=wl.clip,
+                              optimizer=opt)
             else:
                 o.step([0, nk], g, st, f(wl.beta1), f(wl.lr), f(wl.eps), clip=wl.clip, optimizer=opt)
             dt = time.perf_counter() - t
@@ -457,7 +473,7 @@ def run_ours(args):
         # The step's result read back each step: the server scales, or (the
         # momentum-error rule has none) the first C parameters.
         result = opt.s_srv if opt.s_srv is not None else opt.p[: wl.C]
-        s_host = torch.empty(wl.C, dtype=torch.float32, pin_memory=True)
+        s_host = torch.empty(result.shape, dtype=torch.float32, pin_memory=True)
         for i in range(2):
             opt.step(host_g[i % nh])
         torch.cuda.synchronize()
@@ -472,7 +488,7 @@ def run_ours(args):
         barrier(dist)
         ms_e2e = max_over_ranks(dist, e0.elapsed_time(e1) / args.steps, device)
         e2e = {"value": world * n / (ms_e2e / 1e3) / 1e9, "unit": UNIT, "ms_per_step": ms_e2e,
-               "h2d_bytes_per_step": host_bytes, "d2h_bytes_per_step": 4 * wl.C}
+               "h2d_bytes_per_step": host_bytes, "d2h_bytes_per_step": 4 * s_host.numel()}
         del host_g
 
     cpu = None

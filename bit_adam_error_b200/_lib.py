@@ -16,7 +16,7 @@ LIB_PATH = os.path.join(_PKG, "libonebit.so")
 OB_OK, OB_EINVAL, OB_ECUDA, OB_EPHASE, OB_ENOMEM = 0, -1, -2, -3, -4
 OB_F32, OB_BF16 = 0, 1
 OB_ADAM, OB_LAMB = 0, 1
-OB_RULE_SCALED_SIGN, OB_RULE_MOMENTUM_ERROR = 0, 1
+OB_RULE_SCALED_SIGN, OB_RULE_MOMENTUM_ERROR, OB_RULE_TWO_BIT = 0, 1, 2
 OB_STATUS_NONFINITE = 1
 
 ERR_NAMES = {OB_OK: "OB_OK", OB_EINVAL: "OB_EINVAL", OB_ECUDA: "OB_ECUDA",
@@ -72,7 +72,7 @@ _SIGS = {
     "ob_last_error": (ctypes.c_char_p, []),
 }
 
-OB_K_KINDS = 12
+OB_K_KINDS = 16
 
 _lib = None
 

@@ -21,7 +21,7 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libonebit.so")
 SOURCES = [os.path.join(CSRC, "onebit.cu")]
 DEPS = SOURCES + [os.path.join(CSRC, "kernels.cuh"), os.path.join(CSRC, "ternary.cuh"),
-                  os.path.join(INCLUDE, "onebit.h")]
+                  os.path.join(CSRC, "twobit.cuh"), os.path.join(INCLUDE, "onebit.h")]
 
 # -fmad=false: no FMA contraction, so every fp32 expression rounds as written;
 # IEEE division and square root; no fast-math.

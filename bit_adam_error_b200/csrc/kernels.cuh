@@ -344,10 +344,13 @@ __device__ __forceinline__ double block_sum_fixed(double x, double* sm) {
   return r;
 }
 
+// The result of (row r, chunk k) goes to out[(r * C + k) * planes + plane]: one
+// scale per chunk (planes = 1), or one of the two interleaved scales of the
+// 2-bit rule.
 template <bool RMS>
 __global__ void __launch_bounds__(kFinalizeThreads)
 k_finalize_scale(Layout L, const double* __restrict__ part, const int64_t* __restrict__ tpx,
-                 int mult, int64_t row_stride, float* __restrict__ out) {
+                 int mult, int64_t row_stride, float* __restrict__ out, int planes, int plane) {
   __shared__ double sm[kFinalizeThreads];
   const int k = blockIdx.x, r = blockIdx.y;
   const double* pr = part + static_cast<int64_t>(r) * row_stride;
@@ -359,7 +362,7 @@ k_finalize_scale(Layout L, const double* __restrict__ part, const int64_t* __res
     float o = 0.0f;
     if (!RMS) o = __double2float_rn(__dsqrt_rn(S));   // plain L2 norm (monitoring)
     else if (nk > 0) o = __double2float_rn(__ddiv_rn(__dsqrt_rn(S), __dsqrt_rn(static_cast<double>(nk))));
-    out[static_cast<int64_t>(r) * L.C + k] = o;
+    out[(static_cast<int64_t>(r) * L.C + k) * planes + plane] = o;
   }
 }
 

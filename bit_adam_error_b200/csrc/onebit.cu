@@ -22,6 +22,7 @@
 #include "onebit.h"
 #include "kernels.cuh"
 #include "ternary.cuh"
+#include "twobit.cuh"
 
 namespace {
 
@@ -47,10 +48,16 @@ constexpr uintptr_t kAlignElems = 32, kAlignWords = 4;
 int64_t words_of(int64_t n) { return (n + 31) / 32; }
 
 bool momentum_rule(const ob_config* c) { return c->rule == OB_RULE_MOMENTUM_ERROR; }
+bool two_bit_rule(const ob_config* c) { return c->rule == OB_RULE_TWO_BIT; }
 
-// Words of one chunk in a packed row: sign bits, or int8 codes four to a word.
+// Scales per chunk: one, or two for the two planes of the 2-bit rule.
+int64_t scale_planes(const ob_config* c) { return two_bit_rule(c) ? 2 : 1; }
+
+// Words of one chunk in a packed row: sign bits, int8 codes four to a word, or
+// two sign planes.
 int64_t row_words_of(const ob_config* c, int64_t nk) {
-  return momentum_rule(c) ? (nk + 3) / 4 : words_of(nk);
+  if (momentum_rule(c)) return (nk + 3) / 4;
+  return scale_planes(c) * words_of(nk);
 }
 
 // The int8 sum of W codes in {-1, 0, 1} is exact up to this many workers.
@@ -80,8 +87,9 @@ ob_err check_config(const ob_config* c) {
   if (c->freeze_step < 0) return fail(OB_EINVAL, "freeze_step = %d < 0", c->freeze_step);
   if (c->err_dtype != OB_F32 && c->err_dtype != OB_BF16)
     return fail(OB_EINVAL, "err_dtype = %d is neither OB_F32 nor OB_BF16", c->err_dtype);
-  if (c->rule != OB_RULE_SCALED_SIGN && c->rule != OB_RULE_MOMENTUM_ERROR)
-    return fail(OB_EINVAL, "rule = %d is neither OB_RULE_SCALED_SIGN nor OB_RULE_MOMENTUM_ERROR", c->rule);
+  if (c->rule != OB_RULE_SCALED_SIGN && c->rule != OB_RULE_MOMENTUM_ERROR && c->rule != OB_RULE_TWO_BIT)
+    return fail(OB_EINVAL, "rule = %d is not OB_RULE_SCALED_SIGN, OB_RULE_MOMENTUM_ERROR or OB_RULE_TWO_BIT",
+                c->rule);
   if (momentum_rule(c) && c->W > kMaxMomentumWorkers)
     return fail(OB_EINVAL, "W = %d > %d: the int8 sum of the codes could overflow", c->W, kMaxMomentumWorkers);
   // Element and word indices of [W][n] rows must fit in int64 comfortably.
@@ -211,11 +219,14 @@ ob_err check_grads(ob_ctx* c, const void* grads) {
 // ---- enqueue helpers (no validation) ----------------------------------------------
 
 // Per-chunk scales from partial slots [tpx[k]*mult, tpx[k+1]*mult) of each row.
+// planes / plane: where the scales land (one per chunk, or plane `plane` of the
+// two interleaved scales of the 2-bit rule).
 void enqueue_finalize_scale(ob_ctx* c, const double* part, float* out, int rows,
-                            const int64_t* tpx, int mult, int64_t row_stride, cudaStream_t st) {
+                            const int64_t* tpx, int mult, int64_t row_stride, cudaStream_t st,
+                            int planes = 1, int plane = 0) {
   launch(c, OB_K_FINALIZE_SCALE, st, [&] {
     ob::k_finalize_scale<true><<<dim3(c->cfg.num_chunks, rows), ob::kFinalizeThreads, 0, st>>>(
-        c->L, part, tpx, mult, row_stride, out);
+        c->L, part, tpx, mult, row_stride, out, planes, plane);
   });
 }
 
@@ -428,7 +439,145 @@ void enqueue_ternary_update(ob_ctx* c, cudaStream_t st) {
   if (lamb) enqueue_lamb_param(c, st);
 }
 
+// ---- the 2-bit rule (two residual sign planes) ------------------------------------------
+
+// Worker stage (passes 1, 1b, 2) and, when with_server, the server scales
+// (finalise s1', pass 2b, finalise s2').
+template <typename GT, typename ET, bool CLIP, bool POW2>
+void enqueue_tb_worker_t(ob_ctx* c, const GT* grads, bool with_server, cudaStream_t st) {
+  const int W = c->cfg.W;
+  ET* err = static_cast<ET*>(c->err);
+  const ET* srv_err = static_cast<const ET*>(c->srv_err);
+  if (c->T > 0) {
+    auto k1 = ob::k_worker_norm<GT, ET, CLIP>;
+    const int g1 = grid_for(c, k1, W * c->T);
+    launch(c, OB_K_WORKER_NORM, st, [&] {
+      k1<<<g1, ob::kBlock, 0, st>>>(c->L, W, grads, err, c->h.clip, c->part_w, c->status);
+    });
+  }
+  enqueue_finalize_scale(c, c->part_w, c->s_w, W, c->L.tp, 1, c->T, st, 2, 0);
+  if (c->T > 0) {
+    auto k1b = ob::k_tb_resid_norm<GT, ET, CLIP>;
+    const int g = grid_for(c, k1b, W * c->T);
+    launch(c, OB_K_TB_RESID_NORM, st, [&] {
+      k1b<<<g, ob::kBlock, 0, st>>>(c->L, W, grads, err, c->s_w, c->h.clip, c->part_w);
+    });
+  }
+  enqueue_finalize_scale(c, c->part_w, c->s_w, W, c->L.tp, 1, c->T, st, 2, 1);
+  if (c->T > 0) {
+    auto k2 = with_server ? ob::k_tb_pack<GT, ET, true, CLIP, POW2> : ob::k_tb_pack<GT, ET, false, CLIP, false>;
+    const int g2 = grid_for(c, k2, c->T);
+    launch(c, OB_K_TB_PACK, st, [&] {
+      k2<<<g2, ob::kBlock, 0, st>>>(c->L, W, grads, err, c->s_w, c->bits_w, srv_err, c->part_srv,
+                                    c->h.clip, c->status);
+    });
+  }
+  if (!with_server) return;
+  enqueue_finalize_scale(c, c->part_srv, c->s_srv, 1, c->L.tp, 1, 0, st, 2, 0);
+  if (c->T > 0) {
+    auto k = ob::k_tb_server_norm<ET, POW2, true>;
+    const int g = grid_for(c, k, c->T);
+    launch(c, OB_K_TB_SERVER_NORM, st, [&] {
+      k<<<g, ob::kBlock, 0, st>>>(c->L, W, c->bits_w, c->s_w, srv_err, c->s_srv, c->part_srv, c->status);
+    });
+  }
+  enqueue_finalize_scale(c, c->part_srv, c->s_srv, 1, c->L.tp, 1, 0, st, 2, 1);
+}
+
+template <typename GT, typename ET>
+void enqueue_tb_worker_e(ob_ctx* c, const GT* grads, bool with_server, cudaStream_t st) {
+  const bool clip = c->h.clip > 0.0f, p2 = pow2_workers(c);
+  if (clip && p2) enqueue_tb_worker_t<GT, ET, true, true>(c, grads, with_server, st);
+  else if (clip) enqueue_tb_worker_t<GT, ET, true, false>(c, grads, with_server, st);
+  else if (p2) enqueue_tb_worker_t<GT, ET, false, true>(c, grads, with_server, st);
+  else enqueue_tb_worker_t<GT, ET, false, false>(c, grads, with_server, st);
+}
+
+void enqueue_tb_worker(ob_ctx* c, const void* grads, bool with_server, cudaStream_t st) {
+  const bool bf16_err = c->cfg.err_dtype == OB_BF16;
+  if (c->cfg.grad_dtype == OB_BF16) {
+    const uint16_t* g = static_cast<const uint16_t*>(grads);
+    if (bf16_err) enqueue_tb_worker_e<uint16_t, uint16_t>(c, g, with_server, st);
+    else enqueue_tb_worker_e<uint16_t, float>(c, g, with_server, st);
+  } else {
+    const float* g = static_cast<const float*>(grads);
+    if (bf16_err) enqueue_tb_worker_e<float, uint16_t>(c, g, with_server, st);
+    else enqueue_tb_worker_e<float, float>(c, g, with_server, st);
+  }
+}
+
+template <ob::Upd U, bool FROM_WORKERS, typename ET>
+void enqueue_tb_server_update_e(ob_ctx* c, cudaStream_t st) {
+  if (c->T == 0) return;
+  auto k = pow2_workers(c) ? ob::k_tb_server_update<U, FROM_WORKERS, true, ET>
+                           : ob::k_tb_server_update<U, FROM_WORKERS, false, ET>;
+  const int g = grid_for(c, k, c->T);
+  launch(c, OB_K_TB_SERVER_UPDATE, st, [&] {
+    k<<<g, ob::kBlock, 0, st>>>(c->L, c->cfg.W, c->bits_w, c->s_w, c->s_srv, static_cast<ET*>(c->srv_err),
+                                c->bits_srv, c->m, c->v, c->p, c->h, c->partP, c->partU, c->status);
+  });
+}
+
+template <ob::Upd U, bool FROM_WORKERS>
+void enqueue_tb_server_update(ob_ctx* c, cudaStream_t st) {
+  if (FROM_WORKERS && c->cfg.err_dtype == OB_BF16) enqueue_tb_server_update_e<U, FROM_WORKERS, uint16_t>(c, st);
+  else enqueue_tb_server_update_e<U, FROM_WORKERS, float>(c, st);
+}
+
+// Update from the worker planes (fused step) or from bits_srv (stage call).
+void enqueue_tb_update(ob_ctx* c, bool from_workers, cudaStream_t st) {
+  const bool lamb = c->cfg.optimizer == OB_LAMB;
+  if (from_workers) {
+    if (lamb) enqueue_tb_server_update<ob::Upd::kLambM, true>(c, st);
+    else enqueue_tb_server_update<ob::Upd::kAdam, true>(c, st);
+  } else {
+    if (lamb) enqueue_tb_server_update<ob::Upd::kLambM, false>(c, st);
+    else enqueue_tb_server_update<ob::Upd::kAdam, false>(c, st);
+  }
+  if (lamb) enqueue_lamb_param(c, st);
+}
+
+// Server stage alone: s1' (pass over the planes), s2' (residual pass), then the
+// server planes and error.
+template <typename ET, bool POW2>
+void enqueue_tb_server_stage_t(ob_ctx* c, cudaStream_t st) {
+  const ET* srv_err = static_cast<const ET*>(c->srv_err);
+  if (c->T > 0) {
+    auto k = ob::k_tb_server_norm<ET, POW2, false>;
+    const int g = grid_for(c, k, c->T);
+    launch(c, OB_K_TB_SERVER_NORM, st, [&] {
+      k<<<g, ob::kBlock, 0, st>>>(c->L, c->cfg.W, c->bits_w, c->s_w, srv_err, c->s_srv, c->part_srv, c->status);
+    });
+  }
+  enqueue_finalize_scale(c, c->part_srv, c->s_srv, 1, c->L.tp, 1, 0, st, 2, 0);
+  if (c->T > 0) {
+    auto k = ob::k_tb_server_norm<ET, POW2, true>;
+    const int g = grid_for(c, k, c->T);
+    launch(c, OB_K_TB_SERVER_NORM, st, [&] {
+      k<<<g, ob::kBlock, 0, st>>>(c->L, c->cfg.W, c->bits_w, c->s_w, srv_err, c->s_srv, c->part_srv, c->status);
+    });
+  }
+  enqueue_finalize_scale(c, c->part_srv, c->s_srv, 1, c->L.tp, 1, 0, st, 2, 1);
+  enqueue_tb_server_update<ob::Upd::kNone, true>(c, st);
+}
+
+void enqueue_tb_server_stage(ob_ctx* c, cudaStream_t st) {
+  const bool p2 = pow2_workers(c);
+  if (c->cfg.err_dtype == OB_BF16) {
+    if (p2) enqueue_tb_server_stage_t<uint16_t, true>(c, st); else enqueue_tb_server_stage_t<uint16_t, false>(c, st);
+  } else {
+    if (p2) enqueue_tb_server_stage_t<float, true>(c, st); else enqueue_tb_server_stage_t<float, false>(c, st);
+  }
+}
+
 ob_err fused_step(ob_ctx* c, const void* grads, cudaStream_t st) {
+  if (two_bit_rule(&c->cfg)) {
+    enqueue_tb_worker(c, grads, true, st);
+    enqueue_tb_update(c, true, st);
+    ob_err r = check_launch("ob_step");
+    if (r == OB_OK) ++c->step;
+    return r;
+  }
   if (momentum_rule(&c->cfg)) {
     enqueue_ternary(c, grads, true, st);
     ob_err r = check_launch("ob_step");
@@ -471,9 +620,9 @@ ob_err require_buffers(const ob_ctx* c, unsigned need, const char* call) {
       {kNeedWorker | kNeedErr, c->err, W * n, "err"},
       {kNeedServer & scaled, c->srv_err, n, "srv_err"},
       {kNeedWorker | kNeedServer, c->bits_w, W * c->words, "bits_w"},
-      {(kNeedWorker | kNeedServer) & scaled, c->s_w, W * C, "s_w"},
+      {(kNeedWorker | kNeedServer) & scaled, c->s_w, W * C * scale_planes(&c->cfg), "s_w"},
       {kNeedUpdate | kNeedServer, c->bits_srv, c->words, "bits_srv"},
-      {(kNeedUpdate | kNeedServer) & scaled, c->s_srv, C, "s_srv"}};
+      {(kNeedUpdate | kNeedServer) & scaled, c->s_srv, C * scale_planes(&c->cfg), "s_srv"}};
   for (const auto& b : list)
     if ((b.mask & need) && b.count > 0 && !b.p)
       return fail(OB_EINVAL, "%s: the ctx was created without %s", call, b.name);
@@ -517,8 +666,8 @@ ob_err ob_create(const ob_config* cfg, float* p, float* m, float* v, void* err, 
   struct { const void* p; int64_t count; const char* name; uintptr_t align; } bufs[] = {
       {p, n, "p", kAlignElems}, {m, n, "m", kAlignElems}, {v, n, "v", kAlignElems},
       {err, W * n, "err", kAlignElems}, {srv_err, n, "srv_err", kAlignElems},
-      {bits_w, W * words, "bits_w", kAlignWords}, {s_w, W * C, "s_w", kAlignWords},
-      {bits_srv, words, "bits_srv", kAlignWords}, {s_srv, C, "s_srv", kAlignWords}};
+      {bits_w, W * words, "bits_w", kAlignWords}, {s_w, W * C * scale_planes(cfg), "s_w", kAlignWords},
+      {bits_srv, words, "bits_srv", kAlignWords}, {s_srv, C * scale_planes(cfg), "s_srv", kAlignWords}};
   for (auto& b : bufs)  // NULL: the ctx is created without that buffer (see require_buffers)
     if (b.p && (r = check_dev(b.p, b.count, b.name, device, b.align)) != OB_OK) return r;
 
@@ -655,6 +804,7 @@ ob_err ob_compress(ob_ctx* c, const void* grads, void* stream) {
   if ((r = check_grads(c, grads)) != OB_OK) return r;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (momentum_rule(&c->cfg)) enqueue_ternary(c, grads, false, st);
+  else if (two_bit_rule(&c->cfg)) enqueue_tb_worker(c, grads, false, st);
   else if (c->cfg.grad_dtype == OB_BF16) enqueue_worker<uint16_t>(c, static_cast<const uint16_t*>(grads), false, st);
   else enqueue_worker<float>(c, static_cast<const float*>(grads), false, st);
   return check_launch("ob_compress");
@@ -668,6 +818,7 @@ ob_err ob_server_reduce(ob_ctx* c, void* stream) {
   DeviceGuard dg(c->device);
   if (!dg.ok) return fail(OB_ECUDA, "cannot select device %d", c->device);
   if (momentum_rule(&c->cfg)) enqueue_ternary_server(c, static_cast<cudaStream_t>(stream));
+  else if (two_bit_rule(&c->cfg)) enqueue_tb_server_stage(c, static_cast<cudaStream_t>(stream));
   else enqueue_server_stage(c, static_cast<cudaStream_t>(stream));
   return check_launch("ob_server_reduce");
 }
@@ -689,6 +840,7 @@ ob_err ob_step(ob_ctx* c, const void* grads, void* stream) {
     return fused_step(c, grads, st);
   }
   if (momentum_rule(&c->cfg)) enqueue_ternary_update(c, st);
+  else if (two_bit_rule(&c->cfg)) enqueue_tb_update(c, false, st);
   else enqueue_update(c, false, st);
   if ((r = check_launch("ob_step")) != OB_OK) return r;
   ++c->step;
@@ -834,7 +986,7 @@ ob_err ob_error_norms(ob_ctx* c, float* worker_norms, float* server_norms, void*
     }
     launch(c, OB_K_FINALIZE_SCALE, st, [&] {
       ob::k_finalize_scale<false><<<dim3(unsigned(C), unsigned(rows)), ob::kFinalizeThreads, 0, st>>>(
-          c->L, part, c->L.tp, 1, c->T, out);
+          c->L, part, c->L.tp, 1, c->T, out, 1, 0);
     });
   };
   if (worker_norms) norms(c->err, int(W), c->part_w, worker_norms);
@@ -894,7 +1046,8 @@ const char* ob_kernel_name(int32_t kind) {
   static const char* names[OB_K_KINDS] = {
       "k_worker_norm", "k_finalize_scale", "k_worker_pack", "k_server_norm",
       "k_server_update", "k_lamb_param", "k_warmup", "k_finalize_ratio",
-      "k_ternary_step", "k_ternary_compress", "k_ternary_server", "k_ternary_update"};
+      "k_ternary_step", "k_ternary_compress", "k_ternary_server", "k_ternary_update",
+      "k_tb_resid_norm", "k_tb_pack", "k_tb_server_norm", "k_tb_server_update"};
   return (kind >= 0 && kind < OB_K_KINDS) ? names[kind] : "";
 }
 
@@ -1050,7 +1203,7 @@ extern "C" ob_err ob_compress_noalloc(const ob_config* cfg, const void* grads, f
     else if (cl) ob::k_worker_norm<float, float, true><<<g1, ob::kBlock, 0, st>>>(L, int(W), gf, err, clip, part, status);
     else ob::k_worker_norm<float, float, false><<<g1, ob::kBlock, 0, st>>>(L, int(W), gf, err, clip, part, status);
   }
-  ob::k_finalize_scale<true><<<dim3(unsigned(C), unsigned(W)), ob::kFinalizeThreads, 0, st>>>(L, part, L.tp, 1, T, s_w);
+  ob::k_finalize_scale<true><<<dim3(unsigned(C), unsigned(W)), ob::kFinalizeThreads, 0, st>>>(L, part, L.tp, 1, T, s_w, 1, 0);
   if (T > 0) {
     const int g2 = noalloc_grid(d->num_sms, d->occ_pack[bf], T);
     const uint16_t* gh = static_cast<const uint16_t*>(grads);

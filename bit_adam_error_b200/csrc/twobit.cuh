@@ -1,0 +1,383 @@
+// twobit.cuh -- sm_100a kernels of 2-bit Adam (two residual sign planes).
+//
+// 2-bit Adam is named by the CANN 1-bit Adam article (section 5.1 table: 6.25% of
+// the traffic; section 8: weaker compression for embedding layers) without a
+// quantiser.  Here it is the 1-bit quantiser of kernels.cuh applied twice:
+//   s1 = ||c|| / sqrt(n_k),  q1 = (c >= 0),   r   = c - s1 sign(q1)
+//   s2 = ||r|| / sqrt(n_k),  q2 = (r >= 0),   err = r - s2 sign(q2)
+//   dequantised value = s1 sign(q1) + s2 sign(q2)
+// for the workers and, on their average plus the server error, for the server.
+//
+// Each extra norm is another streaming pass: s2 needs s1 before r exists, and
+// the server's s2 needs its s1.  The fused step is five passes (plus finalisers):
+//   1  k_worker_norm        g, err            -> sum c^2          -> s1
+//   1b k_tb_resid_norm      g, err            -> sum r^2          -> s2
+//   2  k_tb_pack<SERVER>    g, err, srv_err   -> err, planes, sum c_srv^2 -> s1'
+//   2b k_tb_server_norm<R>  planes, srv_err   -> sum r_srv^2      -> s2'
+//   3  k_tb_server_update   planes, srv_err, m, v, p -> server planes, srv_err, m, p
+// Layout: chunk k owns 2 ceil(n_k / 32) words of a row, plane 1 then plane 2,
+// from word wo[k]; scales are [row][C][2].  Tiling, vector/scalar paths and the
+// floating-point order are those of kernels.cuh (every value equals the plain C
+// statement of the rule for the same scales).
+#pragma once
+
+#include "kernels.cuh"
+
+namespace ob {
+
+__device__ __forceinline__ int64_t plane_words(int64_t nk) { return (nk + 31) / 32; }
+
+// acc[j] += s1 sign1 + s2 sign2 of worker w, ascending w (the order of pass 2).
+__device__ __forceinline__ void tb_server_sum8(const Layout& L, int W, const uint32_t* __restrict__ bits_w,
+                                               const float* __restrict__ s_w, const Tile& tl, int64_t wrel,
+                                               int64_t nwk, bool word_in, int lane, float (&acc)[8]) {
+  zero8(acc);
+  for (int w = 0; w < W; ++w) {
+    const float* sc = s_w + (static_cast<int64_t>(w) * L.C + tl.k) * 2;
+    const float s1 = __ldg(sc), s2 = __ldg(sc + 1);
+    const uint32_t* row = bits_w + static_cast<int64_t>(w) * L.words + tl.w0;
+    const uint32_t w1 = word_in ? __ldg(row + wrel) : 0u;
+    const uint32_t w2 = word_in ? __ldg(row + nwk + wrel) : 0u;
+    const uint32_t b1 = lane_byte(w1, lane), b2 = lane_byte(w2, lane);
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      acc[j] = acc[j] + (signed_scale((b1 >> j) & 1u, s1) + signed_scale((b2 >> j) & 1u, s2));
+  }
+}
+
+__device__ __forceinline__ float tb_server_sum1(const Layout& L, int W, const uint32_t* __restrict__ bits_w,
+                                                const float* __restrict__ s_w, const Tile& tl, int64_t wi,
+                                                int64_t nwk, int lane) {
+  float acc = 0.0f;
+  for (int w = 0; w < W; ++w) {
+    const float* sc = s_w + (static_cast<int64_t>(w) * L.C + tl.k) * 2;
+    const uint32_t* row = bits_w + static_cast<int64_t>(w) * L.words + tl.w0;
+    const bool b1 = (__ldg(row + wi) >> lane) & 1u, b2 = (__ldg(row + nwk + wi) >> lane) & 1u;
+    acc = acc + (signed_scale(b1, __ldg(sc)) + signed_scale(b2, __ldg(sc + 1)));
+  }
+  return acc;
+}
+
+// ---- pass 1b: per-tile sum of r^2, r = c - s1 sign(c) ---------------------------------
+template <typename GT, typename ET, bool CLIP>
+__global__ void __launch_bounds__(kBlock)
+k_tb_resid_norm(Layout L, int W, const GT* __restrict__ grads, const ET* __restrict__ err,
+                const float* __restrict__ s_w, float clip, double* __restrict__ part) {
+  const int lane = threadIdx.x & 31;
+  const int64_t items = static_cast<int64_t>(W) * L.T;
+  int hint = 0;
+  for (int64_t it = warp_id(); it < items; it += warp_count()) {
+    const int w = static_cast<int>(it / L.T);
+    const int64_t t = it - static_cast<int64_t>(w) * L.T;
+    const Tile tl = tile_at(L, t, hint);
+    const GT* g = grads + static_cast<int64_t>(w) * L.n + tl.ck0;
+    const ET* e = err + static_cast<int64_t>(w) * L.n + tl.ck0;
+    const float s1 = __ldg(s_w + (static_cast<int64_t>(w) * L.C + tl.k) * 2);
+    double acc = 0.0;
+    if (tl.vec) {
+#pragma unroll
+      for (int gq = 0; gq < kGroups; ++gq) {
+        const int64_t i0 = tl.rel + gq * kGroupElems + lane * kVec;
+        if (i0 < tl.nk) {
+          float gv[8], ev[8];
+          ld8_ro(g + i0, gv);
+          ld8_ro(e + i0, ev);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const float c = (CLIP ? clip_grad(gv[j], clip) : gv[j]) + ev[j];
+            const float r = c - signed_scale(c >= 0.0f, s1);
+            acc = fma(static_cast<double>(r), static_cast<double>(r), acc);
+          }
+        }
+      }
+    } else {
+      for (int j = 0; j < kTileWords; ++j) {
+        const int64_t i = tl.rel + j * 32 + lane;
+        if (i < tl.nk) {
+          const float c = (CLIP ? clip_grad(ld1_ro(g + i), clip) : ld1_ro(g + i)) + ld1_ro(e + i);
+          const float r = c - signed_scale(c >= 0.0f, s1);
+          acc = fma(static_cast<double>(r), static_cast<double>(r), acc);
+        }
+      }
+    }
+    acc = warp_sum(acc);
+    if (lane == 0) part[it] = acc;
+  }
+}
+
+// ---- pass 2: both planes, worker error (+ server sums) ---------------------------------
+template <typename GT, typename ET, bool SERVER, bool CLIP, bool POW2>
+__global__ void __launch_bounds__(kBlock)
+k_tb_pack(Layout L, int W, const GT* __restrict__ grads, ET* __restrict__ err,
+          const float* __restrict__ s_w, uint32_t* __restrict__ bits_w, const ET* __restrict__ srv_err,
+          double* __restrict__ part_srv, float clip, uint32_t* __restrict__ status) {
+  const int lane = threadIdx.x & 31;
+  const auto mean = make_mean<POW2>(W);
+  int hint = 0;
+  for (int64_t t = warp_id(); t < L.T; t += warp_count()) {
+    const Tile tl = tile_at(L, t, hint);
+    const int64_t nwk = plane_words(tl.nk);
+    double tsum = 0.0;
+    if (tl.vec) {
+#pragma unroll 1
+      for (int gq = 0; gq < kGroups; ++gq) {
+        const int64_t i0 = tl.rel + gq * kGroupElems + lane * kVec;
+        const bool in = i0 < tl.nk;
+        const int64_t wrel = (tl.rel + gq * kGroupElems) / 32 + (lane >> 2);
+        float acc[8], sv[8];
+        zero8(acc);
+        if (SERVER) {
+          if (in) ld8_ro(srv_err + tl.ck0 + i0, sv); else zero8(sv);
+        }
+        for (int w = 0; w < W; ++w) {
+          const GT* g = grads + static_cast<int64_t>(w) * L.n + tl.ck0;
+          ET* e = err + static_cast<int64_t>(w) * L.n + tl.ck0;
+          const float* sc = s_w + (static_cast<int64_t>(w) * L.C + tl.k) * 2;
+          const float s1 = __ldg(sc), s2 = __ldg(sc + 1);
+          float gv[8], ev[8];
+          if (in) { ld8_ro(g + i0, gv); ld8(e + i0, ev); }
+          else { zero8(gv); zero8(ev); }
+          uint32_t byte1 = 0, byte2 = 0;
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const float c = (CLIP ? clip_grad(gv[j], clip) : gv[j]) + ev[j];
+            const bool b1 = c >= 0.0f;
+            const float d1 = signed_scale(b1, s1);
+            const float r = c - d1;
+            const bool b2 = r >= 0.0f;
+            const float d2 = signed_scale(b2, s2);
+            byte1 |= static_cast<uint32_t>(b1) << j;
+            byte2 |= static_cast<uint32_t>(b2) << j;
+            ev[j] = r - d2;
+            acc[j] = acc[j] + (d1 + d2);
+          }
+          if (in) st8(e + i0, ev);
+          else { byte1 = 0; byte2 = 0; }
+          const uint32_t word1 = quad_word(byte1, lane), word2 = quad_word(byte2, lane);
+          if ((lane & 3) == 0 && wrel * 32 < tl.nk) {
+            uint32_t* row = bits_w + static_cast<int64_t>(w) * L.words + tl.w0;
+            row[wrel] = word1;
+            row[nwk + wrel] = word2;
+          }
+        }
+        if (SERVER && in) {
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const float cs = mean(acc[j]) + sv[j];
+            tsum = fma(static_cast<double>(cs), static_cast<double>(cs), tsum);
+          }
+        }
+      }
+    } else {
+      for (int j = 0; j < kTileWords; ++j) {
+        const int64_t i = tl.rel + j * 32 + lane;
+        const bool inb = i < tl.nk;
+        const int64_t wi = tl.rel / 32 + j;
+        float acc = 0.0f;
+        for (int w = 0; w < W; ++w) {
+          const float* sc = s_w + (static_cast<int64_t>(w) * L.C + tl.k) * 2;
+          ET* e = err + static_cast<int64_t>(w) * L.n + tl.ck0;
+          bool b1 = false, b2 = false;
+          if (inb) {
+            const float g = ld1_ro(grads + static_cast<int64_t>(w) * L.n + tl.ck0 + i);
+            const float c = (CLIP ? clip_grad(g, clip) : g) + ld1(e + i);
+            b1 = c >= 0.0f;
+            const float d1 = signed_scale(b1, __ldg(sc));
+            const float r = c - d1;
+            b2 = r >= 0.0f;
+            const float d2 = signed_scale(b2, __ldg(sc + 1));
+            st1(e + i, r - d2);
+            acc = acc + (d1 + d2);
+          }
+          const uint32_t word1 = __ballot_sync(kFull, b1), word2 = __ballot_sync(kFull, b2);
+          if (lane == 0 && (tl.rel + j * 32) < tl.nk) {
+            uint32_t* row = bits_w + static_cast<int64_t>(w) * L.words + tl.w0;
+            row[wi] = word1;
+            row[nwk + wi] = word2;
+          }
+        }
+        if (SERVER && inb) {
+          const float cs = mean(acc) + ld1_ro(srv_err + tl.ck0 + i);
+          tsum = fma(static_cast<double>(cs), static_cast<double>(cs), tsum);
+        }
+      }
+    }
+    if (SERVER) {
+      tsum = warp_sum(tsum);
+      if (lane == 0) {
+        part_srv[t] = tsum;
+        flag_tile_sum(tsum, status);
+      }
+    }
+  }
+}
+
+// ---- server norms from the worker planes --------------------------------------------
+// RESID = false: sum c_srv^2 (for s1'; the stage call).  RESID = true: sum of
+// (c_srv - s1' sign(c_srv))^2 (for s2'), s1' read from s_srv.
+template <typename ET, bool POW2, bool RESID>
+__global__ void __launch_bounds__(kBlock)
+k_tb_server_norm(Layout L, int W, const uint32_t* __restrict__ bits_w, const float* __restrict__ s_w,
+                 const ET* __restrict__ srv_err, const float* __restrict__ s_srv,
+                 double* __restrict__ part, uint32_t* __restrict__ status) {
+  const int lane = threadIdx.x & 31;
+  const auto mean = make_mean<POW2>(W);
+  int hint = 0;
+  for (int64_t t = warp_id(); t < L.T; t += warp_count()) {
+    const Tile tl = tile_at(L, t, hint);
+    const int64_t nwk = plane_words(tl.nk);
+    const float s1 = RESID ? __ldg(s_srv + 2 * tl.k) : 0.0f;
+    double tsum = 0.0;
+    auto add = [&](float cs) {
+      const float x = RESID ? cs - signed_scale(cs >= 0.0f, s1) : cs;
+      tsum = fma(static_cast<double>(x), static_cast<double>(x), tsum);
+    };
+    if (tl.vec) {
+#pragma unroll
+      for (int gq = 0; gq < kGroups; ++gq) {
+        const int64_t i0 = tl.rel + gq * kGroupElems + lane * kVec;
+        const int64_t wrel = (tl.rel + gq * kGroupElems) / 32 + (lane >> 2);
+        const bool in = i0 < tl.nk;
+        float sv[8], acc[8];
+        if (in) ld8_ro(srv_err + tl.ck0 + i0, sv); else zero8(sv);
+        tb_server_sum8(L, W, bits_w, s_w, tl, wrel, nwk, wrel * 32 < tl.nk, lane, acc);
+        if (in) {
+#pragma unroll
+          for (int j = 0; j < 8; ++j) add(mean(acc[j]) + sv[j]);
+        }
+      }
+    } else {
+      for (int j = 0; j < kTileWords; ++j) {
+        const int64_t i = tl.rel + j * 32 + lane;
+        if (i < tl.nk) add(mean(tb_server_sum1(L, W, bits_w, s_w, tl, tl.rel / 32 + j, nwk, lane)) +
+                           ld1_ro(srv_err + tl.ck0 + i));
+      }
+    }
+    tsum = warp_sum(tsum);
+    if (lane == 0) {
+      part[t] = tsum;
+      if (!RESID) flag_tile_sum(tsum, status);
+    }
+  }
+}
+
+// ---- pass 3: server planes + server error, and/or the update --------------------------
+// FROM_WORKERS: c_srv from the worker planes and srv_err, quantised to two planes
+// with s_srv (bits_srv and srv_err written).  Otherwise g_hat from bits_srv.
+template <Upd U, bool FROM_WORKERS, bool POW2, typename ET>
+__global__ void __launch_bounds__(kBlock, kUpdateMinBlocks)
+k_tb_server_update(Layout L, int W, const uint32_t* __restrict__ bits_w, const float* __restrict__ s_w,
+                   const float* __restrict__ s_srv, ET* __restrict__ srv_err,
+                   uint32_t* __restrict__ bits_srv, float* __restrict__ m, const float* __restrict__ v,
+                   float* __restrict__ p, Hyper h, double* __restrict__ partP,
+                   double* __restrict__ partU, uint32_t* __restrict__ status) {
+  const int lane = threadIdx.x & 31;
+  const auto mean = make_mean<POW2>(W);
+  int hint = 0;
+  for (int64_t t = warp_id(); t < L.T; t += warp_count()) {
+    const Tile tl = tile_at(L, t, hint);
+    const int64_t nwk = plane_words(tl.nk);
+    const float s1 = __ldg(s_srv + 2 * tl.k), s2 = __ldg(s_srv + 2 * tl.k + 1);
+    uint32_t* srow = bits_srv + tl.w0;
+    double Psum = 0.0, Usum = 0.0;
+    bool bad = false;
+    if (tl.vec) {
+#pragma unroll 1
+      for (int gq = 0; gq < kGroups; ++gq) {
+        const int64_t i0 = tl.rel + gq * kGroupElems + lane * kVec;
+        const int64_t wrel = (tl.rel + gq * kGroupElems) / 32 + (lane >> 2);
+        const bool word_in = wrel * 32 < tl.nk;
+        const bool in = i0 < tl.nk;
+        const int64_t gi = tl.ck0 + i0;
+        float sv[8], mv[8], vv[8], pv[8];
+        if (in) {
+          if (FROM_WORKERS) ld8(srv_err + gi, sv);
+          if (U != Upd::kNone) { ld8(m + gi, mv); ld8_ro(v + gi, vv); ld8(p + gi, pv); }
+        }
+        if (FROM_WORKERS) {
+          float acc[8];
+          tb_server_sum8(L, W, bits_w, s_w, tl, wrel, nwk, word_in, lane, acc);
+          uint32_t byte1 = 0, byte2 = 0;
+          if (in) {
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              const float cs = mean(acc[j]) + sv[j];
+              const bool b1 = cs >= 0.0f;
+              const float d1 = signed_scale(b1, s1);
+              const float r = cs - d1;
+              const bool b2 = r >= 0.0f;
+              const float d2 = signed_scale(b2, s2);
+              byte1 |= static_cast<uint32_t>(b1) << j;
+              byte2 |= static_cast<uint32_t>(b2) << j;
+              sv[j] = r - d2;
+              update_elem<U>(d1 + d2, mv[j], vv[j], pv[j], h, Psum, Usum, bad);
+            }
+            st8(srv_err + gi, sv);
+          }
+          const uint32_t word1 = quad_word(byte1, lane), word2 = quad_word(byte2, lane);
+          if ((lane & 3) == 0 && word_in) {
+            srow[wrel] = word1;
+            srow[nwk + wrel] = word2;
+          }
+        } else {
+          const uint32_t w1 = word_in ? __ldg(srow + wrel) : 0u;
+          const uint32_t w2 = word_in ? __ldg(srow + nwk + wrel) : 0u;
+          const uint32_t byte1 = lane_byte(w1, lane), byte2 = lane_byte(w2, lane);
+          if (in) {
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+              update_elem<U>(signed_scale((byte1 >> j) & 1u, s1) + signed_scale((byte2 >> j) & 1u, s2),
+                             mv[j], vv[j], pv[j], h, Psum, Usum, bad);
+          }
+        }
+        if (in && U != Upd::kNone) {
+          st8(m + gi, mv);
+          if (U == Upd::kAdam) st8(p + gi, pv);
+        }
+      }
+    } else {
+      for (int j = 0; j < kTileWords; ++j) {
+        const int64_t i = tl.rel + j * 32 + lane;
+        const bool inb = i < tl.nk;
+        const int64_t gi = tl.ck0 + i;
+        const int64_t wi = tl.rel / 32 + j;
+        float d = 0.0f;
+        if (FROM_WORKERS) {
+          bool b1 = false, b2 = false;
+          if (inb) {
+            const float cs = mean(tb_server_sum1(L, W, bits_w, s_w, tl, wi, nwk, lane)) + ld1(srv_err + gi);
+            b1 = cs >= 0.0f;
+            const float d1 = signed_scale(b1, s1);
+            const float r = cs - d1;
+            b2 = r >= 0.0f;
+            const float d2 = signed_scale(b2, s2);
+            st1(srv_err + gi, r - d2);
+            d = d1 + d2;
+          }
+          const uint32_t word1 = __ballot_sync(kFull, b1), word2 = __ballot_sync(kFull, b2);
+          if (lane == 0 && (tl.rel + j * 32) < tl.nk) {
+            srow[wi] = word1;
+            srow[nwk + wi] = word2;
+          }
+        } else if (inb) {
+          d = signed_scale((__ldg(srow + wi) >> lane) & 1u, s1) +
+              signed_scale((__ldg(srow + nwk + wi) >> lane) & 1u, s2);
+        }
+        if (inb && U != Upd::kNone) {
+          float mv = m[gi], pv = p[gi];
+          update_elem<U>(d, mv, __ldg(v + gi), pv, h, Psum, Usum, bad);
+          m[gi] = mv;
+          if (U == Upd::kAdam) p[gi] = pv;
+        }
+      }
+    }
+    if (U == Upd::kLambM) {
+      Psum = warp_sum(Psum);
+      Usum = warp_sum(Usum);
+      if (lane == 0) { partP[t] = Psum; partU[t] = Usum; }
+    }
+    flag_nonfinite(bad, status);
+  }
+}
+
+}  // namespace ob

@@ -15,7 +15,9 @@ in HBM as flat buffers:
 With ``rule="momentum"`` (the momentum-error rule of the CANN 1-bit Adam
 article, sections 2.1-3.2) bits_w / bits_srv hold int8 codes and their sums
 (``codes_w`` / ``codes_srv`` give int8 views), and srv_err, s_w, s_srv are
-absent (None): that rule has no scale and no server error.
+absent (None): that rule has no scale and no server error.  With
+``rule="twobit"`` (2-bit Adam: two residual sign planes) bits_w / bits_srv
+hold both planes of every chunk and s_w / s_srv are [W, C, 2] / [C, 2].
 
 Phases follow "DeepSpeed Communication Compression and Hiding" (section
 "1-bit Adam", 机制): ``step()`` runs the full-precision warmup while
@@ -55,8 +57,10 @@ class OneBitAdam:
         self.optimizer = {"adam": L.OB_ADAM, "lamb": L.OB_LAMB}[optimizer]
         self.err_dtype = {"f32": L.OB_F32, "bf16": L.OB_BF16}[err_dtype]
         edt = torch.float32 if self.err_dtype == L.OB_F32 else torch.bfloat16
-        self.rule = {"scaled": L.OB_RULE_SCALED_SIGN, "momentum": L.OB_RULE_MOMENTUM_ERROR}[rule]
-        scaled = self.rule == L.OB_RULE_SCALED_SIGN
+        self.rule = {"scaled": L.OB_RULE_SCALED_SIGN, "momentum": L.OB_RULE_MOMENTUM_ERROR,
+                     "twobit": L.OB_RULE_TWO_BIT}[rule]
+        scaled = self.rule != L.OB_RULE_MOMENTUM_ERROR        # has scales and a server error
+        planes = (2,) if self.rule == L.OB_RULE_TWO_BIT else ()
         self.cfg, self._off_keep = L.make_config(self.n, self.offsets, self.W, self.grad_dtype,
                                                  self.optimizer, lr, beta1, beta2, eps, clip,
                                                  freeze_step, self.err_dtype, self.rule)
@@ -75,9 +79,9 @@ class OneBitAdam:
         self.err = torch.zeros((self.W, self.n), dtype=edt, device=dev)
         self.srv_err = torch.zeros(self.n, dtype=edt, device=dev) if scaled else None
         self.bits_w = torch.zeros((self.W, self.words), dtype=torch.int32, device=dev)
-        self.s_w = torch.zeros((self.W, self.C), dtype=f32, device=dev) if scaled else None
+        self.s_w = torch.zeros((self.W, self.C, *planes), dtype=f32, device=dev) if scaled else None
         self.bits_srv = torch.zeros(self.words, dtype=torch.int32, device=dev)
-        self.s_srv = torch.zeros(self.C, dtype=f32, device=dev) if scaled else None
+        self.s_srv = torch.zeros((self.C, *planes), dtype=f32, device=dev) if scaled else None
         with torch.cuda.device(dev):
             self.ctx = L.ob_create(self.cfg, _ptr(self.p), _ptr(self.m), _ptr(self.v),
                                    _ptr(self.err), _ptr(self.srv_err), _ptr(self.bits_w),

@@ -38,6 +38,14 @@
  * int8, so W <= 127), g_hat = sum / W, and m, p move as above (v frozen).
  * There is no server error and no scale under this rule.
  *
+ * A third rule, 2-bit Adam (named by the CANN article, section 5.1, without a
+ * quantiser), is selected by OB_RULE_TWO_BIT: the 1-bit quantiser applied twice,
+ * the second time to what the first left over --
+ *   s1 = ||c|| / sqrt(n_k), q1 = sign(c), r = c - s1 q1,
+ *   s2 = ||r|| / sqrt(n_k), q2 = sign(r), err = r - s2 q2,
+ * dequantised as s1 q1 + s2 q2 -- for the workers and, on their average plus
+ * the server error, for the server.
+ *
  * Conventions for every call:
  *   - Device buffers are caller-owned and must stay valid for the ctx's life.
  *     The ctx stores their pointers and owns only its own scratch (per-tile
@@ -80,7 +88,8 @@ enum { OB_F32 = 0, OB_BF16 = 1 };  /* gradient element type */
 enum { OB_ADAM = 0, OB_LAMB = 1 }; /* update rule after the compressed allreduce */
 enum {                             /* compression rule (ob_config.rule) */
   OB_RULE_SCALED_SIGN = 0,         /* sign bits + per-chunk scale, worker and server error */
-  OB_RULE_MOMENTUM_ERROR = 1       /* int8 ternary codes, momentum-form worker error */
+  OB_RULE_MOMENTUM_ERROR = 1,      /* int8 ternary codes, momentum-form worker error */
+  OB_RULE_TWO_BIT = 2              /* two residual sign planes, two scales per chunk */
 };
 
 #define OB_STATUS_NONFINITE 1u /* a compensated value, server value or parameter was NaN/Inf */
@@ -99,14 +108,16 @@ typedef struct {
   int32_t err_dtype;            /* OB_F32, or OB_BF16: err and srv_err stored as bfloat16
                                    (rounded to nearest even; arithmetic stays float32) --
                                    half the error-buffer bytes, different rounding */
-  int32_t rule;                 /* OB_RULE_SCALED_SIGN (default 0) or OB_RULE_MOMENTUM_ERROR
-                                   (then W <= 127) */
+  int32_t rule;                 /* OB_RULE_SCALED_SIGN (default 0), OB_RULE_MOMENTUM_ERROR
+                                   (then W <= 127) or OB_RULE_TWO_BIT */
 } ob_config;
 
 /* Number of uint32 words one packed row holds.  OB_RULE_SCALED_SIGN: sign bits,
  * sum_k ceil(n_k / 32).  OB_RULE_MOMENTUM_ERROR: int8 codes, sum_k ceil(n_k / 4);
  * element i of chunk k is byte i of the chunk's words (byte b of a word is bits
  * 8b..8b+7), every chunk starts on a fresh word, padding bytes are 0.
+ * OB_RULE_TWO_BIT: sum_k 2 ceil(n_k / 32) -- chunk k's words hold plane 1 then
+ * plane 2, each laid out like the sign bits.
  * Host-only; validates the config.  words_total must be non-NULL. */
 ob_err ob_layout(const ob_config* cfg, int64_t* words_total);
 
@@ -127,6 +138,8 @@ ob_err ob_layout(const ob_config* cfg, int64_t* words_total);
  * s_w and s_srv are never used (pass NULL); ob_compress needs err and bits_w,
  * ob_server_reduce bits_w and bits_srv, ob_step(NULL) p, m, v and bits_srv, and
  * ob_step(grads) p, m, v and err only.
+ * Under OB_RULE_TWO_BIT: bits_w / bits_srv hold both planes (ob_layout words),
+ * and s_w is [W][C][2], s_srv [C][2] (plane 1, plane 2 of each chunk).
  * Allocates the ctx scratch with cudaMalloc on the current device and
  * synchronises once.  *out receives the ctx (NULL on failure). */
 ob_err ob_create(const ob_config* cfg, float* p, float* m, float* v, void* err,
@@ -218,7 +231,11 @@ enum {
   OB_K_TERNARY_COMPRESS = 9, /* momentum-error rule: codes + worker error (stage call) */
   OB_K_TERNARY_SERVER = 10,  /* momentum-error rule: sum of the workers' codes */
   OB_K_TERNARY_UPDATE = 11,  /* momentum-error rule: update from the code sums */
-  OB_K_KINDS = 12
+  OB_K_TB_RESID_NORM = 12,   /* 2-bit: per-tile sums of the first plane's residual^2 */
+  OB_K_TB_PACK = 13,         /* 2-bit: both planes, worker error (+ server sums) */
+  OB_K_TB_SERVER_NORM = 14,  /* 2-bit: server sums (or residual sums) from the planes */
+  OB_K_TB_SERVER_UPDATE = 15,/* 2-bit: server planes + error, and/or the update */
+  OB_K_KINDS = 16
 };
 
 /* Start recording a CUDA event pair around each of the next `capacity`

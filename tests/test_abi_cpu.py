@@ -46,6 +46,11 @@ def test_layout_counts_code_words_under_the_momentum_rule():
     assert L.ob_layout(cfg) == 2
 
 
+def test_layout_counts_two_planes_under_the_two_bit_rule():
+    cfg, _k = L.make_config(100, [0, 33, 33, 97, 100], 3, rule=L.OB_RULE_TWO_BIT)
+    assert L.ob_layout(cfg) == 2 * (2 + 0 + 2 + 1)
+
+
 @pytest.mark.parametrize("kw,frag", [
     (dict(n=10, offsets=[0, 5, 9], W=1), "!= n"),
     (dict(n=10, offsets=[1, 10], W=1), "[0] must be 0"),
@@ -57,7 +62,7 @@ def test_layout_counts_code_words_under_the_momentum_rule():
     (dict(n=10, offsets=[0, 10], W=1, lr=float("nan")), "finite"),
     (dict(n=10, offsets=[0, 10], W=1, freeze_step=-1), "freeze_step"),
     (dict(n=-1, offsets=[0, -1], W=1), "n = -1"),
-    (dict(n=10, offsets=[0, 10], W=1, rule=2), "rule = 2"),
+    (dict(n=10, offsets=[0, 10], W=1, rule=3), "rule = 3"),
     (dict(n=10, offsets=[0, 10], W=128, rule=1), "W = 128 > 127"),
 ])
 def test_layout_rejects_bad_configs(kw, frag):

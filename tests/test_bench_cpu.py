@@ -54,3 +54,19 @@ def test_byte_model_of_the_one_pass_step():
     assert bench.step_bytes_per_elem(bl, "compressed", "momentum") == 16 * 12 + 20
     lamb = WL.get_workload("lamb-1.3b")
     assert bench.step_bytes_per_elem(lamb, "compressed", "momentum") == 4 * 12 + 16 + 16
+
+
+def test_byte_model_of_the_two_bit_step():
+    """Five passes: two worker norm passes, the two-plane pack, the server
+    residual norm and the server/update pass."""
+    sys.path.insert(0, ROOT)
+    import bench
+    import workloads as WL
+    wl = WL.get_workload("gpt2xl-flat")
+    assert bench.step_bytes_per_elem(wl, "compressed", "twobit") == 6 + 6 + 14.25 + 4.25 + 28.5
+
+
+def test_reference_arm_two_bit_rule():
+    d = run_bench("--impl", "reference", "--workload", "tiny", "--rule", "twobit", "--steps", "2",
+                  "--warmup", "3")
+    assert d["config"]["rule"] == "twobit" and d["value"] > 0

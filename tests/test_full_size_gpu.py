@@ -143,3 +143,43 @@ def test_full_size_momentum_rule(name):
             assert_state(tag + key, np_of(getattr(opt, key)[lo:hi]), ref[key], off)
         assert_state(tag + "err", np_of(opt.err[:, lo:hi]), ref["err"], off)
     opt.close()
+
+
+@pytest.mark.parametrize("name", ["gpt2xl-flat", "bert-large"])
+def test_full_size_two_bit_rule(name):
+    """2-bit Adam at full size (one compressed step from the seeded state),
+    compared with the oracle on sampled chunks."""
+    wl = WL.get_workload(name)
+    torch.cuda.empty_cache()
+    opt = OneBitAdam(wl.offsets, wl.W, grad_dtype=wl.grad_dtype, optimizer=wl.optimizer,
+                     clip=wl.clip, rule="twobit", device=dev(), **HP)
+    upload_state(wl, opt.p, opt.v)
+    gdt = torch.bfloat16 if wl.grad_dtype == "bf16" else torch.float32
+    G = torch.empty((wl.W, wl.n), dtype=gdt, device=dev())
+    upload_grads(wl, 0, G)
+    opt.step(G)
+    torch.cuda.synchronize()
+    assert opt.status() == 0
+    del G
+    o = oracle.get()
+    wb = np.zeros(wl.C + 1, np.int64)
+    np.cumsum([2 * ((s + 31) // 32) for s in wl.sizes], out=wb[1:])
+    opt_code = oracle.LAMB if wl.optimizer == "lamb" else oracle.ADAM
+    for k in sampled_chunks(wl):
+        nk = wl.sizes[k]
+        lo, hi = int(wl.offsets[k]), int(wl.offsets[k + 1])
+        off = np.array([0, nk], np.int64)
+        pk, vk = WL.chunk_state(wl, k)
+        ref = {"p": pk, "m": np.zeros(nk, np.float32), "v": vk,
+               "err": np.zeros((wl.W, nk), np.float32), "srv_err": np.zeros(nk, np.float32)}
+        g = np.stack([WL.chunk_grads(wl, 0, w, k) for w in range(wl.W)])
+        o.twobit_step(off, g, ref, F["beta1"], F["lr"], F["eps"], clip=wl.clip, optimizer=opt_code)
+        tag = f"{name} chunk {k}: "
+        for key in ("p", "m", "v", "srv_err"):
+            assert_state(tag + key, np_of(getattr(opt, key)[lo:hi]), ref[key], off)
+        assert_state(tag + "err", np_of(opt.err[:, lo:hi]), ref["err"], off)
+        assert_bits(tag + "bits_w", np_of(opt.bits_w[:, wb[k]:wb[k + 1]]), ref["bits_w"])
+        assert_bits(tag + "bits_srv", np_of(opt.bits_srv[wb[k]:wb[k + 1]]), ref["bits_srv"])
+        assert_scales(tag + "s_w", np_of(opt.s_w[:, k]), ref["s_w"][:, 0])
+        assert_scales(tag + "s_srv", np_of(opt.s_srv[k]), ref["s_srv"][0])
+    opt.close()
