@@ -186,24 +186,36 @@ class CudaStages:
             if warmup:
                 self.warm = L.ob_create(cfg(layout.offsets, W, 1 << 30), ptr(self.p), ptr(self.m),
                                         ptr(self.v), 0, 0, 0, 0, 0, 0)
+            # The momentum-error rule's update divides the code sums by W, so it runs
+            # on a ctx of W = world workers (the worker stage's ctx has one).  The
+            # scaled rules' update reads averaged scales: the local ctx serves.
+            self.update = 0
+            if momentum:
+                self.update = L.ob_create(cfg(layout.offsets, W, 0), ptr(self.p), ptr(self.m), ptr(self.v),
+                                          0, 0, 0, 0, ptr(self.bits_srv), 0)
             # One worker+update ctx per owner slice (views into the same buffers), so a
             # slice can be compressed and sent while the next one is compressed.  Element
             # arrays of a slice must start 32-byte aligned (16 bf16 elements).
             self.slice_ctx: Optional[List[int]] = None
+            self.slice_upd: Optional[List[int]] = None
             if pipelined and W > 1 and all(layout.eslice(o).start % 16 == 0 for o in range(W)):
-                self.slice_ctx = []
+                self.slice_ctx, self.slice_upd = [], []
                 for o in range(W):
                     ks, es, ws = layout.kslice(o), layout.eslice(o), layout.wslice(o)
                     if ks.stop == ks.start:
                         self.slice_ctx.append(0)
+                        self.slice_upd.append(0)
                         continue
                     so = layout.offsets[ks.start: ks.stop + 1] - es.start
                     e4, w4, k4 = 4 * es.start, 4 * ws.start, 4 * ks.start
                     at = lambda t, b: ptr(t) + b if t.numel() else 0  # noqa: E731
-                    self.slice_ctx.append(L.ob_create(
-                        cfg(so, 1, 0), at(self.p, e4), at(self.m, e4), at(self.v, e4),
-                        at(self.err, e4), 0, at(self.bits_w, w4), at(self.s_w, k4),
-                        at(self.bits_srv, w4), at(self.s_srv, k4)))
+                    h = L.ob_create(cfg(so, 1, 0), at(self.p, e4), at(self.m, e4), at(self.v, e4),
+                                    at(self.err, e4), 0, at(self.bits_w, w4), at(self.s_w, k4),
+                                    at(self.bits_srv, w4), at(self.s_srv, k4))
+                    self.slice_ctx.append(h)
+                    self.slice_upd.append(L.ob_create(cfg(so, W, 0), at(self.p, e4), at(self.m, e4),
+                                                      at(self.v, e4), 0, 0, 0, 0, at(self.bits_srv, w4), 0)
+                                          if momentum else h)
 
     def _stream(self) -> int:
         return int(torch.cuda.current_stream(self.device).cuda_stream)
@@ -223,15 +235,15 @@ class CudaStages:
             self.L.ob_compress(self.slice_ctx[o], int(grad_slice.data_ptr()), self._stream())
 
     def apply_slice(self, o: int) -> None:
-        if self.slice_ctx[o]:
-            self.L.ob_step(self.slice_ctx[o], None, self._stream())
+        if self.slice_upd[o]:
+            self.L.ob_step(self.slice_upd[o], None, self._stream())
 
     def server_reduce(self) -> None:
         if self.server:
             self.L.ob_server_reduce(self.server, self._stream())
 
     def apply(self) -> None:
-        self.L.ob_step(self.local, None, self._stream())
+        self.L.ob_step(self.update or self.local, None, self._stream())
 
     def status(self) -> int:
         st = self._stream()
@@ -240,21 +252,23 @@ class CudaStages:
             f |= self.L.ob_get_status(self.server, False, st)
         if self.warm:
             f |= self.L.ob_get_status(self.warm, False, st)
-        for h in self.slice_ctx or []:
+        if self.update:
+            f |= self.L.ob_get_status(self.update, False, st)
+        for h in set(self.slice_ctx or []) | set(self.slice_upd or []):
             if h:
                 f |= self.L.ob_get_status(h, False, st)
         return f
 
     def close(self) -> None:
-        for name in ("local", "server", "warm"):
+        for name in ("local", "server", "warm", "update"):
             h = getattr(self, name, 0)
             if h:
                 self.L.ob_destroy(h)
                 setattr(self, name, 0)
-        for h in self.slice_ctx or []:
+        for h in set(self.slice_ctx or []) | set(self.slice_upd or []):
             if h:
                 self.L.ob_destroy(h)
-        self.slice_ctx = None
+        self.slice_ctx = self.slice_upd = None
 
 
 # ---- the data-parallel optimizer -------------------------------------------------------
