@@ -398,7 +398,7 @@ def run_ours(args):
     torch.cuda.synchronize()
 
     # -- timed region: inputs resident in HBM ------------------------------------
-    per_step_launches = 8
+    per_step_launches = 16
     L.ob_profile_start(opt.ctx, args.steps * per_step_launches)
     launches0 = L.ob_launch_count(opt.ctx)
     sampler = ClockSampler(gpu_id(device))
