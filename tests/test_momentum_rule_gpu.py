@@ -252,3 +252,34 @@ def test_error_norms_of_worker_buffers():
     off = wl.offsets
     want = np.array([[np.sqrt((e[w, off[k]:off[k + 1]] ** 2).sum()) for k in range(wl.C)] for w in range(3)])
     assert np.allclose(np_of(wn), want, rtol=1e-6, atol=0)
+
+
+@pytest.mark.parametrize("rule", ["momentum", "twobit"])
+def test_step_replays_from_a_cuda_graph(rule):
+    """The fused step of the other rules captures into a CUDA graph too; replays
+    equal eager steps bit for bit."""
+    wl = WL.get_workload("tiny")
+    p, v = state_for(wl)
+    kw = dict(rule=rule, device=dev(), p=to_dev(p), v=to_dev(v), **HP)
+    eager = OneBitAdam(wl.offsets, wl.W, **kw)
+    graphed = OneBitAdam(wl.offsets, wl.W, **kw)
+    G = torch.empty((wl.W, wl.n), dtype=torch.float32, device=dev())
+    s = torch.cuda.Stream(device=dev())
+    s.wait_stream(torch.cuda.current_stream())
+    graph = torch.cuda.CUDAGraph()
+    G.copy_(to_dev(grads_for(wl, 0)))
+    with torch.cuda.stream(s):
+        graphed.step(G)
+    torch.cuda.current_stream().wait_stream(s)
+    with torch.cuda.graph(graph, stream=s):
+        graphed.step(G)
+    graphed.set_step(1)
+    eager.step(to_dev(grads_for(wl, 0)))
+    for t in range(1, 4):
+        gt = to_dev(grads_for(wl, t))
+        eager.step(gt)
+        G.copy_(gt)
+        graph.replay()
+    torch.cuda.synchronize()
+    for k in ("p", "m", "err"):
+        assert np.array_equal(np_of(getattr(eager, k)), np_of(getattr(graphed, k))), k
