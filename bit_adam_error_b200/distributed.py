@@ -62,6 +62,7 @@ class DPLayout:
     words: np.ndarray                # [C+1] packed-word offsets, layout order
     kbounds: Tuple[int, ...]         # [world+1] layout positions: rank r owns [kbounds[r], kbounds[r+1])
     codes_per_word: int = 32         # 32 sign bits, or 4 int8 codes (momentum-error rule)
+    planes: int = 1                  # sign planes per chunk (2: 2-bit Adam)
 
     @property
     def n(self) -> int:
@@ -88,13 +89,16 @@ class DPLayout:
         return self.order.index(k)
 
 
-def plan(sizes: Sequence[int], world: int, codes_per_word: int = 32) -> DPLayout:
+def plan(sizes: Sequence[int], world: int, codes_per_word: int = 32, planes: int = 1) -> DPLayout:
     """Assign chunks to ranks (largest first to the least-loaded rank, ties to the
     lower rank) and lay the buffer out grouped by owner.  ``codes_per_word``: 32
     for the sign bits of the scaled-sign rule, 4 for the int8 codes of the
-    momentum-error rule (every chunk starts on a fresh word either way)."""
+    momentum-error rule; ``planes``: 2 for the two sign planes of 2-bit Adam.
+    Every chunk starts on a fresh word."""
     if codes_per_word not in (4, 32):
         raise ValueError("codes_per_word must be 32 (sign bits) or 4 (int8 codes)")
+    if planes not in (1, 2) or (planes == 2 and codes_per_word != 32):
+        raise ValueError("planes must be 1, or 2 with sign bits")
     sizes = tuple(int(s) for s in sizes)
     if world < 1:
         raise ValueError("world must be >= 1")
@@ -110,11 +114,11 @@ def plan(sizes: Sequence[int], world: int, codes_per_word: int = 32) -> DPLayout
     np.cumsum(np.asarray(lay_sizes, np.int64), out=offsets[1:])
     words = np.zeros(len(sizes) + 1, np.int64)
     cpw = codes_per_word
-    np.cumsum(np.asarray([(s + cpw - 1) // cpw for s in lay_sizes], np.int64), out=words[1:])
+    np.cumsum(np.asarray([planes * ((s + cpw - 1) // cpw) for s in lay_sizes], np.int64), out=words[1:])
     kb = [0] * (world + 1)
     for r in range(world):
         kb[r + 1] = kb[r] + sum(1 for k in order if owner[k] == r)
-    return DPLayout(sizes, world, tuple(owner), order, offsets, words, tuple(kb), cpw)
+    return DPLayout(sizes, world, tuple(owner), order, offsets, words, tuple(kb), cpw, planes)
 
 
 # ---- CUDA stage backend ------------------------------------------------------------------
@@ -140,12 +144,16 @@ class CudaStages:
         self.device = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
         self.layout, self.rank = layout, rank
         W, n = layout.world, layout.n
-        momentum = rule == "momentum"
-        if layout.codes_per_word != (4 if momentum else 32):
-            raise ValueError(f"layout planned with {layout.codes_per_word} codes per word for rule {rule!r}")
-        # The momentum-error rule has no scales and no server error: those are empty.
+        momentum, twobit = rule == "momentum", rule == "twobit"
+        if (layout.codes_per_word, layout.planes) != ((4, 1) if momentum else (32, 2) if twobit else (32, 1)):
+            raise ValueError(f"layout planned with {layout.codes_per_word} codes per word and "
+                             f"{layout.planes} plane(s), not for rule {rule!r}")
+        # The momentum-error rule has no scales and no server error: those are
+        # empty.  2-bit Adam has two scales per chunk: [.., C, 2].
         C = 0 if momentum else layout.C
-        code_rule = L.OB_RULE_MOMENTUM_ERROR if momentum else L.OB_RULE_SCALED_SIGN
+        sp = (2,) if twobit else ()
+        code_rule = (L.OB_RULE_MOMENTUM_ERROR if momentum else L.OB_RULE_TWO_BIT if twobit
+                     else L.OB_RULE_SCALED_SIGN)
         gd = L.OB_BF16 if grad_dtype == "bf16" else L.OB_F32
         opt = L.OB_LAMB if optimizer == "lamb" else L.OB_ADAM
         hp = dict(lr=lr, beta1=beta1, beta2=beta2, eps=eps, clip=clip)
@@ -154,8 +162,8 @@ class CudaStages:
         z = lambda shape, dt=f32: torch.zeros(shape, dtype=dt, device=dev)  # noqa: E731
         self.p, self.m, self.v = z(n), z(n), z(n)
         self.err = z((1, n))
-        self.bits_w, self.s_w = z((1, words), i32), z((1, C))
-        self.bits_srv, self.s_srv = z(words, i32), z(C)
+        self.bits_w, self.s_w = z((1, words), i32), z((1, C, *sp))
+        self.bits_srv, self.s_srv = z(words, i32), z((C, *sp))
         ptr = lambda t: 0 if t is None or t.numel() == 0 else int(t.data_ptr())  # noqa: E731
         self._keep = []
 
@@ -175,8 +183,8 @@ class CudaStages:
             w_own = layout.wslice(rank).stop - layout.wslice(rank).start
             self.srv_err = z(0 if momentum else self.n_own)
             C_own_scales = 0 if momentum else self.C_own
-            self.bits_w_srv, self.s_w_srv = z((W, w_own), i32), z((W, C_own_scales))
-            self.bits_srv_own, self.s_srv_own = z(w_own, i32), z(C_own_scales)
+            self.bits_w_srv, self.s_w_srv = z((W, w_own), i32), z((W, C_own_scales, *sp))
+            self.bits_srv_own, self.s_srv_own = z(w_own, i32), z((C_own_scales, *sp))
             self.server = 0
             if self.C_own > 0:
                 self.server = L.ob_create(cfg(off_own, W, 0), 0, 0, 0, 0, ptr(self.srv_err),
@@ -207,7 +215,7 @@ class CudaStages:
                         self.slice_upd.append(0)
                         continue
                     so = layout.offsets[ks.start: ks.stop + 1] - es.start
-                    e4, w4, k4 = 4 * es.start, 4 * ws.start, 4 * ks.start
+                    e4, w4, k4 = 4 * es.start, 4 * ws.start, 4 * (2 if twobit else 1) * ks.start
                     at = lambda t, b: ptr(t) + b if t.numel() else 0  # noqa: E731
                     h = L.ob_create(cfg(so, 1, 0), at(self.p, e4), at(self.m, e4), at(self.v, e4),
                                     at(self.err, e4), 0, at(self.bits_w, w4), at(self.s_w, k4),

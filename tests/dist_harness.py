@@ -33,23 +33,24 @@ class OracleStages:
         self.opt = oracle.LAMB if optimizer == "lamb" else oracle.ADAM
         self.clip = clip
         self.device = torch.device("cpu")
-        self.momentum = rule == "momentum"
+        self.momentum, self.twobit = rule == "momentum", rule == "twobit"
         W, n = layout.world, layout.n
         C = 0 if self.momentum else layout.C
+        sp = (2,) if self.twobit else ()
         words = int(layout.words[-1])
         f32, i32 = torch.float32, torch.int32
         self.p, self.m, self.v = torch.zeros(n), torch.zeros(n), torch.zeros(n)
         self.err = torch.zeros((1, n))
-        self.bits_w, self.s_w = torch.zeros((1, words), dtype=i32), torch.zeros((1, C))
-        self.bits_srv, self.s_srv = torch.zeros(words, dtype=i32), torch.zeros(C)
+        self.bits_w, self.s_w = torch.zeros((1, words), dtype=i32), torch.zeros((1, C, *sp))
+        self.bits_srv, self.s_srv = torch.zeros(words, dtype=i32), torch.zeros((C, *sp))
         ks, wsl = layout.kslice(rank), layout.wslice(rank)
         self.off_own = layout.offsets[ks.start: ks.stop + 1] - layout.offsets[ks.start]
         c_own = 0 if self.momentum else ks.stop - ks.start
         self.srv_err = torch.zeros(0 if self.momentum else int(self.off_own[-1]))
         self.bits_w_srv = torch.zeros((W, wsl.stop - wsl.start), dtype=i32)
-        self.s_w_srv = torch.zeros((W, c_own), dtype=f32)
+        self.s_w_srv = torch.zeros((W, c_own, *sp), dtype=f32)
         self.bits_srv_own = torch.zeros(wsl.stop - wsl.start, dtype=i32)
-        self.s_srv_own = torch.zeros(c_own, dtype=f32)
+        self.s_srv_own = torch.zeros((c_own, *sp), dtype=f32)
         self.flags = 0
         self.pipelined = bool(pipelined) and layout.world > 1
 
@@ -76,8 +77,8 @@ class OracleStages:
             self.bits_w.numpy().view(np.int8)[:] = codes
             self.flags |= fl
             return
-        bits, s, fl = self.o.compress(self.layout.offsets, self._grad_rows(grad), self.err.numpy(),
-                                      clip=self.clip)
+        fn = self.o.twobit_compress if self.twobit else self.o.compress
+        bits, s, fl = fn(self.layout.offsets, self._grad_rows(grad), self.err.numpy(), clip=self.clip)
         self._u32(self.bits_w)[:] = bits
         self.s_w.numpy()[:] = s
         self.flags |= fl
@@ -98,8 +99,8 @@ class OracleStages:
             self.bits_w.numpy().view(np.int8)[0, 4 * wsl.start: 4 * wsl.stop] = codes[0]
             self.flags |= fl
             return
-        bits, s, fl = self.o.compress(self._slice_offsets(o), self._grad_rows(grad_slice), err,
-                                      clip=self.clip)
+        fn = self.o.twobit_compress if self.twobit else self.o.compress
+        bits, s, fl = fn(self._slice_offsets(o), self._grad_rows(grad_slice), err, clip=self.clip)
         self._u32(self.bits_w)[0, wsl] = bits[0]
         self.s_w.numpy()[0, ks] = s[0]
         self.flags |= fl
@@ -112,8 +113,9 @@ class OracleStages:
             return
         if self.s_w_srv.shape[1] == 0:
             return
-        bits, s, fl = self.o.server_reduce(self.off_own, np.ascontiguousarray(self._u32(self.bits_w_srv)),
-                                           np.ascontiguousarray(self.s_w_srv.numpy()), self.srv_err.numpy())
+        fn = self.o.twobit_server if self.twobit else self.o.server_reduce
+        bits, s, fl = fn(self.off_own, np.ascontiguousarray(self._u32(self.bits_w_srv)),
+                         np.ascontiguousarray(self.s_w_srv.numpy()), self.srv_err.numpy())
         self._u32(self.bits_srv_own)[:] = bits
         self.s_srv_own.numpy()[:] = s
         self.flags |= fl
@@ -128,7 +130,9 @@ class OracleStages:
             return
         args = (self.layout.offsets, self._u32(self.bits_srv), self.s_srv.numpy(), self.m.numpy(),
                 self.v.numpy(), self.p.numpy(), f["beta1"], f["lr"], f["eps"])
-        if self.opt:
+        if self.twobit:
+            self.flags |= self.o.twobit_apply(*args, optimizer=self.opt)[1]
+        elif self.opt:
             self.flags |= self.o.lamb_apply(*args)[1]
         else:
             self.flags |= self.o.adam_apply(*args)
@@ -147,7 +151,9 @@ class OracleStages:
             return
         args = (self._slice_offsets(o), self._u32(self.bits_srv)[wsl], self.s_srv.numpy()[ks],
                 self.m.numpy()[es], self.v.numpy()[es], self.p.numpy()[es], f["beta1"], f["lr"], f["eps"])
-        if self.opt:
+        if self.twobit:
+            self.flags |= self.o.twobit_apply(*args, optimizer=self.opt)[1]
+        elif self.opt:
             self.flags |= self.o.lamb_apply(*args)[1]
         else:
             self.flags |= self.o.adam_apply(*args)
@@ -194,7 +200,7 @@ def _rank_main(rank, world, port, sizes, wl_kw, steps, backend, device, q, die=N
         dist.init_process_group(backend, rank=rank, world_size=world,
                                 timeout=datetime.timedelta(seconds=timeout_s))
         wl = workload(sizes, world, **wl_kw)
-        layout = plan(sizes, world, 4 if rule == "momentum" else 32)
+        layout = plan(sizes, world, 4 if rule == "momentum" else 32, 2 if rule == "twobit" else 1)
         if device == "cpu":
             stages = OracleStages(layout, rank, optimizer=wl.optimizer, clip=wl.clip, pipelined=pipelined,
                                   rule=rule)
@@ -283,12 +289,15 @@ def reference(sizes, world, wl_kw, steps, rule="scaled"):
                      optimizer=opt)
         elif rule == "momentum":
             o.ternary_step(wl.offsets, g, st, f["beta1"], f["lr"], f["eps"], clip=wl.clip, optimizer=opt)
+        elif rule == "twobit":
+            o.twobit_step(wl.offsets, g, st, f["beta1"], f["lr"], f["eps"], clip=wl.clip, optimizer=opt)
         else:
             o.step(wl.offsets, g, st, f["beta1"], f["lr"], f["eps"], clip=wl.clip, optimizer=opt)
     return wl, st
 
 
 def compare(layout, wl, ref, outs, exact=True):
+    planes = layout.planes
     """Every rank's state against the W-worker oracle, mapped to layout order:
     bit for bit (exact) or to the parity bar of the GPU tests."""
     off = wl.offsets
@@ -299,7 +308,7 @@ def compare(layout, wl, ref, outs, exact=True):
 
     if "bits_srv" in ref:          # the scaled-sign rule: server words, scales, server error
         wb = np.zeros(wl.C + 1, np.int64)
-        np.cumsum([(s + 31) // 32 for s in wl.sizes], out=wb[1:])
+        np.cumsum([planes * ((s + 31) // 32) for s in wl.sizes], out=wb[1:])
         bits_ref = layout.to_layout([ref["bits_srv"][wb[k]:wb[k + 1]] for k in range(wl.C)]).astype(np.uint32)
         s_ref = np.array([ref["s_srv"][k] for k in layout.order], np.float32)
         srv_ref = lay(ref["srv_err"])

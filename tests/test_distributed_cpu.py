@@ -87,3 +87,22 @@ def test_plan_code_words():
     assert int(lay.words[-1]) == sum((s + 3) // 4 for s in SIZES)
     with pytest.raises(ValueError):
         plan(SIZES, 2, 8)
+    two = plan(SIZES, 3, 32, 2)
+    assert int(two.words[-1]) == sum(2 * ((s + 31) // 32) for s in SIZES)
+    with pytest.raises(ValueError):
+        plan(SIZES, 2, 4, 2)
+
+
+@pytest.mark.parametrize("pipelined", [False, True], ids=["grouped", "pipelined"])
+@pytest.mark.parametrize("world,wl_kw,steps", [
+    (2, dict(freeze_step=1), 3),
+    (3, dict(grad_dtype="bf16", clip=5.0, grad_dist="student_t_zeros", zero_frac=0.05), 3),
+    (3, dict(optimizer="lamb"), 2),
+])
+def test_two_bit_ranks_match_single_process_oracle(world, wl_kw, steps, pipelined):
+    """2-bit Adam across ranks: both planes and both scales of owned chunks to
+    the owners, the server planes back; bit for bit with the W-worker oracle."""
+    outs = run_ranks(SIZES, world, wl_kw, steps, pipelined=pipelined, rule="twobit")
+    wl, ref = reference(SIZES, world, wl_kw, steps, rule="twobit")
+    compare(plan(SIZES, world, 32, 2), wl, ref, outs)
+    assert all(o["flags"] == 0 for o in outs)

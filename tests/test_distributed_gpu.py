@@ -47,3 +47,16 @@ def test_gpu_ranks_momentum_rule(world, pipelined):
     assert all(o["flags"] == 0 for o in outs)
     want = "pipelined" if pipelined and world > 1 else "grouped"
     assert all(o["schedule"] == want for o in outs)
+
+
+@pytest.mark.parametrize("world,pipelined", [(1, True), (2, True), (3, False)])
+def test_gpu_ranks_two_bit_rule(world, pipelined):
+    backend = "nccl" if world == 1 else "gloo"
+    wl_kw = dict(grad_dtype="bf16", freeze_step=1)
+    outs = run_ranks(SIZES, world, wl_kw, 3, backend=backend, device="cuda:0", pipelined=pipelined,
+                     rule="twobit")
+    wl, ref = reference(SIZES, world, wl_kw, 3, rule="twobit")
+    compare(plan(SIZES, world, 32, 2), wl, ref, outs, exact=False)
+    assert all(o["flags"] == 0 for o in outs)
+    want = "pipelined" if pipelined and world > 1 else "grouped"
+    assert all(o["schedule"] == want for o in outs)
