@@ -131,8 +131,15 @@ class CudaStages:
     server (W = world, owned chunks only): srv_err, the W workers' words/scales
                     of the owned chunks (filled by exchange 1) -> server stage.
     warm   (W = world, shares p, m, v): the full-precision warmup step.
+    update (momentum-error rule only; W = world, shares p, m, v, bits_srv): the
+                    update divides the code sums by W, which the local ctx's W = 1
+                    would get wrong.
+    slice_ctx / slice_upd (pipelined schedule): the local (and update) ctxs again,
+                    one per owner slice, as views into the same buffers.
+    ``rule``: "scaled" (default), "momentum" or "twobit"; the layout must be
+    planned for it (codes per word, planes).
     Phases are the driver's: every ctx is created with freeze_step 0 (local,
-    server) or never leaving warmup (warm).
+    server, update) or never leaving warmup (warm).
     """
 
     def __init__(self, layout: DPLayout, rank: int, *, grad_dtype: str = "f32",
