@@ -553,9 +553,10 @@ def run_dp(args):
     import workloads as WL
     from bit_adam_error_b200.distributed import CudaStages, DistributedOneBitAdam, plan
     wl = select_workload(args).with_(W=world, freeze_step=0)
-    layout = plan(wl.sizes, world)
+    layout = plan(wl.sizes, world, 4 if args.rule == "momentum" else 32, 2 if args.rule == "twobit" else 1)
     stages = CudaStages(layout, rank, grad_dtype=wl.grad_dtype, optimizer=wl.optimizer, clip=wl.clip,
-                        lr=wl.lr, beta1=wl.beta1, beta2=wl.beta2, eps=wl.eps, warmup=False, device=device)
+                        lr=wl.lr, beta1=wl.beta1, beta2=wl.beta2, eps=wl.eps, warmup=False,
+                        rule=args.rule, device=device)
     bf = wl.grad_dtype == "bf16"
     gdt = torch.bfloat16 if bf else torch.float32
     nbuf = max(1, args.grad_buffers)
@@ -590,14 +591,18 @@ def run_dp(args):
     flags = drv.status()
     if rank == 0:
         own = [layout.eslice(r).stop - layout.eslice(r).start for r in range(world)]
-        line = {"metric": METRIC, "value": world * layout.n / (ms / 1e3) / 1e9, "unit": UNIT,
+        scales_per_chunk = {"scaled": 1, "momentum": 0, "twobit": 2}[args.rule]
+        # One job, one model of n parameters per step (the W = world workers are the
+        # ranks), so the rate is n / step time, as for W virtual workers on one GPU.
+        line = {"metric": METRIC, "value": layout.n / (ms / 1e3) / 1e9, "unit": UNIT,
                 "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
                 "data": "synthetic (seeded Philox streams; shapes and distributions of the workload)",
-                "config": dict(workload_config(wl, world), parallelism=f"dp{world}: worker w = rank w, "
-                               f"chunk-owner server stage, NCCL point-to-point exchanges",
+                "config": dict(workload_config(wl, world, args.rule),
+                               parallelism=f"dp{world}: worker w = rank w, chunk-owner server stage, "
+                                           f"NCCL point-to-point exchanges ({'pipelined' if stages.pipelined else 'grouped'})",
                                owned_elements=own),
-                "exchange_bytes_per_step_per_rank": 2 * 4 * (int(layout.words[-1]) + layout.C),
+                "exchange_bytes_per_step_per_rank": 2 * 4 * (int(layout.words[-1]) + scales_per_chunk * layout.C),
                 "status_flags": flags, "e2e": None}
         print(json.dumps(line), flush=True)
     stages.close()
