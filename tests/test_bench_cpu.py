@@ -70,3 +70,14 @@ def test_reference_arm_two_bit_rule():
     d = run_bench("--impl", "reference", "--workload", "tiny", "--rule", "twobit", "--steps", "2",
                   "--warmup", "3")
     assert d["config"]["rule"] == "twobit" and d["value"] > 0
+
+
+def test_small_workloads_are_timed_with_an_l2_flush():
+    sys.path.insert(0, ROOT)
+    import bench
+    import workloads as WL
+    assert bench.flushes_l2(WL.get_workload("tiny"))
+    assert "flushed" in bench.workload_config(WL.get_workload("tiny"), 1)["l2"]
+    for name in ("bert-base", "gpt2xl-flat", "bert-large", "lamb-1.3b"):
+        assert not bench.flushes_l2(WL.get_workload(name))
+        assert bench.workload_config(WL.get_workload(name), 1)["l2"].startswith("inputs larger than L2")
