@@ -10,7 +10,7 @@ when it has not been built.
 from . import _lib
 from ._lib import (  # noqa: F401
     OB_ADAM, OB_BF16, OB_ECUDA, OB_EINVAL, OB_ENOMEM, OB_EPHASE, OB_F32, OB_LAMB, OB_OK,
-    OB_STATUS_NONFINITE, OneBitError, make_config, ob_compress, ob_create, ob_destroy,
+    OB_RULE_MOMENTUM_ERROR, OB_RULE_SCALED_SIGN, OB_RULE_TWO_BIT, OB_STATUS_NONFINITE, OneBitError, make_config, ob_compress, ob_create, ob_destroy,
     ob_get_status, ob_get_step, ob_layout, ob_refresh_step, ob_server_reduce, ob_set_step,
     ob_step, ob_step_host, ob_warmup_step,
 )
