@@ -445,7 +445,9 @@ def run_ours(args):
 
     # Dominant kernel roofline (this rank's CUDA events on the launch stream).
     peak, peak_src = measured_peak()
-    dom = max(prof, key=lambda k: prof[k][0])
+    # Dominant kernel: the one with the most time among those that stream the
+    # step's bytes (on a launch-bound workload a finaliser can take longer).
+    dom = max((k for k in prof if algo_bytes_per_elem(k, wl) > 0), key=lambda k: prof[k][0])
     dom_ms = prof[dom][0] / prof[dom][1]
     dom_bytes = algo_bytes_per_elem(dom, wl) * n
     achieved = dom_bytes / (dom_ms / 1e3) / 1e9
