@@ -1,8 +1,9 @@
 """Data-parallel driver with the CUDA stages (one GPU here).
 
-world 1 over NCCL (the exchanges reduce to local copies) and world 2 over gloo
-with both ranks on the same GPU (packed words staged through host memory; no
-kernel waits on another process).  Every rank's state is compared with the
+world 1 over NCCL (the exchanges reduce to local copies) and worlds 2 and 3
+over gloo with all ranks on the same GPU (packed words staged through host
+memory; no kernel waits on another process), in the grouped and the pipelined
+schedule, for all three rules.  Every rank's state is compared with the
 single-process W-worker oracle at the GPU parity bar: sign words bit-exact,
 scales and state within 1e-5.
 """

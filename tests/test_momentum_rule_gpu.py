@@ -283,3 +283,28 @@ def test_step_replays_from_a_cuda_graph(rule):
     torch.cuda.synchronize()
     for k in ("p", "m", "err"):
         assert np.array_equal(np_of(getattr(eager, k)), np_of(getattr(graphed, k))), k
+
+
+@pytest.mark.parametrize("rule", ["momentum", "twobit"])
+def test_checkpoint_resume_bitwise(rule):
+    """10 steps equal 5 steps, state_dict, a fresh optimizer, load, 5 more steps."""
+    wl = small(ALIGNED, 2, freeze_step=2)
+    p, v = state_for(wl)
+    kw = dict(rule=rule, device=dev(), freeze_step=2, **HP)
+    a = OneBitAdam(wl.offsets, 2, p=to_dev(p), v=to_dev(v), **kw)
+    for t in range(10):
+        a.step(to_dev(grads_for(wl, t)))
+    b = OneBitAdam(wl.offsets, 2, p=to_dev(p), v=to_dev(v), **kw)
+    for t in range(5):
+        b.step(to_dev(grads_for(wl, t)))
+    sd = b.state_dict()
+    b.close()
+    assert ("srv_err" in sd) == (rule == "twobit")
+    c = OneBitAdam(wl.offsets, 2, **kw)
+    c.load_state_dict(sd)
+    assert c.step_count == 5
+    for t in range(5, 10):
+        c.step(to_dev(grads_for(wl, t)))
+    torch.cuda.synchronize()
+    for k in ("p", "m", "v", "err") + (("srv_err",) if rule == "twobit" else ()):
+        assert np.array_equal(np_of(getattr(a, k)), np_of(getattr(c, k))), k
