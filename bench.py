@@ -120,18 +120,38 @@ def algo_bytes_per_elem(kind: str, wl) -> float:
         return W / 4 + eb
     if kind == "k_tb_server_update":     # planes, srv_err r/w, server planes (+ m, v, p as Adam/LAMB)
         return W / 4 + 2 * eb + 1 / 4 + (16 if wl.optimizer == "lamb" else 20)
+    # W >= 4: pass 2 also stores c_srv (4 B); the server passes read it instead of
+    # the W workers' words and the server error
+    upd = 16 if wl.optimizer == "lamb" else 20
+    if kind == "k_worker_pack_cached":
+        return algo_bytes_per_elem("k_worker_pack", wl) + 4
+    if kind == "k_server_update_cached":  # c_srv, srv_err written, server signs, m, v, p
+        return 4 + eb + 1 / 8 + upd
+    if kind == "k_tb_pack_cached":
+        return algo_bytes_per_elem("k_tb_pack", wl) + 4
+    if kind == "k_tb_server_norm_cached":
+        return 4.0
+    if kind == "k_tb_server_update_cached":
+        return 4 + eb + 1 / 4 + upd
     return 0.0                           # finalisers: a few bytes per chunk
 
 
+CACHE_MIN_W = 4     # the library's fused step stores c_srv from this many workers on
+
+
 def step_bytes_per_elem(wl, phase: str = "compressed", rule: str = "scaled") -> float:
+    """The step's algorithmic bytes per element, from the kernels it launches
+    (bench.py also sums them from the kernels the timed steps actually ran)."""
     if phase == "refresh":
         return algo_bytes_per_elem("k_warmup", wl) + (16.0 if wl.optimizer == "lamb" else 0.0)
     if rule == "momentum":
         return algo_bytes_per_elem("k_ternary_step", wl) + (16.0 if wl.optimizer == "lamb" else 0.0)
+    cached = "_cached" if wl.W >= CACHE_MIN_W else ""
     if rule == "twobit":
-        kinds = ["k_worker_norm", "k_tb_resid_norm", "k_tb_pack", "k_tb_server_norm", "k_tb_server_update"]
+        kinds = ["k_worker_norm", "k_tb_resid_norm", "k_tb_pack" + cached, "k_tb_server_norm" + cached,
+                 "k_tb_server_update" + cached]
         return sum(algo_bytes_per_elem(k, wl) for k in kinds) + (16.0 if wl.optimizer == "lamb" else 0.0)
-    kinds = ["k_worker_norm", "k_worker_pack", "k_server_update"]
+    kinds = ["k_worker_norm", "k_worker_pack" + cached, "k_server_update" + cached]
     if wl.optimizer == "lamb":
         kinds.append("k_lamb_param")
     return sum(algo_bytes_per_elem(k, wl) for k in kinds)
@@ -462,7 +482,9 @@ def run_ours(args):
                    "algorithmic_GBps": (algo_bytes_per_elem(k, wl) * n / (v[0] / v[1] / 1e3) / 1e9)
                    if algo_bytes_per_elem(k, wl) else None}
                for k, v in prof.items()}
-    step_gbs = step_bytes_per_elem(wl, args.phase, args.rule) * n / (ms_max / 1e3) / 1e9
+    # Step bytes from the kernels the timed steps ran (the library picks the schedule).
+    step_bpe = sum(algo_bytes_per_elem(k, wl) * v[1] for k, v in prof.items()) / args.steps
+    step_gbs = step_bpe * n / (ms_max / 1e3) / 1e9
 
     # -- error-buffer monitoring (one call, timed alone) -----------------------------
     monitor = None
@@ -531,8 +553,7 @@ def run_ours(args):
                 "config": workload_config(wl, world, args.rule),
                 "phase": args.phase,
                 "hbm": {"step_achieved_GBps": step_gbs, "step_frac": step_gbs / peak,
-                        "algorithmic_bytes_per_elem": step_bytes_per_elem(wl, args.phase, args.rule),
-                        "peak": peak,
+                        "algorithmic_bytes_per_elem": step_bpe, "peak": peak,
                         "peak_source": peak_src},
                 "roofline": roofline, "kernels": kernels, "error_norms_call": monitor,
                 "cpu_baseline": cpu, "e2e": e2e,

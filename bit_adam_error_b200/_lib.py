@@ -72,7 +72,7 @@ _SIGS = {
     "ob_last_error": (ctypes.c_char_p, []),
 }
 
-OB_K_KINDS = 16
+OB_K_KINDS = 21
 
 _lib = None
 

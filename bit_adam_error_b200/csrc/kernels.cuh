@@ -391,12 +391,14 @@ k_finalize_ratio(Layout L, const double* __restrict__ partP, const double* __res
 // GP = groups of one tile whose loads are issued together: 1 keeps the kernel
 // under 80 registers (3 CTAs per SM), best when W is small and a tile carries few
 // bytes per instruction; 2 keeps more bytes in flight per warp, best for large W.
-template <typename GT, typename ET, bool SERVER, bool CLIP, bool POW2, int GP>
+// CACHE (with SERVER): also store c_srv to csrv[n], so pass 3 reads one float
+// per element instead of rebuilding the sum from the W workers' words.
+template <typename GT, typename ET, bool SERVER, bool CLIP, bool POW2, int GP, bool CACHE>
 __global__ void __launch_bounds__(kBlock, GP == 1 ? 3 : 2)
 k_worker_pack(Layout L, int W, const GT* __restrict__ grads, ET* __restrict__ err,
               const float* __restrict__ s_w, uint32_t* __restrict__ bits_w,
-              const ET* __restrict__ srv_err, double* __restrict__ part_srv, float clip,
-              uint32_t* __restrict__ status) {
+              const ET* __restrict__ srv_err, double* __restrict__ part_srv, float* __restrict__ csrv,
+              float clip, uint32_t* __restrict__ status) {
   const int lane = threadIdx.x & 31;
   const auto mean = make_mean<POW2>(W);
   int hint = 0;
@@ -454,10 +456,11 @@ k_worker_pack(Layout L, int W, const GT* __restrict__ grads, ET* __restrict__ er
           for (int u = 0; u < GP; ++u)
             if (in[u]) {
 #pragma unroll
-              for (int j = 0; j < 8; ++j) {
-                const float cs = mean(acc[u][j]) + sv[u][j];
-                tsum = fma(static_cast<double>(cs), static_cast<double>(cs), tsum);
+              for (int j = 0; j < 8; ++j) {        // c_srv in place of the sum
+                acc[u][j] = mean(acc[u][j]) + sv[u][j];
+                tsum = fma(static_cast<double>(acc[u][j]), static_cast<double>(acc[u][j]), tsum);
               }
+              if (CACHE) st8(csrv + tl.ck0 + tl.rel + (q0 + u) * kGroupElems + lane * kVec, acc[u]);
             }
         }
       }
@@ -485,6 +488,7 @@ k_worker_pack(Layout L, int W, const GT* __restrict__ grads, ET* __restrict__ er
         if (SERVER && inb) {
           const float cs = mean(acc) + ld1_ro(srv_err + tl.ck0 + i);
           tsum = fma(static_cast<double>(cs), static_cast<double>(cs), tsum);
+          if (CACHE) csrv[tl.ck0 + i] = cs;
         }
       }
     }
@@ -592,11 +596,13 @@ __device__ __forceinline__ void update_elem(float d, float& m, float v, float& p
 
 // FROM_WORKERS: c_srv from bits_w/s_w/srv_err, quantised with s_srv, bits_srv and
 // srv_err written (the compressed allreduce's second half).  Otherwise g_hat is
-// read back from bits_srv/s_srv (the update-only stage call).
-template <Upd U, bool FROM_WORKERS, bool POW2, typename ET>
+// read back from bits_srv/s_srv (the update-only stage call).  CACHED (with
+// FROM_WORKERS): c_srv is read from csrv, where pass 2 stored it, and srv_err is
+// only written.
+template <Upd U, bool FROM_WORKERS, bool POW2, typename ET, bool CACHED>
 __global__ void __launch_bounds__(kBlock, kUpdateMinBlocks)
 k_server_update(Layout L, int W, const uint32_t* __restrict__ bits_w, const float* __restrict__ s_w,
-                const float* __restrict__ s_srv, ET* __restrict__ srv_err,
+                const float* __restrict__ csrv, const float* __restrict__ s_srv, ET* __restrict__ srv_err,
                 uint32_t* __restrict__ bits_srv, float* __restrict__ m, const float* __restrict__ v,
                 float* __restrict__ p, Hyper h, double* __restrict__ partP,
                 double* __restrict__ partU, uint32_t* __restrict__ status) {
@@ -618,17 +624,18 @@ k_server_update(Layout L, int W, const uint32_t* __restrict__ bits_w, const floa
         const int64_t gi = tl.ck0 + i0;
         float sv[8], mv[8], vv[8], pv[8];
         if (in) {
-          if (FROM_WORKERS) ld8(srv_err + gi, sv);
+          if (FROM_WORKERS && !CACHED) ld8(srv_err + gi, sv);
+          if (FROM_WORKERS && CACHED) ld8_ro(csrv + gi, sv);      // sv holds c_srv itself
           if (U != Upd::kNone) { ld8(m + gi, mv); ld8_ro(v + gi, vv); ld8(p + gi, pv); }
         }
         uint32_t byte = 0;
         if (FROM_WORKERS) {
           float acc[8];
-          server_sum8(L, W, bits_w, s_w, tl, wrel, word_in, lane, acc);
+          if (!CACHED) server_sum8(L, W, bits_w, s_w, tl, wrel, word_in, lane, acc);
           if (in) {
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
-              const float cs = mean(acc[j]) + sv[j];
+              const float cs = CACHED ? sv[j] : mean(acc[j]) + sv[j];
               const bool b = cs >= 0.0f;
               const float d = signed_scale(b, s2);
               byte |= static_cast<uint32_t>(b) << j;
@@ -664,12 +671,13 @@ k_server_update(Layout L, int W, const uint32_t* __restrict__ bits_w, const floa
         if (FROM_WORKERS) {
           if (inb) {
             float acc = 0.0f;
-            for (int w = 0; w < W; ++w) {
-              const float s = __ldg(s_w + static_cast<int64_t>(w) * L.C + tl.k);
-              const uint32_t word = __ldg(bits_w + static_cast<int64_t>(w) * L.words + wi);
-              acc = acc + signed_scale((word >> lane) & 1u, s);
-            }
-            const float cs = mean(acc) + ld1(srv_err + gi);
+            if (!CACHED)
+              for (int w = 0; w < W; ++w) {
+                const float s = __ldg(s_w + static_cast<int64_t>(w) * L.C + tl.k);
+                const uint32_t word = __ldg(bits_w + static_cast<int64_t>(w) * L.words + wi);
+                acc = acc + signed_scale((word >> lane) & 1u, s);
+              }
+            const float cs = CACHED ? __ldg(csrv + gi) : mean(acc) + ld1(srv_err + gi);
             b = cs >= 0.0f;
             d = signed_scale(b, s2);
             st1(srv_err + gi, cs - d);

@@ -45,6 +45,11 @@ ob_err cuda_fail(cudaError_t e, const char* what) {
 // at a time, so 4 bytes suffice (slices of them can start on any word).
 constexpr uintptr_t kAlignElems = 32, kAlignWords = 4;
 
+// From this many workers on, the fused step's pass 2 stores c_srv (4 bytes per
+// element) and pass 3 reads it back instead of rebuilding the server sum from
+// the W workers' words, which is bound by per-element work at large W.
+constexpr int32_t kCacheMinW = 4;
+
 int64_t words_of(int64_t n) { return (n + 31) / 32; }
 
 bool momentum_rule(const ob_config* c) { return c->rule == OB_RULE_MOMENTUM_ERROR; }
@@ -133,6 +138,7 @@ struct ob_ctx {
   void* scratch = nullptr;
   ob::Layout L{};
   double *part_w = nullptr, *part_srv = nullptr, *partP = nullptr, *partU = nullptr;
+  float* csrv = nullptr;            // c_srv of the fused step's pass 2 (W >= kCacheMinW), else NULL
   float* ratio = nullptr;
   uint32_t* status = nullptr;
   ob::Hyper h{};
@@ -253,13 +259,18 @@ void enqueue_worker_t(ob_ctx* c, const GT* grads, bool with_server, cudaStream_t
   enqueue_finalize_scale(c, c->part_w, c->s_w, W, c->L.tp, 1, c->T, st);
   if (c->T > 0) {
     // The stage call (no server part) never uses the mean: one instantiation each.
-    const bool one = W <= kPackOneGroupMaxW;
-    auto k2 = with_server ? (one ? ob::k_worker_pack<GT, ET, true, CLIP, POW2, 1> : ob::k_worker_pack<GT, ET, true, CLIP, POW2, 2>)
-                          : (one ? ob::k_worker_pack<GT, ET, false, CLIP, false, 1> : ob::k_worker_pack<GT, ET, false, CLIP, false, 2>);
+    // Many workers: the fused step also stores c_srv for pass 3 (CACHE).
+    const bool one = W <= kPackOneGroupMaxW, cache = with_server && c->csrv;
+    auto k2 = with_server ? (cache ? (one ? ob::k_worker_pack<GT, ET, true, CLIP, POW2, 1, true>
+                                          : ob::k_worker_pack<GT, ET, true, CLIP, POW2, 2, true>)
+                                   : (one ? ob::k_worker_pack<GT, ET, true, CLIP, POW2, 1, false>
+                                          : ob::k_worker_pack<GT, ET, true, CLIP, POW2, 2, false>))
+                          : (one ? ob::k_worker_pack<GT, ET, false, CLIP, false, 1, false>
+                                 : ob::k_worker_pack<GT, ET, false, CLIP, false, 2, false>);
     const int g2 = grid_for(c, k2, c->T);
-    launch(c, OB_K_WORKER_PACK, st, [&] {
+    launch(c, cache ? OB_K_WORKER_PACK_CACHED : OB_K_WORKER_PACK, st, [&] {
       k2<<<g2, ob::kBlock, 0, st>>>(c->L, W, grads, err, c->s_w, c->bits_w, srv_err,
-                                    c->part_srv, c->h.clip, c->status);
+                                    c->part_srv, c->csrv, c->h.clip, c->status);
     });
   }
   if (with_server) enqueue_finalize_scale(c, c->part_srv, c->s_srv, 1, c->L.tp, 1, 0, st);
@@ -280,25 +291,36 @@ void enqueue_worker(ob_ctx* c, const GT* grads, bool with_server, cudaStream_t s
   else enqueue_worker_e<GT, float>(c, grads, with_server, st);
 }
 
-template <ob::Upd U, bool FROM_WORKERS, typename ET>
-void enqueue_server_update_e(ob_ctx* c, cudaStream_t st) {
-  auto k3 = pow2_workers(c) ? ob::k_server_update<U, FROM_WORKERS, true, ET>
-                            : ob::k_server_update<U, FROM_WORKERS, false, ET>;
+// CACHED: c_srv comes from c->csrv (the fused step's pass 2 stored it).
+template <ob::Upd U, bool FROM_WORKERS, typename ET, bool CACHED>
+void launch_server_update(ob_ctx* c, cudaStream_t st) {
+  auto k3 = pow2_workers(c) ? ob::k_server_update<U, FROM_WORKERS, true, ET, CACHED>
+                            : ob::k_server_update<U, FROM_WORKERS, false, ET, CACHED>;
   const int g3 = grid_for(c, k3, c->T);
   ET* srv_err = static_cast<ET*>(c->srv_err);
-  launch(c, OB_K_SERVER_UPDATE, st, [&] {
-    k3<<<g3, ob::kBlock, 0, st>>>(c->L, c->cfg.W, c->bits_w, c->s_w, c->s_srv, srv_err,
+  launch(c, CACHED ? OB_K_SERVER_UPDATE_CACHED : OB_K_SERVER_UPDATE, st, [&] {
+    k3<<<g3, ob::kBlock, 0, st>>>(c->L, c->cfg.W, c->bits_w, c->s_w, c->csrv, c->s_srv, srv_err,
                                   c->bits_srv, c->m, c->v, c->p, c->h, c->partP, c->partU,
                                   c->status);
   });
 }
 
+template <ob::Upd U, bool FROM_WORKERS, typename ET>
+void enqueue_server_update_e(ob_ctx* c, bool cached, cudaStream_t st) {
+  if constexpr (FROM_WORKERS) {
+    if (cached) launch_server_update<U, true, ET, true>(c, st);
+    else launch_server_update<U, true, ET, false>(c, st);
+  } else {
+    launch_server_update<U, false, ET, false>(c, st);
+  }
+}
+
 template <ob::Upd U, bool FROM_WORKERS>
-void enqueue_server_update(ob_ctx* c, cudaStream_t st) {
+void enqueue_server_update(ob_ctx* c, cudaStream_t st, bool cached = false) {
   if (c->T == 0) return;
   // The update-only call never reads the server error: one instantiation.
-  if (FROM_WORKERS && c->cfg.err_dtype == OB_BF16) enqueue_server_update_e<U, FROM_WORKERS, uint16_t>(c, st);
-  else enqueue_server_update_e<U, FROM_WORKERS, float>(c, st);
+  if (FROM_WORKERS && c->cfg.err_dtype == OB_BF16) enqueue_server_update_e<U, FROM_WORKERS, uint16_t>(c, cached, st);
+  else enqueue_server_update_e<U, FROM_WORKERS, float>(c, cached, st);
 }
 
 // LAMB: trust ratio per layer from the tile partials, then the parameter step.
@@ -316,11 +338,12 @@ void enqueue_lamb_param(ob_ctx* c, cudaStream_t st) {
 }
 
 // Update from the packed worker signs (fused) or from bits_srv (stage call).
+// from_workers is the fused step: its pass 2 stored c_srv when the ctx has csrv.
 void enqueue_update(ob_ctx* c, bool from_workers, cudaStream_t st) {
-  const bool lamb = c->cfg.optimizer == OB_LAMB;
+  const bool lamb = c->cfg.optimizer == OB_LAMB, cached = from_workers && c->csrv;
   if (from_workers) {
-    if (lamb) enqueue_server_update<ob::Upd::kLambM, true>(c, st);
-    else enqueue_server_update<ob::Upd::kAdam, true>(c, st);
+    if (lamb) enqueue_server_update<ob::Upd::kLambM, true>(c, st, cached);
+    else enqueue_server_update<ob::Upd::kAdam, true>(c, st, cached);
   } else {
     if (lamb) enqueue_server_update<ob::Upd::kLambM, false>(c, st);
     else enqueue_server_update<ob::Upd::kAdam, false>(c, st);
@@ -464,17 +487,26 @@ void enqueue_tb_worker_t(ob_ctx* c, const GT* grads, bool with_server, cudaStrea
     });
   }
   enqueue_finalize_scale(c, c->part_w, c->s_w, W, c->L.tp, 1, c->T, st, 2, 1);
+  const bool cache = with_server && c->csrv;       // many workers: keep c_srv for 2b and 3
   if (c->T > 0) {
-    auto k2 = with_server ? ob::k_tb_pack<GT, ET, true, CLIP, POW2> : ob::k_tb_pack<GT, ET, false, CLIP, false>;
+    auto k2 = !with_server ? ob::k_tb_pack<GT, ET, false, CLIP, false, false>
+              : cache      ? ob::k_tb_pack<GT, ET, true, CLIP, POW2, true>
+                           : ob::k_tb_pack<GT, ET, true, CLIP, POW2, false>;
     const int g2 = grid_for(c, k2, c->T);
-    launch(c, OB_K_TB_PACK, st, [&] {
+    launch(c, cache ? OB_K_TB_PACK_CACHED : OB_K_TB_PACK, st, [&] {
       k2<<<g2, ob::kBlock, 0, st>>>(c->L, W, grads, err, c->s_w, c->bits_w, srv_err, c->part_srv,
-                                    c->h.clip, c->status);
+                                    c->csrv, c->h.clip, c->status);
     });
   }
   if (!with_server) return;
   enqueue_finalize_scale(c, c->part_srv, c->s_srv, 1, c->L.tp, 1, 0, st, 2, 0);
-  if (c->T > 0) {
+  if (c->T > 0 && cache) {
+    auto k = ob::k_tb_server_norm_cached;
+    const int g = grid_for(c, k, c->T);
+    launch(c, OB_K_TB_SERVER_NORM_CACHED, st, [&] {
+      k<<<g, ob::kBlock, 0, st>>>(c->L, c->csrv, c->s_srv, c->part_srv);
+    });
+  } else if (c->T > 0) {
     auto k = ob::k_tb_server_norm<ET, POW2, true>;
     const int g = grid_for(c, k, c->T);
     launch(c, OB_K_TB_SERVER_NORM, st, [&] {
@@ -506,30 +538,40 @@ void enqueue_tb_worker(ob_ctx* c, const void* grads, bool with_server, cudaStrea
   }
 }
 
-template <ob::Upd U, bool FROM_WORKERS, typename ET>
-void enqueue_tb_server_update_e(ob_ctx* c, cudaStream_t st) {
+template <ob::Upd U, bool FROM_WORKERS, typename ET, bool CACHED>
+void launch_tb_server_update(ob_ctx* c, cudaStream_t st) {
   if (c->T == 0) return;
-  auto k = pow2_workers(c) ? ob::k_tb_server_update<U, FROM_WORKERS, true, ET>
-                           : ob::k_tb_server_update<U, FROM_WORKERS, false, ET>;
+  auto k = pow2_workers(c) ? ob::k_tb_server_update<U, FROM_WORKERS, true, ET, CACHED>
+                           : ob::k_tb_server_update<U, FROM_WORKERS, false, ET, CACHED>;
   const int g = grid_for(c, k, c->T);
-  launch(c, OB_K_TB_SERVER_UPDATE, st, [&] {
-    k<<<g, ob::kBlock, 0, st>>>(c->L, c->cfg.W, c->bits_w, c->s_w, c->s_srv, static_cast<ET*>(c->srv_err),
-                                c->bits_srv, c->m, c->v, c->p, c->h, c->partP, c->partU, c->status);
+  launch(c, CACHED ? OB_K_TB_SERVER_UPDATE_CACHED : OB_K_TB_SERVER_UPDATE, st, [&] {
+    k<<<g, ob::kBlock, 0, st>>>(c->L, c->cfg.W, c->bits_w, c->s_w, c->csrv, c->s_srv,
+                                static_cast<ET*>(c->srv_err), c->bits_srv, c->m, c->v, c->p, c->h,
+                                c->partP, c->partU, c->status);
   });
 }
 
+// cached: the fused step's pass 2 stored c_srv in c->csrv.
 template <ob::Upd U, bool FROM_WORKERS>
-void enqueue_tb_server_update(ob_ctx* c, cudaStream_t st) {
-  if (FROM_WORKERS && c->cfg.err_dtype == OB_BF16) enqueue_tb_server_update_e<U, FROM_WORKERS, uint16_t>(c, st);
-  else enqueue_tb_server_update_e<U, FROM_WORKERS, float>(c, st);
+void enqueue_tb_server_update(ob_ctx* c, cudaStream_t st, bool cached = false) {
+  const bool bf = FROM_WORKERS && c->cfg.err_dtype == OB_BF16;
+  if constexpr (FROM_WORKERS) {
+    if (cached) {
+      if (bf) launch_tb_server_update<U, true, uint16_t, true>(c, st);
+      else launch_tb_server_update<U, true, float, true>(c, st);
+      return;
+    }
+  }
+  if (bf) launch_tb_server_update<U, FROM_WORKERS, uint16_t, false>(c, st);
+  else launch_tb_server_update<U, FROM_WORKERS, float, false>(c, st);
 }
 
 // Update from the worker planes (fused step) or from bits_srv (stage call).
 void enqueue_tb_update(ob_ctx* c, bool from_workers, cudaStream_t st) {
-  const bool lamb = c->cfg.optimizer == OB_LAMB;
+  const bool lamb = c->cfg.optimizer == OB_LAMB, cached = from_workers && c->csrv;
   if (from_workers) {
-    if (lamb) enqueue_tb_server_update<ob::Upd::kLambM, true>(c, st);
-    else enqueue_tb_server_update<ob::Upd::kAdam, true>(c, st);
+    if (lamb) enqueue_tb_server_update<ob::Upd::kLambM, true>(c, st, cached);
+    else enqueue_tb_server_update<ob::Upd::kAdam, true>(c, st, cached);
   } else {
     if (lamb) enqueue_tb_server_update<ob::Upd::kLambM, false>(c, st);
     else enqueue_tb_server_update<ob::Upd::kAdam, false>(c, st);
@@ -713,7 +755,12 @@ ob_err ob_create(const ob_config* cfg, float* p, float* m, float* v, void* err, 
   const size_t sz_pw = up256(sizeof(double) * size_t(W) * size_t(c->T));
   const size_t sz_pt = up256(sizeof(double) * size_t(c->T));
   const size_t sz_ratio = up256(sizeof(float) * size_t(C));
-  const size_t total = 3 * sz_tab + sz_vec + sz_pw + 3 * sz_pt + sz_ratio + 256;
+  // c_srv cache of the fused step: scaled-sign rules with many workers, on a ctx
+  // that holds every buffer the fused step needs.
+  const bool fused_capable = p && m && v && err && srv_err && bits_w && s_w && bits_srv && s_srv;
+  const bool cache = !momentum_rule(cfg) && W >= kCacheMinW && fused_capable && n > 0;
+  const size_t sz_cs = cache ? up256(sizeof(float) * size_t(n)) : 0;
+  const size_t total = 3 * sz_tab + sz_vec + sz_pw + 3 * sz_pt + sz_ratio + sz_cs + 256;
   if ((e = cudaMalloc(&c->scratch, total)) != cudaSuccess) {
     cudaGetLastError();
     delete c;
@@ -729,6 +776,7 @@ ob_err ob_create(const ob_config* cfg, float* p, float* m, float* v, void* err, 
   c->partP = reinterpret_cast<double*>(base); base += sz_pt;
   c->partU = reinterpret_cast<double*>(base); base += sz_pt;
   c->ratio = reinterpret_cast<float*>(base); base += sz_ratio;
+  c->csrv = cache ? reinterpret_cast<float*>(base) : nullptr; base += sz_cs;
   c->status = reinterpret_cast<uint32_t*>(base);
 
   const struct { void* dst; const void* src; size_t bytes; } copies[] = {
@@ -1047,7 +1095,9 @@ const char* ob_kernel_name(int32_t kind) {
       "k_worker_norm", "k_finalize_scale", "k_worker_pack", "k_server_norm",
       "k_server_update", "k_lamb_param", "k_warmup", "k_finalize_ratio",
       "k_ternary_step", "k_ternary_compress", "k_ternary_server", "k_ternary_update",
-      "k_tb_resid_norm", "k_tb_pack", "k_tb_server_norm", "k_tb_server_update"};
+      "k_tb_resid_norm", "k_tb_pack", "k_tb_server_norm", "k_tb_server_update",
+      "k_worker_pack_cached", "k_server_update_cached", "k_tb_pack_cached", "k_tb_server_norm_cached",
+      "k_tb_server_update_cached"};
   return (kind >= 0 && kind < OB_K_KINDS) ? names[kind] : "";
 }
 
@@ -1108,8 +1158,8 @@ ob_err noalloc_setup(int device, NoAllocDevice** out) {
       return cuda_fail(e, "cudaDeviceGetAttribute");
     d.occ_norm[0] = occupancy(reinterpret_cast<const void*>(ob::k_worker_norm<float, float, true>));
     d.occ_norm[1] = occupancy(reinterpret_cast<const void*>(ob::k_worker_norm<uint16_t, float, true>));
-    d.occ_pack[0] = occupancy(reinterpret_cast<const void*>(ob::k_worker_pack<float, float, false, true, false, 2>));
-    d.occ_pack[1] = occupancy(reinterpret_cast<const void*>(ob::k_worker_pack<uint16_t, float, false, true, false, 2>));
+    d.occ_pack[0] = occupancy(reinterpret_cast<const void*>(ob::k_worker_pack<float, float, false, true, false, 2, false>));
+    d.occ_pack[1] = occupancy(reinterpret_cast<const void*>(ob::k_worker_pack<uint16_t, float, false, true, false, 2, false>));
     d.scratch = static_cast<char*>(ptr);
     d.ready = true;
   }
@@ -1208,10 +1258,10 @@ extern "C" ob_err ob_compress_noalloc(const ob_config* cfg, const void* grads, f
     const int g2 = noalloc_grid(d->num_sms, d->occ_pack[bf], T);
     const uint16_t* gh = static_cast<const uint16_t*>(grads);
     const float* gf = static_cast<const float*>(grads);
-    if (bf && cl) ob::k_worker_pack<uint16_t, float, false, true, false, 2><<<g2, ob::kBlock, 0, st>>>(L, int(W), gh, err, s_w, bits_w, nullptr, nullptr, clip, status);
-    else if (bf) ob::k_worker_pack<uint16_t, float, false, false, false, 2><<<g2, ob::kBlock, 0, st>>>(L, int(W), gh, err, s_w, bits_w, nullptr, nullptr, clip, status);
-    else if (cl) ob::k_worker_pack<float, float, false, true, false, 2><<<g2, ob::kBlock, 0, st>>>(L, int(W), gf, err, s_w, bits_w, nullptr, nullptr, clip, status);
-    else ob::k_worker_pack<float, float, false, false, false, 2><<<g2, ob::kBlock, 0, st>>>(L, int(W), gf, err, s_w, bits_w, nullptr, nullptr, clip, status);
+    if (bf && cl) ob::k_worker_pack<uint16_t, float, false, true, false, 2, false><<<g2, ob::kBlock, 0, st>>>(L, int(W), gh, err, s_w, bits_w, nullptr, nullptr, nullptr, clip, status);
+    else if (bf) ob::k_worker_pack<uint16_t, float, false, false, false, 2, false><<<g2, ob::kBlock, 0, st>>>(L, int(W), gh, err, s_w, bits_w, nullptr, nullptr, nullptr, clip, status);
+    else if (cl) ob::k_worker_pack<float, float, false, true, false, 2, false><<<g2, ob::kBlock, 0, st>>>(L, int(W), gf, err, s_w, bits_w, nullptr, nullptr, nullptr, clip, status);
+    else ob::k_worker_pack<float, float, false, false, false, 2, false><<<g2, ob::kBlock, 0, st>>>(L, int(W), gf, err, s_w, bits_w, nullptr, nullptr, nullptr, clip, status);
   }
   return check_launch("ob_compress_noalloc");
 }

@@ -106,11 +106,14 @@ k_tb_resid_norm(Layout L, int W, const GT* __restrict__ grads, const ET* __restr
 }
 
 // ---- pass 2: both planes, worker error (+ server sums) ---------------------------------
-template <typename GT, typename ET, bool SERVER, bool CLIP, bool POW2>
-__global__ void __launch_bounds__(kBlock)
+// CACHE (with SERVER): c_srv also goes to csrv[n] for passes 2b and 3.
+// Three CTAs per SM (at most 80 registers): the cached, clipped variant would
+// otherwise take 92 and drop to two.
+template <typename GT, typename ET, bool SERVER, bool CLIP, bool POW2, bool CACHE>
+__global__ void __launch_bounds__(kBlock, 3)
 k_tb_pack(Layout L, int W, const GT* __restrict__ grads, ET* __restrict__ err,
           const float* __restrict__ s_w, uint32_t* __restrict__ bits_w, const ET* __restrict__ srv_err,
-          double* __restrict__ part_srv, float clip, uint32_t* __restrict__ status) {
+          double* __restrict__ part_srv, float* __restrict__ csrv, float clip, uint32_t* __restrict__ status) {
   const int lane = threadIdx.x & 31;
   const auto mean = make_mean<POW2>(W);
   int hint = 0;
@@ -162,10 +165,11 @@ k_tb_pack(Layout L, int W, const GT* __restrict__ grads, ET* __restrict__ err,
         }
         if (SERVER && in) {
 #pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const float cs = mean(acc[j]) + sv[j];
-            tsum = fma(static_cast<double>(cs), static_cast<double>(cs), tsum);
+          for (int j = 0; j < 8; ++j) {            // c_srv in place of the sum
+            acc[j] = mean(acc[j]) + sv[j];
+            tsum = fma(static_cast<double>(acc[j]), static_cast<double>(acc[j]), tsum);
           }
+          if (CACHE) st8(csrv + tl.ck0 + i0, acc);
         }
       }
     } else {
@@ -199,6 +203,7 @@ k_tb_pack(Layout L, int W, const GT* __restrict__ grads, ET* __restrict__ err,
         if (SERVER && inb) {
           const float cs = mean(acc) + ld1_ro(srv_err + tl.ck0 + i);
           tsum = fma(static_cast<double>(cs), static_cast<double>(cs), tsum);
+          if (CACHE) csrv[tl.ck0 + i] = cs;
         }
       }
     }
@@ -261,13 +266,53 @@ k_tb_server_norm(Layout L, int W, const uint32_t* __restrict__ bits_w, const flo
   }
 }
 
+// Pass 2b when pass 2 stored c_srv: sum of (c_srv - s1' sign(c_srv))^2 from csrv.
+__global__ void __launch_bounds__(kBlock)
+k_tb_server_norm_cached(Layout L, const float* __restrict__ csrv, const float* __restrict__ s_srv,
+                        double* __restrict__ part) {
+  const int lane = threadIdx.x & 31;
+  int hint = 0;
+  for (int64_t t = warp_id(); t < L.T; t += warp_count()) {
+    const Tile tl = tile_at(L, t, hint);
+    const float s1 = __ldg(s_srv + 2 * tl.k);
+    double tsum = 0.0;
+    if (tl.vec) {
+#pragma unroll
+      for (int gq = 0; gq < kGroups; ++gq) {
+        const int64_t i0 = tl.rel + gq * kGroupElems + lane * kVec;
+        if (i0 < tl.nk) {
+          float cv[8];
+          ld8_ro(csrv + tl.ck0 + i0, cv);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const float x = cv[j] - signed_scale(cv[j] >= 0.0f, s1);
+            tsum = fma(static_cast<double>(x), static_cast<double>(x), tsum);
+          }
+        }
+      }
+    } else {
+      for (int j = 0; j < kTileWords; ++j) {
+        const int64_t i = tl.rel + j * 32 + lane;
+        if (i < tl.nk) {
+          const float cs = __ldg(csrv + tl.ck0 + i);
+          const float x = cs - signed_scale(cs >= 0.0f, s1);
+          tsum = fma(static_cast<double>(x), static_cast<double>(x), tsum);
+        }
+      }
+    }
+    tsum = warp_sum(tsum);
+    if (lane == 0) part[t] = tsum;
+  }
+}
+
 // ---- pass 3: server planes + server error, and/or the update --------------------------
 // FROM_WORKERS: c_srv from the worker planes and srv_err, quantised to two planes
 // with s_srv (bits_srv and srv_err written).  Otherwise g_hat from bits_srv.
-template <Upd U, bool FROM_WORKERS, bool POW2, typename ET>
+// CACHED (with FROM_WORKERS): c_srv read from csrv; srv_err only written.
+template <Upd U, bool FROM_WORKERS, bool POW2, typename ET, bool CACHED>
 __global__ void __launch_bounds__(kBlock, kUpdateMinBlocks)
 k_tb_server_update(Layout L, int W, const uint32_t* __restrict__ bits_w, const float* __restrict__ s_w,
-                   const float* __restrict__ s_srv, ET* __restrict__ srv_err,
+                   const float* __restrict__ csrv, const float* __restrict__ s_srv, ET* __restrict__ srv_err,
                    uint32_t* __restrict__ bits_srv, float* __restrict__ m, const float* __restrict__ v,
                    float* __restrict__ p, Hyper h, double* __restrict__ partP,
                    double* __restrict__ partU, uint32_t* __restrict__ status) {
@@ -291,17 +336,18 @@ k_tb_server_update(Layout L, int W, const uint32_t* __restrict__ bits_w, const f
         const int64_t gi = tl.ck0 + i0;
         float sv[8], mv[8], vv[8], pv[8];
         if (in) {
-          if (FROM_WORKERS) ld8(srv_err + gi, sv);
+          if (FROM_WORKERS && !CACHED) ld8(srv_err + gi, sv);
+          if (FROM_WORKERS && CACHED) ld8_ro(csrv + gi, sv);      // sv holds c_srv itself
           if (U != Upd::kNone) { ld8(m + gi, mv); ld8_ro(v + gi, vv); ld8(p + gi, pv); }
         }
         if (FROM_WORKERS) {
           float acc[8];
-          tb_server_sum8(L, W, bits_w, s_w, tl, wrel, nwk, word_in, lane, acc);
+          if (!CACHED) tb_server_sum8(L, W, bits_w, s_w, tl, wrel, nwk, word_in, lane, acc);
           uint32_t byte1 = 0, byte2 = 0;
           if (in) {
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
-              const float cs = mean(acc[j]) + sv[j];
+              const float cs = CACHED ? sv[j] : mean(acc[j]) + sv[j];
               const bool b1 = cs >= 0.0f;
               const float d1 = signed_scale(b1, s1);
               const float r = cs - d1;
@@ -345,7 +391,8 @@ k_tb_server_update(Layout L, int W, const uint32_t* __restrict__ bits_w, const f
         if (FROM_WORKERS) {
           bool b1 = false, b2 = false;
           if (inb) {
-            const float cs = mean(tb_server_sum1(L, W, bits_w, s_w, tl, wi, nwk, lane)) + ld1(srv_err + gi);
+            const float cs = CACHED ? __ldg(csrv + gi)
+                                    : mean(tb_server_sum1(L, W, bits_w, s_w, tl, wi, nwk, lane)) + ld1(srv_err + gi);
             b1 = cs >= 0.0f;
             const float d1 = signed_scale(b1, s1);
             const float r = cs - d1;

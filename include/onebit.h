@@ -141,7 +141,10 @@ ob_err ob_layout(const ob_config* cfg, int64_t* words_total);
  * Under OB_RULE_TWO_BIT: bits_w / bits_srv hold both planes (ob_layout words),
  * and s_w is [W][C][2], s_srv [C][2] (plane 1, plane 2 of each chunk).
  * Allocates the ctx scratch with cudaMalloc on the current device and
- * synchronises once.  *out receives the ctx (NULL on failure). */
+ * synchronises once.  The scratch holds the chunk tables and per-tile partial
+ * sums; with W >= 4 and every buffer of the fused step given (scaled-sign and
+ * 2-bit rules) it also holds one float per element for the fused step's server
+ * value.  *out receives the ctx (NULL on failure). */
 ob_err ob_create(const ob_config* cfg, float* p, float* m, float* v, void* err,
                  void* srv_err, uint32_t* bits_w, float* s_w, uint32_t* bits_srv,
                  float* s_srv, ob_ctx** out);
@@ -235,7 +238,15 @@ enum {
   OB_K_TB_PACK = 13,         /* 2-bit: both planes, worker error (+ server sums) */
   OB_K_TB_SERVER_NORM = 14,  /* 2-bit: server sums (or residual sums) from the planes */
   OB_K_TB_SERVER_UPDATE = 15,/* 2-bit: server planes + error, and/or the update */
-  OB_K_KINDS = 16
+  /* The fused step with W >= 4 workers: pass 2 also stores the server value
+   * c_srv (one float per element, in the ctx scratch) and the server passes read
+   * it instead of rebuilding it from the W workers' words. */
+  OB_K_WORKER_PACK_CACHED = 16,
+  OB_K_SERVER_UPDATE_CACHED = 17,
+  OB_K_TB_PACK_CACHED = 18,
+  OB_K_TB_SERVER_NORM_CACHED = 19,
+  OB_K_TB_SERVER_UPDATE_CACHED = 20,
+  OB_K_KINDS = 21
 };
 
 /* Start recording a CUDA event pair around each of the next `capacity`

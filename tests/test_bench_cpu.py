@@ -81,3 +81,14 @@ def test_small_workloads_are_timed_with_an_l2_flush():
     for name in ("bert-base", "gpt2xl-flat", "bert-large", "lamb-1.3b"):
         assert not bench.flushes_l2(WL.get_workload(name))
         assert bench.workload_config(WL.get_workload(name), 1)["l2"].startswith("inputs larger than L2")
+
+
+def test_byte_model_with_the_cached_server_value():
+    """From W = 4 on pass 2 also writes c_srv and pass 3 reads it instead of the
+    workers' words and the server error."""
+    sys.path.insert(0, ROOT)
+    import bench
+    import workloads as WL
+    bl = WL.get_workload("bert-large")          # W = 16, fp32 gradients and errors
+    assert bench.step_bytes_per_elem(bl) == 8 * 16 + (12 * 16 + 2 + 4 + 4) + (4 + 4 + 0.125 + 20)
+    assert bench.step_bytes_per_elem(bl.with_(W=2)) == 8 * 2 + (12 * 2 + 0.25 + 4) + (0.25 + 8 + 0.125 + 20)

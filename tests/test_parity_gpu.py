@@ -435,3 +435,23 @@ def test_error_norms_monitoring(layout):
     assert_scales("worker error norms", np_of(wn), want_w)
     assert_scales("server error norms", np_of(sn), want_s)
     assert np.all(np_of(wn)[:, np.diff(off) == 0] == 0)
+
+
+@pytest.mark.parametrize("W", [2, 4, 16])
+def test_fused_equals_stages_bitwise(W):
+    """From W = 4 on the fused step keeps the server value of pass 2 for pass 3
+    instead of rebuilding it from the workers' words; it must equal the stage
+    calls (which rebuild it) bit for bit, as it does below that."""
+    wl = small(RAGGED, W)
+    p, v = state_for(wl)
+    a = OneBitAdam(wl.offsets, W, device=dev(), p=to_dev(p), v=to_dev(v), **HP)
+    b = OneBitAdam(wl.offsets, W, device=dev(), p=to_dev(p), v=to_dev(v), **HP)
+    for t in range(3):
+        g = to_dev(grads_for(wl, t))
+        a.step(g)
+        b.compress(g)
+        b.server_reduce()
+        b.apply()
+    torch.cuda.synchronize()
+    for k in ("p", "m", "err", "srv_err", "bits_w", "s_w", "bits_srv", "s_srv"):
+        assert torch.equal(getattr(a, k), getattr(b, k)), k

@@ -176,11 +176,14 @@ def test_warmup_then_compressed():
     run_chain(small(ALIGNED, 4, freeze_step=2), 5)
 
 
-def test_fused_equals_stages():
-    wl = small(RAGGED, 3)
+@pytest.mark.parametrize("W", [3, 8])
+def test_fused_equals_stages(W):
+    """Bit for bit; from W = 4 on the fused step's server passes read the server
+    value pass 2 kept, the stage calls rebuild it."""
+    wl = small(RAGGED, W)
     p, v = state_for(wl)
-    a = make_gpu(wl.offsets, 3, p=to_dev(p), v=to_dev(v))
-    b = make_gpu(wl.offsets, 3, p=to_dev(p), v=to_dev(v))
+    a = make_gpu(wl.offsets, W, p=to_dev(p), v=to_dev(v))
+    b = make_gpu(wl.offsets, W, p=to_dev(p), v=to_dev(v))
     for t in range(3):
         g = to_dev(grads_for(wl, t))
         a.step(g)
