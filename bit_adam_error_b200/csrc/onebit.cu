@@ -1,8 +1,10 @@
 // onebit.cu -- host side of the C ABI declared in include/onebit.h.
 //
 // Validates arguments, owns the per-ctx scratch (chunk tables, per-tile partial
-// norms, LAMB ratios, status word) and enqueues the kernels of kernels.cuh on the
-// caller's stream.  After ob_create no call allocates device memory; the step
+// norms, LAMB ratios, status word, and for W >= 4 the fused step's server values)
+// and enqueues the kernels of the ctx's rule on the caller's stream: kernels.cuh
+// (scaled sign bits), ternary.cuh (the momentum-error rule's int8 codes),
+// twobit.cuh (2-bit Adam's two planes).  After ob_create no call allocates device memory; the step
 // calls only enqueue work.  ob_get_status synchronises the stream (one 4-byte
 // read-back); ob_step_host creates its copy stream and events on first use;
 // ob_profile_start/stop create, wait for and destroy CUDA events; ob_destroy
