@@ -8,7 +8,6 @@ and the two exchanges must not change a single operation.
 
 import time
 
-import numpy as np
 import pytest
 
 from bit_adam_error_b200.distributed import plan
