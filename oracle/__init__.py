@@ -22,6 +22,10 @@ import numpy as np
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "onebit_oracle.c")
 _LIB = os.path.join(_HERE, "libonebit_oracle.so")
+# The multi-threaded step (onebit_oracle_mt.c compiles onebit_oracle.c into the
+# same unit, so this library also exports every single-thread function).
+_SRC_MT = os.path.join(_HERE, "onebit_oracle_mt.c")
+_LIB_MT = os.path.join(_HERE, "libonebit_oracle_mt.so")
 
 F32, BF16 = 0, 1
 ADAM, LAMB = 0, 1
@@ -30,13 +34,27 @@ STATUS_NONFINITE = 1
 CFLAGS = ["-O2", "-ffp-contract=off", "-fno-fast-math", "-fPIC", "-shared", "-std=c11"]
 
 
-def build(force: bool = False, src: str = _SRC, out: str = _LIB, defines=()) -> str:
-    """Compile the oracle with gcc (no FMA contraction).  Returns the .so path."""
-    if not force and os.path.exists(out) and os.path.getmtime(out) >= os.path.getmtime(src):
+def build(force: bool = False, src: str = _SRC, out: str = _LIB, defines=(), threads: bool = False) -> str:
+    """Compile the oracle with gcc (no FMA contraction).  Returns the .so path.
+
+    ``threads``: the multi-threaded step (``onebit_oracle_mt.c``, linked with
+    ``-pthread``) when ``src``/``out`` are left at their defaults.
+    """
+    if threads and src == _SRC and out == _LIB:
+        src, out = _SRC_MT, _LIB_MT
+    deps = [src] + ([_SRC] if src == _SRC_MT else [])
+    if not force and os.path.exists(out) and all(os.path.getmtime(out) >= os.path.getmtime(d) for d in deps):
         return out
-    cmd = ["gcc", *CFLAGS, *[f"-D{d}" for d in defines], "-o", out, src, "-lm"]
+    extra = ["-pthread"] if src == _SRC_MT else []
+    cmd = ["gcc", *CFLAGS, *extra, *[f"-D{d}" for d in defines], "-o", out, src, "-lm"]
     subprocess.run(cmd, check=True)
     return out
+
+
+def build_all(force: bool = False) -> None:
+    """Both oracle libraries: the plain one and the multi-threaded step."""
+    build(force=force)
+    build(force=force, threads=True)
 
 
 _P = ctypes.c_void_p
@@ -67,6 +85,10 @@ _SIGS = {
     "orc_twobit_step": (_U32, [_I32, _I64, _I32, _P, _P, _I32, _I32, _F, _F, _F, _F,
                                _P, _P, _P, _P, _P, _I32, _P, _P, _P, _P]),
 }
+_SIGS_MT = {
+    "orc_step_mt": (_U32, [_I32, _I32, _I64, _I32, _P, _P, _I32, _I32, _F, _F, _F, _F,
+                           _P, _P, _P, _P, _P, _I32, _P, _P, _P, _P]),
+}
 
 MAX_TERNARY_WORKERS = 127   # the int8 sum of W codes in {-1, 0, 1} is exact up to here
 
@@ -77,7 +99,10 @@ class Oracle:
     def __init__(self, path: Optional[str] = None):
         self.path = path or build()
         self.lib = ctypes.CDLL(self.path)
-        for name, (res, args) in _SIGS.items():
+        sigs = dict(_SIGS)
+        if hasattr(self.lib, "orc_step_mt"):
+            sigs.update(_SIGS_MT)
+        for name, (res, args) in sigs.items():
             fn = getattr(self.lib, name)
             fn.restype = res
             fn.argtypes = args
@@ -170,10 +195,15 @@ class Oracle:
                                        self._dtype_of(grads), optimizer, beta1, beta2, lr, eps,
                                        self._ptr(m), self._ptr(v), self._ptr(p)))
 
-    def step(self, offsets, grads, state: dict, beta1, lr, eps, clip=0.0, optimizer=ADAM) -> int:
+    def step(self, offsets, grads, state: dict, beta1, lr, eps, clip=0.0, optimizer=ADAM,
+             threads: int = 1) -> int:
         """One compressed step.  ``state`` holds p, m, v, err, srv_err (updated in place;
         err and srv_err float32, or both uint16 bfloat16 patterns) and receives
-        bits_w, s_w, bits_srv, s_srv."""
+        bits_w, s_w, bits_srv, s_srv.
+
+        ``threads`` > 1 runs the multi-threaded step (bit-identical results); it
+        needs an ``Oracle`` loaded from the multi-threaded library (``get_mt()``).
+        """
         off = self._off(offsets)
         W, n = grads.shape
         C = len(off) - 1
@@ -182,13 +212,20 @@ class Oracle:
                                ("bits_srv", (words,), np.uint32), ("s_srv", (C,), np.float32)):
             if key not in state or state[key].shape != shape:
                 state[key] = np.zeros(shape, dt)
-        return int(self.lib.orc_step(
-            W, n, C, self._ptr(off), self._ptr(grads), self._dtype_of(grads), optimizer,
-            float(clip), beta1, lr, eps, self._ptr(state["p"]), self._ptr(state["m"]),
-            self._ptr(state["v"]), self._ptr(state["err"]), self._ptr(state["srv_err"]),
-            self._err_dtype(state["err"]),
-            self._ptr(state["bits_w"]), self._ptr(state["s_w"]), self._ptr(state["bits_srv"]),
-            self._ptr(state["s_srv"])))
+        args = (W, n, C, self._ptr(off), self._ptr(grads), self._dtype_of(grads), optimizer,
+                float(clip), beta1, lr, eps, self._ptr(state["p"]), self._ptr(state["m"]),
+                self._ptr(state["v"]), self._ptr(state["err"]), self._ptr(state["srv_err"]),
+                self._err_dtype(state["err"]),
+                self._ptr(state["bits_w"]), self._ptr(state["s_w"]), self._ptr(state["bits_srv"]),
+                self._ptr(state["s_srv"]))
+        if threads > 1:
+            if not hasattr(self.lib, "orc_step_mt"):
+                raise RuntimeError("this oracle build has no multi-threaded step; use oracle.get_mt()")
+            flags = int(self.lib.orc_step_mt(int(threads), *args))
+            if flags & 0x80000000:
+                raise MemoryError("orc_step_mt: scratch allocation failed")
+            return flags
+        return int(self.lib.orc_step(*args))
 
     # -- the momentum-error rule (int8 ternary codes) --------------------------------
     def code_words_total(self, offsets) -> int:
@@ -312,6 +349,7 @@ class Oracle:
 
 
 _default: Optional[Oracle] = None
+_default_mt: Optional[Oracle] = None
 
 
 def get() -> Oracle:
@@ -320,3 +358,20 @@ def get() -> Oracle:
     if _default is None:
         _default = Oracle()
     return _default
+
+
+def get_mt() -> Oracle:
+    """The multi-threaded build: every function of ``get()``, plus ``step(...,
+    threads=N)`` on N host threads."""
+    global _default_mt
+    if _default_mt is None:
+        _default_mt = Oracle(build(threads=True))
+    return _default_mt
+
+
+def host_threads() -> int:
+    """Threads this process may run on (its CPU affinity), at least 1."""
+    try:
+        return max(1, len(os.sched_getaffinity(0)))
+    except (AttributeError, OSError):
+        return max(1, os.cpu_count() or 1)
