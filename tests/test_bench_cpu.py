@@ -6,6 +6,8 @@ import subprocess
 import sys
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
 
 
 def run_bench(*args):
@@ -24,7 +26,11 @@ def test_reference_arm_json_line():
         assert key in d, key
     assert d["impl"] == "reference" and d["unit"] == "Gelem/s" and d["higher_is_better"] is True
     assert d["steps"] == 2 and d["warmup"] == 3 and d["value"] > 0
-    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] == 1
+    import oracle
+    assert d["cpu_baseline"]["kind"] == "oracle"
+    assert d["cpu_baseline"]["cores"] == oracle.host_threads()      # every host core
+    assert d["cpu_baseline"]["nproc"] == os.cpu_count()
+    assert "multi-threaded oracle step" in d["cpu_baseline"]["sample"]
     assert d["e2e"] == {"value": d["value"], "unit": "Gelem/s", "h2d_bytes_per_step": 0,
                         "d2h_bytes_per_step": 0}
     assert d["config"]["workload"].startswith("tiny")
@@ -92,3 +98,21 @@ def test_byte_model_with_the_cached_server_value():
     bl = WL.get_workload("bert-large")          # W = 16, fp32 gradients and errors
     assert bench.step_bytes_per_elem(bl) == 8 * 16 + (12 * 16 + 2 + 4 + 4) + (4 + 4 + 0.125 + 20)
     assert bench.step_bytes_per_elem(bl.with_(W=2)) == 8 * 2 + (12 * 2 + 0.25 + 4) + (0.25 + 8 + 0.125 + 20)
+
+
+def test_cpu_baseline_both_legs():
+    """The bench's cpu_baseline record: the single-thread leg and the all-cores
+    leg on the same chunk sample, the all-cores figure as its value."""
+    import types
+
+    import bench
+    import oracle
+    import workloads as WL
+    wl = WL.get_workload("tiny").with_(sizes=(70_000, 4_096, 33), W=2)
+    args = types.SimpleNamespace(phase="compressed", rule="scaled")
+    rec = bench.cpu_baseline(wl, args)
+    assert rec["kind"] == "oracle" and rec["unit"] == "Gelem/s"
+    assert rec["cores"] == oracle.host_threads() and rec["nproc"] == os.cpu_count()
+    one, allc = rec["legs"]
+    assert one["cores"] == 1 and allc["cores"] == rec["cores"]
+    assert rec["value"] == allc["value"] and one["value"] > 0 and allc["value"] > 0
