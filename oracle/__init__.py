@@ -85,6 +85,10 @@ _SIGS = {
     "orc_twobit_step": (_U32, [_I32, _I64, _I32, _P, _P, _I32, _I32, _F, _F, _F, _F,
                                _P, _P, _P, _P, _P, _I32, _P, _P, _P, _P]),
 }
+_SIGS.update({
+    "orc_sign_rates": (None, [_I32, _I32, _P, _I32, _P, _P]),
+    "orc_local_step": (_U32, [_I32, _I64, _I32, _P, _P, _I32, _I32, _F, _F, _F, _P, _P, _P, _P, _I32]),
+})
 _SIGS_MT = {
     "orc_step_mt": (_U32, [_I32, _I32, _I64, _I32, _P, _P, _I32, _I32, _F, _F, _F, _F,
                            _P, _P, _P, _P, _P, _I32, _P, _P, _P, _P]),
@@ -346,6 +350,30 @@ class Oracle:
             self._err_dtype(state["err"]),
             self._ptr(state["bits_w"]), self._ptr(state["s_w"]), self._ptr(state["bits_srv"]),
             self._ptr(state["s_srv"])))
+
+
+    # -- monitoring and 0/1 Adam's local step ----------------------------------------
+    def sign_rates(self, offsets, bits: np.ndarray, planes: int = 1) -> np.ndarray:
+        """Quantisation rate: per row, chunk and plane the fraction of the chunk's
+        elements whose sign bit is set.  ``bits`` [rows, words] (or one row).
+        Returns float32 [rows, C, planes]."""
+        off = self._off(offsets)
+        C = len(off) - 1
+        b = np.ascontiguousarray(np.atleast_2d(bits), dtype=np.uint32)
+        rows = b.shape[0]
+        out = np.zeros((rows, C, planes), np.float32)
+        self.lib.orc_sign_rates(rows, C, self._ptr(off), int(planes), self._ptr(b), self._ptr(out))
+        return out
+
+    def local_step(self, offsets, grads, state: dict, lr, eps, clip=0.0, optimizer=ADAM) -> int:
+        """0/1 Adam local step: err += clip(g) per worker; p moves with the current
+        m and v (both unchanged).  ``state`` holds p, m, v, err (in place)."""
+        off = self._off(offsets)
+        W, n = grads.shape
+        return int(self.lib.orc_local_step(
+            W, n, len(off) - 1, self._ptr(off), self._ptr(grads), self._dtype_of(grads), optimizer,
+            float(clip), lr, eps, self._ptr(state["p"]), self._ptr(state["m"]), self._ptr(state["v"]),
+            self._ptr(state["err"]), self._err_dtype(state["err"])))
 
 
 _default: Optional[Oracle] = None

@@ -646,3 +646,88 @@ uint32_t orc_twobit_step(int32_t W, int64_t n, int32_t C, const int64_t* off,
   flags |= orc_twobit_apply(n, C, off, bits_srv, s_srv, optimizer, beta1, lr, eps, m, v, p, NULL);
   return flags;
 }
+
+/* ---- monitoring: the quantisation rate ---------------------------------------------
+ *
+ * The CANN 1-bit Adam article, section 8 ("监控指标"), watches the gradient
+ * quantisation rate ("梯度量化率") next to the error-buffer L2 norm and expects it
+ * near its theoretical value.  The article gives no formula.  Reading: the
+ * rate of a chunk is the fraction of its n_k elements sent as +1, i.e. whose
+ * sign bit is set; for a message symmetric about zero its theoretical value is
+ * 1/2.  A rate far from 1/2 means the error feedback is carrying a bias.
+ *
+ * rows: packed rows, each laid out as the sign words are: chunk k starts at
+ * word planes * sum_{j<k} ceil(n_j / 32), its `planes` planes follow one
+ * another, ceil(n_k / 32) words each (planes = 2 for 2-bit Adam, else 1).
+ * rates[(r * C + k) * planes + p] = (float)((double)count / (double)n_k), the
+ * count taken over the n_k real bits only (padding bits never count); an
+ * empty chunk has rate 0.
+ */
+void orc_sign_rates(int32_t rows, int32_t C, const int64_t* off, int32_t planes,
+                    const uint32_t* bits, float* rates) {
+  int64_t row_words = 0;
+  for (int32_t k = 0; k < C; ++k) row_words += planes * words_of(off[k + 1] - off[k]);
+  for (int32_t r = 0; r < rows; ++r) {
+    int64_t base = (int64_t)r * row_words;
+    for (int32_t k = 0; k < C; ++k) {
+      int64_t nk = off[k + 1] - off[k], nw = words_of(nk);
+      for (int32_t pl = 0; pl < planes; ++pl) {
+        const uint32_t* q = bits + base + pl * nw;
+        int64_t count = 0;
+        for (int64_t i = 0; i < nk; ++i) count += sign_bit(q, i);
+        rates[((int64_t)r * C + k) * planes + pl] = nk > 0 ? (float)((double)count / (double)nk) : 0.0f;
+      }
+      base += planes * nw;
+    }
+  }
+}
+
+/* ---- 0/1 Adam: the local step ------------------------------------------------------
+ *
+ * "DeepSpeed Communication Compression and Hiding", section "0/1 Adam": 0/1
+ * Adam alternates full-precision variance refreshes with 1-bit synchronised
+ * steps, and adds local updates that lower the synchronisation frequency: its
+ * listing updates m only from a synchronised g_hat, applies
+ * param = adam_update(param, m, v) on every step, and notes that local steps
+ * may proceed before the next global synchronisation.  The page gives no
+ * formula for a local step.  Reading:
+ *   - a local step sends nothing;
+ *   - the parameters take the update of the listing's last line with the
+ *     current m and v, which stay as they are:
+ *       p = p - lr m / (sqrtf(v) + eps)
+ *     (1-bit LAMB: u = m / (sqrtf(v) + eps), r_l = ||p_l|| / ||u_l||,
+ *     p -= lr r_l u, as orc_lamb_apply);
+ *   - the gradient was not sent, so, as error feedback keeps whatever a step
+ *     did not transmit, each worker adds it to its error buffer and it reaches
+ *     the next synchronised step inside the compensated value:
+ *       err_w = clip(g_w) + err_w
+ *     (the same float addition the worker stage makes).
+ * Rules with additive error feedback only (the scaled-sign rule and 2-bit Adam).
+ * grads: [W][n]; err: [W][n] in/out.  Returns status flags (non-finite error or
+ * parameter).
+ */
+uint32_t orc_local_step(int32_t W, int64_t n, int32_t C, const int64_t* off, const void* grads,
+                        int32_t dtype, int32_t optimizer, float clip, float lr, float eps, float* p,
+                        const float* m, const float* v, void* err, int32_t err_dtype) {
+  uint32_t flags = 0;
+  for (int32_t w = 0; w < W; ++w)
+    for (int64_t i = 0; i < n; ++i) {
+      const int64_t e = (int64_t)w * n + i;
+      float kept = clip_grad(grad_at(grads, dtype, e), clip) + err_get(err, err_dtype, e);
+      if (is_nonfinite(kept)) flags |= ORC_STATUS_NONFINITE;
+      err_set(err, err_dtype, e, kept);
+    }
+  for (int32_t k = 0; k < C; ++k) {
+    int64_t o = off[k], nk = off[k + 1] - off[k];
+    if (optimizer == ORC_LAMB) {
+      flags |= lamb_update_layer(p + o, m + o, v + o, lr, eps, nk);
+      continue;
+    }
+    for (int64_t i = 0; i < nk; ++i) {
+      float pi = p[o + i] - lr * m[o + i] / (sqrtf(v[o + i]) + eps);
+      if (is_nonfinite(pi)) flags |= ORC_STATUS_NONFINITE;
+      p[o + i] = pi;
+    }
+  }
+  return flags;
+}

@@ -935,4 +935,143 @@ def pin_twobit_step_composition(o):
         assert np.array_equal(st["bits_srv"], bs) and np.array_equal(st["s_srv"], ss)
 
 
+
+
+# -- monitoring: the quantisation rate ---------------------------------------------------
+
+def pin_sign_rates_hand_cases(o):
+    """The hand-worked packing cases: rate = popcount / n (5/8, 17/33, 32/64)."""
+    cases = json.load(open(os.path.join(GOLDEN, "pack_hand_cases.json")))["cases"]
+    for case in cases:
+        c = _case_c(case)
+        n = len(c)
+        words = np.array([int(w, 16) for w in case["words"]], np.uint32)
+        rate = o.sign_rates([0, n], words)
+        assert rate.shape == (1, 1, 1)
+        assert float(rate[0, 0, 0]) == float(np.float32(Fraction(case["popcount"], n))), case["name"]
+
+
+def pin_sign_rates_count_real_bits_only(o):
+    """Rates count the n_k real bits of each chunk: set padding bits change
+    nothing; an empty chunk has rate 0; rows are independent."""
+    sizes = [33, 0, 64, 5, 100]
+    off, wb = offsets_of(sizes), word_base(sizes)
+    c = aux_normal(SEED, (300,), 2 * int(off[-1]), 1.0).reshape(2, -1)
+    rows = np.stack([np.concatenate([pack_ref(c[r, off[k]:off[k + 1]] >= 0) for k in range(len(sizes))])
+                     for r in range(2)])
+    want = np.zeros((2, len(sizes), 1), np.float32)
+    for r in range(2):
+        for k, nk in enumerate(sizes):
+            if nk:
+                want[r, k, 0] = np.float32(Fraction(int(np.count_nonzero(c[r, off[k]:off[k + 1]] >= 0)), nk))
+    assert np.array_equal(o.sign_rates(off, rows), want)
+    dirty = rows.copy()
+    for k, nk in enumerate(sizes):
+        if nk % 32:
+            dirty[:, wb[k + 1] - 1] |= np.uint32((0xFFFFFFFF << (nk % 32)) & 0xFFFFFFFF)
+    assert np.array_equal(o.sign_rates(off, dirty), want)
+    assert np.array_equal(o.sign_rates(off, rows[1]), want[1:2])
+
+
+def pin_sign_rates_of_the_stages(o):
+    """Worker rates equal the fraction of compensated values c >= 0 (numpy, from c
+    itself); the 2-bit layout has two planes per chunk, plane 1 the signs of c,
+    plane 2 the bits numpy unpacks from the second plane's words."""
+    W, sizes = 2, [70, 33, 0, 128]
+    off = offsets_of(sizes)
+    g, err0 = _worker_inputs(W, sizes, (301,))
+    err = err0.copy()
+    bits, _, _ = o.compress(off, g, err)
+    c = g + err0
+    rates = o.sign_rates(off, bits)
+    err2 = err0.copy()
+    bits2, _, _ = o.twobit_compress(off, g, err2)
+    rates2 = o.sign_rates(off, bits2, planes=2)
+    assert rates2.shape == (W, len(sizes), 2)
+    base = 0
+    for k, nk in enumerate(sizes):
+        nw = (nk + 31) // 32
+        for w in range(W):
+            want = np.float32(Fraction(int(np.count_nonzero(c[w, off[k]:off[k + 1]] >= 0)), nk)) if nk else 0.0
+            assert rates[w, k, 0] == want and rates2[w, k, 0] == want, (w, k)
+            plane2 = unpack_ref(bits2[w, base + nw: base + 2 * nw], nk)
+            want2 = np.float32(Fraction(int(plane2.sum()), nk)) if nk else 0.0
+            assert rates2[w, k, 1] == want2, (w, k)
+        base += 2 * nw
+
+
+# -- 0/1 Adam: the local step ------------------------------------------------------------
+
+def _local_state(sizes, W, key):
+    off = offsets_of(sizes)
+    n = int(off[-1])
+    return off, n, {"p": aux_normal(SEED, (key, 1), n, 0.02), "m": aux_normal(SEED, (key, 2), n, 1e-3),
+                    "v": aux_uniform(SEED, (key, 3), n, 1e-8, 1e-6),
+                    "err": aux_normal(SEED, (key, 4), W * n, 1e-3).reshape(W, n),
+                    "srv_err": aux_normal(SEED, (key, 5), n, 1e-4)}
+
+
+def pin_local_step_moves_p_with_the_current_momentum(o):
+    """A local step's parameter move is the compressed-phase update with beta1 = 1
+    (m kept, whatever g_hat): equal p bit for bit, Adam and LAMB; m and v are
+    untouched."""
+    sizes = [48, 33, 0, 64]
+    for opt in (0, 1):
+        off, n, st = _local_state(sizes, 2, 310 + opt)
+        m0, v0 = st["m"].copy(), st["v"].copy()
+        p_ref = st["p"].copy()
+        bits = _fixed_direction(sizes, (312,))
+        s = np.array([0.5, 0.25, 0.0, 0.125], np.float32)
+        if opt == 0:
+            o.adam_apply(off, bits, s, st["m"].copy(), st["v"], p_ref, np.float32(1.0), LR, EPS)
+        else:
+            o.lamb_apply(off, bits, s, st["m"].copy(), st["v"], p_ref, np.float32(1.0), LR, EPS)
+        g = aux_normal(SEED, (313,), 2 * n, 1e-3).reshape(2, n)
+        flags = o.local_step(off, g, st, LR, EPS, optimizer=opt)
+        assert flags == 0
+        assert np.array_equal(st["p"], p_ref), opt
+        assert np.array_equal(st["m"], m0) and np.array_equal(st["v"], v0)
+
+
+def pin_local_steps_telescope_with_error_feedback(o):
+    """Over a schedule mixing synchronised and local steps, the transmitted
+    directions still add up to all the gradients minus the final residuals:
+    sum over synchronised t of g_hat_t = mean_w(sum over all t of g_w,t - err_w,T)
+    - srv_err_T.  The local steps' gradients are not lost."""
+    W, sizes = 3, [50, 64, 33]
+    off, wb = offsets_of(sizes), word_base(sizes)
+    n = int(off[-1])
+    st = {"p": aux_normal(SEED, (320,), n, 0.02), "m": np.zeros(n, np.float32),
+          "v": aux_uniform(SEED, (321,), n, 1e-8, 1e-6),
+          "err": np.zeros((W, n), np.float32), "srv_err": np.zeros(n, np.float32)}
+    gsum = np.zeros((W, n))
+    ghat_sum = np.zeros(n)
+    for t, kind in enumerate("SLLSLSLLLS"):
+        g = aux_normal(SEED, (322, t), W * n, 1e-3).reshape(W, n)
+        gsum += g
+        if kind == "L":
+            assert o.local_step(off, g, st, LR, EPS) == 0
+            continue
+        o.step(off, g, st, B1, LR, EPS)
+        for k, nk in enumerate(sizes):
+            sg = np.where(unpack_ref(st["bits_srv"][wb[k]: wb[k + 1]], nk), 1.0, -1.0)
+            ghat_sum[off[k]: off[k + 1]] += float(st["s_srv"][k]) * sg
+    want = (gsum - st["err"]).mean(0) - st["srv_err"]
+    assert np.max(np.abs(ghat_sum - want)) <= 2e-8, np.max(np.abs(ghat_sum - want))
+
+
+def pin_local_step_clip_and_nonfinite(o):
+    """The kept gradient is clipped like the worker stage's (numpy's clamp), and
+    a NaN gradient raises the flag."""
+    sizes = [40]
+    off, n, st = _local_state(sizes, 1, 330)
+    g = aux_normal(SEED, (331,), n, 3.0).reshape(1, n)
+    e0 = st["err"].copy()
+    assert o.local_step(off, g, st, LR, EPS, clip=2.5) == 0
+    want = (np.clip(g, np.float32(-2.5), np.float32(2.5)).astype(np.float32) + e0).astype(np.float32)
+    assert np.array_equal(st["err"], want)
+    g[0, 7] = np.nan
+    assert o.local_step(off, g, st, LR, EPS) == 1
+
+
 ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_") and callable(v)]

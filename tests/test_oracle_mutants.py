@@ -87,6 +87,22 @@ MUTANTS = {
                                            "return dequantize(words, s[0], i);"),
     "twobit_second_plane_shifted": ("  quantize_signs(r, nk, words + nw);", "  quantize_signs(r, nk, words + nw - 1);"),
     "twobit_apply_word_step": ("    wo += 2 * nw;", "    wo += nw;"),
+    # the quantisation rate
+    "rates_count_padding": ("for (int64_t i = 0; i < nk; ++i) count += sign_bit(q, i);",
+                            "for (int64_t i = 0; i < 32 * nw; ++i) count += sign_bit(q, i);"),
+    "rates_plane_offset": ("const uint32_t* q = bits + base + pl * nw;", "const uint32_t* q = bits + base;"),
+    "rates_divisor": ("(float)((double)count / (double)nk)", "(float)((double)count / (double)(32 * nw))"),
+    "rates_row_stride": ("int64_t base = (int64_t)r * row_words;", "int64_t base = 0;"),
+    # 0/1 Adam's local step
+    "local_gradient_dropped": ("float kept = clip_grad(grad_at(grads, dtype, e), clip) + err_get(err, err_dtype, e);",
+                               "float kept = 0.0f + err_get(err, err_dtype, e);"),
+    "local_clip_ignored": ("float kept = clip_grad(grad_at(grads, dtype, e), clip) + err_get(err, err_dtype, e);",
+                           "float kept = grad_at(grads, dtype, e) + err_get(err, err_dtype, e);"),
+    "local_param_sign": ("float pi = p[o + i] - lr * m[o + i] / (sqrtf(v[o + i]) + eps);",
+                         "float pi = p[o + i] + lr * m[o + i] / (sqrtf(v[o + i]) + eps);"),
+    "local_lamb_skipped": ("      flags |= lamb_update_layer(p + o, m + o, v + o, lr, eps, nk);\n      continue;",
+                           "      continue;"),
+    "local_nan_not_flagged": ("if (is_nonfinite(kept)) flags |= ORC_STATUS_NONFINITE;", ""),
     "ternary_clip_after_error": ("float c = clip_grad(grad_at(grads, dtype, e), clip) + eps_old;",
                                  "float c = clip_grad(grad_at(grads, dtype, e) + eps_old, clip);"),
 }
