@@ -269,6 +269,16 @@ __device__ __forceinline__ void flag_nonfinite(bool bad, uint32_t* status) {
   if (__any_sync(kFull, bad) && (threadIdx.x & 31) == 0) atomicOr(status, kStatusNonfinite);
 }
 
+// Programmatic dependent launch: every kernel first waits until the kernels
+// before it in the stream have completed and their writes are visible (a no-op
+// when it was launched without the programmatic-serialization attribute), then
+// lets the next kernel's launch begin, so its set-up overlaps this kernel's
+// tail.  Nothing is read or written before the wait.
+__device__ __forceinline__ void pdl_enter() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 __device__ __forceinline__ int64_t warp_id() {
   return (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
 }
@@ -276,12 +286,55 @@ __device__ __forceinline__ int64_t warp_count() {
   return (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
 }
 
+// ---- fused finaliser (small problems) ---------------------------------------------
+// On small problems a separate finaliser launch costs as much as a pass, so the
+// pass's last CTA computes the scales itself.  Every thread fences its partial
+// stores; one thread per CTA then takes a ticket; the CTA that draws the last
+// ticket has every partial visible and turns each (row, chunk)'s tile partials
+// into its scale, one warp per (row, chunk): lane l sums slots tp[k] + l,
+// tp[k] + l + 32, ... in order, then the fixed xor butterfly of warp_sum, so
+// the scale is the same on every launch.  It resets the ticket for the next
+// launch.  No thread waits on another CTA.  The stage calls use the same
+// finaliser on the same problems, so the fused step and the stages agree bit
+// for bit.
+struct Fin {
+  unsigned* ticket;    // zero at the start of the launch (ctx scratch)
+  const double* part;  // [rows][row_stride] tile partials
+  int64_t row_stride;
+  int rows;
+  float* out;          // [rows][C]: ||.|| / sqrt(n_k)
+};
+
+__device__ __forceinline__ void fused_finalize(const Layout& L, const Fin& f) {
+  __shared__ unsigned s_last;
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) s_last = atomicAdd(f.ticket, 1u) == gridDim.x - 1 ? 1u : 0u;
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  for (int task = warp; task < f.rows * L.C; task += kWarpsPerBlock) {
+    const int r = task / L.C, k = task - r * L.C;
+    const double* pr = f.part + static_cast<int64_t>(r) * f.row_stride;
+    double acc = 0.0;
+    for (int64_t t = L.tp[k] + lane; t < L.tp[k + 1]; t += kWarp) acc += __ldcg(pr + t);
+    acc = warp_sum(acc);
+    if (lane == 0) {
+      const int64_t nk = L.off[k + 1] - L.off[k];
+      f.out[static_cast<int64_t>(r) * L.C + k] =
+          nk > 0 ? __double2float_rn(__ddiv_rn(__dsqrt_rn(acc), __dsqrt_rn(static_cast<double>(nk)))) : 0.0f;
+    }
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) *f.ticket = 0u;
+}
+
 // ---- pass 1: per-tile sum of c^2 for every worker ----------------------------------
 // part[w * T + t] = sum over tile t of (clip(g_w) + err_w)^2; a non-finite sum
 // (some c is NaN/Inf) raises the status flag.
 template <typename GT, typename ET, bool CLIP>
-__global__ void __launch_bounds__(kBlock)
-k_worker_norm(Layout L, int W, const GT* __restrict__ grads, const ET* __restrict__ err,
+__device__ __forceinline__ void worker_norm_tiles(Layout L, int W, const GT* __restrict__ grads, const ET* __restrict__ err,
               float clip, double* __restrict__ part, uint32_t* __restrict__ status) {
   const int lane = threadIdx.x & 31;
   const int64_t items = static_cast<int64_t>(W) * L.T;
@@ -325,6 +378,25 @@ k_worker_norm(Layout L, int W, const GT* __restrict__ grads, const ET* __restric
   }
 }
 
+template <typename GT, typename ET, bool CLIP>
+__global__ void __launch_bounds__(kBlock)
+k_worker_norm(Layout L, int W, const GT* __restrict__ grads, const ET* __restrict__ err,
+              float clip, double* __restrict__ part, uint32_t* __restrict__ status) {
+  pdl_enter();
+  worker_norm_tiles<GT, ET, CLIP>(L, W, grads, err, clip, part, status);
+}
+
+// Small problems: pass 1 and the worker scales (fin: rows = W, part, s_w) in one launch.
+template <typename GT, typename ET, bool CLIP>
+__global__ void __launch_bounds__(kBlock)
+k_worker_norm_fin(Layout L, int W, const GT* __restrict__ grads, const ET* __restrict__ err,
+              float clip, double* __restrict__ part, uint32_t* __restrict__ status, Fin fin) {
+  pdl_enter();
+  worker_norm_tiles<GT, ET, CLIP>(L, W, grads, err, clip, part, status);
+  fused_finalize(L, fin);
+}
+
+
 // ---- finalize: per-chunk scale from tile partials ----------------------------------
 // Partial slots of chunk k are [tpx[k] * mult, tpx[k+1] * mult) of each row (tpx =
 // warp-tile prefix with mult 1, or block-tile prefix with one slot per consumer
@@ -351,6 +423,7 @@ template <bool RMS>
 __global__ void __launch_bounds__(kFinalizeThreads)
 k_finalize_scale(Layout L, const double* __restrict__ part, const int64_t* __restrict__ tpx,
                  int mult, int64_t row_stride, float* __restrict__ out, int planes, int plane) {
+  pdl_enter();
   __shared__ double sm[kFinalizeThreads];
   const int k = blockIdx.x, r = blockIdx.y;
   const double* pr = part + static_cast<int64_t>(r) * row_stride;
@@ -370,6 +443,7 @@ k_finalize_scale(Layout L, const double* __restrict__ part, const int64_t* __res
 __global__ void __launch_bounds__(kFinalizeThreads)
 k_finalize_ratio(Layout L, const double* __restrict__ partP, const double* __restrict__ partU,
                  const int64_t* __restrict__ tpx, int mult, float* __restrict__ ratio) {
+  pdl_enter();
   __shared__ double sm[kFinalizeThreads];
   const int k = blockIdx.x;
   double a = 0.0, b = 0.0;
@@ -394,8 +468,7 @@ k_finalize_ratio(Layout L, const double* __restrict__ partP, const double* __res
 // CACHE (with SERVER): also store c_srv to csrv[n], so pass 3 reads one float
 // per element instead of rebuilding the sum from the W workers' words.
 template <typename GT, typename ET, bool SERVER, bool CLIP, bool POW2, int GP, bool CACHE>
-__global__ void __launch_bounds__(kBlock, GP == 1 ? 3 : 2)
-k_worker_pack(Layout L, int W, const GT* __restrict__ grads, ET* __restrict__ err,
+__device__ __forceinline__ void worker_pack_tiles(Layout L, int W, const GT* __restrict__ grads, ET* __restrict__ err,
               const float* __restrict__ s_w, uint32_t* __restrict__ bits_w,
               const ET* __restrict__ srv_err, double* __restrict__ part_srv, float* __restrict__ csrv,
               float clip, uint32_t* __restrict__ status) {
@@ -502,14 +575,43 @@ k_worker_pack(Layout L, int W, const GT* __restrict__ grads, ET* __restrict__ er
   }
 }
 
+template <typename GT, typename ET, bool SERVER, bool CLIP, bool POW2, int GP, bool CACHE>
+__global__ void __launch_bounds__(kBlock, GP == 1 ? 3 : 2)
+k_worker_pack(Layout L, int W, const GT* __restrict__ grads, ET* __restrict__ err,
+              const float* __restrict__ s_w, uint32_t* __restrict__ bits_w,
+              const ET* __restrict__ srv_err, double* __restrict__ part_srv, float* __restrict__ csrv,
+              float clip, uint32_t* __restrict__ status) {
+  pdl_enter();
+  worker_pack_tiles<GT, ET, SERVER, CLIP, POW2, GP, CACHE>(L, W, grads, err, s_w, bits_w, srv_err, part_srv, csrv, clip, status);
+}
+
+// Small problems (SERVER): pass 2 and the server scale (fin: rows = 1, part_srv, s_srv) in one launch.
+template <typename GT, typename ET, bool SERVER, bool CLIP, bool POW2, int GP, bool CACHE>
+__global__ void __launch_bounds__(kBlock, GP == 1 ? 3 : 2)
+k_worker_pack_fin(Layout L, int W, const GT* __restrict__ grads, ET* __restrict__ err,
+              const float* __restrict__ s_w, uint32_t* __restrict__ bits_w,
+              const ET* __restrict__ srv_err, double* __restrict__ part_srv, float* __restrict__ csrv,
+              float clip, uint32_t* __restrict__ status, Fin fin) {
+  pdl_enter();
+  worker_pack_tiles<GT, ET, SERVER, CLIP, POW2, GP, CACHE>(L, W, grads, err, s_w, bits_w, srv_err, part_srv, csrv, clip, status);
+  fused_finalize(L, fin);
+}
+
+
 // ---- server average recomputed from the packed worker signs ---------------------------
 // acc[j] = sum_w s_w[w][k] * sign_w(element), in ascending w (the same float
 // additions pass 2 made), for the 8 elements of this lane in group (rel0).
+// W1: exactly one worker, known at compile time -- the loop and its per-worker
+// address arithmetic disappear (acc is still 0.0f + the one scaled sign, the
+// same float operation), which is what lets pass 3 at W = 1 keep two groups of
+// loads in flight under 96 registers.
+template <bool W1>
 __device__ __forceinline__ void server_sum8(const Layout& L, int W, const uint32_t* __restrict__ bits_w,
                                             const float* __restrict__ s_w, const Tile& tl,
                                             int64_t wrel, bool word_in, int lane, float (&acc)[8]) {
   zero8(acc);
-  for (int w = 0; w < W; ++w) {
+  const int nw = W1 ? 1 : W;
+  for (int w = 0; w < nw; ++w) {
     const float s = __ldg(s_w + static_cast<int64_t>(w) * L.C + tl.k);
     const uint32_t word =
         word_in ? __ldg(bits_w + static_cast<int64_t>(w) * L.words + tl.w0 + wrel) : 0u;
@@ -521,8 +623,7 @@ __device__ __forceinline__ void server_sum8(const Layout& L, int W, const uint32
 
 // Server norm only (stage-wise call): part_srv[t] = sum over the tile of c_srv^2.
 template <typename ET, bool POW2>
-__global__ void __launch_bounds__(kBlock)
-k_server_norm(Layout L, int W, const uint32_t* __restrict__ bits_w, const float* __restrict__ s_w,
+__device__ __forceinline__ void server_norm_tiles(Layout L, int W, const uint32_t* __restrict__ bits_w, const float* __restrict__ s_w,
               const ET* __restrict__ srv_err, double* __restrict__ part_srv,
               uint32_t* __restrict__ status) {
   const int lane = threadIdx.x & 31;
@@ -537,7 +638,7 @@ k_server_norm(Layout L, int W, const uint32_t* __restrict__ bits_w, const float*
         const int64_t i0 = tl.rel + q * kGroupElems + lane * kVec;
         const int64_t wrel = (tl.rel + q * kGroupElems) / 32 + (lane >> 2);
         float acc[8];
-        server_sum8(L, W, bits_w, s_w, tl, wrel, wrel * 32 < tl.nk, lane, acc);
+        server_sum8<false>(L, W, bits_w, s_w, tl, wrel, wrel * 32 < tl.nk, lane, acc);
         if (i0 < tl.nk) {
           float sv[8];
           ld8_ro(srv_err + tl.ck0 + i0, sv);
@@ -571,6 +672,28 @@ k_server_norm(Layout L, int W, const uint32_t* __restrict__ bits_w, const float*
   }
 }
 
+template <typename ET, bool POW2>
+__global__ void __launch_bounds__(kBlock)
+k_server_norm(Layout L, int W, const uint32_t* __restrict__ bits_w, const float* __restrict__ s_w,
+              const ET* __restrict__ srv_err, double* __restrict__ part_srv,
+              uint32_t* __restrict__ status) {
+  pdl_enter();
+  server_norm_tiles<ET, POW2>(L, W, bits_w, s_w, srv_err, part_srv, status);
+}
+
+// Small problems: the server sums and the server scale in one launch (the stage
+// call's counterpart of k_worker_pack_fin, so both give the same scale).
+template <typename ET, bool POW2>
+__global__ void __launch_bounds__(kBlock)
+k_server_norm_fin(Layout L, int W, const uint32_t* __restrict__ bits_w, const float* __restrict__ s_w,
+              const ET* __restrict__ srv_err, double* __restrict__ part_srv,
+              uint32_t* __restrict__ status, Fin fin) {
+  pdl_enter();
+  server_norm_tiles<ET, POW2>(L, W, bits_w, s_w, srv_err, part_srv, status);
+  fused_finalize(L, fin);
+}
+
+
 // ---- pass 3: server pack + update ------------------------------------------------------
 enum class Upd : int {
   kNone = 0,   // server pack + server error only (stage-wise call)
@@ -598,14 +721,15 @@ __device__ __forceinline__ void update_elem(float d, float& m, float v, float& p
 // srv_err written (the compressed allreduce's second half).  Otherwise g_hat is
 // read back from bits_srv/s_srv (the update-only stage call).  CACHED (with
 // FROM_WORKERS): c_srv is read from csrv, where pass 2 stored it, and srv_err is
-// only written.
-template <Upd U, bool FROM_WORKERS, bool POW2, typename ET, bool CACHED>
+// only written.  W1 (with FROM_WORKERS, POW2): one worker (see server_sum8).
+template <Upd U, bool FROM_WORKERS, bool POW2, typename ET, bool CACHED, bool W1>
 __global__ void __launch_bounds__(kBlock, kUpdateMinBlocks)
 k_server_update(Layout L, int W, const uint32_t* __restrict__ bits_w, const float* __restrict__ s_w,
                 const float* __restrict__ csrv, const float* __restrict__ s_srv, ET* __restrict__ srv_err,
                 uint32_t* __restrict__ bits_srv, float* __restrict__ m, const float* __restrict__ v,
                 float* __restrict__ p, Hyper h, double* __restrict__ partP,
                 double* __restrict__ partU, uint32_t* __restrict__ status) {
+  pdl_enter();
   const int lane = threadIdx.x & 31;
   const auto mean = make_mean<POW2>(W);
   int hint = 0;
@@ -631,7 +755,7 @@ k_server_update(Layout L, int W, const uint32_t* __restrict__ bits_w, const floa
         uint32_t byte = 0;
         if (FROM_WORKERS) {
           float acc[8];
-          if (!CACHED) server_sum8(L, W, bits_w, s_w, tl, wrel, word_in, lane, acc);
+          if (!CACHED) server_sum8<W1>(L, W, bits_w, s_w, tl, wrel, word_in, lane, acc);
           if (in) {
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
@@ -672,7 +796,7 @@ k_server_update(Layout L, int W, const uint32_t* __restrict__ bits_w, const floa
           if (inb) {
             float acc = 0.0f;
             if (!CACHED)
-              for (int w = 0; w < W; ++w) {
+              for (int w = 0; w < (W1 ? 1 : W); ++w) {
                 const float s = __ldg(s_w + static_cast<int64_t>(w) * L.C + tl.k);
                 const uint32_t word = __ldg(bits_w + static_cast<int64_t>(w) * L.words + wi);
                 acc = acc + signed_scale((word >> lane) & 1u, s);
@@ -708,6 +832,7 @@ k_server_update(Layout L, int W, const uint32_t* __restrict__ bits_w, const floa
 template <typename ET>
 __global__ void __launch_bounds__(kBlock)
 k_rows_sumsq(Layout L, int R, const ET* __restrict__ x, double* __restrict__ part) {
+  pdl_enter();
   const int lane = threadIdx.x & 31;
   const int64_t items = static_cast<int64_t>(R) * L.T;
   int hint = 0;
@@ -742,11 +867,148 @@ k_rows_sumsq(Layout L, int R, const ET* __restrict__ x, double* __restrict__ par
   }
 }
 
+// ---- monitoring: the quantisation rate ------------------------------------------------------
+// The rate of a chunk is the fraction of its n_k elements sent as +1 (sign bit
+// set); for a message symmetric about zero its theoretical value is 1/2.
+// part[r * T + t] = set bits among the real elements of warp tile t in plane
+// `plane` of packed row r (chunk k's plane p starts at word wo[k] + p ceil(n_k / 32)).
+// Bits past n_k are masked off; a count is exact in a double.
+__global__ void __launch_bounds__(kBlock)
+k_sign_count(Layout L, int R, const uint32_t* __restrict__ bits, int plane, double* __restrict__ part) {
+  pdl_enter();
+  const int lane = threadIdx.x & 31;
+  const int64_t items = static_cast<int64_t>(R) * L.T;
+  int hint = 0;
+  for (int64_t it = warp_id(); it < items; it += warp_count()) {
+    const int r = static_cast<int>(it / L.T);
+    const int64_t t = it - static_cast<int64_t>(r) * L.T;
+    const Tile tl = tile_at(L, t, hint);
+    const int64_t nwk = (tl.nk + 31) / 32;
+    const int64_t wi = tl.rel / 32 + lane;        // lanes 0..15 hold the tile's words
+    unsigned cnt = 0;
+    if (lane < kTileWords && wi < nwk) {
+      uint32_t word = __ldg(bits + static_cast<int64_t>(r) * L.words + tl.w0 + plane * nwk + wi);
+      const int64_t left = tl.nk - wi * 32;       // real bits in this word
+      if (left < 32) word &= (1u << left) - 1u;
+      cnt = __popc(word);
+    }
+    cnt = __reduce_add_sync(kFull, cnt);
+    if (lane == 0) part[it] = static_cast<double>(cnt);
+  }
+}
+
+// out[(r * C + k) * planes + plane] = (float)(count / n_k) (double division, one
+// rounding), 0 for an empty chunk.  grid = (C, R).
+__global__ void __launch_bounds__(kFinalizeThreads)
+k_finalize_rate(Layout L, const double* __restrict__ part, int64_t row_stride, float* __restrict__ out,
+                int planes, int plane) {
+  pdl_enter();
+  __shared__ double sm[kFinalizeThreads];
+  const int k = blockIdx.x, r = blockIdx.y;
+  const double* pr = part + static_cast<int64_t>(r) * row_stride;
+  double acc = 0.0;
+  for (int64_t t = L.tp[k] + threadIdx.x; t < L.tp[k + 1]; t += kFinalizeThreads) acc += pr[t];
+  const double S = block_sum_fixed(acc, sm);
+  if (threadIdx.x == 0) {
+    const int64_t nk = L.off[k + 1] - L.off[k];
+    out[(static_cast<int64_t>(r) * L.C + k) * planes + plane] =
+        nk > 0 ? __double2float_rn(__ddiv_rn(S, static_cast<double>(nk))) : 0.0f;
+  }
+}
+
+// ---- 0/1 Adam local step ------------------------------------------------------------------
+// A local step sends nothing: every worker keeps its gradient in its error
+// buffer for the next synchronised step, err_w = clip(g_w) + err_w, and the
+// parameters move with the current m and v, which stay as they are:
+//   Adam: p -= lr m / (sqrt(v) + eps);
+//   LAMB (kLambM): per-tile sums of p^2 and u^2, u = m / (sqrt(v) + eps), for the
+//   trust ratio; the parameter step follows in k_lamb_param.
+// A non-finite kept value or parameter raises the status flag.
+template <Upd U>
+__device__ __forceinline__ void local_elem(float m, float v, float& p, const Hyper& h, double& P,
+                                           double& Usum, bool& bad) {
+  if (U == Upd::kAdam) {
+    p = p - __fdiv_rn(h.lr * m, __fsqrt_rn(v) + h.eps);
+    bad |= !isfinite(p);
+  } else {
+    const float u = __fdiv_rn(m, __fsqrt_rn(v) + h.eps);
+    P = fma(static_cast<double>(p), static_cast<double>(p), P);
+    Usum = fma(static_cast<double>(u), static_cast<double>(u), Usum);
+  }
+}
+
+template <typename GT, typename ET, bool CLIP, Upd U>
+__global__ void __launch_bounds__(kBlock)
+k_local_step(Layout L, int W, const GT* __restrict__ grads, ET* __restrict__ err,
+             const float* __restrict__ m, const float* __restrict__ v, float* __restrict__ p, Hyper h,
+             double* __restrict__ partP, double* __restrict__ partU, uint32_t* __restrict__ status) {
+  pdl_enter();
+  const int lane = threadIdx.x & 31;
+  int hint = 0;
+  for (int64_t t = warp_id(); t < L.T; t += warp_count()) {
+    const Tile tl = tile_at(L, t, hint);
+    double Psum = 0.0, Usum = 0.0;
+    bool bad = false;
+    if (tl.vec) {
+#pragma unroll
+      for (int q = 0; q < kGroups; ++q) {
+        const int64_t i0 = tl.rel + q * kGroupElems + lane * kVec;
+        if (i0 < tl.nk) {
+          const int64_t gi = tl.ck0 + i0;
+          float mv[8], vv[8], pv[8];
+          ld8_ro(m + gi, mv);
+          ld8_ro(v + gi, vv);
+          ld8(p + gi, pv);
+          for (int w = 0; w < W; ++w) {
+            const int64_t e = static_cast<int64_t>(w) * L.n + gi;
+            float gv[8], ev[8];
+            ld8_ro(grads + e, gv);
+            ld8(err + e, ev);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              ev[j] = (CLIP ? clip_grad(gv[j], h.clip) : gv[j]) + ev[j];
+              bad |= !isfinite(ev[j]);
+            }
+            st8(err + e, ev);
+          }
+#pragma unroll
+          for (int j = 0; j < 8; ++j) local_elem<U>(mv[j], vv[j], pv[j], h, Psum, Usum, bad);
+          if (U == Upd::kAdam) st8(p + gi, pv);
+        }
+      }
+    } else {
+      for (int j = 0; j < kTileWords; ++j) {
+        const int64_t i = tl.rel + j * 32 + lane;
+        if (i < tl.nk) {
+          const int64_t gi = tl.ck0 + i;
+          for (int w = 0; w < W; ++w) {
+            const int64_t e = static_cast<int64_t>(w) * L.n + gi;
+            const float g = ld1_ro(grads + e);
+            const float kept = (CLIP ? clip_grad(g, h.clip) : g) + ld1(err + e);
+            bad |= !isfinite(kept);
+            st1(err + e, kept);
+          }
+          float pv = p[gi];
+          local_elem<U>(__ldg(m + gi), __ldg(v + gi), pv, h, Psum, Usum, bad);
+          if (U == Upd::kAdam) p[gi] = pv;
+        }
+      }
+    }
+    if (U == Upd::kLambM) {
+      Psum = warp_sum(Psum);
+      Usum = warp_sum(Usum);
+      if (lane == 0) { partP[t] = Psum; partU[t] = Usum; }
+    }
+    flag_nonfinite(bad, status);
+  }
+}
+
 // ---- LAMB parameter step: p -= lr * r_k * m / (sqrt(v) + eps) ---------------------------
 __global__ void __launch_bounds__(kBlock)
 k_lamb_param(Layout L, const float* __restrict__ m, const float* __restrict__ v,
              float* __restrict__ p, const float* __restrict__ ratio, Hyper h,
              uint32_t* __restrict__ status) {
+  pdl_enter();
   const int lane = threadIdx.x & 31;
   int hint = 0;
   for (int64_t t = warp_id(); t < L.T; t += warp_count()) {
@@ -786,6 +1048,61 @@ k_lamb_param(Layout L, const float* __restrict__ m, const float* __restrict__ v,
   }
 }
 
+// ---- the warmup's full-precision average ----------------------------------------------------
+// mean[i] = (sum_{w=0..W-1} g_w[i]) / W: float additions in ascending w, one
+// division (the average k_warmup forms before its moments).  A one-worker
+// float32 warmup on `mean` then takes the same steps as the W-worker warmup.
+// A non-finite mean raises the status flag.
+template <typename GT, bool POW2>
+__global__ void __launch_bounds__(kBlock)
+k_grad_mean(Layout L, int W, const GT* __restrict__ grads, float* __restrict__ out,
+            uint32_t* __restrict__ status) {
+  pdl_enter();
+  const int lane = threadIdx.x & 31;
+  const auto mean = make_mean<POW2>(W);
+  int hint = 0;
+  for (int64_t t = warp_id(); t < L.T; t += warp_count()) {
+    const Tile tl = tile_at(L, t, hint);
+    bool bad = false;
+    if (tl.vec) {
+#pragma unroll
+      for (int q = 0; q < kGroups; ++q) {
+        const int64_t i0 = tl.rel + q * kGroupElems + lane * kVec;
+        if (i0 < tl.nk) {
+          const int64_t gi = tl.ck0 + i0;
+          float acc[8];
+          zero8(acc);
+          for (int w = 0; w < W; ++w) {
+            float gv[8];
+            ld8_ro(grads + static_cast<int64_t>(w) * L.n + gi, gv);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) acc[j] = acc[j] + gv[j];
+          }
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            acc[j] = mean(acc[j]);
+            bad |= !isfinite(acc[j]);
+          }
+          st8(out + gi, acc);
+        }
+      }
+    } else {
+      for (int j = 0; j < kTileWords; ++j) {
+        const int64_t i = tl.rel + j * 32 + lane;
+        if (i < tl.nk) {
+          const int64_t gi = tl.ck0 + i;
+          float acc = 0.0f;
+          for (int w = 0; w < W; ++w) acc = acc + ld1_ro(grads + static_cast<int64_t>(w) * L.n + gi);
+          acc = mean(acc);
+          bad |= !isfinite(acc);
+          out[gi] = acc;
+        }
+      }
+    }
+    flag_nonfinite(bad, status);
+  }
+}
+
 // ---- full-precision warmup -------------------------------------------------------------
 // g = (sum_w g_w) / W; m = b1 m + (1-b1) g; v = b2 v + (1-b2) g^2;
 // Adam: p -= lr m / (sqrt(v) + eps).  LAMB: per-tile sums of p^2 and u^2 instead
@@ -795,6 +1112,7 @@ __global__ void __launch_bounds__(kBlock)
 k_warmup(Layout L, int W, const GT* __restrict__ grads, float* __restrict__ m,
          float* __restrict__ v, float* __restrict__ p, Hyper h, double* __restrict__ partP,
          double* __restrict__ partU, uint32_t* __restrict__ status) {
+  pdl_enter();
   const int lane = threadIdx.x & 31;
   const auto mean = make_mean<POW2>(W);
   int hint = 0;

@@ -28,9 +28,28 @@ namespace ob {
 __device__ __forceinline__ int64_t plane_words(int64_t nk) { return (nk + 31) / 32; }
 
 // acc[j] += s1 sign1 + s2 sign2 of worker w, ascending w (the order of pass 2).
+// W1: exactly one worker.  Its four possible dequantised values
+// (+-s1) + (+-s2) are formed once per group -- the same float additions the
+// per-element form makes -- and each element selects one of them.
+template <bool W1>
 __device__ __forceinline__ void tb_server_sum8(const Layout& L, int W, const uint32_t* __restrict__ bits_w,
                                                const float* __restrict__ s_w, const Tile& tl, int64_t wrel,
                                                int64_t nwk, bool word_in, int lane, float (&acc)[8]) {
+  if constexpr (W1) {
+    const float* sc = s_w + static_cast<int64_t>(tl.k) * 2;
+    const float s1 = __ldg(sc), s2 = __ldg(sc + 1);
+    const float d00 = -s1 + -s2, d10 = s1 + -s2, d01 = -s1 + s2, d11 = s1 + s2;  // d<b1><b2>
+    const uint32_t* row = bits_w + tl.w0;
+    const uint32_t w1 = word_in ? __ldg(row + wrel) : 0u;
+    const uint32_t w2 = word_in ? __ldg(row + nwk + wrel) : 0u;
+    const uint32_t b1 = lane_byte(w1, lane), b2 = lane_byte(w2, lane);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const bool x1 = (b1 >> j) & 1u, x2 = (b2 >> j) & 1u;
+      acc[j] = 0.0f + (x2 ? (x1 ? d11 : d01) : (x1 ? d10 : d00));
+    }
+    return;
+  }
   zero8(acc);
   for (int w = 0; w < W; ++w) {
     const float* sc = s_w + (static_cast<int64_t>(w) * L.C + tl.k) * 2;
@@ -45,11 +64,12 @@ __device__ __forceinline__ void tb_server_sum8(const Layout& L, int W, const uin
   }
 }
 
+template <bool W1>
 __device__ __forceinline__ float tb_server_sum1(const Layout& L, int W, const uint32_t* __restrict__ bits_w,
                                                 const float* __restrict__ s_w, const Tile& tl, int64_t wi,
                                                 int64_t nwk, int lane) {
   float acc = 0.0f;
-  for (int w = 0; w < W; ++w) {
+  for (int w = 0; w < (W1 ? 1 : W); ++w) {
     const float* sc = s_w + (static_cast<int64_t>(w) * L.C + tl.k) * 2;
     const uint32_t* row = bits_w + static_cast<int64_t>(w) * L.words + tl.w0;
     const bool b1 = (__ldg(row + wi) >> lane) & 1u, b2 = (__ldg(row + nwk + wi) >> lane) & 1u;
@@ -63,6 +83,7 @@ template <typename GT, typename ET, bool CLIP>
 __global__ void __launch_bounds__(kBlock)
 k_tb_resid_norm(Layout L, int W, const GT* __restrict__ grads, const ET* __restrict__ err,
                 const float* __restrict__ s_w, float clip, double* __restrict__ part) {
+  pdl_enter();
   const int lane = threadIdx.x & 31;
   const int64_t items = static_cast<int64_t>(W) * L.T;
   int hint = 0;
@@ -114,6 +135,7 @@ __global__ void __launch_bounds__(kBlock, 3)
 k_tb_pack(Layout L, int W, const GT* __restrict__ grads, ET* __restrict__ err,
           const float* __restrict__ s_w, uint32_t* __restrict__ bits_w, const ET* __restrict__ srv_err,
           double* __restrict__ part_srv, float* __restrict__ csrv, float clip, uint32_t* __restrict__ status) {
+  pdl_enter();
   const int lane = threadIdx.x & 31;
   const auto mean = make_mean<POW2>(W);
   int hint = 0;
@@ -219,12 +241,14 @@ k_tb_pack(Layout L, int W, const GT* __restrict__ grads, ET* __restrict__ err,
 
 // ---- server norms from the worker planes --------------------------------------------
 // RESID = false: sum c_srv^2 (for s1'; the stage call).  RESID = true: sum of
-// (c_srv - s1' sign(c_srv))^2 (for s2'), s1' read from s_srv.
-template <typename ET, bool POW2, bool RESID>
+// (c_srv - s1' sign(c_srv))^2 (for s2'), s1' read from s_srv.  W1 (with POW2):
+// one worker (see tb_server_sum8).
+template <typename ET, bool POW2, bool RESID, bool W1>
 __global__ void __launch_bounds__(kBlock)
 k_tb_server_norm(Layout L, int W, const uint32_t* __restrict__ bits_w, const float* __restrict__ s_w,
                  const ET* __restrict__ srv_err, const float* __restrict__ s_srv,
                  double* __restrict__ part, uint32_t* __restrict__ status) {
+  pdl_enter();
   const int lane = threadIdx.x & 31;
   const auto mean = make_mean<POW2>(W);
   int hint = 0;
@@ -245,7 +269,7 @@ k_tb_server_norm(Layout L, int W, const uint32_t* __restrict__ bits_w, const flo
         const bool in = i0 < tl.nk;
         float sv[8], acc[8];
         if (in) ld8_ro(srv_err + tl.ck0 + i0, sv); else zero8(sv);
-        tb_server_sum8(L, W, bits_w, s_w, tl, wrel, nwk, wrel * 32 < tl.nk, lane, acc);
+        tb_server_sum8<W1>(L, W, bits_w, s_w, tl, wrel, nwk, wrel * 32 < tl.nk, lane, acc);
         if (in) {
 #pragma unroll
           for (int j = 0; j < 8; ++j) add(mean(acc[j]) + sv[j]);
@@ -254,7 +278,7 @@ k_tb_server_norm(Layout L, int W, const uint32_t* __restrict__ bits_w, const flo
     } else {
       for (int j = 0; j < kTileWords; ++j) {
         const int64_t i = tl.rel + j * 32 + lane;
-        if (i < tl.nk) add(mean(tb_server_sum1(L, W, bits_w, s_w, tl, tl.rel / 32 + j, nwk, lane)) +
+        if (i < tl.nk) add(mean(tb_server_sum1<W1>(L, W, bits_w, s_w, tl, tl.rel / 32 + j, nwk, lane)) +
                            ld1_ro(srv_err + tl.ck0 + i));
       }
     }
@@ -270,6 +294,7 @@ k_tb_server_norm(Layout L, int W, const uint32_t* __restrict__ bits_w, const flo
 __global__ void __launch_bounds__(kBlock)
 k_tb_server_norm_cached(Layout L, const float* __restrict__ csrv, const float* __restrict__ s_srv,
                         double* __restrict__ part) {
+  pdl_enter();
   const int lane = threadIdx.x & 31;
   int hint = 0;
   for (int64_t t = warp_id(); t < L.T; t += warp_count()) {
@@ -308,14 +333,16 @@ k_tb_server_norm_cached(Layout L, const float* __restrict__ csrv, const float* _
 // ---- pass 3: server planes + server error, and/or the update --------------------------
 // FROM_WORKERS: c_srv from the worker planes and srv_err, quantised to two planes
 // with s_srv (bits_srv and srv_err written).  Otherwise g_hat from bits_srv.
-// CACHED (with FROM_WORKERS): c_srv read from csrv; srv_err only written.
-template <Upd U, bool FROM_WORKERS, bool POW2, typename ET, bool CACHED>
+// CACHED (with FROM_WORKERS): c_srv read from csrv; srv_err only written.  W1
+// (with FROM_WORKERS, POW2): one worker (see tb_server_sum8).
+template <Upd U, bool FROM_WORKERS, bool POW2, typename ET, bool CACHED, bool W1>
 __global__ void __launch_bounds__(kBlock, kUpdateMinBlocks)
 k_tb_server_update(Layout L, int W, const uint32_t* __restrict__ bits_w, const float* __restrict__ s_w,
                    const float* __restrict__ csrv, const float* __restrict__ s_srv, ET* __restrict__ srv_err,
                    uint32_t* __restrict__ bits_srv, float* __restrict__ m, const float* __restrict__ v,
                    float* __restrict__ p, Hyper h, double* __restrict__ partP,
                    double* __restrict__ partU, uint32_t* __restrict__ status) {
+  pdl_enter();
   const int lane = threadIdx.x & 31;
   const auto mean = make_mean<POW2>(W);
   int hint = 0;
@@ -342,7 +369,7 @@ k_tb_server_update(Layout L, int W, const uint32_t* __restrict__ bits_w, const f
         }
         if (FROM_WORKERS) {
           float acc[8];
-          if (!CACHED) tb_server_sum8(L, W, bits_w, s_w, tl, wrel, nwk, word_in, lane, acc);
+          if (!CACHED) tb_server_sum8<W1>(L, W, bits_w, s_w, tl, wrel, nwk, word_in, lane, acc);
           uint32_t byte1 = 0, byte2 = 0;
           if (in) {
 #pragma unroll
@@ -392,7 +419,7 @@ k_tb_server_update(Layout L, int W, const uint32_t* __restrict__ bits_w, const f
           bool b1 = false, b2 = false;
           if (inb) {
             const float cs = CACHED ? __ldg(csrv + gi)
-                                    : mean(tb_server_sum1(L, W, bits_w, s_w, tl, wi, nwk, lane)) + ld1(srv_err + gi);
+                                    : mean(tb_server_sum1<W1>(L, W, bits_w, s_w, tl, wi, nwk, lane)) + ld1(srv_err + gi);
             b1 = cs >= 0.0f;
             const float d1 = signed_scale(b1, s1);
             const float r = cs - d1;
