@@ -69,10 +69,13 @@ _SIGS = {
     "ob_launch_count": (ctypes.c_int64, [_P]),
     "ob_compress_noalloc": (ctypes.c_int, [ctypes.POINTER(ob_config), _P, _P, _P, _P, _P]),
     "ob_error_norms": (ctypes.c_int, [_P, _P, _P, _P]),
+    "ob_quant_rates": (ctypes.c_int, [_P, _P, _P, _P]),
+    "ob_local_step": (ctypes.c_int, [_P, _P, _P]),
+    "ob_mean_grads": (ctypes.c_int, [_P, _P, _P, _P]),
     "ob_last_error": (ctypes.c_char_p, []),
 }
 
-OB_K_KINDS = 21
+OB_K_KINDS = 24
 
 _lib = None
 
@@ -178,6 +181,18 @@ def ob_set_step(ctx: int, step: int) -> None:
 
 def ob_error_norms(ctx: int, worker_norms: int, server_norms: int, stream: int) -> None:
     check(load().ob_error_norms(ctx, worker_norms, server_norms, stream), "ob_error_norms")
+
+
+def ob_quant_rates(ctx: int, worker_rates: int, server_rates: int, stream: int) -> None:
+    check(load().ob_quant_rates(ctx, worker_rates, server_rates, stream), "ob_quant_rates")
+
+
+def ob_local_step(ctx: int, grads: int, stream: int) -> None:
+    check(load().ob_local_step(ctx, grads, stream), "ob_local_step")
+
+
+def ob_mean_grads(ctx: int, grads: int, mean: int, stream: int) -> None:
+    check(load().ob_mean_grads(ctx, grads, mean, stream), "ob_mean_grads")
 
 
 def ob_profile_start(ctx: int, capacity: int) -> None:

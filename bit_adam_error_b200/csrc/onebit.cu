@@ -17,6 +17,7 @@
 #include <cstring>
 #include <mutex>
 #include <new>
+#include <utility>
 #include <vector>
 
 #include <cuda_runtime.h>
@@ -143,6 +144,7 @@ struct ob_ctx {
   float* csrv = nullptr;            // c_srv of the fused step's pass 2 (W >= kCacheMinW), else NULL
   float* ratio = nullptr;
   uint32_t* status = nullptr;
+  unsigned* ticket = nullptr;       // the fused finaliser's CTA counter (zero between launches)
   ob::Hyper h{};
   const void* grads_checked = nullptr;   // last grads pointer that passed check_dev
   std::vector<std::pair<const void*, int>> occ;  // kernel -> resident CTAs per SM
@@ -197,6 +199,25 @@ struct DeviceGuard {
   }
 };
 
+// Launch with programmatic stream serialisation: the kernel may be scheduled
+// while the stream's previous kernel finishes, and waits for it (every kernel
+// starts with pdl_enter) before touching memory.  Launch errors surface through
+// cudaGetLastError like those of <<<>>> launches.
+template <typename... P, typename... A>
+void pdl(void (*kernel)(P...), dim3 grid, unsigned block, cudaStream_t st, A&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(block);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaLaunchKernelEx(&cfg, kernel, std::forward<A>(args)...);
+}
+
 // Enqueue one kernel launch (fn), with an event pair around it while profiling.
 template <typename Fn>
 void launch(ob_ctx* c, int kind, cudaStream_t st, Fn&& fn) {
@@ -233,7 +254,7 @@ void enqueue_finalize_scale(ob_ctx* c, const double* part, float* out, int rows,
                             const int64_t* tpx, int mult, int64_t row_stride, cudaStream_t st,
                             int planes = 1, int plane = 0) {
   launch(c, OB_K_FINALIZE_SCALE, st, [&] {
-    ob::k_finalize_scale<true><<<dim3(c->cfg.num_chunks, rows), ob::kFinalizeThreads, 0, st>>>(
+    pdl(ob::k_finalize_scale<true>, dim3(c->cfg.num_chunks, rows), ob::kFinalizeThreads, st, 
         c->L, part, tpx, mult, row_stride, out, planes, plane);
   });
 }
@@ -246,36 +267,70 @@ bool pow2_workers(const ob_ctx* c) { return (c->cfg.W & (c->cfg.W - 1)) == 0; }
 // W = 1 bf16 3.19 vs 3.47 ms per 1.5e9 elements, W = 16 fp32 10.30 vs 10.05 ms.
 constexpr int kPackOneGroupMaxW = 2;
 
+// Problems this small take the fused finaliser (the pass's last CTA computes the
+// scales, see ob::fused_finalize) instead of a separate finaliser launch: at most
+// this many tile partials and (row, chunk) pairs, so the last CTA's share stays
+// a few microseconds.  The stage calls decide the same way, so on a given
+// problem the fused step and the stages compute every scale alike.
+constexpr int64_t kFinMaxPartials = int64_t(1) << 15;
+constexpr int64_t kFinMaxTasks = 64;
+
+bool fused_fin(const ob_ctx* c, int64_t rows) {
+  return c->T > 0 && rows * c->T <= kFinMaxPartials && rows * c->cfg.num_chunks <= kFinMaxTasks;
+}
+
 template <typename GT, typename ET, bool CLIP, bool POW2>
 void enqueue_worker_t(ob_ctx* c, const GT* grads, bool with_server, cudaStream_t st) {
   const int W = c->cfg.W;
   ET* err = static_cast<ET*>(c->err);
   const ET* srv_err = static_cast<const ET*>(c->srv_err);
-  if (c->T > 0) {
+  const bool fin1 = fused_fin(c, W), fin2 = with_server && fused_fin(c, 1);
+  if (c->T > 0 && fin1) {
+    auto k1 = ob::k_worker_norm_fin<GT, ET, CLIP>;
+    const int g1 = grid_for(c, k1, W * c->T);
+    const ob::Fin f{c->ticket, c->part_w, c->T, W, c->s_w};
+    launch(c, OB_K_WORKER_NORM, st, [&] {
+      pdl(k1, g1, ob::kBlock, st, c->L, W, grads, err, c->h.clip, c->part_w, c->status, f);
+    });
+  } else if (c->T > 0) {
     auto k1 = ob::k_worker_norm<GT, ET, CLIP>;
     const int g1 = grid_for(c, k1, W * c->T);
     launch(c, OB_K_WORKER_NORM, st, [&] {
-      k1<<<g1, ob::kBlock, 0, st>>>(c->L, W, grads, err, c->h.clip, c->part_w, c->status);
+      pdl(k1, g1, ob::kBlock, st, c->L, W, grads, err, c->h.clip, c->part_w, c->status);
     });
   }
-  enqueue_finalize_scale(c, c->part_w, c->s_w, W, c->L.tp, 1, c->T, st);
+  if (!fin1) enqueue_finalize_scale(c, c->part_w, c->s_w, W, c->L.tp, 1, c->T, st);
   if (c->T > 0) {
     // The stage call (no server part) never uses the mean: one instantiation each.
     // Many workers: the fused step also stores c_srv for pass 3 (CACHE).
     const bool one = W <= kPackOneGroupMaxW, cache = with_server && c->csrv;
-    auto k2 = with_server ? (cache ? (one ? ob::k_worker_pack<GT, ET, true, CLIP, POW2, 1, true>
-                                          : ob::k_worker_pack<GT, ET, true, CLIP, POW2, 2, true>)
-                                   : (one ? ob::k_worker_pack<GT, ET, true, CLIP, POW2, 1, false>
-                                          : ob::k_worker_pack<GT, ET, true, CLIP, POW2, 2, false>))
-                          : (one ? ob::k_worker_pack<GT, ET, false, CLIP, false, 1, false>
-                                 : ob::k_worker_pack<GT, ET, false, CLIP, false, 2, false>);
-    const int g2 = grid_for(c, k2, c->T);
-    launch(c, cache ? OB_K_WORKER_PACK_CACHED : OB_K_WORKER_PACK, st, [&] {
-      k2<<<g2, ob::kBlock, 0, st>>>(c->L, W, grads, err, c->s_w, c->bits_w, srv_err,
-                                    c->part_srv, c->csrv, c->h.clip, c->status);
-    });
+    const int kind = cache ? OB_K_WORKER_PACK_CACHED : OB_K_WORKER_PACK;
+    if (fin2) {
+      auto k2 = cache ? (one ? ob::k_worker_pack_fin<GT, ET, true, CLIP, POW2, 1, true>
+                             : ob::k_worker_pack_fin<GT, ET, true, CLIP, POW2, 2, true>)
+                      : (one ? ob::k_worker_pack_fin<GT, ET, true, CLIP, POW2, 1, false>
+                             : ob::k_worker_pack_fin<GT, ET, true, CLIP, POW2, 2, false>);
+      const int g2 = grid_for(c, k2, c->T);
+      const ob::Fin f{c->ticket, c->part_srv, 0, 1, c->s_srv};
+      launch(c, kind, st, [&] {
+        pdl(k2, g2, ob::kBlock, st, c->L, W, grads, err, c->s_w, c->bits_w, srv_err, c->part_srv, c->csrv,
+            c->h.clip, c->status, f);
+      });
+    } else {
+      auto k2 = with_server ? (cache ? (one ? ob::k_worker_pack<GT, ET, true, CLIP, POW2, 1, true>
+                                            : ob::k_worker_pack<GT, ET, true, CLIP, POW2, 2, true>)
+                                     : (one ? ob::k_worker_pack<GT, ET, true, CLIP, POW2, 1, false>
+                                            : ob::k_worker_pack<GT, ET, true, CLIP, POW2, 2, false>))
+                            : (one ? ob::k_worker_pack<GT, ET, false, CLIP, false, 1, false>
+                                   : ob::k_worker_pack<GT, ET, false, CLIP, false, 2, false>);
+      const int g2 = grid_for(c, k2, c->T);
+      launch(c, kind, st, [&] {
+        pdl(k2, g2, ob::kBlock, st, c->L, W, grads, err, c->s_w, c->bits_w, srv_err, c->part_srv, c->csrv,
+            c->h.clip, c->status);
+      });
+    }
   }
-  if (with_server) enqueue_finalize_scale(c, c->part_srv, c->s_srv, 1, c->L.tp, 1, 0, st);
+  if (with_server && !fin2) enqueue_finalize_scale(c, c->part_srv, c->s_srv, 1, c->L.tp, 1, 0, st);
 }
 
 template <typename GT, typename ET>
@@ -294,14 +349,17 @@ void enqueue_worker(ob_ctx* c, const GT* grads, bool with_server, cudaStream_t s
 }
 
 // CACHED: c_srv comes from c->csrv (the fused step's pass 2 stored it).
+// One worker (rebuilding the server value from the words): the W1 instance.
 template <ob::Upd U, bool FROM_WORKERS, typename ET, bool CACHED>
 void launch_server_update(ob_ctx* c, cudaStream_t st) {
-  auto k3 = pow2_workers(c) ? ob::k_server_update<U, FROM_WORKERS, true, ET, CACHED>
-                            : ob::k_server_update<U, FROM_WORKERS, false, ET, CACHED>;
+  constexpr bool kRebuild = FROM_WORKERS && !CACHED;
+  auto k3 = (kRebuild && c->cfg.W == 1) ? ob::k_server_update<U, FROM_WORKERS, true, ET, CACHED, kRebuild>
+            : pow2_workers(c)           ? ob::k_server_update<U, FROM_WORKERS, true, ET, CACHED, false>
+                                        : ob::k_server_update<U, FROM_WORKERS, false, ET, CACHED, false>;
   const int g3 = grid_for(c, k3, c->T);
   ET* srv_err = static_cast<ET*>(c->srv_err);
   launch(c, CACHED ? OB_K_SERVER_UPDATE_CACHED : OB_K_SERVER_UPDATE, st, [&] {
-    k3<<<g3, ob::kBlock, 0, st>>>(c->L, c->cfg.W, c->bits_w, c->s_w, c->csrv, c->s_srv, srv_err,
+    pdl(k3, g3, ob::kBlock, st, c->L, c->cfg.W, c->bits_w, c->s_w, c->csrv, c->s_srv, srv_err,
                                   c->bits_srv, c->m, c->v, c->p, c->h, c->partP, c->partU,
                                   c->status);
   });
@@ -328,14 +386,14 @@ void enqueue_server_update(ob_ctx* c, cudaStream_t st, bool cached = false) {
 // LAMB: trust ratio per layer from the tile partials, then the parameter step.
 void enqueue_lamb_param(ob_ctx* c, cudaStream_t st) {
   launch(c, OB_K_FINALIZE_RATIO, st, [&] {
-    ob::k_finalize_ratio<<<c->cfg.num_chunks, ob::kFinalizeThreads, 0, st>>>(c->L, c->partP, c->partU,
+    pdl(ob::k_finalize_ratio, c->cfg.num_chunks, ob::kFinalizeThreads, st, c->L, c->partP, c->partU,
                                                                              c->L.tp, 1, c->ratio);
   });
   if (c->T == 0) return;
   auto k = ob::k_lamb_param;
   const int g = grid_for(c, k, c->T);
   launch(c, OB_K_LAMB_PARAM, st, [&] {
-    k<<<g, ob::kBlock, 0, st>>>(c->L, c->m, c->v, c->p, c->ratio, c->h, c->status);
+    pdl(k, g, ob::kBlock, st, c->L, c->m, c->v, c->p, c->ratio, c->h, c->status);
   });
 }
 
@@ -361,29 +419,40 @@ void enqueue_warmup(ob_ctx* c, const GT* grads, cudaStream_t st) {
                   : (p2 ? ob::k_warmup<GT, false, true> : ob::k_warmup<GT, false, false>);
     const int g = grid_for(c, k, c->T);
     launch(c, OB_K_WARMUP, st, [&] {
-      k<<<g, ob::kBlock, 0, st>>>(c->L, c->cfg.W, grads, c->m, c->v, c->p, c->h, c->partP,
+      pdl(k, g, ob::kBlock, st, c->L, c->cfg.W, grads, c->m, c->v, c->p, c->h, c->partP,
                                   c->partU, c->status);
     });
   }
   if (lamb) enqueue_lamb_param(c, st);
 }
 
+// fin: the fused finaliser writes s_srv (small problems, as in the fused step).
 template <typename ET>
-void enqueue_server_norm(ob_ctx* c, cudaStream_t st) {
+void enqueue_server_norm(ob_ctx* c, bool fin, cudaStream_t st) {
+  const ET* srv_err = static_cast<const ET*>(c->srv_err);
+  if (fin) {
+    auto k = pow2_workers(c) ? ob::k_server_norm_fin<ET, true> : ob::k_server_norm_fin<ET, false>;
+    const int g = grid_for(c, k, c->T);
+    const ob::Fin f{c->ticket, c->part_srv, 0, 1, c->s_srv};
+    launch(c, OB_K_SERVER_NORM, st, [&] {
+      pdl(k, g, ob::kBlock, st, c->L, c->cfg.W, c->bits_w, c->s_w, srv_err, c->part_srv, c->status, f);
+    });
+    return;
+  }
   auto k = pow2_workers(c) ? ob::k_server_norm<ET, true> : ob::k_server_norm<ET, false>;
   const int g = grid_for(c, k, c->T);
-  const ET* srv_err = static_cast<const ET*>(c->srv_err);
   launch(c, OB_K_SERVER_NORM, st, [&] {
-    k<<<g, ob::kBlock, 0, st>>>(c->L, c->cfg.W, c->bits_w, c->s_w, srv_err, c->part_srv, c->status);
+    pdl(k, g, ob::kBlock, st, c->L, c->cfg.W, c->bits_w, c->s_w, srv_err, c->part_srv, c->status);
   });
 }
 
 void enqueue_server_stage(ob_ctx* c, cudaStream_t st) {
+  const bool fin = fused_fin(c, 1);
   if (c->T > 0) {
-    if (c->cfg.err_dtype == OB_BF16) enqueue_server_norm<uint16_t>(c, st);
-    else enqueue_server_norm<float>(c, st);
+    if (c->cfg.err_dtype == OB_BF16) enqueue_server_norm<uint16_t>(c, fin, st);
+    else enqueue_server_norm<float>(c, fin, st);
   }
-  enqueue_finalize_scale(c, c->part_srv, c->s_srv, 1, c->L.tp, 1, 0, st);
+  if (!fin) enqueue_finalize_scale(c, c->part_srv, c->s_srv, 1, c->L.tp, 1, 0, st);
   enqueue_server_update<ob::Upd::kNone, true>(c, st);
 }
 
@@ -396,7 +465,7 @@ void enqueue_ternary_step_t(ob_ctx* c, const GT* grads, cudaStream_t st) {
                                        : ob::k_ternary_step<GT, ET, CLIP, POW2, ob::Upd::kAdam>;
   const int g = grid_for(c, k, c->T);
   launch(c, OB_K_TERNARY_STEP, st, [&] {
-    k<<<g, ob::kBlock, 0, st>>>(c->L, c->cfg.W, grads, static_cast<ET*>(c->err), c->m, c->v, c->p,
+    pdl(k, g, ob::kBlock, st, c->L, c->cfg.W, grads, static_cast<ET*>(c->err), c->m, c->v, c->p,
                                 c->h, c->partP, c->partU, c->status);
   });
 }
@@ -407,7 +476,7 @@ void enqueue_ternary_compress_t(ob_ctx* c, const GT* grads, cudaStream_t st) {
   auto k = ob::k_ternary_compress<GT, ET, CLIP>;
   const int g = grid_for(c, k, c->cfg.W * c->T);
   launch(c, OB_K_TERNARY_COMPRESS, st, [&] {
-    k<<<g, ob::kBlock, 0, st>>>(c->L, c->cfg.W, grads, static_cast<ET*>(c->err), c->bits_w, c->h,
+    pdl(k, g, ob::kBlock, st, c->L, c->cfg.W, grads, static_cast<ET*>(c->err), c->bits_w, c->h,
                                 c->status);
   });
 }
@@ -446,7 +515,7 @@ void enqueue_ternary_server(ob_ctx* c, cudaStream_t st) {
   auto k = ob::k_ternary_server;
   const int g = grid_for(c, k, (c->words + 31) / 32);
   launch(c, OB_K_TERNARY_SERVER, st, [&] {
-    k<<<g, ob::kBlock, 0, st>>>(c->cfg.W, c->words, c->bits_w, c->bits_srv);
+    pdl(k, g, ob::kBlock, st, c->cfg.W, c->words, c->bits_w, c->bits_srv);
   });
 }
 
@@ -457,7 +526,7 @@ void enqueue_ternary_update(ob_ctx* c, cudaStream_t st) {
                   : (p2 ? ob::k_ternary_update<ob::Upd::kAdam, true> : ob::k_ternary_update<ob::Upd::kAdam, false>);
     const int g = grid_for(c, k, c->T);
     launch(c, OB_K_TERNARY_UPDATE, st, [&] {
-      k<<<g, ob::kBlock, 0, st>>>(c->L, c->cfg.W, c->bits_srv, c->m, c->v, c->p, c->h, c->partP,
+      pdl(k, g, ob::kBlock, st, c->L, c->cfg.W, c->bits_srv, c->m, c->v, c->p, c->h, c->partP,
                                   c->partU, c->status);
     });
   }
@@ -477,7 +546,7 @@ void enqueue_tb_worker_t(ob_ctx* c, const GT* grads, bool with_server, cudaStrea
     auto k1 = ob::k_worker_norm<GT, ET, CLIP>;
     const int g1 = grid_for(c, k1, W * c->T);
     launch(c, OB_K_WORKER_NORM, st, [&] {
-      k1<<<g1, ob::kBlock, 0, st>>>(c->L, W, grads, err, c->h.clip, c->part_w, c->status);
+      pdl(k1, g1, ob::kBlock, st, c->L, W, grads, err, c->h.clip, c->part_w, c->status);
     });
   }
   enqueue_finalize_scale(c, c->part_w, c->s_w, W, c->L.tp, 1, c->T, st, 2, 0);
@@ -485,7 +554,7 @@ void enqueue_tb_worker_t(ob_ctx* c, const GT* grads, bool with_server, cudaStrea
     auto k1b = ob::k_tb_resid_norm<GT, ET, CLIP>;
     const int g = grid_for(c, k1b, W * c->T);
     launch(c, OB_K_TB_RESID_NORM, st, [&] {
-      k1b<<<g, ob::kBlock, 0, st>>>(c->L, W, grads, err, c->s_w, c->h.clip, c->part_w);
+      pdl(k1b, g, ob::kBlock, st, c->L, W, grads, err, c->s_w, c->h.clip, c->part_w);
     });
   }
   enqueue_finalize_scale(c, c->part_w, c->s_w, W, c->L.tp, 1, c->T, st, 2, 1);
@@ -496,7 +565,7 @@ void enqueue_tb_worker_t(ob_ctx* c, const GT* grads, bool with_server, cudaStrea
                            : ob::k_tb_pack<GT, ET, true, CLIP, POW2, false>;
     const int g2 = grid_for(c, k2, c->T);
     launch(c, cache ? OB_K_TB_PACK_CACHED : OB_K_TB_PACK, st, [&] {
-      k2<<<g2, ob::kBlock, 0, st>>>(c->L, W, grads, err, c->s_w, c->bits_w, srv_err, c->part_srv,
+      pdl(k2, g2, ob::kBlock, st, c->L, W, grads, err, c->s_w, c->bits_w, srv_err, c->part_srv,
                                     c->csrv, c->h.clip, c->status);
     });
   }
@@ -506,13 +575,13 @@ void enqueue_tb_worker_t(ob_ctx* c, const GT* grads, bool with_server, cudaStrea
     auto k = ob::k_tb_server_norm_cached;
     const int g = grid_for(c, k, c->T);
     launch(c, OB_K_TB_SERVER_NORM_CACHED, st, [&] {
-      k<<<g, ob::kBlock, 0, st>>>(c->L, c->csrv, c->s_srv, c->part_srv);
+      pdl(k, g, ob::kBlock, st, c->L, c->csrv, c->s_srv, c->part_srv);
     });
   } else if (c->T > 0) {
-    auto k = ob::k_tb_server_norm<ET, POW2, true>;
+    auto k = W == 1 ? ob::k_tb_server_norm<ET, true, true, true> : ob::k_tb_server_norm<ET, POW2, true, false>;
     const int g = grid_for(c, k, c->T);
     launch(c, OB_K_TB_SERVER_NORM, st, [&] {
-      k<<<g, ob::kBlock, 0, st>>>(c->L, W, c->bits_w, c->s_w, srv_err, c->s_srv, c->part_srv, c->status);
+      pdl(k, g, ob::kBlock, st, c->L, W, c->bits_w, c->s_w, srv_err, c->s_srv, c->part_srv, c->status);
     });
   }
   enqueue_finalize_scale(c, c->part_srv, c->s_srv, 1, c->L.tp, 1, 0, st, 2, 1);
@@ -543,11 +612,13 @@ void enqueue_tb_worker(ob_ctx* c, const void* grads, bool with_server, cudaStrea
 template <ob::Upd U, bool FROM_WORKERS, typename ET, bool CACHED>
 void launch_tb_server_update(ob_ctx* c, cudaStream_t st) {
   if (c->T == 0) return;
-  auto k = pow2_workers(c) ? ob::k_tb_server_update<U, FROM_WORKERS, true, ET, CACHED>
-                           : ob::k_tb_server_update<U, FROM_WORKERS, false, ET, CACHED>;
+  constexpr bool kRebuild = FROM_WORKERS && !CACHED;
+  auto k = (kRebuild && c->cfg.W == 1) ? ob::k_tb_server_update<U, FROM_WORKERS, true, ET, CACHED, kRebuild>
+           : pow2_workers(c)           ? ob::k_tb_server_update<U, FROM_WORKERS, true, ET, CACHED, false>
+                                       : ob::k_tb_server_update<U, FROM_WORKERS, false, ET, CACHED, false>;
   const int g = grid_for(c, k, c->T);
   launch(c, CACHED ? OB_K_TB_SERVER_UPDATE_CACHED : OB_K_TB_SERVER_UPDATE, st, [&] {
-    k<<<g, ob::kBlock, 0, st>>>(c->L, c->cfg.W, c->bits_w, c->s_w, c->csrv, c->s_srv,
+    pdl(k, g, ob::kBlock, st, c->L, c->cfg.W, c->bits_w, c->s_w, c->csrv, c->s_srv,
                                 static_cast<ET*>(c->srv_err), c->bits_srv, c->m, c->v, c->p, c->h,
                                 c->partP, c->partU, c->status);
   });
@@ -586,19 +657,20 @@ void enqueue_tb_update(ob_ctx* c, bool from_workers, cudaStream_t st) {
 template <typename ET, bool POW2>
 void enqueue_tb_server_stage_t(ob_ctx* c, cudaStream_t st) {
   const ET* srv_err = static_cast<const ET*>(c->srv_err);
+  const bool one = c->cfg.W == 1;
   if (c->T > 0) {
-    auto k = ob::k_tb_server_norm<ET, POW2, false>;
+    auto k = one ? ob::k_tb_server_norm<ET, true, false, true> : ob::k_tb_server_norm<ET, POW2, false, false>;
     const int g = grid_for(c, k, c->T);
     launch(c, OB_K_TB_SERVER_NORM, st, [&] {
-      k<<<g, ob::kBlock, 0, st>>>(c->L, c->cfg.W, c->bits_w, c->s_w, srv_err, c->s_srv, c->part_srv, c->status);
+      pdl(k, g, ob::kBlock, st, c->L, c->cfg.W, c->bits_w, c->s_w, srv_err, c->s_srv, c->part_srv, c->status);
     });
   }
   enqueue_finalize_scale(c, c->part_srv, c->s_srv, 1, c->L.tp, 1, 0, st, 2, 0);
   if (c->T > 0) {
-    auto k = ob::k_tb_server_norm<ET, POW2, true>;
+    auto k = one ? ob::k_tb_server_norm<ET, true, true, true> : ob::k_tb_server_norm<ET, POW2, true, false>;
     const int g = grid_for(c, k, c->T);
     launch(c, OB_K_TB_SERVER_NORM, st, [&] {
-      k<<<g, ob::kBlock, 0, st>>>(c->L, c->cfg.W, c->bits_w, c->s_w, srv_err, c->s_srv, c->part_srv, c->status);
+      pdl(k, g, ob::kBlock, st, c->L, c->cfg.W, c->bits_w, c->s_w, srv_err, c->s_srv, c->part_srv, c->status);
     });
   }
   enqueue_finalize_scale(c, c->part_srv, c->s_srv, 1, c->L.tp, 1, 0, st, 2, 1);
@@ -611,6 +683,40 @@ void enqueue_tb_server_stage(ob_ctx* c, cudaStream_t st) {
     if (p2) enqueue_tb_server_stage_t<uint16_t, true>(c, st); else enqueue_tb_server_stage_t<uint16_t, false>(c, st);
   } else {
     if (p2) enqueue_tb_server_stage_t<float, true>(c, st); else enqueue_tb_server_stage_t<float, false>(c, st);
+  }
+}
+
+// ---- 0/1 Adam local step ------------------------------------------------------------------
+
+template <typename GT, typename ET, bool CLIP>
+void enqueue_local_t(ob_ctx* c, const GT* grads, cudaStream_t st) {
+  const bool lamb = c->cfg.optimizer == OB_LAMB;
+  if (c->T > 0) {
+    auto k = lamb ? ob::k_local_step<GT, ET, CLIP, ob::Upd::kLambM> : ob::k_local_step<GT, ET, CLIP, ob::Upd::kAdam>;
+    const int g = grid_for(c, k, c->T);
+    launch(c, OB_K_LOCAL_STEP, st, [&] {
+      pdl(k, g, ob::kBlock, st, c->L, c->cfg.W, grads, static_cast<ET*>(c->err), c->m, c->v, c->p, c->h,
+                                  c->partP, c->partU, c->status);
+    });
+  }
+  if (lamb) enqueue_lamb_param(c, st);
+}
+
+template <typename GT, typename ET>
+void enqueue_local_e(ob_ctx* c, const void* grads, cudaStream_t st) {
+  const GT* g = static_cast<const GT*>(grads);
+  if (c->h.clip > 0.0f) enqueue_local_t<GT, ET, true>(c, g, st);
+  else enqueue_local_t<GT, ET, false>(c, g, st);
+}
+
+void enqueue_local(ob_ctx* c, const void* grads, cudaStream_t st) {
+  const bool bf16_err = c->cfg.err_dtype == OB_BF16;
+  if (c->cfg.grad_dtype == OB_BF16) {
+    if (bf16_err) enqueue_local_e<uint16_t, uint16_t>(c, grads, st);
+    else enqueue_local_e<uint16_t, float>(c, grads, st);
+  } else {
+    if (bf16_err) enqueue_local_e<float, uint16_t>(c, grads, st);
+    else enqueue_local_e<float, float>(c, grads, st);
   }
 }
 
@@ -762,7 +868,7 @@ ob_err ob_create(const ob_config* cfg, float* p, float* m, float* v, void* err, 
   const bool fused_capable = p && m && v && err && srv_err && bits_w && s_w && bits_srv && s_srv;
   const bool cache = !momentum_rule(cfg) && W >= kCacheMinW && fused_capable && n > 0;
   const size_t sz_cs = cache ? up256(sizeof(float) * size_t(n)) : 0;
-  const size_t total = 3 * sz_tab + sz_vec + sz_pw + 3 * sz_pt + sz_ratio + sz_cs + 256;
+  const size_t total = 3 * sz_tab + sz_vec + sz_pw + 3 * sz_pt + sz_ratio + sz_cs + 512;
   if ((e = cudaMalloc(&c->scratch, total)) != cudaSuccess) {
     cudaGetLastError();
     delete c;
@@ -780,6 +886,7 @@ ob_err ob_create(const ob_config* cfg, float* p, float* m, float* v, void* err, 
   c->ratio = reinterpret_cast<float*>(base); base += sz_ratio;
   c->csrv = cache ? reinterpret_cast<float*>(base) : nullptr; base += sz_cs;
   c->status = reinterpret_cast<uint32_t*>(base);
+  c->ticket = reinterpret_cast<unsigned*>(base + 256);
 
   const struct { void* dst; const void* src; size_t bytes; } copies[] = {
       {d_off, c->off.data(), sizeof(int64_t) * (C + 1)},
@@ -792,7 +899,7 @@ ob_err ob_create(const ob_config* cfg, float* p, float* m, float* v, void* err, 
       delete c;
       return cuda_fail(e, "cudaMemcpy of chunk tables");
     }
-  if ((e = cudaMemset(c->status, 0, sizeof(uint32_t))) != cudaSuccess ||
+  if ((e = cudaMemset(c->status, 0, 512)) != cudaSuccess ||
       (e = cudaDeviceSynchronize()) != cudaSuccess) {
     cudaFree(c->scratch);
     delete c;
@@ -842,6 +949,46 @@ ob_err ob_refresh_step(ob_ctx* c, const void* grads, void* stream) {
   ob_err r = check_ctx(c);
   if (r != OB_OK) return r;
   return full_precision_step(c, grads, stream, "ob_refresh_step");
+}
+
+ob_err ob_local_step(ob_ctx* c, const void* grads, void* stream) {
+  ob_err r = check_ctx(c);
+  if (r != OB_OK) return r;
+  if (momentum_rule(&c->cfg))
+    return fail(OB_EINVAL, "ob_local_step: the momentum-error rule's error buffer is not additive");
+  if ((r = require_compressed(c, "ob_local_step")) != OB_OK) return r;
+  if ((r = require_buffers(c, kNeedWarm | kNeedErr, "ob_local_step")) != OB_OK) return r;
+  DeviceGuard dg(c->device);
+  if (!dg.ok) return fail(OB_ECUDA, "cannot select device %d", c->device);
+  if ((r = check_grads(c, grads)) != OB_OK) return r;
+  enqueue_local(c, grads, static_cast<cudaStream_t>(stream));
+  if ((r = check_launch("ob_local_step")) != OB_OK) return r;
+  ++c->step;
+  return OB_OK;
+}
+
+ob_err ob_mean_grads(ob_ctx* c, const void* grads, float* mean, void* stream) {
+  ob_err r = check_ctx(c);
+  if (r != OB_OK) return r;
+  DeviceGuard dg(c->device);
+  if (!dg.ok) return fail(OB_ECUDA, "cannot select device %d", c->device);
+  if ((r = check_grads(c, grads)) != OB_OK) return r;
+  if ((r = check_dev(mean, c->cfg.n, "mean", c->device)) != OB_OK) return r;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (c->T > 0) {
+    const bool p2 = pow2_workers(c), bf = c->cfg.grad_dtype == OB_BF16;
+    auto launch_mean = [&](auto k, const auto* g) {
+      const int grid = grid_for(c, k, c->T);
+      launch(c, OB_K_GRAD_MEAN, st, [&] { pdl(k, grid, ob::kBlock, st, c->L, c->cfg.W, g, mean, c->status); });
+    };
+    const uint16_t* gh = static_cast<const uint16_t*>(grads);
+    const float* gf = static_cast<const float*>(grads);
+    if (bf && p2) launch_mean(ob::k_grad_mean<uint16_t, true>, gh);
+    else if (bf) launch_mean(ob::k_grad_mean<uint16_t, false>, gh);
+    else if (p2) launch_mean(ob::k_grad_mean<float, true>, gf);
+    else launch_mean(ob::k_grad_mean<float, false>, gf);
+  }
+  return check_launch("ob_mean_grads");
 }
 
 ob_err ob_compress(ob_ctx* c, const void* grads, void* stream) {
@@ -1024,24 +1171,59 @@ ob_err ob_error_norms(ob_ctx* c, float* worker_norms, float* server_norms, void*
         auto k = ob::k_rows_sumsq<uint16_t>;
         const int g = grid_for(c, k, rows * c->T);
         launch(c, OB_K_WORKER_NORM, st, [&] {
-          k<<<g, ob::kBlock, 0, st>>>(c->L, rows, static_cast<const uint16_t*>(x), part);
+          pdl(k, g, ob::kBlock, st, c->L, rows, static_cast<const uint16_t*>(x), part);
         });
       } else {
         auto k = ob::k_rows_sumsq<float>;
         const int g = grid_for(c, k, rows * c->T);
         launch(c, OB_K_WORKER_NORM, st, [&] {
-          k<<<g, ob::kBlock, 0, st>>>(c->L, rows, static_cast<const float*>(x), part);
+          pdl(k, g, ob::kBlock, st, c->L, rows, static_cast<const float*>(x), part);
         });
       }
     }
     launch(c, OB_K_FINALIZE_SCALE, st, [&] {
-      ob::k_finalize_scale<false><<<dim3(unsigned(C), unsigned(rows)), ob::kFinalizeThreads, 0, st>>>(
+      pdl(ob::k_finalize_scale<false>, dim3(unsigned(C), unsigned(rows)), ob::kFinalizeThreads, st,
           c->L, part, c->L.tp, 1, c->T, out, 1, 0);
     });
   };
   if (worker_norms) norms(c->err, int(W), c->part_w, worker_norms);
   if (server_norms) norms(c->srv_err, 1, c->part_srv, server_norms);
   return check_launch("ob_error_norms");
+}
+
+ob_err ob_quant_rates(ob_ctx* c, float* worker_rates, float* server_rates, void* stream) {
+  ob_err r = check_ctx(c);
+  if (r != OB_OK) return r;
+  if (momentum_rule(&c->cfg))
+    return fail(OB_EINVAL, "ob_quant_rates: the momentum-error rule sends ternary codes, not sign bits");
+  const int64_t W = c->cfg.W, C = c->cfg.num_chunks, planes = scale_planes(&c->cfg);
+  if (!worker_rates && !server_rates) return fail(OB_EINVAL, "ob_quant_rates: no output");
+  if (worker_rates && !c->bits_w && c->words > 0) return fail(OB_EINVAL, "ob_quant_rates: the ctx has no bits_w");
+  if (server_rates && !c->bits_srv && c->words > 0) return fail(OB_EINVAL, "ob_quant_rates: the ctx has no bits_srv");
+  DeviceGuard dg(c->device);
+  if (!dg.ok) return fail(OB_ECUDA, "cannot select device %d", c->device);
+  if (worker_rates && (r = check_dev(worker_rates, W * C * planes, "worker_rates", c->device, kAlignWords)) != OB_OK)
+    return r;
+  if (server_rates && (r = check_dev(server_rates, C * planes, "server_rates", c->device, kAlignWords)) != OB_OK)
+    return r;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // Reuses the partial-sum scratch of the step: call it between steps on the same stream.
+  auto rates = [&](const uint32_t* bits, int rows, double* part, float* out) {
+    for (int pl = 0; pl < int(planes); ++pl) {
+      if (c->T > 0) {
+        auto k = ob::k_sign_count;
+        const int g = grid_for(c, k, rows * c->T);
+        launch(c, OB_K_SIGN_COUNT, st, [&] { pdl(k, g, ob::kBlock, st, c->L, rows, bits, pl, part); });
+      }
+      launch(c, OB_K_FINALIZE_SCALE, st, [&] {
+        pdl(ob::k_finalize_rate, dim3(unsigned(C), unsigned(rows)), ob::kFinalizeThreads, st,
+            c->L, part, c->T, out, int(planes), pl);
+      });
+    }
+  };
+  if (worker_rates) rates(c->bits_w, int(W), c->part_w, worker_rates);
+  if (server_rates) rates(c->bits_srv, 1, c->part_srv, server_rates);
+  return check_launch("ob_quant_rates");
 }
 
 ob_err ob_profile_start(ob_ctx* c, int32_t capacity) {
@@ -1099,7 +1281,7 @@ const char* ob_kernel_name(int32_t kind) {
       "k_ternary_step", "k_ternary_compress", "k_ternary_server", "k_ternary_update",
       "k_tb_resid_norm", "k_tb_pack", "k_tb_server_norm", "k_tb_server_update",
       "k_worker_pack_cached", "k_server_update_cached", "k_tb_pack_cached", "k_tb_server_norm_cached",
-      "k_tb_server_update_cached"};
+      "k_tb_server_update_cached", "k_local_step", "k_sign_count", "k_grad_mean"};
   return (kind >= 0 && kind < OB_K_KINDS) ? names[kind] : "";
 }
 
@@ -1129,8 +1311,8 @@ struct NoAllocDevice {
   bool ready = false;
   char* scratch = nullptr;   // device address of g_noalloc_scratch on this device
   int num_sms = 0;
-  int occ_norm[2] = {1, 1};  // resident CTAs per SM: [f32, bf16]
-  int occ_pack[2] = {1, 1};
+  int occ_norm[2][2] = {{1, 1}, {1, 1}};  // resident CTAs per SM: [bf16 grads][clip]
+  int occ_pack[2][2] = {{1, 1}, {1, 1}};
 };
 
 std::mutex g_noalloc_mu;
@@ -1158,10 +1340,15 @@ ob_err noalloc_setup(int device, NoAllocDevice** out) {
     if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(no-alloc scratch)");
     if ((e = cudaDeviceGetAttribute(&d.num_sms, cudaDevAttrMultiProcessorCount, device)) != cudaSuccess)
       return cuda_fail(e, "cudaDeviceGetAttribute");
-    d.occ_norm[0] = occupancy(reinterpret_cast<const void*>(ob::k_worker_norm<float, float, true>));
-    d.occ_norm[1] = occupancy(reinterpret_cast<const void*>(ob::k_worker_norm<uint16_t, float, true>));
-    d.occ_pack[0] = occupancy(reinterpret_cast<const void*>(ob::k_worker_pack<float, float, false, true, false, 2, false>));
-    d.occ_pack[1] = occupancy(reinterpret_cast<const void*>(ob::k_worker_pack<uint16_t, float, false, true, false, 2, false>));
+    // Every instance that a call may launch, so each grid is sized for its own kernel.
+    d.occ_norm[0][0] = occupancy(reinterpret_cast<const void*>(ob::k_worker_norm<float, float, false>));
+    d.occ_norm[0][1] = occupancy(reinterpret_cast<const void*>(ob::k_worker_norm<float, float, true>));
+    d.occ_norm[1][0] = occupancy(reinterpret_cast<const void*>(ob::k_worker_norm<uint16_t, float, false>));
+    d.occ_norm[1][1] = occupancy(reinterpret_cast<const void*>(ob::k_worker_norm<uint16_t, float, true>));
+    d.occ_pack[0][0] = occupancy(reinterpret_cast<const void*>(ob::k_worker_pack<float, float, false, false, false, 2, false>));
+    d.occ_pack[0][1] = occupancy(reinterpret_cast<const void*>(ob::k_worker_pack<float, float, false, true, false, 2, false>));
+    d.occ_pack[1][0] = occupancy(reinterpret_cast<const void*>(ob::k_worker_pack<uint16_t, float, false, false, false, 2, false>));
+    d.occ_pack[1][1] = occupancy(reinterpret_cast<const void*>(ob::k_worker_pack<uint16_t, float, false, true, false, 2, false>));
     d.scratch = static_cast<char*>(ptr);
     d.ready = true;
   }
@@ -1202,6 +1389,16 @@ extern "C" ob_err ob_compress_noalloc(const ob_config* cfg, const void* grads, f
   int device = 0;
   cudaError_t e = cudaGetDevice(&device);
   if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // The chunk tables travel from a host buffer that the next call rewrites; a
+  // copy recorded into a graph would read whatever that buffer holds at replay.
+  // (Checked before any other runtime call, so a refused call leaves the
+  // capture untouched.)
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  if ((e = cudaStreamIsCapturing(st, &cap)) != cudaSuccess) return cuda_fail(e, "ob_compress_noalloc: cudaStreamIsCapturing");
+  if (cap != cudaStreamCaptureStatusNone)
+    return fail(OB_EINVAL, "ob_compress_noalloc: the stream is being captured into a graph; "
+                           "this call copies its chunk tables from a host buffer that every call rewrites");
   struct { const void* p; int64_t count; const char* name; uintptr_t align; } bufs[] = {
       {grads, W * n, "grads", kAlignElems}, {err, W * n, "err", kAlignElems},
       {bits_w, W * words, "bits_w", kAlignWords}, {s_w, W * C, "s_w", kAlignWords}};
@@ -1227,7 +1424,6 @@ extern "C" ob_err ob_compress_noalloc(const ob_config* cfg, const void* grads, f
     h_tp[k + 1] = h_tp[k] + (nk + ob::kTile - 1) / ob::kTile;
     h_vec[k] = (o % 8 == 0) && (nk % 8 == 0) && (W == 1 || n % 8 == 0);
   }
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
   if ((e = cudaMemcpyAsync(d->scratch, g_noalloc_header, status_at + sizeof(uint32_t),
                            cudaMemcpyHostToDevice, st)) != cudaSuccess)
     return cuda_fail(e, "ob_compress_noalloc: header copy");
@@ -1247,7 +1443,7 @@ extern "C" ob_err ob_compress_noalloc(const ob_config* cfg, const void* grads, f
   const float clip = cfg->clip;
   const bool cl = clip > 0.0f;
   if (T > 0) {
-    const int g1 = noalloc_grid(d->num_sms, d->occ_norm[bf], W * T);
+    const int g1 = noalloc_grid(d->num_sms, d->occ_norm[bf][cl ? 1 : 0], W * T);
     const uint16_t* gh = static_cast<const uint16_t*>(grads);
     const float* gf = static_cast<const float*>(grads);
     if (bf && cl) ob::k_worker_norm<uint16_t, float, true><<<g1, ob::kBlock, 0, st>>>(L, int(W), gh, err, clip, part, status);
@@ -1257,7 +1453,7 @@ extern "C" ob_err ob_compress_noalloc(const ob_config* cfg, const void* grads, f
   }
   ob::k_finalize_scale<true><<<dim3(unsigned(C), unsigned(W)), ob::kFinalizeThreads, 0, st>>>(L, part, L.tp, 1, T, s_w, 1, 0);
   if (T > 0) {
-    const int g2 = noalloc_grid(d->num_sms, d->occ_pack[bf], T);
+    const int g2 = noalloc_grid(d->num_sms, d->occ_pack[bf][cl ? 1 : 0], T);
     const uint16_t* gh = static_cast<const uint16_t*>(grads);
     const float* gf = static_cast<const float*>(grads);
     if (bf && cl) ob::k_worker_pack<uint16_t, float, false, true, false, 2, false><<<g2, ob::kBlock, 0, st>>>(L, int(W), gh, err, s_w, bits_w, nullptr, nullptr, nullptr, clip, status);

@@ -161,6 +161,13 @@ class OneBitAdam:
         error buffers untouched.  Which steps refresh is the caller's schedule."""
         L.ob_refresh_step(self.ctx, self._grads_ptr(grads), self._stream())
 
+    def local_step(self, grads: torch.Tensor) -> None:
+        """0/1 Adam local step (compressed phase): nothing is sent; each worker's
+        gradient is kept in its error buffer for the next synchronised step, and
+        p moves with the current m and v.  Which steps are local is the caller's
+        schedule."""
+        L.ob_local_step(self.ctx, self._grads_ptr(grads), self._stream())
+
     def compress(self, grads: torch.Tensor) -> None:
         """Worker stage: err, bits_w, s_w."""
         L.ob_compress(self.ctx, self._grads_ptr(grads), self._stream())
@@ -182,6 +189,18 @@ class OneBitAdam:
         L.ob_error_norms(self.ctx, _ptr(wn) if wn.numel() else 0,
                          _ptr(sn) if sn is not None and sn.numel() else 0, self._stream())
         return wn, sn
+
+    def quant_rates(self):
+        """(worker rates [W, C(, 2)], server rates [C(, 2)]): per chunk the fraction
+        of elements the last step sent as +1 (theoretical value 1/2), as device
+        tensors (monitoring; the CANN article's quantisation-rate check).  Not
+        available under the momentum-error rule."""
+        planes = (2,) if self.rule == L.OB_RULE_TWO_BIT else ()
+        wr = torch.empty((self.W, self.C, *planes), dtype=torch.float32, device=self.device)
+        sr = torch.empty((self.C, *planes), dtype=torch.float32, device=self.device)
+        L.ob_quant_rates(self.ctx, _ptr(wr) if wr.numel() else 0, _ptr(sr) if sr.numel() else 0,
+                         self._stream())
+        return wr, sr
 
     def status(self, clear: bool = False) -> int:
         return L.ob_get_status(self.ctx, clear, self._stream())

@@ -121,7 +121,12 @@ typedef struct {
  * Host-only; validates the config.  words_total must be non-NULL. */
 ob_err ob_layout(const ob_config* cfg, int64_t* words_total);
 
-/* Create a ctx over caller-owned DEVICE buffers (float32 unless stated):
+/* Create a ctx: the optimizer state of the CANN 1-bit Adam article, section 3.1
+ * (OneBitAdamState: an error-feedback buffer of the parameters' shape, the
+ * first and second moments, beta1/beta2/eps and the step count), here with one
+ * error buffer per worker, the server error buffer, the packed messages and
+ * their scales, all caller-owned.
+ * Create it over caller-owned DEVICE buffers (float32 unless stated):
  *   p, m, v: [n];  err: [W][n] (worker-major), srv_err: [n], both of err_dtype;
  *   bits_w: uint32 [W][words_total];  s_w: [W][C];
  *   bits_srv: uint32 [words_total];  s_srv: [C].
@@ -149,7 +154,11 @@ ob_err ob_create(const ob_config* cfg, float* p, float* m, float* v, void* err,
                  void* srv_err, uint32_t* bits_w, float* s_w, uint32_t* bits_srv,
                  float* s_srv, ob_ctx** out);
 
-/* One full-precision warmup step (step < freeze_step, else OB_EPHASE):
+/* One full-precision warmup step ("DeepSpeed Communication Compression and
+ * Hiding": the `step < freeze_step` branch of the listing in section "1-bit
+ * Adam" 机制 -- average the workers' gradients, then the Adam moments of section
+ * "基线：Adam 为什么难压缩" -- and the listing's last line, the parameter update);
+ * step < freeze_step, else OB_EPHASE:
  *   g = (sum_w g_w) / W;  m = b1 m + (1-b1) g;  v = b2 v + (1-b2) g^2;
  *   Adam: p -= lr m / (sqrt(v) + eps);  LAMB: per-layer trust-ratio update.
  * grads: DEVICE [W][n] of grad_dtype.  Error buffers are not touched. */
@@ -164,20 +173,45 @@ ob_err ob_warmup_step(ob_ctx* ctx, const void* grads, void* stream);
  * step counter. */
 ob_err ob_refresh_step(ob_ctx* ctx, const void* grads, void* stream);
 
-/* Worker stage only (compressed phase): for every worker and chunk,
+/* The warmup's synchronisation alone ("DeepSpeed Communication Compression and
+ * Hiding", section "1-bit Adam" 机制: the listing's `g = allreduce(local_grad)`
+ * line before freeze_step, read as the float32 mean of the workers'
+ * gradients): mean[i] = (sum_{w=0..W-1} g_w[i]) / W, float additions in
+ * ascending w and one division, as ob_warmup_step forms it.  grads: DEVICE
+ * [W][n] of grad_dtype; mean: DEVICE float32 [n], 32-byte aligned.  An
+ * ob_warmup_step on a one-worker float32 ctx over `mean` then leaves p, m and v
+ * as ob_warmup_step on the W gradients does, so a data-parallel driver can
+ * average each owner's slice of the gradients instead of gathering every
+ * worker's whole gradient.  Any phase; the step counter is unchanged; a
+ * non-finite mean raises OB_STATUS_NONFINITE. */
+ob_err ob_mean_grads(ob_ctx* ctx, const void* grads, float* mean, void* stream);
+
+/* Worker stage only ("DeepSpeed Communication Compression and Hiding", section
+ * "1-bit Adam" 机制, the listing's `compensated = local_grad + error`,
+ * `q, scale = one_bit_quantize(compensated)` and -- for the worker's own part of
+ * the residual -- `error = compensated - g_hat` lines; compressed phase): for
+ * every worker and chunk,
  * c = clip(g_w) + err_w, s_w = ||c|| / sqrt(n_k), bits_w = sign(c),
  * err_w = c - s_w sign(c).  grads: DEVICE [W][n].  Step counter unchanged.
  * OB_RULE_MOMENTUM_ERROR: bits_w = int8 codes sign(c), err_w = beta1 err_w +
  * (1 - beta1)(c - sign(c)). */
 ob_err ob_compress(ob_ctx* ctx, const void* grads, void* stream);
 
-/* Server stage only (the compressed allreduce) from bits_w / s_w:
+/* Server stage only ("DeepSpeed Communication Compression and Hiding", section
+ * "1-bit Adam" 机制, the listing's `q_global = compressed_allreduce(q, scale)`
+ * line: average the workers' messages and re-compress them with a server error
+ * buffer) from bits_w / s_w:
  * c_srv = mean_w(s_w sign_w) + srv_err, s_srv = ||c_srv|| / sqrt(n_k),
  * bits_srv = sign(c_srv), srv_err = c_srv - s_srv sign(c_srv).
  * OB_RULE_MOMENTUM_ERROR: bits_srv = per-element sum of the W int8 codes. */
 ob_err ob_server_reduce(ob_ctx* ctx, void* stream);
 
-/* grads != NULL: the whole fused compressed step (worker stage, server stage,
+/* The compressed-phase step ("DeepSpeed Communication Compression and Hiding",
+ * section "1-bit Adam" 机制: the listing's `else` branch, then
+ * `g_hat = dequantize(q_global)`, `m = beta1 * m + (1 - beta1) * g_hat` with v
+ * frozen, and `param -= lr * m / (sqrt(v_frozen) + eps)`; section "1-bit LAMB"
+ * for the trust-ratio update under OB_LAMB).
+ * grads != NULL: the whole fused compressed step (worker stage, server stage,
  * update) on DEVICE grads [W][n].  grads == NULL: the update alone from
  * bits_srv / s_srv (g_hat = s_srv sign), after ob_compress + ob_server_reduce.
  * Advances the step counter.  OB_EPHASE while step < freeze_step.
@@ -186,7 +220,9 @@ ob_err ob_server_reduce(ob_ctx* ctx, void* stream);
  * neither bits_w nor bits_srv. */
 ob_err ob_step(ob_ctx* ctx, const void* grads, void* stream);
 
-/* Same as ob_step(ctx, grads, ...) with the gradients in HOST memory:
+/* The same passage as ob_step ("DeepSpeed Communication Compression and
+ * Hiding", section "1-bit Adam" 机制, the compressed-phase branch and update),
+ * with the gradients in HOST memory:
  * copies [W][n] grad_dtype elements from host_grads into dev_staging (a
  * caller-owned DEVICE buffer of that size, 32-byte aligned), then runs the
  * fused step on `stream`.  The copy runs on an internal copy stream (created on
@@ -219,6 +255,37 @@ ob_err ob_set_step(ob_ctx* ctx, int64_t step);
  * steps (same stream); it does not change any state. */
 ob_err ob_error_norms(ob_ctx* ctx, float* worker_norms, float* server_norms, void* stream);
 
+/* Quantisation-rate monitoring (CANN 1-bit Adam article, section 8, "监控指标":
+ * watch the gradient quantisation rate, which should stay near its theoretical
+ * value).  The article gives no formula; here the rate of a chunk is the
+ * fraction of its n_k elements sent as +1 (sign bit set), whose theoretical
+ * value is 1/2 for a message symmetric about zero.  Writes, from the sign words
+ * the last step or stage call left in bits_w / bits_srv,
+ *   worker_rates[(w * C + k) * planes + p]  and  server_rates[k * planes + p]
+ * (DEVICE float arrays, 4-byte aligned; either may be NULL; planes = 2 under
+ * OB_RULE_TWO_BIT -- plane 1 the signs of c, plane 2 the signs of its residual --
+ * else 1) as (float)(count / n_k), the count taken over the n_k real bits only;
+ * an empty chunk gives 0.  OB_EINVAL under OB_RULE_MOMENTUM_ERROR (ternary codes,
+ * no sign bits).  Uses the ctx scratch, so it must be ordered with the ctx's
+ * steps (same stream); it changes no state. */
+ob_err ob_quant_rates(ob_ctx* ctx, float* worker_rates, float* server_rates, void* stream);
+
+/* 0/1 Adam local step ("DeepSpeed Communication Compression and Hiding",
+ * section "0/1 Adam": local updates lower the synchronisation frequency; the
+ * listing moves param with the current m and v on every step and updates m only
+ * from a synchronised g_hat).  The page gives no formula for a local step; here
+ * it sends nothing, keeps each worker's gradient for the next synchronised
+ * step in its error buffer, and moves the parameters with the current m and v:
+ *   err_w = clip(g_w) + err_w   (every worker; the worker stage's addition)
+ *   Adam: p = p - lr m / (sqrt(v) + eps)
+ *   LAMB: u = m / (sqrt(v) + eps), r_l = ||p_l|| / ||u_l||, p -= lr r_l u
+ * m, v, srv_err and the packed words are untouched.  grads: DEVICE [W][n] of
+ * grad_dtype.  Compressed phase only (OB_EPHASE while step < freeze_step); the
+ * caller chooses which steps are local (the page gives no schedule).  OB_EINVAL
+ * under OB_RULE_MOMENTUM_ERROR, whose error buffer is a momentum, not a sum.
+ * Advances the step counter. */
+ob_err ob_local_step(ob_ctx* ctx, const void* grads, void* stream);
+
 /* ---- profiling (not part of the method) ----------------------------------
  * Kernel kinds the library launches, for per-kernel timing: */
 enum {
@@ -246,7 +313,10 @@ enum {
   OB_K_TB_PACK_CACHED = 18,
   OB_K_TB_SERVER_NORM_CACHED = 19,
   OB_K_TB_SERVER_UPDATE_CACHED = 20,
-  OB_K_KINDS = 21
+  OB_K_LOCAL_STEP = 21,      /* 0/1 Adam local step */
+  OB_K_SIGN_COUNT = 22,      /* quantisation rate: per-tile counts of set sign bits */
+  OB_K_GRAD_MEAN = 23,       /* full-precision average of the workers' gradients */
+  OB_K_KINDS = 24
 };
 
 /* Start recording a CUDA event pair around each of the next `capacity`
@@ -295,9 +365,13 @@ int64_t ob_launch_count(const ob_ctx* ctx);
  * different host threads without ordering) race and give wrong results;
  * order them on one stream.  Each call rewrites the tables and clears the
  * status word it uses.  The first call on each device looks up the array's
- * device address (cudaGetSymbolAddress) with that device current; make that
- * first call before any stream capture begins.  Not-finite flags are not
- * reported by this call (the ctx path's ob_get_status has them). */
+ * device address (cudaGetSymbolAddress) with that device current.  The chunk
+ * tables are copied from a host buffer that every call rewrites, so the call
+ * returns OB_EINVAL while `stream` is being captured into a CUDA graph.
+ * Non-finite input: there is no status word to read back; instead a NaN or
+ * infinite compensated value c in chunk k of worker w makes s_w[w][k] NaN or
+ * infinite (the scale of a chunk of finite values is always finite), so a
+ * caller checks the scales. */
 ob_err ob_compress_noalloc(const ob_config* cfg, const void* grads, float* err,
                            uint32_t* bits_w, float* s_w, void* stream);
 
