@@ -18,8 +18,17 @@ and every float operation are the ones the single-GPU path (and the oracle)
 computes with W workers: the result is the same, bit for bit.  The flat
 buffer groups chunks by owner, so each exchange moves one contiguous slice
 per peer: about n/32 words plus C scales in each direction per step, 1/32 of an
-fp32 allreduce.  Warmup steps all-gather the full-precision gradients and run
-the W-worker warmup kernel, which sums them in rank order like the oracle.
+fp32 allreduce.  A warmup step averages the full-precision gradients owner by
+owner: every rank sends owner o its gradient slice of o's chunks (n / W
+elements to each peer), the owner averages the W slices in rank order (the
+oracle's float sum, then / W), and the owners send the averaged slices to
+every rank (float32), which runs a one-worker warmup on the average.  Per rank
+that moves about n gradient elements plus n floats, instead of the W whole
+gradients an all-gather of gradients would.  The averaging and the one-worker
+warmup round exactly as the W-worker warmup does.
+
+0/1 Adam's local steps (``local_step``) exchange nothing: every rank keeps its
+gradient in its error buffer and moves its replica with the current m and v.
 
 The arithmetic runs in the CUDA library (``CudaStages``); this module only
 plans the layout and moves packed words between ranks (NCCL on GPUs; gloo
@@ -130,7 +139,9 @@ class CudaStages:
                     words/scales (filled by exchange 2) -> worker stage, update.
     server (W = world, owned chunks only): srv_err, the W workers' words/scales
                     of the owned chunks (filled by exchange 1) -> server stage.
-    warm   (W = world, shares p, m, v): the full-precision warmup step.
+    warm   (W = 1, float32 gradients, shares p, m, v): the full-precision warmup
+                    step on the averaged gradient (the server ctx averages the
+                    owned slices of the W ranks' gradients).
     update (momentum-error rule only; W = world, shares p, m, v, bits_srv): the
                     update divides the code sums by W, which the local ctx's W = 1
                     would get wrong.
@@ -199,8 +210,14 @@ class CudaStages:
                                           ptr(self.bits_srv_own), ptr(self.s_srv_own))
             self.warm = 0
             if warmup:
-                self.warm = L.ob_create(cfg(layout.offsets, W, 1 << 30), ptr(self.p), ptr(self.m),
-                                        ptr(self.v), 0, 0, 0, 0, 0, 0)
+                c_warm, arr = L.make_config(n, layout.offsets, 1, L.OB_F32, opt, freeze_step=1 << 30,
+                                            rule=code_rule, **hp)
+                self._keep.append(arr)
+                self.warm = L.ob_create(c_warm, ptr(self.p), ptr(self.m), ptr(self.v), 0, 0, 0, 0, 0, 0)
+            self.grad_dtype = torch.bfloat16 if gd == L.OB_BF16 else f32
+            self._warm_grads: Optional[torch.Tensor] = None   # [W, n_own]: the owned slices of every rank
+            self._warm_own: Optional[torch.Tensor] = None     # [n_own]: their average (aligned for the kernel)
+            self._warm_mean: Optional[torch.Tensor] = None    # [n]: the averaged gradient
             # The momentum-error rule's update divides the code sums by W, so it runs
             # on a ctx of W = world workers (the worker stage's ctx has one).  The
             # scaled rules' update reads averaged scales: the local ctx serves.
@@ -235,8 +252,29 @@ class CudaStages:
     def _stream(self) -> int:
         return int(torch.cuda.current_stream(self.device).cuda_stream)
 
-    def warmup(self, gathered: torch.Tensor) -> None:
-        self.L.ob_warmup_step(self.warm, int(gathered.data_ptr()), self._stream())
+    # -- warmup: average owner by owner, then a one-worker step on the average --
+    def warm_buffers(self) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
+        """([W, n_own] owned gradient slices of every rank, [n_own] their float32
+        average, [n] float32 averaged gradient), allocated on the first warmup step."""
+        if self._warm_grads is None:
+            dev = self.device
+            self._warm_grads = torch.zeros((self.layout.world, self.n_own), dtype=self.grad_dtype, device=dev)
+            self._warm_own = torch.zeros(self.n_own, dtype=torch.float32, device=dev)
+            self._warm_mean = torch.zeros(self.layout.n, dtype=torch.float32, device=dev)
+        return self._warm_grads, self._warm_own, self._warm_mean
+
+    def warm_mean_own(self) -> None:
+        """Average the W ranks' slices of the owned chunks (into the [n_own] buffer)."""
+        if self.server:
+            self.L.ob_mean_grads(self.server, int(self._warm_grads.data_ptr()), int(self._warm_own.data_ptr()),
+                                 self._stream())
+
+    def warmup(self) -> None:
+        """The full-precision step on the averaged gradient."""
+        self.L.ob_warmup_step(self.warm, int(self._warm_mean.data_ptr()), self._stream())
+
+    def local_step(self, grad: torch.Tensor) -> None:
+        self.L.ob_local_step(self.local, int(grad.data_ptr()), self._stream())
 
     def compress(self, grad: torch.Tensor) -> None:
         self.L.ob_compress(self.local, int(grad.data_ptr()), self._stream())
@@ -329,6 +367,9 @@ class DistributedOneBitAdam:
         stream wait for the transfer, so kernels enqueued meanwhile overlap it)."""
         host = self._stage_on_host
         ops, copy_back = [], []
+        as_bits = lambda t: t.view(torch.int16) if t.dtype == torch.bfloat16 else t  # noqa: E731
+        sends = [(as_bits(t), peer) for t, peer in sends]
+        recvs = [(as_bits(t), peer) for t, peer in recvs]
         for t, peer in sends:
             if t.numel():
                 src = t.detach().to("cpu") if host and t.is_cuda else t.contiguous()
@@ -407,15 +448,28 @@ class DistributedOneBitAdam:
             pend.wait()
             s.apply_slice((r - i) % W)
 
-    def _gather_grads(self, grad: torch.Tensor) -> torch.Tensor:
-        """All ranks' full-precision gradients, rank-major [world, n] (warmup)."""
-        if self._stage_on_host and grad.is_cuda:
-            parts = [torch.empty(grad.shape, dtype=grad.dtype) for _ in range(self.world)]
-            dist.all_gather(parts, grad.to("cpu"), group=self.group)
-            return torch.stack(parts).to(grad.device)
-        parts = [torch.empty_like(grad) for _ in range(self.world)]
-        dist.all_gather(parts, grad, group=self.group)
-        return torch.stack(parts)
+    def _warmup_step(self, grad: torch.Tensor) -> None:
+        """Full-precision step: (1) every rank sends owner o its gradient slice of
+        o's chunks; (2) each owner averages the W slices in rank order; (3) the
+        owners send their averaged slices to every rank; (4) every rank runs the
+        one-worker warmup on the averaged gradient."""
+        L, s, r = self.layout, self.stages, self.rank
+        G, own, gbar = s.warm_buffers()
+        sends, recvs = [], []
+        for o in range(self.world):
+            es = L.eslice(o)
+            if o == r:
+                G[r].copy_(grad[es])
+            else:
+                sends.append((grad[es], o))
+                recvs.append((G[o], o))
+        self._p2p(sends, recvs)
+        s.warm_mean_own()
+        gbar[L.eslice(r)].copy_(own)
+        sends = [(own, o) for o in range(self.world) if o != r]
+        recvs = [(gbar[L.eslice(o)], o) for o in range(self.world) if o != r]
+        self._p2p(sends, recvs)
+        s.warmup()
 
     @property
     def in_warmup(self) -> bool:
@@ -425,7 +479,7 @@ class DistributedOneBitAdam:
         if grad.numel() != self.layout.n:
             raise ValueError(f"gradient must hold {self.layout.n} elements (layout order)")
         if self.in_warmup:
-            self.stages.warmup(self._gather_grads(grad.reshape(-1)))
+            self._warmup_step(grad.reshape(-1))
         elif getattr(self.stages, "pipelined", False):
             self._compressed_step_pipelined(grad.reshape(-1))
         else:
@@ -434,6 +488,18 @@ class DistributedOneBitAdam:
             self.stages.server_reduce()
             self._from_owners()
             self.stages.apply()
+        self.step_count += 1
+
+    def local_step(self, grad: torch.Tensor) -> None:
+        """0/1 Adam local step (compressed phase): no exchange; this rank keeps its
+        gradient in its error buffer for the next synchronised step and moves its
+        replica with the current m and v.  Every rank must take the same
+        schedule of local and synchronised steps."""
+        if grad.numel() != self.layout.n:
+            raise ValueError(f"gradient must hold {self.layout.n} elements (layout order)")
+        if self.in_warmup:
+            raise ValueError("local steps belong to the compressed phase")
+        self.stages.local_step(grad.reshape(-1))
         self.step_count += 1
 
     def status(self) -> int:

@@ -26,9 +26,11 @@ class OracleStages:
     """``pipelined``: also offer the per-owner-slice stages (compress_slice,
     apply_slice), so the driver takes its overlapped schedule."""
 
-    def __init__(self, layout, rank, optimizer="adam", clip=0.0, pipelined=False, rule="scaled"):
+    def __init__(self, layout, rank, optimizer="adam", clip=0.0, pipelined=False, rule="scaled",
+                 grad_dtype="f32"):
         import oracle
         self.o = oracle.get()
+        self.grad_dtype = grad_dtype
         self.layout, self.rank = layout, rank
         self.opt = oracle.LAMB if optimizer == "lamb" else oracle.ADAM
         self.clip = clip
@@ -58,11 +60,40 @@ class OracleStages:
     def _u32(t):
         return t.numpy().view(np.uint32)
 
-    def warmup(self, gathered):
+    # -- warmup: the owned slices of every rank are averaged by the owner ------------
+    def warm_buffers(self):
+        if not hasattr(self, "_warm"):
+            n_own = int(self.off_own[-1])
+            gdt = torch.bfloat16 if self.grad_dtype == "bf16" else torch.float32
+            self._warm = (torch.zeros((self.layout.world, n_own), dtype=gdt), torch.zeros(n_own),
+                          torch.zeros(self.layout.n))
+        return self._warm
+
+    def warm_mean_own(self):
+        """The owner's average of the W slices: float32 additions in rank order,
+        then one division by W (numpy's IEEE float32 arithmetic, the statement
+        the oracle's warmup makes before its moments)."""
+        G, own, _ = self._warm
+        rows = self._grad_rows(G) if G.dtype == torch.bfloat16 else G.numpy()
+        if rows.dtype == np.uint16:
+            rows = (rows.astype(np.uint32) << np.uint32(16)).view(np.float32).reshape(G.shape)
+        acc = np.zeros(rows.shape[1], np.float32)
+        for w in range(rows.shape[0]):
+            acc = (acc + rows[w]).astype(np.float32)
+        own.numpy()[:] = (acc / np.float32(rows.shape[0])).astype(np.float32)
+
+    def warmup(self):
+        """The oracle's warmup with one worker on the averaged gradient."""
         f = {k: np.float32(v) for k, v in HP.items()}
-        self.flags |= self.o.warmup(self.layout.offsets, np.ascontiguousarray(gathered.numpy()),
-                                    self.m.numpy(), self.v.numpy(), self.p.numpy(), f["beta1"],
-                                    f["beta2"], f["lr"], f["eps"], optimizer=self.opt)
+        gbar = np.ascontiguousarray(self._warm[2].numpy().reshape(1, -1))
+        self.flags |= self.o.warmup(self.layout.offsets, gbar, self.m.numpy(), self.v.numpy(), self.p.numpy(),
+                                    f["beta1"], f["beta2"], f["lr"], f["eps"], optimizer=self.opt)
+
+    def local_step(self, grad):
+        f = {k: np.float32(v) for k, v in HP.items()}
+        st = {"p": self.p.numpy(), "m": self.m.numpy(), "v": self.v.numpy(), "err": self.err.numpy()}
+        self.flags |= self.o.local_step(self.layout.offsets, self._grad_rows(grad), st, f["lr"], f["eps"],
+                                        clip=self.clip, optimizer=self.opt)
 
     @staticmethod
     def _grad_rows(grad):
@@ -186,7 +217,7 @@ def initial_state(wl, layout):
 
 
 def _rank_main(rank, world, port, sizes, wl_kw, steps, backend, device, q, die=None, timeout_s=120,
-               pipelined=False, rule="scaled"):
+               pipelined=False, rule="scaled", schedule=None):
     try:
         import sys
         sys.path.insert(0, ROOT)
@@ -203,7 +234,7 @@ def _rank_main(rank, world, port, sizes, wl_kw, steps, backend, device, q, die=N
         layout = plan(sizes, world, 4 if rule == "momentum" else 32, 2 if rule == "twobit" else 1)
         if device == "cpu":
             stages = OracleStages(layout, rank, optimizer=wl.optimizer, clip=wl.clip, pipelined=pipelined,
-                                  rule=rule)
+                                  rule=rule, grad_dtype=wl.grad_dtype)
         else:
             from bit_adam_error_b200.distributed import CudaStages
             stages = CudaStages(layout, rank, grad_dtype=wl.grad_dtype, optimizer=wl.optimizer,
@@ -219,7 +250,10 @@ def _rank_main(rank, world, port, sizes, wl_kw, steps, backend, device, q, die=N
             g = rank_inputs(wl, layout, rank, t)
             gt = torch.from_numpy(g.view(np.int16)).view(torch.bfloat16) if g.dtype == np.uint16 \
                 else torch.from_numpy(g)
-            drv.step(gt.to(stages.device))
+            if schedule is not None and schedule[t] == "L":
+                drv.local_step(gt.to(stages.device))
+            else:
+                drv.step(gt.to(stages.device))
         flags = drv.status()
         schedule = "pipelined" if getattr(stages, "pipelined", False) else "grouped"
         if device != "cpu":
@@ -241,14 +275,15 @@ def _rank_main(rank, world, port, sizes, wl_kw, steps, backend, device, q, die=N
 
 
 def run_ranks(sizes, world, wl_kw, steps, backend="gloo", device="cpu", timeout=600, pipelined=False,
-              rule="scaled"):
-    """Spawn `world` ranks; returns the list of per-rank final states."""
+              rule="scaled", schedule=None):
+    """Spawn `world` ranks; returns the list of per-rank final states.  ``schedule``:
+    one letter per step, "L" for a 0/1 Adam local step (else a regular step)."""
     import multiprocessing as mp
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = free_port()
     procs = [ctx.Process(target=_rank_main, args=(r, world, port, sizes, wl_kw, steps, backend, device, q),
-                         kwargs=dict(pipelined=pipelined, rule=rule)) for r in range(world)]
+                         kwargs=dict(pipelined=pipelined, rule=rule, schedule=schedule)) for r in range(world)]
     for pr in procs:
         pr.start()
     results = {}
@@ -266,8 +301,9 @@ def run_ranks(sizes, world, wl_kw, steps, backend="gloo", device="cpu", timeout=
     return [results[r] for r in range(world)]
 
 
-def reference(sizes, world, wl_kw, steps, rule="scaled"):
-    """The same workload as one W-worker oracle problem (caller's chunk order)."""
+def reference(sizes, world, wl_kw, steps, rule="scaled", schedule=None):
+    """The same workload as one W-worker oracle problem (caller's chunk order);
+    ``schedule`` as for run_ranks."""
     import oracle
     import workloads as WL
     wl = workload(sizes, world, **wl_kw)
@@ -287,6 +323,8 @@ def reference(sizes, world, wl_kw, steps, rule="scaled"):
         if t < wl.freeze_step:
             o.warmup(wl.offsets, g, st["m"], st["v"], st["p"], f["beta1"], f["beta2"], f["lr"], f["eps"],
                      optimizer=opt)
+        elif schedule is not None and schedule[t] == "L":
+            o.local_step(wl.offsets, g, st, f["lr"], f["eps"], clip=wl.clip, optimizer=opt)
         elif rule == "momentum":
             o.ternary_step(wl.offsets, g, st, f["beta1"], f["lr"], f["eps"], clip=wl.clip, optimizer=opt)
         elif rule == "twobit":

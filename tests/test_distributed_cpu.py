@@ -105,3 +105,43 @@ def test_two_bit_ranks_match_single_process_oracle(world, wl_kw, steps, pipeline
     wl, ref = reference(SIZES, world, wl_kw, steps, rule="twobit")
     compare(plan(SIZES, world, 32, 2), wl, ref, outs)
     assert all(o["flags"] == 0 for o in outs)
+
+
+@pytest.mark.parametrize("world,wl_kw", [
+    (2, dict(freeze_step=3)),
+    (3, dict(freeze_step=3, grad_dtype="bf16")),
+    (4, dict(freeze_step=2, optimizer="lamb")),
+    (5, dict(freeze_step=3, grad_dtype="bf16", optimizer="lamb")),
+])
+def test_warmup_exchange_owner_average(world, wl_kw):
+    """Warmup steps: every rank sends each owner its slice of the owner's
+    chunks, the owner averages the W slices in rank order, the averaged slices
+    return to every rank, and a one-worker warmup runs on the average.  The
+    result equals the W-worker oracle warmup bit for bit (all-warmup runs)."""
+    steps = wl_kw["freeze_step"]
+    outs = run_ranks(SIZES, world, wl_kw, steps)
+    wl, ref = reference(SIZES, world, wl_kw, steps)
+    lay = plan(SIZES, world)
+    import numpy as np
+    off = wl.offsets
+    for r, out in enumerate(outs):
+        for key in ("p", "m", "v"):
+            want = lay.to_layout([ref[key][off[k]:off[k + 1]] for k in range(wl.C)])
+            np.testing.assert_array_equal(out[key], want, err_msg=f"rank {r} {key}")
+        assert out["flags"] == 0
+
+
+@pytest.mark.parametrize("pipelined", [False, True], ids=["grouped", "pipelined"])
+@pytest.mark.parametrize("world,wl_kw,schedule", [
+    (2, dict(), "SLLSLS"),
+    (3, dict(freeze_step=1, grad_dtype="bf16"), "WSLSLL"),
+    (2, dict(optimizer="lamb", clip=2e-3), "SLSL"),
+])
+def test_local_steps_across_ranks(world, wl_kw, schedule, pipelined):
+    """0/1 Adam local steps in the data-parallel driver: no exchange, each rank
+    keeps its gradient in its error buffer and moves its replica; every rank
+    equals the W-worker oracle with the same schedule, bit for bit."""
+    outs = run_ranks(SIZES, world, wl_kw, len(schedule), pipelined=pipelined, schedule=schedule)
+    wl, ref = reference(SIZES, world, wl_kw, len(schedule), schedule=schedule)
+    compare(plan(SIZES, world), wl, ref, outs)
+    assert all(o["flags"] == 0 for o in outs)

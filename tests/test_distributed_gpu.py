@@ -61,3 +61,20 @@ def test_gpu_ranks_two_bit_rule(world, pipelined):
     assert all(o["flags"] == 0 for o in outs)
     want = "pipelined" if pipelined and world > 1 else "grouped"
     assert all(o["schedule"] == want for o in outs)
+
+
+@pytest.mark.parametrize("world,backend,wl_kw,schedule,pipelined", [
+    (1, "nccl", dict(freeze_step=2, grad_dtype="bf16"), "WWSLLS", True),
+    (2, "gloo", dict(freeze_step=1), "WSLSLL", True),
+    (3, "gloo", dict(freeze_step=2, optimizer="lamb", grad_dtype="bf16"), "WWSLS", False),
+])
+def test_gpu_ranks_warmup_exchange_and_local_steps(world, backend, wl_kw, schedule, pipelined):
+    """The owner-averaged warmup (each owner averages the ranks' slices of its
+    chunks with ob_mean_grads, then every rank runs a one-worker warmup on the
+    average) and 0/1 Adam local steps (ob_local_step, no exchange), against the
+    W-worker oracle with the same schedule."""
+    outs = run_ranks(SIZES, world, wl_kw, len(schedule), backend=backend, device="cuda:0",
+                     pipelined=pipelined, schedule=schedule)
+    wl, ref = reference(SIZES, world, wl_kw, len(schedule), schedule=schedule)
+    compare(plan(SIZES, world), wl, ref, outs, exact=False)
+    assert all(o["flags"] == 0 for o in outs)
