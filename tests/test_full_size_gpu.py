@@ -21,6 +21,11 @@ from gpu_harness import (F, HP, assert_bits, assert_scales, assert_state, dev, n
 
 pytestmark = [pytest.mark.gpu, pytest.mark.slow]
 
+# The scaled-sign rule's oracle step runs on every host core (bit-identical to
+# the single-thread oracle; tests/test_oracle_threads.py), which keeps the
+# full-size comparisons short.
+THREADS = oracle.host_threads()
+
 
 def sampled_chunks(wl):
     C = wl.C
@@ -44,7 +49,7 @@ def test_full_size_sampled_chunks(name):
     assert opt.status() == 0
     del G
 
-    o = oracle.get()
+    o = oracle.get_mt()
     wb = np.zeros(wl.C + 1, np.int64)
     np.cumsum([(s + 31) // 32 for s in wl.sizes], out=wb[1:])
     for k in sampled_chunks(wl):
@@ -61,7 +66,8 @@ def test_full_size_sampled_chunks(name):
                 o.warmup(off, g, ref["m"], ref["v"], ref["p"], F["beta1"], F["beta2"], F["lr"],
                          F["eps"], optimizer=opt_code)
             else:
-                o.step(off, g, ref, F["beta1"], F["lr"], F["eps"], clip=wl.clip, optimizer=opt_code)
+                o.step(off, g, ref, F["beta1"], F["lr"], F["eps"], clip=wl.clip, optimizer=opt_code,
+                       threads=THREADS)
         tag = f"{name} chunk {k}: "
         for key in ("p", "m", "v", "srv_err"):
             assert_state(tag + key, np_of(getattr(opt, key)[lo:hi]), ref[key], off)
@@ -71,6 +77,97 @@ def test_full_size_sampled_chunks(name):
         assert_scales(tag + "s_w", np_of(opt.s_w[:, k]), ref["s_w"][:, 0])
         assert_scales(tag + "s_srv", np_of(opt.s_srv[k:k + 1]), ref["s_srv"])
     opt.close()
+
+
+def test_gpt2xl_flat_hundred_chained_steps():
+    """The headline workload chained at full size: 100 compressed steps of the
+    1.5e9-element gpt2xl-flat buffer (W = 1, bf16 gradients) through
+    OneBitAdam.step, the call the benchmark times.  The gradient of step t is
+    pre-generated batch t mod 4 (four 3 GB batches stay on the device).
+
+    The oracle runs the same 100 steps on the first chunk (2^26 elements) and
+    the 23,604,992-element tail chunk, on their own (chunks are independent).
+    Checked:
+      * after 100 steps, each sampled chunk's p, m, err and srv_err within the
+        per-step parity bar of the oracle's, scales within 1e-5, and the
+        chunk's parameter norm within 1e-3 of the oracle's;
+      * the last step from identical input state: the oracle's step 100 run on
+        the GPU's own state after step 99 gives bit-exact sign words and the
+        same state (within the parity bar) as the GPU's step 100.
+    """
+    wl = WL.get_workload("gpt2xl-flat")
+    steps, batches = 100, 4
+    ks = (0, wl.C - 1)
+    torch.cuda.empty_cache()
+    opt = OneBitAdam(wl.offsets, wl.W, grad_dtype=wl.grad_dtype, optimizer=wl.optimizer,
+                     clip=wl.clip, freeze_step=wl.freeze_step, device=dev(), **HP)
+    upload_state(wl, opt.p, opt.v)
+    Gs = []
+    for j in range(batches):
+        G = torch.empty((wl.W, wl.n), dtype=torch.bfloat16, device=dev())
+        upload_grads(wl, j, G)
+        Gs.append(G)
+    spans = [(int(wl.offsets[k]), int(wl.offsets[k + 1])) for k in ks]
+    before_last = None
+    for t in range(steps):
+        if t == steps - 1:
+            torch.cuda.synchronize()
+            before_last = {key: np.concatenate([np_of(getattr(opt, key)[..., lo:hi]) for lo, hi in spans], axis=-1)
+                           for key in ("p", "m", "v", "err", "srv_err")}
+        opt.step(Gs[t % batches])
+    torch.cuda.synchronize()
+    assert opt.status() == 0
+    del Gs
+    torch.cuda.empty_cache()
+
+    wb = np.zeros(wl.C + 1, np.int64)
+    np.cumsum([(s + 31) // 32 for s in wl.sizes], out=wb[1:])
+    gpu = {key: np.concatenate([np_of(getattr(opt, key)[..., lo:hi]) for lo, hi in spans], axis=-1)
+           for key in ("p", "m", "v", "err", "srv_err")}
+    gpu["bits_w"] = np.concatenate([np_of(opt.bits_w[:, wb[k]:wb[k + 1]]) for k in ks], axis=-1)
+    gpu["bits_srv"] = np.concatenate([np_of(opt.bits_srv[wb[k]:wb[k + 1]]) for k in ks])
+    gpu["s_w"] = np.stack([np_of(opt.s_w[:, k]) for k in ks], axis=-1)
+    gpu["s_srv"] = np.array([np_of(opt.s_srv[k:k + 1])[0] for k in ks], np.float32)
+    opt.close()
+
+    # The two sampled chunks as one two-chunk problem, from the seeded state.
+    sizes = [wl.sizes[k] for k in ks]
+    off = np.array([0, sizes[0], sizes[0] + sizes[1]], np.int64)
+    n2 = int(off[-1])
+    grads = []
+    for j in range(batches):
+        g = np.empty((1, n2), np.uint16)
+        for i, k in enumerate(ks):
+            g[0, off[i]:off[i + 1]] = WL.chunk_grads(wl, j, 0, k)
+        grads.append(g)
+    p0, v0 = zip(*(WL.chunk_state(wl, k) for k in ks))
+    ref = {"p": np.concatenate(p0), "m": np.zeros(n2, np.float32), "v": np.concatenate(v0),
+           "err": np.zeros((1, n2), np.float32), "srv_err": np.zeros(n2, np.float32)}
+    o = oracle.get_mt()
+    for t in range(steps):
+        assert o.step(off, grads[t % batches], ref, F["beta1"], F["lr"], F["eps"], threads=THREADS) == 0
+
+    for key in ("p", "m", "v", "srv_err"):
+        assert_state("100 steps: " + key, gpu[key], ref[key], off)
+    assert_state("100 steps: err", gpu["err"], ref["err"], off)
+    assert_scales("100 steps: s_w", gpu["s_w"], ref["s_w"])
+    assert_scales("100 steps: s_srv", gpu["s_srv"], ref["s_srv"])
+    for i, k in enumerate(ks):
+        pg = gpu["p"][off[i]:off[i + 1]].astype(np.float64)
+        pr = ref["p"][off[i]:off[i + 1]].astype(np.float64)
+        rel = abs(np.linalg.norm(pg) - np.linalg.norm(pr)) / np.linalg.norm(pr)
+        assert rel <= 1e-3, (k, rel)
+
+    # Step 100 again, on the oracle, from the GPU's state after step 99.
+    last = {key: np.ascontiguousarray(val) for key, val in before_last.items()}
+    assert o.step(off, grads[(steps - 1) % batches], last, F["beta1"], F["lr"], F["eps"], threads=THREADS) == 0
+    assert_bits("step 100: bits_w", gpu["bits_w"], last["bits_w"])
+    assert_bits("step 100: bits_srv", gpu["bits_srv"], last["bits_srv"])
+    assert_scales("step 100: s_w", gpu["s_w"], last["s_w"])
+    assert_scales("step 100: s_srv", gpu["s_srv"], last["s_srv"])
+    for key in ("p", "m", "srv_err"):
+        assert_state("step 100: " + key, gpu[key], last[key], off)
+    assert_state("step 100: err", gpu["err"], last["err"], off)
 
 
 def test_row_longer_than_two_to_the_31():
@@ -88,7 +185,7 @@ def test_row_longer_than_two_to_the_31():
     torch.cuda.synchronize()
     assert opt.status() == 0
     del G
-    o = oracle.get()
+    o = oracle.get_mt()
     wb = np.zeros(wl.C + 1, np.int64)
     np.cumsum([(s + 31) // 32 for s in wl.sizes], out=wb[1:])
     for k in (0, wl.C - 2, wl.C - 1):
@@ -98,7 +195,7 @@ def test_row_longer_than_two_to_the_31():
         pk, vk = WL.chunk_state(wl, k)
         ref = {"p": pk, "m": np.zeros(nk, np.float32), "v": vk, "err": np.zeros((1, nk), np.float32),
                "srv_err": np.zeros(nk, np.float32)}
-        o.step(off, WL.chunk_grads(wl, 0, 0, k)[None, :], ref, F["beta1"], F["lr"], F["eps"])
+        o.step(off, WL.chunk_grads(wl, 0, 0, k)[None, :], ref, F["beta1"], F["lr"], F["eps"], threads=THREADS)
         tag = f"chunk {k} [{lo}, {hi}): "
         for key in ("p", "m", "srv_err"):
             assert_state(tag + key, np_of(getattr(opt, key)[lo:hi]), ref[key], off)

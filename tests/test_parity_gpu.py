@@ -197,16 +197,18 @@ def test_warmup_then_compressed(opt):
 
 
 @pytest.mark.parametrize("W,gdt,opt", [(1, "bf16", "adam"), (3, "f32", "adam"), (2, "f32", "lamb")])
-def test_fused_steps_many_tiles_per_cta(W, gdt, opt):
-    # ~12M elements: every CTA of the pipelined passes cycles its stage ring many
-    # times (block tiles of 2048 elements, one CTA per SM); chunks of uneven size.
+def test_fused_steps_many_tiles_per_warp(W, gdt, opt):
+    # ~12M elements: every warp of the persistent grid strides over many
+    # 512-element warp tiles, across chunk boundaries; chunks of uneven size,
+    # one of 40 elements and ones that end part-way through a tile.
     wl = small([1 << 23, 3 * (1 << 20) + 2048 * 7 + 8, 40, 2048 * 300 - 8 * 3], W, grad_dtype=gdt,
                optimizer=opt)
     run_chain(wl, 3)
 
 
-def test_fused_steps_many_workers_fallback():
-    # W = 1024: the pass-3 stage would not fit shared memory; the warp-tile kernel runs.
+def test_fused_steps_1024_workers():
+    # W = 1024, the largest worker count the library accepts: passes 1-2 loop
+    # over 1024 workers per tile, and pass 3 reads the cached server value.
     run_chain(small([2048, 1000, 24], 1024), 2)
 
 
