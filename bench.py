@@ -21,9 +21,12 @@ plain C statement of the method) on one host thread and on all host cores, on
 the same sample of whole chunks.  ``--impl reference`` times the oracle on all
 host cores, one bounded sample (chunk 0) per bench step.
 
-Multi-GPU: every rank runs an independent replica of the workload (the
-virtual workers of one replica live in one GPU's memory); no collective is on
-the data path, so scaling is weak.
+Multi-GPU (N > 1 under torchrun): real data parallelism -- rank w is worker
+w, holding the whole model and its own gradient of the workload; the
+compressed allreduce runs as two NCCL point-to-point exchanges of packed words
+around a chunk-owner server stage.  Per-rank work is fixed, so scaling is weak
+and ``value`` counts the gradient elements of all ranks.  ``--replicas`` times
+independent single-GPU replicas instead (no collective).
 """
 
 from __future__ import annotations
@@ -64,9 +67,9 @@ def parse_args():
                     help="use only the first K chunks of the workload (a smaller case, e.g. for ncu)")
     ap.add_argument("--grad-buffers", type=int, default=2,
                     help="distinct gradient batches cycled through the timed steps")
-    ap.add_argument("--phase", choices=["compressed", "refresh"], default="compressed",
-                    help="time the compressed step (default) or the full-precision variance-refresh "
-                         "step of 0/1 Adam")
+    ap.add_argument("--phase", choices=["compressed", "refresh", "local"], default="compressed",
+                    help="time the compressed step (default), the full-precision variance-refresh "
+                         "step of 0/1 Adam, or its local step")
     ap.add_argument("--rule", choices=["scaled", "momentum", "twobit"], default="scaled",
                     help="compression rule: scaled sign bits with worker and server error "
                          "(default), the momentum-error rule with int8 ternary codes, or "
@@ -74,8 +77,11 @@ def parse_args():
     ap.add_argument("--err-dtype", choices=["f32", "bf16"], default=None,
                     help="storage of the error buffers (default: the workload's, f32)")
     ap.add_argument("--dp", action="store_true",
-                    help="time the real data-parallel path (worker w = rank w, NCCL exchanges) "
-                         "instead of per-GPU replicas of the single-GPU step")
+                    help="time the real data-parallel path (worker w = rank w, NCCL exchanges) even "
+                         "at one GPU (with more than one GPU it is the default)")
+    ap.add_argument("--replicas", action="store_true",
+                    help="with more than one GPU, time independent replicas of the single-GPU step "
+                         "(no collective) instead of the data-parallel step")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     a = ap.parse_args()
@@ -135,6 +141,13 @@ def algo_bytes_per_elem(kind: str, wl) -> float:
         return 4.0
     if kind == "k_tb_server_update_cached":
         return 4 + eb + 1 / 4 + upd
+    # 0/1 Adam's local step: g, err r/w per worker; m, v, p reads (+ p write for Adam)
+    if kind == "k_local_step":
+        return (gb + 2 * eb) * W + (12 if wl.optimizer == "lamb" else 16)
+    if kind == "k_sign_count":           # the packed signs of every worker (monitoring)
+        return W / 8
+    if kind == "k_grad_mean":            # g of every worker in, one float out
+        return gb * W + 4.0
     return 0.0                           # finalisers: a few bytes per chunk
 
 
@@ -146,6 +159,8 @@ def step_bytes_per_elem(wl, phase: str = "compressed", rule: str = "scaled") -> 
     (bench.py also sums them from the kernels the timed steps actually ran)."""
     if phase == "refresh":
         return algo_bytes_per_elem("k_warmup", wl) + (16.0 if wl.optimizer == "lamb" else 0.0)
+    if phase == "local":
+        return algo_bytes_per_elem("k_local_step", wl) + (16.0 if wl.optimizer == "lamb" else 0.0)
     if rule == "momentum":
         return algo_bytes_per_elem("k_ternary_step", wl) + (16.0 if wl.optimizer == "lamb" else 0.0)
     cached = "_cached" if wl.W >= CACHE_MIN_W else ""
@@ -303,6 +318,8 @@ def _oracle_step(o, wl, off, g, st, phase, rule, threads=1):
     if phase == "refresh":
         o.warmup(off, g, st["m"], st["v"], st["p"], f(wl.beta1), f(wl.beta2), f(wl.lr), f(wl.eps),
                  optimizer=opt)
+    elif phase == "local":
+        o.local_step(off, g, st, f(wl.lr), f(wl.eps), clip=wl.clip, optimizer=opt)
     elif rule == "momentum":
         o.ternary_step(off, g, st, f(wl.beta1), f(wl.lr), f(wl.eps), clip=wl.clip, optimizer=opt)
     elif rule == "twobit":
@@ -478,7 +495,7 @@ def run_ours(args):
         dev_g.append(G)
     stream = torch.cuda.current_stream(device)
 
-    step_fn = opt.refresh_step if args.phase == "refresh" else opt.step
+    step_fn = {"refresh": opt.refresh_step, "local": opt.local_step}.get(args.phase, opt.step)
     for i in range(args.warmup):
         step_fn(dev_g[i % nbuf])
     torch.cuda.synchronize()
@@ -651,8 +668,13 @@ def fill_device_grads(wl, step, G) -> None:
 
 
 def run_dp(args):
-    """Data-parallel 1-bit Adam over the ranks: each rank is one worker (W = N),
-    compresses its own gradient, serves the chunks it owns and applies the update."""
+    """Data-parallel 1-bit Adam over the ranks: each rank is one worker (W = N)
+    holding the whole model and its own gradient; it compresses its gradient,
+    serves the chunks it owns (server stage between the two point-to-point
+    exchanges) and applies the update to its replica.  Per-rank work is one
+    gradient of n elements whatever N is, so scaling is weak and ``value`` is
+    the gradient elements of all ranks per second (N n / max-over-ranks step
+    time); ``model_value`` is n / step time."""
     import torch
     world, rank, local = dist_env()
     torch.cuda.set_device(local)
@@ -665,6 +687,7 @@ def run_dp(args):
         os.environ.setdefault("WORLD_SIZE", str(world))
         tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=device)
     import workloads as WL
+    from bit_adam_error_b200 import _lib as L
     from bit_adam_error_b200.distributed import CudaStages, DistributedOneBitAdam, plan
     wl = select_workload(args).with_(W=world, freeze_step=0)
     layout = plan(wl.sizes, world, 4 if args.rule == "momentum" else 32, 2 if args.rule == "twobit" else 1)
@@ -688,36 +711,76 @@ def run_dp(args):
             src = torch.from_numpy(row.view(np.int16)).view(torch.bfloat16) if bf else torch.from_numpy(row)
             G[b][lo:hi].copy_(src)
     drv = DistributedOneBitAdam(layout, stages, freeze_step=0)
+    ctxs = [h for h in {stages.local, stages.server, stages.update, *(stages.slice_ctx or []),
+                        *(stages.slice_upd or [])} if h]
     stream = torch.cuda.current_stream(device)
     for i in range(args.warmup):
         drv.step(G[i % nbuf])
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    launches0 = sum(L.ob_launch_count(h) for h in ctxs)
+    sampler = ClockSampler(gpu_id(device))
+    sampler.start()
+    time.sleep(0.3)
     barrier(tdist)
     torch.cuda.synchronize()
+    w0 = time.time()
     e0.record(stream)
     for i in range(args.steps):
         drv.step(G[i % nbuf])
     e1.record(stream)
     torch.cuda.synchronize()
+    w1 = time.time()
     barrier(tdist)
+    clocks = sampler.stop(w0, w1)
+    launches = sum(L.ob_launch_count(h) for h in ctxs) - launches0
     ms = max_over_ranks(tdist, e0.elapsed_time(e1) / args.steps, device)
+
+    # End to end: this rank's gradient from pinned host memory every step (one
+    # host-to-device copy), the step, and a device-to-host read of the scales.
+    e2e = None
+    if not args.no_e2e:
+        host = [torch.empty(layout.n, dtype=gdt, pin_memory=True) for _ in range(min(2, nbuf))]
+        for b, hb in enumerate(host):
+            hb.copy_(G[b])
+        dev_in = torch.empty(layout.n, dtype=gdt, device=device)
+        result = stages.s_srv if stages.s_srv.numel() else stages.p[: max(1, layout.C)]
+        out_h = torch.empty(result.shape, dtype=torch.float32, pin_memory=True)
+        for i in range(2):
+            dev_in.copy_(host[i % len(host)], non_blocking=True)
+            drv.step(dev_in)
+        torch.cuda.synchronize()
+        barrier(tdist)
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for i in range(args.steps):
+            dev_in.copy_(host[i % len(host)], non_blocking=True)
+            drv.step(dev_in)
+            out_h.copy_(result, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier(tdist)
+        ms_e2e = max_over_ranks(tdist, e0.elapsed_time(e1) / args.steps, device)
+        e2e = {"value": world * layout.n / (ms_e2e / 1e3) / 1e9, "unit": UNIT, "ms_per_step": ms_e2e,
+               "h2d_bytes_per_step": layout.n * wl.grad_bytes, "d2h_bytes_per_step": 4 * out_h.numel()}
     flags = drv.status()
     if rank == 0:
         own = [layout.eslice(r).stop - layout.eslice(r).start for r in range(world)]
         scales_per_chunk = {"scaled": 1, "momentum": 0, "twobit": 2}[args.rule]
-        # One job, one model of n parameters per step (the W = world workers are the
-        # ranks), so the rate is n / step time, as for W virtual workers on one GPU.
-        line = {"metric": METRIC, "value": layout.n / (ms / 1e3) / 1e9, "unit": UNIT,
+        line = {"metric": METRIC, "value": world * layout.n / (ms / 1e3) / 1e9, "unit": UNIT,
                 "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
                 "data": "synthetic (seeded Philox streams; shapes and distributions of the workload)",
                 "config": dict(workload_config(wl, world, args.rule),
-                               parallelism=f"dp{world}: worker w = rank w, chunk-owner server stage, "
-                                           f"NCCL point-to-point exchanges ({'pipelined' if stages.pipelined else 'grouped'})",
-                               owned_elements=own),
+                               parallelism=f"dp{world}: worker w = rank w (whole model and one gradient per "
+                                           f"rank), chunk-owner server stage, NCCL point-to-point exchanges "
+                                           f"({'pipelined' if stages.pipelined else 'grouped'})",
+                               owned_elements=own, units="gradient elements of all ranks per second"),
+                "model_value": layout.n / (ms / 1e3) / 1e9,
                 "exchange_bytes_per_step_per_rank": 2 * 4 * (int(layout.words[-1]) + scales_per_chunk * layout.C),
-                "status_flags": flags, "e2e": None}
+                "roofline": None,
+                "roofline_note": "per-kernel rooflines are reported by the single-GPU line (N = 1)",
+                "gpu_launches": launches, "status_flags": flags, "e2e": e2e, "clocks": clocks}
         print(json.dumps(line), flush=True)
     stages.close()
     tdist.destroy_process_group()
@@ -736,7 +799,8 @@ def main():
     args = parse_args()
     if args.impl == "reference":
         return run_reference(args)
-    if args.dp:
+    world = dist_env()[0]
+    if args.dp or (world > 1 and not args.replicas):
         return run_dp(args)
     return run_ours(args)
 
