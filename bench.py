@@ -557,6 +557,21 @@ def run_ours(args):
     step_bpe = sum(algo_bytes_per_elem(k, wl) * v[1] for k, v in prof.items()) / args.steps
     step_gbs = step_bpe * n / (ms_max / 1e3) / 1e9
 
+    # -- small workloads: the same steps back to back, inputs left in L2 -------------
+    l2_resident = None
+    if flush:
+        for i in range(3):
+            step_fn(dev_g[i % nbuf])
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for i in range(args.steps):
+            step_fn(dev_g[i % nbuf])
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ms_res = max_over_ranks(dist, e0.elapsed_time(e1) / args.steps, device)
+        l2_resident = {"ms_per_step": ms_res, "value": world * n / (ms_res / 1e3) / 1e9, "unit": UNIT,
+                       "note": "no L2 flush between steps: the step's inputs stay in the 126 MB L2"}
+
     # -- error-buffer monitoring (one call, timed alone) -----------------------------
     monitor = None
     if args.phase == "compressed":
@@ -622,6 +637,7 @@ def run_ours(args):
                         "algorithmic_bytes_per_elem": step_bpe, "peak": peak,
                         "peak_source": peak_src},
                 "roofline": roofline, "kernels": kernels, "error_norms_call": monitor,
+                "l2_resident": l2_resident,
                 "cpu_baseline": cpu, "e2e": e2e,
                 "gpu_launches": launches, "status_flags": status, "clocks": clocks}
         print(json.dumps(line), flush=True)

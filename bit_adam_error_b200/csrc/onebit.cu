@@ -201,8 +201,9 @@ struct DeviceGuard {
 
 // Launch with programmatic stream serialisation: the kernel may be scheduled
 // while the stream's previous kernel finishes, and waits for it (every kernel
-// starts with pdl_enter) before touching memory.  Launch errors surface through
-// cudaGetLastError like those of <<<>>> launches.
+// starts with pdl_enter) before touching memory.  Should a stream refuse the
+// attribute, the same kernel is launched plainly (same results, no overlap).
+// Launch errors surface through cudaGetLastError like those of <<<>>> launches.
 template <typename... P, typename... A>
 void pdl(void (*kernel)(P...), dim3 grid, unsigned block, cudaStream_t st, A&&... args) {
   cudaLaunchConfig_t cfg = {};
@@ -215,6 +216,9 @@ void pdl(void (*kernel)(P...), dim3 grid, unsigned block, cudaStream_t st, A&&..
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kernel, args...) == cudaSuccess) return;
+  cudaGetLastError();
+  cfg.numAttrs = 0;
   cudaLaunchKernelEx(&cfg, kernel, std::forward<A>(args)...);
 }
 

@@ -49,8 +49,8 @@ def _run_two_calls(sizes, W, gdt, clip):
     stream = int(torch.cuda.current_stream().cuda_stream)
     for t in range(2):
         g = grads_for(wl, t)
-        if clip:
-            g[:, ::53] = np.float32(-8.0)
+        if clip:                        # values the clip must cut (-8.0; 0xC100 as bfloat16 bits)
+            g[:, ::53] = np.float32(-8.0) if g.dtype == np.float32 else np.uint16(0xC100)
         G = to_dev(g)
         ref.compress(G)
         L.ob_compress_noalloc(cfg, G.data_ptr(), err.data_ptr(), bits.data_ptr(), s.data_ptr(), stream)
