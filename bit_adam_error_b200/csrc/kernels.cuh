@@ -313,16 +313,18 @@ __device__ __forceinline__ void fused_finalize(const Layout& L, const Fin& f) {
   __syncthreads();
   if (!s_last) return;
   __threadfence();
+  // rows * T <= 2^15 on this path: 32-bit slot indices.
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   for (int task = warp; task < f.rows * L.C; task += kWarpsPerBlock) {
     const int r = task / L.C, k = task - r * L.C;
-    const double* pr = f.part + static_cast<int64_t>(r) * f.row_stride;
+    const double* pr = f.part + r * static_cast<int>(f.row_stride);
+    const int t1 = static_cast<int>(L.tp[k + 1]);
     double acc = 0.0;
-    for (int64_t t = L.tp[k] + lane; t < L.tp[k + 1]; t += kWarp) acc += __ldcg(pr + t);
+    for (int t = static_cast<int>(L.tp[k]) + lane; t < t1; t += kWarp) acc += __ldcg(pr + t);
     acc = warp_sum(acc);
     if (lane == 0) {
       const int64_t nk = L.off[k + 1] - L.off[k];
-      f.out[static_cast<int64_t>(r) * L.C + k] =
+      f.out[r * L.C + k] =
           nk > 0 ? __double2float_rn(__ddiv_rn(__dsqrt_rn(acc), __dsqrt_rn(static_cast<double>(nk)))) : 0.0f;
     }
   }
