@@ -313,14 +313,32 @@ __device__ __forceinline__ void fused_finalize(const Layout& L, const Fin& f) {
   __syncthreads();
   if (!s_last) return;
   __threadfence();
-  // rows * T <= 2^15 on this path: 32-bit slot indices.
+  // rows * T <= 2^15 on this path: 32-bit slot indices.  Lane l keeps kFinLanes
+  // running sums (slot t0 + 32 i + l goes to sum i % kFinLanes), so kFinLanes
+  // loads are in flight per lane instead of one; the sums are then added in
+  // index order and across lanes by the butterfly -- a fixed order.
+  constexpr int kFinLanes = 8;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   for (int task = warp; task < f.rows * L.C; task += kWarpsPerBlock) {
     const int r = task / L.C, k = task - r * L.C;
     const double* pr = f.part + r * static_cast<int>(f.row_stride);
-    const int t1 = static_cast<int>(L.tp[k + 1]);
+    const int t0 = static_cast<int>(L.tp[k]), t1 = static_cast<int>(L.tp[k + 1]);
+    double part[kFinLanes];
+#pragma unroll
+    for (int u = 0; u < kFinLanes; ++u) part[u] = 0.0;
+    for (int t = t0 + lane; t < t1; t += kWarp * kFinLanes) {
+      double x[kFinLanes];
+#pragma unroll
+      for (int u = 0; u < kFinLanes; ++u) {
+        const int tu = t + u * kWarp;
+        x[u] = tu < t1 ? __ldcg(pr + tu) : 0.0;
+      }
+#pragma unroll
+      for (int u = 0; u < kFinLanes; ++u) part[u] += x[u];
+    }
     double acc = 0.0;
-    for (int t = static_cast<int>(L.tp[k]) + lane; t < t1; t += kWarp) acc += __ldcg(pr + t);
+#pragma unroll
+    for (int u = 0; u < kFinLanes; ++u) acc += part[u];
     acc = warp_sum(acc);
     if (lane == 0) {
       const int64_t nk = L.off[k + 1] - L.off[k];

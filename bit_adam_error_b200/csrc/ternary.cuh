@@ -61,6 +61,7 @@ __global__ void __launch_bounds__(kBlock)
 k_ternary_step(Layout L, int W, const GT* __restrict__ grads, ET* __restrict__ err,
                float* __restrict__ m, const float* __restrict__ v, float* __restrict__ p, Hyper h,
                double* __restrict__ partP, double* __restrict__ partU, uint32_t* __restrict__ status) {
+  pdl_enter();
   const int lane = threadIdx.x & 31;
   const auto mean = make_mean<POW2>(W);
   int hint = 0;
@@ -130,6 +131,7 @@ template <typename GT, typename ET, bool CLIP>
 __global__ void __launch_bounds__(kBlock)
 k_ternary_compress(Layout L, int W, const GT* __restrict__ grads, ET* __restrict__ err,
                    uint32_t* __restrict__ codes, Hyper h, uint32_t* __restrict__ status) {
+  pdl_enter();
   const int lane = threadIdx.x & 31;
   const int64_t items = static_cast<int64_t>(W) * L.T;
   int hint = 0;
@@ -184,6 +186,7 @@ k_ternary_compress(Layout L, int W, const GT* __restrict__ grads, ET* __restrict
 __global__ void __launch_bounds__(kBlock)
 k_ternary_server(int W, int64_t words, const uint32_t* __restrict__ codes_w,
                  uint32_t* __restrict__ codes_srv) {
+  pdl_enter();
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
   for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < words; i += stride) {
     uint32_t acc = 0u;
@@ -198,6 +201,7 @@ __global__ void __launch_bounds__(kBlock)
 k_ternary_update(Layout L, int W, const uint32_t* __restrict__ codes_srv, float* __restrict__ m,
                  const float* __restrict__ v, float* __restrict__ p, Hyper h,
                  double* __restrict__ partP, double* __restrict__ partU, uint32_t* __restrict__ status) {
+  pdl_enter();
   const int lane = threadIdx.x & 31;
   const auto mean = make_mean<POW2>(W);
   int hint = 0;

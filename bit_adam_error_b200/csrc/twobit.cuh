@@ -27,18 +27,25 @@ namespace ob {
 
 __device__ __forceinline__ int64_t plane_words(int64_t nk) { return (nk + 31) / 32; }
 
+// The four dequantised values (+-s1) + (+-s2) of one worker's chunk, d<b1><b2>,
+// formed once per tile: the same float additions the per-element form makes.
+struct Dq4 {
+  float d00, d10, d01, d11;
+};
+
+__device__ __forceinline__ Dq4 dq4_of(const float* __restrict__ s_w, int k) {
+  const float s1 = __ldg(s_w + static_cast<int64_t>(k) * 2), s2 = __ldg(s_w + static_cast<int64_t>(k) * 2 + 1);
+  return Dq4{-s1 + -s2, s1 + -s2, -s1 + s2, s1 + s2};
+}
+
 // acc[j] += s1 sign1 + s2 sign2 of worker w, ascending w (the order of pass 2).
-// W1: exactly one worker.  Its four possible dequantised values
-// (+-s1) + (+-s2) are formed once per group -- the same float additions the
-// per-element form makes -- and each element selects one of them.
+// W1: exactly one worker; each element selects one of the tile's four values dq.
 template <bool W1>
 __device__ __forceinline__ void tb_server_sum8(const Layout& L, int W, const uint32_t* __restrict__ bits_w,
                                                const float* __restrict__ s_w, const Tile& tl, int64_t wrel,
-                                               int64_t nwk, bool word_in, int lane, float (&acc)[8]) {
+                                               int64_t nwk, bool word_in, int lane, float (&acc)[8],
+                                               const Dq4& dq) {
   if constexpr (W1) {
-    const float* sc = s_w + static_cast<int64_t>(tl.k) * 2;
-    const float s1 = __ldg(sc), s2 = __ldg(sc + 1);
-    const float d00 = -s1 + -s2, d10 = s1 + -s2, d01 = -s1 + s2, d11 = s1 + s2;  // d<b1><b2>
     const uint32_t* row = bits_w + tl.w0;
     const uint32_t w1 = word_in ? __ldg(row + wrel) : 0u;
     const uint32_t w2 = word_in ? __ldg(row + nwk + wrel) : 0u;
@@ -46,7 +53,7 @@ __device__ __forceinline__ void tb_server_sum8(const Layout& L, int W, const uin
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
       const bool x1 = (b1 >> j) & 1u, x2 = (b2 >> j) & 1u;
-      acc[j] = 0.0f + (x2 ? (x1 ? d11 : d01) : (x1 ? d10 : d00));
+      acc[j] = 0.0f + (x2 ? (x1 ? dq.d11 : dq.d01) : (x1 ? dq.d10 : dq.d00));
     }
     return;
   }
@@ -256,6 +263,7 @@ k_tb_server_norm(Layout L, int W, const uint32_t* __restrict__ bits_w, const flo
     const Tile tl = tile_at(L, t, hint);
     const int64_t nwk = plane_words(tl.nk);
     const float s1 = RESID ? __ldg(s_srv + 2 * tl.k) : 0.0f;
+    const Dq4 dq = W1 ? dq4_of(s_w, tl.k) : Dq4{};
     double tsum = 0.0;
     auto add = [&](float cs) {
       const float x = RESID ? cs - signed_scale(cs >= 0.0f, s1) : cs;
@@ -269,7 +277,7 @@ k_tb_server_norm(Layout L, int W, const uint32_t* __restrict__ bits_w, const flo
         const bool in = i0 < tl.nk;
         float sv[8], acc[8];
         if (in) ld8_ro(srv_err + tl.ck0 + i0, sv); else zero8(sv);
-        tb_server_sum8<W1>(L, W, bits_w, s_w, tl, wrel, nwk, wrel * 32 < tl.nk, lane, acc);
+        tb_server_sum8<W1>(L, W, bits_w, s_w, tl, wrel, nwk, wrel * 32 < tl.nk, lane, acc, dq);
         if (in) {
 #pragma unroll
           for (int j = 0; j < 8; ++j) add(mean(acc[j]) + sv[j]);
@@ -350,6 +358,7 @@ k_tb_server_update(Layout L, int W, const uint32_t* __restrict__ bits_w, const f
     const Tile tl = tile_at(L, t, hint);
     const int64_t nwk = plane_words(tl.nk);
     const float s1 = __ldg(s_srv + 2 * tl.k), s2 = __ldg(s_srv + 2 * tl.k + 1);
+    const Dq4 dq = (FROM_WORKERS && !CACHED && W1) ? dq4_of(s_w, tl.k) : Dq4{};
     uint32_t* srow = bits_srv + tl.w0;
     double Psum = 0.0, Usum = 0.0;
     bool bad = false;
@@ -369,7 +378,7 @@ k_tb_server_update(Layout L, int W, const uint32_t* __restrict__ bits_w, const f
         }
         if (FROM_WORKERS) {
           float acc[8];
-          if (!CACHED) tb_server_sum8<W1>(L, W, bits_w, s_w, tl, wrel, nwk, word_in, lane, acc);
+          if (!CACHED) tb_server_sum8<W1>(L, W, bits_w, s_w, tl, wrel, nwk, word_in, lane, acc, dq);
           uint32_t byte1 = 0, byte2 = 0;
           if (in) {
 #pragma unroll
