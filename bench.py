@@ -597,6 +597,17 @@ def run_ours(args):
         monitor = {"ms": mon_ms, "GBps": mon_bytes / (mon_ms / 1e3) / 1e9,
                    "frac": mon_bytes / (mon_ms / 1e3) / 1e9 / peak, "bytes": mon_bytes}
 
+    # -- quantisation-rate monitoring (one call, timed alone; sign-bit rules) ----------
+    rates = None
+    if args.phase == "compressed" and args.rule != "momentum":
+        e0.record(stream)
+        opt.quant_rates()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        r_ms = e0.elapsed_time(e1)
+        r_bytes = 4 * opt.words * (W + 1)          # every worker's packed words and the server's
+        rates = {"ms": r_ms, "GBps": r_bytes / (r_ms / 1e3) / 1e9, "bytes": r_bytes}
+
     # -- end to end: host gradients through the public call ---------------------------
     e2e = None
     host_bytes = W * n * wl.grad_bytes
@@ -652,7 +663,7 @@ def run_ours(args):
                 "roofline": roofline, "kernels": kernels,
                 "kernel_timing": ("a second pass of the same steps with per-kernel CUDA events"
                                   if flush else "per-kernel CUDA events in the timed steps"),
-                "error_norms_call": monitor,
+                "error_norms_call": monitor, "quant_rates_call": rates,
                 "l2_resident": l2_resident,
                 "cpu_baseline": cpu, "e2e": e2e,
                 "gpu_launches": launches, "status_flags": status, "clocks": clocks}
