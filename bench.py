@@ -588,6 +588,8 @@ def run_ours(args):
     # -- error-buffer monitoring (one call, timed alone) -----------------------------
     monitor = None
     if args.phase == "compressed":
+        opt.error_norms()                  # first call: host-side set-up outside the timing
+        torch.cuda.synchronize()
         e0.record(stream)
         opt.error_norms()
         e1.record(stream)
@@ -600,6 +602,8 @@ def run_ours(args):
     # -- quantisation-rate monitoring (one call, timed alone; sign-bit rules) ----------
     rates = None
     if args.phase == "compressed" and args.rule != "momentum":
+        opt.quant_rates()
+        torch.cuda.synchronize()
         e0.record(stream)
         opt.quant_rates()
         e1.record(stream)

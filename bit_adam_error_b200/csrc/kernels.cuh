@@ -313,38 +313,59 @@ __device__ __forceinline__ void fused_finalize(const Layout& L, const Fin& f) {
   __syncthreads();
   if (!s_last) return;
   __threadfence();
-  // rows * T <= 2^15 on this path: 32-bit slot indices.  Lane l keeps kFinLanes
-  // running sums (slot t0 + 32 i + l goes to sum i % kFinLanes), so kFinLanes
-  // loads are in flight per lane instead of one; the sums are then added in
-  // index order and across lanes by the butterfly -- a fixed order.
+  // rows * T <= 2^15 on this path: 32-bit slot indices.  With few (row, chunk)
+  // pairs, wpt warps share one: warp `share` sums the share-th contiguous part
+  // of its slots, each lane keeping kFinLanes running sums (slot a + 32 i + l
+  // goes to sum i % kFinLanes) so that kFinLanes loads are in flight; the sums
+  // are added in index order, across lanes by the butterfly, and across the
+  // shares in warp order -- a fixed order for a given problem.
   constexpr int kFinLanes = 8;
+  __shared__ double s_share[kWarpsPerBlock];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  for (int task = warp; task < f.rows * L.C; task += kWarpsPerBlock) {
-    const int r = task / L.C, k = task - r * L.C;
-    const double* pr = f.part + r * static_cast<int>(f.row_stride);
-    const int t0 = static_cast<int>(L.tp[k]), t1 = static_cast<int>(L.tp[k + 1]);
-    double part[kFinLanes];
+  const int tasks = f.rows * L.C;
+  const int wpt = tasks >= kWarpsPerBlock ? 1 : tasks >= kWarpsPerBlock / 2 ? 2 : tasks >= 2 ? 4 : 8;
+  const int per_round = kWarpsPerBlock / wpt;
+  const int rounds = (tasks + per_round - 1) / per_round;
+  for (int rd = 0; rd < rounds; ++rd) {
+    const int task = rd * per_round + warp / wpt, share = warp % wpt;
+    double acc = 0.0;
+    if (task < tasks) {
+      const int r = task / L.C, k = task - r * L.C;
+      const double* pr = f.part + r * static_cast<int>(f.row_stride);
+      const int t0 = static_cast<int>(L.tp[k]), t1 = static_cast<int>(L.tp[k + 1]);
+      const int len = (t1 - t0 + wpt - 1) / wpt;
+      const int a = t0 + share * len, b = min(t1, a + len);
+      double part[kFinLanes];
 #pragma unroll
-    for (int u = 0; u < kFinLanes; ++u) part[u] = 0.0;
-    for (int t = t0 + lane; t < t1; t += kWarp * kFinLanes) {
-      double x[kFinLanes];
+      for (int u = 0; u < kFinLanes; ++u) part[u] = 0.0;
+      for (int t = a + lane; t < b; t += kWarp * kFinLanes) {
+        double x[kFinLanes];
 #pragma unroll
-      for (int u = 0; u < kFinLanes; ++u) {
-        const int tu = t + u * kWarp;
-        x[u] = tu < t1 ? __ldcg(pr + tu) : 0.0;
+        for (int u = 0; u < kFinLanes; ++u) {
+          const int tu = t + u * kWarp;
+          x[u] = tu < b ? __ldcg(pr + tu) : 0.0;
+        }
+#pragma unroll
+        for (int u = 0; u < kFinLanes; ++u) part[u] += x[u];
       }
 #pragma unroll
-      for (int u = 0; u < kFinLanes; ++u) part[u] += x[u];
+      for (int u = 0; u < kFinLanes; ++u) acc += part[u];
+      acc = warp_sum(acc);
     }
-    double acc = 0.0;
-#pragma unroll
-    for (int u = 0; u < kFinLanes; ++u) acc += part[u];
-    acc = warp_sum(acc);
-    if (lane == 0) {
-      const int64_t nk = L.off[k + 1] - L.off[k];
-      f.out[r * L.C + k] =
-          nk > 0 ? __double2float_rn(__ddiv_rn(__dsqrt_rn(acc), __dsqrt_rn(static_cast<double>(nk)))) : 0.0f;
+    if (lane == 0) s_share[warp] = acc;
+    __syncthreads();
+    if (threadIdx.x < per_round) {
+      const int tk = rd * per_round + threadIdx.x;
+      if (tk < tasks) {
+        double S = 0.0;
+        for (int i = 0; i < wpt; ++i) S += s_share[threadIdx.x * wpt + i];
+        const int r = tk / L.C, k = tk - r * L.C;
+        const int64_t nk = L.off[k + 1] - L.off[k];
+        f.out[r * L.C + k] =
+            nk > 0 ? __double2float_rn(__ddiv_rn(__dsqrt_rn(S), __dsqrt_rn(static_cast<double>(nk)))) : 0.0f;
+      }
     }
+    __syncthreads();
   }
   __syncthreads();
   if (threadIdx.x == 0) *f.ticket = 0u;
@@ -896,24 +917,25 @@ k_rows_sumsq(Layout L, int R, const ET* __restrict__ x, double* __restrict__ par
 __global__ void __launch_bounds__(kBlock)
 k_sign_count(Layout L, int R, const uint32_t* __restrict__ bits, int plane, double* __restrict__ part) {
   pdl_enter();
-  const int lane = threadIdx.x & 31;
+  // One thread per (row, tile): a warp reads 32 consecutive tiles' words, 2 KB.
   const int64_t items = static_cast<int64_t>(R) * L.T;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
   int hint = 0;
-  for (int64_t it = warp_id(); it < items; it += warp_count()) {
+  for (int64_t it = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; it < items; it += stride) {
     const int r = static_cast<int>(it / L.T);
     const int64_t t = it - static_cast<int64_t>(r) * L.T;
     const Tile tl = tile_at(L, t, hint);
-    const int64_t nwk = (tl.nk + 31) / 32;
-    const int64_t wi = tl.rel / 32 + lane;        // lanes 0..15 hold the tile's words
+    const int64_t nwk = (tl.nk + 31) / 32, wi0 = tl.rel / 32;
+    const int nw = static_cast<int>(min(static_cast<int64_t>(kTileWords), nwk - wi0));
+    const uint32_t* q = bits + static_cast<int64_t>(r) * L.words + tl.w0 + plane * nwk + wi0;
     unsigned cnt = 0;
-    if (lane < kTileWords && wi < nwk) {
-      uint32_t word = __ldg(bits + static_cast<int64_t>(r) * L.words + tl.w0 + plane * nwk + wi);
-      const int64_t left = tl.nk - wi * 32;       // real bits in this word
+    for (int j = 0; j < nw; ++j) {
+      uint32_t word = __ldg(q + j);
+      const int64_t left = tl.nk - (wi0 + j) * 32;   // real bits in this word
       if (left < 32) word &= (1u << left) - 1u;
-      cnt = __popc(word);
+      cnt += __popc(word);
     }
-    cnt = __reduce_add_sync(kFull, cnt);
-    if (lane == 0) part[it] = static_cast<double>(cnt);
+    part[it] = static_cast<double>(cnt);
   }
 }
 

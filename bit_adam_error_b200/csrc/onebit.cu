@@ -1216,7 +1216,7 @@ ob_err ob_quant_rates(ob_ctx* c, float* worker_rates, float* server_rates, void*
     for (int pl = 0; pl < int(planes); ++pl) {
       if (c->T > 0) {
         auto k = ob::k_sign_count;
-        const int g = grid_for(c, k, rows * c->T);
+        const int g = grid_for(c, k, (rows * c->T + ob::kWarp - 1) / ob::kWarp);   // a thread per tile
         launch(c, OB_K_SIGN_COUNT, st, [&] { pdl(k, g, ob::kBlock, st, c->L, rows, bits, pl, part); });
       }
       launch(c, OB_K_FINALIZE_SCALE, st, [&] {
