@@ -239,6 +239,17 @@ __device__ __forceinline__ Mean<POW2> make_mean(int W) {
   return m;
 }
 
+// The mean of kernels specialised for one worker (W1): the multiply by 1, known
+// at compile time, so it costs nothing (x * 1 is x exactly).
+template <bool POW2, bool W1>
+__device__ __forceinline__ Mean<POW2> make_mean_w(int W) {
+  if constexpr (W1) {
+    static_assert(POW2, "one worker is a power of two");
+    return Mean<POW2>{1.0f, 1.0f};
+  }
+  return make_mean<POW2>(W);
+}
+
 // A sum of squares of finite floats cannot overflow a double, so a non-finite
 // tile sum means a non-finite value in the tile: one check per tile replaces a
 // check per element.
@@ -772,7 +783,7 @@ k_server_update(Layout L, int W, const uint32_t* __restrict__ bits_w, const floa
                 double* __restrict__ partU, uint32_t* __restrict__ status) {
   pdl_enter();
   const int lane = threadIdx.x & 31;
-  const auto mean = make_mean<POW2>(W);
+  const auto mean = make_mean_w<POW2, W1>(W);
   int hint = 0;
   for (int64_t t = warp_id(); t < L.T; t += warp_count()) {
     const Tile tl = tile_at(L, t, hint);

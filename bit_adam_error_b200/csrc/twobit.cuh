@@ -257,7 +257,7 @@ k_tb_server_norm(Layout L, int W, const uint32_t* __restrict__ bits_w, const flo
                  double* __restrict__ part, uint32_t* __restrict__ status) {
   pdl_enter();
   const int lane = threadIdx.x & 31;
-  const auto mean = make_mean<POW2>(W);
+  const auto mean = make_mean_w<POW2, W1>(W);
   int hint = 0;
   for (int64_t t = warp_id(); t < L.T; t += warp_count()) {
     const Tile tl = tile_at(L, t, hint);
@@ -352,7 +352,7 @@ k_tb_server_update(Layout L, int W, const uint32_t* __restrict__ bits_w, const f
                    double* __restrict__ partU, uint32_t* __restrict__ status) {
   pdl_enter();
   const int lane = threadIdx.x & 31;
-  const auto mean = make_mean<POW2>(W);
+  const auto mean = make_mean_w<POW2, W1>(W);
   int hint = 0;
   for (int64_t t = warp_id(); t < L.T; t += warp_count()) {
     const Tile tl = tile_at(L, t, hint);

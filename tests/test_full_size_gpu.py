@@ -170,6 +170,56 @@ def test_gpt2xl_flat_hundred_chained_steps():
     assert_state("step 100: err", gpu["err"], last["err"], off)
 
 
+def test_gpt2xl_flat_local_step_and_quant_rates():
+    """0/1 Adam's local step and the quantisation rates at full size: on the
+    1.5e9-element workload, a synchronised step, a local step and another
+    synchronised step; chunk 0 and the tail chunk are compared with the oracle
+    (state within the parity bar, sign words bit-exact), and the per-chunk
+    quantisation rates of every chunk equal the oracle's count of the GPU's
+    own sign words (and, on the sampled chunks, of the oracle's)."""
+    wl = WL.get_workload("gpt2xl-flat")
+    ks = (0, wl.C - 1)
+    torch.cuda.empty_cache()
+    opt = OneBitAdam(wl.offsets, 1, grad_dtype="bf16", device=dev(), **HP)
+    upload_state(wl, opt.p, opt.v)
+    G = torch.empty((1, wl.n), dtype=torch.bfloat16, device=dev())
+    for t, kind in enumerate("SLS"):
+        upload_grads(wl, t, G)
+        (opt.local_step if kind == "L" else opt.step)(G)
+    wr, sr = opt.quant_rates()
+    torch.cuda.synchronize()
+    assert opt.status() == 0
+    del G
+    o = oracle.get_mt()
+    bits_w, bits_srv = np_of(opt.bits_w), np_of(opt.bits_srv)
+    assert np.array_equal(np_of(wr), o.sign_rates(wl.offsets, bits_w)[:, :, 0])
+    assert np.array_equal(np_of(sr), o.sign_rates(wl.offsets, bits_srv)[0, :, 0])
+    wb = np.zeros(wl.C + 1, np.int64)
+    np.cumsum([(s + 31) // 32 for s in wl.sizes], out=wb[1:])
+    for k in ks:
+        nk = wl.sizes[k]
+        lo, hi = int(wl.offsets[k]), int(wl.offsets[k + 1])
+        off = np.array([0, nk], np.int64)
+        pk, vk = WL.chunk_state(wl, k)
+        ref = {"p": pk, "m": np.zeros(nk, np.float32), "v": vk,
+               "err": np.zeros((1, nk), np.float32), "srv_err": np.zeros(nk, np.float32)}
+        for t, kind in enumerate("SLS"):
+            g = WL.chunk_grads(wl, t, 0, k)[None, :]
+            if kind == "L":
+                assert o.local_step(off, g, ref, F["lr"], F["eps"]) == 0
+            else:
+                assert o.step(off, g, ref, F["beta1"], F["lr"], F["eps"], threads=THREADS) == 0
+        tag = f"chunk {k}: "
+        for key in ("p", "m", "v", "srv_err"):
+            assert_state(tag + key, np_of(getattr(opt, key)[lo:hi]), ref[key], off)
+        assert_state(tag + "err", np_of(opt.err[:, lo:hi]), ref["err"], off)
+        assert_bits(tag + "bits_w", bits_w[:, wb[k]:wb[k + 1]], ref["bits_w"])
+        assert_bits(tag + "bits_srv", bits_srv[wb[k]:wb[k + 1]], ref["bits_srv"])
+        assert np_of(wr)[0, k] == o.sign_rates(off, ref["bits_w"])[0, 0, 0]
+        assert np_of(sr)[k] == o.sign_rates(off, ref["bits_srv"])[0, 0, 0]
+    opt.close()
+
+
 def test_row_longer_than_two_to_the_31():
     """Maximum-size indexing: one worker row of 2^31 + 2^20 elements (bf16
     gradients; about 48 GB resident), so element, word and tile indices pass
