@@ -268,6 +268,25 @@ class ClockSampler:
 
 # -- distributed plumbing ------------------------------------------------------------------
 
+def dp_bytes_per_elem(kind: str, role: str, wl, world: int, rule: str) -> float:
+    """HBM bytes per element of a data-parallel stage kernel (scaled-sign rule):
+    role "worker" (a one-worker ctx: the worker stage, or the update alone),
+    "server" (the owner's W-worker server stage).  0 when not modelled."""
+    if rule != "scaled":
+        return 0.0
+    gb, eb = wl.grad_bytes, wl.err_bytes
+    upd = 16.0 if wl.optimizer == "lamb" else 20.0
+    if role == "worker":
+        return {"k_worker_norm": gb + eb,                      # g, err
+                "k_worker_pack": gb + 2 * eb + 1 / 8,          # g, err r/w, signs
+                "k_server_update": 1 / 8 + upd,                # server signs, m r/w, v, p (+ p w)
+                "k_lamb_param": 16.0}.get(kind, 0.0)
+    if role == "server":
+        return {"k_server_norm": world / 8 + eb,               # W workers' signs, srv_err
+                "k_server_update": world / 8 + 2 * eb + 1 / 8}.get(kind, 0.0)  # signs, srv_err r/w, server signs
+    return 0.0
+
+
 def dist_env():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -760,12 +779,28 @@ def run_dp(args):
     drv = DistributedOneBitAdam(layout, stages, freeze_step=0)
     ctxs = [h for h in {stages.local, stages.server, stages.update, *(stages.slice_ctx or []),
                         *(stages.slice_upd or [])} if h]
+    # Elements and role of every ctx, for the byte model of its kernels.
+    ctx_info = {stages.local: (layout.n, "worker")}
+    if stages.server:
+        ctx_info[stages.server] = (stages.n_own, "server")
+    if stages.update:
+        ctx_info[stages.update] = (layout.n, "worker")
+    for o, h in enumerate(stages.slice_ctx or []):
+        if h:
+            es = layout.eslice(o)
+            ctx_info[h] = (es.stop - es.start, "worker")
+    for o, h in enumerate(stages.slice_upd or []):
+        if h and h not in ctx_info:
+            es = layout.eslice(o)
+            ctx_info[h] = (es.stop - es.start, "worker")
     stream = torch.cuda.current_stream(device)
     for i in range(args.warmup):
         drv.step(G[i % nbuf])
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     launches0 = sum(L.ob_launch_count(h) for h in ctxs)
+    for h in ctxs:
+        L.ob_profile_start(h, args.steps * 16)
     sampler = ClockSampler(gpu_id(device))
     sampler.start()
     time.sleep(0.3)
@@ -782,6 +817,29 @@ def run_dp(args):
     clocks = sampler.stop(w0, w1)
     launches = sum(L.ob_launch_count(h) for h in ctxs) - launches0
     ms = max_over_ranks(tdist, e0.elapsed_time(e1) / args.steps, device)
+    # Per kernel and ctx role: time (CUDA events on the launch stream) and bytes.
+    agg = {}
+    for h in ctxs:
+        n_ctx, role = ctx_info.get(h, (0, "worker"))
+        for kname, (kms, kl) in L.ob_profile_stop(h).items():
+            key = f"{kname} ({role})"
+            t, c, b = agg.get(key, (0.0, 0, 0.0))
+            agg[key] = (t + kms, c + kl, b + kl * n_ctx * dp_bytes_per_elem(kname, role, wl, world, args.rule))
+    peak, peak_src = measured_peak()
+    streamed = {k: v for k, v in agg.items() if v[2] > 0}
+    roofline, dp_kernels = None, None
+    if streamed:
+        total_ms = sum(v[0] for v in agg.values())
+        dom = max(streamed, key=lambda k: streamed[k][0])
+        t, c, b = streamed[dom]
+        achieved = b / (t / 1e3) / 1e9
+        roofline = {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": peak,
+                    "peak_source": f"{peak_src} (copy bandwidth)", "unit": "GB/s", "frac": achieved / peak,
+                    "traffic": None, "algorithmic_bytes_per_launch": b / c, "launch_ms": t / c,
+                    "share_of_kernel_time": t / total_ms, "rank": rank}
+        dp_kernels = {k: {"ms_per_launch": v[0] / v[1], "launches": v[1], "share": v[0] / total_ms,
+                          "algorithmic_GBps": (v[2] / (v[0] / 1e3) / 1e9) if v[2] else None}
+                      for k, v in agg.items()}
 
     # End to end: this rank's gradient from pinned host memory every step (one
     # host-to-device copy), the step, and a device-to-host read of the scales.
@@ -825,8 +883,7 @@ def run_dp(args):
                                owned_elements=own, units="gradient elements of all ranks per second"),
                 "model_value": layout.n / (ms / 1e3) / 1e9,
                 "exchange_bytes_per_step_per_rank": 2 * 4 * (int(layout.words[-1]) + scales_per_chunk * layout.C),
-                "roofline": None,
-                "roofline_note": "per-kernel rooflines are reported by the single-GPU line (N = 1)",
+                "roofline": roofline, "kernels": dp_kernels,
                 "gpu_launches": launches, "status_flags": flags, "e2e": e2e, "clocks": clocks}
         print(json.dumps(line), flush=True)
     stages.close()

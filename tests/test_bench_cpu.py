@@ -116,3 +116,18 @@ def test_cpu_baseline_both_legs():
     one, allc = rec["legs"]
     assert one["cores"] == 1 and allc["cores"] == rec["cores"]
     assert rec["value"] == allc["value"] and one["value"] > 0 and allc["value"] > 0
+
+
+def test_byte_model_of_the_data_parallel_stages():
+    """Per-element bytes of the data-parallel stage kernels: the worker stage and
+    the update on a one-worker ctx, the server stage on the owner's W-worker ctx."""
+    import bench
+    import workloads as WL
+    wl = WL.get_workload("gpt2xl-flat")              # bf16 gradients, f32 error buffers, Adam
+    assert bench.dp_bytes_per_elem("k_worker_norm", "worker", wl, 8, "scaled") == 2 + 4
+    assert bench.dp_bytes_per_elem("k_worker_pack", "worker", wl, 8, "scaled") == 2 + 8 + 1 / 8
+    assert bench.dp_bytes_per_elem("k_server_update", "worker", wl, 8, "scaled") == 1 / 8 + 20
+    assert bench.dp_bytes_per_elem("k_server_norm", "server", wl, 8, "scaled") == 1 + 4
+    assert bench.dp_bytes_per_elem("k_server_update", "server", wl, 8, "scaled") == 1 + 8 + 1 / 8
+    assert bench.dp_bytes_per_elem("k_finalize_scale", "worker", wl, 8, "scaled") == 0
+    assert bench.dp_bytes_per_elem("k_worker_norm", "worker", wl, 8, "momentum") == 0
