@@ -688,9 +688,9 @@ void orc_sign_rates(int32_t rows, int32_t C, const int64_t* off, int32_t planes,
  * Adam alternates full-precision variance refreshes with 1-bit synchronised
  * steps, and adds local updates that lower the synchronisation frequency: its
  * listing updates m only from a synchronised g_hat, applies
- * param = adam_update(param, m, v) on every step, and notes that local steps
- * may proceed before the next global synchronisation.  The page gives no
- * formula for a local step.  Reading:
+ * param = adam_update(param, m, v) on every step, and lets local steps run
+ * between one global synchronisation and the next.  The page gives no formula
+ * for a local step.  Reading:
  *   - a local step sends nothing;
  *   - the parameters take the update of the listing's last line with the
  *     current m and v, which stay as they are:
