@@ -120,16 +120,16 @@ def algo_bytes_per_elem(kind: str, wl) -> float:
     if kind == "k_ternary_update":       # one sum byte, m r/w, v, p r (+ p w for Adam)
         return 1 + (16 if wl.optimizer == "lamb" else 20)
     # 2-bit Adam: two sign planes per message
-    if kind == "k_tb_resid_norm":        # g, err again for the first plane's residual
+    if kind == "k_tb_worker_norm":       # g, err of every worker (both scales' sums)
         return (gb + eb) * W
     if kind == "k_tb_pack":              # g, err r/w, both planes; srv_err read
         return (gb + 2 * eb) * W + W / 4 + eb
-    if kind == "k_tb_server_norm":       # both planes of every worker, srv_err
+    if kind == "k_tb_server_norm":       # both planes of every worker, srv_err (stage call)
         return W / 4 + eb
     if kind == "k_tb_server_update":     # planes, srv_err r/w, server planes (+ m, v, p as Adam/LAMB)
         return W / 4 + 2 * eb + 1 / 4 + (16 if wl.optimizer == "lamb" else 20)
-    # W >= 4: pass 2 also stores c_srv (4 B); the server passes read it instead of
-    # the W workers' words and the server error
+    # W >= 4: pass 2 also stores c_srv (4 B); pass 3 reads it instead of the W
+    # workers' words and the server error
     upd = 16 if wl.optimizer == "lamb" else 20
     if kind == "k_worker_pack_cached":
         return algo_bytes_per_elem("k_worker_pack", wl) + 4
@@ -137,8 +137,6 @@ def algo_bytes_per_elem(kind: str, wl) -> float:
         return 4 + eb + 1 / 8 + upd
     if kind == "k_tb_pack_cached":
         return algo_bytes_per_elem("k_tb_pack", wl) + 4
-    if kind == "k_tb_server_norm_cached":
-        return 4.0
     if kind == "k_tb_server_update_cached":
         return 4 + eb + 1 / 4 + upd
     # 0/1 Adam's local step: g, err r/w per worker; m, v, p reads (+ p write for Adam)
@@ -165,8 +163,7 @@ def step_bytes_per_elem(wl, phase: str = "compressed", rule: str = "scaled") -> 
         return algo_bytes_per_elem("k_ternary_step", wl) + (16.0 if wl.optimizer == "lamb" else 0.0)
     cached = "_cached" if wl.W >= CACHE_MIN_W else ""
     if rule == "twobit":
-        kinds = ["k_worker_norm", "k_tb_resid_norm", "k_tb_pack" + cached, "k_tb_server_norm" + cached,
-                 "k_tb_server_update" + cached]
+        kinds = ["k_tb_worker_norm", "k_tb_pack" + cached, "k_tb_server_update" + cached]
         return sum(algo_bytes_per_elem(k, wl) for k in kinds) + (16.0 if wl.optimizer == "lamb" else 0.0)
     kinds = ["k_worker_norm", "k_worker_pack" + cached, "k_server_update" + cached]
     if wl.optimizer == "lamb":
@@ -269,11 +266,29 @@ class ClockSampler:
 # -- distributed plumbing ------------------------------------------------------------------
 
 def dp_bytes_per_elem(kind: str, role: str, wl, world: int, rule: str) -> float:
-    """HBM bytes per element of a data-parallel stage kernel (scaled-sign rule):
-    role "worker" (a one-worker ctx: the worker stage, or the update alone),
-    "server" (the owner's W-worker server stage).  0 when not modelled."""
-    if rule != "scaled":
-        return 0.0
+    """HBM bytes per element of a data-parallel stage kernel (scaled-sign and
+    2-bit rules): role "worker" (a one-worker ctx: the worker stage, or the
+    update alone), "server" (the owner's W-worker server stage).  0 when not
+    modelled."""
+    gb, eb = wl.grad_bytes, wl.err_bytes
+    upd = 16.0 if wl.optimizer == "lamb" else 20.0
+    if rule == "scaled" and role == "worker":
+        return {"k_worker_norm": gb + eb,                      # g, err
+                "k_worker_pack": gb + 2 * eb + 1 / 8,          # g, err r/w, signs
+                "k_server_update": 1 / 8 + upd,                # server signs, m r/w, v, p (+ p w)
+                "k_lamb_param": 16.0}.get(kind, 0.0)
+    if rule == "scaled" and role == "server":
+        return {"k_server_norm": world / 8 + eb,               # W workers' signs, srv_err
+                "k_server_update": world / 8 + 2 * eb + 1 / 8}.get(kind, 0.0)  # signs, srv_err r/w, server signs
+    if rule == "twobit" and role == "worker":
+        return {"k_tb_worker_norm": gb + eb,                   # g, err
+                "k_tb_pack": gb + 2 * eb + 1 / 4,              # g, err r/w, both planes
+                "k_tb_server_update": 1 / 4 + upd,             # server planes, m r/w, v, p (+ p w)
+                "k_lamb_param": 16.0}.get(kind, 0.0)
+    if rule == "twobit" and role == "server":
+        return {"k_tb_server_norm": world / 4 + eb,            # W workers' planes, srv_err
+                "k_tb_server_update": world / 4 + 2 * eb + 1 / 4}.get(kind, 0.0)
+    return 0.0
     gb, eb = wl.grad_bytes, wl.err_bytes
     upd = 16.0 if wl.optimizer == "lamb" else 20.0
     if role == "worker":

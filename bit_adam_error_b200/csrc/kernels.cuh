@@ -468,13 +468,11 @@ __device__ __forceinline__ double block_sum_fixed(double x, double* sm) {
   return r;
 }
 
-// The result of (row r, chunk k) goes to out[(r * C + k) * planes + plane]: one
-// scale per chunk (planes = 1), or one of the two interleaved scales of the
-// 2-bit rule.
+// The result of (row r, chunk k) goes to out[r * C + k].
 template <bool RMS>
 __global__ void __launch_bounds__(kFinalizeThreads)
 k_finalize_scale(Layout L, const double* __restrict__ part, const int64_t* __restrict__ tpx,
-                 int mult, int64_t row_stride, float* __restrict__ out, int planes, int plane) {
+                 int mult, int64_t row_stride, float* __restrict__ out) {
   pdl_enter();
   __shared__ double sm[kFinalizeThreads];
   const int k = blockIdx.x, r = blockIdx.y;
@@ -487,7 +485,7 @@ k_finalize_scale(Layout L, const double* __restrict__ part, const int64_t* __res
     float o = 0.0f;
     if (!RMS) o = __double2float_rn(__dsqrt_rn(S));   // plain L2 norm (monitoring)
     else if (nk > 0) o = __double2float_rn(__ddiv_rn(__dsqrt_rn(S), __dsqrt_rn(static_cast<double>(nk))));
-    out[(static_cast<int64_t>(r) * L.C + k) * planes + plane] = o;
+    out[static_cast<int64_t>(r) * L.C + k] = o;
   }
 }
 
@@ -673,30 +671,37 @@ __device__ __forceinline__ void server_sum8(const Layout& L, int W, const uint32
   }
 }
 
-// Server norm only (stage-wise call): part_srv[t] = sum over the tile of c_srv^2.
-template <typename ET, bool POW2>
+// Server norm only (stage-wise call): part_srv[t] = sum over the tile of c_srv^2,
+// the values and the order of the fused pass 2.  The server errors of both groups
+// are loaded before the sums; W1 (with POW2): one worker (see server_sum8).
+template <typename ET, bool POW2, bool W1>
 __device__ __forceinline__ void server_norm_tiles(Layout L, int W, const uint32_t* __restrict__ bits_w, const float* __restrict__ s_w,
               const ET* __restrict__ srv_err, double* __restrict__ part_srv,
               uint32_t* __restrict__ status) {
   const int lane = threadIdx.x & 31;
-  const auto mean = make_mean<POW2>(W);
+  const auto mean = make_mean_w<POW2, W1>(W);
   int hint = 0;
   for (int64_t t = warp_id(); t < L.T; t += warp_count()) {
     const Tile tl = tile_at(L, t, hint);
     double tsum = 0.0;
     if (tl.vec) {
+      float sv[kGroups][8];
+      bool in[kGroups];
 #pragma unroll
       for (int q = 0; q < kGroups; ++q) {
         const int64_t i0 = tl.rel + q * kGroupElems + lane * kVec;
+        in[q] = i0 < tl.nk;
+        if (in[q]) ld8_ro(srv_err + tl.ck0 + i0, sv[q]); else zero8(sv[q]);
+      }
+#pragma unroll
+      for (int q = 0; q < kGroups; ++q) {
         const int64_t wrel = (tl.rel + q * kGroupElems) / 32 + (lane >> 2);
         float acc[8];
-        server_sum8<false>(L, W, bits_w, s_w, tl, wrel, wrel * 32 < tl.nk, lane, acc);
-        if (i0 < tl.nk) {
-          float sv[8];
-          ld8_ro(srv_err + tl.ck0 + i0, sv);
+        server_sum8<W1>(L, W, bits_w, s_w, tl, wrel, wrel * 32 < tl.nk, lane, acc);
+        if (in[q]) {
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
-            const float cs = mean(acc[j]) + sv[j];
+            const float cs = mean(acc[j]) + sv[q][j];
             tsum = fma(static_cast<double>(cs), static_cast<double>(cs), tsum);
           }
         }
@@ -706,7 +711,7 @@ __device__ __forceinline__ void server_norm_tiles(Layout L, int W, const uint32_
         const int64_t i = tl.rel + j * 32 + lane;
         if (i < tl.nk) {
           float acc = 0.0f;
-          for (int w = 0; w < W; ++w) {
+          for (int w = 0; w < (W1 ? 1 : W); ++w) {
             const float s = __ldg(s_w + static_cast<int64_t>(w) * L.C + tl.k);
             const uint32_t word = __ldg(bits_w + static_cast<int64_t>(w) * L.words + tl.w0 + tl.rel / 32 + j);
             acc = acc + signed_scale((word >> lane) & 1u, s);
@@ -724,24 +729,24 @@ __device__ __forceinline__ void server_norm_tiles(Layout L, int W, const uint32_
   }
 }
 
-template <typename ET, bool POW2>
+template <typename ET, bool POW2, bool W1>
 __global__ void __launch_bounds__(kBlock)
 k_server_norm(Layout L, int W, const uint32_t* __restrict__ bits_w, const float* __restrict__ s_w,
               const ET* __restrict__ srv_err, double* __restrict__ part_srv,
               uint32_t* __restrict__ status) {
   pdl_enter();
-  server_norm_tiles<ET, POW2>(L, W, bits_w, s_w, srv_err, part_srv, status);
+  server_norm_tiles<ET, POW2, W1>(L, W, bits_w, s_w, srv_err, part_srv, status);
 }
 
 // Small problems: the server sums and the server scale in one launch (the stage
 // call's counterpart of k_worker_pack_fin, so both give the same scale).
-template <typename ET, bool POW2>
+template <typename ET, bool POW2, bool W1>
 __global__ void __launch_bounds__(kBlock)
 k_server_norm_fin(Layout L, int W, const uint32_t* __restrict__ bits_w, const float* __restrict__ s_w,
               const ET* __restrict__ srv_err, double* __restrict__ part_srv,
               uint32_t* __restrict__ status, Fin fin) {
   pdl_enter();
-  server_norm_tiles<ET, POW2>(L, W, bits_w, s_w, srv_err, part_srv, status);
+  server_norm_tiles<ET, POW2, W1>(L, W, bits_w, s_w, srv_err, part_srv, status);
   fused_finalize(L, fin);
 }
 

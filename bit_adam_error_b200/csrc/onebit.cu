@@ -18,6 +18,7 @@
 #include <mutex>
 #include <new>
 #include <utility>
+#include <type_traits>
 #include <vector>
 
 #include <cuda_runtime.h>
@@ -255,11 +256,10 @@ ob_err check_grads(ob_ctx* c, const void* grads) {
 // planes / plane: where the scales land (one per chunk, or plane `plane` of the
 // two interleaved scales of the 2-bit rule).
 void enqueue_finalize_scale(ob_ctx* c, const double* part, float* out, int rows,
-                            const int64_t* tpx, int mult, int64_t row_stride, cudaStream_t st,
-                            int planes = 1, int plane = 0) {
+                            const int64_t* tpx, int mult, int64_t row_stride, cudaStream_t st) {
   launch(c, OB_K_FINALIZE_SCALE, st, [&] {
     pdl(ob::k_finalize_scale<true>, dim3(c->cfg.num_chunks, rows), ob::kFinalizeThreads, st, 
-        c->L, part, tpx, mult, row_stride, out, planes, plane);
+        c->L, part, tpx, mult, row_stride, out);
   });
 }
 
@@ -269,6 +269,7 @@ bool pow2_workers(const ob_ctx* c) { return (c->cfg.W & (c->cfg.W - 1)) == 0; }
 // Pass 2 issues one group of a tile at a time (3 CTAs per SM) up to this many
 // workers, two groups at a time (2 CTAs per SM) above it -- measured on B200:
 // W = 1 bf16 3.19 vs 3.47 ms per 1.5e9 elements, W = 16 fp32 10.30 vs 10.05 ms.
+// With bf16 error buffers two groups win at W = 1 too (3.13 vs 2.80 ms).
 constexpr int kPackOneGroupMaxW = 2;
 
 // Problems this small take the fused finaliser (the pass's last CTA computes the
@@ -307,7 +308,8 @@ void enqueue_worker_t(ob_ctx* c, const GT* grads, bool with_server, cudaStream_t
   if (c->T > 0) {
     // The stage call (no server part) never uses the mean: one instantiation each.
     // Many workers: the fused step also stores c_srv for pass 3 (CACHE).
-    const bool one = W <= kPackOneGroupMaxW, cache = with_server && c->csrv;
+    const bool one = W <= kPackOneGroupMaxW && !std::is_same<ET, uint16_t>::value;
+    const bool cache = with_server && c->csrv;
     const int kind = cache ? OB_K_WORKER_PACK_CACHED : OB_K_WORKER_PACK;
     if (fin2) {
       auto k2 = cache ? (one ? ob::k_worker_pack_fin<GT, ET, true, CLIP, POW2, 1, true>
@@ -434,8 +436,10 @@ void enqueue_warmup(ob_ctx* c, const GT* grads, cudaStream_t st) {
 template <typename ET>
 void enqueue_server_norm(ob_ctx* c, bool fin, cudaStream_t st) {
   const ET* srv_err = static_cast<const ET*>(c->srv_err);
+  const bool one = c->cfg.W == 1;
   if (fin) {
-    auto k = pow2_workers(c) ? ob::k_server_norm_fin<ET, true> : ob::k_server_norm_fin<ET, false>;
+    auto k = one ? ob::k_server_norm_fin<ET, true, true>
+                 : pow2_workers(c) ? ob::k_server_norm_fin<ET, true, false> : ob::k_server_norm_fin<ET, false, false>;
     const int g = grid_for(c, k, c->T);
     const ob::Fin f{c->ticket, c->part_srv, 0, 1, c->s_srv};
     launch(c, OB_K_SERVER_NORM, st, [&] {
@@ -443,7 +447,8 @@ void enqueue_server_norm(ob_ctx* c, bool fin, cudaStream_t st) {
     });
     return;
   }
-  auto k = pow2_workers(c) ? ob::k_server_norm<ET, true> : ob::k_server_norm<ET, false>;
+  auto k = one ? ob::k_server_norm<ET, true, true>
+               : pow2_workers(c) ? ob::k_server_norm<ET, true, false> : ob::k_server_norm<ET, false, false>;
   const int g = grid_for(c, k, c->T);
   launch(c, OB_K_SERVER_NORM, st, [&] {
     pdl(k, g, ob::kBlock, st, c->L, c->cfg.W, c->bits_w, c->s_w, srv_err, c->part_srv, c->status);
@@ -539,30 +544,29 @@ void enqueue_ternary_update(ob_ctx* c, cudaStream_t st) {
 
 // ---- the 2-bit rule (two residual sign planes) ------------------------------------------
 
-// Worker stage (passes 1, 1b, 2) and, when with_server, the server scales
-// (finalise s1', pass 2b, finalise s2').
+// Both scales of every (row, chunk) from the tile sums of a 2-bit pass (grid C x rows).
+void enqueue_tb_finalize(ob_ctx* c, const double* part, int rows, float* out, cudaStream_t st) {
+  launch(c, OB_K_TB_FINALIZE, st, [&] {
+    pdl(ob::k_tb_finalize, dim3(c->cfg.num_chunks, rows), ob::kFinalizeThreads, st, c->L, part, rows, out);
+  });
+}
+
+// Worker stage (passes 1 and 2, each followed by its scales) and, when
+// with_server, the server scales from pass 2's sums.
 template <typename GT, typename ET, bool CLIP, bool POW2>
 void enqueue_tb_worker_t(ob_ctx* c, const GT* grads, bool with_server, cudaStream_t st) {
   const int W = c->cfg.W;
   ET* err = static_cast<ET*>(c->err);
   const ET* srv_err = static_cast<const ET*>(c->srv_err);
   if (c->T > 0) {
-    auto k1 = ob::k_worker_norm<GT, ET, CLIP>;
+    auto k1 = ob::k_tb_worker_norm<GT, ET, CLIP>;
     const int g1 = grid_for(c, k1, W * c->T);
-    launch(c, OB_K_WORKER_NORM, st, [&] {
+    launch(c, OB_K_TB_WORKER_NORM, st, [&] {
       pdl(k1, g1, ob::kBlock, st, c->L, W, grads, err, c->h.clip, c->part_w, c->status);
     });
   }
-  enqueue_finalize_scale(c, c->part_w, c->s_w, W, c->L.tp, 1, c->T, st, 2, 0);
-  if (c->T > 0) {
-    auto k1b = ob::k_tb_resid_norm<GT, ET, CLIP>;
-    const int g = grid_for(c, k1b, W * c->T);
-    launch(c, OB_K_TB_RESID_NORM, st, [&] {
-      pdl(k1b, g, ob::kBlock, st, c->L, W, grads, err, c->s_w, c->h.clip, c->part_w);
-    });
-  }
-  enqueue_finalize_scale(c, c->part_w, c->s_w, W, c->L.tp, 1, c->T, st, 2, 1);
-  const bool cache = with_server && c->csrv;       // many workers: keep c_srv for 2b and 3
+  enqueue_tb_finalize(c, c->part_w, W, c->s_w, st);
+  const bool cache = with_server && c->csrv;       // many workers: keep c_srv for pass 3
   if (c->T > 0) {
     auto k2 = !with_server ? ob::k_tb_pack<GT, ET, false, CLIP, false, false>
               : cache      ? ob::k_tb_pack<GT, ET, true, CLIP, POW2, true>
@@ -573,22 +577,7 @@ void enqueue_tb_worker_t(ob_ctx* c, const GT* grads, bool with_server, cudaStrea
                                     c->csrv, c->h.clip, c->status);
     });
   }
-  if (!with_server) return;
-  enqueue_finalize_scale(c, c->part_srv, c->s_srv, 1, c->L.tp, 1, 0, st, 2, 0);
-  if (c->T > 0 && cache) {
-    auto k = ob::k_tb_server_norm_cached;
-    const int g = grid_for(c, k, c->T);
-    launch(c, OB_K_TB_SERVER_NORM_CACHED, st, [&] {
-      pdl(k, g, ob::kBlock, st, c->L, c->csrv, c->s_srv, c->part_srv);
-    });
-  } else if (c->T > 0) {
-    auto k = W == 1 ? ob::k_tb_server_norm<ET, true, true, true> : ob::k_tb_server_norm<ET, POW2, true, false>;
-    const int g = grid_for(c, k, c->T);
-    launch(c, OB_K_TB_SERVER_NORM, st, [&] {
-      pdl(k, g, ob::kBlock, st, c->L, W, c->bits_w, c->s_w, srv_err, c->s_srv, c->part_srv, c->status);
-    });
-  }
-  enqueue_finalize_scale(c, c->part_srv, c->s_srv, 1, c->L.tp, 1, 0, st, 2, 1);
+  if (with_server) enqueue_tb_finalize(c, c->part_srv, 1, c->s_srv, st);
 }
 
 template <typename GT, typename ET>
@@ -656,28 +645,19 @@ void enqueue_tb_update(ob_ctx* c, bool from_workers, cudaStream_t st) {
   if (lamb) enqueue_lamb_param(c, st);
 }
 
-// Server stage alone: s1' (pass over the planes), s2' (residual pass), then the
-// server planes and error.
+// Server stage alone: the server sums (one pass over the planes), both server
+// scales, then the server planes and error.
 template <typename ET, bool POW2>
 void enqueue_tb_server_stage_t(ob_ctx* c, cudaStream_t st) {
   const ET* srv_err = static_cast<const ET*>(c->srv_err);
-  const bool one = c->cfg.W == 1;
   if (c->T > 0) {
-    auto k = one ? ob::k_tb_server_norm<ET, true, false, true> : ob::k_tb_server_norm<ET, POW2, false, false>;
+    auto k = c->cfg.W == 1 ? ob::k_tb_server_norm<ET, true, true> : ob::k_tb_server_norm<ET, POW2, false>;
     const int g = grid_for(c, k, c->T);
     launch(c, OB_K_TB_SERVER_NORM, st, [&] {
-      pdl(k, g, ob::kBlock, st, c->L, c->cfg.W, c->bits_w, c->s_w, srv_err, c->s_srv, c->part_srv, c->status);
+      pdl(k, g, ob::kBlock, st, c->L, c->cfg.W, c->bits_w, c->s_w, srv_err, c->part_srv, c->status);
     });
   }
-  enqueue_finalize_scale(c, c->part_srv, c->s_srv, 1, c->L.tp, 1, 0, st, 2, 0);
-  if (c->T > 0) {
-    auto k = one ? ob::k_tb_server_norm<ET, true, true, true> : ob::k_tb_server_norm<ET, POW2, true, false>;
-    const int g = grid_for(c, k, c->T);
-    launch(c, OB_K_TB_SERVER_NORM, st, [&] {
-      pdl(k, g, ob::kBlock, st, c->L, c->cfg.W, c->bits_w, c->s_w, srv_err, c->s_srv, c->part_srv, c->status);
-    });
-  }
-  enqueue_finalize_scale(c, c->part_srv, c->s_srv, 1, c->L.tp, 1, 0, st, 2, 1);
+  enqueue_tb_finalize(c, c->part_srv, 1, c->s_srv, st);
   enqueue_tb_server_update<ob::Upd::kNone, true>(c, st);
 }
 
@@ -864,7 +844,11 @@ ob_err ob_create(const ob_config* cfg, float* p, float* m, float* v, void* err, 
   auto up256 = [](size_t x) { return (x + 255) & ~size_t(255); };
   const size_t sz_tab = up256(sizeof(int64_t) * (C + 1));
   const size_t sz_vec = up256(size_t(C));
-  const size_t sz_pw = up256(sizeof(double) * size_t(W) * size_t(c->T));
+  // The 2-bit rule keeps three sums per tile: c^2, |c| and the squared
+  // deviations of |c| (twobit.cuh).
+  const size_t sums = two_bit_rule(cfg) ? 3 : 1;
+  const size_t sz_pw = up256(sizeof(double) * sums * size_t(W) * size_t(c->T));
+  const size_t sz_ps = up256(sizeof(double) * sums * size_t(c->T));
   const size_t sz_pt = up256(sizeof(double) * size_t(c->T));
   const size_t sz_ratio = up256(sizeof(float) * size_t(C));
   // c_srv cache of the fused step: scaled-sign rules with many workers, on a ctx
@@ -872,7 +856,7 @@ ob_err ob_create(const ob_config* cfg, float* p, float* m, float* v, void* err, 
   const bool fused_capable = p && m && v && err && srv_err && bits_w && s_w && bits_srv && s_srv;
   const bool cache = !momentum_rule(cfg) && W >= kCacheMinW && fused_capable && n > 0;
   const size_t sz_cs = cache ? up256(sizeof(float) * size_t(n)) : 0;
-  const size_t total = 3 * sz_tab + sz_vec + sz_pw + 3 * sz_pt + sz_ratio + sz_cs + 512;
+  const size_t total = 3 * sz_tab + sz_vec + sz_pw + sz_ps + 2 * sz_pt + sz_ratio + sz_cs + 512;
   if ((e = cudaMalloc(&c->scratch, total)) != cudaSuccess) {
     cudaGetLastError();
     delete c;
@@ -884,7 +868,7 @@ ob_err ob_create(const ob_config* cfg, float* p, float* m, float* v, void* err, 
   int64_t* d_tp = reinterpret_cast<int64_t*>(base); base += sz_tab;
   uint8_t* d_vec = reinterpret_cast<uint8_t*>(base); base += sz_vec;
   c->part_w = reinterpret_cast<double*>(base); base += sz_pw;
-  c->part_srv = reinterpret_cast<double*>(base); base += sz_pt;
+  c->part_srv = reinterpret_cast<double*>(base); base += sz_ps;
   c->partP = reinterpret_cast<double*>(base); base += sz_pt;
   c->partU = reinterpret_cast<double*>(base); base += sz_pt;
   c->ratio = reinterpret_cast<float*>(base); base += sz_ratio;
@@ -1187,7 +1171,7 @@ ob_err ob_error_norms(ob_ctx* c, float* worker_norms, float* server_norms, void*
     }
     launch(c, OB_K_FINALIZE_SCALE, st, [&] {
       pdl(ob::k_finalize_scale<false>, dim3(unsigned(C), unsigned(rows)), ob::kFinalizeThreads, st,
-          c->L, part, c->L.tp, 1, c->T, out, 1, 0);
+          c->L, part, c->L.tp, 1, c->T, out);
     });
   };
   if (worker_norms) norms(c->err, int(W), c->part_w, worker_norms);
@@ -1283,8 +1267,8 @@ const char* ob_kernel_name(int32_t kind) {
       "k_worker_norm", "k_finalize_scale", "k_worker_pack", "k_server_norm",
       "k_server_update", "k_lamb_param", "k_warmup", "k_finalize_ratio",
       "k_ternary_step", "k_ternary_compress", "k_ternary_server", "k_ternary_update",
-      "k_tb_resid_norm", "k_tb_pack", "k_tb_server_norm", "k_tb_server_update",
-      "k_worker_pack_cached", "k_server_update_cached", "k_tb_pack_cached", "k_tb_server_norm_cached",
+      "k_tb_worker_norm", "k_tb_pack", "k_tb_server_norm", "k_tb_server_update",
+      "k_worker_pack_cached", "k_server_update_cached", "k_tb_pack_cached", "k_tb_finalize",
       "k_tb_server_update_cached", "k_local_step", "k_sign_count", "k_grad_mean"};
   return (kind >= 0 && kind < OB_K_KINDS) ? names[kind] : "";
 }
@@ -1455,7 +1439,7 @@ extern "C" ob_err ob_compress_noalloc(const ob_config* cfg, const void* grads, f
     else if (cl) ob::k_worker_norm<float, float, true><<<g1, ob::kBlock, 0, st>>>(L, int(W), gf, err, clip, part, status);
     else ob::k_worker_norm<float, float, false><<<g1, ob::kBlock, 0, st>>>(L, int(W), gf, err, clip, part, status);
   }
-  ob::k_finalize_scale<true><<<dim3(unsigned(C), unsigned(W)), ob::kFinalizeThreads, 0, st>>>(L, part, L.tp, 1, T, s_w, 1, 0);
+  ob::k_finalize_scale<true><<<dim3(unsigned(C), unsigned(W)), ob::kFinalizeThreads, 0, st>>>(L, part, L.tp, 1, T, s_w);
   if (T > 0) {
     const int g2 = noalloc_grid(d->num_sms, d->occ_pack[bf][cl ? 1 : 0], T);
     const uint16_t* gh = static_cast<const uint16_t*>(grads);

@@ -8,17 +8,23 @@
 //   dequantised value = s1 sign(q1) + s2 sign(q2)
 // for the workers and, on their average plus the server error, for the server.
 //
-// Each extra norm is another streaming pass: s2 needs s1 before r exists, and
-// the server's s2 needs its s1.  The fused step is five passes (plus finalisers):
-//   1  k_worker_norm        g, err            -> sum c^2          -> s1
-//   1b k_tb_resid_norm      g, err            -> sum r^2          -> s2
-//   2  k_tb_pack<SERVER>    g, err, srv_err   -> err, planes, sum c_srv^2 -> s1'
-//   2b k_tb_server_norm<R>  planes, srv_err   -> sum r_srv^2      -> s2'
+// s2 needs s1, which is known only once the whole chunk has been read.  Since
+// r_i^2 = (|c_i| - s1)^2, the sum over the chunk is, for any split of the chunk
+// into tiles t of n_t elements with mean mu_t of |c|,
+//   ||r||^2 = sum_t [ sum_{i in t} (|c_i| - mu_t)^2 + n_t (mu_t - s1)^2 ],
+// an identity of real arithmetic whose terms are all >= 0 (no cancellation,
+// even when every |c_i| is close to s1).  So the pass that reads c for ||c||
+// also keeps, per warp tile, S = sum |c| and M2 = sum (|c| - S / n_t)^2, and
+// the finaliser forms ||r||^2 from them once s1 is in hand: the fused step is
+// three streaming passes, as for 1 bit.  ||r||^2 differs from the sum of the
+// squared float residuals by their rounding only (at most 2^-23 relative).
+//   1  k_tb_worker_norm     g, err            -> sum c^2, moments of |c|      -> s1, s2
+//   2  k_tb_pack<SERVER>    g, err, srv_err   -> err, planes, the same of c_srv -> s1', s2'
 //   3  k_tb_server_update   planes, srv_err, m, v, p -> server planes, srv_err, m, p
 // Layout: chunk k owns 2 ceil(n_k / 32) words of a row, plane 1 then plane 2,
 // from word wo[k]; scales are [row][C][2].  Tiling, vector/scalar paths and the
-// floating-point order are those of kernels.cuh (every value equals the plain C
-// statement of the rule for the same scales).
+// floating-point order of the per-element values are those of kernels.cuh
+// (every value equals the plain C statement of the rule for the same scales).
 #pragma once
 
 #include "kernels.cuh"
@@ -26,6 +32,40 @@
 namespace ob {
 
 __device__ __forceinline__ int64_t plane_words(int64_t nk) { return (nk + 31) / 32; }
+
+// ---- tile sums of |c| for the second scale -------------------------------------------
+// One sweep, shifted by K = |c| of the tile's first element (lane 0 holds it on
+// both paths): every lane adds d = |c| - K and d^2 of its elements, and after the
+// warp sums
+//   S_t = n_t K + sum d,   M2_t = sum d^2 - (sum d)^2 / n_t   (>= 0, clamped).
+// K is one of the values, so n_t (mean - K)^2 <= n_t M2_t and the subtraction
+// loses at most about 2 n_t ulps of M2_t; equal magnitudes give M2_t = 0 exactly.
+struct Shifted {
+  double K, d1, d2;
+};
+
+__device__ __forceinline__ Shifted shifted_from(float first_lane0) {
+  return Shifted{fabs(static_cast<double>(__shfl_sync(kFull, first_lane0, 0))), 0.0, 0.0};
+}
+
+__device__ __forceinline__ void shifted_add(Shifted& m, double c) {
+  const double d = fabs(c) - m.K;
+  m.d1 += d;
+  m.d2 = fma(d, d, m.d2);
+}
+
+// Warp sums; lane 0 stores S_t at part[P + t] and M2_t at part[2P + t].
+__device__ __forceinline__ void store_shifted(Shifted m, const Tile& tl, double* __restrict__ part, int64_t P,
+                                              int64_t t, int lane) {
+  const double d1 = warp_sum(m.d1), d2 = warp_sum(m.d2);
+  if (lane == 0) {
+    const int64_t left = tl.nk - tl.rel;
+    const int nt = left < kTile ? static_cast<int>(left) : kTile;
+    const double sq = nt == kTile ? d1 * d1 * (1.0 / kTile) : d1 * d1 / nt;
+    part[P + t] = static_cast<double>(nt) * m.K + d1;
+    part[2 * P + t] = fmax(d2 - sq, 0.0);
+  }
+}
 
 // The four dequantised values (+-s1) + (+-s2) of one worker's chunk, d<b1><b2>,
 // formed once per tile: the same float additions the per-element form makes.
@@ -85,11 +125,14 @@ __device__ __forceinline__ float tb_server_sum1(const Layout& L, int W, const ui
   return acc;
 }
 
-// ---- pass 1b: per-tile sum of r^2, r = c - s1 sign(c) ---------------------------------
+// ---- pass 1: per tile, sum c^2 and the sums of |c| of every worker ---------------------
+// Item it = w * T + t (P = W * T items): part[it] = sum c^2 (the order of the 1-bit
+// pass 1), part[P + it] = S_t, part[2P + it] = M2_t (see Shifted).  A non-finite
+// sum c^2 raises the status flag.
 template <typename GT, typename ET, bool CLIP>
 __global__ void __launch_bounds__(kBlock)
-k_tb_resid_norm(Layout L, int W, const GT* __restrict__ grads, const ET* __restrict__ err,
-                const float* __restrict__ s_w, float clip, double* __restrict__ part) {
+k_tb_worker_norm(Layout L, int W, const GT* __restrict__ grads, const ET* __restrict__ err,
+                 float clip, double* __restrict__ part, uint32_t* __restrict__ status) {
   pdl_enter();
   const int lane = threadIdx.x & 31;
   const int64_t items = static_cast<int64_t>(W) * L.T;
@@ -100,41 +143,55 @@ k_tb_resid_norm(Layout L, int W, const GT* __restrict__ grads, const ET* __restr
     const Tile tl = tile_at(L, t, hint);
     const GT* g = grads + static_cast<int64_t>(w) * L.n + tl.ck0;
     const ET* e = err + static_cast<int64_t>(w) * L.n + tl.ck0;
-    const float s1 = __ldg(s_w + (static_cast<int64_t>(w) * L.C + tl.k) * 2);
     double acc = 0.0;
+    Shifted m;
     if (tl.vec) {
+      float gv[kGroups][8], ev[kGroups][8];
+      bool in[kGroups];
 #pragma unroll
-      for (int gq = 0; gq < kGroups; ++gq) {
-        const int64_t i0 = tl.rel + gq * kGroupElems + lane * kVec;
-        if (i0 < tl.nk) {
-          float gv[8], ev[8];
-          ld8_ro(g + i0, gv);
-          ld8_ro(e + i0, ev);
+      for (int q = 0; q < kGroups; ++q) {
+        const int64_t i0 = tl.rel + q * kGroupElems + lane * kVec;
+        in[q] = i0 < tl.nk;
+        if (in[q]) { ld8_ro(g + i0, gv[q]); ld8_ro(e + i0, ev[q]); }
+        else { zero8(gv[q]); zero8(ev[q]); }
+      }
+      m = shifted_from((CLIP ? clip_grad(gv[0][0], clip) : gv[0][0]) + ev[0][0]);
+#pragma unroll
+      for (int q = 0; q < kGroups; ++q)
+        if (in[q]) {
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
-            const float c = (CLIP ? clip_grad(gv[j], clip) : gv[j]) + ev[j];
-            const float r = c - signed_scale(c >= 0.0f, s1);
-            acc = fma(static_cast<double>(r), static_cast<double>(r), acc);
+            const double c = static_cast<double>((CLIP ? clip_grad(gv[q][j], clip) : gv[q][j]) + ev[q][j]);
+            acc = fma(c, c, acc);
+            shifted_add(m, c);
           }
         }
-      }
     } else {
       for (int j = 0; j < kTileWords; ++j) {
         const int64_t i = tl.rel + j * 32 + lane;
+        float c = 0.0f;
+        if (i < tl.nk) c = (CLIP ? clip_grad(ld1_ro(g + i), clip) : ld1_ro(g + i)) + ld1_ro(e + i);
+        if (j == 0) m = shifted_from(c);
         if (i < tl.nk) {
-          const float c = (CLIP ? clip_grad(ld1_ro(g + i), clip) : ld1_ro(g + i)) + ld1_ro(e + i);
-          const float r = c - signed_scale(c >= 0.0f, s1);
-          acc = fma(static_cast<double>(r), static_cast<double>(r), acc);
+          const double cd = static_cast<double>(c);
+          acc = fma(cd, cd, acc);
+          shifted_add(m, cd);
         }
       }
     }
+    store_shifted(m, tl, part, items, it, lane);
     acc = warp_sum(acc);
-    if (lane == 0) part[it] = acc;
+    if (lane == 0) {
+      part[it] = acc;
+      flag_tile_sum(acc, status);
+    }
   }
 }
 
 // ---- pass 2: both planes, worker error (+ server sums) ---------------------------------
-// CACHE (with SERVER): c_srv also goes to csrv[n] for passes 2b and 3.
+// SERVER: also c_srv = (sum_w dequantised_w) / W + srv_err, with part_srv[t] =
+// sum c_srv^2, part_srv[T + t] = S_t and part_srv[2T + t] = M2_t of |c_srv| (see
+// Shifted).  CACHE (with SERVER): c_srv also goes to csrv[n] for pass 3.
 // Three CTAs per SM (at most 80 registers): the cached, clipped variant would
 // otherwise take 92 and drop to two.
 template <typename GT, typename ET, bool SERVER, bool CLIP, bool POW2, bool CACHE>
@@ -150,6 +207,7 @@ k_tb_pack(Layout L, int W, const GT* __restrict__ grads, ET* __restrict__ err,
     const Tile tl = tile_at(L, t, hint);
     const int64_t nwk = plane_words(tl.nk);
     double tsum = 0.0;
+    Shifted mo{0.0, 0.0, 0.0};
     if (tl.vec) {
 #pragma unroll 1
       for (int gq = 0; gq < kGroups; ++gq) {
@@ -192,13 +250,20 @@ k_tb_pack(Layout L, int W, const GT* __restrict__ grads, ET* __restrict__ err,
             row[nwk + wrel] = word2;
           }
         }
-        if (SERVER && in) {
+        if constexpr (SERVER) {
+          if (in) {
 #pragma unroll
-          for (int j = 0; j < 8; ++j) {            // c_srv in place of the sum
-            acc[j] = mean(acc[j]) + sv[j];
-            tsum = fma(static_cast<double>(acc[j]), static_cast<double>(acc[j]), tsum);
+            for (int j = 0; j < 8; ++j) {            // c_srv in place of the sum
+              acc[j] = mean(acc[j]) + sv[j];
+              tsum = fma(static_cast<double>(acc[j]), static_cast<double>(acc[j]), tsum);
+            }
+            if (CACHE) st8(csrv + tl.ck0 + i0, acc);
           }
-          if (CACHE) st8(csrv + tl.ck0 + i0, acc);
+          if (gq == 0) mo = shifted_from(acc[0]);
+          if (in) {
+#pragma unroll
+            for (int j = 0; j < 8; ++j) shifted_add(mo, static_cast<double>(acc[j]));
+          }
         }
       }
     } else {
@@ -229,14 +294,19 @@ k_tb_pack(Layout L, int W, const GT* __restrict__ grads, ET* __restrict__ err,
             row[nwk + wi] = word2;
           }
         }
-        if (SERVER && inb) {
-          const float cs = mean(acc) + ld1_ro(srv_err + tl.ck0 + i);
-          tsum = fma(static_cast<double>(cs), static_cast<double>(cs), tsum);
-          if (CACHE) csrv[tl.ck0 + i] = cs;
+        if constexpr (SERVER) {
+          const float cs = inb ? mean(acc) + ld1_ro(srv_err + tl.ck0 + i) : 0.0f;
+          if (j == 0) mo = shifted_from(cs);
+          if (inb) {
+            tsum = fma(static_cast<double>(cs), static_cast<double>(cs), tsum);
+            if (CACHE) csrv[tl.ck0 + i] = cs;
+            shifted_add(mo, static_cast<double>(cs));
+          }
         }
       }
     }
-    if (SERVER) {
+    if constexpr (SERVER) {
+      store_shifted(mo, tl, part_srv, L.T, t, lane);
       tsum = warp_sum(tsum);
       if (lane == 0) {
         part_srv[t] = tsum;
@@ -246,15 +316,14 @@ k_tb_pack(Layout L, int W, const GT* __restrict__ grads, ET* __restrict__ err,
   }
 }
 
-// ---- server norms from the worker planes --------------------------------------------
-// RESID = false: sum c_srv^2 (for s1'; the stage call).  RESID = true: sum of
-// (c_srv - s1' sign(c_srv))^2 (for s2'), s1' read from s_srv.  W1 (with POW2):
-// one worker (see tb_server_sum8).
-template <typename ET, bool POW2, bool RESID, bool W1>
+// ---- server sums from the worker planes (stage call) ----------------------------------
+// part[t] = sum c_srv^2, part[T + t] = S_t, part[2T + t] = M2_t of |c_srv| (see
+// Shifted; one row): the values and the order of the fused pass 2.  W1 (with
+// POW2): one worker (see tb_server_sum8).
+template <typename ET, bool POW2, bool W1>
 __global__ void __launch_bounds__(kBlock)
 k_tb_server_norm(Layout L, int W, const uint32_t* __restrict__ bits_w, const float* __restrict__ s_w,
-                 const ET* __restrict__ srv_err, const float* __restrict__ s_srv,
-                 double* __restrict__ part, uint32_t* __restrict__ status) {
+                 const ET* __restrict__ srv_err, double* __restrict__ part, uint32_t* __restrict__ status) {
   pdl_enter();
   const int lane = threadIdx.x & 31;
   const auto mean = make_mean_w<POW2, W1>(W);
@@ -262,13 +331,9 @@ k_tb_server_norm(Layout L, int W, const uint32_t* __restrict__ bits_w, const flo
   for (int64_t t = warp_id(); t < L.T; t += warp_count()) {
     const Tile tl = tile_at(L, t, hint);
     const int64_t nwk = plane_words(tl.nk);
-    const float s1 = RESID ? __ldg(s_srv + 2 * tl.k) : 0.0f;
     const Dq4 dq = W1 ? dq4_of(s_w, tl.k) : Dq4{};
     double tsum = 0.0;
-    auto add = [&](float cs) {
-      const float x = RESID ? cs - signed_scale(cs >= 0.0f, s1) : cs;
-      tsum = fma(static_cast<double>(x), static_cast<double>(x), tsum);
-    };
+    Shifted mo{0.0, 0.0, 0.0};
     if (tl.vec) {
 #pragma unroll
       for (int gq = 0; gq < kGroups; ++gq) {
@@ -280,61 +345,76 @@ k_tb_server_norm(Layout L, int W, const uint32_t* __restrict__ bits_w, const flo
         tb_server_sum8<W1>(L, W, bits_w, s_w, tl, wrel, nwk, wrel * 32 < tl.nk, lane, acc, dq);
         if (in) {
 #pragma unroll
-          for (int j = 0; j < 8; ++j) add(mean(acc[j]) + sv[j]);
+          for (int j = 0; j < 8; ++j) {
+            acc[j] = mean(acc[j]) + sv[j];
+            tsum = fma(static_cast<double>(acc[j]), static_cast<double>(acc[j]), tsum);
+          }
+        }
+        if (gq == 0) mo = shifted_from(acc[0]);
+        if (in) {
+#pragma unroll
+          for (int j = 0; j < 8; ++j) shifted_add(mo, static_cast<double>(acc[j]));
         }
       }
     } else {
       for (int j = 0; j < kTileWords; ++j) {
         const int64_t i = tl.rel + j * 32 + lane;
-        if (i < tl.nk) add(mean(tb_server_sum1<W1>(L, W, bits_w, s_w, tl, tl.rel / 32 + j, nwk, lane)) +
-                           ld1_ro(srv_err + tl.ck0 + i));
+        const bool inb = i < tl.nk;
+        const float cs = inb ? mean(tb_server_sum1<W1>(L, W, bits_w, s_w, tl, tl.rel / 32 + j, nwk, lane)) +
+                                   ld1_ro(srv_err + tl.ck0 + i)
+                             : 0.0f;
+        if (j == 0) mo = shifted_from(cs);
+        if (inb) {
+          tsum = fma(static_cast<double>(cs), static_cast<double>(cs), tsum);
+          shifted_add(mo, static_cast<double>(cs));
+        }
       }
     }
+    store_shifted(mo, tl, part, L.T, t, lane);
     tsum = warp_sum(tsum);
     if (lane == 0) {
       part[t] = tsum;
-      if (!RESID) flag_tile_sum(tsum, status);
+      flag_tile_sum(tsum, status);
     }
   }
 }
 
-// Pass 2b when pass 2 stored c_srv: sum of (c_srv - s1' sign(c_srv))^2 from csrv.
-__global__ void __launch_bounds__(kBlock)
-k_tb_server_norm_cached(Layout L, const float* __restrict__ csrv, const float* __restrict__ s_srv,
-                        double* __restrict__ part) {
+// ---- both scales of a chunk from the tile sums ----------------------------------------------
+// Row r, chunk k (P = rows * T): A = sum_t part[r*T + t], s1 = sqrt(A) / sqrt(n_k);
+// then, with S_t = part[P + r*T + t], M2_t = part[2P + r*T + t] and n_t the tile's
+// element count,
+//   R = sum_t [ M2_t + n_t (S_t / n_t - s1)^2 ],   s2 = sqrt(R) / sqrt(n_k);
+// both 0 for an empty chunk.  Fixed-order sums (the order of k_finalize_scale);
+// a full tile's mean is an exact multiply by 1/kTile.
+// out[(r * C + k) * 2 + {0, 1}] = s1, s2.  grid = (C, rows).
+__global__ void __launch_bounds__(kFinalizeThreads)
+k_tb_finalize(Layout L, const double* __restrict__ part, int rows, float* __restrict__ out) {
   pdl_enter();
-  const int lane = threadIdx.x & 31;
-  int hint = 0;
-  for (int64_t t = warp_id(); t < L.T; t += warp_count()) {
-    const Tile tl = tile_at(L, t, hint);
-    const float s1 = __ldg(s_srv + 2 * tl.k);
-    double tsum = 0.0;
-    if (tl.vec) {
-#pragma unroll
-      for (int gq = 0; gq < kGroups; ++gq) {
-        const int64_t i0 = tl.rel + gq * kGroupElems + lane * kVec;
-        if (i0 < tl.nk) {
-          float cv[8];
-          ld8_ro(csrv + tl.ck0 + i0, cv);
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const float x = cv[j] - signed_scale(cv[j] >= 0.0f, s1);
-            tsum = fma(static_cast<double>(x), static_cast<double>(x), tsum);
-          }
-        }
-      }
-    } else {
-      for (int j = 0; j < kTileWords; ++j) {
-        const int64_t i = tl.rel + j * 32 + lane;
-        if (i < tl.nk) {
-          const float cs = __ldg(csrv + tl.ck0 + i);
-          const float x = cs - signed_scale(cs >= 0.0f, s1);
-          tsum = fma(static_cast<double>(x), static_cast<double>(x), tsum);
-        }
-      }
-    }
-    tsum = warp_sum(tsum);
-    if (lane == 0) part[t] = tsum;
+  __shared__ double sm[kFinalizeThreads];
+  const int k = blockIdx.x, r = blockIdx.y;
+  const int64_t P = static_cast<int64_t>(rows) * L.T;
+  const double* pa = part + static_cast<int64_t>(r) * L.T;
+  const double* ps = pa + P;
+  const double* pm = pa + 2 * P;
+  const int64_t t0 = L.tp[k], t1 = L.tp[k + 1], nk = L.off[k + 1] - L.off[k];
+  double acc = 0.0;
+  for (int64_t t = t0 + threadIdx.x; t < t1; t += kFinalizeThreads) acc += pa[t];
+  const double A = block_sum_fixed(acc, sm);
+  const double rn = __dsqrt_rn(static_cast<double>(nk));
+  const float s1 = nk > 0 ? __double2float_rn(__ddiv_rn(__dsqrt_rn(A), rn)) : 0.0f;
+  acc = 0.0;
+  for (int64_t t = t0 + threadIdx.x; t < t1; t += kFinalizeThreads) {
+    const int64_t left = nk - (t - t0) * kTile;
+    const double mu = left >= kTile ? ps[t] * (1.0 / kTile) : ps[t] / static_cast<double>(left);
+    const double nt = static_cast<double>(left < kTile ? left : kTile);
+    const double d = mu - static_cast<double>(s1);
+    acc += pm[t] + nt * d * d;
+  }
+  const double R = block_sum_fixed(acc, sm);
+  if (threadIdx.x == 0) {
+    float* o = out + (static_cast<int64_t>(r) * L.C + k) * 2;
+    o[0] = s1;
+    o[1] = nk > 0 ? __double2float_rn(__ddiv_rn(__dsqrt_rn(R), rn)) : 0.0f;
   }
 }
 

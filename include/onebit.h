@@ -301,17 +301,17 @@ enum {
   OB_K_TERNARY_COMPRESS = 9, /* momentum-error rule: codes + worker error (stage call) */
   OB_K_TERNARY_SERVER = 10,  /* momentum-error rule: sum of the workers' codes */
   OB_K_TERNARY_UPDATE = 11,  /* momentum-error rule: update from the code sums */
-  OB_K_TB_RESID_NORM = 12,   /* 2-bit: per-tile sums of the first plane's residual^2 */
+  OB_K_TB_WORKER_NORM = 12,  /* 2-bit pass 1: per-tile sums of c^2 and moments of |c|, every worker */
   OB_K_TB_PACK = 13,         /* 2-bit: both planes, worker error (+ server sums) */
-  OB_K_TB_SERVER_NORM = 14,  /* 2-bit: server sums (or residual sums) from the planes */
+  OB_K_TB_SERVER_NORM = 14,  /* 2-bit: server sums from the planes (stage call) */
   OB_K_TB_SERVER_UPDATE = 15,/* 2-bit: server planes + error, and/or the update */
   /* The fused step with W >= 4 workers: pass 2 also stores the server value
-   * c_srv (one float per element, in the ctx scratch) and the server passes read
-   * it instead of rebuilding it from the W workers' words. */
+   * c_srv (one float per element, in the ctx scratch) and pass 3 reads it
+   * instead of rebuilding it from the W workers' words. */
   OB_K_WORKER_PACK_CACHED = 16,
   OB_K_SERVER_UPDATE_CACHED = 17,
   OB_K_TB_PACK_CACHED = 18,
-  OB_K_TB_SERVER_NORM_CACHED = 19,
+  OB_K_TB_FINALIZE = 19,     /* 2-bit: both scales of every chunk from the tile sums */
   OB_K_TB_SERVER_UPDATE_CACHED = 20,
   OB_K_LOCAL_STEP = 21,      /* 0/1 Adam local step */
   OB_K_SIGN_COUNT = 22,      /* quantisation rate: per-tile counts of set sign bits */

@@ -63,13 +63,13 @@ def test_byte_model_of_the_one_pass_step():
 
 
 def test_byte_model_of_the_two_bit_step():
-    """Five passes: two worker norm passes, the two-plane pack, the server
-    residual norm and the server/update pass."""
+    """Three passes: the worker sums (both scales), the two-plane pack with the
+    server sums, and the server/update pass."""
     sys.path.insert(0, ROOT)
     import bench
     import workloads as WL
     wl = WL.get_workload("gpt2xl-flat")
-    assert bench.step_bytes_per_elem(wl, "compressed", "twobit") == 6 + 6 + 14.25 + 4.25 + 28.5
+    assert bench.step_bytes_per_elem(wl, "compressed", "twobit") == 6 + 14.25 + 28.5
 
 
 def test_reference_arm_two_bit_rule():
@@ -131,3 +131,5 @@ def test_byte_model_of_the_data_parallel_stages():
     assert bench.dp_bytes_per_elem("k_server_update", "server", wl, 8, "scaled") == 1 + 8 + 1 / 8
     assert bench.dp_bytes_per_elem("k_finalize_scale", "worker", wl, 8, "scaled") == 0
     assert bench.dp_bytes_per_elem("k_worker_norm", "worker", wl, 8, "momentum") == 0
+    assert bench.dp_bytes_per_elem("k_tb_pack", "worker", wl, 8, "twobit") == 2 + 8 + 1 / 4
+    assert bench.dp_bytes_per_elem("k_tb_server_norm", "server", wl, 8, "twobit") == 2 + 4

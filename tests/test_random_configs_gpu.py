@@ -17,7 +17,7 @@ import oracle
 import workloads as WL
 from bit_adam_error_b200 import OneBitAdam
 from gpu_harness import F, HP, as_f32, assert_bits, assert_scales, assert_state, dev, grads_for, np_of, \
-    state_for, to_dev
+    state_for, sync_state, to_dev
 
 pytestmark = pytest.mark.gpu
 
@@ -70,11 +70,14 @@ def test_random_config(rule, case):
         torch.cuda.synchronize()
         for k in keys:
             got = np_of(getattr(gpu, k))
-            assert_state(f"{tag} step {t} {k}", as_f32(got), as_f32(ref[k].reshape(got.shape)), wl.offsets)
+            assert_state(f"{tag} step {t} {k}", as_f32(got), as_f32(ref[k].reshape(got.shape)), wl.offsets,
+                         bf16_step=rule == "twobit" and got.dtype == np.uint16)
         if rule != "momentum":          # (the momentum rule's fused step keeps its codes in registers)
             assert_bits(f"{tag} bits_w", np_of(gpu.bits_w), ref["bits_w"])
             assert_bits(f"{tag} bits_srv", np_of(gpu.bits_srv), ref["bits_srv"])
             assert_scales(f"{tag} s_w", np_of(gpu.s_w), ref["s_w"])
             assert_scales(f"{tag} s_srv", np_of(gpu.s_srv), ref["s_srv"])
+        if rule == "twobit":            # the next step from the oracle's state (second scale to an ulp)
+            sync_state(gpu, ref)
     assert gpu.status() == flags == 0, tag
     gpu.close()

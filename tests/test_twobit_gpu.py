@@ -2,10 +2,12 @@
 the C ABI.
 
 Stage by stage with identical input state (worker planes, scales and errors;
-the server stage from seeded planes and scales; the update), then chained fused
+the server stage from seeded planes and scales; the update), then runs of fused
 steps on ragged and aligned layouts (Adam, LAMB, bf16 gradients and error
-buffers, clip, many workers), fused = stages, and the non-finite flag.  Planes
-compare bit for bit, scales within 1e-5, state at the parity bar.
+buffers, clip, many workers), each step from the oracle's state, fused =
+stages, and the non-finite flag.  Planes compare bit for bit, scales within
+1e-5, state at the parity bar (bf16 error buffers: plus one bf16 step, see
+gpu_harness).
 """
 
 import numpy as np
@@ -16,7 +18,7 @@ import oracle
 import workloads as WL
 from bit_adam_error_b200 import OneBitAdam, _lib as L
 from gpu_harness import (F, HP, as_f32, assert_bits, assert_scales, assert_state, dev, grads_for, np_of,
-                         state_for, to_dev)
+                         state_for, sync_state, to_dev)
 
 pytestmark = pytest.mark.gpu
 
@@ -150,13 +152,15 @@ def run_chain(wl, steps, err_dtype="f32"):
         for k in ("p", "m", "v", "err", "srv_err"):
             got = np_of(getattr(gpu, k))
             want = ref[k].reshape(got.shape)
-            assert_state(f"step {t} {k}", as_f32(got), as_f32(want), wl.offsets)
+            assert_state(f"step {t} {k}", as_f32(got), as_f32(want), wl.offsets,
+                         bf16_step=got.dtype == np.uint16)
             exact &= np.array_equal(got, want)
         if t >= wl.freeze_step:
             assert_bits(f"step {t} bits_w", np_of(gpu.bits_w), ref["bits_w"])
             assert_bits(f"step {t} bits_srv", np_of(gpu.bits_srv), ref["bits_srv"])
             assert_scales(f"step {t} s_w", np_of(gpu.s_w), ref["s_w"])
             assert_scales(f"step {t} s_srv", np_of(gpu.s_srv), ref["s_srv"])
+        sync_state(gpu, ref)
     assert gpu.status() == flags == 0
     return gpu, exact
 
