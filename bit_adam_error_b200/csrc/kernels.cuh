@@ -297,6 +297,28 @@ __device__ __forceinline__ int64_t warp_count() {
   return (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
 }
 
+// Grid-stride loop over items it = r * T + t (rows x tiles) without a 64-bit
+// division per item: the warp's first item is split once, then t advances by the
+// stride and carries into r -- the same items, in the same order, as it += stride.
+struct RowTile {
+  int r;
+  int64_t t;
+};
+
+__device__ __forceinline__ RowTile first_item(int64_t T) {   // T > 0
+  const int64_t it = warp_id();
+  const int r = static_cast<int>(it / T);
+  return RowTile{r, it - static_cast<int64_t>(r) * T};
+}
+
+__device__ __forceinline__ void next_item(RowTile& x, int64_t T, int rows) {
+  x.t += warp_count();
+  while (x.t >= T && x.r < rows) {
+    x.t -= T;
+    ++x.r;
+  }
+}
+
 // ---- fused finaliser (small problems) ---------------------------------------------
 // On small problems a separate finaliser launch costs as much as a pass, so the
 // pass's last CTA computes the scales itself.  Every thread fences its partial

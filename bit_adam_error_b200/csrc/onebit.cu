@@ -552,7 +552,10 @@ void enqueue_tb_finalize(ob_ctx* c, const double* part, int rows, float* out, cu
 }
 
 // Worker stage (passes 1 and 2, each followed by its scales) and, when
-// with_server, the server scales from pass 2's sums.
+// with_server, the server scales from pass 2's sums.  (A fused finaliser in the
+// pass's last CTA, as the 1-bit rule has for small problems, measured slower
+// here: one CTA finishing both sweeps of every (row, chunk) has less
+// parallelism than k_tb_finalize's one block per (row, chunk).)
 template <typename GT, typename ET, bool CLIP, bool POW2>
 void enqueue_tb_worker_t(ob_ctx* c, const GT* grads, bool with_server, cudaStream_t st) {
   const int W = c->cfg.W;

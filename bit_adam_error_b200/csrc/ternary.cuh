@@ -133,11 +133,11 @@ k_ternary_compress(Layout L, int W, const GT* __restrict__ grads, ET* __restrict
                    uint32_t* __restrict__ codes, Hyper h, uint32_t* __restrict__ status) {
   pdl_enter();
   const int lane = threadIdx.x & 31;
-  const int64_t items = static_cast<int64_t>(W) * L.T;
+  if (L.T == 0) return;
   int hint = 0;
-  for (int64_t it = warp_id(); it < items; it += warp_count()) {
-    const int w = static_cast<int>(it / L.T);
-    const int64_t t = it - static_cast<int64_t>(w) * L.T;
+  for (RowTile x = first_item(L.T); x.r < W; next_item(x, L.T, W)) {
+    const int w = x.r;
+    const int64_t t = x.t;
     const Tile tl = tile_at(L, t, hint);
     const GT* g = grads + static_cast<int64_t>(w) * L.n + tl.ck0;
     ET* e = err + static_cast<int64_t>(w) * L.n + tl.ck0;

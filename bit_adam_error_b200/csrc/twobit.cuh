@@ -130,16 +130,16 @@ __device__ __forceinline__ float tb_server_sum1(const Layout& L, int W, const ui
 // pass 1), part[P + it] = S_t, part[2P + it] = M2_t (see Shifted).  A non-finite
 // sum c^2 raises the status flag.
 template <typename GT, typename ET, bool CLIP>
-__global__ void __launch_bounds__(kBlock)
-k_tb_worker_norm(Layout L, int W, const GT* __restrict__ grads, const ET* __restrict__ err,
-                 float clip, double* __restrict__ part, uint32_t* __restrict__ status) {
-  pdl_enter();
+__device__ __forceinline__ void tb_worker_norm_tiles(Layout L, int W, const GT* __restrict__ grads,
+                                                     const ET* __restrict__ err, float clip,
+                                                     double* __restrict__ part, uint32_t* __restrict__ status) {
   const int lane = threadIdx.x & 31;
+  if (L.T == 0) return;
   const int64_t items = static_cast<int64_t>(W) * L.T;
   int hint = 0;
-  for (int64_t it = warp_id(); it < items; it += warp_count()) {
-    const int w = static_cast<int>(it / L.T);
-    const int64_t t = it - static_cast<int64_t>(w) * L.T;
+  for (RowTile x = first_item(L.T); x.r < W; next_item(x, L.T, W)) {
+    const int w = x.r;
+    const int64_t t = x.t, it = static_cast<int64_t>(w) * L.T + t;
     const Tile tl = tile_at(L, t, hint);
     const GT* g = grads + static_cast<int64_t>(w) * L.n + tl.ck0;
     const ET* e = err + static_cast<int64_t>(w) * L.n + tl.ck0;
@@ -188,6 +188,14 @@ k_tb_worker_norm(Layout L, int W, const GT* __restrict__ grads, const ET* __rest
   }
 }
 
+template <typename GT, typename ET, bool CLIP>
+__global__ void __launch_bounds__(kBlock)
+k_tb_worker_norm(Layout L, int W, const GT* __restrict__ grads, const ET* __restrict__ err,
+                 float clip, double* __restrict__ part, uint32_t* __restrict__ status) {
+  pdl_enter();
+  tb_worker_norm_tiles<GT, ET, CLIP>(L, W, grads, err, clip, part, status);
+}
+
 // ---- pass 2: both planes, worker error (+ server sums) ---------------------------------
 // SERVER: also c_srv = (sum_w dequantised_w) / W + srv_err, with part_srv[t] =
 // sum c_srv^2, part_srv[T + t] = S_t and part_srv[2T + t] = M2_t of |c_srv| (see
@@ -195,11 +203,9 @@ k_tb_worker_norm(Layout L, int W, const GT* __restrict__ grads, const ET* __rest
 // Three CTAs per SM (at most 80 registers): the cached, clipped variant would
 // otherwise take 92 and drop to two.
 template <typename GT, typename ET, bool SERVER, bool CLIP, bool POW2, bool CACHE>
-__global__ void __launch_bounds__(kBlock, 3)
-k_tb_pack(Layout L, int W, const GT* __restrict__ grads, ET* __restrict__ err,
+__device__ __forceinline__ void tb_pack_tiles(Layout L, int W, const GT* __restrict__ grads, ET* __restrict__ err,
           const float* __restrict__ s_w, uint32_t* __restrict__ bits_w, const ET* __restrict__ srv_err,
           double* __restrict__ part_srv, float* __restrict__ csrv, float clip, uint32_t* __restrict__ status) {
-  pdl_enter();
   const int lane = threadIdx.x & 31;
   const auto mean = make_mean<POW2>(W);
   int hint = 0;
@@ -316,15 +322,24 @@ k_tb_pack(Layout L, int W, const GT* __restrict__ grads, ET* __restrict__ err,
   }
 }
 
+template <typename GT, typename ET, bool SERVER, bool CLIP, bool POW2, bool CACHE>
+__global__ void __launch_bounds__(kBlock, 3)
+k_tb_pack(Layout L, int W, const GT* __restrict__ grads, ET* __restrict__ err,
+          const float* __restrict__ s_w, uint32_t* __restrict__ bits_w, const ET* __restrict__ srv_err,
+          double* __restrict__ part_srv, float* __restrict__ csrv, float clip, uint32_t* __restrict__ status) {
+  pdl_enter();
+  tb_pack_tiles<GT, ET, SERVER, CLIP, POW2, CACHE>(L, W, grads, err, s_w, bits_w, srv_err, part_srv, csrv, clip,
+                                                    status);
+}
+
 // ---- server sums from the worker planes (stage call) ----------------------------------
 // part[t] = sum c_srv^2, part[T + t] = S_t, part[2T + t] = M2_t of |c_srv| (see
 // Shifted; one row): the values and the order of the fused pass 2.  W1 (with
 // POW2): one worker (see tb_server_sum8).
 template <typename ET, bool POW2, bool W1>
-__global__ void __launch_bounds__(kBlock)
-k_tb_server_norm(Layout L, int W, const uint32_t* __restrict__ bits_w, const float* __restrict__ s_w,
-                 const ET* __restrict__ srv_err, double* __restrict__ part, uint32_t* __restrict__ status) {
-  pdl_enter();
+__device__ __forceinline__ void tb_server_norm_tiles(Layout L, int W, const uint32_t* __restrict__ bits_w,
+                                                     const float* __restrict__ s_w, const ET* __restrict__ srv_err,
+                                                     double* __restrict__ part, uint32_t* __restrict__ status) {
   const int lane = threadIdx.x & 31;
   const auto mean = make_mean_w<POW2, W1>(W);
   int hint = 0;
@@ -379,6 +394,14 @@ k_tb_server_norm(Layout L, int W, const uint32_t* __restrict__ bits_w, const flo
   }
 }
 
+template <typename ET, bool POW2, bool W1>
+__global__ void __launch_bounds__(kBlock)
+k_tb_server_norm(Layout L, int W, const uint32_t* __restrict__ bits_w, const float* __restrict__ s_w,
+                 const ET* __restrict__ srv_err, double* __restrict__ part, uint32_t* __restrict__ status) {
+  pdl_enter();
+  tb_server_norm_tiles<ET, POW2, W1>(L, W, bits_w, s_w, srv_err, part, status);
+}
+
 // ---- both scales of a chunk from the tile sums ----------------------------------------------
 // Row r, chunk k (P = rows * T): A = sum_t part[r*T + t], s1 = sqrt(A) / sqrt(n_k);
 // then, with S_t = part[P + r*T + t], M2_t = part[2P + r*T + t] and n_t the tile's
@@ -402,13 +425,19 @@ k_tb_finalize(Layout L, const double* __restrict__ part, int rows, float* __rest
   const double A = block_sum_fixed(acc, sm);
   const double rn = __dsqrt_rn(static_cast<double>(nk));
   const float s1 = nk > 0 ? __double2float_rn(__ddiv_rn(__dsqrt_rn(A), rn)) : 0.0f;
+  // Full tiles in the loop (no division, so loads pipeline); a ragged last tile
+  // after it, by the thread whose stride reaches it.
+  const int64_t tf = t0 + nk / kTile;
+  const double s1d = static_cast<double>(s1);
   acc = 0.0;
-  for (int64_t t = t0 + threadIdx.x; t < t1; t += kFinalizeThreads) {
-    const int64_t left = nk - (t - t0) * kTile;
-    const double mu = left >= kTile ? ps[t] * (1.0 / kTile) : ps[t] / static_cast<double>(left);
-    const double nt = static_cast<double>(left < kTile ? left : kTile);
-    const double d = mu - static_cast<double>(s1);
-    acc += pm[t] + nt * d * d;
+  for (int64_t t = t0 + threadIdx.x; t < tf; t += kFinalizeThreads) {
+    const double d = ps[t] * (1.0 / kTile) - s1d;
+    acc += pm[t] + static_cast<double>(kTile) * d * d;
+  }
+  if (tf < t1 && (tf - t0) % kFinalizeThreads == threadIdx.x) {
+    const double nt = static_cast<double>(nk - (tf - t0) * kTile);
+    const double d = ps[tf] / nt - s1d;
+    acc += pm[tf] + nt * d * d;
   }
   const double R = block_sum_fixed(acc, sm);
   if (threadIdx.x == 0) {
