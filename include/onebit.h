@@ -44,7 +44,10 @@
  *   s1 = ||c|| / sqrt(n_k), q1 = sign(c), r = c - s1 q1,
  *   s2 = ||r|| / sqrt(n_k), q2 = sign(r), err = r - s2 q2,
  * dequantised as s1 q1 + s2 q2 -- for the workers and, on their average plus
- * the server error, for the server.
+ * the server error, for the server.  ||r||^2 is formed from per-tile sums of
+ * |c| and of its squared deviations (sum (|c| - s1)^2, an identity), so it
+ * equals the sum of the squared float residuals to within their rounding
+ * (2^-23 relative at most); the planes depend on s1 and c only.
  *
  * Conventions for every call:
  *   - Device buffers are caller-owned and must stay valid for the ctx's life.
