@@ -899,6 +899,7 @@ def run_dp(args):
                 "model_value": layout.n / (ms / 1e3) / 1e9,
                 "exchange_bytes_per_step_per_rank": 2 * 4 * (int(layout.words[-1]) + scales_per_chunk * layout.C),
                 "roofline": roofline, "kernels": dp_kernels,
+                "kernel_timing": "per-kernel CUDA events of every ctx in the timed steps",
                 "gpu_launches": launches, "status_flags": flags, "e2e": e2e, "clocks": clocks}
         print(json.dumps(line), flush=True)
     stages.close()
