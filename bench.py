@@ -266,10 +266,10 @@ class ClockSampler:
 # -- distributed plumbing ------------------------------------------------------------------
 
 def dp_bytes_per_elem(kind: str, role: str, wl, world: int, rule: str) -> float:
-    """HBM bytes per element of a data-parallel stage kernel (scaled-sign and
-    2-bit rules): role "worker" (a one-worker ctx: the worker stage, or the
-    update alone), "server" (the owner's W-worker server stage).  0 when not
-    modelled."""
+    """HBM bytes per element of a data-parallel stage kernel: role "worker" (a
+    ctx over the rank's gradient or a slice of it: the worker stage, or the
+    update alone), "server" (the owner's W-worker server stage).  0 for the
+    finalisers and the monitoring kernels."""
     gb, eb = wl.grad_bytes, wl.err_bytes
     upd = 16.0 if wl.optimizer == "lamb" else 20.0
     if rule == "scaled" and role == "worker":
@@ -288,6 +288,12 @@ def dp_bytes_per_elem(kind: str, role: str, wl, world: int, rule: str) -> float:
     if rule == "twobit" and role == "server":
         return {"k_tb_server_norm": world / 4 + eb,            # W workers' planes, srv_err
                 "k_tb_server_update": world / 4 + 2 * eb + 1 / 4}.get(kind, 0.0)
+    if rule == "momentum" and role == "worker":
+        return {"k_ternary_compress": gb + 2 * eb + 1,         # g, err r/w, one code byte
+                "k_ternary_update": 1 + upd,                   # one sum byte, m r/w, v, p (+ p w)
+                "k_lamb_param": 16.0}.get(kind, 0.0)
+    if rule == "momentum" and role == "server":
+        return {"k_ternary_server": world + 1.0}.get(kind, 0.0)  # W code bytes in, one sum byte out
     return 0.0
     gb, eb = wl.grad_bytes, wl.err_bytes
     upd = 16.0 if wl.optimizer == "lamb" else 20.0

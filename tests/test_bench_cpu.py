@@ -133,3 +133,6 @@ def test_byte_model_of_the_data_parallel_stages():
     assert bench.dp_bytes_per_elem("k_worker_norm", "worker", wl, 8, "momentum") == 0
     assert bench.dp_bytes_per_elem("k_tb_pack", "worker", wl, 8, "twobit") == 2 + 8 + 1 / 4
     assert bench.dp_bytes_per_elem("k_tb_server_norm", "server", wl, 8, "twobit") == 2 + 4
+    assert bench.dp_bytes_per_elem("k_ternary_compress", "worker", wl, 8, "momentum") == 2 + 8 + 1
+    assert bench.dp_bytes_per_elem("k_ternary_server", "server", wl, 8, "momentum") == 9
+    assert bench.dp_bytes_per_elem("k_ternary_update", "worker", wl, 8, "momentum") == 21
