@@ -472,10 +472,9 @@ k_worker_norm_fin(Layout L, int W, const GT* __restrict__ grads, const ET* __res
 
 
 // ---- finalize: per-chunk scale from tile partials ----------------------------------
-// Partial slots of chunk k are [tpx[k] * mult, tpx[k+1] * mult) of each row (tpx =
-// warp-tile prefix with mult 1, or block-tile prefix with one slot per consumer
-// warp).  out[r * C + k] = sqrt(sum of the slots, fixed order) / sqrt(n_k); 0 for
-// an empty chunk.  grid = (C, R).
+// The partials of chunk k are the slots [tp[k], tp[k+1]) of each row (one per
+// warp tile).  out[r * C + k] = sqrt(sum of the slots, fixed order) / sqrt(n_k);
+// 0 for an empty chunk.  grid = (C, R).
 __device__ __forceinline__ double block_sum_fixed(double x, double* sm) {
   const int tid = threadIdx.x;
   sm[tid] = x;
@@ -493,14 +492,13 @@ __device__ __forceinline__ double block_sum_fixed(double x, double* sm) {
 // The result of (row r, chunk k) goes to out[r * C + k].
 template <bool RMS>
 __global__ void __launch_bounds__(kFinalizeThreads)
-k_finalize_scale(Layout L, const double* __restrict__ part, const int64_t* __restrict__ tpx,
-                 int mult, int64_t row_stride, float* __restrict__ out) {
+k_finalize_scale(Layout L, const double* __restrict__ part, int64_t row_stride, float* __restrict__ out) {
   pdl_enter();
   __shared__ double sm[kFinalizeThreads];
   const int k = blockIdx.x, r = blockIdx.y;
   const double* pr = part + static_cast<int64_t>(r) * row_stride;
   double acc = 0.0;
-  for (int64_t t = tpx[k] * mult + threadIdx.x; t < tpx[k + 1] * mult; t += kFinalizeThreads) acc += pr[t];
+  for (int64_t t = L.tp[k] + threadIdx.x; t < L.tp[k + 1]; t += kFinalizeThreads) acc += pr[t];
   const double S = block_sum_fixed(acc, sm);
   if (threadIdx.x == 0) {
     const int64_t nk = L.off[k + 1] - L.off[k];
@@ -514,12 +512,12 @@ k_finalize_scale(Layout L, const double* __restrict__ part, const int64_t* __res
 // LAMB trust ratio per layer (chunk): r = sqrt(P) / sqrt(U), 1 if either is 0.  grid = C.
 __global__ void __launch_bounds__(kFinalizeThreads)
 k_finalize_ratio(Layout L, const double* __restrict__ partP, const double* __restrict__ partU,
-                 const int64_t* __restrict__ tpx, int mult, float* __restrict__ ratio) {
+                 float* __restrict__ ratio) {
   pdl_enter();
   __shared__ double sm[kFinalizeThreads];
   const int k = blockIdx.x;
   double a = 0.0, b = 0.0;
-  for (int64_t t = tpx[k] * mult + threadIdx.x; t < tpx[k + 1] * mult; t += kFinalizeThreads) {
+  for (int64_t t = L.tp[k] + threadIdx.x; t < L.tp[k + 1]; t += kFinalizeThreads) {
     a += partP[t];
     b += partU[t];
   }

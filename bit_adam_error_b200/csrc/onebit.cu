@@ -252,14 +252,12 @@ ob_err check_grads(ob_ctx* c, const void* grads) {
 
 // ---- enqueue helpers (no validation) ----------------------------------------------
 
-// Per-chunk scales from partial slots [tpx[k]*mult, tpx[k+1]*mult) of each row.
-// planes / plane: where the scales land (one per chunk, or plane `plane` of the
-// two interleaved scales of the 2-bit rule).
-void enqueue_finalize_scale(ob_ctx* c, const double* part, float* out, int rows,
-                            const int64_t* tpx, int mult, int64_t row_stride, cudaStream_t st) {
+// Per-chunk scales from the tile partials of each row (rows of row_stride slots).
+void enqueue_finalize_scale(ob_ctx* c, const double* part, float* out, int rows, int64_t row_stride,
+                            cudaStream_t st) {
   launch(c, OB_K_FINALIZE_SCALE, st, [&] {
-    pdl(ob::k_finalize_scale<true>, dim3(c->cfg.num_chunks, rows), ob::kFinalizeThreads, st, 
-        c->L, part, tpx, mult, row_stride, out);
+    pdl(ob::k_finalize_scale<true>, dim3(c->cfg.num_chunks, rows), ob::kFinalizeThreads, st, c->L, part,
+        row_stride, out);
   });
 }
 
@@ -304,7 +302,7 @@ void enqueue_worker_t(ob_ctx* c, const GT* grads, bool with_server, cudaStream_t
       pdl(k1, g1, ob::kBlock, st, c->L, W, grads, err, c->h.clip, c->part_w, c->status);
     });
   }
-  if (!fin1) enqueue_finalize_scale(c, c->part_w, c->s_w, W, c->L.tp, 1, c->T, st);
+  if (!fin1) enqueue_finalize_scale(c, c->part_w, c->s_w, W, c->T, st);
   if (c->T > 0) {
     // The stage call (no server part) never uses the mean: one instantiation each.
     // Many workers: the fused step also stores c_srv for pass 3 (CACHE).
@@ -336,7 +334,7 @@ void enqueue_worker_t(ob_ctx* c, const GT* grads, bool with_server, cudaStream_t
       });
     }
   }
-  if (with_server && !fin2) enqueue_finalize_scale(c, c->part_srv, c->s_srv, 1, c->L.tp, 1, 0, st);
+  if (with_server && !fin2) enqueue_finalize_scale(c, c->part_srv, c->s_srv, 1, 0, st);
 }
 
 template <typename GT, typename ET>
@@ -393,7 +391,7 @@ void enqueue_server_update(ob_ctx* c, cudaStream_t st, bool cached = false) {
 void enqueue_lamb_param(ob_ctx* c, cudaStream_t st) {
   launch(c, OB_K_FINALIZE_RATIO, st, [&] {
     pdl(ob::k_finalize_ratio, c->cfg.num_chunks, ob::kFinalizeThreads, st, c->L, c->partP, c->partU,
-                                                                             c->L.tp, 1, c->ratio);
+        c->ratio);
   });
   if (c->T == 0) return;
   auto k = ob::k_lamb_param;
@@ -461,7 +459,7 @@ void enqueue_server_stage(ob_ctx* c, cudaStream_t st) {
     if (c->cfg.err_dtype == OB_BF16) enqueue_server_norm<uint16_t>(c, fin, st);
     else enqueue_server_norm<float>(c, fin, st);
   }
-  if (!fin) enqueue_finalize_scale(c, c->part_srv, c->s_srv, 1, c->L.tp, 1, 0, st);
+  if (!fin) enqueue_finalize_scale(c, c->part_srv, c->s_srv, 1, 0, st);
   enqueue_server_update<ob::Upd::kNone, true>(c, st);
 }
 
@@ -1174,7 +1172,7 @@ ob_err ob_error_norms(ob_ctx* c, float* worker_norms, float* server_norms, void*
     }
     launch(c, OB_K_FINALIZE_SCALE, st, [&] {
       pdl(ob::k_finalize_scale<false>, dim3(unsigned(C), unsigned(rows)), ob::kFinalizeThreads, st,
-          c->L, part, c->L.tp, 1, c->T, out);
+          c->L, part, c->T, out);
     });
   };
   if (worker_norms) norms(c->err, int(W), c->part_w, worker_norms);
@@ -1442,7 +1440,7 @@ extern "C" ob_err ob_compress_noalloc(const ob_config* cfg, const void* grads, f
     else if (cl) ob::k_worker_norm<float, float, true><<<g1, ob::kBlock, 0, st>>>(L, int(W), gf, err, clip, part, status);
     else ob::k_worker_norm<float, float, false><<<g1, ob::kBlock, 0, st>>>(L, int(W), gf, err, clip, part, status);
   }
-  ob::k_finalize_scale<true><<<dim3(unsigned(C), unsigned(W)), ob::kFinalizeThreads, 0, st>>>(L, part, L.tp, 1, T, s_w);
+  ob::k_finalize_scale<true><<<dim3(unsigned(C), unsigned(W)), ob::kFinalizeThreads, 0, st>>>(L, part, T, s_w);
   if (T > 0) {
     const int g2 = noalloc_grid(d->num_sms, d->occ_pack[bf][cl ? 1 : 0], T);
     const uint16_t* gh = static_cast<const uint16_t*>(grads);
