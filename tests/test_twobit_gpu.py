@@ -190,6 +190,39 @@ def test_fused_steps_free_running(layout, W, gdt, opt, clip):
     print(f"2-bit free-running {layout} W={W} {gdt} {opt}: bit-identical to the oracle: {exact}")
 
 
+@pytest.mark.parametrize("W", [1, 2])
+def test_equal_magnitudes_give_an_exact_zero_second_scale(W):
+    """Gradients of one magnitude per chunk (random signs, the same for every
+    worker): |c| equals s1 everywhere, so the residual is exactly 0 and both
+    second scales are exactly 0 -- on the GPU, whose second scale comes from
+    shifted tile sums of |c|, as in the oracle.  Chunks of 1, 33, 512, 1000 and
+    4104 elements (ragged tiles, the scalar and 8-wide paths) and an empty one."""
+    sizes = [1, 33, 512, 0, 1000, 4104]
+    wl = small(sizes, W)
+    p, v = state_for(wl)
+    rng = np.random.default_rng(17)
+    mags = np.float32([3.0517578e-05, 1e-3, 0.25, 1.0, 7.5e-4, 2.0 ** -20])
+    row = np.concatenate([np.where(rng.random(n) < 0.5, -1.0, 1.0).astype(np.float32) * mags[k]
+                          for k, n in enumerate(sizes)]).astype(np.float32)
+    g = np.stack([row] * W)
+    gpu = make_gpu(wl.offsets, W, p=to_dev(p), v=to_dev(v))
+    gpu.step(to_dev(g))
+    torch.cuda.synchronize()
+    ref = {"p": p.copy(), "m": np.zeros(wl.n, np.float32), "v": v.copy(),
+           "err": np.zeros((W, wl.n), np.float32), "srv_err": np.zeros(wl.n, np.float32)}
+    o = oracle.get()
+    assert o.twobit_step(wl.offsets, g, ref, F["beta1"], F["lr"], F["eps"]) == 0
+    s_w, s_srv = np_of(gpu.s_w).reshape(W, len(sizes), 2), np_of(gpu.s_srv).reshape(len(sizes), 2)
+    assert np.array_equal(s_w, ref["s_w"]) and np.array_equal(s_srv, ref["s_srv"])
+    assert np.all(s_w[:, :, 1] == 0) and np.all(s_srv[:, 1] == 0)
+    assert np.array_equal(s_w[0, :, 0], np.where(np.array(sizes) > 0, mags, 0))
+    assert_bits("bits_w", np_of(gpu.bits_w), ref["bits_w"])
+    assert_bits("bits_srv", np_of(gpu.bits_srv), ref["bits_srv"])
+    for k in ("p", "m", "err", "srv_err"):
+        assert np.array_equal(np_of(getattr(gpu, k)), ref[k].reshape(np_of(getattr(gpu, k)).shape)), k
+    assert gpu.status() == 0
+
+
 def test_warmup_then_compressed():
     run_chain(small(ALIGNED, 4, freeze_step=2), 5)
 
